@@ -1,0 +1,166 @@
+"""fp64 CPU oracle for the AttentionPack decode hot path (numpy front end).
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+cpu_baseline / reference leg of bench.py may import this package.  It shares
+no code with the product (rank_compressed_kv_b200), and neither imports the
+other.
+
+The arithmetic lives in oracle.c (plain C, fp64, OpenMP over independent
+units); this module converts numpy arrays and calls it.  What each routine
+computes, and the passage of the method it follows:
+
+  compress  -- multi-head SVD compression (AttentionPack pages, Technical
+               summary 2.A): K (T x 512, the 4 KV heads of a group side by
+               side) = C . B with C = U_r Sigma_r and B = V_r^T, by Householder
+               QR followed by one-sided Jacobi (Hestenes) SVD.
+  decode    -- one decode step with attention-aware partial decompression
+               (pages 2.B): each visual token decompressed at rank r or r_lo
+               by its mask bit, then dense softmax attention over visual
+               tokens plus the uncompressed text tail; also the attention
+               mass each visual token received.
+  select    -- importance = moving average (alpha) of attention mass; the k
+               largest get the full rank next step, ties to the lower index.
+
+Parity pins for every routine are in tests/test_oracle_*.py.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_fp = ctypes.POINTER(ctypes.c_float)
+_u32p = ctypes.POINTER(ctypes.c_uint32)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_i64 = ctypes.c_int64
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        L.ora_bf16_to_f64_array.argtypes = [_u16p, _dp, _i64]
+        L.ora_f64_to_bf16_array.argtypes = [_dp, _u16p, _i64]
+        L.ora_svd.argtypes = [_dp, _i64, ctypes.c_int, _dp, _dp]
+        L.ora_svd.restype = ctypes.c_int
+        L.ora_compress_units.argtypes = [_i64, _dp, _i64, ctypes.c_int, ctypes.c_int, _dp, _dp, _dp]
+        L.ora_compress_units.restype = ctypes.c_int
+        L.ora_decode_units.argtypes = [_i64, _i64, _i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       _dp, _dp, _dp, _dp, _dp, _dp, _u32p, _dp, ctypes.c_double, _dp, _dp]
+        L.ora_select_units.argtypes = [_i64, _i64, _fp, _fp, ctypes.c_float, _i64, _u32p]
+        _lib = L
+    return _lib
+
+
+def _ptr(a, t):
+    return a.ctypes.data_as(t)
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+# ------------------------------------------------------------------ bf16
+
+def bf16_to_f64(bits) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (uint16) to float64."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    out = np.empty(b.shape, dtype=np.float64)
+    lib().ora_bf16_to_f64_array(_ptr(b, _u16p), _ptr(out, _dp), b.size)
+    return out
+
+
+def f64_to_bf16(x) -> np.ndarray:
+    """Round float64 to the nearest bf16 (ties to even), one rounding step; uint16 bits."""
+    a = _f64(x)
+    out = np.empty(a.shape, dtype=np.uint16)
+    lib().ora_f64_to_bf16_array(_ptr(a, _dp), _ptr(out, _u16p), a.size)
+    return out
+
+
+# ------------------------------------------------------------- compress
+
+def svd(X):
+    """Singular values (descending) and right singular vectors (columns of V) of X (T x n)."""
+    X = _f64(X)
+    T, n = X.shape
+    sig = np.empty(min(T, n), dtype=np.float64)
+    V = np.empty((n, n), dtype=np.float64)
+    sweeps = lib().ora_svd(_ptr(X, _dp), T, n, _ptr(sig, _dp), _ptr(V, _dp))
+    if sweeps < 0:
+        raise RuntimeError("oracle Jacobi SVD did not converge")
+    return sig, V
+
+
+def compress(X, r=64):
+    """Truncated factors of units X [U, T, n] (fp64): C [U,T,r], B [U,r,n], sigma [U,min(T,n)]."""
+    X = _f64(X)
+    if X.ndim == 2:
+        X = X[None]
+    U, T, n = X.shape
+    C = np.empty((U, T, r))
+    B = np.empty((U, r, n))
+    sig = np.empty((U, min(T, n)))
+    s = lib().ora_compress_units(U, _ptr(X, _dp), T, n, r, _ptr(C, _dp), _ptr(B, _dp), _ptr(sig, _dp))
+    if s < 0:
+        raise RuntimeError("oracle Jacobi SVD did not converge")
+    return C, B, sig
+
+
+# --------------------------------------------------------------- decode
+
+def decode(CK, BK, CV, BV, Ktext, Vtext, mask, q, r_lo=16, scale=1.0, want_mass=True):
+    """One decode step over U independent units (fp64).
+
+    CK, CV [U,T,r]; BK, BV [U,r,512]; Ktext, Vtext [U,L,4,128]; mask uint32
+    [U, ceil(T/32)]; q [U,Hg,128].  Returns out [U,Hg,128] and mass [U,T].
+    """
+    CK, BK, CV, BV = (_f64(a) for a in (CK, BK, CV, BV))
+    Ktext, Vtext, q = _f64(Ktext), _f64(Vtext), _f64(q)
+    U, T, r = CK.shape
+    L = Ktext.shape[1]
+    Hg = q.shape[1]
+    assert BK.shape == (U, r, 512) and Ktext.shape == (U, L, 4, 128) and q.shape == (U, Hg, 128)
+    assert Hg % 4 == 0
+    m = np.ascontiguousarray(mask, dtype=np.uint32).reshape(U, (T + 31) // 32)
+    out = np.empty((U, Hg, 128))
+    mass = np.empty((U, T)) if want_mass else None
+    if L == 0:   # keep valid pointers for empty tails
+        Ktext = np.zeros((U, 1, 4, 128))
+        Vtext = np.zeros((U, 1, 4, 128))
+    lib().ora_decode_units(U, T, L, Hg, r, r_lo, _ptr(CK, _dp), _ptr(BK, _dp), _ptr(CV, _dp), _ptr(BV, _dp),
+                           _ptr(Ktext, _dp), _ptr(Vtext, _dp), _ptr(m, _u32p), _ptr(q, _dp), float(scale),
+                           _ptr(out, _dp), _ptr(mass, _dp) if want_mass else None)
+    return out, mass
+
+
+# --------------------------------------------------------------- select
+
+def select(mass, k, alpha=0.0, score=None):
+    """Rank mask for the next step from fp32 mass [U,T] (and EMA score, updated in place).
+
+    Returns (mask uint32 [U, ceil(T/32)], score fp32 [U,T]).
+    """
+    mass = np.ascontiguousarray(mass, dtype=np.float32)
+    if mass.ndim == 1:
+        mass = mass[None]
+    U, T = mass.shape
+    if score is None:
+        score = np.zeros_like(mass)
+    score = np.ascontiguousarray(score, dtype=np.float32).reshape(U, T).copy()
+    mask = np.empty((U, (T + 31) // 32), dtype=np.uint32)
+    lib().ora_select_units(U, T, _ptr(mass, _fp), _ptr(score, _fp), ctypes.c_float(alpha), int(k),
+                           _ptr(mask, _u32p))
+    return mask, score
+
+
+def mask_bits(mask, T) -> np.ndarray:
+    """Bool [.., T] view of a packed rank mask (bit t of word t>>5)."""
+    m = np.asarray(mask, dtype=np.uint32)
+    idx = np.arange(T)
+    return ((m[..., idx >> 5] >> (idx & 31).astype(np.uint32)) & 1).astype(bool)
