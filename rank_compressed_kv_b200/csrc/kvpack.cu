@@ -1,0 +1,296 @@
+// kvpack.cu -- the C ABI of libkvpack (see include/kvpack.h): argument
+// validation, workspace planning and kernel launches.  Everything that
+// computes runs in the kernels of decode.cuh, select.cuh and compress.cuh.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "kvpack.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "select.cuh"
+#include "compress.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxT = 65536;
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+kvpack_status check_dims(const kvpack_dims *d, int32_t n_layers) {
+    if (d == nullptr || n_layers <= 0) return KVPACK_ERR_INVALID_ARG;
+    if (d->batch <= 0 || d->n_q_heads <= 0 || d->n_kv_heads <= 0 || d->T_vis <= 0 || d->L_text_cap < 0)
+        return KVPACK_ERR_INVALID_ARG;
+    if (d->group != KVPACK_GROUP || d->head_dim != KVPACK_HEAD_DIM || d->rank != KVPACK_RANK ||
+        d->rank_lo != KVPACK_RANK_LO)
+        return KVPACK_ERR_UNSUPPORTED;
+    if (d->n_kv_heads % KVPACK_GROUP != 0 || d->n_q_heads % d->n_kv_heads != 0) return KVPACK_ERR_UNSUPPORTED;
+    if ((d->n_q_heads / d->n_kv_heads) * KVPACK_GROUP > 32) return KVPACK_ERR_UNSUPPORTED;
+    if (d->T_vis > kMaxT) return KVPACK_ERR_UNSUPPORTED;
+    const long long units = (long long)n_layers * d->batch * (d->n_kv_heads / KVPACK_GROUP);
+    if (units > (1LL << 30)) return KVPACK_ERR_UNSUPPORTED;
+    return KVPACK_OK;
+}
+
+inline int n_units(const kvpack_dims *d, int32_t n_layers) {
+    return n_layers * d->batch * (d->n_kv_heads / KVPACK_GROUP);
+}
+
+inline int hg(const kvpack_dims *d) { return (d->n_q_heads / d->n_kv_heads) * KVPACK_GROUP; }
+
+struct DecodePlan {
+    int nmb, S, tps, units, Hg;
+    size_t off_qt, off_part, off_arrive, total;
+};
+
+DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
+    DecodePlan pl{};
+    pl.Hg = hg(d);
+    pl.nmb = (pl.Hg <= 16) ? 1 : 2;
+    const int tps_max = (pl.nmb == 1) ? kvpack::decode::Cfg<1>::kTPS : kvpack::decode::Cfg<2>::kTPS;
+    const int lot = (pl.nmb == 1) ? kvpack::decode::Cfg<1>::kLoT : kvpack::decode::Cfg<2>::kLoT;
+    pl.S = (d->T_vis + tps_max - 1) / tps_max;
+    const int per = (d->T_vis + pl.S - 1) / pl.S;
+    pl.tps = (per + lot - 1) / lot * lot;
+    pl.units = n_units(d, n_layers);
+    size_t off = 0;
+    pl.off_qt = off;
+    off = align256(off + (size_t)pl.units * 2 * pl.Hg * 64 * sizeof(uint16_t));
+    pl.off_part = off;
+    if (pl.S > 1) off = align256(off + (size_t)pl.units * pl.S * pl.Hg * kvpack::decode::kPartFloats * sizeof(float));
+    pl.off_arrive = off;
+    off = align256(off + (size_t)pl.units * sizeof(unsigned int));
+    pl.total = off;
+    return pl;
+}
+
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+    int attn_blocks[2] = {0, 0};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+kvpack_status device_info(DeviceInfo **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVPACK_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo &di = g_dev[dev];
+    if (!di.ready) {
+        if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return KVPACK_ERR_CUDA;
+        const int s1 = (int)sizeof(kvpack::decode::Smem<1>), s2 = (int)sizeof(kvpack::decode::Smem<2>);
+        if (cudaFuncSetAttribute(kvpack::decode::attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1) != cudaSuccess)
+            return KVPACK_ERR_CUDA;
+        if (cudaFuncSetAttribute(kvpack::decode::attn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2) != cudaSuccess)
+            return KVPACK_ERR_CUDA;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.attn_blocks[0], kvpack::decode::attn_kernel<1>,
+                                                          kvpack::decode::kThreads, s1) != cudaSuccess)
+            return KVPACK_ERR_CUDA;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.attn_blocks[1], kvpack::decode::attn_kernel<2>,
+                                                          kvpack::decode::kThreads, s2) != cudaSuccess)
+            return KVPACK_ERR_CUDA;
+        if (di.attn_blocks[0] < 1 || di.attn_blocks[1] < 1) return KVPACK_ERR_CUDA;
+        kvpack_status cs = kvpack::compress::prepare_device();
+        if (cs != KVPACK_OK) return cs;
+        di.ready = true;
+    }
+    *out = &di;
+    return KVPACK_OK;
+}
+
+template <int KPT, int NW>
+cudaError_t launch_select(const kvpack::select::Params &p, cudaStream_t st) {
+    if (NW == 1) {
+        const int grid = (p.n_units + 7) / 8;
+        kvpack::select::select_kernel<KPT, 1><<<grid, 256, 0, st>>>(p);
+    } else {
+        kvpack::select::select_kernel<KPT, 32><<<p.n_units, 1024, 0, st>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+template <int NW>
+cudaError_t select_dispatch(int kpt, const kvpack::select::Params &p, cudaStream_t st) {
+    switch (kpt) {
+        case 1: return launch_select<1, NW>(p, st);
+        case 2: return launch_select<2, NW>(p, st);
+        case 4: return launch_select<4, NW>(p, st);
+        case 8: return launch_select<8, NW>(p, st);
+        case 16: return launch_select<16, NW>(p, st);
+        case 32: return launch_select<32, NW>(p, st);
+        default: return launch_select<64, NW>(p, st);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t kvpack_version(void) { return KVPACK_VERSION; }
+
+const char *kvpack_status_string(kvpack_status s) {
+    switch (s) {
+        case KVPACK_OK: return "KVPACK_OK";
+        case KVPACK_ERR_INVALID_ARG: return "KVPACK_ERR_INVALID_ARG";
+        case KVPACK_ERR_ALIGNMENT: return "KVPACK_ERR_ALIGNMENT";
+        case KVPACK_ERR_UNSUPPORTED: return "KVPACK_ERR_UNSUPPORTED";
+        case KVPACK_ERR_WORKSPACE: return "KVPACK_ERR_WORKSPACE";
+        case KVPACK_ERR_CUDA: return "KVPACK_ERR_CUDA";
+        case KVPACK_ERR_NOCONVERGE: return "KVPACK_ERR_NOCONVERGE";
+        case KVPACK_ERR_TIMEOUT: return "KVPACK_ERR_TIMEOUT";
+    }
+    return "KVPACK_ERR_UNKNOWN";
+}
+
+kvpack_status kvpack_last_device_status(void *stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KVPACK_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, kvpack::g_error_word, sizeof(v)) != cudaSuccess) return KVPACK_ERR_CUDA;
+    if (cudaMemcpyToSymbol(kvpack::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return KVPACK_ERR_CUDA;
+    return static_cast<kvpack_status>(v);
+}
+
+kvpack_status kvpack_footprint(const kvpack_dims *d, int32_t n_layers, int32_t L_text, uint64_t out[3]) {
+    kvpack_status s = check_dims(d, n_layers);
+    if (s != KVPACK_OK) return s;
+    if (out == nullptr || L_text < 0) return KVPACK_ERR_INVALID_ARG;
+    const uint64_t units = (uint64_t)n_units(d, n_layers);
+    const uint64_t T = (uint64_t)d->T_vis, L = (uint64_t)L_text, n = KVPACK_GROUP * KVPACK_HEAD_DIM;
+    out[0] = units * (T + L) * n * 2 * 2;
+    out[1] = units * (T * KVPACK_RANK * 2 * 2 + L * n * 2 * 2);
+    out[2] = units * (uint64_t)KVPACK_RANK * n * 2 * 2;
+    return KVPACK_OK;
+}
+
+// ------------------------------------------------------------------ decode
+
+size_t kvpack_decode_workspace(const kvpack_dims *d, int32_t n_layers) {
+    if (check_dims(d, n_layers) != KVPACK_OK) return 0;
+    return plan_decode(d, n_layers).total;
+}
+
+kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const uint16_t *q,
+                                 const uint16_t *CK_lo, const uint16_t *CK_hi, const uint16_t *BK,
+                                 const uint16_t *CV_lo, const uint16_t *CV_hi, const uint16_t *BV,
+                                 const uint16_t *K_text, const uint16_t *V_text, int32_t L_text,
+                                 const uint32_t *mask, float softmax_scale, uint16_t *out, float *mass,
+                                 void *ws, size_t ws_bytes, void *stream) {
+    kvpack_status s = check_dims(d, n_layers);
+    if (s != KVPACK_OK) return s;
+    if (L_text < 0 || L_text > d->L_text_cap) return KVPACK_ERR_INVALID_ARG;
+    if (!q || !CK_lo || !CK_hi || !BK || !CV_lo || !CV_hi || !BV || !mask || !out) return KVPACK_ERR_INVALID_ARG;
+    if (L_text > 0 && (!K_text || !V_text)) return KVPACK_ERR_INVALID_ARG;
+    if (!(softmax_scale == softmax_scale) || softmax_scale <= 0.f) return KVPACK_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, mask, out, mass, ws,
+                          L_text > 0 ? K_text : nullptr, L_text > 0 ? V_text : nullptr};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KVPACK_ERR_ALIGNMENT;
+    const DecodePlan pl = plan_decode(d, n_layers);
+    if (ws == nullptr || ws_bytes < pl.total) return KVPACK_ERR_WORKSPACE;
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != KVPACK_OK) return s;
+
+    kvpack::decode::Params p{};
+    p.q = q; p.CK_lo = CK_lo; p.CK_hi = CK_hi; p.BK = BK; p.CV_lo = CV_lo; p.CV_hi = CV_hi; p.BV = BV;
+    p.Kt = K_text; p.Vt = V_text; p.mask = mask; p.out = out; p.mass = mass;
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    p.qt = reinterpret_cast<uint16_t *>(w + pl.off_qt);
+    p.part = reinterpret_cast<float *>(w + pl.off_part);
+    p.arrive = reinterpret_cast<unsigned int *>(w + pl.off_arrive);
+    p.n_units = pl.units; p.T = d->T_vis; p.L = L_text; p.Lcap = d->L_text_cap;
+    p.Hg = pl.Hg; p.per_kv = d->n_q_heads / d->n_kv_heads; p.n_q = d->n_q_heads;
+    p.groups = d->n_kv_heads / KVPACK_GROUP; p.S = pl.S; p.tps = pl.tps;
+    p.txs = (L_text + pl.S - 1) / pl.S;
+    p.txs = (p.txs + kvpack::decode::kTextTokens - 1) / kvpack::decode::kTextTokens * kvpack::decode::kTextTokens;
+    p.n_items = pl.units * pl.S;
+    p.nwords = (d->T_vis + 31) / 32;
+    p.scale2 = softmax_scale * 1.4426950408889634f;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    kvpack::decode::qproj_kernel<<<pl.units, 256, 0, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
+
+    const int blocks = di->attn_blocks[pl.nmb - 1] * di->sms;
+    const int grid = p.n_items < blocks ? p.n_items : blocks;
+    if (pl.S > grid) return KVPACK_ERR_UNSUPPORTED;   // every split of a unit must be co-resident
+    void *args[] = {&p};
+    cudaError_t e;
+    if (pl.nmb == 1) {
+        const size_t sm = sizeof(kvpack::decode::Smem<1>);
+        if (pl.S > 1)
+            e = cudaLaunchCooperativeKernel((const void *)kvpack::decode::attn_kernel<1>, dim3(grid),
+                                            dim3(kvpack::decode::kThreads), args, sm, st);
+        else {
+            kvpack::decode::attn_kernel<1><<<grid, kvpack::decode::kThreads, sm, st>>>(p);
+            e = cudaGetLastError();
+        }
+    } else {
+        const size_t sm = sizeof(kvpack::decode::Smem<2>);
+        if (pl.S > 1)
+            e = cudaLaunchCooperativeKernel((const void *)kvpack::decode::attn_kernel<2>, dim3(grid),
+                                            dim3(kvpack::decode::kThreads), args, sm, st);
+        else {
+            kvpack::decode::attn_kernel<2><<<grid, kvpack::decode::kThreads, sm, st>>>(p);
+            e = cudaGetLastError();
+        }
+    }
+    return (e == cudaSuccess) ? KVPACK_OK : KVPACK_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ select
+
+kvpack_status kvpack_select(const kvpack_dims *d, int32_t n_layers, const float *mass, float *score, float alpha,
+                            int32_t k_hi, uint32_t *mask_out, void *stream) {
+    kvpack_status s = check_dims(d, n_layers);
+    if (s != KVPACK_OK) return s;
+    if (!mass || !mask_out) return KVPACK_ERR_INVALID_ARG;
+    if (k_hi < 0 || k_hi > d->T_vis) return KVPACK_ERR_INVALID_ARG;
+    if (!(alpha >= 0.f && alpha < 1.f)) return KVPACK_ERR_INVALID_ARG;
+    if (alpha != 0.f && score == nullptr) return KVPACK_ERR_INVALID_ARG;
+    if (!aligned16(mass) || !aligned16(mask_out) || (score && !aligned16(score))) return KVPACK_ERR_ALIGNMENT;
+    kvpack::select::Params p{};
+    p.mass = mass; p.score = score; p.alpha = alpha; p.k = k_hi; p.T = d->T_vis;
+    p.nwords = (d->T_vis + 31) / 32; p.n_units = n_units(d, n_layers); p.mask = mask_out;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    const int T = d->T_vis;
+    if (T <= 32 * 64) {
+        int kpt = 1;
+        while (32 * kpt < T) kpt <<= 1;
+        e = select_dispatch<1>(kpt, p, st);
+    } else {
+        int kpt = 1;
+        while (1024 * kpt < T) kpt <<= 1;
+        e = select_dispatch<32>(kpt, p, st);
+    }
+    return (e == cudaSuccess) ? KVPACK_OK : KVPACK_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ compress
+
+size_t kvpack_compress_workspace(const kvpack_dims *d, int32_t n_layers) {
+    if (check_dims(d, n_layers) != KVPACK_OK) return 0;
+    return kvpack::compress::workspace_bytes(n_units(d, n_layers), d->T_vis);
+}
+
+kvpack_status kvpack_compress(const kvpack_dims *d, int32_t n_layers, const uint16_t *X, uint16_t *C_lo,
+                              uint16_t *C_hi, uint16_t *B, float *sigma, void *ws, size_t ws_bytes, void *stream) {
+    kvpack_status s = check_dims(d, n_layers);
+    if (s != KVPACK_OK) return s;
+    if (!X || !C_lo || !C_hi || !B) return KVPACK_ERR_INVALID_ARG;
+    const void *ptrs[] = {X, C_lo, C_hi, B, sigma, ws};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KVPACK_ERR_ALIGNMENT;
+    const int units = n_units(d, n_layers);
+    if (ws == nullptr || ws_bytes < kvpack::compress::workspace_bytes(units, d->T_vis)) return KVPACK_ERR_WORKSPACE;
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != KVPACK_OK) return s;
+    return kvpack::compress::run(units, d->T_vis, X, C_lo, C_hi, B, sigma, ws, di->sms,
+                                 static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
