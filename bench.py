@@ -1,0 +1,457 @@
+"""Benchmark of the compressed-KV decode step on B200 (one JSON line on rank 0).
+
+A step is one decode step of every unit of every layer of the workload:
+kvpack_select (rank mask from the previous step's attention mass) followed by
+kvpack_decode_attn (rank-space scores, split-T online softmax, V-coefficient
+sum, projection through B_V, uncompressed text tail, attention mass).  The
+text tail grows by one token per step.  The compressed cache is synthetic
+(seeded; shapes of the LLaVA-1.5-7B-style workload by default) and resident
+in HBM; every step reads far more than the 126 MB L2, so no flush is needed.
+
+    python bench.py [--gpus N --steps K --warmup W] [--config C1] [--hi-frac 0.25]
+    python bench.py --impl reference ...      # the fp64 CPU oracle on a bounded sample
+
+Multi-GPU (torchrun, one process per GPU): every rank decodes its own batch of
+the workload (independent units, no collective on the data path); the step
+time is the max over ranks and value counts the units of all ranks.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from synth import cases  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+POOL = 8   # distinct host-generated units tiled over the cache
+
+
+# ------------------------------------------------------------------ accounting
+
+def step_bytes(w: synth.Workload, L_text: int, k_hi: int) -> int:
+    """Algorithmic HBM bytes of one step (select + decode), all units:
+    coefficients at each token's rank (K and V), both bases, the text tail,
+    q and out, the mask, the mass written by decode and read by select, the
+    new mask written by select."""
+    T, Hg = w.T, w.Hg
+    per_unit = ((k_hi * 64 + (T - k_hi) * 16) * 2 * 2
+                + 2 * 64 * 512 * 2
+                + L_text * 512 * 2 * 2
+                + 2 * Hg * 128 * 2
+                + ((T + 31) // 32) * 4 * 2
+                + T * 4 * 2)
+    return per_unit * w.units
+
+
+def decode_bytes(w: synth.Workload, L_text: int, k_hi: int) -> int:
+    """Algorithmic bytes of kvpack_decode_attn alone (everything above but select's mass read and mask write)."""
+    T = w.T
+    return step_bytes(w, L_text, k_hi) - w.units * (T * 4 + ((T + 31) // 32) * 4)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            mp = json.load(f)
+        return float(mp["hbm_gbs"]), float(mp["bf16_tflops"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback (profiling recipe)"
+
+
+def recorded_traffic(kernel: str, config: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    ent = rec.get(f"{kernel}:{config}")
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "rank_compressed_kv_b200", "csrc", ent["source"])
+    try:
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return ent["bytes_per_launch"] if digest == ent["sha256_16"] else None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="kvpack_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", str(self.dev)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), reasons=parts[4:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        active = set()
+        for r in rows:
+            for n, v in zip(names, r["reasons"][1:]):
+                if v.lower().startswith("active"):
+                    active.add(n)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(active), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def build_cache(kv, torch, w: synth.Workload, Lcap: int, dev):
+    """Device-resident compressed cache of the whole workload: POOL host-generated
+    units (seeded, per the workload's recipe) tiled over all units."""
+    U, T = w.units, w.T
+    pool = [cases.unit_inputs(w, 0, i % w.batch, i % w.groups, T, Lcap, mask="ones") for i in range(POOL)]
+
+    def tile(key, shape, sl=None):
+        arr = np.stack([p[key] if sl is None else p[key][..., sl] for p in pool])
+        src = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).to(dev)
+        full = torch.empty((U,) + shape, dtype=torch.int16, device=dev)
+        reps = U // POOL
+        full[:reps * POOL].view(reps, POOL, *shape).copy_(src.unsqueeze(0).expand(reps, *src.shape))
+        if U % POOL:
+            full[reps * POOL:].copy_(src[:U % POOL])
+        return full.view(torch.bfloat16)
+
+    c = {}
+    c["CK_lo"] = tile("CK", (T, 16), slice(0, 16))
+    c["CK_hi"] = tile("CK", (T, 48), slice(16, 64))
+    c["CV_lo"] = tile("CV", (T, 16), slice(0, 16))
+    c["CV_hi"] = tile("CV", (T, 48), slice(16, 64))
+    c["BK"] = tile("BK", (64, 512))
+    c["BV"] = tile("BV", (64, 512))
+    c["K_text"] = tile("K_text", (Lcap, 4, 128))
+    c["V_text"] = tile("V_text", (Lcap, 4, 128))
+    return c
+
+
+def run_ours(args, w: synth.Workload, rank: int, world: int):
+    import torch
+    import rank_compressed_kv_b200 as kv
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    K, W = args.steps, args.warmup
+    T, L0 = w.T, w.text0
+    Lcap = L0 + W + K + 1
+    k_hi = w.k_hi
+    dims = kv.Dims(batch=w.batch, n_q_heads=w.n_q, n_kv_heads=w.n_kv, T_vis=T, L_text_cap=Lcap)
+    n_layers = w.layers
+    c = build_cache(kv, torch, w, Lcap, dev)
+    NQ = 4
+    q_host = [torch.from_numpy(np.stack([synth.query(w, l, b, s) for l in range(n_layers) for b in range(w.batch)])
+                               .view(np.int16)).view(torch.bfloat16).pin_memory() for s in range(NQ)]
+    q_dev = [qh.to(dev) for qh in q_host]
+    out = torch.empty(n_layers * w.batch, w.n_q, 128, dtype=torch.bfloat16, device=dev)
+    out_host = torch.empty_like(out, device="cpu").pin_memory()
+    mass = torch.zeros(w.units, T, dtype=torch.float32, device=dev)
+    nwords = (T + 31) // 32
+    mask = torch.empty(w.units, nwords, dtype=torch.int32, device=dev)
+    mask.copy_(torch.from_numpy(synth.all_ones_mask(T).view(np.int32)).to(dev).unsqueeze(0).expand(w.units, nwords))
+    ws = torch.empty(kv.decode_workspace(dims, n_layers), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def decode(step, q):
+        kv.decode_attn(dims, n_layers, q, c["CK_lo"], c["CK_hi"], c["BK"], c["CV_lo"], c["CV_hi"], c["BV"],
+                       c["K_text"], c["V_text"], L0 + step, mask, 1.0, out, mass, ws)
+
+    def step_fn(step, q):
+        kv.select(dims, n_layers, mass, None, 0.0, k_hi, mask)
+        decode(step, q)
+
+    # step 0: all tokens at full rank (no previous mass), then warm-up steps
+    decode(0, q_dev[0])
+    for s in range(1, W + 1):
+        step_fn(s, q_dev[s % NQ])
+    torch.cuda.synchronize()
+
+    # device-resident timed region: events per decode launch and around the whole run
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    ev0.record(stream)
+    for i in range(K):
+        s = W + 1 + i
+        kv.select(dims, n_layers, mass, None, 0.0, k_hi, mask)
+        ev_dec[i][0].record(stream)
+        decode(s, q_dev[s % NQ])
+        ev_dec[i][1].record(stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop()
+    st = kv.last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {kv.STATUS_NAMES[st]} during the timed region")
+    ms_total = ev0.elapsed_time(ev1)
+    dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
+    if dist:
+        t = torch.tensor([ms_total, sum(dec_ms)], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total, dec_sum = float(t[0]), float(t[1])
+    else:
+        dec_sum = sum(dec_ms)
+    ms_step = ms_total / K
+    value = world * w.batch / (ms_step / 1e3)
+
+    # end-to-end through the public API with host buffers: q from pinned host memory in,
+    # the step's output back to pinned host memory, every step
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        s = W + 1 + K + i
+        qd = q_dev[0]
+        qd.copy_(q_host[s % NQ], non_blocking=True)
+        kv.select(dims, n_layers, mass, None, 0.0, k_hi, mask)
+        kv.decode_attn(dims, n_layers, qd, c["CK_lo"], c["CK_hi"], c["BK"], c["CV_lo"], c["CV_hi"], c["BV"],
+                       c["K_text"], c["V_text"], min(L0 + s, Lcap), mask, 1.0, out, mass, ws)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / K
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_value = world * w.batch / (e2e_ms / 1e3)
+    qbytes = q_host[0].numel() * 2
+    obytes = out.numel() * 2
+
+    # roofline of the dominant launch (kvpack_decode_attn), algorithmic bytes per launch
+    hbm, _, peak_kind = measured_peaks()
+    L_mean = L0 + W + 1 + (K - 1) / 2.0
+    dbytes = decode_bytes(w, L_mean, k_hi)
+    dec_avg_ms = dec_sum / K
+    achieved = dbytes / (dec_avg_ms / 1e3) / 1e9
+    sbytes = step_bytes(w, L_mean, k_hi)
+    line = {
+        "metric": "compressed-KV decode attn query-tokens/s and achieved HBM GB/s vs 8 TB/s peak",
+        "value": round(value, 1),
+        "unit": "query-tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded low-rank-plus-noise compressed cache, 8 generated units tiled)",
+        "config": {"workload": f"{w.name}: batch {w.batch} x {w.layers} layers, {w.n_q} q / {w.n_kv} kv heads, "
+                               f"T={T} visual + {L0}+step text, r=64/16, top {int(w.hi_frac * 100)}% full rank",
+                   "global_batch": world * w.batch, "units": w.units, "hi_frac": w.hi_frac,
+                   "parallelism": f"dp{world}" if world > 1 else "single-gpu",
+                   "l2": "inputs larger than L2 (no flush needed)",
+                   "step": "kvpack_select + kvpack_decode_attn over all layers"},
+        "step_bytes": int(sbytes),
+        "step_GBps": round(sbytes / (ms_step / 1e3) / 1e9, 1),
+        "roofline": {"bound": "hbm", "kernel": "kvpack_decode_attn (qproj_kernel + attn_kernel)",
+                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "frac_of_8TBps": round(achieved / 8000.0, 4),
+                     "peak_kind": peak_kind,
+                     "bytes_per_launch": int(dbytes), "avg_launch_ms": round(dec_avg_ms, 4),
+                     "traffic": recorded_traffic("decode", w.name)},
+        "e2e": {"value": round(e2e_value, 1), "unit": "query-tokens/s", "h2d_bytes_per_step": qbytes,
+                "d2h_bytes_per_step": obytes, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": 3 * K,
+        "clocks": clk,
+        "wall_s_timed": round(wall, 3),
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
+    if args.compress and rank == 0:
+        line["compress"] = bench_compress(kv, torch, w, dev)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+def bench_compress(kv, torch, w, dev):
+    return None
+
+
+# ------------------------------------------------------------------ oracle (CPU) arm
+
+def _oracle_inputs(w: synth.Workload, n_units: int, L_text: int):
+    import oracle
+    f = oracle.bf16_to_f64
+    pool = [cases.unit_inputs(w, 0, i % w.batch, i % w.groups, w.T, L_text, mask="random") for i in range(POOL)]
+    idx = [i % POOL for i in range(n_units)]
+    q = np.stack([synth.query(w, 0, i % w.batch, 0)[: w.Hg] for i in range(POOL)])
+    return dict(
+        CK=f(np.stack([pool[i]["CK"] for i in idx])), BK=f(np.stack([pool[i]["BK"] for i in idx])),
+        CV=f(np.stack([pool[i]["CV"] for i in idx])), BV=f(np.stack([pool[i]["BV"] for i in idx])),
+        Kt=f(np.stack([pool[i]["K_text"] for i in idx])), Vt=f(np.stack([pool[i]["V_text"] for i in idx])),
+        mask=np.stack([pool[i]["mask"] for i in idx]), q=f(np.stack([q[i] for i in idx])),
+    )
+
+
+def _oracle_step(inp, k_hi, mass_prev):
+    import oracle
+    mask, _ = oracle.select(mass_prev, k_hi)
+    out, mass = oracle.decode(inp["CK"], inp["BK"], inp["CV"], inp["BV"], inp["Kt"], inp["Vt"], mask, inp["q"])
+    return mass.astype(np.float32)
+
+
+def cpu_baseline(w: synth.Workload, budget_s: float = 15.0):
+    """The oracle as it stands (fp64 decompress-then-attend + fp32 top-k), OpenMP over
+    units on the host cores, on a bounded sample of the workload's units; the metric
+    is extrapolated to a full step of all units."""
+    import oracle
+    L = w.text0
+    probe = _oracle_inputs(w, 2 * oracle.num_threads(), L)
+    m0 = np.random.default_rng(0).random((probe["CK"].shape[0], w.T)).astype(np.float32)
+    t0 = time.perf_counter()
+    _oracle_step(probe, w.k_hi, m0)
+    per_unit = (time.perf_counter() - t0) / probe["CK"].shape[0]
+    n = int(max(oracle.num_threads(), min(w.units, 2048, budget_s / max(per_unit, 1e-6))))
+    n = max(oracle.num_threads(), (n // oracle.num_threads()) * oracle.num_threads())
+    inp = _oracle_inputs(w, n, L)
+    m0 = np.random.default_rng(1).random((n, w.T)).astype(np.float32)
+    t0 = time.perf_counter()
+    _oracle_step(inp, w.k_hi, m0)
+    el = time.perf_counter() - t0
+    step_s = el * w.units / n
+    return {"value": round(w.batch / step_s, 3), "unit": "query-tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{n} of {w.units} units of one step (select + decode, fp64), {el:.1f} s, extrapolated"}
+
+
+def run_reference(args, w: synth.Workload):
+    """--impl reference: the fp64 CPU oracle timed on the host cores, each step a bounded
+    sample of the workload's units, extrapolated to the full step."""
+    import oracle
+    K, W = args.steps, args.warmup
+    threads = oracle.num_threads()
+    # size the per-step sample so that W + K steps take about args.cpu_seconds in total
+    probe = _oracle_inputs(w, 2 * threads, w.text0)
+    m0 = np.random.default_rng(0).random((probe["CK"].shape[0], w.T)).astype(np.float32)
+    t0 = time.perf_counter()
+    _oracle_step(probe, w.k_hi, m0)
+    per_unit = (time.perf_counter() - t0) / probe["CK"].shape[0]
+    n = int(args.cpu_seconds / max(per_unit, 1e-6) / (K + W))
+    n = max(threads, min(w.units, 2048, (n // threads) * threads))
+    inp = _oracle_inputs(w, n, w.text0)
+    mass = np.random.default_rng(1).random((n, w.T)).astype(np.float32)
+    for _ in range(W):
+        mass = _oracle_step(inp, w.k_hi, mass)
+    t0 = time.perf_counter()
+    for _ in range(K):
+        mass = _oracle_step(inp, w.k_hi, mass)
+    el = time.perf_counter() - t0
+    step_s = el / K * w.units / n
+    value = w.batch / step_s
+    sample = f"{n} of {w.units} units per step (select + decode, fp64), extrapolated to the full step"
+    return {
+        "impl": "reference",
+        "metric": "compressed-KV decode attn query-tokens/s and achieved HBM GB/s vs 8 TB/s peak",
+        "value": round(value, 4), "unit": "query-tokens/s", "n_gpus": 1, "steps": K, "warmup": W,
+        "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.batch, "units": w.units},
+        "cpu_baseline": {"value": round(value, 4), "unit": "query-tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "query-tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="C1", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--hi-frac", type=float, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--compress", action="store_true", help="also time kvpack_compress on the workload")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = synth.WORKLOADS[args.config]
+    if args.hi_frac is not None:
+        w = w.with_hi_frac(args.hi_frac)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus != world and args.impl == "ours":
+        ap.error(f"--gpus {args.gpus} needs one process per GPU: launch with torchrun --nproc-per-node {args.gpus}")
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return
+    line = run_ours(args, w, rank, world)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

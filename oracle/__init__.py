@@ -53,8 +53,14 @@ def lib():
         L.ora_decode_units.argtypes = [_i64, _i64, _i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        _dp, _dp, _dp, _dp, _dp, _dp, _u32p, _dp, ctypes.c_double, _dp, _dp]
         L.ora_select_units.argtypes = [_i64, _i64, _fp, _fp, ctypes.c_float, _i64, _u32p]
+        L.ora_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle runs on."""
+    return int(lib().ora_num_threads())
 
 
 def _ptr(a, t):

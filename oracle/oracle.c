@@ -31,6 +31,7 @@
  * an integer (which bit of the rank mask is set).
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -413,3 +414,6 @@ int ora_compress_units(int64_t n_units, const double *X, int64_t T, int n, int r
     }
     return worst;
 }
+
+/* Threads the OpenMP loops above use (reported next to any timing of the oracle). */
+int ora_num_threads(void) { return omp_get_max_threads(); }
