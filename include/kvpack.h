@@ -142,6 +142,43 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *dims, int32_t n_layers,
                                  uint16_t *out, float *mass,
                                  void *ws, size_t ws_bytes, void *stream);
 
+/* ---------------------------------------------------- decode step, no allocation
+ * kvpack_decode_attn_noalloc -- the same decode step as kvpack_decode_attn,
+ * for callers that cannot hand the library any device memory of their own:
+ * for example a plugin or custom operator hosted by a framework that owns
+ * all device memory and offers no workspace hook, or a serving loop that
+ * forbids allocator calls after start-up because cudaMalloc and cudaFree
+ * can stall on device-wide synchronisation.  This entry point has no
+ * counterpart in the paper; it only changes where the scratch lives.
+ *
+ * The scratch (rank-space queries, per-split partial results and arrival
+ * counters) is a fixed array of KVPACK_NOALLOC_SCRATCH_BYTES compiled into
+ * the library as device memory.  Every GPU that loads the library holds
+ * that array until the process exits.  The call itself allocates nothing
+ * and calls no allocating routine.
+ *
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and sets the kernels'
+ *   attributes; make that first call before any stream capture.
+ * - A call whose kvpack_decode_workspace(dims, n_layers) exceeds
+ *   KVPACK_NOALLOC_SCRATCH_BYTES returns KVPACK_ERR_WORKSPACE and launches
+ *   nothing; split the layers over several calls instead.
+ * - All calls on a device share the one array, and it keeps the last call's
+ *   contents.  The kernels rewrite every part they read, and clear the
+ *   arrival counters themselves before use.  Calls that overlap on the GPU
+ *   (two streams, or two threads with their own streams) race on the array
+ *   and give wrong results: order them on one stream or with events.
+ * Arguments and results are those of kvpack_decode_attn minus ws / ws_bytes.
+ */
+#define KVPACK_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+kvpack_status kvpack_decode_attn_noalloc(const kvpack_dims *dims, int32_t n_layers,
+                                         const uint16_t *q,
+                                         const uint16_t *CK_lo, const uint16_t *CK_hi, const uint16_t *BK,
+                                         const uint16_t *CV_lo, const uint16_t *CV_hi, const uint16_t *BV,
+                                         const uint16_t *K_text, const uint16_t *V_text, int32_t L_text,
+                                         const uint32_t *mask, float softmax_scale,
+                                         uint16_t *out, float *mass, void *stream);
+
 /* ------------------------------------------------------------------ rank choice
  * kvpack_select -- importance update and rank mask for the next step, every
  * unit of n_layers layers (Methodologie 2.B on the fr page: a moving average,

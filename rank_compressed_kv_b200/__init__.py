@@ -24,6 +24,8 @@ from ._lib import (  # noqa: F401
     compress,
     compress_workspace,
     decode_attn,
+    decode_attn_noalloc,
+    NOALLOC_SCRATCH_BYTES,
     decode_workspace,
     footprint,
     last_device_status,

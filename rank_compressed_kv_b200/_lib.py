@@ -79,6 +79,9 @@ _L.kvpack_decode_workspace.restype = _sz
 _L.kvpack_decode_attn.argtypes = [_dims_p, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
                                   ctypes.c_float, _vp, _vp, _vp, _sz, _vp]
 _L.kvpack_decode_attn.restype = ctypes.c_int
+_L.kvpack_decode_attn_noalloc.argtypes = [_dims_p, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
+                                          _vp, ctypes.c_float, _vp, _vp, _vp]
+_L.kvpack_decode_attn_noalloc.restype = ctypes.c_int
 _L.kvpack_select.argtypes = [_dims_p, _i32, _vp, _vp, ctypes.c_float, _i32, _vp, _vp]
 _L.kvpack_select.restype = ctypes.c_int
 
@@ -147,6 +150,18 @@ def decode_attn(dims: Dims, n_layers: int, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV
                                  _ptr(CV_lo), _ptr(CV_hi), _ptr(BV), _ptr(K_text), _ptr(V_text), L_text,
                                  _ptr(mask), float(scale), _ptr(out), _ptr(mass), _ptr(ws), _nbytes(ws),
                                  _stream(stream)), "kvpack_decode_attn")
+
+
+def decode_attn_noalloc(dims: Dims, n_layers: int, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, K_text, V_text,
+                        L_text: int, mask, scale: float, out, mass, stream=None):
+    """decode_attn with the library's built-in scratch, for callers that cannot allocate device memory."""
+    _check(_L.kvpack_decode_attn_noalloc(ctypes.byref(dims.c()), n_layers, _ptr(q), _ptr(CK_lo), _ptr(CK_hi),
+                                         _ptr(BK), _ptr(CV_lo), _ptr(CV_hi), _ptr(BV), _ptr(K_text), _ptr(V_text),
+                                         L_text, _ptr(mask), float(scale), _ptr(out), _ptr(mass), _stream(stream)),
+           "kvpack_decode_attn_noalloc")
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 def select(dims: Dims, n_layers: int, mass, score, alpha: float, k_hi: int, mask_out, stream=None):

@@ -241,6 +241,57 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     return (e == cudaSuccess) ? KVPACK_OK : KVPACK_ERR_CUDA;
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------------ decode without allocation
+//
+// For callers that cannot give the library device memory (a framework-owned
+// plugin with no workspace hook, a serving loop that bans allocator calls):
+// the decode scratch lives in this fixed device array, which every GPU that
+// loads the library holds until exit.  Host code must not pass the array's
+// name to a kernel -- on the host it is only a stand-in -- so its device
+// address is looked up once per device and cached.
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KVPACK_NOALLOC_SCRATCH_BYTES];
+
+void *g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// First call on a device: look the array up with that device current.
+kvpack_status noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVPACK_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KVPACK_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return KVPACK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvpack_status kvpack_decode_attn_noalloc(const kvpack_dims *d, int32_t n_layers, const uint16_t *q,
+                                         const uint16_t *CK_lo, const uint16_t *CK_hi, const uint16_t *BK,
+                                         const uint16_t *CV_lo, const uint16_t *CV_hi, const uint16_t *BV,
+                                         const uint16_t *K_text, const uint16_t *V_text, int32_t L_text,
+                                         const uint32_t *mask, float softmax_scale, uint16_t *out, float *mass,
+                                         void *stream) {
+    kvpack_status s = check_dims(d, n_layers);
+    if (s != KVPACK_OK) return s;
+    if (plan_decode(d, n_layers).total > KVPACK_NOALLOC_SCRATCH_BYTES) return KVPACK_ERR_WORKSPACE;
+    void *ws = nullptr;
+    if ((s = noalloc_scratch(&ws)) != KVPACK_OK) return s;
+    return kvpack_decode_attn(d, n_layers, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, K_text, V_text, L_text, mask,
+                              softmax_scale, out, mass, ws, KVPACK_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 // ------------------------------------------------------------------ select
 
 kvpack_status kvpack_select(const kvpack_dims *d, int32_t n_layers, const float *mass, float *score, float alpha,
