@@ -118,6 +118,17 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float x) {
     return *reinterpret_cast<uint16_t *>(&v);
 }
 
+// Split an fp32 pair into bf16 hi and lo pairs (x = hi + lo to ~2^-16 relative).
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+    const float r0 = x0 - __bfloat162float(h0), r1 = x1 - __bfloat162float(h1);
+    __nv_bfloat162 hv;
+    hv.x = h0;
+    hv.y = h1;
+    hi = *reinterpret_cast<uint32_t *>(&hv);
+    lo = pack_bf16(r0, r1);
+}
+
 // Named barrier over the first `threads` threads of the block (id != 0).
 __device__ __forceinline__ void named_bar(int id, int threads) {
     asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(threads) : "memory");

@@ -75,15 +75,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
 
-// split an fp32 pair into bf16 hi and lo pairs (x = hi + lo to ~2^-16 relative)
-__device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
-    const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-    const float r0 = x0 - __bfloat162float(h0), r1 = x1 - __bfloat162float(h1);
-    __nv_bfloat162 hv; hv.x = h0; hv.y = h1;
-    hi = *reinterpret_cast<uint32_t *>(&hv);
-    lo = pack_bf16(r0, r1);
-}
-
 // ================================================================== Gram (mma.sync)
 
 constexpr int kGramThreads = 256;

@@ -10,29 +10,34 @@
 // softmax-weighted V coefficients are summed in rank space and projected back
 // through B_V once per head.  K and V are never materialised.
 //
-// Kernels
-//   qproj_kernel  one block per unit: q~ for the unit's Hg heads, stored as a
-//                 bf16 pair (hi + lo) so that the score MMA keeps ~16
-//                 significant bits of q~; also clears the unit's arrival count.
-//   attn_kernel   persistent; work item = (unit, split of the visual tokens and
-//                 of the text tail).  Warp 8 is the producer: it walks the
-//                 item's tokens and stages them into a 6-slot ring with
-//                 cp.async (16-byte copies), one mbarrier pair per slot:
-//                   LO   128 (or 64) tokens' 32-byte C_lo rows of K and V
-//                   HI   32 full-rank tokens: C_lo + C_hi rows (128 B) of K and V
-//                   TEXT 16 text tokens of one KV head: 256-byte K and V rows
-//                 Warps 0-7 consume: mma.sync m16n8k16 bf16 with heads on M,
-//                 tokens on N; online softmax in registers; P re-used from the
-//                 score accumulators as the A operand of the value MMA.  A
-//                 token with its mask bit set is scored in the HI stream at
-//                 rank 64 and excluded (logit -inf) from the LO stream.
-//                 Logits are kept on chip (fp32) for the attention mass.
-//                 When a unit has S > 1 splits, the splits publish
-//                 (max, sum, u, w) per head, count arrivals on a per-unit
-//                 counter and wait (bounded) for their siblings; then each
-//                 split writes the mass of its own tokens and the outputs of
-//                 the heads h with h % S == split.
+// attn_kernel is persistent (one 288-thread block per SM).  A work item is a
+// unit's split of the visual tokens and of the text tail.  Warp 8 produces:
+// it stages the item into a 6-slot shared-memory ring (8 KB per slot, a
+// full / empty mbarrier pair per slot):
+//   Q     the unit's query rows (cp.async)
+//   BK    32 rows of B_K for one KV head (TMA, 128-byte swizzle)
+//   QDONE barrier: q~ complete
+//   LO    128 (Hg <= 16) or 64 tokens' 32-byte C_lo rows of K and V (TMA, 32-byte swizzle)
+//   HI    32 full-rank tokens: C_lo + C_hi rows of K and V gathered with cp.async
+//   TEXT  16 text tokens of one KV head, K and V (TMA, 128-byte swizzle)
+//   END   the item's tokens are done
+//   BV    32 rows of B_V for one KV head (TMA)
+//   FIN   outputs complete
+// Warps 0-7 consume.  q~ = q B_K^T by mma.sync from the BK stages, kept as a
+// bf16 hi + lo pair (~16 significant bits).  Scores and values run on
+// mma.sync m16n8k16 (bf16 in, fp32 accumulate) with heads on M and tokens on
+// N; the online softmax stays in registers and P is reused from the score
+// accumulators as the A operand of the value MMA.  A token with its mask bit
+// set is scored at rank 64 in the HI stream and gets logit -inf in the LO
+// stream (rank 16).  Logits stay in shared memory for the attention mass.
+// When a unit has S > 1 splits, each split publishes (max, sum) and (u, w)
+// per head, counts itself on a per-unit counter and waits (bounded) for its
+// siblings; a static round-robin schedule on a cooperative launch keeps the
+// wait deadlock-free.  Split s then writes the mass of its own tokens and the
+// outputs of heads h with h % S == s, projecting u through B_V.
 #pragma once
+
+#include <cuda.h>
 
 #include "common.cuh"
 
@@ -42,14 +47,17 @@ namespace decode {
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
-constexpr int kStages = 6;
+constexpr int kStages = 11;
 constexpr int kStageBytes = 8192;
 constexpr int kHiTokens = 32;
 constexpr int kTextTokens = 16;
 constexpr int kMaxHeads = 32;
-constexpr int kPartFloats = 196;     // per (unit, split, head): m, l, pad2, u[64], w[128]
+constexpr int kUW = 192;              // per (unit, split, head): u[64] then w[128]
 
-enum : int { ST_QT = 0, ST_Q = 1, ST_LO = 2, ST_HI = 3, ST_TEXT = 4, ST_END = 5, ST_STOP = 6 };
+enum : int {
+    ST_Q = 0, ST_BK = 1, ST_QDONE = 2, ST_LO = 3, ST_HI = 4, ST_TEXT = 5, ST_END = 6, ST_BV = 7, ST_FIN = 8,
+    ST_STOP = 9
+};
 
 template <int NMB>
 struct Cfg {
@@ -57,7 +65,7 @@ struct Cfg {
     static constexpr int kWPM = kConsumerWarps / NMB; // consumer warps per 16-head block
     static constexpr int kLoT = 16 * kWPM;            // tokens per LO stage
     static constexpr int kLS = kMRows + 4;            // logits row stride (floats), bank-conflict free
-    static constexpr int kTPS = (NMB == 1) ? 1536 : 832;  // max visual tokens per split
+    static constexpr int kTPS = (NMB == 1) ? 1024 : 512;  // max visual tokens per split
 };
 
 struct StageHdr {
@@ -70,34 +78,46 @@ static_assert(sizeof(StageHdr) == 128, "stage header size");
 
 template <int NMB>
 struct Smem {
-    alignas(128) unsigned char ring[kStages][kStageBytes];
+    alignas(1024) unsigned char ring[kStages][kStageBytes];
     StageHdr hdr[kStages];
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t hbar[kStages];     // header published (1 arrival): warps that skip a stage need only this
+    uint64_t full[kStages];     // header and data landed
+    uint64_t empty[kStages];    // every consumer warp is done with the slot
     uint64_t cbar;                                  // consumer-wide barrier (bounded waits)
-    alignas(128) uint16_t qa[2][kMaxHeads][64];     // q~ hi / lo, 128-byte rows, 16-B chunks XOR-swizzled
-    alignas(128) uint16_t qtxt[4][16][128];         // q rows of each KV head, 256-byte rows, swizzled
-    float acc_u[kMaxHeads][64];
-    float acc_w[kMaxHeads][128];
+    union {
+        struct {   // while an item's tokens stream
+            alignas(128) uint16_t qa[2][kMaxHeads][64];   // q~ hi / lo, 128-byte rows, 16-B chunks XOR-swizzled
+            alignas(128) uint16_t qtxt[4][16][128];       // q rows of each KV head, 256-byte rows, swizzled
+        };
+        struct {   // in the item's epilogue: block-wide sums in register order (bank-conflict-free atomics)
+            float frag_u[2][32][32];                      // [head block][register][lane]
+            float frag_w[4][32][32];                      // [KV head][register][lane]
+        };
+    };
+    float acc_u[kMaxHeads][64];                     // u / l of the unit (rank space)
+    float acc_w[kMaxHeads][128];                    // w / l of the unit (text part)
     float acc_l[kMaxHeads];
     float mcta[kMaxHeads];
     float mfin[kMaxHeads];
     float invl[kMaxHeads];
     float wmax_v[kConsumerWarps][16];
     float wmax_t[kConsumerWarps][16];
-    float ucomb[2][64];
     uint16_t hi_pend[kHiTokens + 128];
+    uint32_t mask_words[Cfg<NMB>::kTPS / 32];    // producer's copy of the item's rank-mask words
     int abort;
     alignas(16) float logits[Cfg<NMB>::kTPS * Cfg<NMB>::kLS];
 };
 
 struct Params {
-    const uint16_t *q, *CK_lo, *CK_hi, *BK, *CV_lo, *CV_hi, *BV, *Kt, *Vt;
+    CUtensorMap tm_ck, tm_cv;    // C_lo planes of K and V: 2D [units*T][16], box {16, LoT}, 32-byte swizzle
+    CUtensorMap tm_kt, tm_vt;    // text tails: 3D [units*Lcap][4][128], box {64, 1, 16}, 128-byte swizzle
+    CUtensorMap tm_bk, tm_bv;    // bases: 2D [units*64][512], box {64, 32}, 128-byte swizzle
+    const uint16_t *q, *CK_lo, *CK_hi, *CV_lo, *CV_hi;
     const uint32_t *mask;
     uint16_t *out;
     float *mass;
-    uint16_t *qt;            // workspace: [units][2][Hg][64] bf16 q~ (hi, lo)
-    float *part;             // workspace: [units][S][Hg][kPartFloats]
+    float *ml;               // workspace: [units][S][Hg][2]  (max, sum) of each split
+    float *uw;               // workspace: [units][S][Hg][kUW] (u, w) of each split
     unsigned int *arrive;    // workspace: [units]
     int n_units, T, L, Lcap, Hg, per_kv, n_q, groups, S, tps, txs, n_items, nwords;
     float scale2;            // softmax scale * log2(e)
@@ -109,47 +129,39 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// ------------------------------------------------------------------ qproj
+// -------------------------------------------------------------- TMA helpers
 
-__global__ void __launch_bounds__(256) qproj_kernel(Params p) {
-    __shared__ float qs[kMaxHeads][128];
-    const int unit = blockIdx.x;
-    const int lb = unit / p.groups, G = unit % p.groups;
-    const uint16_t *qsrc = p.q + ((size_t)lb * p.n_q + (size_t)G * p.Hg) * 128;
-    for (int i = threadIdx.x; i < p.Hg * 128; i += blockDim.x) qs[i >> 7][i & 127] = bf16_bits_to_float(qsrc[i]);
-    if (threadIdx.x == 0) p.arrive[unit] = 0u;
-    __syncthreads();
-    const uint16_t *bk = p.BK + (size_t)unit * 64 * 512;
-    uint16_t *dst = p.qt + (size_t)unit * 2 * p.Hg * 64;
-    for (int o = threadIdx.x; o < p.Hg * 64; o += blockDim.x) {
-        const int h = o >> 6, i = o & 63;
-        float acc = 0.f;
-        {
-            const int j = h / p.per_kv;
-            const uint4 *row = reinterpret_cast<const uint4 *>(bk + (size_t)i * 512 + j * 128);
-            #pragma unroll 4
-            for (int c = 0; c < 16; ++c) {
-                uint4 v = __ldg(row + c);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    acc = fmaf(__uint_as_float(w[e] << 16), qs[h][8 * c + 2 * e], acc);
-                    acc = fmaf(__uint_as_float(w[e] & 0xffff0000u), qs[h][8 * c + 2 * e + 1], acc);
-                }
-            }
-        }
-        const uint16_t hi = float_to_bf16_bits(acc);
-        const uint16_t lo = float_to_bf16_bits(acc - bf16_bits_to_float(hi));
-        dst[o] = hi;
-        dst[p.Hg * 64 + o] = lo;
-    }
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void tma_2d(void *dst, const CUtensorMap *tm, int c0, int c1, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tma_3d(void *dst, const CUtensorMap *tm, int c0, int c1, int c2, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// byte offset of element (row, col) of a 128-byte-swizzled box of 64 bf16 per row
+__device__ __forceinline__ uint32_t sw128(int row, int col) {
+    return row * 128 + ((((col >> 3) ^ (row & 7)) & 7) << 4) + (col & 7) * 2;
 }
 
 // -------------------------------------------------------------- helpers
 
-// Consumer-wide barrier on an mbarrier (count = kConsumers) with a bounded wait.
+// Consumer-wide barrier on an mbarrier (one arrival per consumer warp, after a
+// warp-level sync that orders the warp's earlier shared-memory writes) with a
+// bounded wait.
 __device__ __forceinline__ void csync(uint64_t *bar, uint32_t &phase, volatile int *abort) {
-    mbar_arrive(bar);
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+    __syncwarp();   // no lane polls before lane 0 has arrived
     mbar_wait(bar, phase, abort);
     phase ^= 1u;
 }
@@ -195,6 +207,14 @@ __device__ __forceinline__ void zero16(void *dst) {
     *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
 }
 
+// Heads of this split's output: h % S == split.  Bit j of the result is set if
+// a head of KV head j is among them.
+__device__ __forceinline__ int output_kv_heads(const Params &p, int split) {
+    int m = 0;
+    for (int h = split; h < p.Hg; h += p.S) m |= 1 << (h / p.per_kv);
+    return m;
+}
+
 // ---------------------------------------------------------------- producer
 
 template <int NMB>
@@ -202,14 +222,18 @@ __device__ void producer(const Params &p, Smem<NMB> &sm, int lane) {
     using C = Cfg<NMB>;
     uint32_t seq = 0;
     auto acquire = [&]() -> int {
+        __syncwarp();   // lane 0's arrivals and copy issues of the previous stage are done
         const int slot = seq % kStages;
         const uint32_t k = seq / kStages;
         if (!mbar_wait(&sm.empty[slot], (k & 1u) ^ 1u, &sm.abort)) return -1;
         return slot;
     };
-    auto commit = [&](int slot) {
-        cp_async_arrive(&sm.full[slot]);
-        mbar_arrive(&sm.full[slot]);
+    // arrivals: lane 0 announces the TMA bytes (0 for none); lanes that issued cp.async
+    // copies arrive again when those land
+    auto commit = [&](int slot, uint32_t tma_bytes, bool used_cp_async) {
+        if (used_cp_async) cp_async_arrive(&sm.full[slot]);
+        if (lane == 0 && tma_bytes) mbar_arrive_tx(&sm.full[slot], tma_bytes);
+        else mbar_arrive(&sm.full[slot]);
         ++seq;
     };
     auto header = [&](int slot, int type, int item, int base, int n, int aux, int aux2) {
@@ -217,6 +241,13 @@ __device__ void producer(const Params &p, Smem<NMB> &sm, int lane) {
             StageHdr &h = sm.hdr[slot];
             h.type = type; h.item = item; h.base = base; h.n = n; h.aux = aux; h.aux2 = aux2;
         }
+    };
+    auto bar_of = [&](int slot) { return &sm.full[slot]; };
+    // the header (and any per-stage fields the lanes wrote) becomes visible to the consumers
+    auto publish = [&](int slot) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.hbar[slot]);
+        __syncwarp();
     };
 
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
@@ -226,32 +257,53 @@ __device__ void producer(const Params &p, Smem<NMB> &sm, int lane) {
         const size_t ubase = (size_t)unit * p.T;
         int slot;
 
-        // q~ (bf16 hi and lo parts, 2 x Hg x 128 B)
-        if ((slot = acquire()) < 0) break;
-        header(slot, ST_QT, item, 0, 0, 0, 0);
-        {
-            const unsigned char *src = reinterpret_cast<const unsigned char *>(p.qt + (size_t)unit * 2 * p.Hg * 64);
-            for (int c = lane; c < p.Hg * 16; c += 32) cp_async16(sm.ring[slot] + 16 * c, src + 16 * c);
+        // rank-mask words of this split, once per item
+        for (int i = lane; i < (t1 - t0 + 31) / 32; i += 32) {
+            const int widx = t0 / 32 + i;
+            sm.mask_words[i] = (widx < p.nwords) ? p.mask[(size_t)unit * p.nwords + widx] : 0u;
         }
-        commit(slot);
+        __syncwarp();
 
-        // q rows of the unit's heads (Hg x 256 B)
+        // query rows of the unit's heads (Hg x 256 B)
         if ((slot = acquire()) < 0) break;
         header(slot, ST_Q, item, 0, 0, 0, 0);
+        publish(slot);
         {
             const uint16_t *src = p.q + ((size_t)(unit / p.groups) * p.n_q + (size_t)(unit % p.groups) * p.Hg) * 128;
             for (int c = lane; c < p.Hg * 16; c += 32) cp_async16(sm.ring[slot] + 16 * c, src + 8 * c);
         }
-        commit(slot);
+        commit(slot, 0, true);
+
+        // B_K, 32 rank rows of one KV head per stage
+        bool ok = true;
+        for (int j = 0; j < 4 && ok; ++j)
+            for (int sub = 0; sub < 2; ++sub) {
+                if ((slot = acquire()) < 0) { ok = false; break; }
+                header(slot, ST_BK, item, 0, 0, j, sub);
+                publish(slot);
+                if (lane == 0) {
+                    mbar_arrive_tx(bar_of(slot), kStageBytes);
+                    tma_2d(sm.ring[slot], &p.tm_bk, j * 128, unit * 64 + 32 * sub, bar_of(slot));
+                    tma_2d(sm.ring[slot] + 4096, &p.tm_bk, j * 128 + 64, unit * 64 + 32 * sub, bar_of(slot));
+                } else {
+                    mbar_arrive(bar_of(slot));
+                }
+                ++seq;
+            }
+        if (!ok) break;
+        if ((slot = acquire()) < 0) break;
+        header(slot, ST_QDONE, item, 0, 0, 0, 0);
+        publish(slot);
+        commit(slot, 0, false);
 
         // visual tokens: LO tiles, HI stages of 32 pending full-rank tokens
-        int npend = 0, hi_count = 0, lo_count = 0;
-        bool ok = true;
+        int npend = 0, hi_count = 0;
         auto emit_hi = [&](int cnt) -> bool {
             int s2 = acquire();
             if (s2 < 0) return false;
             header(s2, ST_HI, item, t0, cnt, hi_count, 0);
             for (int i = lane; i < cnt; i += 32) sm.hdr[s2].tok[i] = sm.hi_pend[i];
+            publish(s2);
             unsigned char *dk = sm.ring[s2];
             unsigned char *dv = sm.ring[s2] + 4096;
             for (int idx = lane; idx < kHiTokens * 8; idx += 32) {
@@ -271,7 +323,7 @@ __device__ void producer(const Params &p, Smem<NMB> &sm, int lane) {
                     zero16(dv + r * 128 + pos);
                 }
             }
-            commit(s2);
+            commit(s2, 0, true);
             ++hi_count;
             return true;
         };
@@ -279,34 +331,26 @@ __device__ void producer(const Params &p, Smem<NMB> &sm, int lane) {
         for (int tb = t0; tb < t1 && ok; tb += C::kLoT) {
             const int n = min(C::kLoT, t1 - tb);
             if ((slot = acquire()) < 0) { ok = false; break; }
-            header(slot, ST_LO, item, tb, n, lo_count, 0);
-            // mask words of this tile (bits of tokens past n cleared)
+            header(slot, ST_LO, item, tb, n, 0, 0);
             uint32_t word = 0u;
             const int nw = C::kLoT / 32;
             if (lane < nw) {
                 const int widx = tb / 32 + lane;
-                word = (widx < p.nwords) ? p.mask[(size_t)unit * p.nwords + widx] : 0u;
+                word = (widx < p.nwords) ? sm.mask_words[widx - t0 / 32] : 0u;
                 const int lo_tok = 32 * lane;
                 if (lo_tok >= n) word = 0u;
                 else if (n - lo_tok < 32) word &= (1u << (n - lo_tok)) - 1u;
                 sm.hdr[slot].mask[lane] = word;
             }
-            unsigned char *dk = sm.ring[slot];
-            unsigned char *dv = sm.ring[slot] + 4096;
-            for (int idx = lane; idx < C::kLoT * 2; idx += 32) {
-                const int r = idx >> 1, ch = idx & 1;
-                const int pos = (ch ^ ((r >> 2) & 1)) * 16;
-                if (r < n) {
-                    const size_t row = ubase + tb + r;
-                    cp_async16(dk + r * 32 + pos, p.CK_lo + row * 16 + ch * 8);
-                    cp_async16(dv + r * 32 + pos, p.CV_lo + row * 16 + ch * 8);
-                } else {
-                    zero16(dk + r * 32 + pos);
-                    zero16(dv + r * 32 + pos);
-                }
+            publish(slot);
+            if (lane == 0) {
+                mbar_arrive_tx(bar_of(slot), C::kLoT * 64);
+                tma_2d(sm.ring[slot], &p.tm_ck, 0, (int)(ubase + tb), bar_of(slot));
+                tma_2d(sm.ring[slot] + 4096, &p.tm_cv, 0, (int)(ubase + tb), bar_of(slot));
+            } else {
+                mbar_arrive(bar_of(slot));
             }
-            commit(slot);
-            ++lo_count;
+            ++seq;
 
             // append the tile's full-rank tokens (split-relative) to the pending list
             const int cnt = __popc(word);
@@ -356,33 +400,56 @@ __device__ void producer(const Params &p, Smem<NMB> &sm, int lane) {
             for (int j = 0; j < 4; ++j) {
                 if ((slot = acquire()) < 0) { ok = false; break; }
                 header(slot, ST_TEXT, item, ct, n, j, tt);
-                unsigned char *dk = sm.ring[slot];
-                unsigned char *dv = sm.ring[slot] + 4096;
-                for (int idx = lane; idx < kTextTokens * 16; idx += 32) {
-                    const int r = idx >> 4, ch = idx & 15;
-                    const int pos = (ch ^ (r & 7)) * 16;
-                    if (r < n) {
-                        const size_t row = (((size_t)unit * p.Lcap + ct + r) * 4 + j) * 128;
-                        cp_async16(dk + r * 256 + pos, p.Kt + row + ch * 8);
-                        cp_async16(dv + r * 256 + pos, p.Vt + row + ch * 8);
-                    } else {
-                        zero16(dk + r * 256 + pos);
-                        zero16(dv + r * 256 + pos);
-                    }
+                publish(slot);
+                if (lane == 0) {
+                    const int row = unit * p.Lcap + ct;
+                    mbar_arrive_tx(bar_of(slot), kStageBytes);
+                    tma_3d(sm.ring[slot], &p.tm_kt, 0, j, row, bar_of(slot));
+                    tma_3d(sm.ring[slot] + 2048, &p.tm_kt, 64, j, row, bar_of(slot));
+                    tma_3d(sm.ring[slot] + 4096, &p.tm_vt, 0, j, row, bar_of(slot));
+                    tma_3d(sm.ring[slot] + 6144, &p.tm_vt, 64, j, row, bar_of(slot));
+                } else {
+                    mbar_arrive(bar_of(slot));
                 }
-                commit(slot);
+                ++seq;
             }
         }
         if (!ok) break;
 
         if ((slot = acquire()) < 0) break;
         header(slot, ST_END, item, 0, 0, 0, 0);
-        commit(slot);
+        publish(slot);
+        commit(slot, 0, false);
+
+        // B_V rows of the KV heads this split writes outputs for
+        const int jm = output_kv_heads(p, split);
+        for (int j = 0; j < 4 && ok; ++j) {
+            if (!((jm >> j) & 1)) continue;
+            for (int sub = 0; sub < 2; ++sub) {
+                if ((slot = acquire()) < 0) { ok = false; break; }
+                header(slot, ST_BV, item, 0, 0, j, sub);
+                publish(slot);
+                if (lane == 0) {
+                    mbar_arrive_tx(bar_of(slot), kStageBytes);
+                    tma_2d(sm.ring[slot], &p.tm_bv, j * 128, unit * 64 + 32 * sub, bar_of(slot));
+                    tma_2d(sm.ring[slot] + 4096, &p.tm_bv, j * 128 + 64, unit * 64 + 32 * sub, bar_of(slot));
+                } else {
+                    mbar_arrive(bar_of(slot));
+                }
+                ++seq;
+            }
+        }
+        if (!ok) break;
+        if ((slot = acquire()) < 0) break;
+        header(slot, ST_FIN, item, 0, 0, 0, 0);
+        publish(slot);
+        commit(slot, 0, false);
     }
     int slot = acquire();
     if (slot >= 0) {
         header(slot, ST_STOP, -1, 0, 0, 0, 0);
-        commit(slot);
+        publish(slot);
+        commit(slot, 0, false);
     }
     cp_async_wait_all();
 }
@@ -400,10 +467,8 @@ __device__ void consumers(const Params &p, Smem<NMB> &sm, int warp, int lane) {
     volatile int *abort = &sm.abort;
     uint32_t cphase = 0;
 
-    // visual softmax state (rows g, g+8 of block mb) and rank-space accumulator u^T
-    float vm[2], vl[2], u[8][4];
-    // text softmax state (rows g, g+8 of KV head jt) and head-space accumulator w^T
-    float tm[2], tl[2], w[16][4];
+    float vm[2], vl[2], u[8][4];          // visual softmax state, u^T accumulator (rank space)
+    float tm[2], tl[2], w[16][4];         // text softmax state, w^T accumulator (head space)
     uint32_t qah[4], qal[4];              // q~ A fragments, rank 0..15 (hi / lo)
 
     auto reset_state = [&]() {
@@ -414,51 +479,99 @@ __device__ void consumers(const Params &p, Smem<NMB> &sm, int warp, int lane) {
         #pragma unroll
         for (int a = 0; a < 16; ++a) w[a][0] = w[a][1] = w[a][2] = w[a][3] = 0.f;
     };
+    auto clear_acc = [&]() {
+        if (ctid < kMaxHeads) sm.acc_l[ctid] = 0.f;
+    };
     reset_state();
-    for (int i = ctid; i < kMaxHeads * 64; i += kConsumers) (&sm.acc_u[0][0])[i] = 0.f;
-    for (int i = ctid; i < kMaxHeads * 128; i += kConsumers) (&sm.acc_w[0][0])[i] = 0.f;
-    if (ctid < kMaxHeads) sm.acc_l[ctid] = 0.f;
+    clear_acc();
     csync(&sm.cbar, cphase, abort);
 
     const uint32_t qa_base[2] = {smem_u32(&sm.qa[0][0][0]), smem_u32(&sm.qa[1][0][0])};
     int item = -1, unit = 0, split = 0, t0 = 0, t1 = 0;
+    int held_slot = -1;       // first B_V stage of a pair, kept until the second arrives
 
     for (uint32_t seq = 0;; ++seq) {
         const int slot = seq % kStages;
         const uint32_t k = seq / kStages;
-        const bool ok = mbar_wait(&sm.full[slot], k & 1u, abort);
+        __syncwarp();   // every lane is past the previous stage's release
+        const bool hok = mbar_wait(&sm.hbar[slot], k & 1u, abort);
         const StageHdr &hd = sm.hdr[slot];
-        const int type = ok ? hd.type : ST_STOP;
+        int type = hok ? hd.type : ST_STOP;
+        // does this warp read the stage's data?  Stages it skips are released without
+        // waiting for their data to land.
+        bool mine = true;
+        if (type == ST_BK) mine = warp == ((2 * hd.aux + hd.aux2) & 7);
+        else if (type == ST_BV) mine = (warp >> 1) == hd.aux;
+        else if (type == ST_TEXT) mine = warp == 4 * (hd.aux2 & 1) + hd.aux;
+        else if (type == ST_HI) mine = ((win - 2 * hd.aux) % C::kWPM + C::kWPM) % C::kWPM < 2;
+        if (type != ST_STOP && mine && !mbar_wait(&sm.full[slot], k & 1u, abort)) type = ST_STOP;
         const unsigned char *st = sm.ring[slot];
         const uint32_t sbase = smem_u32(st);
 
-        if (type == ST_QT) {
+        if (type == ST_Q) {
             item = hd.item;
             unit = item / p.S; split = item % p.S;
             t0 = split * p.tps; t1 = min(p.T, t0 + p.tps);
-            for (int c = ctid; c < 512; c += kConsumers) {
-                const int part = c >> 8, row = (c >> 3) & 31, ch = c & 7;
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (row < p.Hg) v = *reinterpret_cast<const uint4 *>(st + (part * p.Hg + row) * 128 + 16 * ch);
-                *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(&sm.qa[part][row][0]) + ((ch ^ (row & 7)) << 4)) = v;
-            }
-            csync(&sm.cbar, cphase, abort);
-            const int row = 16 * mb + (lane & 7) + (((lane >> 3) & 1) << 3);
-            const int ch = lane >> 4;
-            const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
-            ldsm_x4(qa_base[0] + off, qah[0], qah[1], qah[2], qah[3]);
-            ldsm_x4(qa_base[1] + off, qal[0], qal[1], qal[2], qal[3]);
-        } else if (type == ST_Q) {
             for (int c = ctid; c < 4 * 16 * 16; c += kConsumers) {
                 const int j = c >> 8, rr = (c >> 4) & 15, ch = c & 15;
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
                 if (rr < p.per_kv) v = *reinterpret_cast<const uint4 *>(st + (j * p.per_kv + rr) * 256 + 16 * ch);
                 *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(&sm.qtxt[j][rr][0]) + ((ch ^ (rr & 7)) << 4)) = v;
             }
+            for (int i = ctid; i < 2 * kMaxHeads * 64 / 8; i += kConsumers) zero16(reinterpret_cast<uint4 *>(&sm.qa[0][0][0]) + i);
             csync(&sm.cbar, cphase, abort);
+        } else if (type == ST_BK) {
+            // q~[h][32 sub + n] = sum_d q_h[d] B_K[32 sub + n][128 j + d] for the heads of KV head j
+            const int j = hd.aux, sub = hd.aux2;
+            if (warp == ((2 * j + sub) & 7)) {
+                const uint32_t qb = smem_u32(&sm.qtxt[j][0][0]);
+                float acc[4][4];
+                #pragma unroll
+                for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = acc[a][2] = acc[a][3] = 0.f;
+                #pragma unroll
+                for (int kb = 0; kb < 8; ++kb) {
+                    uint32_t a[4];
+                    {
+                        const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
+                        const int ch = 2 * kb + (lane >> 4);
+                        ldsm_x4(qb + row * 256 + ((ch ^ (row & 7)) << 4), a[0], a[1], a[2], a[3]);
+                    }
+                    #pragma unroll
+                    for (int np = 0; np < 2; ++np) {
+                        uint32_t b0, b1, b2, b3;
+                        const int row = 16 * np + (lane & 7) + ((lane >> 4) << 3);
+                        const int c = 2 * kb + ((lane >> 3) & 1);
+                        ldsm_x4(sbase + (c >> 3) * 4096 + row * 128 + ((((c & 7) ^ (row & 7))) << 4), b0, b1, b2, b3);
+                        mma_bf16(acc[2 * np], a, b0, b1);
+                        mma_bf16(acc[2 * np + 1], a, b2, b3);
+                    }
+                }
+                #pragma unroll
+                for (int nb = 0; nb < 4; ++nb)
+                    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int rr = g + 8 * (e >> 1);
+                        if (rr < p.per_kv) {
+                            const int h = j * p.per_kv + rr;
+                            const int i = 32 * sub + 8 * nb + 2 * tig + (e & 1);
+                            const float v = acc[nb][e];
+                            const uint16_t hi = float_to_bf16_bits(v);
+                            const uint16_t lo = float_to_bf16_bits(v - bf16_bits_to_float(hi));
+                            const uint32_t off = ((((i >> 3) ^ (h & 7)) & 7) << 4) + (i & 7) * 2;
+                            *reinterpret_cast<uint16_t *>(reinterpret_cast<unsigned char *>(&sm.qa[0][h][0]) + off) = hi;
+                            *reinterpret_cast<uint16_t *>(reinterpret_cast<unsigned char *>(&sm.qa[1][h][0]) + off) = lo;
+                        }
+                    }
+            }
+        } else if (type == ST_QDONE) {
+            csync(&sm.cbar, cphase, abort);
+            const int row = 16 * mb + (lane & 7) + (((lane >> 3) & 1) << 3);
+            const int ch = lane >> 4;
+            const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
+            ldsm_x4(qa_base[0] + off, qah[0], qah[1], qah[2], qah[3]);
+            ldsm_x4(qa_base[1] + off, qal[0], qal[1], qal[2], qal[3]);
         } else if (type == ST_LO) {
             const int base = hd.base, n = hd.n;
-            // scores S^T[h, t] for 16 heads x 16 tokens at rank 0..15
             uint32_t b0, b1, b2, b3;
             {
                 const int row = win * 16 + (lane & 7) + ((lane >> 4) << 3);
@@ -572,8 +685,8 @@ __device__ void consumers(const Params &p, Smem<NMB> &sm, int warp, int lane) {
                     }
                     {
                         const int row = (lane & 7) + ((lane >> 4) << 3);
-                        const int ch = 2 * kb + ((lane >> 3) & 1);
-                        ldsm_x4(sbase + row * 256 + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
+                        const int c = 2 * kb + ((lane >> 3) & 1);
+                        ldsm_x4(sbase + (c >> 3) * 2048 + row * 128 + ((((c & 7) ^ (row & 7))) << 4), b0, b1, b2, b3);
                     }
                     mma_bf16(s[0], a, b0, b1);
                     mma_bf16(s[1], a, b2, b3);
@@ -593,20 +706,90 @@ __device__ void consumers(const Params &p, Smem<NMB> &sm, int warp, int lane) {
                 for (int pr = 0; pr < 8; ++pr) {
                     uint32_t b0, b1, b2, b3;
                     const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
-                    const int ch = 2 * pr + (lane >> 4);
-                    ldsm_x4_t(sbase + 4096 + row * 256 + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
+                    const int c = 2 * pr + (lane >> 4);
+                    ldsm_x4_t(sbase + 4096 + (c >> 3) * 2048 + row * 128 + ((((c & 7) ^ (row & 7))) << 4), b0, b1, b2, b3);
                     mma_bf16(w[2 * pr], pa, b0, b1);
                     mma_bf16(w[2 * pr + 1], pa, b2, b3);
+                }
+            }
+        } else if (type == ST_BV) {
+            // o_h = (u_h / l_h) B_V[:, 128 j + d] + w_h / l_h for the output heads of KV head j:
+            // warps 2j and 2j+1 take output columns [0, 64) and [64, 128); they keep the first of
+            // the two 32-row stages until the second arrives and run both through mma.sync
+            const int j = hd.aux, sub = hd.aux2;
+            if ((warp >> 1) == j) {
+                if (sub == 0) {
+                    held_slot = slot;
+                } else if (held_slot >= 0) {
+                    const int dh = warp & 1;
+                    const int h = j * p.per_kv + g;
+                    const bool valid = (g < p.per_kv) && (h % p.S == split);
+                    float o[8][4];
+                    #pragma unroll
+                    for (int a2 = 0; a2 < 8; ++a2) o[a2][0] = o[a2][1] = o[a2][2] = o[a2][3] = 0.f;
+                    #pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const uint32_t bbase = smem_u32(sm.ring[half == 0 ? held_slot : slot]) + dh * 4096;
+                        #pragma unroll
+                        for (int kb = 0; kb < 2; ++kb) {
+                            const int i0 = 32 * half + 16 * kb + 2 * tig;
+                            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                            if (valid) {
+                                a0 = sm.acc_u[h][i0]; a1 = sm.acc_u[h][i0 + 1];
+                                a2 = sm.acc_u[h][i0 + 8]; a3 = sm.acc_u[h][i0 + 9];
+                            }
+                            uint32_t ah[4], al[4];
+                            split2(a0, a1, ah[0], al[0]);
+                            split2(a2, a3, ah[2], al[2]);
+                            ah[1] = ah[3] = al[1] = al[3] = 0u;
+                            #pragma unroll
+                            for (int np = 0; np < 4; ++np) {
+                                uint32_t b0, b1, b2, b3;
+                                const int row = 16 * kb + (lane & 7) + (((lane >> 3) & 1) << 3);
+                                const int ch = 2 * np + (lane >> 4);
+                                ldsm_x4_t(bbase + row * 128 + ((((ch ^ (row & 7))) & 7) << 4), b0, b1, b2, b3);
+                                mma_bf16(o[2 * np], ah, b0, b1);
+                                mma_bf16(o[2 * np], al, b0, b1);
+                                mma_bf16(o[2 * np + 1], ah, b2, b3);
+                                mma_bf16(o[2 * np + 1], al, b2, b3);
+                            }
+                        }
+                    }
+                    if (valid) {
+                        const int lb = unit / p.groups, G = unit % p.groups;
+                        uint16_t *orow = p.out + ((size_t)lb * p.n_q + (size_t)G * p.Hg + h) * 128;
+                        #pragma unroll
+                        for (int nb = 0; nb < 8; ++nb) {
+                            const int d = 64 * dh + 8 * nb + 2 * tig;
+                            const uint32_t v = pack_bf16(o[nb][0] + sm.acc_w[h][d], o[nb][1] + sm.acc_w[h][d + 1]);
+                            *reinterpret_cast<uint32_t *>(orow + d) = v;
+                        }
+                    }
                 }
             }
         }
 
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.empty[slot]);
+        if (lane == 0) {
+            if (type == ST_BV && held_slot == slot) {
+                // released together with the second stage of the pair
+            } else {
+                mbar_arrive(&sm.empty[slot]);
+                if (type == ST_BV && held_slot >= 0 && held_slot != slot) mbar_arrive(&sm.empty[held_slot]);
+            }
+        }
+        if (type == ST_BV && held_slot >= 0 && held_slot != slot) held_slot = -1;
         if (type == ST_STOP) break;
+
+        if (type == ST_FIN) {
+            csync(&sm.cbar, cphase, abort);
+            clear_acc();
+            reset_state();
+            continue;
+        }
         if (type != ST_END) continue;
 
-        // ============================ epilogue of one work item
+        // ============================ epilogue of the item's tokens
         const int Hg = p.Hg;
         #pragma unroll
         for (int r = 0; r < 2; ++r) {
@@ -622,6 +805,8 @@ __device__ void consumers(const Params &p, Smem<NMB> &sm, int warp, int lane) {
             sm.wmax_t[warp][g + 8] = tm[1];
         }
         csync(&sm.cbar, cphase, abort);
+        // every warp is past its token stages: the q staging area is dead and becomes the merge buffer
+        for (int i = ctid; i < 6 * 32 * 32; i += kConsumers) (&sm.frag_u[0][0][0])[i] = 0.f;
         if (ctid < Hg) {
             const int h = ctid;
             float mx = -INFINITY;
@@ -633,48 +818,55 @@ __device__ void consumers(const Params &p, Smem<NMB> &sm, int warp, int lane) {
             sm.mcta[h] = mx;
         }
         csync(&sm.cbar, cphase, abort);
-        // rescale this warp's partials to the block maximum and add them up
+        // rescale this warp's partials to the block maximum and add them up in register order:
+        // one warp-wide atomic touches 32 consecutive words (no bank conflicts)
         #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const int h = 16 * mb + g + 8 * r;
-            if (h < Hg) {
-                const float mc = sm.mcta[h];
-                const float f = (vm[r] == -INFINITY) ? 0.f : ex2(vm[r] - mc);
-                #pragma unroll
-                for (int nb = 0; nb < 8; ++nb) {
-                    atomicAdd(&sm.acc_u[h][8 * nb + 2 * tig], u[nb][2 * r] * f);
-                    atomicAdd(&sm.acc_u[h][8 * nb + 2 * tig + 1], u[nb][2 * r + 1] * f);
-                }
-                if (tig == 0) atomicAdd(&sm.acc_l[h], vl[r] * f);
+            const float f = (h < Hg && vm[r] != -INFINITY) ? ex2(vm[r] - sm.mcta[h]) : 0.f;
+            #pragma unroll
+            for (int nb = 0; nb < 8; ++nb) {
+                atomicAdd(&sm.frag_u[mb][4 * nb + 2 * r][lane], u[nb][2 * r] * f);
+                atomicAdd(&sm.frag_u[mb][4 * nb + 2 * r + 1][lane], u[nb][2 * r + 1] * f);
             }
-            const int rr = g + 8 * r;
-            if (rr < p.per_kv) {
-                const int ht = jt * p.per_kv + rr;
-                const float mc = sm.mcta[ht];
-                const float f = (tm[r] == -INFINITY) ? 0.f : ex2(tm[r] - mc);
-                if (f != 0.f) {
-                    #pragma unroll
-                    for (int nb = 0; nb < 16; ++nb) {
-                        atomicAdd(&sm.acc_w[ht][8 * nb + 2 * tig], w[nb][2 * r] * f);
-                        atomicAdd(&sm.acc_w[ht][8 * nb + 2 * tig + 1], w[nb][2 * r + 1] * f);
-                    }
-                    if (tig == 0) atomicAdd(&sm.acc_l[ht], tl[r] * f);
-                }
+            if (tig == 0 && f != 0.f) atomicAdd(&sm.acc_l[h], vl[r] * f);
+        }
+        {
+            // text rows: KV head jt has per_kv <= 8 query heads, all in row g (r = 0)
+            const bool row_ok = g < p.per_kv;
+            const int ht = jt * p.per_kv + g;
+            const float f = (row_ok && tm[0] != -INFINITY) ? ex2(tm[0] - sm.mcta[ht]) : 0.f;
+            #pragma unroll
+            for (int nb = 0; nb < 16; ++nb) {
+                atomicAdd(&sm.frag_w[jt][2 * nb][lane], w[nb][0] * f);
+                atomicAdd(&sm.frag_w[jt][2 * nb + 1][lane], w[nb][1] * f);
             }
+            if (tig == 0 && f != 0.f) atomicAdd(&sm.acc_l[ht], tl[0] * f);
+        }
+        csync(&sm.cbar, cphase, abort);
+        // register order -> [head][column]
+        for (int i = ctid; i < Hg * 64; i += kConsumers) {
+            const int h = i >> 6, c = i & 63, hh = h & 15;
+            sm.acc_u[h][c] = sm.frag_u[h >> 4][4 * (c >> 3) + 2 * (hh >> 3) + (c & 1)][4 * (hh & 7) + ((c & 7) >> 1)];
+        }
+        for (int i = ctid; i < Hg * 128; i += kConsumers) {
+            const int h = i >> 7, d = i & 127;
+            const int j = h / p.per_kv, rr = h % p.per_kv;
+            sm.acc_w[h][d] = sm.frag_w[j][2 * (d >> 3) + (d & 1)][4 * rr + ((d & 7) >> 1)];
         }
         csync(&sm.cbar, cphase, abort);
 
         if (p.S > 1) {
-            float *mine = p.part + ((size_t)unit * p.S + split) * Hg * kPartFloats;
-            for (int i = ctid; i < Hg * kPartFloats; i += kConsumers) {
-                const int h = i / kPartFloats, f = i % kPartFloats;
-                float v;
-                if (f == 0) v = sm.mcta[h];
-                else if (f == 1) v = sm.acc_l[h];
-                else if (f < 4) v = 0.f;
-                else if (f < 68) v = sm.acc_u[h][f - 4];
-                else v = sm.acc_w[h][f - 68];
-                mine[i] = v;
+            // publish this split's (max, sum) and (u, w), then wait for the unit's other splits
+            float *mlu = p.ml + (size_t)unit * p.S * Hg * 2;
+            float *uwu = p.uw + (size_t)unit * p.S * Hg * kUW;
+            if (ctid < Hg) {
+                mlu[((size_t)split * Hg + ctid) * 2] = sm.mcta[ctid];
+                mlu[((size_t)split * Hg + ctid) * 2 + 1] = sm.acc_l[ctid];
+            }
+            for (int i = ctid; i < Hg * kUW; i += kConsumers) {
+                const int h = i / kUW, f = i % kUW;
+                uwu[(size_t)split * Hg * kUW + i] = (f < 64) ? sm.acc_u[h][f] : sm.acc_w[h][f - 64];
             }
             __threadfence();
             csync(&sm.cbar, cphase, abort);
@@ -691,27 +883,69 @@ __device__ void consumers(const Params &p, Smem<NMB> &sm, int warp, int lane) {
                         *abort = 1;
                         break;
                     }
-                    __nanosleep(256);
+                    __nanosleep(128);
                 }
             }
             csync(&sm.cbar, cphase, abort);
-            if (ctid < Hg) {
-                const int h = ctid;
-                const float *ph = p.part + (size_t)unit * p.S * Hg * kPartFloats + (size_t)h * kPartFloats;
-                float M = -INFINITY;
-                for (int s2 = 0; s2 < p.S; ++s2) M = fmaxf(M, __ldcg(ph + (size_t)s2 * Hg * kPartFloats));
-                float Lsum = 0.f;
-                for (int s2 = 0; s2 < p.S; ++s2) {
-                    const float ms = __ldcg(ph + (size_t)s2 * Hg * kPartFloats);
-                    if (ms != -INFINITY) Lsum += __ldcg(ph + (size_t)s2 * Hg * kPartFloats + 1) * ex2(ms - M);
+            // unit-wide max and sum per head: one warp per head, lanes over splits
+            for (int h = warp; h < Hg; h += kConsumerWarps) {
+                float mloc = -INFINITY;
+                for (int s2 = lane; s2 < p.S; s2 += 32) mloc = fmaxf(mloc, __ldcg(mlu + ((size_t)s2 * Hg + h) * 2));
+                #pragma unroll
+                for (int d = 16; d > 0; d >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, d));
+                float lsum = 0.f;
+                for (int s2 = lane; s2 < p.S; s2 += 32) {
+                    const float ms = __ldcg(mlu + ((size_t)s2 * Hg + h) * 2);
+                    if (ms != -INFINITY) lsum += __ldcg(mlu + ((size_t)s2 * Hg + h) * 2 + 1) * ex2(ms - mloc);
                 }
-                sm.mfin[h] = M;
-                sm.invl[h] = 1.f / Lsum;
+                #pragma unroll
+                for (int d = 16; d > 0; d >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, d);
+                if (lane == 0) {
+                    sm.mfin[h] = mloc;
+                    sm.invl[h] = 1.f / lsum;
+                }
+            }
+            csync(&sm.cbar, cphase, abort);
+            // combined u / l and w / l of this split's output heads, all (head, feature) pairs in parallel
+            const int n_out = (split < Hg) ? (Hg - split + p.S - 1) / p.S : 0;
+            for (int task = ctid; task < n_out * kUW; task += kConsumers) {
+                const int h = split + (task / kUW) * p.S, f = task % kUW;
+                const float mh = sm.mfin[h];
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                int s2 = 0;
+                for (; s2 + 4 <= p.S; s2 += 4) {
+                    const float m0 = __ldcg(mlu + ((size_t)(s2 + 0) * Hg + h) * 2);
+                    const float m1 = __ldcg(mlu + ((size_t)(s2 + 1) * Hg + h) * 2);
+                    const float m2 = __ldcg(mlu + ((size_t)(s2 + 2) * Hg + h) * 2);
+                    const float m3 = __ldcg(mlu + ((size_t)(s2 + 3) * Hg + h) * 2);
+                    const float x0 = __ldcg(uwu + ((size_t)(s2 + 0) * Hg + h) * kUW + f);
+                    const float x1 = __ldcg(uwu + ((size_t)(s2 + 1) * Hg + h) * kUW + f);
+                    const float x2 = __ldcg(uwu + ((size_t)(s2 + 2) * Hg + h) * kUW + f);
+                    const float x3 = __ldcg(uwu + ((size_t)(s2 + 3) * Hg + h) * kUW + f);
+                    if (m0 != -INFINITY) a0 = fmaf(x0, ex2(m0 - mh), a0);
+                    if (m1 != -INFINITY) a1 = fmaf(x1, ex2(m1 - mh), a1);
+                    if (m2 != -INFINITY) a2 = fmaf(x2, ex2(m2 - mh), a2);
+                    if (m3 != -INFINITY) a3 = fmaf(x3, ex2(m3 - mh), a3);
+                }
+                for (; s2 < p.S; ++s2) {
+                    const float m0 = __ldcg(mlu + ((size_t)s2 * Hg + h) * 2);
+                    const float x0 = __ldcg(uwu + ((size_t)s2 * Hg + h) * kUW + f);
+                    if (m0 != -INFINITY) a0 = fmaf(x0, ex2(m0 - mh), a0);
+                }
+                const float v = ((a0 + a1) + (a2 + a3)) * sm.invl[h];
+                if (f < 64) sm.acc_u[h][f] = v;
+                else sm.acc_w[h][f - 64] = v;
             }
         } else {
             if (ctid < Hg) {
                 sm.mfin[ctid] = sm.mcta[ctid];
                 sm.invl[ctid] = 1.f / sm.acc_l[ctid];
+            }
+            csync(&sm.cbar, cphase, abort);
+            for (int i = ctid; i < Hg * kUW; i += kConsumers) {
+                const int h = i / kUW, f = i % kUW;
+                if (f < 64) sm.acc_u[h][f] *= sm.invl[h];
+                else sm.acc_w[h][f - 64] *= sm.invl[h];
             }
         }
         csync(&sm.cbar, cphase, abort);
@@ -725,74 +959,25 @@ __device__ void consumers(const Params &p, Smem<NMB> &sm, int warp, int lane) {
                 p.mass[(size_t)unit * p.T + t] = acc;
             }
         }
-
-        // outputs of the heads assigned to this split, two heads at a time
-        {
-            const int lb = unit / p.groups, G = unit % p.groups;
-            const int half = ctid >> 7, d = ctid & 127;
-            const float *pu = p.part + (size_t)unit * p.S * Hg * kPartFloats;
-            for (int h0 = split; h0 < Hg; h0 += 2 * p.S) {
-                const int h = h0 + half * p.S;
-                const bool act = h < Hg;
-                // combined u (rank space) of head h into ucomb[half]
-                if (act && d < 64) {
-                    float uv;
-                    if (p.S == 1) {
-                        uv = sm.acc_u[h][d];
-                    } else {
-                        uv = 0.f;
-                        for (int s2 = 0; s2 < p.S; ++s2) {
-                            const float *ps = pu + ((size_t)s2 * Hg + h) * kPartFloats;
-                            const float ms = __ldcg(ps);
-                            if (ms != -INFINITY) uv += __ldcg(ps + 4 + d) * ex2(ms - sm.mfin[h]);
-                        }
-                    }
-                    sm.ucomb[half][d] = uv;
-                }
-                csync(&sm.cbar, cphase, abort);
-                if (act) {
-                    const int j = h / p.per_kv;
-                    float wv;
-                    if (p.S == 1) {
-                        wv = sm.acc_w[h][d];
-                    } else {
-                        wv = 0.f;
-                        for (int s2 = 0; s2 < p.S; ++s2) {
-                            const float *ps = pu + ((size_t)s2 * Hg + h) * kPartFloats;
-                            const float ms = __ldcg(ps);
-                            if (ms != -INFINITY) wv += __ldcg(ps + 68 + d) * ex2(ms - sm.mfin[h]);
-                        }
-                    }
-                    const uint16_t *bv = p.BV + (size_t)unit * 64 * 512 + j * 128 + d;
-                    float o = wv;
-                    #pragma unroll 8
-                    for (int i = 0; i < 64; ++i) o = fmaf(sm.ucomb[half][i], bf16_bits_to_float(__ldg(bv + (size_t)i * 512)), o);
-                    p.out[((size_t)lb * p.n_q + (size_t)G * Hg + h) * 128 + d] = float_to_bf16_bits(o * sm.invl[h]);
-                }
-                csync(&sm.cbar, cphase, abort);
-            }
-        }
-
-        // clear the block accumulators and the warp state for the next item
-        for (int i = ctid; i < kMaxHeads * 64; i += kConsumers) (&sm.acc_u[0][0])[i] = 0.f;
-        for (int i = ctid; i < kMaxHeads * 128; i += kConsumers) (&sm.acc_w[0][0])[i] = 0.f;
-        if (ctid < kMaxHeads) sm.acc_l[ctid] = 0.f;
-        reset_state();
-        csync(&sm.cbar, cphase, abort);
+        // the BV stages that follow add u B_V into acc_w; FIN writes the outputs
     }
 }
 
 template <int NMB>
-__global__ void __launch_bounds__(kThreads, 1) attn_kernel(Params p) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    Smem<NMB> &sm = *reinterpret_cast<Smem<NMB> *>(smem_raw);
+__global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ Params p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // the ring must start on a 1024-byte boundary (128-byte swizzle pattern)
+    const uint32_t base = smem_u32(smem_raw);
+    unsigned char *aligned = smem_raw + ((1024u - (base & 1023u)) & 1023u);
+    Smem<NMB> &sm = *reinterpret_cast<Smem<NMB> *>(aligned);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.hbar[s], 1);
             mbar_init(&sm.full[s], 32);
             mbar_init(&sm.empty[s], kConsumerWarps);
         }
-        mbar_init(&sm.cbar, kConsumers);
+        mbar_init(&sm.cbar, kConsumerWarps);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -800,6 +985,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(Params p) {
     if (warp == kConsumerWarps) producer<NMB>(p, sm, lane);
     else consumers<NMB>(p, sm, warp, lane);
 }
+
+template <int NMB>
+constexpr size_t smem_bytes() { return sizeof(Smem<NMB>) + 1024; }
 
 }  // namespace decode
 }  // namespace kvpack

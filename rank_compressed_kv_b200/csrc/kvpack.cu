@@ -5,6 +5,9 @@
 #include <cstring>
 #include <mutex>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "kvpack.h"
 #include "common.cuh"
 #include "decode.cuh"
@@ -43,7 +46,7 @@ inline int hg(const kvpack_dims *d) { return (d->n_q_heads / d->n_kv_heads) * KV
 
 struct DecodePlan {
     int nmb, S, tps, units, Hg;
-    size_t off_qt, off_part, off_arrive, total;
+    size_t off_ml, off_uw, off_arrive, total;
 };
 
 DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
@@ -57,10 +60,10 @@ DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
     pl.tps = (per + lot - 1) / lot * lot;
     pl.units = n_units(d, n_layers);
     size_t off = 0;
-    pl.off_qt = off;
-    off = align256(off + (size_t)pl.units * 2 * pl.Hg * 64 * sizeof(uint16_t));
-    pl.off_part = off;
-    if (pl.S > 1) off = align256(off + (size_t)pl.units * pl.S * pl.Hg * kvpack::decode::kPartFloats * sizeof(float));
+    pl.off_ml = off;
+    if (pl.S > 1) off = align256(off + (size_t)pl.units * pl.S * pl.Hg * 2 * sizeof(float));
+    pl.off_uw = off;
+    if (pl.S > 1) off = align256(off + (size_t)pl.units * pl.S * pl.Hg * kvpack::decode::kUW * sizeof(float));
     pl.off_arrive = off;
     off = align256(off + (size_t)pl.units * sizeof(unsigned int));
     pl.total = off;
@@ -82,7 +85,7 @@ kvpack_status device_info(DeviceInfo **out) {
     DeviceInfo &di = g_dev[dev];
     if (!di.ready) {
         if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return KVPACK_ERR_CUDA;
-        const int s1 = (int)sizeof(kvpack::decode::Smem<1>), s2 = (int)sizeof(kvpack::decode::Smem<2>);
+        const int s1 = (int)kvpack::decode::smem_bytes<1>(), s2 = (int)kvpack::decode::smem_bytes<2>();
         if (cudaFuncSetAttribute(kvpack::decode::attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1) != cudaSuccess)
             return KVPACK_ERR_CUDA;
         if (cudaFuncSetAttribute(kvpack::decode::attn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2) != cudaSuccess)
@@ -100,6 +103,33 @@ kvpack_status device_info(DeviceInfo **out) {
     }
     *out = &di;
     return KVPACK_OK;
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_encode_mu;
+
+kvpack_status tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000 *out) {
+    std::lock_guard<std::mutex> lk(g_encode_mu);
+    if (g_encode == nullptr) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return KVPACK_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    *out = g_encode;
+    return KVPACK_OK;
+}
+
+// bf16 tensor map of `rank` dims (innermost first), byte strides of dims 1.., box, swizzle
+bool encode_bf16(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const void *ptr, int rank,
+                 const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapSwizzle sw) {
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int KPT, int NW>
@@ -194,12 +224,41 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     DeviceInfo *di = nullptr;
     if ((s = device_info(&di)) != KVPACK_OK) return s;
 
-    kvpack::decode::Params p{};
-    p.q = q; p.CK_lo = CK_lo; p.CK_hi = CK_hi; p.BK = BK; p.CV_lo = CV_lo; p.CV_hi = CV_hi; p.BV = BV;
-    p.Kt = K_text; p.Vt = V_text; p.mask = mask; p.out = out; p.mass = mass;
+    PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+    if ((s = tensor_map_encoder(&enc)) != KVPACK_OK) return s;
+
+    kvpack::decode::Params p;
+    std::memset(&p, 0, sizeof(p));
+    const int lot = (pl.nmb == 1) ? kvpack::decode::Cfg<1>::kLoT : kvpack::decode::Cfg<2>::kLoT;
+    {
+        const cuuint64_t dims[2] = {16, (cuuint64_t)pl.units * d->T_vis};
+        const cuuint64_t strides[1] = {32};
+        const cuuint32_t box[2] = {16, (cuuint32_t)lot};
+        if (!encode_bf16(enc, &p.tm_ck, CK_lo, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B) ||
+            !encode_bf16(enc, &p.tm_cv, CV_lo, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B))
+            return KVPACK_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {512, (cuuint64_t)pl.units * 64};
+        const cuuint64_t strides[1] = {1024};
+        const cuuint32_t box[2] = {64, 32};
+        if (!encode_bf16(enc, &p.tm_bk, BK, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_bf16(enc, &p.tm_bv, BV, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return KVPACK_ERR_CUDA;
+    }
+    if (L_text > 0) {
+        const cuuint64_t dims[3] = {128, 4, (cuuint64_t)pl.units * d->L_text_cap};
+        const cuuint64_t strides[2] = {256, 1024};
+        const cuuint32_t box[3] = {64, 1, 16};
+        if (!encode_bf16(enc, &p.tm_kt, K_text, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_bf16(enc, &p.tm_vt, V_text, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return KVPACK_ERR_CUDA;
+    }
+    p.q = q; p.CK_lo = CK_lo; p.CK_hi = CK_hi; p.CV_lo = CV_lo; p.CV_hi = CV_hi;
+    p.mask = mask; p.out = out; p.mass = mass;
     unsigned char *w = static_cast<unsigned char *>(ws);
-    p.qt = reinterpret_cast<uint16_t *>(w + pl.off_qt);
-    p.part = reinterpret_cast<float *>(w + pl.off_part);
+    p.ml = reinterpret_cast<float *>(w + pl.off_ml);
+    p.uw = reinterpret_cast<float *>(w + pl.off_uw);
     p.arrive = reinterpret_cast<unsigned int *>(w + pl.off_arrive);
     p.n_units = pl.units; p.T = d->T_vis; p.L = L_text; p.Lcap = d->L_text_cap;
     p.Hg = pl.Hg; p.per_kv = d->n_q_heads / d->n_kv_heads; p.n_q = d->n_q_heads;
@@ -211,16 +270,15 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     p.scale2 = softmax_scale * 1.4426950408889634f;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    kvpack::decode::qproj_kernel<<<pl.units, 256, 0, st>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
-
     const int blocks = di->attn_blocks[pl.nmb - 1] * di->sms;
     const int grid = p.n_items < blocks ? p.n_items : blocks;
     if (pl.S > grid) return KVPACK_ERR_UNSUPPORTED;   // every split of a unit must be co-resident
+    if (pl.S > 1 && cudaMemsetAsync(p.arrive, 0, (size_t)pl.units * sizeof(unsigned int), st) != cudaSuccess)
+        return KVPACK_ERR_CUDA;
     void *args[] = {&p};
     cudaError_t e;
     if (pl.nmb == 1) {
-        const size_t sm = sizeof(kvpack::decode::Smem<1>);
+        const size_t sm = kvpack::decode::smem_bytes<1>();
         if (pl.S > 1)
             e = cudaLaunchCooperativeKernel((const void *)kvpack::decode::attn_kernel<1>, dim3(grid),
                                             dim3(kvpack::decode::kThreads), args, sm, st);
@@ -229,7 +287,7 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
             e = cudaGetLastError();
         }
     } else {
-        const size_t sm = sizeof(kvpack::decode::Smem<2>);
+        const size_t sm = kvpack::decode::smem_bytes<2>();
         if (pl.S > 1)
             e = cudaLaunchCooperativeKernel((const void *)kvpack::decode::attn_kernel<2>, dim3(grid),
                                             dim3(kvpack::decode::kThreads), args, sm, st);
