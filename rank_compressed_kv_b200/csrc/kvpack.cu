@@ -44,28 +44,49 @@ inline int n_units(const kvpack_dims *d, int32_t n_layers) {
 
 inline int hg(const kvpack_dims *d) { return (d->n_q_heads / d->n_kv_heads) * KVPACK_GROUP; }
 
+// Text tail: work items of kTextChunk tokens per (unit, KV head).
+constexpr int kTextChunk = 64;
+
 struct DecodePlan {
-    int nmb, S, tps, units, Hg;
-    size_t off_ml, off_uw, off_arrive, total;
+    int nmb, S, tps, units, Hg, Sc_max;
+    size_t off_qt, off_tp, off_vp, off_arrive, off_counter, total;
 };
 
+// Visual splits: at most Cfg<NMB>::kItemTok tokens each, 32-aligned, and of
+// equal size where a few more splits make them so.
 DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
     DecodePlan pl{};
     pl.Hg = hg(d);
     pl.nmb = (pl.Hg <= 16) ? 1 : 2;
-    const int tps_max = (pl.nmb == 1) ? kvpack::decode::Cfg<1>::kTPS : kvpack::decode::Cfg<2>::kTPS;
-    const int lot = (pl.nmb == 1) ? kvpack::decode::Cfg<1>::kLoT : kvpack::decode::Cfg<2>::kLoT;
-    pl.S = (d->T_vis + tps_max - 1) / tps_max;
-    const int per = (d->T_vis + pl.S - 1) / pl.S;
-    pl.tps = (per + lot - 1) / lot * lot;
+    const int item_max = (pl.nmb == 1) ? kvpack::decode::vis::Cfg<1>::kItemTok : kvpack::decode::vis::Cfg<2>::kItemTok;
+    const int T = d->T_vis;
+    const int s0 = (T + item_max - 1) / item_max;
+    long long best_waste = -1;
+    for (int S = s0; S <= s0 + 8; ++S) {
+        int tps = (T + S - 1) / S;
+        tps = (tps + 31) & ~31;
+        if (tps > item_max) continue;
+        const int Se = (T + tps - 1) / tps;
+        const long long waste = (long long)Se * tps - T;
+        if (best_waste < 0 || waste < best_waste) {
+            best_waste = waste;
+            pl.S = Se;
+            pl.tps = tps;
+        }
+    }
     pl.units = n_units(d, n_layers);
+    pl.Sc_max = (d->L_text_cap + kTextChunk - 1) / kTextChunk;
     size_t off = 0;
-    pl.off_ml = off;
-    if (pl.S > 1) off = align256(off + (size_t)pl.units * pl.S * pl.Hg * 2 * sizeof(float));
-    pl.off_uw = off;
-    if (pl.S > 1) off = align256(off + (size_t)pl.units * pl.S * pl.Hg * kvpack::decode::kUW * sizeof(float));
+    pl.off_qt = off;
+    off = align256(off + (size_t)pl.units * 2 * pl.Hg * 64 * sizeof(uint16_t));
+    pl.off_tp = off;
+    off = align256(off + (size_t)pl.units * pl.Sc_max * pl.Hg * kvpack::decode::kTxtPart * sizeof(float));
+    pl.off_vp = off;
+    off = align256(off + (size_t)pl.units * pl.S * pl.Hg * kvpack::decode::kVisPart * sizeof(float));
     pl.off_arrive = off;
-    off = align256(off + (size_t)pl.units * sizeof(unsigned int));
+    off += (size_t)pl.units * sizeof(unsigned int);
+    pl.off_counter = off;
+    off = align256(off + sizeof(unsigned int));
     pl.total = off;
     return pl;
 }
@@ -73,7 +94,6 @@ DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
 struct DeviceInfo {
     bool ready = false;
     int sms = 0;
-    int attn_blocks[2] = {0, 0};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -85,18 +105,24 @@ kvpack_status device_info(DeviceInfo **out) {
     DeviceInfo &di = g_dev[dev];
     if (!di.ready) {
         if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return KVPACK_ERR_CUDA;
-        const int s1 = (int)kvpack::decode::smem_bytes<1>(), s2 = (int)kvpack::decode::smem_bytes<2>();
-        if (cudaFuncSetAttribute(kvpack::decode::attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1) != cudaSuccess)
+        namespace dc = kvpack::decode;
+        if (cudaFuncSetAttribute(dc::vis::vis_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)dc::vis::smem_bytes<1>()) != cudaSuccess ||
+            cudaFuncSetAttribute(dc::vis::vis_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)dc::vis::smem_bytes<2>()) != cudaSuccess ||
+            cudaFuncSetAttribute(dc::text::text_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)dc::text::smem_bytes()) != cudaSuccess)
             return KVPACK_ERR_CUDA;
-        if (cudaFuncSetAttribute(kvpack::decode::attn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2) != cudaSuccess)
+        int b1 = 0, b2 = 0, bt = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b1, dc::vis::vis_kernel<1>, dc::vis::kThreads,
+                                                          dc::vis::smem_bytes<1>()) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b2, dc::vis::vis_kernel<2>, dc::vis::kThreads,
+                                                          dc::vis::smem_bytes<2>()) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bt, dc::text::text_kernel, dc::text::kThreads,
+                                                          dc::text::smem_bytes()) != cudaSuccess)
             return KVPACK_ERR_CUDA;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.attn_blocks[0], kvpack::decode::attn_kernel<1>,
-                                                          kvpack::decode::kThreads, s1) != cudaSuccess)
-            return KVPACK_ERR_CUDA;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.attn_blocks[1], kvpack::decode::attn_kernel<2>,
-                                                          kvpack::decode::kThreads, s2) != cudaSuccess)
-            return KVPACK_ERR_CUDA;
-        if (di.attn_blocks[0] < 1 || di.attn_blocks[1] < 1) return KVPACK_ERR_CUDA;
+        // the visual kernel holds all 512 tensor-memory columns of its SM: exactly one block per SM
+        if (b1 != 1 || b2 != 1 || bt < 1) return KVPACK_ERR_CUDA;
         kvpack_status cs = kvpack::compress::prepare_device();
         if (cs != KVPACK_OK) return cs;
         di.ready = true;
@@ -126,7 +152,7 @@ kvpack_status tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000 *out) {
 // bf16 tensor map of `rank` dims (innermost first), byte strides of dims 1.., box, swizzle
 bool encode_bf16(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const void *ptr, int rank,
                  const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapSwizzle sw) {
-    cuuint32_t es[3] = {1, 1, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(ptr), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -220,83 +246,86 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     for (const void *ptr : ptrs)
         if (ptr && !aligned16(ptr)) return KVPACK_ERR_ALIGNMENT;
     const DecodePlan pl = plan_decode(d, n_layers);
+    if (pl.S <= 0) return KVPACK_ERR_UNSUPPORTED;
     if (ws == nullptr || ws_bytes < pl.total) return KVPACK_ERR_WORKSPACE;
     DeviceInfo *di = nullptr;
     if ((s = device_info(&di)) != KVPACK_OK) return s;
 
     PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
     if ((s = tensor_map_encoder(&enc)) != KVPACK_OK) return s;
+    namespace dc = kvpack::decode;
 
-    kvpack::decode::Params p;
-    std::memset(&p, 0, sizeof(p));
-    const int lot = (pl.nmb == 1) ? kvpack::decode::Cfg<1>::kLoT : kvpack::decode::Cfg<2>::kLoT;
-    {
-        const cuuint64_t dims[2] = {16, (cuuint64_t)pl.units * d->T_vis};
-        const cuuint64_t strides[1] = {32};
-        const cuuint32_t box[2] = {16, (cuuint32_t)lot};
-        if (!encode_bf16(enc, &p.tm_ck, CK_lo, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B) ||
-            !encode_bf16(enc, &p.tm_cv, CV_lo, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B))
-            return KVPACK_ERR_CUDA;
-    }
-    {
-        const cuuint64_t dims[2] = {512, (cuuint64_t)pl.units * 64};
-        const cuuint64_t strides[1] = {1024};
-        const cuuint32_t box[2] = {64, 32};
-        if (!encode_bf16(enc, &p.tm_bk, BK, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !encode_bf16(enc, &p.tm_bv, BV, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return KVPACK_ERR_CUDA;
-    }
-    if (L_text > 0) {
-        const cuuint64_t dims[3] = {128, 4, (cuuint64_t)pl.units * d->L_text_cap};
-        const cuuint64_t strides[2] = {256, 1024};
-        const cuuint32_t box[3] = {64, 1, 16};
-        if (!encode_bf16(enc, &p.tm_kt, K_text, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !encode_bf16(enc, &p.tm_vt, V_text, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return KVPACK_ERR_CUDA;
-    }
-    p.q = q; p.CK_lo = CK_lo; p.CK_hi = CK_hi; p.CV_lo = CV_lo; p.CV_hi = CV_hi;
-    p.mask = mask; p.out = out; p.mass = mass;
+    const int T = d->T_vis, Hg = pl.Hg, per_kv = d->n_q_heads / d->n_kv_heads;
+    const int groups = d->n_kv_heads / KVPACK_GROUP;
+    const int Sc = (L_text + kTextChunk - 1) / kTextChunk;
+    const float scale2 = softmax_scale * 1.4426950408889634f;
     unsigned char *w = static_cast<unsigned char *>(ws);
-    p.ml = reinterpret_cast<float *>(w + pl.off_ml);
-    p.uw = reinterpret_cast<float *>(w + pl.off_uw);
-    p.arrive = reinterpret_cast<unsigned int *>(w + pl.off_arrive);
-    p.n_units = pl.units; p.T = d->T_vis; p.L = L_text; p.Lcap = d->L_text_cap;
-    p.Hg = pl.Hg; p.per_kv = d->n_q_heads / d->n_kv_heads; p.n_q = d->n_q_heads;
-    p.groups = d->n_kv_heads / KVPACK_GROUP; p.S = pl.S; p.tps = pl.tps;
-    p.txs = (L_text + pl.S - 1) / pl.S;
-    p.txs = (p.txs + kvpack::decode::kTextTokens - 1) / kvpack::decode::kTextTokens * kvpack::decode::kTextTokens;
-    p.n_items = pl.units * pl.S;
-    p.nwords = (d->T_vis + 31) / 32;
-    p.scale2 = softmax_scale * 1.4426950408889634f;
-
+    uint16_t *qt = reinterpret_cast<uint16_t *>(w + pl.off_qt);
+    float *tpart = reinterpret_cast<float *>(w + pl.off_tp);
+    float *vpart = reinterpret_cast<float *>(w + pl.off_vp);
+    unsigned int *arrive = reinterpret_cast<unsigned int *>(w + pl.off_arrive);
+    unsigned int *counter = reinterpret_cast<unsigned int *>(w + pl.off_counter);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int blocks = di->attn_blocks[pl.nmb - 1] * di->sms;
-    const int grid = p.n_items < blocks ? p.n_items : blocks;
-    if (pl.S > grid) return KVPACK_ERR_UNSUPPORTED;   // every split of a unit must be co-resident
-    if (pl.S > 1 && cudaMemsetAsync(p.arrive, 0, (size_t)pl.units * sizeof(unsigned int), st) != cudaSuccess)
+
+    // arrival counters and the text work counter start at zero
+    if (cudaMemsetAsync(arrive, 0, pl.off_counter + sizeof(unsigned int) - pl.off_arrive, st) != cudaSuccess)
         return KVPACK_ERR_CUDA;
-    void *args[] = {&p};
-    cudaError_t e;
-    if (pl.nmb == 1) {
-        const size_t sm = kvpack::decode::smem_bytes<1>();
-        if (pl.S > 1)
-            e = cudaLaunchCooperativeKernel((const void *)kvpack::decode::attn_kernel<1>, dim3(grid),
-                                            dim3(kvpack::decode::kThreads), args, sm, st);
-        else {
-            kvpack::decode::attn_kernel<1><<<grid, kvpack::decode::kThreads, sm, st>>>(p);
-            e = cudaGetLastError();
-        }
-    } else {
-        const size_t sm = kvpack::decode::smem_bytes<2>();
-        if (pl.S > 1)
-            e = cudaLaunchCooperativeKernel((const void *)kvpack::decode::attn_kernel<2>, dim3(grid),
-                                            dim3(kvpack::decode::kThreads), args, sm, st);
-        else {
-            kvpack::decode::attn_kernel<2><<<grid, kvpack::decode::kThreads, sm, st>>>(p);
-            e = cudaGetLastError();
-        }
+
+    // 1. q~ per unit
+    dc::QProjParams qp{q, BK, qt, Hg, per_kv, d->n_q_heads, groups, scale2};
+    dc::qproj_kernel<<<pl.units, 256, 0, st>>>(qp);
+    if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
+
+    // 2. text tail partials
+    if (L_text > 0) {
+        dc::text::Params tp;
+        std::memset(&tp, 0, sizeof(tp));
+        const cuuint64_t dims[4] = {128, 4, (cuuint64_t)L_text, (cuuint64_t)pl.units};
+        const cuuint64_t strides[3] = {256, 1024, (cuuint64_t)d->L_text_cap * 1024};
+        const cuuint32_t box[4] = {64, 1, 16, 1};
+        if (!encode_bf16(enc, &tp.tm_k, K_text, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_bf16(enc, &tp.tm_v, V_text, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return KVPACK_ERR_CUDA;
+        tp.q = q; tp.part = tpart; tp.counter = counter;
+        tp.n_units = pl.units; tp.L = L_text; tp.Hg = Hg; tp.per_kv = per_kv; tp.n_q = d->n_q_heads;
+        tp.groups = groups; tp.Sc = Sc; tp.ct = kTextChunk; tp.n_items = pl.units * 4 * Sc; tp.scale2 = scale2;
+        const int grid = tp.n_items < di->sms ? tp.n_items : di->sms;
+        dc::text::text_kernel<<<grid, dc::text::kThreads, dc::text::smem_bytes(), st>>>(tp);
+        if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
     }
-    return (e == cudaSuccess) ? KVPACK_OK : KVPACK_ERR_CUDA;
+
+    // 3. visual partials and the attention mass
+    {
+        dc::vis::Params vp;
+        std::memset(&vp, 0, sizeof(vp));
+        const cuuint64_t dims[3] = {16, (cuuint64_t)T, (cuuint64_t)pl.units};
+        const cuuint64_t strides[2] = {32, (cuuint64_t)T * 32};
+        const cuuint32_t box[3] = {16, 32, 1};
+        if (!encode_bf16(enc, &vp.tm_ck, CK_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B) ||
+            !encode_bf16(enc, &vp.tm_cv, CV_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B))
+            return KVPACK_ERR_CUDA;
+        vp.CK_lo = CK_lo; vp.CK_hi = CK_hi; vp.CV_lo = CV_lo; vp.CV_hi = CV_hi;
+        vp.qt = qt; vp.mask = mask; vp.mass = mass; vp.part = vpart; vp.tpart = Sc > 0 ? tpart : nullptr;
+        vp.arrive = arrive;
+        vp.n_units = pl.units; vp.T = T; vp.Hg = Hg; vp.S = pl.S; vp.tps = pl.tps; vp.nwords = (T + 31) / 32;
+        vp.Sc = Sc; vp.n_items = pl.units * pl.S;
+        const int grid = vp.n_items < di->sms ? vp.n_items : di->sms;
+        if (pl.S > grid) return KVPACK_ERR_UNSUPPORTED;   // every split of a unit must be co-resident
+        void *args[] = {&vp};
+        const void *fn = (pl.nmb == 1) ? (const void *)dc::vis::vis_kernel<1> : (const void *)dc::vis::vis_kernel<2>;
+        const size_t smem = (pl.nmb == 1) ? dc::vis::smem_bytes<1>() : dc::vis::smem_bytes<2>();
+        cudaError_t e;
+        if (pl.S > 1 && mass != nullptr)
+            e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(dc::vis::kThreads), args, smem, st);
+        else
+            e = cudaLaunchKernel(fn, dim3(grid), dim3(dc::vis::kThreads), args, smem, st);
+        if (e != cudaSuccess) return KVPACK_ERR_CUDA;
+    }
+
+    // 4. combine and project through B_V
+    dc::FinishParams fp{BV, vpart, Sc > 0 ? tpart : nullptr, out, Hg, per_kv, d->n_q_heads, groups, pl.S, Sc};
+    dc::finish_kernel<<<pl.units, 256, 0, st>>>(fp);
+    return (cudaGetLastError() == cudaSuccess) ? KVPACK_OK : KVPACK_ERR_CUDA;
 }
 
 }  // extern "C"
