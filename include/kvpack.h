@@ -61,6 +61,8 @@ extern "C" {
 #define KVPACK_HEAD_DIM 128  /* d */
 #define KVPACK_RANK 64       /* r: rank of the compressed cache */
 #define KVPACK_RANK_LO 16    /* r_lo = r / 4: rank of low-importance tokens */
+#define KVPACK_MAX_T 65536        /* visual tokens per unit, at most */
+#define KVPACK_MAX_TEXT 65536     /* text-tail capacity per unit, at most */
 
 typedef enum {
     KVPACK_OK = 0,
@@ -77,7 +79,7 @@ typedef enum {
  * Shape of the cache.  Supported: group == 4, head_dim == 128, rank == 64,
  * rank_lo == 16, n_kv_heads a positive multiple of 4, n_q_heads a positive
  * multiple of n_kv_heads with Hg = 4 * n_q / n_kv <= 32, batch >= 1,
- * 1 <= T_vis <= 1 << 20, 0 <= L_text_cap.
+ * 1 <= T_vis <= KVPACK_MAX_T, 0 <= L_text_cap <= KVPACK_MAX_TEXT.
  */
 typedef struct {
     int32_t batch;

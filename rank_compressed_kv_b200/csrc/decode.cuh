@@ -23,6 +23,8 @@
 
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace kvpack {
@@ -34,24 +36,118 @@ constexpr int kVisPart = 66;    // per (unit, visual split, head): max, sum, u[6
 
 // ======================================================================== qproj
 
+// Per unit, the query block the visual kernel copies in one piece:
+//   [2][Hg][64] bf16  q~ hi then lo (128-byte rows, 16-byte chunk c stored at c ^ (h & 7))
+//   [Hg][2]     f32   the text tail's (max, sum) per head, combined over its chunks
+__host__ __device__ constexpr size_t qblock_bytes(int Hg) { return (size_t)Hg * (2 * 128 + 8); }
+
 struct QProjParams {
     const uint16_t *q;     // [(layer, batch)][n_q][128]
     const uint16_t *BK;    // [units][64][512]
-    uint16_t *qt;          // [units][2][Hg][64]: hi then lo, 128-byte rows, 16-byte chunk c stored at c ^ (h & 7)
-    int Hg, per_kv, n_q, groups;
+    unsigned char *qt;     // [units][qblock_bytes(Hg)]
+    const float *tpart;    // [units][Sc][Hg][kTxtPart] from text_kernel, or null (Sc == 0)
+    int Hg, per_kv, n_q, groups, Sc;
     float scale2;
 };
 
-// One block per unit.  Warp w takes rank rows 8w..8w+7 of B_K; lane L holds
-// columns 8L..8L+7 and 256+8L..256+8L+7 of a row, so a 16-lane half covers one
-// KV head's 128 columns and a shuffle tree finishes each dot product.
-__global__ void __launch_bounds__(256) qproj_kernel(const QProjParams p) {
+// The text tail's (max, sum) per head of one unit, folded over its chunks: warp
+// per head, lanes over the chunks.
+__device__ __forceinline__ void text_stats(const QProjParams &p, int unit, int warp, int lane) {
+    float *ts = reinterpret_cast<float *>(p.qt + (size_t)unit * qblock_bytes(p.Hg) + (size_t)p.Hg * 256);
+    for (int h = warp; h < p.Hg; h += 8) {
+        const float *tp = p.tpart + (size_t)unit * p.Sc * p.Hg * kTxtPart + (size_t)h * kTxtPart;
+        float mx = -INFINITY, mc[2], lc[2];
+        #pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int c = lane + 32 * k;
+            mc[k] = c < p.Sc ? tp[(size_t)c * p.Hg * kTxtPart] : -INFINITY;
+            lc[k] = c < p.Sc ? tp[(size_t)c * p.Hg * kTxtPart + 1] : 0.f;
+            mx = fmaxf(mx, mc[k]);
+        }
+        for (int c = lane + 64; c < p.Sc; c += 32) mx = fmaxf(mx, tp[(size_t)c * p.Hg * kTxtPart]);
+        #pragma unroll
+        for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+        float sum = 0.f;
+        #pragma unroll
+        for (int k = 0; k < 2; ++k)
+            if (mc[k] != -INFINITY) sum += lc[k] * ex2(mc[k] - mx);
+        for (int c = lane + 64; c < p.Sc; c += 32) {
+            const float m2 = tp[(size_t)c * p.Hg * kTxtPart];
+            if (m2 != -INFINITY) sum += tp[(size_t)c * p.Hg * kTxtPart + 1] * ex2(m2 - mx);
+        }
+        #pragma unroll
+        for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
+        if (lane == 0) {
+            ts[2 * h] = mx;
+            ts[2 * h + 1] = sum;
+        }
+    }
+}
+
+// One block per unit (several query heads per KV head); thread (i, j) =
+// (tid / 4, tid % 4) owns rank row i of B_K restricted to KV head j (256
+// contiguous bytes) and forms q~_h[i] for the KV head's query heads with plain
+// fp32 FMAs.  Runs after text_kernel.
+__global__ void __launch_bounds__(256) qproj_cols_kernel(const QProjParams p) {
+    __shared__ float qs[kMaxHeads][132];   // q rows in fp32; the pad spreads the 4 KV heads over banks
+    const int unit = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int lb = unit / p.groups, G = unit % p.groups;
+    const int i = tid >> 2, j = tid & 3;
+
+    // the thread's 256 bytes of B_K first, so that they are in flight before anything waits
+    uint4 raw[16];
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.BK + ((size_t)unit * 64 + i) * 512 + 128 * j);
+    #pragma unroll
+    for (int k = 0; k < 16; ++k) raw[k] = __ldg(src + k);
+
+    const uint32_t *qsrc = reinterpret_cast<const uint32_t *>(p.q + ((size_t)lb * p.n_q + (size_t)G * p.Hg) * 128);
+    for (int x = tid; x < p.Hg * 64; x += 256) {
+        const uint32_t v = __ldg(qsrc + x);
+        qs[x >> 6][2 * (x & 63)] = __uint_as_float(v << 16);
+        qs[x >> 6][2 * (x & 63) + 1] = __uint_as_float(v & 0xffff0000u);
+    }
+
+    text_stats(p, unit, warp, lane);
+    __syncthreads();
+
+    float acc[8];
+    #pragma unroll
+    for (int hh = 0; hh < 8; ++hh) acc[hh] = 0.f;
+    const int h0 = j * p.per_kv;
+    #pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+        #pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float b = (e & 1) ? __uint_as_float(w4[e >> 1] & 0xffff0000u) : __uint_as_float(w4[e >> 1] << 16);
+            #pragma unroll
+            for (int hh = 0; hh < 8; ++hh)
+                if (hh < p.per_kv) acc[hh] = fmaf(b, qs[h0 + hh][8 * k + e], acc[hh]);
+        }
+    }
+    uint16_t *qt = reinterpret_cast<uint16_t *>(p.qt + (size_t)unit * qblock_bytes(p.Hg));
+    #pragma unroll
+    for (int hh = 0; hh < 8; ++hh) {
+        if (hh < p.per_kv) {
+            const int h = h0 + hh;
+            const float v = acc[hh] * p.scale2;
+            const uint16_t hi = float_to_bf16_bits(v);
+            const uint16_t lo = float_to_bf16_bits(v - bf16_bits_to_float(hi));
+            const int off = h * 64 + ((((i >> 3) ^ (h & 7)) & 7) << 3) + (i & 7);
+            qt[off] = hi;
+            qt[p.Hg * 64 + off] = lo;
+        }
+    }
+}
+
+// One block per unit (one or two query heads per KV head): warp w takes rank
+// rows 8w..8w+7 of B_K; lane L holds columns 8L..8L+7 and 256+8L..256+8L+7 of a
+// row (coalesced), so a 16-lane half covers one KV head's 128 columns and a
+// shuffle tree finishes each dot product.  Runs after text_kernel.
+__global__ void __launch_bounds__(256) qproj_rows_kernel(const QProjParams p) {
     __shared__ float qs[kMaxHeads][128];
     const int unit = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int lb = unit / p.groups, G = unit % p.groups;
-    const uint16_t *qsrc = p.q + ((size_t)lb * p.n_q + (size_t)G * p.Hg) * 128;
-    for (int i = threadIdx.x; i < p.Hg * 128; i += 256) qs[i >> 7][i & 127] = bf16_bits_to_float(qsrc[i]);
-
     uint4 raw[8][2];
     const uint16_t *bk = p.BK + (size_t)unit * 64 * 512;
     #pragma unroll
@@ -59,9 +155,15 @@ __global__ void __launch_bounds__(256) qproj_kernel(const QProjParams p) {
         #pragma unroll
         for (int sg = 0; sg < 2; ++sg)
             raw[r][sg] = __ldcs(reinterpret_cast<const uint4 *>(bk + (size_t)(8 * warp + r) * 512 + 256 * sg + 8 * lane));
+    const uint32_t *qsrc = reinterpret_cast<const uint32_t *>(p.q + ((size_t)lb * p.n_q + (size_t)G * p.Hg) * 128);
+    for (int x = threadIdx.x; x < p.Hg * 64; x += 256) {
+        const uint32_t v = __ldg(qsrc + x);
+        qs[x >> 6][2 * (x & 63)] = __uint_as_float(v << 16);
+        qs[x >> 6][2 * (x & 63) + 1] = __uint_as_float(v & 0xffff0000u);
+    }
+    text_stats(p, unit, warp, lane);
     __syncthreads();
-
-    uint16_t *qt = p.qt + (size_t)unit * 2 * p.Hg * 64;
+    uint16_t *qt = reinterpret_cast<uint16_t *>(p.qt + (size_t)unit * qblock_bytes(p.Hg));
     #pragma unroll
     for (int r = 0; r < 8; ++r) {
         const int i = 8 * warp + r;
@@ -75,21 +177,24 @@ __global__ void __launch_bounds__(256) qproj_kernel(const QProjParams p) {
                 b[2 * e] = __uint_as_float(w4[e] << 16);
                 b[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
             }
-            for (int hh = 0; hh < p.per_kv; ++hh) {
-                const int h = j * p.per_kv + hh;
-                const float *qr = &qs[h][dd];
-                float acc = 0.f;
-                #pragma unroll
-                for (int e = 0; e < 8; ++e) acc = fmaf(b[e], qr[e], acc);
-                #pragma unroll
-                for (int d = 1; d < 16; d <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
-                if ((lane & 15) == 0) {
-                    const float v = acc * p.scale2;
-                    const uint16_t hi = float_to_bf16_bits(v);
-                    const uint16_t lo = float_to_bf16_bits(v - bf16_bits_to_float(hi));
-                    const int off = h * 64 + ((((i >> 3) ^ (h & 7)) & 7) << 3) + (i & 7);
-                    qt[off] = hi;
-                    qt[p.Hg * 64 + off] = lo;
+            #pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                if (hh < p.per_kv) {
+                    const int h = j * p.per_kv + hh;
+                    const float *qr = &qs[h][dd];
+                    float acc = 0.f;
+                    #pragma unroll
+                    for (int e = 0; e < 8; ++e) acc = fmaf(b[e], qr[e], acc);
+                    #pragma unroll
+                    for (int d = 1; d < 16; d <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
+                    if ((lane & 15) == 0) {
+                        const float v = acc * p.scale2;
+                        const uint16_t hi = float_to_bf16_bits(v);
+                        const uint16_t lo = float_to_bf16_bits(v - bf16_bits_to_float(hi));
+                        const int off = h * 64 + ((((i >> 3) ^ (h & 7)) & 7) << 3) + (i & 7);
+                        qt[off] = hi;
+                        qt[p.Hg * 64 + off] = lo;
+                    }
                 }
             }
         }
@@ -322,81 +427,111 @@ namespace vis {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kSlots = 3;
-constexpr int kSlotBytes = 8192;
-constexpr int kHiTok = 32;          // full-rank tokens per HI stage
 constexpr int kMeta = 4;            // item metadata ring (the issue side runs up to two items ahead)
 
+// Geometry per head-block count.  Up to 16 query heads per unit: two blocks per
+// SM (their serial phases overlap), 4 KB ring slots.  Up to 32: one block per SM.
 template <int NMB>
 struct Cfg {
-    static constexpr int kRows = 16 * NMB;                 // query-head rows (padded)
-    static constexpr int kLoTok = (NMB == 1) ? 128 : 64;   // visual tokens per warp per item
-    static constexpr int kItemTok = kWarps * kLoTok;       // 1024 / 512 tokens per item
-    static constexpr int kHiMax = kLoTok / kHiTok;         // HI stages per warp per item, at most
-    static constexpr int kUpd = kLoTok / 64 + kHiMax;      // softmax updates per warp per item, at most
+    static constexpr int kRows = 16 * NMB;                      // query-head rows (padded)
+    static constexpr int kBlocks = (NMB == 1) ? 2 : 1;          // resident blocks per SM
+    static constexpr int kSlots = 2;                            // ring slots per warp
+    static constexpr int kSlotBytes = (NMB == 1) ? 4096 : 8192; // K rows in the first half, V in the second
+    static constexpr int kHiTok = (NMB == 1) ? 16 : 32;         // full-rank tokens per HI stage
+    static constexpr int kNTH = kHiTok / 8;                     // m16n8 token tiles per HI stage
+    static constexpr int kLoTok = 64;                           // visual tokens per warp per item
+    static constexpr int kItemTok = kWarps * kLoTok;            // tokens per item
+    static constexpr int kHiMax = kLoTok / kHiTok;              // HI stages per warp per item, at most
+    static constexpr int kUpd = 1 + kHiMax;                     // softmax updates per warp per item, at most
+    // tensor-memory columns of one warp's stash of one item: LO p (32 per head block), then HI p
+    static constexpr int kBufCols = 32 * NMB + 4 * kNTH * NMB * kHiMax;
+    static constexpr int kTmemCols = 4 * kBufCols;              // two warps per lane quarter, two items each
+    static_assert(kHiTok * 128 == kSlotBytes / 2, "HI stage rows fill half a slot");
+    static_assert(kLoTok * 32 <= kSlotBytes / 2, "LO stage rows fit half a slot");
 };
 
 struct Params {
     CUtensorMap tm_ck, tm_cv;   // C_lo planes: 3D {16, T, units}, box {16, 32, 1}, 32-byte swizzle
     const uint16_t *CK_lo, *CK_hi, *CV_lo, *CV_hi;
-    const uint16_t *qt;         // [units][2][Hg][64] from qproj_kernel
+    const unsigned char *qt;    // [units][qblock_bytes(Hg)] from qproj_kernel
     const uint32_t *mask;       // [units][nwords]
     float *mass;                // [units][T] or null
     float *part;                // [units][S][Hg][kVisPart]
-    const float *tpart;         // [units][Sc][Hg][kTxtPart] (max and sum read) or null
+    float *ustat;               // [units][Hg][2]: unit-wide (max, 1/sum); NaN at launch (S > 1)
     unsigned int *arrive;       // [units], zero at launch
-    int n_units, T, Hg, S, tps, nwords, Sc, n_items;
+    int n_units, T, Hg, S, tps, nwords, n_items;
 };
 
 template <int NMB>
 struct Smem {
     using C = Cfg<NMB>;
-    alignas(1024) unsigned char ring[kWarps][kSlots][kSlotBytes];
+    alignas(1024) unsigned char ring[kWarps][C::kSlots][C::kSlotBytes];
     alignas(128) uint16_t qt[2][C::kRows][64];              // q~ hi / lo of the current item
-    float u_acc[C::kRows][64];                               // block-wide u of the item
+    alignas(16) float tst[C::kRows][2];                      // text (max, sum) of the current item's unit
+    float tcur[C::kRows][2];                                 // the same, kept through the epilogue
+    float ubuf[4][16][64];                                   // merge staging: 4 warps x one 16-row block of u
     float wm[kWarps][C::kRows], wl[kWarps][C::kRows];
     float mcta[C::kRows], lcta[C::kRows], mfin[C::kRows], invl[C::kRows];
-    float mref[2][kWarps][C::kUpd][C::kRows];               // running max at each stashed update
+    float mref[2][kWarps][C::kUpd][C::kRows];               // reference max of each stashed update
+    float upf[C::kRows][2];                                  // prefetched unit (max, 1/sum) of the previous item
     uint16_t hi_list[kMeta][kWarps][C::kLoTok];             // this warp's full-rank tokens (item-relative)
-    int meta[kMeta][kWarps][8];                             // lo0, n_lo, n_hi, item, 4 mask words of the LO range
-    uint64_t full[kWarps][kSlots];
+    int meta[kMeta][kWarps][12];                            // lo0, n_lo, n_hi, item, 4 mask words of the LO range, unit, t0
+    uint64_t full[kWarps][C::kSlots];
     uint64_t qbar;
     uint32_t tmem_base;
     int abort;
+    int last;
 };
 
 template <int NMB>
 constexpr size_t smem_bytes() { return sizeof(Smem<NMB>) + 1024; }
 
-// One online-softmax update of row r over NT m16n8 score tiles; returns the
-// new running max.  p overwrites s.
+// Reference a row starts from: any finite logit exceeds it by more than kLazy.
+constexpr float kRefInit = -1e30f;
+// The reference max of a row moves only when a logit exceeds it by more than
+// kLazy (log2 units), so p = 2^(s - m) stays below 2^kLazy and the (rare)
+// rescale of l and u is a warp-uniform branch.
+constexpr float kLazy = 8.f;
+
+// One online-softmax update of the block's rows g and g + 8 over NT m16n8
+// score tiles (log2 domain, masked logits -inf).  p overwrites s.
 template <int NT>
-__device__ __forceinline__ float softmax_row(float (&s)[NT][4], int r, float &m, float &l, float (&u)[8][4]) {
-    float mx = -INFINITY;
+__device__ __forceinline__ void lazy_update(float (&s)[NT][4], float (&m)[2], float (&l)[2], float (&u)[8][4]) {
+    float mx0 = fmaxf(s[0][0], s[0][1]), mx1 = fmaxf(s[0][2], s[0][3]);
     #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) mx = fmaxf(mx, fmaxf(s[nt][2 * r], s[nt][2 * r + 1]));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float mn = fmaxf(m, mx);
-    const bool live = mn != -INFINITY;
-    const float alpha = live ? ex2(m - mn) : 1.f;
-    float sum = 0.f;
+    for (int nt = 1; nt < NT; ++nt) {
+        mx0 = fmaxf(mx0, fmaxf(s[nt][0], s[nt][1]));
+        mx1 = fmaxf(mx1, fmaxf(s[nt][2], s[nt][3]));
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const bool up0 = mx0 > m[0] + kLazy, up1 = mx1 > m[1] + kLazy;
+    if (__any_sync(0xffffffffu, up0 || up1)) {
+        const float n0 = up0 ? mx0 : m[0], n1 = up1 ? mx1 : m[1];
+        const float a0 = ex2(m[0] - n0), a1 = ex2(m[1] - n1);
+        l[0] *= a0;
+        l[1] *= a1;
+        #pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            u[nt][0] *= a0; u[nt][1] *= a0; u[nt][2] *= a1; u[nt][3] *= a1;
+        }
+        m[0] = n0;
+        m[1] = n1;
+    }
+    float sum0 = 0.f, sum1 = 0.f;
     #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-        const float x0 = live ? ex2(s[nt][2 * r] - mn) : 0.f;
-        const float x1 = live ? ex2(s[nt][2 * r + 1] - mn) : 0.f;
-        s[nt][2 * r] = x0;
-        s[nt][2 * r + 1] = x1;
-        sum += x0 + x1;
+        s[nt][0] = ex2(s[nt][0] - m[0]);
+        s[nt][1] = ex2(s[nt][1] - m[0]);
+        s[nt][2] = ex2(s[nt][2] - m[1]);
+        s[nt][3] = ex2(s[nt][3] - m[1]);
+        sum0 += s[nt][0] + s[nt][1];
+        sum1 += s[nt][2] + s[nt][3];
     }
-    l = l * alpha + sum;
-    m = mn;
-    #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-        u[nt][2 * r] *= alpha;
-        u[nt][2 * r + 1] *= alpha;
-    }
-    return mn;
+    l[0] += sum0;
+    l[1] += sum1;
 }
 
 // Sum over the 8 lanes that share lane & 3 of 16 per-lane values, scattered:
@@ -440,7 +575,22 @@ __device__ __forceinline__ float reduce_scatter8(const float (&x)[8], int lane) 
     return (b2 ? t2[1] : t2[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
 }
 
-// Persistent, one 256-thread block per SM, a static round-robin over items
+// 4 values -> lanes with bit 2 clear hold the total of slot 2 b4 + b3 (the
+// lanes with bit 2 set hold the same totals)
+__device__ __forceinline__ float reduce_scatter4(const float (&x)[4], int lane) {
+    float t2[2];
+    const bool b4 = lane & 16, b3 = lane & 8;
+    #pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = b4 ? x[i] : x[2 + i];
+        t2[i] = (b4 ? x[2 + i] : x[i]) + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    const float send = b3 ? t2[0] : t2[1];
+    const float t = (b3 ? t2[1] : t2[0]) + __shfl_xor_sync(0xffffffffu, send, 8);
+    return t + __shfl_xor_sync(0xffffffffu, t, 4);
+}
+
+// Persistent, one or two 256-thread blocks per SM, a static round-robin over items
 // (unit, split).  Each warp streams its own share of the item -- a contiguous
 // range of C_lo rows (TMA) and an equal share of the item's full-rank tokens
 // (C_lo + C_hi rows gathered with cp.async) -- through a private 3-slot ring,
@@ -455,8 +605,9 @@ __device__ __forceinline__ float reduce_scatter8(const float (&x)[8], int lane) 
 // item is written one item later, when every split of the unit (and the text
 // partials) fix the unit's max and sum: mass_t = sum_h p_ht 2^(m_ref - M_h) / L_h.
 template <int NMB>
-__global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const __grid_constant__ Params p) {
     using C = Cfg<NMB>;
+    constexpr int kSlots = C::kSlots, kHiTok = C::kHiTok, kNTH = C::kNTH, kHalf = C::kSlotBytes / 2;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t sbase0 = smem_u32(smem_raw);
     Smem<NMB> &sm = *reinterpret_cast<Smem<NMB> *>(smem_raw + ((1024u - (sbase0 & 1023u)) & 1023u));
@@ -472,21 +623,21 @@ __global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant_
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     for (int i = tid; i < 2 * C::kRows * 64; i += kThreads) (&sm.qt[0][0][0])[i] = 0;
-    for (int i = tid; i < C::kRows * 64; i += kThreads) (&sm.u_acc[0][0])[i] = 0.f;
-    if (warp == 0) tmem_alloc(&sm.tmem_base, 512);
+    if (warp == 0) tmem_alloc(&sm.tmem_base, C::kTmemCols);
     tmem_fence_before();
     __syncthreads();
     tmem_fence_after();
-    const uint32_t tmem = sm.tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + 256u * (uint32_t)(warp >> 2);
+    const uint32_t tmem = sm.tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(2 * C::kBufCols * (warp >> 2));
 
     auto item_of = [&](int K) { return (int)blockIdx.x + K * (int)gridDim.x; };
-    auto issue_q = [&](int K) {   // q~ of item K into sm.qt (one thread)
-        const int unit = item_of(K) / p.S;
+    auto issue_q = [&](int K) {   // query block of item K's unit into sm.qt / sm.tst (one thread)
+        const unsigned char *src = p.qt + (size_t)(item_of(K) / p.S) * qblock_bytes(p.Hg);
         const uint32_t bytes = (uint32_t)p.Hg * 128u;
         fence_proxy_async();
-        mbar_arrive_tx(&sm.qbar, 2 * bytes);
-        bulk_g2s(&sm.qt[0][0][0], p.qt + (size_t)unit * 2 * p.Hg * 64, bytes, &sm.qbar);
-        bulk_g2s(&sm.qt[1][0][0], p.qt + (size_t)unit * 2 * p.Hg * 64 + (size_t)p.Hg * 64, bytes, &sm.qbar);
+        mbar_arrive_tx(&sm.qbar, (uint32_t)qblock_bytes(p.Hg));
+        bulk_g2s(&sm.qt[0][0][0], src, bytes, &sm.qbar);
+        bulk_g2s(&sm.qt[1][0][0], src + bytes, bytes, &sm.qbar);
+        bulk_g2s(&sm.tst[0][0], src + 2 * bytes, (uint32_t)p.Hg * 8u, &sm.qbar);
     };
     if (tid == 0) issue_q(0);
 
@@ -551,6 +702,8 @@ __global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant_
             sm.meta[ms][warp][1] = n_lo;
             sm.meta[ms][warp][2] = h1 - h0;
             sm.meta[ms][warp][3] = item;
+            sm.meta[ms][warp][8] = item / p.S;
+            sm.meta[ms][warp][9] = t0;
         }
         __syncwarp();
         i_nst = (n_lo > 0 ? 1 : 0) + (h1 - h0 + kHiTok - 1) / kHiTok;
@@ -561,8 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant_
     auto issue_stage = [&]() {
         const int ms = iK % kMeta;
         const int lo0 = sm.meta[ms][warp][0], n_lo = sm.meta[ms][warp][1], nh = sm.meta[ms][warp][2];
-        const int item = sm.meta[ms][warp][3];
-        const int unit = item / p.S, t0 = (item % p.S) * p.tps;
+        const int unit = sm.meta[ms][warp][8], t0 = sm.meta[ms][warp][9];
         const int slot = i_seq % kSlots;
         unsigned char *dst = sm.ring[warp][slot];
         uint64_t *bar = &sm.full[warp][slot];
@@ -576,22 +728,24 @@ __global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant_
                 mbar_arrive_tx(bar, (uint32_t)nb * 2048u);
                 for (int b = 0; b < nb; ++b) {
                     tma_3d(dst + 1024 * b, &p.tm_ck, 0, t0 + lo0 + 32 * b, unit, bar);
-                    tma_3d(dst + 4096 + 1024 * b, &p.tm_cv, 0, t0 + lo0 + 32 * b, unit, bar);
+                    tma_3d(dst + kHalf + 1024 * b, &p.tm_cv, 0, t0 + lo0 + 32 * b, unit, bar);
                 }
             } else {
                 mbar_arrive(bar);
             }
         } else {
+            // 32 full-rank tokens: C_lo + C_hi rows of K and V gathered into 128-byte rows
+            // (16-byte chunk c of row r stored at c ^ (r & 7)); rows past the count are zero
             const int hs = i_st - (n_lo > 0 ? 1 : 0);
             const int cnt = min(kHiTok, nh - kHiTok * hs);
             const size_t ubase = (size_t)unit * p.T + t0;
             #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < kHiTok / 4; ++i) {
                 const int idx = lane + 32 * i;
                 const int r = idx >> 3, ch = idx & 7;
                 const int pos = (ch ^ (r & 7)) << 4;
                 unsigned char *dk = dst + r * 128 + pos;
-                unsigned char *dv = dst + 4096 + r * 128 + pos;
+                unsigned char *dv = dst + kHalf + r * 128 + pos;
                 if (r < cnt) {
                     const size_t row = ubase + sm.hi_list[ms][warp][kHiTok * hs + r];
                     if (ch < 2) {
@@ -634,75 +788,76 @@ __global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant_
     uint32_t qah[NMB][4], qal[NMB][4];
     const uint32_t qt0 = smem_u32(&sm.qt[0][0][0]), qt1 = smem_u32(&sm.qt[1][0][0]);
 
-    // deferred: attention mass of item K (meta slot K % kMeta, stash buffer K & 1); block-wide
-    auto mass_of = [&](int K) {
+    // Attention mass of this warp's tokens of item K (meta slot K % kMeta, stash
+    // buffer K & 1), one warp alone.  The unit's (max, 1/sum) per head come from
+    // shared memory (single-split units) or from ustat, polled until the unit's
+    // last split has written them.
+    auto mass_warp = [&](int K, int src) {
         const int item = item_of(K);
         const int unit = item / p.S;
-        if (tid == 0) {
+        float Mr[NMB][2], IL[NMB][2];
+        bool ready = true;
+        #pragma unroll
+        for (int mb = 0; mb < NMB; ++mb)
+            #pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int row = 16 * mb + g + 8 * r;
+                const bool ok = row < p.Hg;
+                Mr[mb][r] = ok ? (src == 0 ? sm.mfin[row] : sm.upf[row][0]) : 0.f;
+                IL[mb][r] = ok ? (src == 0 ? sm.invl[row] : sm.upf[row][1]) : 0.f;
+                ready = ready && !(Mr[mb][r] != Mr[mb][r]) && !(IL[mb][r] != IL[mb][r]);
+            }
+        if (src == 1 || (src == 2 && !__all_sync(0xffffffffu, ready))) {
             const long long start = clock64();
-            while (!*abort) {
-                unsigned int v;
-                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&p.arrive[unit]) : "memory");
-                if (v >= (unsigned int)p.S) break;
+            while (true) {
+                ready = true;
+                #pragma unroll
+                for (int mb = 0; mb < NMB; ++mb)
+                    #pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int row = 16 * mb + g + 8 * r;
+                        float a = 0.f, b2 = 0.f;
+                        if (row < p.Hg) {
+                            const float *us = p.ustat + ((size_t)unit * p.Hg + row) * 2;
+                            asm volatile("ld.relaxed.gpu.global.v2.f32 {%0, %1}, [%2];" : "=f"(a), "=f"(b2) : "l"(us) : "memory");
+                        }
+                        Mr[mb][r] = a;
+                        IL[mb][r] = b2;
+                        ready = ready && !(a != a) && !(b2 != b2);
+                    }
+                if (__all_sync(0xffffffffu, ready)) break;
+                if (*abort) return;
                 if (clock64() - start > kWaitCycles) {
                     report_error(KVPACK_ERR_TIMEOUT);
                     *abort = 1;
-                    break;
+                    return;
                 }
-                __nanosleep(64);
+                __nanosleep(100);
             }
         }
-        __syncthreads();
-        if (*abort) return;
-        // unit-wide max and 1/sum per head from the visual and text partials
-        for (int h = warp; h < p.Hg; h += kWarps) {
-            const float *vp = p.part + (size_t)unit * p.S * p.Hg * kVisPart + (size_t)h * kVisPart;
-            const float *tp = p.tpart + (size_t)unit * p.Sc * p.Hg * kTxtPart + (size_t)h * kTxtPart;
-            float mx = -INFINITY;
-            for (int s = lane; s < p.S; s += 32) mx = fmaxf(mx, __ldcg(vp + (size_t)s * p.Hg * kVisPart));
-            for (int c = lane; c < p.Sc; c += 32) mx = fmaxf(mx, __ldcg(tp + (size_t)c * p.Hg * kTxtPart));
-            #pragma unroll
-            for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
-            float sum = 0.f;
-            for (int s = lane; s < p.S; s += 32) {
-                const float ms = __ldcg(vp + (size_t)s * p.Hg * kVisPart);
-                if (ms != -INFINITY) sum += __ldcg(vp + (size_t)s * p.Hg * kVisPart + 1) * ex2(ms - mx);
-            }
-            for (int c = lane; c < p.Sc; c += 32) {
-                const float ms = __ldcg(tp + (size_t)c * p.Hg * kTxtPart);
-                if (ms != -INFINITY) sum += __ldcg(tp + (size_t)c * p.Hg * kTxtPart + 1) * ex2(ms - mx);
-            }
-            #pragma unroll
-            for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
-            if (lane == 0) {
-                sm.mfin[h] = mx;
-                sm.invl[h] = 1.f / sum;
-            }
-        }
-        __syncthreads();
         const int ms = K % kMeta, b = K & 1;
         const int lo0 = sm.meta[ms][warp][0], n_lo = sm.meta[ms][warp][1], nh = sm.meta[ms][warp][2];
         const int t0 = (item % p.S) * p.tps;
         float *mrow = p.mass + (size_t)unit * p.T + t0;
-        auto fac = [&](int upd, int row) -> float {
-            const float mr = sm.mref[b][warp][upd][row];
-            return (row < p.Hg && mr != -INFINITY) ? ex2(mr - sm.mfin[row]) * sm.invl[row] : 0.f;
+        auto fac = [&](int upd, int mb, int r) -> float {
+            const int row = 16 * mb + g + 8 * r;
+            return row < p.Hg ? ex2(sm.mref[b][warp][upd][row] - Mr[mb][r]) * IL[mb][r] : 0.f;
         };
         tmem_fence_after();
-        // LO range, 64 tokens per pass
-        for (int hf = 0; hf < C::kLoTok / 64; ++hf) {
-            if (64 * hf >= n_lo) break;
+        // LO range (64 tokens)
+        const uint32_t bcol = (uint32_t)(C::kBufCols * b);
+        if (n_lo > 0) {
             float acc[16];
             #pragma unroll
             for (int i = 0; i < 16; ++i) acc[i] = 0.f;
             #pragma unroll
             for (int mb = 0; mb < NMB; ++mb) {
                 float v0[16], v1[16];
-                const uint32_t col = (uint32_t)(128 * b + 32 * (NMB == 1 ? hf : mb));
+                const uint32_t col = bcol + (uint32_t)(32 * mb);
                 tmem_ld16(tmem + col, v0);
                 tmem_ld16(tmem + col + 16, v1);
                 tmem_wait_ld();
-                const float f0 = fac(hf, 16 * mb + g), f1 = fac(hf, 16 * mb + g + 8);
+                const float f0 = fac(0, mb, 0), f1 = fac(0, mb, 1);
                 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt)
                     #pragma unroll
@@ -716,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant_
             const int nt = 4 * ((lane >> 4) & 1) + 2 * ((lane >> 3) & 1) + ((lane >> 2) & 1);
             #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const int r = 64 * hf + 8 * nt + 2 * tig + e;
+                const int r = 8 * nt + 2 * tig + e;
                 const bool hb = ((uint32_t)sm.meta[ms][warp][4 + (r >> 5)] >> (r & 31)) & 1u;
                 if (r < n_lo && !hb) mrow[lo0 + r] = out[e];
             }
@@ -724,26 +879,47 @@ __global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant_
         // full-rank tokens
         for (int hs = 0; hs * kHiTok < nh; ++hs) {
             const int n = min(kHiTok, nh - kHiTok * hs);
-            float acc[8];
+            float acc[2 * kNTH];
             #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-            const int upd = C::kLoTok / 64 + hs;
+            for (int i = 0; i < 2 * kNTH; ++i) acc[i] = 0.f;
+            const int upd = 1 + hs;
             #pragma unroll
             for (int mb = 0; mb < NMB; ++mb) {
                 float v[16];
-                const uint32_t col = (uint32_t)(128 * b + 64 + (NMB == 1 ? 16 * hs : 32 * hs + 16 * mb));
-                tmem_ld16(tmem + col, v);
+                const uint32_t col = bcol + (uint32_t)(32 * NMB + (hs * NMB + mb) * 4 * kNTH);
+                if (kNTH == 4) {
+                    tmem_ld16(tmem + col, v);
+                } else {
+                    float v8[8];
+                    tmem_ld8(tmem + col, v8);
+                    #pragma unroll
+                    for (int i = 0; i < 8; ++i) v[i] = v8[i];
+                }
                 tmem_wait_ld();
-                const float f0 = fac(upd, 16 * mb + g), f1 = fac(upd, 16 * mb + g + 8);
+                const float f0 = fac(upd, mb, 0), f1 = fac(upd, mb, 1);
                 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
+                for (int nt = 0; nt < kNTH; ++nt)
                     #pragma unroll
                     for (int e = 0; e < 2; ++e) acc[2 * nt + e] += v[4 * nt + e] * f0 + v[4 * nt + 2 + e] * f1;
             }
-            const float val = reduce_scatter8(acc, lane);
-            const int j = 4 * ((lane >> 4) & 1) + 2 * ((lane >> 3) & 1) + ((lane >> 2) & 1);
+            int j;
+            float val;
+            if (kNTH == 4) {
+                float a8[8];
+                #pragma unroll
+                for (int i = 0; i < 8; ++i) a8[i] = acc[i];
+                val = reduce_scatter8(a8, lane);
+                j = 4 * ((lane >> 4) & 1) + 2 * ((lane >> 3) & 1) + ((lane >> 2) & 1);
+            } else {
+                float a4[4];
+                #pragma unroll
+                for (int i = 0; i < 4; ++i) a4[i] = acc[i];
+                val = reduce_scatter4(a4, lane);
+                j = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+            }
             const int colt = 8 * (j >> 1) + 2 * tig + (j & 1);
-            if (colt < n) mrow[sm.hi_list[ms][warp][kHiTok * hs + colt]] = val;
+            const bool writer = kNTH == 4 || ((lane >> 2) & 1) == 0;
+            if (writer && colt < n) mrow[sm.hi_list[ms][warp][kHiTok * hs + colt]] = val;
         }
         tmem_fence_before();
     };
@@ -768,95 +944,92 @@ __global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant_
             const uint32_t off = row * 128 + (((lane >> 4) ^ (row & 7)) << 4);
             ldsm_x4(qt0 + off, qah[mb][0], qah[mb][1], qah[mb][2], qah[mb][3]);
             ldsm_x4(qt1 + off, qal[mb][0], qal[mb][1], qal[mb][2], qal[mb][3]);
-            m[mb][0] = m[mb][1] = -INFINITY;
+            m[mb][0] = m[mb][1] = kRefInit;
             l[mb][0] = l[mb][1] = 0.f;
             #pragma unroll
             for (int a = 0; a < 8; ++a) u[mb][a][0] = u[mb][a][1] = u[mb][a][2] = u[mb][a][3] = 0.f;
         }
-        const uint32_t tcol = tmem + 128u * (uint32_t)b;
+        const uint32_t tcol = tmem + (uint32_t)(C::kBufCols * b);
         const int nst = (n_lo > 0 ? 1 : 0) + (nh + kHiTok - 1) / kHiTok;
+
+        // LO range: one softmax update over all of this warp's C_lo rows (NT m16n8 tiles of tokens)
+        auto do_lo = [&](uint32_t sb, auto ntc) {
+            constexpr int NT = decltype(ntc)::value;
+            uint32_t x[NT / 4];   // mask words shifted so that bit 8 (nt & 3) + e is token 8 nt + 2 tig + e
+            #pragma unroll
+            for (int w4 = 0; w4 < NT / 4; ++w4) x[w4] = lw[w4] >> (2 * tig);
+            const bool partial = n_lo < 8 * NT;
+            #pragma unroll
+            for (int mb = 0; mb < NMB; ++mb) {
+                float s[NT][4];
+                #pragma unroll
+                for (int a = 0; a < NT; ++a) s[a][0] = s[a][1] = s[a][2] = s[a][3] = 0.f;
+                #pragma unroll
+                for (int np = 0; np < NT / 2; ++np) {
+                    uint32_t b0, b1, b2, b3;
+                    const int row = 16 * np + (lane & 7) + ((lane >> 4) << 3);
+                    const int ch = (lane >> 3) & 1;
+                    ldsm_x4(sb + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), b0, b1, b2, b3);
+                    mma_bf16(s[2 * np], qah[mb], b0, b1);
+                    mma_bf16(s[2 * np + 1], qah[mb], b2, b3);
+                    mma_bf16(s[2 * np], qal[mb], b0, b1);
+                    mma_bf16(s[2 * np + 1], qal[mb], b2, b3);
+                }
+                #pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    #pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const bool hb = (x[nt >> 2] >> (8 * (nt & 3) + e)) & 1u;
+                        const bool out = hb || (partial && 8 * nt + 2 * tig + e >= n_lo);
+                        if (out) s[nt][e] = s[nt][2 + e] = -INFINITY;
+                    }
+                lazy_update<NT>(s, m[mb], l[mb], u[mb]);
+                if (p.mass != nullptr) {
+                    if (tig == 0) {
+                        sm.mref[b][warp][0][16 * mb + g] = m[mb][0];
+                        sm.mref[b][warp][0][16 * mb + g + 8] = m[mb][1];
+                    }
+                    #pragma unroll
+                    for (int c4 = 0; c4 < NT / 4; ++c4) {
+                        float v[16];
+                        #pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = s[4 * c4 + (i >> 2)][i & 3];
+                        tmem_st16(tcol + (uint32_t)(32 * mb + 16 * c4), v);
+                    }
+                }
+                #pragma unroll
+                for (int kk = 0; kk < NT / 2; ++kk) {
+                    uint32_t a[4];
+                    a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+                    a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+                    a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+                    a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+                    uint32_t b0, b1, b2, b3;
+                    const int row = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
+                    const int ch = lane >> 4;
+                    ldsm_x4_t(sb + kHalf + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), b0, b1, b2, b3);
+                    mma_bf16(u[mb][0], a, b0, b1);
+                    mma_bf16(u[mb][1], a, b2, b3);
+                }
+            }
+        };
 
         for (int st = 0; st < nst && ok; ++st) {
             const int slot = c_seq % kSlots;
             if (!mbar_wait(&sm.full[warp][slot], (c_seq / kSlots) & 1u, abort)) { ok = false; break; }
             const uint32_t sb = smem_u32(sm.ring[warp][slot]);
             if (st == 0 && n_lo > 0) {
-                // ------------------------------------------------ LO range
-                #pragma unroll
-                for (int hf = 0; hf < C::kLoTok / 64; ++hf) {
-                    if (64 * hf < n_lo) {
-                        uint32_t kf[4][4];
-                        #pragma unroll
-                        for (int np = 0; np < 4; ++np) {
-                            const int row = 64 * hf + 16 * np + (lane & 7) + ((lane >> 4) << 3);
-                            const int ch = (lane >> 3) & 1;
-                            ldsm_x4(sb + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), kf[np][0], kf[np][1], kf[np][2],
-                                    kf[np][3]);
-                        }
-                        #pragma unroll
-                        for (int mb = 0; mb < NMB; ++mb) {
-                            float s[8][4];
-                            #pragma unroll
-                            for (int a = 0; a < 8; ++a) s[a][0] = s[a][1] = s[a][2] = s[a][3] = 0.f;
-                            #pragma unroll
-                            for (int np = 0; np < 4; ++np) {
-                                mma_bf16(s[2 * np], qah[mb], kf[np][0], kf[np][1]);
-                                mma_bf16(s[2 * np], qal[mb], kf[np][0], kf[np][1]);
-                                mma_bf16(s[2 * np + 1], qah[mb], kf[np][2], kf[np][3]);
-                                mma_bf16(s[2 * np + 1], qal[mb], kf[np][2], kf[np][3]);
-                            }
-                            #pragma unroll
-                            for (int nt = 0; nt < 8; ++nt)
-                                #pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    const int r = 64 * hf + 8 * nt + 2 * tig + e;
-                                    const bool hb = (lw[r >> 5] >> (r & 31)) & 1u;
-                                    if (r >= n_lo || hb) s[nt][e] = s[nt][2 + e] = -INFINITY;
-                                }
-                            const float mn0 = softmax_row<8>(s, 0, m[mb][0], l[mb][0], u[mb]);
-                            const float mn1 = softmax_row<8>(s, 1, m[mb][1], l[mb][1], u[mb]);
-                            if (p.mass != nullptr) {
-                                if (tig == 0) {
-                                    sm.mref[b][warp][hf][16 * mb + g] = mn0;
-                                    sm.mref[b][warp][hf][16 * mb + g + 8] = mn1;
-                                }
-                                const uint32_t col = tcol + (uint32_t)(32 * (NMB == 1 ? hf : mb));
-                                float v0[16], v1[16];
-                                #pragma unroll
-                                for (int i = 0; i < 16; ++i) {
-                                    v0[i] = s[i >> 2][i & 3];
-                                    v1[i] = s[4 + (i >> 2)][i & 3];
-                                }
-                                tmem_st16(col, v0);
-                                tmem_st16(col + 16, v1);
-                            }
-                            #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk) {
-                                uint32_t a[4];
-                                a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-                                a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-                                a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-                                a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-                                uint32_t b0, b1, b2, b3;
-                                const int row = 64 * hf + 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
-                                const int ch = lane >> 4;
-                                ldsm_x4_t(sb + 4096 + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), b0, b1, b2, b3);
-                                mma_bf16(u[mb][0], a, b0, b1);
-                                mma_bf16(u[mb][1], a, b2, b3);
-                            }
-                        }
-                    }
-                }
+                do_lo(sb, std::integral_constant<int, 8>{});
             } else {
-                // ------------------------------------------------ HI stage
+                // ------------------------------------------------ HI stage: kHiTok full-rank tokens
                 const int hs = st - (n_lo > 0 ? 1 : 0);
                 const int n = min(kHiTok, nh - kHiTok * hs);
-                const int upd = C::kLoTok / 64 + hs;
+                const int upd = 1 + hs;
                 #pragma unroll
                 for (int mb = 0; mb < NMB; ++mb) {
-                    float s[4][4];
+                    float s[kNTH][4];
                     #pragma unroll
-                    for (int a = 0; a < 4; ++a) s[a][0] = s[a][1] = s[a][2] = s[a][3] = 0.f;
+                    for (int a = 0; a < kNTH; ++a) s[a][0] = s[a][1] = s[a][2] = s[a][3] = 0.f;
                     #pragma unroll
                     for (int kb = 0; kb < 4; ++kb) {
                         uint32_t ah[4], al[4];
@@ -871,37 +1044,45 @@ __global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant_
                             ldsm_x4(qt1 + off, al[0], al[1], al[2], al[3]);
                         }
                         #pragma unroll
-                        for (int np = 0; np < 2; ++np) {
+                        for (int np = 0; np < kNTH / 2; ++np) {
                             uint32_t b0, b1, b2, b3;
                             const int row = 16 * np + (lane & 7) + ((lane >> 4) << 3);
                             const int ch = 2 * kb + ((lane >> 3) & 1);
                             ldsm_x4(sb + row * 128 + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
                             mma_bf16(s[2 * np], ah, b0, b1);
-                            mma_bf16(s[2 * np], al, b0, b1);
                             mma_bf16(s[2 * np + 1], ah, b2, b3);
+                            mma_bf16(s[2 * np], al, b0, b1);
                             mma_bf16(s[2 * np + 1], al, b2, b3);
                         }
                     }
-                    #pragma unroll
-                    for (int nt = 0; nt < 4; ++nt)
+                    if (n < kHiTok) {
                         #pragma unroll
-                        for (int e = 0; e < 2; ++e)
-                            if (8 * nt + 2 * tig + e >= n) s[nt][e] = s[nt][2 + e] = -INFINITY;
-                    const float mn0 = softmax_row<4>(s, 0, m[mb][0], l[mb][0], u[mb]);
-                    const float mn1 = softmax_row<4>(s, 1, m[mb][1], l[mb][1], u[mb]);
+                        for (int nt = 0; nt < kNTH; ++nt)
+                            #pragma unroll
+                            for (int e = 0; e < 2; ++e)
+                                if (8 * nt + 2 * tig + e >= n) s[nt][e] = s[nt][2 + e] = -INFINITY;
+                    }
+                    lazy_update<kNTH>(s, m[mb], l[mb], u[mb]);
                     if (p.mass != nullptr) {
                         if (tig == 0) {
-                            sm.mref[b][warp][upd][16 * mb + g] = mn0;
-                            sm.mref[b][warp][upd][16 * mb + g + 8] = mn1;
+                            sm.mref[b][warp][upd][16 * mb + g] = m[mb][0];
+                            sm.mref[b][warp][upd][16 * mb + g + 8] = m[mb][1];
                         }
-                        const uint32_t col = tcol + (uint32_t)(64 + (NMB == 1 ? 16 * hs : 32 * hs + 16 * mb));
-                        float v0[16];
-                        #pragma unroll
-                        for (int i = 0; i < 16; ++i) v0[i] = s[i >> 2][i & 3];
-                        tmem_st16(col, v0);
+                        const uint32_t col = tcol + (uint32_t)(32 * NMB + (hs * NMB + mb) * 4 * kNTH);
+                        if (kNTH == 4) {
+                            float v0[16];
+                            #pragma unroll
+                            for (int i = 0; i < 16; ++i) v0[i] = s[(i >> 2) % kNTH][i & 3];
+                            tmem_st16(col, v0);
+                        } else {
+                            float v0[8];
+                            #pragma unroll
+                            for (int i = 0; i < 8; ++i) v0[i] = s[(i >> 2) % kNTH][i & 3];
+                            tmem_st8(col, v0);
+                        }
                     }
                     #pragma unroll
-                    for (int kk = 0; kk < 2; ++kk) {
+                    for (int kk = 0; kk < kNTH / 2; ++kk) {
                         uint32_t a[4];
                         a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
                         a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
@@ -912,7 +1093,7 @@ __global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant_
                             uint32_t b0, b1, b2, b3;
                             const int row = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
                             const int ch = 2 * pr + (lane >> 4);
-                            ldsm_x4_t(sb + 4096 + row * 128 + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
+                            ldsm_x4_t(sb + kHalf + row * 128 + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
                             mma_bf16(u[mb][2 * pr], a, b0, b1);
                             mma_bf16(u[mb][2 * pr + 1], a, b2, b3);
                         }
@@ -939,58 +1120,143 @@ __global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant_
                     sm.wl[warp][16 * mb + g + 8 * r] = lt;
                 }
             }
+        if (tid < C::kRows) {   // the next item's query block lands in sm.tst after the barrier
+            sm.tcur[tid][0] = tid < p.Hg ? sm.tst[tid][0] : -INFINITY;
+            sm.tcur[tid][1] = tid < p.Hg ? sm.tst[tid][1] : 0.f;
+        }
+        // the previous item's unit (max, 1/sum), read now and stored after the merge
+        float pf0 = 0.f, pf1 = 0.f;
+        const bool prefetch = p.mass != nullptr && p.S > 1 && K >= 1 && tid < p.Hg;
+        if (prefetch) {
+            const float *us = p.ustat + ((size_t)(item_of(K - 1) / p.S) * p.Hg + tid) * 2;
+            asm volatile("ld.relaxed.gpu.global.v2.f32 {%0, %1}, [%2];" : "=f"(pf0), "=f"(pf1) : "l"(us) : "memory");
+        }
         tmem_fence_before();
         __syncthreads();
         if (*abort) break;
         if (tid == 0 && item_of(K + 1) < p.n_items) issue_q(K + 1);
         if (tid < C::kRows) {
-            float mx = -INFINITY;
-            for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, sm.wm[w][tid]);
+            float mx = sm.wm[0][tid];
+            #pragma unroll
+            for (int w = 1; w < kWarps; ++w) mx = fmaxf(mx, sm.wm[w][tid]);
             float sum = 0.f;
-            if (mx != -INFINITY)
-                for (int w = 0; w < kWarps; ++w) {
-                    const float mw_ = sm.wm[w][tid];
-                    if (mw_ != -INFINITY) sum += sm.wl[w][tid] * ex2(mw_ - mx);
-                }
+            #pragma unroll
+            for (int w = 0; w < kWarps; ++w) sum += sm.wl[w][tid] * ex2(sm.wm[w][tid] - mx);
             sm.mcta[tid] = mx;
             sm.lcta[tid] = sum;
+            if (p.S == 1) {   // the unit's max and sum: this block's visual part and the text tail
+                const float t0m = sm.tcur[tid][0];
+                const float M = fmaxf(mx, t0m);
+                float L = sum * ex2(mx - M);
+                if (t0m != -INFINITY) L += sm.tcur[tid][1] * ex2(t0m - M);
+                sm.mfin[tid] = M;
+                sm.invl[tid] = 1.f / L;
+            }
         }
-        __syncthreads();
+        // every thread rescales its u rows to the block reference (the max of the warps' references)
         #pragma unroll
         for (int mb = 0; mb < NMB; ++mb)
             #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const int row = 16 * mb + g + 8 * r;
-                const float f = (row < p.Hg && m[mb][r] != -INFINITY) ? ex2(m[mb][r] - sm.mcta[row]) : 0.f;
-                if (f != 0.f) {
+                float mc = sm.wm[0][row];
+                #pragma unroll
+                for (int w = 1; w < kWarps; ++w) mc = fmaxf(mc, sm.wm[w][row]);
+                const float f = row < p.Hg ? ex2(m[mb][r] - mc) : 0.f;
+                #pragma unroll
+                for (int nt = 0; nt < 8; ++nt) {
+                    u[mb][nt][2 * r] *= f;
+                    u[mb][nt][2 * r + 1] *= f;
+                }
+            }
+        // sum over the 8 warps, one 16-row block at a time: warps 4-7 hand their u to warps
+        // 0-3, which hand the pair sums on; every thread then adds the four for 4 outputs
+        {
+            float *dst = p.part + ((size_t)unit * p.S + split) * p.Hg * kVisPart;
+            #pragma unroll
+            for (int mb = 0; mb < NMB; ++mb) {
+                float *ub = &sm.ubuf[warp & 3][0][0];
+                if (mb > 0) __syncthreads();   // the previous block's sums have been read
+                if (warp >= 4) {
+                    #pragma unroll
+                    for (int nt = 0; nt < 8; ++nt)
+                        *reinterpret_cast<float4 *>(ub + 4 * (32 * nt + lane)) =
+                            make_float4(u[mb][nt][0], u[mb][nt][1], u[mb][nt][2], u[mb][nt][3]);
+                }
+                __syncthreads();
+                if (warp < 4) {
                     #pragma unroll
                     for (int nt = 0; nt < 8; ++nt) {
-                        atomicAdd(&sm.u_acc[row][8 * nt + 2 * tig], u[mb][nt][2 * r] * f);
-                        atomicAdd(&sm.u_acc[row][8 * nt + 2 * tig + 1], u[mb][nt][2 * r + 1] * f);
+                        const float4 v = *reinterpret_cast<const float4 *>(ub + 4 * (32 * nt + lane));
+                        *reinterpret_cast<float4 *>(ub + 4 * (32 * nt + lane)) =
+                            make_float4(u[mb][nt][0] + v.x, u[mb][nt][1] + v.y, u[mb][nt][2] + v.z, u[mb][nt][3] + v.w);
+                    }
+                }
+                __syncthreads();
+                // output (row, col) of the block: fragment (nt = col / 8, lane = 4 (row % 8) + (col % 8) / 2,
+                // element 2 (row / 8) + col % 2)
+                for (int o = tid; o < 16 * 64; o += kThreads) {
+                    const int row = o >> 6, col = o & 63;
+                    const int h = 16 * mb + row;
+                    if (h < p.Hg) {
+                        const int off = 4 * (32 * (col >> 3) + 4 * (row & 7) + ((col & 7) >> 1)) + 2 * (row >> 3) + (col & 1);
+                        const float v = sm.ubuf[0][0][off] + sm.ubuf[1][0][off] + sm.ubuf[2][0][off] + sm.ubuf[3][0][off];
+                        dst[(size_t)h * kVisPart + 2 + col] = v;
                     }
                 }
             }
-        __syncthreads();
-        {
-            float *dst = p.part + ((size_t)unit * p.S + split) * p.Hg * kVisPart;
-            for (int i = tid; i < p.Hg * kVisPart; i += kThreads) {
-                const int h = i / kVisPart, f = i % kVisPart;
-                float v;
-                if (f == 0) v = sm.mcta[h];
-                else if (f == 1) v = sm.lcta[h];
-                else { v = sm.u_acc[h][f - 2]; sm.u_acc[h][f - 2] = 0.f; }
-                dst[i] = v;
+            if (tid < p.Hg) {
+                dst[(size_t)tid * kVisPart] = sm.mcta[tid];
+                dst[(size_t)tid * kVisPart + 1] = sm.lcta[tid];
             }
         }
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" :: "l"(&p.arrive[unit]) : "memory");
-        if (p.mass != nullptr && K >= 1) {
-            mass_of(K - 1);
-            if (*abort) break;
+        if (prefetch) { sm.upf[tid][0] = pf0; sm.upf[tid][1] = pf1; }
+        if (p.mass == nullptr) continue;
+        if (p.S == 1) {
+            mass_warp(K, 0);
+            continue;
         }
+        // several splits: the last one to publish fixes the unit's (max, 1/sum), warp per head
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            unsigned int old;
+            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&p.arrive[unit]) : "memory");
+            sm.last = (old == (unsigned int)(p.S - 1));
+        }
+        __syncthreads();
+        if (sm.last) {
+            for (int h = warp; h < p.Hg; h += kWarps) {
+                const float *vp = p.part + (size_t)unit * p.S * p.Hg * kVisPart + (size_t)h * kVisPart;
+                float mx = sm.tcur[h][0], ml[4], ll[4];
+                #pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int sp = lane + 32 * k;
+                    ml[k] = sp < p.S ? __ldcg(vp + (size_t)sp * p.Hg * kVisPart) : kRefInit;
+                    ll[k] = sp < p.S ? __ldcg(vp + (size_t)sp * p.Hg * kVisPart + 1) : 0.f;
+                    mx = fmaxf(mx, ml[k]);
+                }
+                for (int sp = lane + 128; sp < p.S; sp += 32) mx = fmaxf(mx, __ldcg(vp + (size_t)sp * p.Hg * kVisPart));
+                #pragma unroll
+                for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+                float sum = 0.f;
+                #pragma unroll
+                for (int k = 0; k < 4; ++k) sum += ll[k] * ex2(ml[k] - mx);
+                for (int sp = lane + 128; sp < p.S; sp += 32)
+                    sum += __ldcg(vp + (size_t)sp * p.Hg * kVisPart + 1) * ex2(__ldcg(vp + (size_t)sp * p.Hg * kVisPart) - mx);
+                #pragma unroll
+                for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
+                if (lane == 0) {
+                    if (sm.tcur[h][0] != -INFINITY) sum += sm.tcur[h][1] * ex2(sm.tcur[h][0] - mx);
+                    float *us = p.ustat + ((size_t)unit * p.Hg + h) * 2;
+                    const float inv = 1.f / sum;
+                    asm volatile("st.relaxed.gpu.global.v2.f32 [%0], {%1, %2};" :: "l"(us), "f"(mx), "f"(inv) : "memory");
+                }
+            }
+        }
+        if (K >= 1) mass_warp(K - 1, 2);
     }
-    if (p.mass != nullptr && K >= 1 && !*abort) mass_of(K - 1);
+    if (p.mass != nullptr && p.S > 1 && K >= 1 && !*abort) mass_warp(K - 1, 1);
 
     // copies still in flight (only after an abort) must land before the block exits
     while (c_seq < i_seq) {
@@ -1005,7 +1271,7 @@ __global__ void __launch_bounds__(kThreads, 1) vis_kernel(const __grid_constant_
     __syncthreads();
     if (warp == 0) {
         tmem_fence_after();
-        tmem_dealloc(sm.tmem_base, 512);
+        tmem_dealloc(sm.tmem_base, C::kTmemCols);
     }
 }
 
@@ -1021,79 +1287,111 @@ struct FinishParams {
     int Hg, per_kv, n_q, groups, S, Sc;
 };
 
-// One block per unit: unit-wide max and sum per head, u / l and w / l from the
-// partials, then o_h = (u_h / l_h) B_V[:, 128 j(h) ..] + w_h / l_h with thread
-// t owning output columns 2t, 2t+1 of the unit's 512 (KV head t / 64).
+// dynamic shared memory of finish_kernel: weights of every partial, then u / l and w / l
+__host__ __device__ constexpr size_t finish_smem_bytes(int S, int Sc) {
+    return (size_t)(S + Sc) * kMaxHeads * sizeof(float) + (size_t)kMaxHeads * (64 + 128) * sizeof(float);
+}
+
+// One block per unit.  Per head, the unit-wide max M and sum L over every
+// visual and text partial give each partial the weight 2^(m - M) / L; u / l and
+// w / l are weighted sums with the feature index across threads (coalesced).
+// Then o_h = (u_h / l_h) B_V[:, 128 j(h) ..] + w_h / l_h, thread t owning output
+// columns 2t, 2t+1 of the unit's 512 (KV head t / 64).
 __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
-    __shared__ float mfin[kMaxHeads], invl[kMaxHeads];
-    __shared__ float uf[kMaxHeads][64];
-    __shared__ float wf[kMaxHeads][128];
+    extern __shared__ float fsm[];
+    float *wv = fsm;                                  // [S][kMaxHeads]
+    float *wt = wv + p.S * kMaxHeads;                 // [Sc][kMaxHeads]
+    float (*uf)[64] = reinterpret_cast<float (*)[64]>(wt + p.Sc * kMaxHeads);
+    float (*wf)[128] = reinterpret_cast<float (*)[128]>(&uf[kMaxHeads][0]);
     const int unit = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const float *vp0 = p.vpart + (size_t)unit * p.S * p.Hg * kVisPart;
     const float *tp0 = p.tpart + (size_t)unit * p.Sc * p.Hg * kTxtPart;
 
-    // B_V columns 2t, 2t+1 of all 64 rank rows (issued first: independent of the partials)
-    const uint32_t *bv = reinterpret_cast<const uint32_t *>(p.BV + (size_t)unit * 64 * 512) + tid;
-    uint32_t braw[64];
-    #pragma unroll
-    for (int i = 0; i < 64; ++i) braw[i] = __ldcs(bv + i * 256);
-
     for (int h = warp; h < p.Hg; h += 8) {
         float mx = -INFINITY;
-        for (int s = lane; s < p.S; s += 32) mx = fmaxf(mx, vp0[((size_t)s * p.Hg + h) * kVisPart]);
-        for (int c = lane; c < p.Sc; c += 32) mx = fmaxf(mx, tp0[((size_t)c * p.Hg + h) * kTxtPart]);
+        for (int s = lane; s < p.S; s += 32) mx = fmaxf(mx, __ldcg(vp0 + ((size_t)s * p.Hg + h) * kVisPart));
+        for (int c = lane; c < p.Sc; c += 32) mx = fmaxf(mx, __ldcg(tp0 + ((size_t)c * p.Hg + h) * kTxtPart));
         #pragma unroll
         for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
         float sum = 0.f;
         for (int s = lane; s < p.S; s += 32) {
             const float *r = vp0 + ((size_t)s * p.Hg + h) * kVisPart;
-            if (r[0] != -INFINITY) sum += r[1] * ex2(r[0] - mx);
+            const float e = ex2(__ldcg(r) - mx);
+            wv[s * kMaxHeads + h] = e;
+            sum += __ldcg(r + 1) * e;
         }
         for (int c = lane; c < p.Sc; c += 32) {
             const float *r = tp0 + ((size_t)c * p.Hg + h) * kTxtPart;
-            if (r[0] != -INFINITY) sum += r[1] * ex2(r[0] - mx);
+            const float m = __ldcg(r);
+            const float e = (m != -INFINITY) ? ex2(m - mx) : 0.f;
+            wt[c * kMaxHeads + h] = e;
+            sum += (m != -INFINITY) ? __ldcg(r + 1) * e : 0.f;
         }
         #pragma unroll
         for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
-        if (lane == 0) {
-            mfin[h] = mx;
-            invl[h] = 1.f / sum;
-        }
+        const float inv = 1.f / sum;
+        __syncwarp();
+        for (int s = lane; s < p.S; s += 32) wv[s * kMaxHeads + h] *= inv;
+        for (int c = lane; c < p.Sc; c += 32) wt[c * kMaxHeads + h] *= inv;
     }
     __syncthreads();
-    for (int task = tid; task < p.Hg * 192; task += 256) {
-        const int h = task / 192, f = task % 192;
-        const float mh = mfin[h];
-        float acc = 0.f;
-        if (f < 64) {
-            for (int s = 0; s < p.S; ++s) {
-                const float *r = vp0 + ((size_t)s * p.Hg + h) * kVisPart;
-                if (r[0] != -INFINITY) acc = fmaf(r[2 + f], ex2(r[0] - mh), acc);
-            }
-            uf[h][f] = acc * invl[h];
-        } else {
-            for (int c = 0; c < p.Sc; ++c) {
-                const float *r = tp0 + ((size_t)c * p.Hg + h) * kTxtPart;
-                if (r[0] != -INFINITY) acc = fmaf(r[2 + f - 64], ex2(r[0] - mh), acc);
-            }
-            wf[h][f - 64] = acc * invl[h];
+    for (int task = tid; task < p.Hg * 64; task += 256) {
+        const int h = task >> 6, f = task & 63;
+        const float *r = vp0 + (size_t)h * kVisPart + 2 + f;
+        float a0 = 0.f, a1 = 0.f;
+        int s = 0;
+        for (; s + 2 <= p.S; s += 2) {
+            a0 = fmaf(__ldcg(r + (size_t)s * p.Hg * kVisPart), wv[s * kMaxHeads + h], a0);
+            a1 = fmaf(__ldcg(r + (size_t)(s + 1) * p.Hg * kVisPart), wv[(s + 1) * kMaxHeads + h], a1);
         }
+        if (s < p.S) a0 = fmaf(__ldcg(r + (size_t)s * p.Hg * kVisPart), wv[s * kMaxHeads + h], a0);
+        uf[h][f] = a0 + a1;
+    }
+    for (int task = tid; task < p.Hg * 128; task += 256) {
+        const int h = task >> 7, f = task & 127;
+        const float *r = tp0 + (size_t)h * kTxtPart + 2 + f;
+        float a0 = 0.f, a1 = 0.f;
+        int c = 0;
+        for (; c + 2 <= p.Sc; c += 2) {
+            a0 = fmaf(__ldcg(r + (size_t)c * p.Hg * kTxtPart), wt[c * kMaxHeads + h], a0);
+            a1 = fmaf(__ldcg(r + (size_t)(c + 1) * p.Hg * kTxtPart), wt[(c + 1) * kMaxHeads + h], a1);
+        }
+        if (c < p.Sc) a0 = fmaf(__ldcg(r + (size_t)c * p.Hg * kTxtPart), wt[c * kMaxHeads + h], a0);
+        wf[h][f] = a0 + a1;
     }
     __syncthreads();
     const int j = tid >> 6, d = (2 * tid) & 127;
     const int lb = unit / p.groups, G = unit % p.groups;
-    for (int hh = 0; hh < p.per_kv; ++hh) {
-        const int h = j * p.per_kv + hh;
-        float a0 = 0.f, a1 = 0.f;
+    const uint32_t *bv = reinterpret_cast<const uint32_t *>(p.BV + (size_t)unit * 64 * 512) + tid;
+    float acc[8][2];
+    #pragma unroll
+    for (int hh = 0; hh < 8; ++hh) acc[hh][0] = acc[hh][1] = 0.f;
+    const int h0 = j * p.per_kv;
+    #pragma unroll 4
+    for (int i0 = 0; i0 < 64; i0 += 16) {
+        uint32_t braw[16];
         #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            const float x = uf[h][i];
-            a0 = fmaf(x, __uint_as_float(braw[i] << 16), a0);
-            a1 = fmaf(x, __uint_as_float(braw[i] & 0xffff0000u), a1);
+        for (int i = 0; i < 16; ++i) braw[i] = __ldcs(bv + (i0 + i) * 256);
+        #pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float b0 = __uint_as_float(braw[i] << 16), b1 = __uint_as_float(braw[i] & 0xffff0000u);
+            #pragma unroll
+            for (int hh = 0; hh < 8; ++hh) {
+                if (hh < p.per_kv) {
+                    const float x = uf[h0 + hh][i0 + i];
+                    acc[hh][0] = fmaf(x, b0, acc[hh][0]);
+                    acc[hh][1] = fmaf(x, b1, acc[hh][1]);
+                }
+            }
         }
-        a0 += wf[h][d];
-        a1 += wf[h][d + 1];
-        *reinterpret_cast<uint32_t *>(p.out + ((size_t)lb * p.n_q + (size_t)G * p.Hg + h) * 128 + d) = pack_bf16(a0, a1);
+    }
+    #pragma unroll
+    for (int hh = 0; hh < 8; ++hh) {
+        if (hh < p.per_kv) {
+            const int h = h0 + hh;
+            *reinterpret_cast<uint32_t *>(p.out + ((size_t)lb * p.n_q + (size_t)G * p.Hg + h) * 128 + d) =
+                pack_bf16(acc[hh][0] + wf[h][d], acc[hh][1] + wf[h][d + 1]);
+        }
     }
 }
 
@@ -1103,7 +1401,7 @@ __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
 namespace kvpack {
 namespace decode {
 // one block per SM: the opt-in shared-memory limit per block on sm_100 is 232448 bytes
-static_assert(vis::smem_bytes<1>() <= 232448, "visual kernel (16 head rows) shared memory");
+static_assert(2 * (vis::smem_bytes<1>() + 1024) <= 233472, "visual kernel (16 head rows): two blocks per SM");
 static_assert(vis::smem_bytes<2>() <= 232448, "visual kernel (32 head rows) shared memory");
 static_assert(text::smem_bytes() <= 232448, "text kernel shared memory");
 }  // namespace decode

@@ -17,7 +17,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxT = 65536;
+constexpr int kMaxT = KVPACK_MAX_T;
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -32,7 +32,7 @@ kvpack_status check_dims(const kvpack_dims *d, int32_t n_layers) {
         return KVPACK_ERR_UNSUPPORTED;
     if (d->n_kv_heads % KVPACK_GROUP != 0 || d->n_q_heads % d->n_kv_heads != 0) return KVPACK_ERR_UNSUPPORTED;
     if ((d->n_q_heads / d->n_kv_heads) * KVPACK_GROUP > 32) return KVPACK_ERR_UNSUPPORTED;
-    if (d->T_vis > kMaxT) return KVPACK_ERR_UNSUPPORTED;
+    if (d->T_vis > kMaxT || d->L_text_cap > KVPACK_MAX_TEXT) return KVPACK_ERR_UNSUPPORTED;
     const long long units = (long long)n_layers * d->batch * (d->n_kv_heads / KVPACK_GROUP);
     if (units > (1LL << 30)) return KVPACK_ERR_UNSUPPORTED;
     return KVPACK_OK;
@@ -49,7 +49,7 @@ constexpr int kTextChunk = 64;
 
 struct DecodePlan {
     int nmb, S, tps, units, Hg, Sc_max;
-    size_t off_qt, off_tp, off_vp, off_arrive, off_counter, total;
+    size_t off_qt, off_tp, off_vp, off_ustat, off_arrive, off_counter, total;
 };
 
 // Visual splits: at most Cfg<NMB>::kItemTok tokens each, 32-aligned, and of
@@ -78,11 +78,13 @@ DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
     pl.Sc_max = (d->L_text_cap + kTextChunk - 1) / kTextChunk;
     size_t off = 0;
     pl.off_qt = off;
-    off = align256(off + (size_t)pl.units * 2 * pl.Hg * 64 * sizeof(uint16_t));
+    off = align256(off + (size_t)pl.units * kvpack::decode::qblock_bytes(pl.Hg));
     pl.off_tp = off;
     off = align256(off + (size_t)pl.units * pl.Sc_max * pl.Hg * kvpack::decode::kTxtPart * sizeof(float));
     pl.off_vp = off;
     off = align256(off + (size_t)pl.units * pl.S * pl.Hg * kvpack::decode::kVisPart * sizeof(float));
+    pl.off_ustat = off;
+    off = align256(off + (size_t)pl.units * pl.Hg * 2 * sizeof(float));
     pl.off_arrive = off;
     off += (size_t)pl.units * sizeof(unsigned int);
     pl.off_counter = off;
@@ -111,7 +113,14 @@ kvpack_status device_info(DeviceInfo **out) {
             cudaFuncSetAttribute(dc::vis::vis_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)dc::vis::smem_bytes<2>()) != cudaSuccess ||
             cudaFuncSetAttribute(dc::text::text_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)dc::text::smem_bytes()) != cudaSuccess)
+                                 (int)dc::text::smem_bytes()) != cudaSuccess ||
+            cudaFuncSetAttribute(dc::finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)dc::finish_smem_bytes(kMaxT / 512 + 8, (KVPACK_MAX_TEXT + kTextChunk - 1) / kTextChunk)) != cudaSuccess)
+            return KVPACK_ERR_CUDA;
+        // all of the SM's shared memory for these kernels (two visual blocks of the 16-row variant)
+        if (cudaFuncSetAttribute(dc::vis::vis_kernel<1>, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
+            cudaFuncSetAttribute(dc::vis::vis_kernel<2>, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
+            cudaFuncSetAttribute(dc::text::text_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
             return KVPACK_ERR_CUDA;
         int b1 = 0, b2 = 0, bt = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b1, dc::vis::vis_kernel<1>, dc::vis::kThreads,
@@ -121,8 +130,11 @@ kvpack_status device_info(DeviceInfo **out) {
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bt, dc::text::text_kernel, dc::text::kThreads,
                                                           dc::text::smem_bytes()) != cudaSuccess)
             return KVPACK_ERR_CUDA;
-        // the visual kernel holds all 512 tensor-memory columns of its SM: exactly one block per SM
-        if (b1 != 1 || b2 != 1 || bt < 1) return KVPACK_ERR_CUDA;
+        // The occupancy calculator counts a kernel that allocates tensor memory as one block per
+        // SM; the 16-row visual kernel is sized for two (124 registers x 256 threads, 88 KB of
+        // shared memory and 256 of the SM's 512 tensor-memory columns each), and B200s run two
+        // such blocks side by side.  Its grid is therefore sized from Cfg::kBlocks.
+        if (b1 < 1 || b2 != dc::vis::Cfg<2>::kBlocks || bt < 1) return KVPACK_ERR_CUDA;
         kvpack_status cs = kvpack::compress::prepare_device();
         if (cs != KVPACK_OK) return cs;
         di.ready = true;
@@ -247,6 +259,7 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
         if (ptr && !aligned16(ptr)) return KVPACK_ERR_ALIGNMENT;
     const DecodePlan pl = plan_decode(d, n_layers);
     if (pl.S <= 0) return KVPACK_ERR_UNSUPPORTED;
+    if ((long long)pl.units * d->T_vis * 3 >= (1LL << 31)) return KVPACK_ERR_UNSUPPORTED;   // int32 gather rows
     if (ws == nullptr || ws_bytes < pl.total) return KVPACK_ERR_WORKSPACE;
     DeviceInfo *di = nullptr;
     if ((s = device_info(&di)) != KVPACK_OK) return s;
@@ -260,23 +273,23 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     const int Sc = (L_text + kTextChunk - 1) / kTextChunk;
     const float scale2 = softmax_scale * 1.4426950408889634f;
     unsigned char *w = static_cast<unsigned char *>(ws);
-    uint16_t *qt = reinterpret_cast<uint16_t *>(w + pl.off_qt);
+    unsigned char *qt = w + pl.off_qt;
     float *tpart = reinterpret_cast<float *>(w + pl.off_tp);
     float *vpart = reinterpret_cast<float *>(w + pl.off_vp);
+    float *ustat = reinterpret_cast<float *>(w + pl.off_ustat);
     unsigned int *arrive = reinterpret_cast<unsigned int *>(w + pl.off_arrive);
     unsigned int *counter = reinterpret_cast<unsigned int *>(w + pl.off_counter);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    // arrival counters and the text work counter start at zero
+    // arrival counters and the text work counter start at zero; the unit statistics
+    // that several splits wait for start as NaN (all-ones bytes)
     if (cudaMemsetAsync(arrive, 0, pl.off_counter + sizeof(unsigned int) - pl.off_arrive, st) != cudaSuccess)
         return KVPACK_ERR_CUDA;
+    if (pl.S > 1 && mass != nullptr &&
+        cudaMemsetAsync(ustat, 0xff, (size_t)pl.units * Hg * 2 * sizeof(float), st) != cudaSuccess)
+        return KVPACK_ERR_CUDA;
 
-    // 1. q~ per unit
-    dc::QProjParams qp{q, BK, qt, Hg, per_kv, d->n_q_heads, groups, scale2};
-    dc::qproj_kernel<<<pl.units, 256, 0, st>>>(qp);
-    if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
-
-    // 2. text tail partials
+    // 1. text tail partials
     if (L_text > 0) {
         dc::text::Params tp;
         std::memset(&tp, 0, sizeof(tp));
@@ -294,6 +307,12 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
         if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
     }
 
+    // 2. q~ per unit, with the text tail's (max, sum) per head
+    dc::QProjParams qp{q, BK, qt, Sc > 0 ? tpart : nullptr, Hg, per_kv, d->n_q_heads, groups, Sc, scale2};
+    if (per_kv <= 2) dc::qproj_rows_kernel<<<pl.units, 256, 0, st>>>(qp);
+    else dc::qproj_cols_kernel<<<pl.units, 256, 0, st>>>(qp);
+    if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
+
     // 3. visual partials and the attention mass
     {
         dc::vis::Params vp;
@@ -305,17 +324,19 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
             !encode_bf16(enc, &vp.tm_cv, CV_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return KVPACK_ERR_CUDA;
         vp.CK_lo = CK_lo; vp.CK_hi = CK_hi; vp.CV_lo = CV_lo; vp.CV_hi = CV_hi;
-        vp.qt = qt; vp.mask = mask; vp.mass = mass; vp.part = vpart; vp.tpart = Sc > 0 ? tpart : nullptr;
-        vp.arrive = arrive;
+        vp.qt = qt; vp.mask = mask; vp.mass = mass; vp.part = vpart; vp.ustat = ustat; vp.arrive = arrive;
         vp.n_units = pl.units; vp.T = T; vp.Hg = Hg; vp.S = pl.S; vp.tps = pl.tps; vp.nwords = (T + 31) / 32;
-        vp.Sc = Sc; vp.n_items = pl.units * pl.S;
-        const int grid = vp.n_items < di->sms ? vp.n_items : di->sms;
+        vp.n_items = pl.units * pl.S;
+        const int resident = di->sms * (pl.nmb == 1 ? dc::vis::Cfg<1>::kBlocks : dc::vis::Cfg<2>::kBlocks);
+        const int grid = vp.n_items < resident ? vp.n_items : resident;
         if (pl.S > grid) return KVPACK_ERR_UNSUPPORTED;   // every split of a unit must be co-resident
         void *args[] = {&vp};
         const void *fn = (pl.nmb == 1) ? (const void *)dc::vis::vis_kernel<1> : (const void *)dc::vis::vis_kernel<2>;
         const size_t smem = (pl.nmb == 1) ? dc::vis::smem_bytes<1>() : dc::vis::smem_bytes<2>();
+        // Splits of a unit wait (boundedly) for one another: the grid never exceeds what is
+        // resident at once.  The 32-row variant asks for that guarantee with a cooperative launch.
         cudaError_t e;
-        if (pl.S > 1 && mass != nullptr)
+        if (pl.nmb == 2 && pl.S > 1 && mass != nullptr)
             e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(dc::vis::kThreads), args, smem, st);
         else
             e = cudaLaunchKernel(fn, dim3(grid), dim3(dc::vis::kThreads), args, smem, st);
@@ -324,7 +345,7 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
 
     // 4. combine and project through B_V
     dc::FinishParams fp{BV, vpart, Sc > 0 ? tpart : nullptr, out, Hg, per_kv, d->n_q_heads, groups, pl.S, Sc};
-    dc::finish_kernel<<<pl.units, 256, 0, st>>>(fp);
+    dc::finish_kernel<<<pl.units, 256, dc::finish_smem_bytes(pl.S, Sc), st>>>(fp);
     return (cudaGetLastError() == cudaSuccess) ? KVPACK_OK : KVPACK_ERR_CUDA;
 }
 
