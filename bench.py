@@ -16,6 +16,7 @@ the workload (independent units, no collective on the data path); the step
 time is the max over ranks and value counts the units of all ranks.
 """
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -73,23 +74,27 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback (profiling recipe)"
 
 
+DECODE_SOURCES = ("decode.cuh", "common.cuh", "kvpack.cu")
+
+
+def sources_digest(names=DECODE_SOURCES) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "rank_compressed_kv_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def recorded_traffic(kernel: str, config: str):
-    """dram bytes per launch from the committed ncu summary, if it was taken on the current kernel source."""
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current kernel sources."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
-    except Exception:
+        ent = rec[f"{kernel}:{config}"]
+        return ent["bytes_per_launch"] if ent["sources_sha256_16"] == sources_digest() else None
+    except (OSError, KeyError, ValueError):
         return None
-    ent = rec.get(f"{kernel}:{config}")
-    if not ent:
-        return None
-    src = os.path.join(ROOT, "rank_compressed_kv_b200", "csrc", ent["source"])
-    try:
-        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    except OSError:
-        return None
-    return ent["bytes_per_launch"] if digest == ent["sha256_16"] else None
 
 
 # ------------------------------------------------------------------ clocks
@@ -311,7 +316,8 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
                    "step": "kvpack_select + kvpack_decode_attn over all layers"},
         "step_bytes": int(sbytes),
         "step_GBps": round(sbytes / (ms_step / 1e3) / 1e9, 1),
-        "roofline": {"bound": "hbm", "kernel": "kvpack_decode_attn (qproj_kernel + attn_kernel)",
+        "roofline": {"bound": "hbm",
+                     "kernel": "kvpack_decode_attn (text_kernel, qproj_*_kernel, vis_kernel, finish_kernel on one stream)",
                      "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4), "frac_of_8TBps": round(achieved / 8000.0, 4),
                      "peak_kind": peak_kind,
@@ -319,7 +325,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
                      "traffic": recorded_traffic("decode", w.name)},
         "e2e": {"value": round(e2e_value, 1), "unit": "query-tokens/s", "h2d_bytes_per_step": qbytes,
                 "d2h_bytes_per_step": obytes, "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": 3 * K,
+        "gpu_launches": (5 if L0 > 0 else 4) * K,   # per step: select + text + q~ projection + visual + finish
         "clocks": clk,
         "wall_s_timed": round(wall, 3),
     }
@@ -334,7 +340,51 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
 
 
 def bench_compress(kv, torch, w, dev):
-    return None
+    """kvpack_compress on one layer of the workload (K side), timed with CUDA events; per-kernel
+    device times from the CUDA profiler give the Gram's rate against the measured bf16 peak."""
+    from torch.profiler import profile, ProfilerActivity
+    units = w.batch * (w.n_kv // 4)
+    dims = kv.Dims(batch=units, n_q_heads=4, n_kv_heads=4, T_vis=w.T, L_text_cap=1)
+    pool = [synth.visual_kv(w, 0, b, 0, synth.K_VIS) for b in range(min(POOL, units))]
+    X = torch.empty(units, w.T, 512, dtype=torch.bfloat16, device=dev)
+    for u in range(units):
+        X[u].copy_(torch.from_numpy(pool[u % len(pool)].view(np.int16)).view(torch.bfloat16))
+    C_lo = torch.empty(units, w.T, 16, dtype=torch.bfloat16, device=dev)
+    C_hi = torch.empty(units, w.T, 48, dtype=torch.bfloat16, device=dev)
+    B = torch.empty(units, 64, 512, dtype=torch.bfloat16, device=dev)
+    sig = torch.empty(units, 64, dtype=torch.float32, device=dev)
+    ws = torch.empty(kv.compress_workspace(dims, 1), dtype=torch.uint8, device=dev)
+
+    def run():
+        kv.compress(dims, 1, X, C_lo, C_hi, B, sig, ws)
+
+    run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    run()
+    e1.record()
+    torch.cuda.synchronize()
+    st = kv.last_device_status()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        run()
+        torch.cuda.synchronize()
+    kern = {}
+    for e in prof.events():
+        if e.device_type.name == "CUDA":
+            name = e.name.split("(")[0].split("::")[-1]
+            kern[name] = kern.get(name, 0.0) + e.device_time_total / 1e3
+    _, bf16, peak_kind = measured_peaks()
+    gram_ms = kern.get("gram_tc_kernel", float("nan"))
+    full = 2.0 * units * w.T * 512 * 512                  # the full product X^T X
+    executed = full * (128 * (512 + 384 + 256 + 128)) / (512 * 512)   # upper bands as computed
+    return {"units": units, "T": w.T, "ms_per_layer_matrix": round(e0.elapsed_time(e1), 3), "status": st,
+            "kernel_ms": {k: round(v, 3) for k, v in kern.items()},
+            "gram": {"full_2Tn2_tflops": round(full / (gram_ms / 1e3) / 1e12, 1),
+                     "executed_tflops": round(executed / (gram_ms / 1e3) / 1e12, 1),
+                     "peak_tflops": bf16, "peak_kind": peak_kind,
+                     "frac_full_2Tn2": round(full / (gram_ms / 1e3) / 1e12 / bf16, 4),
+                     "frac_executed": round(executed / (gram_ms / 1e3) / 1e12 / bf16, 4)}}
 
 
 # ------------------------------------------------------------------ oracle (CPU) arm
@@ -434,12 +484,18 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--compress", action="store_true", help="also time kvpack_compress on the workload")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="run the config with fewer layers (a small case for profiler captures; named in the line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = synth.WORKLOADS[args.config]
     if args.hi_frac is not None:
         w = w.with_hi_frac(args.hi_frac)
+    if args.layers is not None:
+        if not 1 <= args.layers <= w.layers:
+            ap.error(f"--layers must be in 1..{w.layers}")
+        w = dataclasses.replace(w, name=f"{w.name}[{args.layers} of {w.layers} layers]", layers=args.layers)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.gpus != world and args.impl == "ours":

@@ -5,9 +5,10 @@
 // storage falls from T x H x D to T x R + R x H x D).
 //
 // Per unit X (T x 512, bf16) the rank-64 truncated SVD X ~ C B is computed as
-//   1. gram_kernel     G = X^T X (512 x 512, fp32 accumulation) on the tensor
-//                      cores; only the 10 upper-triangle 128 x 128 blocks are
-//                      computed, each written with its mirror.
+//   1. gram_tc_kernel  G = X^T X (512 x 512, fp32 accumulation) on the 5th-
+//                      generation tensor cores (tcgen05.mma, accumulator in tensor
+//                      memory, operands staged by TMA); only the upper 128-row bands
+//                      right of the diagonal are computed, then mirrored.
 //   2. eig_kernel      top-64 eigenpairs of G by blocked subspace iteration
 //                      with p = 96 columns: Y = G Q (three-product bf16 split
 //                      on the tensor cores, ~fp32 accurate), then Y is
@@ -75,95 +76,7 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
 
-// ================================================================== Gram (mma.sync)
 
-constexpr int kGramThreads = 256;
-constexpr int kGramKT = 32;   // tokens per k-step
-
-__global__ void __launch_bounds__(kGramThreads) gram_kernel(const uint16_t *__restrict__ X, int T, float *__restrict__ G) {
-    __shared__ __align__(128) unsigned char sA[2][kGramKT * 256];
-    __shared__ __align__(128) unsigned char sB[2][kGramKT * 256];
-    const int unit = blockIdx.x / 10, blk = blockIdx.x % 10;
-    // upper-triangle block (bi <= bj) of the 4 x 4 grid of 128 x 128 blocks
-    int bi = 0, bj = blk;
-    if (blk >= 4) { bi = 1; bj = blk - 3; }
-    if (blk >= 7) { bi = 2; bj = blk - 5; }
-    if (blk == 9) { bi = 3; bj = 3; }
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, tig = lane & 3;
-    const int wm = warp >> 2, wn = warp & 3;
-    const uint16_t *xu = X + (size_t)unit * T * kN;
-
-    auto load = [&](int stage, int k0) {
-        // A: X[k0 .. k0+32][128 bi .. +128], B: X[k0 .. k0+32][128 bj .. +128]; 16-byte chunk c of
-        // row k stored at chunk c ^ (k & 7) (conflict-free ldmatrix on 256-byte rows)
-        for (int idx = threadIdx.x; idx < kGramKT * 16 * 2; idx += kGramThreads) {
-            const int which = idx >= kGramKT * 16;
-            const int j = idx - which * kGramKT * 16;
-            const int k = j >> 4, c = j & 15;
-            const int tok = k0 + k;
-            const bool ok = tok < T;
-            const uint16_t *src = xu + (size_t)(ok ? tok : 0) * kN + (which ? bj : bi) * 128 + c * 8;
-            unsigned char *dst = (which ? sB[stage] : sA[stage]) + k * 256 + ((c ^ (k & 7)) << 4);
-            cp_async16_zfill(dst, src, ok);
-        }
-        cp_async_commit();
-    };
-
-    float acc[4][4][4];
-    #pragma unroll
-    for (int a = 0; a < 4; ++a)
-        #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b][0] = acc[a][b][1] = acc[a][b][2] = acc[a][b][3] = 0.f;
-
-    const int nk = (T + kGramKT - 1) / kGramKT;
-    load(0, 0);
-    for (int ks = 0; ks < nk; ++ks) {
-        if (ks + 1 < nk) load((ks + 1) & 1, (ks + 1) * kGramKT);
-        else cp_async_commit();
-        cp_async_wait<1>();
-        __syncthreads();
-        const uint32_t aBase = smem_u32(sA[ks & 1]), bBase = smem_u32(sB[ks & 1]);
-        #pragma unroll
-        for (int kk = 0; kk < kGramKT; kk += 16) {
-            uint32_t af[4][4], bfr[4][2];
-            #pragma unroll
-            for (int mt = 0; mt < 4; ++mt) {
-                const int mat = lane >> 3;
-                const int krow = kk + (lane & 7) + 8 * (mat >> 1);
-                const int chunk = (64 * wm + 16 * mt) / 8 + (mat & 1);
-                ldsm_x4_t(aBase + krow * 256 + ((chunk ^ (krow & 7)) << 4), af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
-            }
-            #pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                const int mat = lane >> 3;
-                const int krow = kk + (lane & 7) + 8 * (mat & 1);
-                const int chunk = (32 * wn + 16 * np) / 8 + (mat >> 1);
-                ldsm_x4_t(bBase + krow * 256 + ((chunk ^ (krow & 7)) << 4), bfr[2 * np][0], bfr[2 * np][1],
-                          bfr[2 * np + 1][0], bfr[2 * np + 1][1]);
-            }
-            #pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
-                #pragma unroll
-                for (int nt = 0; nt < 4; ++nt) mma_bf16(acc[mt][nt], af[mt], bfr[nt][0], bfr[nt][1]);
-        }
-        __syncthreads();
-    }
-    cp_async_wait<0>();
-
-    float *gu = G + (size_t)unit * kN * kN;
-    #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
-        #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-            #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int r = 128 * bi + 64 * wm + 16 * mt + g + 8 * (e >> 1);
-                const int c = 128 * bj + 32 * wn + 8 * nt + 2 * tig + (e & 1);
-                gu[(size_t)r * kN + c] = acc[mt][nt][e];
-                if (bi != bj) gu[(size_t)c * kN + r] = acc[mt][nt][e];
-            }
-}
 
 // ================================================================== eigen-solver
 
@@ -533,7 +446,198 @@ __global__ void __launch_bounds__(kProjThreads, 1) project_kernel(const uint16_t
 
 // ================================================================== host side
 
+// ------------------------------------------------------------ Gram on tcgen05
+//
+// G = X^T X per unit with the 5th-generation tensor cores.  A block owns one
+// 128-row band I of G (feature rows 128 I ..) and its columns 128 I .. 511 (the
+// upper triangle and the diagonal block), for one range of tokens:
+//   * TMA streams 64-token chunks of X restricted to features 128 I .. 511
+//     (boxes of 64 features x 64 tokens, 128-byte swizzle) through a 3-stage ring;
+//   * one thread issues tcgen05.mma kind::f16 (bf16 in, fp32 accumulate in tensor
+//     memory), M = 128 (the band's features), N <= 256 (columns), K = 16 tokens,
+//     both operands read "MN-major" straight from the swizzled X tiles (a token is a
+//     K row; the band's own 128 features are the first two boxes of the stage);
+//   * tcgen05.commit releases a stage once its MMAs have read it;
+//   * four warps move the accumulator (one tensor-memory lane per feature row) to
+//     G and mirror the off-diagonal part into the lower triangle.
+// Long token ranges are split 4:3:2:1 over the bands (equal work per block) and
+// the splits add into a zeroed G with fp32 atomics.
+constexpr int kGtTok = 64;         // tokens per stage
+constexpr int kGtStages = 3;
+constexpr int kGtThreads = 128;
+constexpr uint32_t kGtStageBytes = 64 * 1024;   // the widest band: 8 boxes of 64 features x 64 tokens
+
+struct GramTcParams {
+    CUtensorMap tm_x;      // 3D {512, T, units} bf16, box {64, 64, 1}, 128-byte swizzle
+    float *G;              // [units][512][512]
+    int T, units;
+    int splits[4];         // token splits of band I (the block count per unit is their sum)
+    int atomic;            // add into a zeroed G (any band split) instead of storing
+};
+
+struct GramTcSmem {
+    alignas(1024) unsigned char stage[kGtStages][kGtStageBytes];
+    uint64_t full[kGtStages], empty[kGtStages], done;
+    uint32_t tmem_base;
+};
+
+// tcgen05 shared-memory descriptor of an MN-major operand in 128-byte-swizzled
+// tiles: 64-element MN blocks kLbo bytes apart, 8-row K groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t saddr, uint32_t lbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((1024u >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;          // descriptor version of sm_100
+    d |= (uint64_t)2 << 61;          // 128-byte swizzle
+    return d;
+}
+
+// tcgen05 instruction descriptor: bf16 x bf16 -> fp32, both operands MN-major, M x N
+__device__ __forceinline__ uint32_t umma_idesc_bf16_mn(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        :: "r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
+          "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15]),
+          "=f"(v[16]), "=f"(v[17]), "=f"(v[18]), "=f"(v[19]), "=f"(v[20]), "=f"(v[21]), "=f"(v[22]), "=f"(v[23]),
+          "=f"(v[24]), "=f"(v[25]), "=f"(v[26]), "=f"(v[27]), "=f"(v[28]), "=f"(v[29]), "=f"(v[30]), "=f"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+__global__ void __launch_bounds__(kGtThreads, 1) gram_tc_kernel(const __grid_constant__ GramTcParams p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t base0 = smem_u32(smem_raw);
+    GramTcSmem &sm = *reinterpret_cast<GramTcSmem *>(smem_raw + ((1024u - (base0 & 1023u)) & 1023u));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ int abort_flag;
+    volatile int *abort = &abort_flag;
+
+    // block -> (unit, band I, split s)
+    const int per_unit = p.splits[0] + p.splits[1] + p.splits[2] + p.splits[3];
+    const int unit = blockIdx.x / per_unit;
+    int r = blockIdx.x % per_unit, I = 0;
+    while (r >= p.splits[I]) { r -= p.splits[I]; ++I; }
+    const int nsplit = p.splits[I], s = r;
+    const int nch = (p.T + kGtTok - 1) / kGtTok;
+    const int c0 = (int)(((long long)s * nch) / nsplit), c1 = (int)(((long long)(s + 1) * nch) / nsplit);
+    const int NI = 512 - 128 * I;          // accumulator columns (features 128 I .. 511)
+    const int nbox = NI / 64;
+    const uint32_t sbytes = (uint32_t)nbox * 8192u;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kGtStages; ++i) { mbar_init(&sm.full[i], 1); mbar_init(&sm.empty[i], 1); }
+        mbar_init(&sm.done, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+    tmem_fence_before();
+    __syncthreads();
+    tmem_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (c1 > c0) {
+        if (warp == 0 && lane == 0) {
+            // producer
+            for (int c = c0; c < c1; ++c) {
+                const int i = c - c0, slot = i % kGtStages;
+                if (i >= kGtStages && !mbar_wait(&sm.empty[slot], ((i / kGtStages) - 1) & 1u, abort)) break;
+                mbar_arrive_tx(&sm.full[slot], sbytes);
+                for (int b = 0; b < nbox; ++b)
+                    tma_3d(sm.stage[slot] + 8192 * b, &p.tm_x, 128 * I + 64 * b, kGtTok * c, unit, &sm.full[slot]);
+            }
+        } else if (warp == 1 && lane == 0) {
+            // MMA issuer
+            const uint32_t id256 = umma_idesc_bf16_mn(128, 256), id128 = umma_idesc_bf16_mn(128, 128);
+            for (int c = c0; c < c1; ++c) {
+                const int i = c - c0, slot = i % kGtStages;
+                if (!mbar_wait(&sm.full[slot], (i / kGtStages) & 1u, abort)) break;
+                tmem_fence_after();
+                const uint32_t st = smem_u32(sm.stage[slot]);
+                #pragma unroll
+                for (int k = 0; k < kGtTok / 16; ++k) {
+                    const uint64_t a = umma_desc_mn_sw128(st + 2048u * k, 8192u);
+                    for (int n0 = 0; n0 < NI; n0 += 256) {
+                        const int nn = min(256, NI - n0);
+                        const uint64_t b = umma_desc_mn_sw128(st + 8192u * (n0 / 64) + 2048u * k, 8192u);
+                        umma_bf16(tmem + (uint32_t)n0, a, b, nn == 256 ? id256 : id128, (c > c0 || k > 0) ? 1u : 0u);
+                    }
+                }
+                umma_commit(&sm.empty[slot]);
+            }
+            umma_commit(&sm.done);
+        }
+        __syncwarp();
+        // epilogue: warp w holds feature rows 32 w .. 32 w + 31 of the band (tensor-memory lanes)
+        const bool ok = mbar_wait(&sm.done, 0u, abort);
+        tmem_fence_after();
+        if (ok) {
+            const int row = 128 * I + 32 * warp + lane;
+            float *grow = p.G + ((size_t)unit * 512 + row) * 512;
+            for (int col0 = 0; col0 < NI; col0 += 32) {
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)col0, v);
+                tmem_wait_ld();
+                const int J0 = 128 * I + col0;
+                if (p.atomic) {
+                    #pragma unroll
+                    for (int j = 0; j < 32; ++j) atomicAdd(grow + J0 + j, v[j]);
+                } else {
+                    #pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4 *>(grow + J0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                }
+                if (J0 >= 128 * (I + 1)) {   // off the diagonal block: mirror (lanes write consecutive rows)
+                    float *gcol = p.G + (size_t)unit * 512 * 512 + row;
+                    #pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        if (p.atomic) atomicAdd(gcol + (size_t)(J0 + j) * 512, v[j]);
+                        else gcol[(size_t)(J0 + j) * 512] = v[j];
+                    }
+                }
+            }
+        }
+    }
+    tmem_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tmem_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// block counts of the four bands: equal work per block (4:3:2:1) once T is long
+inline void gram_tc_splits(int T, int (&sp)[4]) {
+    const int f = T >= 8192 ? (T + 8191) / 8192 : 0;
+    for (int I = 0; I < 4; ++I) sp[I] = f ? f * (4 - I) : 1;
+}
+
+inline size_t gram_tc_smem() { return sizeof(GramTcSmem) + 1024; }
+
 inline kvpack_status prepare_device() {
+    if (cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gram_tc_smem()) != cudaSuccess)
+        return KVPACK_ERR_CUDA;
     if (cudaFuncSetAttribute(eig_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EigSmem)) != cudaSuccess)
         return KVPACK_ERR_CUDA;
     if (cudaFuncSetAttribute(project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ProjSmem)) !=
@@ -542,11 +646,21 @@ inline kvpack_status prepare_device() {
     return KVPACK_OK;
 }
 
-inline kvpack_status run(int units, int T, const uint16_t *X, uint16_t *C_lo, uint16_t *C_hi, uint16_t *B,
-                         float *sigma, void *ws, int sms, cudaStream_t st) {
+inline kvpack_status run(int units, int T, const uint16_t *X, const CUtensorMap &tm_x, uint16_t *C_lo,
+                         uint16_t *C_hi, uint16_t *B, float *sigma, void *ws, int sms, cudaStream_t st) {
     (void)sms;
     Workspace w = carve(ws, units);
-    gram_kernel<<<units * 10, kGramThreads, 0, st>>>(X, T, w.G);
+    GramTcParams gp;
+    gp.tm_x = tm_x;
+    gp.G = w.G;
+    gp.T = T;
+    gp.units = units;
+    gram_tc_splits(T, gp.splits);
+    gp.atomic = gp.splits[3] > 1 ? 1 : 0;
+    if (gp.atomic && cudaMemsetAsync(w.G, 0, (size_t)units * 512 * 512 * sizeof(float), st) != cudaSuccess)
+        return KVPACK_ERR_CUDA;
+    const int per_unit = gp.splits[0] + gp.splits[1] + gp.splits[2] + gp.splits[3];
+    gram_tc_kernel<<<units * per_unit, kGtThreads, gram_tc_smem(), st>>>(gp);
     if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
     EigParams ep{w, B, sigma, units};
     eig_kernel<<<units, kEigThreads, sizeof(EigSmem), st>>>(ep);

@@ -448,7 +448,16 @@ kvpack_status kvpack_compress(const kvpack_dims *d, int32_t n_layers, const uint
     if (ws == nullptr || ws_bytes < kvpack::compress::workspace_bytes(units, d->T_vis)) return KVPACK_ERR_WORKSPACE;
     DeviceInfo *di = nullptr;
     if ((s = device_info(&di)) != KVPACK_OK) return s;
-    return kvpack::compress::run(units, d->T_vis, X, C_lo, C_hi, B, sigma, ws, di->sms,
+    PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+    if ((s = tensor_map_encoder(&enc)) != KVPACK_OK) return s;
+    CUtensorMap tm_x;
+    {
+        const cuuint64_t dims[3] = {512, (cuuint64_t)d->T_vis, (cuuint64_t)units};
+        const cuuint64_t strides[2] = {1024, (cuuint64_t)d->T_vis * 1024};
+        const cuuint32_t box[3] = {64, 64, 1};
+        if (!encode_bf16(enc, &tm_x, X, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVPACK_ERR_CUDA;
+    }
+    return kvpack::compress::run(units, d->T_vis, X, tm_x, C_lo, C_hi, B, sigma, ws, di->sms,
                                  static_cast<cudaStream_t>(stream));
 }
 
