@@ -11,9 +11,10 @@
 // per head.  K and V are never materialised.
 //
 // Four launches, each streaming its own bytes once:
-//   qproj_kernel   q~ = scale * log2(e) * B_K[:, 128 j(h) ..] q_h per unit, split into bf16 hi + lo
-//   text_kernel    the text tail (plain bf16 K/V) per (unit, KV head, chunk of tokens):
-//                  partial (max, sum, w = sum p V) per query head
+//   text_kernel    q~ = scale * log2(e) * B_K[:, 128 j(h) ..] q_h per (unit, KV head), split into
+//                  bf16 hi + lo; and the text tail (plain bf16 K/V) per (unit, KV head, chunk of
+//                  tokens): partial (max, sum, w = sum p V) per query head
+//   text_stats     the text tail's (max, sum) per head folded over its chunks, one warp per unit
 //   vis_kernel     the compressed visual tokens per (unit, split of tokens): partial
 //                  (max, sum, u = sum p C_V) per query head, then -- once every split
 //                  of the unit has published -- the attention mass of each token
@@ -34,172 +35,12 @@ constexpr int kMaxHeads = 32;
 constexpr int kTxtPart = 130;   // per (unit, text chunk, head): max, sum, w[128]
 constexpr int kVisPart = 66;    // per (unit, visual split, head): max, sum, u[64]
 
-// ======================================================================== qproj
+// =================================================================== query block
 
 // Per unit, the query block the visual kernel copies in one piece:
 //   [2][Hg][64] bf16  q~ hi then lo (128-byte rows, 16-byte chunk c stored at c ^ (h & 7))
 //   [Hg][2]     f32   the text tail's (max, sum) per head, combined over its chunks
 __host__ __device__ constexpr size_t qblock_bytes(int Hg) { return (size_t)Hg * (2 * 128 + 8); }
-
-struct QProjParams {
-    const uint16_t *q;     // [(layer, batch)][n_q][128]
-    const uint16_t *BK;    // [units][64][512]
-    unsigned char *qt;     // [units][qblock_bytes(Hg)]
-    const float *tpart;    // [units][Sc][Hg][kTxtPart] from text_kernel, or null (Sc == 0)
-    int Hg, per_kv, n_q, groups, Sc;
-    float scale2;
-};
-
-// The text tail's (max, sum) per head of one unit, folded over its chunks: warp
-// per head, lanes over the chunks.
-__device__ __forceinline__ void text_stats(const QProjParams &p, int unit, int warp, int lane) {
-    float *ts = reinterpret_cast<float *>(p.qt + (size_t)unit * qblock_bytes(p.Hg) + (size_t)p.Hg * 256);
-    for (int h = warp; h < p.Hg; h += 8) {
-        const float *tp = p.tpart + (size_t)unit * p.Sc * p.Hg * kTxtPart + (size_t)h * kTxtPart;
-        float mx = -INFINITY, mc[2], lc[2];
-        #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const int c = lane + 32 * k;
-            mc[k] = c < p.Sc ? tp[(size_t)c * p.Hg * kTxtPart] : -INFINITY;
-            lc[k] = c < p.Sc ? tp[(size_t)c * p.Hg * kTxtPart + 1] : 0.f;
-            mx = fmaxf(mx, mc[k]);
-        }
-        for (int c = lane + 64; c < p.Sc; c += 32) mx = fmaxf(mx, tp[(size_t)c * p.Hg * kTxtPart]);
-        #pragma unroll
-        for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
-        float sum = 0.f;
-        #pragma unroll
-        for (int k = 0; k < 2; ++k)
-            if (mc[k] != -INFINITY) sum += lc[k] * ex2(mc[k] - mx);
-        for (int c = lane + 64; c < p.Sc; c += 32) {
-            const float m2 = tp[(size_t)c * p.Hg * kTxtPart];
-            if (m2 != -INFINITY) sum += tp[(size_t)c * p.Hg * kTxtPart + 1] * ex2(m2 - mx);
-        }
-        #pragma unroll
-        for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
-        if (lane == 0) {
-            ts[2 * h] = mx;
-            ts[2 * h + 1] = sum;
-        }
-    }
-}
-
-// One block per unit (several query heads per KV head); thread (i, j) =
-// (tid / 4, tid % 4) owns rank row i of B_K restricted to KV head j (256
-// contiguous bytes) and forms q~_h[i] for the KV head's query heads with plain
-// fp32 FMAs.  Runs after text_kernel.
-__global__ void __launch_bounds__(256) qproj_cols_kernel(const QProjParams p) {
-    __shared__ float qs[kMaxHeads][132];   // q rows in fp32; the pad spreads the 4 KV heads over banks
-    const int unit = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int lb = unit / p.groups, G = unit % p.groups;
-    const int i = tid >> 2, j = tid & 3;
-
-    // the thread's 256 bytes of B_K first, so that they are in flight before anything waits
-    uint4 raw[16];
-    const uint4 *src = reinterpret_cast<const uint4 *>(p.BK + ((size_t)unit * 64 + i) * 512 + 128 * j);
-    #pragma unroll
-    for (int k = 0; k < 16; ++k) raw[k] = __ldg(src + k);
-
-    const uint32_t *qsrc = reinterpret_cast<const uint32_t *>(p.q + ((size_t)lb * p.n_q + (size_t)G * p.Hg) * 128);
-    for (int x = tid; x < p.Hg * 64; x += 256) {
-        const uint32_t v = __ldg(qsrc + x);
-        qs[x >> 6][2 * (x & 63)] = __uint_as_float(v << 16);
-        qs[x >> 6][2 * (x & 63) + 1] = __uint_as_float(v & 0xffff0000u);
-    }
-
-    text_stats(p, unit, warp, lane);
-    __syncthreads();
-
-    float acc[8];
-    #pragma unroll
-    for (int hh = 0; hh < 8; ++hh) acc[hh] = 0.f;
-    const int h0 = j * p.per_kv;
-    #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
-        #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float b = (e & 1) ? __uint_as_float(w4[e >> 1] & 0xffff0000u) : __uint_as_float(w4[e >> 1] << 16);
-            #pragma unroll
-            for (int hh = 0; hh < 8; ++hh)
-                if (hh < p.per_kv) acc[hh] = fmaf(b, qs[h0 + hh][8 * k + e], acc[hh]);
-        }
-    }
-    uint16_t *qt = reinterpret_cast<uint16_t *>(p.qt + (size_t)unit * qblock_bytes(p.Hg));
-    #pragma unroll
-    for (int hh = 0; hh < 8; ++hh) {
-        if (hh < p.per_kv) {
-            const int h = h0 + hh;
-            const float v = acc[hh] * p.scale2;
-            const uint16_t hi = float_to_bf16_bits(v);
-            const uint16_t lo = float_to_bf16_bits(v - bf16_bits_to_float(hi));
-            const int off = h * 64 + ((((i >> 3) ^ (h & 7)) & 7) << 3) + (i & 7);
-            qt[off] = hi;
-            qt[p.Hg * 64 + off] = lo;
-        }
-    }
-}
-
-// One block per unit (one or two query heads per KV head): warp w takes rank
-// rows 8w..8w+7 of B_K; lane L holds columns 8L..8L+7 and 256+8L..256+8L+7 of a
-// row (coalesced), so a 16-lane half covers one KV head's 128 columns and a
-// shuffle tree finishes each dot product.  Runs after text_kernel.
-__global__ void __launch_bounds__(256) qproj_rows_kernel(const QProjParams p) {
-    __shared__ float qs[kMaxHeads][128];
-    const int unit = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int lb = unit / p.groups, G = unit % p.groups;
-    uint4 raw[8][2];
-    const uint16_t *bk = p.BK + (size_t)unit * 64 * 512;
-    #pragma unroll
-    for (int r = 0; r < 8; ++r)
-        #pragma unroll
-        for (int sg = 0; sg < 2; ++sg)
-            raw[r][sg] = __ldcs(reinterpret_cast<const uint4 *>(bk + (size_t)(8 * warp + r) * 512 + 256 * sg + 8 * lane));
-    const uint32_t *qsrc = reinterpret_cast<const uint32_t *>(p.q + ((size_t)lb * p.n_q + (size_t)G * p.Hg) * 128);
-    for (int x = threadIdx.x; x < p.Hg * 64; x += 256) {
-        const uint32_t v = __ldg(qsrc + x);
-        qs[x >> 6][2 * (x & 63)] = __uint_as_float(v << 16);
-        qs[x >> 6][2 * (x & 63) + 1] = __uint_as_float(v & 0xffff0000u);
-    }
-    text_stats(p, unit, warp, lane);
-    __syncthreads();
-    uint16_t *qt = reinterpret_cast<uint16_t *>(p.qt + (size_t)unit * qblock_bytes(p.Hg));
-    #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int i = 8 * warp + r;
-        #pragma unroll
-        for (int sg = 0; sg < 2; ++sg) {
-            const int j = 2 * sg + (lane >> 4), dd = 8 * (lane & 15);
-            const uint32_t w4[4] = {raw[r][sg].x, raw[r][sg].y, raw[r][sg].z, raw[r][sg].w};
-            float b[8];
-            #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                b[2 * e] = __uint_as_float(w4[e] << 16);
-                b[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
-            }
-            #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                if (hh < p.per_kv) {
-                    const int h = j * p.per_kv + hh;
-                    const float *qr = &qs[h][dd];
-                    float acc = 0.f;
-                    #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc = fmaf(b[e], qr[e], acc);
-                    #pragma unroll
-                    for (int d = 1; d < 16; d <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
-                    if ((lane & 15) == 0) {
-                        const float v = acc * p.scale2;
-                        const uint16_t hi = float_to_bf16_bits(v);
-                        const uint16_t lo = float_to_bf16_bits(v - bf16_bits_to_float(hi));
-                        const int off = h * 64 + ((((i >> 3) ^ (h & 7)) & 7) << 3) + (i & 7);
-                        qt[off] = hi;
-                        qt[p.Hg * 64 + off] = lo;
-                    }
-                }
-            }
-        }
-    }
-}
 
 // ========================================================================= text
 
@@ -208,15 +49,17 @@ namespace text {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSlots = 3;
-constexpr int kSlotBytes = 8192;   // 16 tokens x (K 256 B + V 256 B) of one KV head
+constexpr int kSlotBytes = 8192;   // 16 text tokens x (K 256 B + V 256 B) of one KV head, or 64 B_K rows x 128 B
 constexpr int kTile = 16;
 
 struct Params {
-    CUtensorMap tm_k, tm_v;    // 4D {128, 4, L, units}, box {64, 1, 16, 1}, 128-byte swizzle
+    CUtensorMap tm_k, tm_v;    // text: 4D {128, 4, L, units}, box {64, 1, 16, 1}, 128-byte swizzle
+    CUtensorMap tm_bk;         // B_K: 3D {512, 64, units}, box {64, 64, 1}, 128-byte swizzle
     const uint16_t *q;
     float *part;               // [units][Sc][Hg][kTxtPart]
+    unsigned char *qt;         // [units][qblock_bytes(Hg)]: q~ written here
     unsigned int *counter;     // work counter, zero at launch
-    int n_units, L, Hg, per_kv, n_q, groups, Sc, ct, n_items;
+    int n_units, L, Hg, per_kv, n_q, groups, Sc, ct, n_qitems, n_items;
     float scale2;
 };
 
@@ -229,12 +72,15 @@ struct Smem {
 
 constexpr size_t smem_bytes() { return sizeof(Smem) + 1024; }
 
-// Every warp streams whole work items -- (unit, KV head j, chunk of ct text
-// tokens) -- through its own 3-slot ring, fetched from a global counter.  Per
-// 16-token tile: S = K q^T with tokens on M and the KV head's query heads on N
-// (mma.sync m16n8k16), an online softmax over the columns, and w^T += V^T P
-// (the transposed P comes from movmatrix).  At the end of an item the warp
-// writes the partial (max, sum, w) of each of its query heads.
+// Every warp streams whole work items through its own 3-slot ring, fetched from
+// a global counter.  Items 0 .. n_qitems-1 project the query to rank space for
+// (unit, KV head j): two stages of B_K (64 rank rows x 64 columns each), q~^T =
+// B_K[:, 128 j ..] q^T on mma.sync (ranks on M, the KV head's query heads on N),
+// written as the bf16 hi + lo pair of the unit's query block.  The others are
+// text items -- (unit, KV head j, chunk of ct text tokens): per 16-token tile,
+// S = K q^T with tokens on M and the query heads on N, an online softmax down
+// the columns, and w^T += V^T P (the transposed P from movmatrix); at the end of
+// an item the partial (max, sum, w) of each query head.
 __global__ void __launch_bounds__(kThreads, 1) text_kernel(const __grid_constant__ Params p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t base = smem_u32(smem_raw);
@@ -255,7 +101,11 @@ __global__ void __launch_bounds__(kThreads, 1) text_kernel(const __grid_constant
         if (lane == 0) v = (int)atomicAdd(p.counter, 1u);
         return __shfl_sync(0xffffffffu, v, 0);
     };
-    auto n_tok = [&](int it) { const int c = it % p.Sc; return min(p.ct, p.L - c * p.ct); };
+    // (unit, KV head) of an item
+    auto unit_of = [&](int it) { return it < p.n_qitems ? it >> 2 : (it - p.n_qitems) / (4 * p.Sc); };
+    auto kvh_of = [&](int it) { return it < p.n_qitems ? it & 3 : ((it - p.n_qitems) / p.Sc) & 3; };
+    auto n_tok = [&](int it) { const int c = (it - p.n_qitems) % p.Sc; return min(p.ct, p.L - c * p.ct); };
+    auto n_tiles = [&](int it) { return it < p.n_qitems ? 2 : (n_tok(it) + kTile - 1) / kTile; };
 
     // ---- issue side
     int i_item = -1, i_tile = 0, i_ntiles = 0, q_push = 0;
@@ -266,23 +116,27 @@ __global__ void __launch_bounds__(kThreads, 1) text_kernel(const __grid_constant
         if (i_tile == i_ntiles) {
             const int it = fetch();
             if (it >= p.n_items) { i_done = true; return; }
-            i_item = it; i_tile = 0; i_ntiles = (n_tok(it) + kTile - 1) / kTile;
+            i_item = it; i_tile = 0; i_ntiles = n_tiles(it);
             if (lane == 0) sm.itemq[warp][q_push & 7] = it;
             ++q_push;
         }
         const int slot = i_seq % kSlots;
-        const int unit = i_item / (4 * p.Sc), j = (i_item / p.Sc) % 4, c = i_item % p.Sc;
-        const int tok = c * p.ct + i_tile * kTile;
+        const int unit = unit_of(i_item), j = kvh_of(i_item);
         __syncwarp();
         if (lane == 0) {
             unsigned char *dst = sm.ring[warp][slot];
             uint64_t *bar = &sm.full[warp][slot];
             fence_proxy_async();
             mbar_arrive_tx(bar, kSlotBytes);
-            tma_4d(dst, &p.tm_k, 0, j, tok, unit, bar);
-            tma_4d(dst + 2048, &p.tm_k, 64, j, tok, unit, bar);
-            tma_4d(dst + 4096, &p.tm_v, 0, j, tok, unit, bar);
-            tma_4d(dst + 6144, &p.tm_v, 64, j, tok, unit, bar);
+            if (i_item < p.n_qitems) {
+                tma_3d(dst, &p.tm_bk, 128 * j + 64 * i_tile, 0, unit, bar);
+            } else {
+                const int tok = ((i_item - p.n_qitems) % p.Sc) * p.ct + i_tile * kTile;
+                tma_4d(dst, &p.tm_k, 0, j, tok, unit, bar);
+                tma_4d(dst + 2048, &p.tm_k, 64, j, tok, unit, bar);
+                tma_4d(dst + 4096, &p.tm_v, 0, j, tok, unit, bar);
+                tma_4d(dst + 6144, &p.tm_v, 64, j, tok, unit, bar);
+            }
         }
         ++i_tile;
         ++i_seq;
@@ -290,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1) text_kernel(const __grid_constant
 
     // query rows of (unit, j) as B fragments: b0 = q[g][16 kb + 2 tig ..], b1 = q[g][16 kb + 8 + 2 tig ..]
     auto load_q = [&](int it, uint32_t (&qf)[8][2]) {
-        const int unit = it / (4 * p.Sc), j = (it / p.Sc) % 4;
+        const int unit = unit_of(it), j = kvh_of(it);
         const int lb = unit / p.groups, G = unit % p.groups;
         const bool ok = g < p.per_kv;
         const uint32_t *row = reinterpret_cast<const uint32_t *>(
@@ -314,8 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1) text_kernel(const __grid_constant
             c_item = sm.itemq[warp][q_pop & 7];
             ++q_pop;
             c_tile = 0;
-            c_n = n_tok(c_item);
-            c_ntiles = (c_n + kTile - 1) / kTile;
+            c_ntiles = n_tiles(c_item);
+            c_n = c_item < p.n_qitems ? 0 : n_tok(c_item);
             if (qn_item == c_item) {
                 #pragma unroll
                 for (int kb = 0; kb < 8; ++kb) { qf[kb][0] = qn[kb][0]; qf[kb][1] = qn[kb][1]; }
@@ -335,8 +189,54 @@ __global__ void __launch_bounds__(kThreads, 1) text_kernel(const __grid_constant
         const int slot = c_seq % kSlots;
         if (!mbar_wait(&sm.full[warp][slot], (c_seq / kSlots) & 1u, abort)) break;
         const uint32_t sb = smem_u32(sm.ring[warp][slot]);
-        const int n = min(kTile, c_n - c_tile * kTile);
 
+        if (c_item < p.n_qitems) {
+            // ---------------- q~ projection: this stage holds B_K[64 ranks][64 columns] of KV head j,
+            // k-steps 4 c_tile .. 4 c_tile + 3 of the 128-column product, accumulated in wt[0..3]
+            auto proj = [&](auto half) {
+                constexpr int H = decltype(half)::value;
+                #pragma unroll
+                for (int kq = 0; kq < 4; ++kq) {
+                    #pragma unroll
+                    for (int mt = 0; mt < 4; ++mt) {
+                        uint32_t a[4];
+                        const int row = 16 * mt + (lane & 7) + (((lane >> 3) & 1) << 3);
+                        const int ch = 2 * kq + (lane >> 4);
+                        ldsm_x4(sb + row * 128 + ((ch ^ (row & 7)) << 4), a[0], a[1], a[2], a[3]);
+                        mma_bf16(wt[mt], a, qf[4 * H + kq][0], qf[4 * H + kq][1]);
+                    }
+                }
+            };
+            if (c_tile == 0) proj(std::integral_constant<int, 0>());
+            else proj(std::integral_constant<int, 1>());
+            ++c_tile;
+            ++c_seq;
+            if (c_tile == c_ntiles) {
+                // wt[mt][e]: rank 16 mt + g (+8 for e >= 2), head 2 tig + (e & 1) of KV head j
+                const int unit = unit_of(c_item), j = kvh_of(c_item);
+                uint16_t *qt = reinterpret_cast<uint16_t *>(p.qt + (size_t)unit * qblock_bytes(p.Hg));
+                #pragma unroll
+                for (int mt = 0; mt < 4; ++mt)
+                    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int hh = 2 * tig + (e & 1);
+                        if (hh < p.per_kv) {
+                            const int h = j * p.per_kv + hh, i = 16 * mt + g + 8 * (e >> 1);
+                            const float v = wt[mt][e] * p.scale2;
+                            const uint16_t hi = float_to_bf16_bits(v);
+                            const uint16_t lo = float_to_bf16_bits(v - bf16_bits_to_float(hi));
+                            const int off = h * 64 + ((((i >> 3) ^ (h & 7)) & 7) << 3) + (i & 7);
+                            qt[off] = hi;
+                            qt[p.Hg * 64 + off] = lo;
+                        }
+                    }
+            }
+            __syncwarp();
+            if (i_seq - c_seq < (uint32_t)kSlots) issue();
+            continue;
+        }
+
+        const int n = min(kTile, c_n - c_tile * kTile);
         // S[tok][h] = K[tok][:] . q_h
         float s[4] = {0.f, 0.f, 0.f, 0.f};
         #pragma unroll
@@ -390,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) text_kernel(const __grid_constant
             for (int e = 0; e < 2; ++e)
                 #pragma unroll
                 for (int d = 4; d < 32; d <<= 1) l[e] += __shfl_xor_sync(0xffffffffu, l[e], d);
-            const int unit = c_item / (4 * p.Sc), j = (c_item / p.Sc) % 4, c = c_item % p.Sc;
+            const int unit = unit_of(c_item), j = kvh_of(c_item), c = (c_item - p.n_qitems) % p.Sc;
             float *dst = p.part + (((size_t)unit * p.Sc + c) * p.Hg + j * p.per_kv) * kTxtPart;
             #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -417,6 +317,25 @@ __global__ void __launch_bounds__(kThreads, 1) text_kernel(const __grid_constant
         while (!mbar_try_wait(&sm.full[warp][slot], par) && clock64() - t0 < kWaitCycles) {}
         ++c_seq;
     }
+}
+
+// The text tail's (max, sum) per head of every unit, folded over its chunks
+// into the unit's query block (one warp per unit, a lane per head).
+__global__ void __launch_bounds__(256) text_stats_kernel(const float *__restrict__ part, unsigned char *qt, int units,
+                                                         int Hg, int Sc) {
+    const int unit = blockIdx.x * 8 + (threadIdx.x >> 5), h = threadIdx.x & 31;
+    if (unit >= units || h >= Hg) return;
+    const float *tp = part + (size_t)unit * Sc * Hg * kTxtPart + (size_t)h * kTxtPart;
+    float mx = -INFINITY;
+    for (int c = 0; c < Sc; ++c) mx = fmaxf(mx, tp[(size_t)c * Hg * kTxtPart]);
+    float sum = 0.f;
+    for (int c = 0; c < Sc; ++c) {
+        const float mc = tp[(size_t)c * Hg * kTxtPart];
+        if (mc != -INFINITY) sum += tp[(size_t)c * Hg * kTxtPart + 1] * ex2(mc - mx);
+    }
+    float *ts = reinterpret_cast<float *>(qt + (size_t)unit * qblock_bytes(Hg) + (size_t)Hg * 256);
+    ts[2 * h] = mx;
+    ts[2 * h + 1] = sum;
 }
 
 }  // namespace text
@@ -453,7 +372,7 @@ struct Cfg {
 struct Params {
     CUtensorMap tm_ck, tm_cv;   // C_lo planes: 3D {16, T, units}, box {16, 32, 1}, 32-byte swizzle
     const uint16_t *CK_lo, *CK_hi, *CV_lo, *CV_hi;
-    const unsigned char *qt;    // [units][qblock_bytes(Hg)] from qproj_kernel
+    const unsigned char *qt;    // [units][qblock_bytes(Hg)] from text_kernel and text_stats_kernel
     const uint32_t *mask;       // [units][nwords]
     float *mass;                // [units][T] or null
     float *part;                // [units][S][Hg][kVisPart]
@@ -1216,43 +1135,59 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
             mass_warp(K, 0);
             continue;
         }
-        // several splits: the last one to publish fixes the unit's (max, 1/sum), warp per head
+        // several splits: the last one to publish fixes the unit's (max, 1/sum).  Only warp 0
+        // takes the arrival count (lanes over splits); the other warps go on to the mass.
         __syncthreads();
-        if (tid == 0) {
-            __threadfence();
-            unsigned int old;
-            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&p.arrive[unit]) : "memory");
-            sm.last = (old == (unsigned int)(p.S - 1));
-        }
-        __syncthreads();
-        if (sm.last) {
-            for (int h = warp; h < p.Hg; h += kWarps) {
-                const float *vp = p.part + (size_t)unit * p.S * p.Hg * kVisPart + (size_t)h * kVisPart;
-                float mx = sm.tcur[h][0], ml[4], ll[4];
-                #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int sp = lane + 32 * k;
-                    ml[k] = sp < p.S ? __ldcg(vp + (size_t)sp * p.Hg * kVisPart) : kRefInit;
-                    ll[k] = sp < p.S ? __ldcg(vp + (size_t)sp * p.Hg * kVisPart + 1) : 0.f;
-                    mx = fmaxf(mx, ml[k]);
-                }
-                for (int sp = lane + 128; sp < p.S; sp += 32) mx = fmaxf(mx, __ldcg(vp + (size_t)sp * p.Hg * kVisPart));
-                #pragma unroll
-                for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
-                float sum = 0.f;
-                #pragma unroll
-                for (int k = 0; k < 4; ++k) sum += ll[k] * ex2(ml[k] - mx);
-                for (int sp = lane + 128; sp < p.S; sp += 32)
-                    sum += __ldcg(vp + (size_t)sp * p.Hg * kVisPart + 1) * ex2(__ldcg(vp + (size_t)sp * p.Hg * kVisPart) - mx);
-                #pragma unroll
-                for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
-                if (lane == 0) {
-                    if (sm.tcur[h][0] != -INFINITY) sum += sm.tcur[h][1] * ex2(sm.tcur[h][0] - mx);
-                    float *us = p.ustat + ((size_t)unit * p.Hg + h) * 2;
-                    const float inv = 1.f / sum;
-                    asm volatile("st.relaxed.gpu.global.v2.f32 [%0], {%1, %2};" :: "l"(us), "f"(mx), "f"(inv) : "memory");
+        if (warp == 0) {
+            unsigned int old = 0;
+            if (lane == 0) {
+                __threadfence();
+                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&p.arrive[unit]) : "memory");
+            }
+            old = __shfl_sync(0xffffffffu, old, 0);
+            if (old == (unsigned int)(p.S - 1)) {
+                // lanes over the splits, four heads at a time with all their loads in flight
+                const float *vu = p.part + (size_t)unit * p.S * p.Hg * kVisPart;
+                for (int h0 = 0; h0 < p.Hg; h0 += 4) {
+                    float ml[4][4], ll[4][4];
+                    #pragma unroll
+                    for (int hh = 0; hh < 4; ++hh)
+                        #pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int sp = lane + 32 * k;
+                            const float *r2 = vu + ((size_t)sp * p.Hg + h0 + hh) * kVisPart;
+                            ml[hh][k] = sp < p.S ? __ldcg(r2) : kRefInit;
+                            ll[hh][k] = sp < p.S ? __ldcg(r2 + 1) : 0.f;
+                        }
+                    #pragma unroll
+                    for (int hh = 0; hh < 4; ++hh) {
+                        const int h = h0 + hh;
+                        float mx = sm.tcur[h][0];
+                        #pragma unroll
+                        for (int k = 0; k < 4; ++k) mx = fmaxf(mx, ml[hh][k]);
+                        for (int sp = lane + 128; sp < p.S; sp += 32)
+                            mx = fmaxf(mx, __ldcg(vu + ((size_t)sp * p.Hg + h) * kVisPart));
+                        #pragma unroll
+                        for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+                        float sum = 0.f;
+                        #pragma unroll
+                        for (int k = 0; k < 4; ++k) sum += ll[hh][k] * ex2(ml[hh][k] - mx);
+                        for (int sp = lane + 128; sp < p.S; sp += 32) {
+                            const float *r2 = vu + ((size_t)sp * p.Hg + h) * kVisPart;
+                            sum += __ldcg(r2 + 1) * ex2(__ldcg(r2) - mx);
+                        }
+                        #pragma unroll
+                        for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
+                        if (lane == 0) {
+                            if (sm.tcur[h][0] != -INFINITY) sum += sm.tcur[h][1] * ex2(sm.tcur[h][0] - mx);
+                            float *us = p.ustat + ((size_t)unit * p.Hg + h) * 2;
+                            const float inv = 1.f / sum;
+                            asm volatile("st.relaxed.gpu.global.v2.f32 [%0], {%1, %2};" :: "l"(us), "f"(mx), "f"(inv) : "memory");
+                        }
+                    }
                 }
             }
+            __syncwarp();
         }
         if (K >= 1) mass_warp(K - 1, 2);
     }
@@ -1284,6 +1219,7 @@ struct FinishParams {
     const float *vpart;       // [units][S][Hg][kVisPart]
     const float *tpart;       // [units][Sc][Hg][kTxtPart] or null
     uint16_t *out;            // [(layer, batch)][n_q][128]
+    float *ustat;             // [units][Hg][2]: the unit-wide (max, 1/sum) per head, or null
     int Hg, per_kv, n_q, groups, S, Sc;
 };
 
@@ -1330,6 +1266,8 @@ __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
         #pragma unroll
         for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
         const float inv = 1.f / sum;
+        if (lane == 0 && p.ustat != nullptr)
+            *reinterpret_cast<float2 *>(p.ustat + ((size_t)unit * p.Hg + h) * 2) = make_float2(mx, inv);
         __syncwarp();
         for (int s = lane; s < p.S; s += 32) wv[s * kMaxHeads + h] *= inv;
         for (int c = lane; c < p.Sc; c += 32) wt[c * kMaxHeads + h] *= inv;

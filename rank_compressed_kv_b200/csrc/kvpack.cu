@@ -11,6 +11,7 @@
 #include "kvpack.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "mass.cuh"
 #include "select.cuh"
 #include "compress.cuh"
 
@@ -96,6 +97,7 @@ DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
 struct DeviceInfo {
     bool ready = false;
     int sms = 0;
+    int mass_blocks[4] = {0, 0, 0, 0};   // resident blocks per SM of mass_kernel<1..4>
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -122,6 +124,18 @@ kvpack_status device_info(DeviceInfo **out) {
             cudaFuncSetAttribute(dc::vis::vis_kernel<2>, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
             cudaFuncSetAttribute(dc::text::text_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
             return KVPACK_ERR_CUDA;
+        {
+            const void *mk[4] = {(const void *)dc::mass::mass_kernel<1>, (const void *)dc::mass::mass_kernel<2>,
+                                 (const void *)dc::mass::mass_kernel<3>, (const void *)dc::mass::mass_kernel<4>};
+            for (int i = 0; i < 4; ++i) {
+                if (cudaFuncSetAttribute(mk[i], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dc::mass::smem_bytes()) != cudaSuccess ||
+                    cudaFuncSetAttribute(mk[i], cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
+                    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.mass_blocks[i], mk[i], dc::mass::kThreads,
+                                                                  dc::mass::smem_bytes()) != cudaSuccess ||
+                    di.mass_blocks[i] < 1)
+                    return KVPACK_ERR_CUDA;
+            }
+        }
         int b1 = 0, b2 = 0, bt = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b1, dc::vis::vis_kernel<1>, dc::vis::kThreads,
                                                           dc::vis::smem_bytes<1>()) != cudaSuccess ||
@@ -285,32 +299,37 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     // that several splits wait for start as NaN (all-ones bytes)
     if (cudaMemsetAsync(arrive, 0, pl.off_counter + sizeof(unsigned int) - pl.off_arrive, st) != cudaSuccess)
         return KVPACK_ERR_CUDA;
-    if (pl.S > 1 && mass != nullptr &&
-        cudaMemsetAsync(ustat, 0xff, (size_t)pl.units * Hg * 2 * sizeof(float), st) != cudaSuccess)
-        return KVPACK_ERR_CUDA;
 
-    // 1. text tail partials
-    if (L_text > 0) {
+    // 1. q~ per (unit, KV head) and the text tail partials, one persistent launch
+    {
         dc::text::Params tp;
         std::memset(&tp, 0, sizeof(tp));
-        const cuuint64_t dims[4] = {128, 4, (cuuint64_t)L_text, (cuuint64_t)pl.units};
-        const cuuint64_t strides[3] = {256, 1024, (cuuint64_t)d->L_text_cap * 1024};
-        const cuuint32_t box[4] = {64, 1, 16, 1};
-        if (!encode_bf16(enc, &tp.tm_k, K_text, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !encode_bf16(enc, &tp.tm_v, V_text, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return KVPACK_ERR_CUDA;
-        tp.q = q; tp.part = tpart; tp.counter = counter;
+        if (L_text > 0) {
+            const cuuint64_t dims[4] = {128, 4, (cuuint64_t)L_text, (cuuint64_t)pl.units};
+            const cuuint64_t strides[3] = {256, 1024, (cuuint64_t)d->L_text_cap * 1024};
+            const cuuint32_t box[4] = {64, 1, 16, 1};
+            if (!encode_bf16(enc, &tp.tm_k, K_text, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                !encode_bf16(enc, &tp.tm_v, V_text, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+                return KVPACK_ERR_CUDA;
+        }
+        {
+            const cuuint64_t dims[3] = {512, 64, (cuuint64_t)pl.units};
+            const cuuint64_t strides[2] = {1024, 64 * 1024};
+            const cuuint32_t box[3] = {64, 64, 1};
+            if (!encode_bf16(enc, &tp.tm_bk, BK, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+                return KVPACK_ERR_CUDA;
+        }
+        tp.q = q; tp.part = tpart; tp.qt = qt; tp.counter = counter;
         tp.n_units = pl.units; tp.L = L_text; tp.Hg = Hg; tp.per_kv = per_kv; tp.n_q = d->n_q_heads;
-        tp.groups = groups; tp.Sc = Sc; tp.ct = kTextChunk; tp.n_items = pl.units * 4 * Sc; tp.scale2 = scale2;
+        tp.groups = groups; tp.Sc = Sc; tp.ct = kTextChunk; tp.n_qitems = pl.units * 4;
+        tp.n_items = tp.n_qitems + pl.units * 4 * Sc; tp.scale2 = scale2;
         const int grid = tp.n_items < di->sms ? tp.n_items : di->sms;
         dc::text::text_kernel<<<grid, dc::text::kThreads, dc::text::smem_bytes(), st>>>(tp);
         if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
     }
 
-    // 2. q~ per unit, with the text tail's (max, sum) per head
-    dc::QProjParams qp{q, BK, qt, Sc > 0 ? tpart : nullptr, Hg, per_kv, d->n_q_heads, groups, Sc, scale2};
-    if (per_kv <= 2) dc::qproj_rows_kernel<<<pl.units, 256, 0, st>>>(qp);
-    else dc::qproj_cols_kernel<<<pl.units, 256, 0, st>>>(qp);
+    // 2. the text tail's (max, sum) per head of each unit, into its query block
+    dc::text::text_stats_kernel<<<(pl.units + 7) / 8, 256, 0, st>>>(tpart, qt, pl.units, Hg, Sc);
     if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
 
     // 3. visual partials and the attention mass
@@ -324,28 +343,55 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
             !encode_bf16(enc, &vp.tm_cv, CV_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return KVPACK_ERR_CUDA;
         vp.CK_lo = CK_lo; vp.CK_hi = CK_hi; vp.CV_lo = CV_lo; vp.CV_hi = CV_hi;
-        vp.qt = qt; vp.mask = mask; vp.mass = mass; vp.part = vpart; vp.ustat = ustat; vp.arrive = arrive;
+        vp.qt = qt; vp.mask = mask; vp.mass = nullptr; vp.part = vpart; vp.ustat = ustat; vp.arrive = arrive;
         vp.n_units = pl.units; vp.T = T; vp.Hg = Hg; vp.S = pl.S; vp.tps = pl.tps; vp.nwords = (T + 31) / 32;
         vp.n_items = pl.units * pl.S;
         const int resident = di->sms * (pl.nmb == 1 ? dc::vis::Cfg<1>::kBlocks : dc::vis::Cfg<2>::kBlocks);
-        const int grid = vp.n_items < resident ? vp.n_items : resident;
+        int grid = vp.n_items < resident ? vp.n_items : resident;
         if (pl.S > grid) return KVPACK_ERR_UNSUPPORTED;   // every split of a unit must be co-resident
+        // a whole number of units per round (items b, b + grid, ...): no unit's splits straddle
+        // two rounds, so they finish together -- unless that idles more than a fifth of the blocks
+        if (pl.S > 1 && grid == resident && (resident / pl.S) * pl.S * 5 >= resident * 4) grid = (resident / pl.S) * pl.S;
         void *args[] = {&vp};
         const void *fn = (pl.nmb == 1) ? (const void *)dc::vis::vis_kernel<1> : (const void *)dc::vis::vis_kernel<2>;
         const size_t smem = (pl.nmb == 1) ? dc::vis::smem_bytes<1>() : dc::vis::smem_bytes<2>();
         // Splits of a unit wait (boundedly) for one another: the grid never exceeds what is
         // resident at once.  The 32-row variant asks for that guarantee with a cooperative launch.
         cudaError_t e;
-        if (pl.nmb == 2 && pl.S > 1 && mass != nullptr)
-            e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(dc::vis::kThreads), args, smem, st);
-        else
-            e = cudaLaunchKernel(fn, dim3(grid), dim3(dc::vis::kThreads), args, smem, st);
+        e = cudaLaunchKernel(fn, dim3(grid), dim3(dc::vis::kThreads), args, smem, st);
         if (e != cudaSuccess) return KVPACK_ERR_CUDA;
     }
 
     // 4. combine and project through B_V
-    dc::FinishParams fp{BV, vpart, Sc > 0 ? tpart : nullptr, out, Hg, per_kv, d->n_q_heads, groups, pl.S, Sc};
+    dc::FinishParams fp{BV, vpart, Sc > 0 ? tpart : nullptr, out, mass != nullptr ? ustat : nullptr,
+                        Hg, per_kv, d->n_q_heads, groups, pl.S, Sc};
     dc::finish_kernel<<<pl.units, 256, dc::finish_smem_bytes(pl.S, Sc), st>>>(fp);
+    if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
+    if (mass == nullptr) return KVPACK_OK;
+
+    // 5. the attention mass of every visual token under the unit's final (max, sum)
+    {
+        dc::mass::Params mp;
+        std::memset(&mp, 0, sizeof(mp));
+        const cuuint64_t dims[3] = {16, (cuuint64_t)T, (cuuint64_t)pl.units};
+        const cuuint64_t strides[2] = {32, (cuuint64_t)T * 32};
+        const cuuint32_t box[3] = {16, 32, 1};
+        if (!encode_bf16(enc, &mp.tm_ck, CK_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B)) return KVPACK_ERR_CUDA;
+        mp.CK_lo = CK_lo; mp.CK_hi = CK_hi; mp.qt = qt; mp.ustat = ustat; mp.mask = mask; mp.mass = mass;
+        mp.T = T; mp.Hg = Hg; mp.nwords = (T + 31) / 32; mp.cpu = (T + dc::mass::kChunk - 1) / dc::mass::kChunk;
+        mp.n_chunks = pl.units * mp.cpu;
+        const int nt = (Hg + 7) / 8;
+        const int resident = di->sms * di->mass_blocks[nt - 1];
+        const int need = (mp.n_chunks + dc::mass::kWarps - 1) / dc::mass::kWarps;
+        const int grid = need < resident ? need : resident;
+        const size_t smem = dc::mass::smem_bytes();
+        switch (nt) {
+            case 1: dc::mass::mass_kernel<1><<<grid, dc::mass::kThreads, smem, st>>>(mp); break;
+            case 2: dc::mass::mass_kernel<2><<<grid, dc::mass::kThreads, smem, st>>>(mp); break;
+            case 3: dc::mass::mass_kernel<3><<<grid, dc::mass::kThreads, smem, st>>>(mp); break;
+            default: dc::mass::mass_kernel<4><<<grid, dc::mass::kThreads, smem, st>>>(mp); break;
+        }
+    }
     return (cudaGetLastError() == cudaSuccess) ? KVPACK_OK : KVPACK_ERR_CUDA;
 }
 
