@@ -346,38 +346,31 @@ namespace vis {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kMeta = 4;            // item metadata ring (the issue side runs up to two items ahead)
+constexpr int kSub = 64;        // tokens per sub-chunk: one LO stage
+constexpr int kSubMeta = 8;     // sub-chunk metadata ring per warp (at most kSlots sub-chunks are in flight)
+constexpr int kItemQ = 4;       // fetched-item ring per warp
 
 // Geometry per head-block count.  Up to 16 query heads per unit: two blocks per
-// SM (their serial phases overlap), 4 KB ring slots.  Up to 32: one block per SM.
+// SM.  Up to 32: one block per SM with a deeper ring.
 template <int NMB>
 struct Cfg {
     static constexpr int kRows = 16 * NMB;                      // query-head rows (padded)
     static constexpr int kBlocks = (NMB == 1) ? 2 : 1;          // resident blocks per SM
-    static constexpr int kSlots = 2;                            // ring slots per warp
-    static constexpr int kSlotBytes = (NMB == 1) ? 4096 : 8192; // K rows in the first half, V in the second
-    static constexpr int kHiTok = (NMB == 1) ? 16 : 32;         // full-rank tokens per HI stage
+    static constexpr int kSlots = (NMB == 1) ? 2 : 4;           // ring slots per warp
+    static constexpr int kSlotBytes = 4096;                     // K rows in the first half, V in the second
+    static constexpr int kHiTok = 16;                           // full-rank tokens per HI stage
     static constexpr int kNTH = kHiTok / 8;                     // m16n8 token tiles per HI stage
-    static constexpr int kLoTok = 64;                           // visual tokens per warp per item
-    static constexpr int kItemTok = kWarps * kLoTok;            // tokens per item
-    static constexpr int kHiMax = kLoTok / kHiTok;              // HI stages per warp per item, at most
-    static constexpr int kUpd = 1 + kHiMax;                     // softmax updates per warp per item, at most
-    // tensor-memory columns of one warp's stash of one item: LO p (32 per head block), then HI p
-    static constexpr int kBufCols = 32 * NMB + 4 * kNTH * NMB * kHiMax;
-    static constexpr int kTmemCols = 4 * kBufCols;              // two warps per lane quarter, two items each
     static_assert(kHiTok * 128 == kSlotBytes / 2, "HI stage rows fill half a slot");
-    static_assert(kLoTok * 32 <= kSlotBytes / 2, "LO stage rows fit half a slot");
+    static_assert(kSub * 32 == kSlotBytes / 2, "LO stage rows fill half a slot");
 };
 
 struct Params {
     CUtensorMap tm_ck, tm_cv;   // C_lo planes: 3D {16, T, units}, box {16, 32, 1}, 32-byte swizzle
     const uint16_t *CK_lo, *CK_hi, *CV_lo, *CV_hi;
-    const unsigned char *qt;    // [units][qblock_bytes(Hg)] from text_kernel and text_stats_kernel
+    const unsigned char *qt;    // [units][qblock_bytes(Hg)] from text_kernel
     const uint32_t *mask;       // [units][nwords]
-    float *mass;                // [units][T] or null
     float *part;                // [units][S][Hg][kVisPart]
-    float *ustat;               // [units][Hg][2]: unit-wide (max, 1/sum); NaN at launch (S > 1)
-    unsigned int *arrive;       // [units], zero at launch
+    unsigned int *counter;      // work counter, zero at launch
     int n_units, T, Hg, S, tps, nwords, n_items;
 };
 
@@ -385,21 +378,13 @@ template <int NMB>
 struct Smem {
     using C = Cfg<NMB>;
     alignas(1024) unsigned char ring[kWarps][C::kSlots][C::kSlotBytes];
-    alignas(128) uint16_t qt[2][C::kRows][64];              // q~ hi / lo of the current item
-    alignas(16) float tst[C::kRows][2];                      // text (max, sum) of the current item's unit
-    float tcur[C::kRows][2];                                 // the same, kept through the epilogue
-    float ubuf[4][16][64];                                   // merge staging: 4 warps x one 16-row block of u
-    float wm[kWarps][C::kRows], wl[kWarps][C::kRows];
-    float mcta[C::kRows], lcta[C::kRows], mfin[C::kRows], invl[C::kRows];
-    float mref[2][kWarps][C::kUpd][C::kRows];               // reference max of each stashed update
-    float upf[C::kRows][2];                                  // prefetched unit (max, 1/sum) of the previous item
-    uint16_t hi_list[kMeta][kWarps][C::kLoTok];             // this warp's full-rank tokens (item-relative)
-    int meta[kMeta][kWarps][12];                            // lo0, n_lo, n_hi, item, 4 mask words of the LO range, unit, t0
+    alignas(128) uint16_t qt[kWarps][2][C::kRows][64];       // per warp: the next item's q~ hi / lo
+    uint8_t hi_list[kWarps][kSubMeta][kSub];                 // sub-chunk-relative positions of full-rank tokens
+    int meta[kWarps][kSubMeta][8];                           // K, unit, t0, n, n_hi, w0, w1, flags
+    int itemq[kWarps][kItemQ];
     uint64_t full[kWarps][C::kSlots];
-    uint64_t qbar;
-    uint32_t tmem_base;
+    uint64_t qbar[kWarps];
     int abort;
-    int last;
 };
 
 template <int NMB>
@@ -453,76 +438,19 @@ __device__ __forceinline__ void lazy_update(float (&s)[NT][4], float (&m)[2], fl
     l[1] += sum1;
 }
 
-// Sum over the 8 lanes that share lane & 3 of 16 per-lane values, scattered:
-// afterwards the lane holds the totals of slots 8 b4 + 4 b3 + 2 b2 + {0, 1}
-// (b = bits 4, 3, 2 of the lane).
-__device__ __forceinline__ void reduce_scatter16(const float (&x)[16], float (&out)[2], int lane) {
-    float t8[8], t4[4];
-    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-    #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float send = b4 ? x[i] : x[8 + i];
-        t8[i] = (b4 ? x[8 + i] : x[i]) + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-    #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float send = b3 ? t8[i] : t8[4 + i];
-        t4[i] = (b3 ? t8[4 + i] : t8[i]) + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-    #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const float send = b2 ? t4[i] : t4[2 + i];
-        out[i] = (b2 ? t4[2 + i] : t4[i]) + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-}
-
-// 8 values -> the lane holds the total of slot 4 b4 + 2 b3 + b2
-__device__ __forceinline__ float reduce_scatter8(const float (&x)[8], int lane) {
-    float t4[4], t2[2];
-    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-    #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float send = b4 ? x[i] : x[4 + i];
-        t4[i] = (b4 ? x[4 + i] : x[i]) + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-    #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const float send = b3 ? t4[i] : t4[2 + i];
-        t2[i] = (b3 ? t4[2 + i] : t4[i]) + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-    const float send = b2 ? t2[0] : t2[1];
-    return (b2 ? t2[1] : t2[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
-}
-
-// 4 values -> lanes with bit 2 clear hold the total of slot 2 b4 + b3 (the
-// lanes with bit 2 set hold the same totals)
-__device__ __forceinline__ float reduce_scatter4(const float (&x)[4], int lane) {
-    float t2[2];
-    const bool b4 = lane & 16, b3 = lane & 8;
-    #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const float send = b4 ? x[i] : x[2 + i];
-        t2[i] = (b4 ? x[2 + i] : x[i]) + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-    const float send = b3 ? t2[0] : t2[1];
-    const float t = (b3 ? t2[1] : t2[0]) + __shfl_xor_sync(0xffffffffu, send, 8);
-    return t + __shfl_xor_sync(0xffffffffu, t, 4);
-}
-
-// Persistent, one or two 256-thread blocks per SM, a static round-robin over items
-// (unit, split).  Each warp streams its own share of the item -- a contiguous
-// range of C_lo rows (TMA) and an equal share of the item's full-rank tokens
-// (C_lo + C_hi rows gathered with cp.async) -- through a private 3-slot ring,
-// with heads on M and tokens on N of mma.sync m16n8k16:
+// Persistent, one or two 256-thread blocks per SM; every warp works alone.
+// A warp fetches items (unit, chunk of tps tokens) from a global counter and
+// streams each through a private ring, 64 tokens (a sub-chunk) at a time: one
+// TMA stage of C_lo rows of K and V (skipped when every token is full-rank)
+// and one gathered stage (C_lo + C_hi rows of K and V, cp.async) per 16
+// full-rank tokens.  With heads on M and tokens on N of mma.sync m16n8k16:
 //   scores  s = q~ C_K^T  (q~ as a bf16 hi + lo pair, C_K exact in bf16)
 //   softmax online per head row; P stays in registers as the A operand of
-//   values  u += P C_V    (rank 16 over the LO range, rank 64 for HI tokens;
+//   values  u += P C_V    (rank 16 over the LO tokens, rank 64 for HI tokens;
 //                          a token with its mask bit set gets logit -inf in LO)
-// Each softmax update also stores its p (fp32) to tensor memory together with
-// the running max it was taken against.  At the item's end the warps merge
-// (max, sum, u) and publish the split's partial; the attention mass of the
-// item is written one item later, when every split of the unit (and the text
-// partials) fix the unit's max and sum: mass_t = sum_h p_ht 2^(m_ref - M_h) / L_h.
+// At the item's end the warp writes the partial (max, sum, u) of each head.
+// The unit's q~ block comes into one of two per-warp buffers by bulk copy
+// when the issue side begins an item.
 template <int NMB>
 __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const __grid_constant__ Params p) {
     using C = Cfg<NMB>;
@@ -535,128 +463,102 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
     volatile int *abort = &sm.abort;
 
     if (tid == 0) {
-        for (int w = 0; w < kWarps; ++w)
+        for (int w = 0; w < kWarps; ++w) {
             for (int s = 0; s < kSlots; ++s) mbar_init(&sm.full[w][s], 32);
-        mbar_init(&sm.qbar, 1);
+            mbar_init(&sm.qbar[w], 1);
+        }
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    for (int i = tid; i < 2 * C::kRows * 64; i += kThreads) (&sm.qt[0][0][0])[i] = 0;
-    if (warp == 0) tmem_alloc(&sm.tmem_base, C::kTmemCols);
-    tmem_fence_before();
+    // query rows past Hg stay zero
+    for (int i = tid; i < kWarps * 2 * C::kRows * 64 / 8; i += kThreads)
+        reinterpret_cast<uint4 *>(&sm.qt[0][0][0][0])[i] = make_uint4(0u, 0u, 0u, 0u);
     __syncthreads();
-    tmem_fence_after();
-    const uint32_t tmem = sm.tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(2 * C::kBufCols * (warp >> 2));
-
-    auto item_of = [&](int K) { return (int)blockIdx.x + K * (int)gridDim.x; };
-    auto issue_q = [&](int K) {   // query block of item K's unit into sm.qt / sm.tst (one thread)
-        const unsigned char *src = p.qt + (size_t)(item_of(K) / p.S) * qblock_bytes(p.Hg);
-        const uint32_t bytes = (uint32_t)p.Hg * 128u;
-        fence_proxy_async();
-        mbar_arrive_tx(&sm.qbar, (uint32_t)qblock_bytes(p.Hg));
-        bulk_g2s(&sm.qt[0][0][0], src, bytes, &sm.qbar);
-        bulk_g2s(&sm.qt[1][0][0], src + bytes, bytes, &sm.qbar);
-        bulk_g2s(&sm.tst[0][0], src + 2 * bytes, (uint32_t)p.Hg * 8u, &sm.qbar);
-    };
-    if (tid == 0) issue_q(0);
 
     // ------------------------------------------------------------ issue side
-    auto load_words = [&](int K) -> uint32_t {   // lane i: mask word i of item K
-        const int item = item_of(K);
-        if (item >= p.n_items) return 0u;
-        const int unit = item / p.S, t0 = (item % p.S) * p.tps;
-        const int n = min(p.T, t0 + p.tps) - t0;
-        const int nw = (n + 31) >> 5;
-        if (lane >= nw) return 0u;
-        uint32_t v = __ldg(p.mask + (size_t)unit * p.nwords + (t0 >> 5) + lane);
-        if (lane == nw - 1 && (n & 31)) v &= (1u << (n & 31)) - 1u;
-        return v;
-    };
-    int iK = 0, i_st = 0, i_nst = 0;
+    int iK = -1, i_item = 0, i_sc = 0, i_nsc = 0, i_st = 0, i_nst = 0;
+    uint32_t i_seq = 0, c_seq = 0, i_sub = 0, c_sub = 0;
     bool i_done = false;
-    uint32_t i_seq = 0, c_seq = 0;
-    int Kc = 0;                          // item the consumer is on
-    uint32_t mw = load_words(0), mw_nx = load_words(1);
-
-    // metadata of item K for this warp (meta slot K % kMeta); false if there is no item K
-    auto begin_item = [&](int K) -> bool {
-        const int item = item_of(K);
-        if (item >= p.n_items) return false;
-        const int t0 = (item % p.S) * p.tps;
-        const int n = min(p.T, t0 + p.tps) - t0;
-        int wt = (n + kWarps - 1) / kWarps;
-        wt = (wt + 31) & ~31;
-        const int lo0 = warp * wt;
-        int n_lo = max(0, min(wt, n - lo0));
-        const int wl0 = lo0 >> 5;
-        if (n_lo > 0) {
-            // the LO range is skipped when every token in it is full-rank
-            const int wln = (n_lo + 31) >> 5;
-            const bool in = lane >= wl0 && lane < wl0 + wln;
-            uint32_t need = 0xffffffffu;
-            if (in && lane == wl0 + wln - 1 && (n_lo & 31)) need = (1u << (n_lo & 31)) - 1u;
-            if (__all_sync(0xffffffffu, !in || (mw & need) == need)) n_lo = 0;
+    int cK = -1;   // item the consumer is on
+    auto fetch = [&]() -> int {
+        int v = 0;
+        if (lane == 0) v = (int)atomicAdd(p.counter, 1u);
+        return __shfl_sync(0xffffffffu, v, 0);
+    };
+    // sub-chunk i_sc of the issue side's item into meta slot i_sub % kSubMeta
+    auto begin_sub = [&]() {
+        const int ms = i_sub % kSubMeta;
+        const int unit = i_item / p.S, t0 = (i_item % p.S) * p.tps + kSub * i_sc;
+        const int n = min(kSub, p.T - t0);
+        uint32_t w = 0u;
+        if (lane < 2 && 32 * lane < n) {
+            w = __ldg(p.mask + (size_t)unit * p.nwords + (t0 >> 5) + lane);
+            const int nb = n - 32 * lane;
+            if (nb < 32) w &= (1u << nb) - 1u;
         }
-        const int cnt = __popc(mw);
-        int incl = cnt;
-        #pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, d);
-            if (lane >= d) incl += v;
-        }
-        const int n_hi = __shfl_sync(0xffffffffu, incl, 31);
-        const int h0 = (warp * n_hi) / kWarps, h1 = ((warp + 1) * n_hi) / kWarps;
-        const int ms = K % kMeta;
-        int gi = incl - cnt;
-        uint32_t bits = mw;
-        while (bits) {
-            const int b = __ffs(bits) - 1;
-            if (gi >= h0 && gi < h1) sm.hi_list[ms][warp][gi - h0] = (uint16_t)(32 * lane + b);
-            ++gi;
-            bits &= bits - 1u;
-        }
-        if (lane >= wl0 && lane < wl0 + 4) sm.meta[ms][warp][4 + lane - wl0] = (int)mw;
+        const uint32_t w0 = __shfl_sync(0xffffffffu, w, 0), w1 = __shfl_sync(0xffffffffu, w, 1);
+        const int c0 = __popc(w0), n_hi = c0 + __popc(w1);
+        const uint32_t below = (1u << lane) - 1u;
+        if ((w0 >> lane) & 1u) sm.hi_list[warp][ms][__popc(w0 & below)] = (uint8_t)lane;
+        if ((w1 >> lane) & 1u) sm.hi_list[warp][ms][c0 + __popc(w1 & below)] = (uint8_t)(32 + lane);
         if (lane == 0) {
-            sm.meta[ms][warp][0] = lo0;
-            sm.meta[ms][warp][1] = n_lo;
-            sm.meta[ms][warp][2] = h1 - h0;
-            sm.meta[ms][warp][3] = item;
-            sm.meta[ms][warp][8] = item / p.S;
-            sm.meta[ms][warp][9] = t0;
+            int *m = sm.meta[warp][ms];
+            m[0] = iK; m[1] = unit; m[2] = t0; m[3] = n; m[4] = n_hi; m[5] = (int)w0; m[6] = (int)w1;
+            m[7] = (i_sc == 0 ? 1 : 0) | (i_sc + 1 == i_nsc ? 2 : 0);
         }
         __syncwarp();
-        i_nst = (n_lo > 0 ? 1 : 0) + (h1 - h0 + kHiTok - 1) / kHiTok;
+        i_nst = (n_hi < n ? 1 : 0) + (n_hi + kHiTok - 1) / kHiTok;
         i_st = 0;
+    };
+    // the next item: its q~ block into the warp's staging buffer (free once the consumer
+    // has taken the current item's q~ into registers)
+    auto begin_item = [&]() -> bool {
+        const int it = fetch();
+        if (it >= p.n_items) return false;
+        ++iK;
+        i_item = it;
+        if (lane == 0) sm.itemq[warp][iK % kItemQ] = it;
+        const int t0 = (it % p.S) * p.tps;
+        i_nsc = (min(p.tps, p.T - t0) + kSub - 1) / kSub;
+        i_sc = 0;
+        if (lane == 0) {
+            const unsigned char *src = p.qt + (size_t)(it / p.S) * qblock_bytes(p.Hg);
+            const uint32_t bytes = (uint32_t)p.Hg * 128u;
+            uint64_t *qb = &sm.qbar[warp];
+            fence_proxy_async();
+            mbar_arrive_tx(qb, 2 * bytes);
+            bulk_g2s(&sm.qt[warp][0][0][0], src, bytes, qb);
+            bulk_g2s(&sm.qt[warp][1][0][0], src + bytes, bytes, qb);
+        }
+        __syncwarp();
         return true;
     };
-
     auto issue_stage = [&]() {
-        const int ms = iK % kMeta;
-        const int lo0 = sm.meta[ms][warp][0], n_lo = sm.meta[ms][warp][1], nh = sm.meta[ms][warp][2];
-        const int unit = sm.meta[ms][warp][8], t0 = sm.meta[ms][warp][9];
+        const int ms = i_sub % kSubMeta;
+        const int *m = sm.meta[warp][ms];
+        const int unit = m[1], t0 = m[2], n = m[3], n_hi = m[4];
         const int slot = i_seq % kSlots;
         unsigned char *dst = sm.ring[warp][slot];
         uint64_t *bar = &sm.full[warp][slot];
         __syncwarp();
-        if (i_st == 0 && n_lo > 0) {
-            // whole 64-row halves: the value MMA reads every row of a half (masked rows get p = 0,
+        if (i_st == 0 && n_hi < n) {
+            // all 64 rows of K and V: the value MMA reads every row (masked rows get p = 0,
             // which must meet finite data -- neighbouring rows, or zeros past the unit's end)
-            const int nb = 2 * ((n_lo + 63) >> 6);
             if (lane == 0) {
                 fence_proxy_async();
-                mbar_arrive_tx(bar, (uint32_t)nb * 2048u);
-                for (int b = 0; b < nb; ++b) {
-                    tma_3d(dst + 1024 * b, &p.tm_ck, 0, t0 + lo0 + 32 * b, unit, bar);
-                    tma_3d(dst + kHalf + 1024 * b, &p.tm_cv, 0, t0 + lo0 + 32 * b, unit, bar);
-                }
+                mbar_arrive_tx(bar, 4u * 1024u);
+                tma_3d(dst, &p.tm_ck, 0, t0, unit, bar);
+                tma_3d(dst + 1024, &p.tm_ck, 0, t0 + 32, unit, bar);
+                tma_3d(dst + kHalf, &p.tm_cv, 0, t0, unit, bar);
+                tma_3d(dst + kHalf + 1024, &p.tm_cv, 0, t0 + 32, unit, bar);
             } else {
                 mbar_arrive(bar);
             }
         } else {
-            // 32 full-rank tokens: C_lo + C_hi rows of K and V gathered into 128-byte rows
+            // kHiTok full-rank tokens: C_lo + C_hi rows of K and V gathered into 128-byte rows
             // (16-byte chunk c of row r stored at c ^ (r & 7)); rows past the count are zero
-            const int hs = i_st - (n_lo > 0 ? 1 : 0);
-            const int cnt = min(kHiTok, nh - kHiTok * hs);
+            const int hs = i_st - (n_hi < n ? 1 : 0);
+            const int cnt = min(kHiTok, n_hi - kHiTok * hs);
             const size_t ubase = (size_t)unit * p.T + t0;
             #pragma unroll
             for (int i = 0; i < kHiTok / 4; ++i) {
@@ -666,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
                 unsigned char *dk = dst + r * 128 + pos;
                 unsigned char *dv = dst + kHalf + r * 128 + pos;
                 if (r < cnt) {
-                    const size_t row = ubase + sm.hi_list[ms][warp][kHiTok * hs + r];
+                    const size_t row = ubase + sm.hi_list[warp][ms][kHiTok * hs + r];
                     if (ch < 2) {
                         cp_async16(dk, p.CK_lo + row * 16 + ch * 8);
                         cp_async16(dv, p.CV_lo + row * 16 + ch * 8);
@@ -682,517 +584,206 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
             cp_async_arrive_noinc(bar);
         }
         ++i_st;
+        if (i_st == i_nst) ++i_sub;
         ++i_seq;
     };
-
-    // issue while the ring has room; the issue side may begin items up to Kc + 2
+    // issue while the ring has room; the issue side may begin item cK + 1 at most
+    // (its q~ overwrites the staging buffer, which the consumer emptied when it began item cK)
     auto pump = [&]() {
         while (!i_done && i_seq - c_seq < (uint32_t)kSlots) {
             if (i_st == i_nst) {
-                if (iK + 1 > Kc + 2) return;
-                ++iK;
-                mw = mw_nx;
-                mw_nx = load_words(iK + 1);
-                if (!begin_item(iK)) { i_done = true; return; }
+                if (i_sub - c_sub >= (uint32_t)kSubMeta) return;
+                if (iK >= 0 && i_sc + 1 < i_nsc) {
+                    ++i_sc;
+                } else {
+                    if (iK + 1 > cK + 1) return;
+                    if (!begin_item()) { i_done = true; return; }
+                }
+                begin_sub();
                 continue;
             }
             issue_stage();
         }
     };
-    if (!begin_item(0)) i_done = true;
     pump();
 
     // ---------------------------------------------------------- consumer side
     float m[NMB][2], l[NMB][2], u[NMB][8][4];
-    uint32_t qah[NMB][4], qal[NMB][4];
-    const uint32_t qt0 = smem_u32(&sm.qt[0][0][0]), qt1 = smem_u32(&sm.qt[1][0][0]);
+    uint32_t qh[NMB][4][4], ql[NMB][4][4];   // q~ hi / lo as A fragments: head block, k-step
+    bool ok = true;
 
-    // Attention mass of this warp's tokens of item K (meta slot K % kMeta, stash
-    // buffer K & 1), one warp alone.  The unit's (max, 1/sum) per head come from
-    // shared memory (single-split units) or from ustat, polled until the unit's
-    // last split has written them.
-    auto mass_warp = [&](int K, int src) {
-        const int item = item_of(K);
-        const int unit = item / p.S;
-        float Mr[NMB][2], IL[NMB][2];
-        bool ready = true;
+    // LO tokens: one softmax update over 8 NT C_lo rows of a stage (NT m16n8 tiles of tokens;
+    // n of them inside the unit; mask words w0, w1 cover them)
+    auto do_lo = [&](uint32_t sb, uint32_t w0, uint32_t w1, int n, auto ntc) {
+        constexpr int NT = decltype(ntc)::value;
+        const uint32_t x[2] = {w0 >> (2 * tig), w1 >> (2 * tig)};   // bit 8 (nt & 3) + e: token 8 nt + 2 tig + e
+        const bool partial = n < 8 * NT;
         #pragma unroll
-        for (int mb = 0; mb < NMB; ++mb)
+        for (int mb = 0; mb < NMB; ++mb) {
+            float s[NT][4];
             #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int row = 16 * mb + g + 8 * r;
-                const bool ok = row < p.Hg;
-                Mr[mb][r] = ok ? (src == 0 ? sm.mfin[row] : sm.upf[row][0]) : 0.f;
-                IL[mb][r] = ok ? (src == 0 ? sm.invl[row] : sm.upf[row][1]) : 0.f;
-                ready = ready && !(Mr[mb][r] != Mr[mb][r]) && !(IL[mb][r] != IL[mb][r]);
+            for (int a = 0; a < NT; ++a) s[a][0] = s[a][1] = s[a][2] = s[a][3] = 0.f;
+            #pragma unroll
+            for (int np = 0; np < NT / 2; ++np) {
+                uint32_t b0, b1, b2, b3;
+                const int row = 16 * np + (lane & 7) + ((lane >> 4) << 3);
+                const int ch = (lane >> 3) & 1;
+                ldsm_x4(sb + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), b0, b1, b2, b3);
+                mma_bf16(s[2 * np], qh[mb][0], b0, b1);
+                mma_bf16(s[2 * np + 1], qh[mb][0], b2, b3);
+                mma_bf16(s[2 * np], ql[mb][0], b0, b1);
+                mma_bf16(s[2 * np + 1], ql[mb][0], b2, b3);
             }
-        if (src == 1 || (src == 2 && !__all_sync(0xffffffffu, ready))) {
-            const long long start = clock64();
-            while (true) {
-                ready = true;
+            #pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
                 #pragma unroll
-                for (int mb = 0; mb < NMB; ++mb)
-                    #pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        const int row = 16 * mb + g + 8 * r;
-                        float a = 0.f, b2 = 0.f;
-                        if (row < p.Hg) {
-                            const float *us = p.ustat + ((size_t)unit * p.Hg + row) * 2;
-                            asm volatile("ld.relaxed.gpu.global.v2.f32 {%0, %1}, [%2];" : "=f"(a), "=f"(b2) : "l"(us) : "memory");
-                        }
-                        Mr[mb][r] = a;
-                        IL[mb][r] = b2;
-                        ready = ready && !(a != a) && !(b2 != b2);
-                    }
-                if (__all_sync(0xffffffffu, ready)) break;
-                if (*abort) return;
-                if (clock64() - start > kWaitCycles) {
-                    report_error(KVPACK_ERR_TIMEOUT);
-                    *abort = 1;
-                    return;
+                for (int e = 0; e < 2; ++e) {
+                    const bool hb = (x[nt >> 2] >> (8 * (nt & 3) + e)) & 1u;
+                    const bool out = hb || (partial && 8 * nt + 2 * tig + e >= n);
+                    if (out) s[nt][e] = s[nt][2 + e] = -INFINITY;
                 }
-                __nanosleep(100);
+            lazy_update<NT>(s, m[mb], l[mb], u[mb]);
+            #pragma unroll
+            for (int kk = 0; kk < NT / 2; ++kk) {
+                uint32_t a[4];
+                a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+                a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+                a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+                a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+                uint32_t b0, b1, b2, b3;
+                const int row = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
+                const int ch = lane >> 4;
+                ldsm_x4_t(sb + kHalf + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), b0, b1, b2, b3);
+                mma_bf16(u[mb][0], a, b0, b1);
+                mma_bf16(u[mb][1], a, b2, b3);
             }
         }
-        const int ms = K % kMeta, b = K & 1;
-        const int lo0 = sm.meta[ms][warp][0], n_lo = sm.meta[ms][warp][1], nh = sm.meta[ms][warp][2];
-        const int t0 = (item % p.S) * p.tps;
-        float *mrow = p.mass + (size_t)unit * p.T + t0;
-        auto fac = [&](int upd, int mb, int r) -> float {
-            const int row = 16 * mb + g + 8 * r;
-            return row < p.Hg ? ex2(sm.mref[b][warp][upd][row] - Mr[mb][r]) * IL[mb][r] : 0.f;
-        };
-        tmem_fence_after();
-        // LO range (64 tokens)
-        const uint32_t bcol = (uint32_t)(C::kBufCols * b);
-        if (n_lo > 0) {
-            float acc[16];
+    };
+
+    // kHiTok full-rank tokens (n of them valid)
+    auto do_hi = [&](uint32_t sb, int n) {
+        #pragma unroll
+        for (int mb = 0; mb < NMB; ++mb) {
+            float s[kNTH][4];
             #pragma unroll
-            for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+            for (int a = 0; a < kNTH; ++a) s[a][0] = s[a][1] = s[a][2] = s[a][3] = 0.f;
             #pragma unroll
-            for (int mb = 0; mb < NMB; ++mb) {
-                float v0[16], v1[16];
-                const uint32_t col = bcol + (uint32_t)(32 * mb);
-                tmem_ld16(tmem + col, v0);
-                tmem_ld16(tmem + col + 16, v1);
-                tmem_wait_ld();
-                const float f0 = fac(0, mb, 0), f1 = fac(0, mb, 1);
+            for (int kb = 0; kb < 4; ++kb) {
                 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
-                    #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        acc[2 * nt + e] += v0[4 * nt + e] * f0 + v0[4 * nt + 2 + e] * f1;
-                        acc[8 + 2 * nt + e] += v1[4 * nt + e] * f0 + v1[4 * nt + 2 + e] * f1;
-                    }
-            }
-            float out[2];
-            reduce_scatter16(acc, out, lane);
-            const int nt = 4 * ((lane >> 4) & 1) + 2 * ((lane >> 3) & 1) + ((lane >> 2) & 1);
-            #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int r = 8 * nt + 2 * tig + e;
-                const bool hb = ((uint32_t)sm.meta[ms][warp][4 + (r >> 5)] >> (r & 31)) & 1u;
-                if (r < n_lo && !hb) mrow[lo0 + r] = out[e];
-            }
-        }
-        // full-rank tokens
-        for (int hs = 0; hs * kHiTok < nh; ++hs) {
-            const int n = min(kHiTok, nh - kHiTok * hs);
-            float acc[2 * kNTH];
-            #pragma unroll
-            for (int i = 0; i < 2 * kNTH; ++i) acc[i] = 0.f;
-            const int upd = 1 + hs;
-            #pragma unroll
-            for (int mb = 0; mb < NMB; ++mb) {
-                float v[16];
-                const uint32_t col = bcol + (uint32_t)(32 * NMB + (hs * NMB + mb) * 4 * kNTH);
-                if (kNTH == 4) {
-                    tmem_ld16(tmem + col, v);
-                } else {
-                    float v8[8];
-                    tmem_ld8(tmem + col, v8);
-                    #pragma unroll
-                    for (int i = 0; i < 8; ++i) v[i] = v8[i];
+                for (int np = 0; np < kNTH / 2; ++np) {
+                    uint32_t b0, b1, b2, b3;
+                    const int row = 16 * np + (lane & 7) + ((lane >> 4) << 3);
+                    const int ch = 2 * kb + ((lane >> 3) & 1);
+                    ldsm_x4(sb + row * 128 + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
+                    mma_bf16(s[2 * np], qh[mb][kb], b0, b1);
+                    mma_bf16(s[2 * np + 1], qh[mb][kb], b2, b3);
+                    mma_bf16(s[2 * np], ql[mb][kb], b0, b1);
+                    mma_bf16(s[2 * np + 1], ql[mb][kb], b2, b3);
                 }
-                tmem_wait_ld();
-                const float f0 = fac(upd, mb, 0), f1 = fac(upd, mb, 1);
+            }
+            if (n < kHiTok) {
                 #pragma unroll
                 for (int nt = 0; nt < kNTH; ++nt)
                     #pragma unroll
-                    for (int e = 0; e < 2; ++e) acc[2 * nt + e] += v[4 * nt + e] * f0 + v[4 * nt + 2 + e] * f1;
+                    for (int e = 0; e < 2; ++e)
+                        if (8 * nt + 2 * tig + e >= n) s[nt][e] = s[nt][2 + e] = -INFINITY;
             }
-            int j;
-            float val;
-            if (kNTH == 4) {
-                float a8[8];
-                #pragma unroll
-                for (int i = 0; i < 8; ++i) a8[i] = acc[i];
-                val = reduce_scatter8(a8, lane);
-                j = 4 * ((lane >> 4) & 1) + 2 * ((lane >> 3) & 1) + ((lane >> 2) & 1);
-            } else {
-                float a4[4];
-                #pragma unroll
-                for (int i = 0; i < 4; ++i) a4[i] = acc[i];
-                val = reduce_scatter4(a4, lane);
-                j = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-            }
-            const int colt = 8 * (j >> 1) + 2 * tig + (j & 1);
-            const bool writer = kNTH == 4 || ((lane >> 2) & 1) == 0;
-            if (writer && colt < n) mrow[sm.hi_list[ms][warp][kHiTok * hs + colt]] = val;
-        }
-        tmem_fence_before();
-    };
-
-    int K = 0;
-    for (;; ++K) {
-        const int item = item_of(K);
-        if (item >= p.n_items) break;
-        Kc = K;
-        pump();
-        const int ms = K % kMeta, b = K & 1;
-        const int n_lo = sm.meta[ms][warp][1], nh = sm.meta[ms][warp][2];
-        uint32_t lw[4];
-        #pragma unroll
-        for (int k = 0; k < 4; ++k) lw[k] = (uint32_t)sm.meta[ms][warp][4 + k];
-        const int unit = item / p.S, split = item % p.S;
-
-        bool ok = mbar_wait(&sm.qbar, (uint32_t)(K & 1), abort);
-        #pragma unroll
-        for (int mb = 0; mb < NMB; ++mb) {
-            const int row = 16 * mb + (lane & 7) + (((lane >> 3) & 1) << 3);
-            const uint32_t off = row * 128 + (((lane >> 4) ^ (row & 7)) << 4);
-            ldsm_x4(qt0 + off, qah[mb][0], qah[mb][1], qah[mb][2], qah[mb][3]);
-            ldsm_x4(qt1 + off, qal[mb][0], qal[mb][1], qal[mb][2], qal[mb][3]);
-            m[mb][0] = m[mb][1] = kRefInit;
-            l[mb][0] = l[mb][1] = 0.f;
+            lazy_update<kNTH>(s, m[mb], l[mb], u[mb]);
             #pragma unroll
-            for (int a = 0; a < 8; ++a) u[mb][a][0] = u[mb][a][1] = u[mb][a][2] = u[mb][a][3] = 0.f;
-        }
-        const uint32_t tcol = tmem + (uint32_t)(C::kBufCols * b);
-        const int nst = (n_lo > 0 ? 1 : 0) + (nh + kHiTok - 1) / kHiTok;
-
-        // LO range: one softmax update over all of this warp's C_lo rows (NT m16n8 tiles of tokens)
-        auto do_lo = [&](uint32_t sb, auto ntc) {
-            constexpr int NT = decltype(ntc)::value;
-            uint32_t x[NT / 4];   // mask words shifted so that bit 8 (nt & 3) + e is token 8 nt + 2 tig + e
-            #pragma unroll
-            for (int w4 = 0; w4 < NT / 4; ++w4) x[w4] = lw[w4] >> (2 * tig);
-            const bool partial = n_lo < 8 * NT;
-            #pragma unroll
-            for (int mb = 0; mb < NMB; ++mb) {
-                float s[NT][4];
+            for (int kk = 0; kk < kNTH / 2; ++kk) {
+                uint32_t a[4];
+                a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+                a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+                a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+                a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
                 #pragma unroll
-                for (int a = 0; a < NT; ++a) s[a][0] = s[a][1] = s[a][2] = s[a][3] = 0.f;
-                #pragma unroll
-                for (int np = 0; np < NT / 2; ++np) {
-                    uint32_t b0, b1, b2, b3;
-                    const int row = 16 * np + (lane & 7) + ((lane >> 4) << 3);
-                    const int ch = (lane >> 3) & 1;
-                    ldsm_x4(sb + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), b0, b1, b2, b3);
-                    mma_bf16(s[2 * np], qah[mb], b0, b1);
-                    mma_bf16(s[2 * np + 1], qah[mb], b2, b3);
-                    mma_bf16(s[2 * np], qal[mb], b0, b1);
-                    mma_bf16(s[2 * np + 1], qal[mb], b2, b3);
-                }
-                #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                    #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const bool hb = (x[nt >> 2] >> (8 * (nt & 3) + e)) & 1u;
-                        const bool out = hb || (partial && 8 * nt + 2 * tig + e >= n_lo);
-                        if (out) s[nt][e] = s[nt][2 + e] = -INFINITY;
-                    }
-                lazy_update<NT>(s, m[mb], l[mb], u[mb]);
-                if (p.mass != nullptr) {
-                    if (tig == 0) {
-                        sm.mref[b][warp][0][16 * mb + g] = m[mb][0];
-                        sm.mref[b][warp][0][16 * mb + g + 8] = m[mb][1];
-                    }
-                    #pragma unroll
-                    for (int c4 = 0; c4 < NT / 4; ++c4) {
-                        float v[16];
-                        #pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] = s[4 * c4 + (i >> 2)][i & 3];
-                        tmem_st16(tcol + (uint32_t)(32 * mb + 16 * c4), v);
-                    }
-                }
-                #pragma unroll
-                for (int kk = 0; kk < NT / 2; ++kk) {
-                    uint32_t a[4];
-                    a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-                    a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-                    a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-                    a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+                for (int pr = 0; pr < 4; ++pr) {
                     uint32_t b0, b1, b2, b3;
                     const int row = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
-                    const int ch = lane >> 4;
-                    ldsm_x4_t(sb + kHalf + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), b0, b1, b2, b3);
-                    mma_bf16(u[mb][0], a, b0, b1);
-                    mma_bf16(u[mb][1], a, b2, b3);
+                    const int ch = 2 * pr + (lane >> 4);
+                    ldsm_x4_t(sb + kHalf + row * 128 + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
+                    mma_bf16(u[mb][2 * pr], a, b0, b1);
+                    mma_bf16(u[mb][2 * pr + 1], a, b2, b3);
                 }
             }
-        };
+        }
+    };
 
-        for (int st = 0; st < nst && ok; ++st) {
+    while (ok) {
+        pump();
+        if (c_sub == i_sub && c_seq == i_seq) break;   // nothing issued and nothing left to issue
+        const int ms = c_sub % kSubMeta;
+        const int *mt = sm.meta[warp][ms];
+        const int K = mt[0], n = mt[3], n_hi = mt[4], flags = mt[7];
+        const uint32_t w0 = (uint32_t)mt[5], w1 = (uint32_t)mt[6];
+        if (flags & 1) {
+            // first sub-chunk of item K: its q~ block, fresh softmax state
+            if (!mbar_wait(&sm.qbar[warp], (uint32_t)(K & 1), abort)) { ok = false; break; }
+            const uint32_t qt0 = smem_u32(&sm.qt[warp][0][0][0]), qt1 = smem_u32(&sm.qt[warp][1][0][0]);
+            #pragma unroll
+            for (int mb = 0; mb < NMB; ++mb) {
+                const int row = 16 * mb + (lane & 7) + (((lane >> 3) & 1) << 3);
+                #pragma unroll
+                for (int kb = 0; kb < 4; ++kb) {
+                    const int ch = 2 * kb + (lane >> 4);
+                    const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
+                    ldsm_x4(qt0 + off, qh[mb][kb][0], qh[mb][kb][1], qh[mb][kb][2], qh[mb][kb][3]);
+                    ldsm_x4(qt1 + off, ql[mb][kb][0], ql[mb][kb][1], ql[mb][kb][2], ql[mb][kb][3]);
+                }
+                m[mb][0] = m[mb][1] = kRefInit;
+                l[mb][0] = l[mb][1] = 0.f;
+                #pragma unroll
+                for (int a = 0; a < 8; ++a) u[mb][a][0] = u[mb][a][1] = u[mb][a][2] = u[mb][a][3] = 0.f;
+            }
+            __syncwarp();
+            cK = K;   // the staging buffer is free for the next item
+        }
+        const int nst = (n_hi < n ? 1 : 0) + (n_hi + kHiTok - 1) / kHiTok;
+        for (int st = 0; st < nst; ++st) {
             const int slot = c_seq % kSlots;
             if (!mbar_wait(&sm.full[warp][slot], (c_seq / kSlots) & 1u, abort)) { ok = false; break; }
             const uint32_t sb = smem_u32(sm.ring[warp][slot]);
-            if (st == 0 && n_lo > 0) {
-                do_lo(sb, std::integral_constant<int, 8>{});
-            } else {
-                // ------------------------------------------------ HI stage: kHiTok full-rank tokens
-                const int hs = st - (n_lo > 0 ? 1 : 0);
-                const int n = min(kHiTok, nh - kHiTok * hs);
-                const int upd = 1 + hs;
-                #pragma unroll
-                for (int mb = 0; mb < NMB; ++mb) {
-                    float s[kNTH][4];
-                    #pragma unroll
-                    for (int a = 0; a < kNTH; ++a) s[a][0] = s[a][1] = s[a][2] = s[a][3] = 0.f;
-                    #pragma unroll
-                    for (int kb = 0; kb < 4; ++kb) {
-                        uint32_t ah[4], al[4];
-                        if (kb == 0) {
-                            #pragma unroll
-                            for (int e = 0; e < 4; ++e) { ah[e] = qah[mb][e]; al[e] = qal[mb][e]; }
-                        } else {
-                            const int row = 16 * mb + (lane & 7) + (((lane >> 3) & 1) << 3);
-                            const int ch = 2 * kb + (lane >> 4);
-                            const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
-                            ldsm_x4(qt0 + off, ah[0], ah[1], ah[2], ah[3]);
-                            ldsm_x4(qt1 + off, al[0], al[1], al[2], al[3]);
-                        }
-                        #pragma unroll
-                        for (int np = 0; np < kNTH / 2; ++np) {
-                            uint32_t b0, b1, b2, b3;
-                            const int row = 16 * np + (lane & 7) + ((lane >> 4) << 3);
-                            const int ch = 2 * kb + ((lane >> 3) & 1);
-                            ldsm_x4(sb + row * 128 + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
-                            mma_bf16(s[2 * np], ah, b0, b1);
-                            mma_bf16(s[2 * np + 1], ah, b2, b3);
-                            mma_bf16(s[2 * np], al, b0, b1);
-                            mma_bf16(s[2 * np + 1], al, b2, b3);
-                        }
-                    }
-                    if (n < kHiTok) {
-                        #pragma unroll
-                        for (int nt = 0; nt < kNTH; ++nt)
-                            #pragma unroll
-                            for (int e = 0; e < 2; ++e)
-                                if (8 * nt + 2 * tig + e >= n) s[nt][e] = s[nt][2 + e] = -INFINITY;
-                    }
-                    lazy_update<kNTH>(s, m[mb], l[mb], u[mb]);
-                    if (p.mass != nullptr) {
-                        if (tig == 0) {
-                            sm.mref[b][warp][upd][16 * mb + g] = m[mb][0];
-                            sm.mref[b][warp][upd][16 * mb + g + 8] = m[mb][1];
-                        }
-                        const uint32_t col = tcol + (uint32_t)(32 * NMB + (hs * NMB + mb) * 4 * kNTH);
-                        if (kNTH == 4) {
-                            float v0[16];
-                            #pragma unroll
-                            for (int i = 0; i < 16; ++i) v0[i] = s[(i >> 2) % kNTH][i & 3];
-                            tmem_st16(col, v0);
-                        } else {
-                            float v0[8];
-                            #pragma unroll
-                            for (int i = 0; i < 8; ++i) v0[i] = s[(i >> 2) % kNTH][i & 3];
-                            tmem_st8(col, v0);
-                        }
-                    }
-                    #pragma unroll
-                    for (int kk = 0; kk < kNTH / 2; ++kk) {
-                        uint32_t a[4];
-                        a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-                        a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-                        a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-                        a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-                        #pragma unroll
-                        for (int pr = 0; pr < 4; ++pr) {
-                            uint32_t b0, b1, b2, b3;
-                            const int row = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
-                            const int ch = 2 * pr + (lane >> 4);
-                            ldsm_x4_t(sb + kHalf + row * 128 + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
-                            mma_bf16(u[mb][2 * pr], a, b0, b1);
-                            mma_bf16(u[mb][2 * pr + 1], a, b2, b3);
-                        }
-                    }
+            if (st == 0 && n_hi < n) {
+                if (NMB == 1) {   // two 32-token halves: fewer live scores
+                    do_lo(sb, w0, 0u, n, std::integral_constant<int, 4>{});
+                    if (n > 32) do_lo(sb + 1024, w1, 0u, n - 32, std::integral_constant<int, 4>{});
+                } else {
+                    do_lo(sb, w0, w1, n, std::integral_constant<int, 8>{});
                 }
+            } else {
+                const int hs = st - (n_hi < n ? 1 : 0);
+                do_hi(sb, min(kHiTok, n_hi - kHiTok * hs));
             }
             ++c_seq;
             __syncwarp();
             pump();
         }
-        if (!ok) *abort = 1;
-        if (p.mass != nullptr) tmem_wait_st();
-
-        // ================================================ item epilogue
-        #pragma unroll
-        for (int mb = 0; mb < NMB; ++mb)
+        if (!ok) break;
+        ++c_sub;
+        if (flags & 2) {
+            // last sub-chunk: the partial of item K -- per head row: max, sum, u[64]
+            const int item = sm.itemq[warp][K % kItemQ];
+            float *dst = p.part + (size_t)item * p.Hg * kVisPart;
             #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                float lt = l[mb][r];
-                lt += __shfl_xor_sync(0xffffffffu, lt, 1);
-                lt += __shfl_xor_sync(0xffffffffu, lt, 2);
-                if (tig == 0) {
-                    sm.wm[warp][16 * mb + g + 8 * r] = m[mb][r];
-                    sm.wl[warp][16 * mb + g + 8 * r] = lt;
-                }
-            }
-        if (tid < C::kRows) {   // the next item's query block lands in sm.tst after the barrier
-            sm.tcur[tid][0] = tid < p.Hg ? sm.tst[tid][0] : -INFINITY;
-            sm.tcur[tid][1] = tid < p.Hg ? sm.tst[tid][1] : 0.f;
-        }
-        // the previous item's unit (max, 1/sum), read now and stored after the merge
-        float pf0 = 0.f, pf1 = 0.f;
-        const bool prefetch = p.mass != nullptr && p.S > 1 && K >= 1 && tid < p.Hg;
-        if (prefetch) {
-            const float *us = p.ustat + ((size_t)(item_of(K - 1) / p.S) * p.Hg + tid) * 2;
-            asm volatile("ld.relaxed.gpu.global.v2.f32 {%0, %1}, [%2];" : "=f"(pf0), "=f"(pf1) : "l"(us) : "memory");
-        }
-        tmem_fence_before();
-        __syncthreads();
-        if (*abort) break;
-        if (tid == 0 && item_of(K + 1) < p.n_items) issue_q(K + 1);
-        if (tid < C::kRows) {
-            float mx = sm.wm[0][tid];
-            #pragma unroll
-            for (int w = 1; w < kWarps; ++w) mx = fmaxf(mx, sm.wm[w][tid]);
-            float sum = 0.f;
-            #pragma unroll
-            for (int w = 0; w < kWarps; ++w) sum += sm.wl[w][tid] * ex2(sm.wm[w][tid] - mx);
-            sm.mcta[tid] = mx;
-            sm.lcta[tid] = sum;
-            if (p.S == 1) {   // the unit's max and sum: this block's visual part and the text tail
-                const float t0m = sm.tcur[tid][0];
-                const float M = fmaxf(mx, t0m);
-                float L = sum * ex2(mx - M);
-                if (t0m != -INFINITY) L += sm.tcur[tid][1] * ex2(t0m - M);
-                sm.mfin[tid] = M;
-                sm.invl[tid] = 1.f / L;
-            }
-        }
-        // every thread rescales its u rows to the block reference (the max of the warps' references)
-        #pragma unroll
-        for (int mb = 0; mb < NMB; ++mb)
-            #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int row = 16 * mb + g + 8 * r;
-                float mc = sm.wm[0][row];
+            for (int mb = 0; mb < NMB; ++mb)
                 #pragma unroll
-                for (int w = 1; w < kWarps; ++w) mc = fmaxf(mc, sm.wm[w][row]);
-                const float f = row < p.Hg ? ex2(m[mb][r] - mc) : 0.f;
-                #pragma unroll
-                for (int nt = 0; nt < 8; ++nt) {
-                    u[mb][nt][2 * r] *= f;
-                    u[mb][nt][2 * r + 1] *= f;
-                }
-            }
-        // sum over the 8 warps, one 16-row block at a time: warps 4-7 hand their u to warps
-        // 0-3, which hand the pair sums on; every thread then adds the four for 4 outputs
-        {
-            float *dst = p.part + ((size_t)unit * p.S + split) * p.Hg * kVisPart;
-            #pragma unroll
-            for (int mb = 0; mb < NMB; ++mb) {
-                float *ub = &sm.ubuf[warp & 3][0][0];
-                if (mb > 0) __syncthreads();   // the previous block's sums have been read
-                if (warp >= 4) {
-                    #pragma unroll
-                    for (int nt = 0; nt < 8; ++nt)
-                        *reinterpret_cast<float4 *>(ub + 4 * (32 * nt + lane)) =
-                            make_float4(u[mb][nt][0], u[mb][nt][1], u[mb][nt][2], u[mb][nt][3]);
-                }
-                __syncthreads();
-                if (warp < 4) {
-                    #pragma unroll
-                    for (int nt = 0; nt < 8; ++nt) {
-                        const float4 v = *reinterpret_cast<const float4 *>(ub + 4 * (32 * nt + lane));
-                        *reinterpret_cast<float4 *>(ub + 4 * (32 * nt + lane)) =
-                            make_float4(u[mb][nt][0] + v.x, u[mb][nt][1] + v.y, u[mb][nt][2] + v.z, u[mb][nt][3] + v.w);
-                    }
-                }
-                __syncthreads();
-                // output (row, col) of the block: fragment (nt = col / 8, lane = 4 (row % 8) + (col % 8) / 2,
-                // element 2 (row / 8) + col % 2)
-                for (int o = tid; o < 16 * 64; o += kThreads) {
-                    const int row = o >> 6, col = o & 63;
-                    const int h = 16 * mb + row;
+                for (int r = 0; r < 2; ++r) {
+                    float lt = l[mb][r];
+                    lt += __shfl_xor_sync(0xffffffffu, lt, 1);
+                    lt += __shfl_xor_sync(0xffffffffu, lt, 2);
+                    const int h = 16 * mb + g + 8 * r;
                     if (h < p.Hg) {
-                        const int off = 4 * (32 * (col >> 3) + 4 * (row & 7) + ((col & 7) >> 1)) + 2 * (row >> 3) + (col & 1);
-                        const float v = sm.ubuf[0][0][off] + sm.ubuf[1][0][off] + sm.ubuf[2][0][off] + sm.ubuf[3][0][off];
-                        dst[(size_t)h * kVisPart + 2 + col] = v;
+                        float *row = dst + (size_t)h * kVisPart;
+                        if (tig == 0) *reinterpret_cast<float2 *>(row) = make_float2(m[mb][r], lt);
+                        #pragma unroll
+                        for (int nt = 0; nt < 8; ++nt)
+                            *reinterpret_cast<float2 *>(row + 2 + 8 * nt + 2 * tig) =
+                                make_float2(u[mb][nt][2 * r], u[mb][nt][2 * r + 1]);
                     }
                 }
-            }
-            if (tid < p.Hg) {
-                dst[(size_t)tid * kVisPart] = sm.mcta[tid];
-                dst[(size_t)tid * kVisPart + 1] = sm.lcta[tid];
-            }
         }
-        if (prefetch) { sm.upf[tid][0] = pf0; sm.upf[tid][1] = pf1; }
-        if (p.mass == nullptr) continue;
-        if (p.S == 1) {
-            mass_warp(K, 0);
-            continue;
-        }
-        // several splits: the last one to publish fixes the unit's (max, 1/sum).  Only warp 0
-        // takes the arrival count (lanes over splits); the other warps go on to the mass.
-        __syncthreads();
-        if (warp == 0) {
-            unsigned int old = 0;
-            if (lane == 0) {
-                __threadfence();
-                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&p.arrive[unit]) : "memory");
-            }
-            old = __shfl_sync(0xffffffffu, old, 0);
-            if (old == (unsigned int)(p.S - 1)) {
-                // lanes over the splits, four heads at a time with all their loads in flight
-                const float *vu = p.part + (size_t)unit * p.S * p.Hg * kVisPart;
-                for (int h0 = 0; h0 < p.Hg; h0 += 4) {
-                    float ml[4][4], ll[4][4];
-                    #pragma unroll
-                    for (int hh = 0; hh < 4; ++hh)
-                        #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const int sp = lane + 32 * k;
-                            const float *r2 = vu + ((size_t)sp * p.Hg + h0 + hh) * kVisPart;
-                            ml[hh][k] = sp < p.S ? __ldcg(r2) : kRefInit;
-                            ll[hh][k] = sp < p.S ? __ldcg(r2 + 1) : 0.f;
-                        }
-                    #pragma unroll
-                    for (int hh = 0; hh < 4; ++hh) {
-                        const int h = h0 + hh;
-                        float mx = sm.tcur[h][0];
-                        #pragma unroll
-                        for (int k = 0; k < 4; ++k) mx = fmaxf(mx, ml[hh][k]);
-                        for (int sp = lane + 128; sp < p.S; sp += 32)
-                            mx = fmaxf(mx, __ldcg(vu + ((size_t)sp * p.Hg + h) * kVisPart));
-                        #pragma unroll
-                        for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
-                        float sum = 0.f;
-                        #pragma unroll
-                        for (int k = 0; k < 4; ++k) sum += ll[hh][k] * ex2(ml[hh][k] - mx);
-                        for (int sp = lane + 128; sp < p.S; sp += 32) {
-                            const float *r2 = vu + ((size_t)sp * p.Hg + h) * kVisPart;
-                            sum += __ldcg(r2 + 1) * ex2(__ldcg(r2) - mx);
-                        }
-                        #pragma unroll
-                        for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
-                        if (lane == 0) {
-                            if (sm.tcur[h][0] != -INFINITY) sum += sm.tcur[h][1] * ex2(sm.tcur[h][0] - mx);
-                            float *us = p.ustat + ((size_t)unit * p.Hg + h) * 2;
-                            const float inv = 1.f / sum;
-                            asm volatile("st.relaxed.gpu.global.v2.f32 [%0], {%1, %2};" :: "l"(us), "f"(mx), "f"(inv) : "memory");
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-        }
-        if (K >= 1) mass_warp(K - 1, 2);
     }
-    if (p.mass != nullptr && p.S > 1 && K >= 1 && !*abort) mass_warp(K - 1, 1);
-
+    if (!ok) *abort = 1;
     // copies still in flight (only after an abort) must land before the block exits
     while (c_seq < i_seq) {
         const int slot = c_seq % kSlots;
@@ -1201,13 +792,11 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
         while (!mbar_try_wait(&sm.full[warp][slot], par) && clock64() - t0 < kWaitCycles) {}
         ++c_seq;
     }
-    cp_async_wait_all();
-    tmem_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tmem_fence_after();
-        tmem_dealloc(sm.tmem_base, C::kTmemCols);
+    if (iK > cK) {   // a q~ copy the consumer never waited for
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&sm.qbar[warp], (uint32_t)(iK & 1)) && clock64() - t0 < kWaitCycles) {}
     }
+    cp_async_wait_all();
 }
 
 }  // namespace vis

@@ -50,32 +50,28 @@ constexpr int kTextChunk = 64;
 
 struct DecodePlan {
     int nmb, S, tps, units, Hg, Sc_max;
-    size_t off_qt, off_tp, off_vp, off_ustat, off_arrive, off_counter, total;
+    size_t off_qt, off_tp, off_vp, off_ustat, off_counter, total;
 };
 
-// Visual splits: at most Cfg<NMB>::kItemTok tokens each, 32-aligned, and of
-// equal size where a few more splits make them so.
 DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
     DecodePlan pl{};
     pl.Hg = hg(d);
     pl.nmb = (pl.Hg <= 16) ? 1 : 2;
-    const int item_max = (pl.nmb == 1) ? kvpack::decode::vis::Cfg<1>::kItemTok : kvpack::decode::vis::Cfg<2>::kItemTok;
-    const int T = d->T_vis;
-    const int s0 = (T + item_max - 1) / item_max;
-    long long best_waste = -1;
-    for (int S = s0; S <= s0 + 8; ++S) {
-        int tps = (T + S - 1) / S;
-        tps = (tps + 31) & ~31;
-        if (tps > item_max) continue;
-        const int Se = (T + tps - 1) / tps;
-        const long long waste = (long long)Se * tps - T;
-        if (best_waste < 0 || waste < best_waste) {
-            best_waste = waste;
-            pl.S = Se;
-            pl.tps = tps;
-        }
-    }
     pl.units = n_units(d, n_layers);
+    // Visual items (unit, chunk of tps tokens) for warps that fetch work from a counter:
+    // about six per warp of a full B200 (148 SMs x 16 or 8 warps), so the last round is
+    // short; chunks are whole 64-token sub-chunks, between 256 and 2048 tokens, and a
+    // unit's chunks are as even as the 64-token grain allows.  The plan depends on the
+    // shapes alone, so the workspace size does too.
+    const int T = d->T_vis;
+    const long long warps = (pl.nmb == 1) ? 148LL * 16 : 148LL * 8;
+    long long tgt = ((long long)pl.units * T) / (6 * warps);
+    tgt = (tgt + 63) / 64 * 64;
+    if (tgt < 256) tgt = 256;
+    if (tgt > 2048) tgt = 2048;
+    const int S0 = (int)((T + tgt - 1) / tgt);
+    pl.tps = ((T + S0 - 1) / S0 + 63) / 64 * 64;
+    pl.S = (T + pl.tps - 1) / pl.tps;
     pl.Sc_max = (d->L_text_cap + kTextChunk - 1) / kTextChunk;
     size_t off = 0;
     pl.off_qt = off;
@@ -86,10 +82,8 @@ DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
     off = align256(off + (size_t)pl.units * pl.S * pl.Hg * kvpack::decode::kVisPart * sizeof(float));
     pl.off_ustat = off;
     off = align256(off + (size_t)pl.units * pl.Hg * 2 * sizeof(float));
-    pl.off_arrive = off;
-    off += (size_t)pl.units * sizeof(unsigned int);
-    pl.off_counter = off;
-    off = align256(off + sizeof(unsigned int));
+    pl.off_counter = off;   // work counters: [0] text kernel, [1] visual kernel
+    off = align256(off + 4 * sizeof(unsigned int));
     pl.total = off;
     return pl;
 }
@@ -117,7 +111,7 @@ kvpack_status device_info(DeviceInfo **out) {
             cudaFuncSetAttribute(dc::text::text_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)dc::text::smem_bytes()) != cudaSuccess ||
             cudaFuncSetAttribute(dc::finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)dc::finish_smem_bytes(kMaxT / 512 + 8, (KVPACK_MAX_TEXT + kTextChunk - 1) / kTextChunk)) != cudaSuccess)
+                                 (int)dc::finish_smem_bytes((kMaxT + 255) / 256, (KVPACK_MAX_TEXT + kTextChunk - 1) / kTextChunk)) != cudaSuccess)
             return KVPACK_ERR_CUDA;
         // all of the SM's shared memory for these kernels (two visual blocks of the 16-row variant)
         if (cudaFuncSetAttribute(dc::vis::vis_kernel<1>, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
@@ -144,11 +138,8 @@ kvpack_status device_info(DeviceInfo **out) {
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bt, dc::text::text_kernel, dc::text::kThreads,
                                                           dc::text::smem_bytes()) != cudaSuccess)
             return KVPACK_ERR_CUDA;
-        // The occupancy calculator counts a kernel that allocates tensor memory as one block per
-        // SM; the 16-row visual kernel is sized for two (124 registers x 256 threads, 88 KB of
-        // shared memory and 256 of the SM's 512 tensor-memory columns each), and B200s run two
-        // such blocks side by side.  Its grid is therefore sized from Cfg::kBlocks.
-        if (b1 < 1 || b2 != dc::vis::Cfg<2>::kBlocks || bt < 1) return KVPACK_ERR_CUDA;
+        // the visual kernels are sized for Cfg::kBlocks resident blocks per SM
+        if (b1 != dc::vis::Cfg<1>::kBlocks || b2 != dc::vis::Cfg<2>::kBlocks || bt < 1) return KVPACK_ERR_CUDA;
         kvpack_status cs = kvpack::compress::prepare_device();
         if (cs != KVPACK_OK) return cs;
         di.ready = true;
@@ -291,14 +282,11 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     float *tpart = reinterpret_cast<float *>(w + pl.off_tp);
     float *vpart = reinterpret_cast<float *>(w + pl.off_vp);
     float *ustat = reinterpret_cast<float *>(w + pl.off_ustat);
-    unsigned int *arrive = reinterpret_cast<unsigned int *>(w + pl.off_arrive);
     unsigned int *counter = reinterpret_cast<unsigned int *>(w + pl.off_counter);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    // arrival counters and the text work counter start at zero; the unit statistics
-    // that several splits wait for start as NaN (all-ones bytes)
-    if (cudaMemsetAsync(arrive, 0, pl.off_counter + sizeof(unsigned int) - pl.off_arrive, st) != cudaSuccess)
-        return KVPACK_ERR_CUDA;
+    // the work counters start at zero
+    if (cudaMemsetAsync(counter, 0, 4 * sizeof(unsigned int), st) != cudaSuccess) return KVPACK_ERR_CUDA;
 
     // 1. q~ per (unit, KV head) and the text tail partials, one persistent launch
     {
@@ -343,22 +331,16 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
             !encode_bf16(enc, &vp.tm_cv, CV_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return KVPACK_ERR_CUDA;
         vp.CK_lo = CK_lo; vp.CK_hi = CK_hi; vp.CV_lo = CV_lo; vp.CV_hi = CV_hi;
-        vp.qt = qt; vp.mask = mask; vp.mass = nullptr; vp.part = vpart; vp.ustat = ustat; vp.arrive = arrive;
+        vp.qt = qt; vp.mask = mask; vp.part = vpart; vp.counter = counter + 1;
         vp.n_units = pl.units; vp.T = T; vp.Hg = Hg; vp.S = pl.S; vp.tps = pl.tps; vp.nwords = (T + 31) / 32;
         vp.n_items = pl.units * pl.S;
         const int resident = di->sms * (pl.nmb == 1 ? dc::vis::Cfg<1>::kBlocks : dc::vis::Cfg<2>::kBlocks);
-        int grid = vp.n_items < resident ? vp.n_items : resident;
-        if (pl.S > grid) return KVPACK_ERR_UNSUPPORTED;   // every split of a unit must be co-resident
-        // a whole number of units per round (items b, b + grid, ...): no unit's splits straddle
-        // two rounds, so they finish together -- unless that idles more than a fifth of the blocks
-        if (pl.S > 1 && grid == resident && (resident / pl.S) * pl.S * 5 >= resident * 4) grid = (resident / pl.S) * pl.S;
+        const int need = (vp.n_items + dc::vis::kWarps - 1) / dc::vis::kWarps;
+        const int grid = need < resident ? need : resident;
         void *args[] = {&vp};
         const void *fn = (pl.nmb == 1) ? (const void *)dc::vis::vis_kernel<1> : (const void *)dc::vis::vis_kernel<2>;
         const size_t smem = (pl.nmb == 1) ? dc::vis::smem_bytes<1>() : dc::vis::smem_bytes<2>();
-        // Splits of a unit wait (boundedly) for one another: the grid never exceeds what is
-        // resident at once.  The 32-row variant asks for that guarantee with a cooperative launch.
-        cudaError_t e;
-        e = cudaLaunchKernel(fn, dim3(grid), dim3(dc::vis::kThreads), args, smem, st);
+        const cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(dc::vis::kThreads), args, smem, st);
         if (e != cudaSuccess) return KVPACK_ERR_CUDA;
     }
 
