@@ -74,7 +74,7 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback (profiling recipe)"
 
 
-DECODE_SOURCES = ("decode.cuh", "common.cuh", "kvpack.cu")
+DECODE_SOURCES = ("decode.cuh", "mass.cuh", "common.cuh", "kvpack.cu")
 
 
 def sources_digest(names=DECODE_SOURCES) -> str:
@@ -317,7 +317,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
         "step_bytes": int(sbytes),
         "step_GBps": round(sbytes / (ms_step / 1e3) / 1e9, 1),
         "roofline": {"bound": "hbm",
-                     "kernel": "kvpack_decode_attn (text_kernel, qproj_*_kernel, vis_kernel, finish_kernel on one stream)",
+                     "kernel": "kvpack_decode_attn (text_kernel, text_stats_kernel, vis_kernel, finish_kernel, mass_kernel on one stream)",
                      "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4), "frac_of_8TBps": round(achieved / 8000.0, 4),
                      "peak_kind": peak_kind,
@@ -325,7 +325,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
                      "traffic": recorded_traffic("decode", w.name)},
         "e2e": {"value": round(e2e_value, 1), "unit": "query-tokens/s", "h2d_bytes_per_step": qbytes,
                 "d2h_bytes_per_step": obytes, "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": (5 if L0 > 0 else 4) * K,   # per step: select + text + q~ projection + visual + finish
+        "gpu_launches": 6 * K,   # per step: select, text (q~ projection + text tail), text statistics, visual, finish, mass
         "clocks": clk,
         "wall_s_timed": round(wall, 3),
     }

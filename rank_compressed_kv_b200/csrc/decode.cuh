@@ -348,7 +348,6 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSub = 64;        // tokens per sub-chunk: one LO stage
 constexpr int kSubMeta = 8;     // sub-chunk metadata ring per warp (at most kSlots sub-chunks are in flight)
-constexpr int kItemQ = 4;       // fetched-item ring per warp
 
 // Geometry per head-block count.  Up to 16 query heads per unit: two blocks per
 // SM.  Up to 32: one block per SM with a deeper ring.
@@ -358,6 +357,7 @@ struct Cfg {
     static constexpr int kBlocks = (NMB == 1) ? 2 : 1;          // resident blocks per SM
     static constexpr int kSlots = (NMB == 1) ? 2 : 4;           // ring slots per warp
     static constexpr int kSlotBytes = 4096;                     // K rows in the first half, V in the second
+    static constexpr int kQStages = NMB;                        // ring stages of an item's q~ (hi, lo planes)
     static constexpr int kHiTok = 16;                           // full-rank tokens per HI stage
     static constexpr int kNTH = kHiTok / 8;                     // m16n8 token tiles per HI stage
     static_assert(kHiTok * 128 == kSlotBytes / 2, "HI stage rows fill half a slot");
@@ -378,12 +378,9 @@ template <int NMB>
 struct Smem {
     using C = Cfg<NMB>;
     alignas(1024) unsigned char ring[kWarps][C::kSlots][C::kSlotBytes];
-    alignas(128) uint16_t qt[kWarps][2][C::kRows][64];       // per warp: the next item's q~ hi / lo
     uint8_t hi_list[kWarps][kSubMeta][kSub];                 // sub-chunk-relative positions of full-rank tokens
-    int meta[kWarps][kSubMeta][8];                           // K, unit, t0, n, n_hi, w0, w1, flags
-    int itemq[kWarps][kItemQ];
+    int meta[kWarps][kSubMeta][8];                           // item, unit, t0, n, n_hi, w0, w1, flags
     uint64_t full[kWarps][C::kSlots];
-    uint64_t qbar[kWarps];
     int abort;
 };
 
@@ -449,8 +446,9 @@ __device__ __forceinline__ void lazy_update(float (&s)[NT][4], float (&m)[2], fl
 //   values  u += P C_V    (rank 16 over the LO tokens, rank 64 for HI tokens;
 //                          a token with its mask bit set gets logit -inf in LO)
 // At the item's end the warp writes the partial (max, sum, u) of each head.
-// The unit's q~ block comes into one of two per-warp buffers by bulk copy
-// when the issue side begins an item.
+// The unit's q~ (hi and lo planes) travels through the same ring: an item's
+// first sub-chunk begins with kQStages bulk-copied stages that the consumer
+// takes into registers.
 template <int NMB>
 __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const __grid_constant__ Params p) {
     using C = Cfg<NMB>;
@@ -463,23 +461,17 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
     volatile int *abort = &sm.abort;
 
     if (tid == 0) {
-        for (int w = 0; w < kWarps; ++w) {
+        for (int w = 0; w < kWarps; ++w)
             for (int s = 0; s < kSlots; ++s) mbar_init(&sm.full[w][s], 32);
-            mbar_init(&sm.qbar[w], 1);
-        }
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // query rows past Hg stay zero
-    for (int i = tid; i < kWarps * 2 * C::kRows * 64 / 8; i += kThreads)
-        reinterpret_cast<uint4 *>(&sm.qt[0][0][0][0])[i] = make_uint4(0u, 0u, 0u, 0u);
     __syncthreads();
 
     // ------------------------------------------------------------ issue side
-    int iK = -1, i_item = 0, i_sc = 0, i_nsc = 0, i_st = 0, i_nst = 0;
+    int i_item = -1, i_sc = 0, i_nsc = 0, i_st = 0, i_nst = 0, i_nq = 0;
     uint32_t i_seq = 0, c_seq = 0, i_sub = 0, c_sub = 0;
     bool i_done = false;
-    int cK = -1;   // item the consumer is on
     auto fetch = [&]() -> int {
         int v = 0;
         if (lane == 0) v = (int)atomicAdd(p.counter, 1u);
@@ -503,34 +495,21 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
         if ((w1 >> lane) & 1u) sm.hi_list[warp][ms][c0 + __popc(w1 & below)] = (uint8_t)(32 + lane);
         if (lane == 0) {
             int *m = sm.meta[warp][ms];
-            m[0] = iK; m[1] = unit; m[2] = t0; m[3] = n; m[4] = n_hi; m[5] = (int)w0; m[6] = (int)w1;
+            m[0] = i_item; m[1] = unit; m[2] = t0; m[3] = n; m[4] = n_hi; m[5] = (int)w0; m[6] = (int)w1;
             m[7] = (i_sc == 0 ? 1 : 0) | (i_sc + 1 == i_nsc ? 2 : 0);
         }
         __syncwarp();
-        i_nst = (n_hi < n ? 1 : 0) + (n_hi + kHiTok - 1) / kHiTok;
+        i_nq = i_sc == 0 ? C::kQStages : 0;
+        i_nst = i_nq + (n_hi < n ? 1 : 0) + (n_hi + kHiTok - 1) / kHiTok;
         i_st = 0;
     };
-    // the next item: its q~ block into the warp's staging buffer (free once the consumer
-    // has taken the current item's q~ into registers)
     auto begin_item = [&]() -> bool {
         const int it = fetch();
         if (it >= p.n_items) return false;
-        ++iK;
         i_item = it;
-        if (lane == 0) sm.itemq[warp][iK % kItemQ] = it;
         const int t0 = (it % p.S) * p.tps;
         i_nsc = (min(p.tps, p.T - t0) + kSub - 1) / kSub;
         i_sc = 0;
-        if (lane == 0) {
-            const unsigned char *src = p.qt + (size_t)(it / p.S) * qblock_bytes(p.Hg);
-            const uint32_t bytes = (uint32_t)p.Hg * 128u;
-            uint64_t *qb = &sm.qbar[warp];
-            fence_proxy_async();
-            mbar_arrive_tx(qb, 2 * bytes);
-            bulk_g2s(&sm.qt[warp][0][0][0], src, bytes, qb);
-            bulk_g2s(&sm.qt[warp][1][0][0], src + bytes, bytes, qb);
-        }
-        __syncwarp();
         return true;
     };
     auto issue_stage = [&]() {
@@ -541,7 +520,25 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
         unsigned char *dst = sm.ring[warp][slot];
         uint64_t *bar = &sm.full[warp][slot];
         __syncwarp();
-        if (i_st == 0 && n_hi < n) {
+        if (i_st < i_nq) {
+            // q~ of the unit: the hi plane (NMB == 1: then the lo plane in the slot's second half),
+            // Hg rows of 128 bytes; the consumer zeroes the rows past Hg in registers
+            if (lane == 0) {
+                const unsigned char *src = p.qt + (size_t)unit * qblock_bytes(p.Hg);
+                const uint32_t bytes = (uint32_t)p.Hg * 128u;
+                fence_proxy_async();
+                if (C::kQStages == 1) {
+                    mbar_arrive_tx(bar, 2 * bytes);
+                    bulk_g2s(dst, src, bytes, bar);
+                    bulk_g2s(dst + kHalf, src + bytes, bytes, bar);
+                } else {
+                    mbar_arrive_tx(bar, bytes);
+                    bulk_g2s(dst, src + (size_t)i_st * bytes, bytes, bar);
+                }
+            } else {
+                mbar_arrive(bar);
+            }
+        } else if (i_st == i_nq && n_hi < n) {
             // all 64 rows of K and V: the value MMA reads every row (masked rows get p = 0,
             // which must meet finite data -- neighbouring rows, or zeros past the unit's end)
             if (lane == 0) {
@@ -557,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
         } else {
             // kHiTok full-rank tokens: C_lo + C_hi rows of K and V gathered into 128-byte rows
             // (16-byte chunk c of row r stored at c ^ (r & 7)); rows past the count are zero
-            const int hs = i_st - (n_hi < n ? 1 : 0);
+            const int hs = i_st - i_nq - (n_hi < n ? 1 : 0);
             const int cnt = min(kHiTok, n_hi - kHiTok * hs);
             const size_t ubase = (size_t)unit * p.T + t0;
             #pragma unroll
@@ -587,16 +584,14 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
         if (i_st == i_nst) ++i_sub;
         ++i_seq;
     };
-    // issue while the ring has room; the issue side may begin item cK + 1 at most
-    // (its q~ overwrites the staging buffer, which the consumer emptied when it began item cK)
+    // issue while the ring has room and the metadata ring has a free entry
     auto pump = [&]() {
         while (!i_done && i_seq - c_seq < (uint32_t)kSlots) {
             if (i_st == i_nst) {
                 if (i_sub - c_sub >= (uint32_t)kSubMeta) return;
-                if (iK >= 0 && i_sc + 1 < i_nsc) {
+                if (i_item >= 0 && i_sc + 1 < i_nsc) {
                     ++i_sc;
                 } else {
-                    if (iK + 1 > cK + 1) return;
                     if (!begin_item()) { i_done = true; return; }
                 }
                 begin_sub();
@@ -709,41 +704,55 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
         }
     };
 
+    // a q~ plane (kRows rows of 128 bytes, chunk c of row r at c ^ (r & 7)) into A fragments;
+    // rows past Hg hold stale bytes and are zeroed here
+    auto load_plane = [&](uint32_t base, uint32_t (&q)[NMB][4][4]) {
+        #pragma unroll
+        for (int mb = 0; mb < NMB; ++mb) {
+            const int row = 16 * mb + (lane & 7) + (((lane >> 3) & 1) << 3);
+            const bool z0 = 16 * mb + g >= p.Hg, z1 = 16 * mb + g + 8 >= p.Hg;
+            #pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+                const int ch = 2 * kb + (lane >> 4);
+                ldsm_x4(base + row * 128 + ((ch ^ (row & 7)) << 4), q[mb][kb][0], q[mb][kb][1], q[mb][kb][2], q[mb][kb][3]);
+                if (z0) q[mb][kb][0] = q[mb][kb][2] = 0u;
+                if (z1) q[mb][kb][1] = q[mb][kb][3] = 0u;
+            }
+        }
+    };
+
     while (ok) {
         pump();
         if (c_sub == i_sub && c_seq == i_seq) break;   // nothing issued and nothing left to issue
         const int ms = c_sub % kSubMeta;
         const int *mt = sm.meta[warp][ms];
-        const int K = mt[0], n = mt[3], n_hi = mt[4], flags = mt[7];
+        const int item = mt[0], n = mt[3], n_hi = mt[4], flags = mt[7];
         const uint32_t w0 = (uint32_t)mt[5], w1 = (uint32_t)mt[6];
-        if (flags & 1) {
-            // first sub-chunk of item K: its q~ block, fresh softmax state
-            if (!mbar_wait(&sm.qbar[warp], (uint32_t)(K & 1), abort)) { ok = false; break; }
-            const uint32_t qt0 = smem_u32(&sm.qt[warp][0][0][0]), qt1 = smem_u32(&sm.qt[warp][1][0][0]);
-            #pragma unroll
-            for (int mb = 0; mb < NMB; ++mb) {
-                const int row = 16 * mb + (lane & 7) + (((lane >> 3) & 1) << 3);
-                #pragma unroll
-                for (int kb = 0; kb < 4; ++kb) {
-                    const int ch = 2 * kb + (lane >> 4);
-                    const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
-                    ldsm_x4(qt0 + off, qh[mb][kb][0], qh[mb][kb][1], qh[mb][kb][2], qh[mb][kb][3]);
-                    ldsm_x4(qt1 + off, ql[mb][kb][0], ql[mb][kb][1], ql[mb][kb][2], ql[mb][kb][3]);
-                }
-                m[mb][0] = m[mb][1] = kRefInit;
-                l[mb][0] = l[mb][1] = 0.f;
-                #pragma unroll
-                for (int a = 0; a < 8; ++a) u[mb][a][0] = u[mb][a][1] = u[mb][a][2] = u[mb][a][3] = 0.f;
-            }
-            __syncwarp();
-            cK = K;   // the staging buffer is free for the next item
-        }
-        const int nst = (n_hi < n ? 1 : 0) + (n_hi + kHiTok - 1) / kHiTok;
+        const int nq = (flags & 1) ? C::kQStages : 0;   // an item's first sub-chunk starts with its q~
+        const int nst = nq + (n_hi < n ? 1 : 0) + (n_hi + kHiTok - 1) / kHiTok;
         for (int st = 0; st < nst; ++st) {
             const int slot = c_seq % kSlots;
             if (!mbar_wait(&sm.full[warp][slot], (c_seq / kSlots) & 1u, abort)) { ok = false; break; }
             const uint32_t sb = smem_u32(sm.ring[warp][slot]);
-            if (st == 0 && n_hi < n) {
+            if (st < nq) {
+                if (st == 0) {   // a new item: fresh softmax state
+                    #pragma unroll
+                    for (int mb = 0; mb < NMB; ++mb) {
+                        m[mb][0] = m[mb][1] = kRefInit;
+                        l[mb][0] = l[mb][1] = 0.f;
+                        #pragma unroll
+                        for (int a = 0; a < 8; ++a) u[mb][a][0] = u[mb][a][1] = u[mb][a][2] = u[mb][a][3] = 0.f;
+                    }
+                }
+                if (C::kQStages == 1) {
+                    load_plane(sb, qh);
+                    load_plane(sb + kHalf, ql);
+                } else if (st == 0) {
+                    load_plane(sb, qh);
+                } else {
+                    load_plane(sb, ql);
+                }
+            } else if (st == nq && n_hi < n) {
                 if (NMB == 1) {   // two 32-token halves: fewer live scores
                     do_lo(sb, w0, 0u, n, std::integral_constant<int, 4>{});
                     if (n > 32) do_lo(sb + 1024, w1, 0u, n - 32, std::integral_constant<int, 4>{});
@@ -751,7 +760,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
                     do_lo(sb, w0, w1, n, std::integral_constant<int, 8>{});
                 }
             } else {
-                const int hs = st - (n_hi < n ? 1 : 0);
+                const int hs = st - nq - (n_hi < n ? 1 : 0);
                 do_hi(sb, min(kHiTok, n_hi - kHiTok * hs));
             }
             ++c_seq;
@@ -761,8 +770,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
         if (!ok) break;
         ++c_sub;
         if (flags & 2) {
-            // last sub-chunk: the partial of item K -- per head row: max, sum, u[64]
-            const int item = sm.itemq[warp][K % kItemQ];
+            // last sub-chunk: the partial of the item -- per head row: max, sum, u[64]
             float *dst = p.part + (size_t)item * p.Hg * kVisPart;
             #pragma unroll
             for (int mb = 0; mb < NMB; ++mb)
@@ -791,10 +799,6 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
         const long long t0 = clock64();
         while (!mbar_try_wait(&sm.full[warp][slot], par) && clock64() - t0 < kWaitCycles) {}
         ++c_seq;
-    }
-    if (iK > cK) {   // a q~ copy the consumer never waited for
-        const long long t0 = clock64();
-        while (!mbar_try_wait(&sm.qbar[warp], (uint32_t)(iK & 1)) && clock64() - t0 < kWaitCycles) {}
     }
     cp_async_wait_all();
 }
