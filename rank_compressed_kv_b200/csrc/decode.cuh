@@ -816,25 +816,27 @@ struct FinishParams {
     int Hg, per_kv, n_q, groups, S, Sc;
 };
 
-// dynamic shared memory of finish_kernel: weights of every partial, then u / l and w / l
-__host__ __device__ constexpr size_t finish_smem_bytes(int S, int Sc) {
-    return (size_t)(S + Sc) * kMaxHeads * sizeof(float) + (size_t)kMaxHeads * (64 + 128) * sizeof(float);
+// dynamic shared memory of finish_kernel: the weight of every partial, then u / l and w / l
+__host__ __device__ constexpr size_t finish_smem_bytes(int S, int Sc, int Hg) {
+    return ((size_t)(S + Sc) * Hg + (size_t)Hg * (64 + 128)) * sizeof(float);
 }
+constexpr size_t kFinishSmemMax = 200 * 1024;
 
-// One block per unit.  Per head, the unit-wide max M and sum L over every
-// visual and text partial give each partial the weight 2^(m - M) / L; u / l and
-// w / l are weighted sums with the feature index across threads (coalesced).
-// Then o_h = (u_h / l_h) B_V[:, 128 j(h) ..] + w_h / l_h, thread t owning output
+// One block per unit.  Per head, the unit-wide max M and sum L over every visual and text
+// partial give each partial the weight 2^(m - M) / L; u / l and w / l are
+// weighted sums with the feature index across threads (coalesced).  Then
+// o_h = (u_h / l_h) B_V[:, 128 j(h) ..] + w_h / l_h, thread t owning output
 // columns 2t, 2t+1 of the unit's 512 (KV head t / 64).
 __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
     extern __shared__ float fsm[];
-    float *wv = fsm;                                  // [S][kMaxHeads]
-    float *wt = wv + p.S * kMaxHeads;                 // [Sc][kMaxHeads]
-    float (*uf)[64] = reinterpret_cast<float (*)[64]>(wt + p.Sc * kMaxHeads);
-    float (*wf)[128] = reinterpret_cast<float (*)[128]>(&uf[kMaxHeads][0]);
+    float *wv = fsm;                              // [S][Hg]
+    float *wt = wv + (size_t)p.S * p.Hg;          // [Sc][Hg]
+    float *uf = wt + (size_t)p.Sc * p.Hg;         // [Hg][64]
+    float *wf = uf + (size_t)p.Hg * 64;           // [Hg][128]
     const int unit = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const float *vp0 = p.vpart + (size_t)unit * p.S * p.Hg * kVisPart;
     const float *tp0 = p.tpart + (size_t)unit * p.Sc * p.Hg * kTxtPart;
+    const uint16_t *bvg = p.BV + (size_t)unit * 64 * 512;
 
     for (int h = warp; h < p.Hg; h += 8) {
         float mx = -INFINITY;
@@ -846,14 +848,14 @@ __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
         for (int s = lane; s < p.S; s += 32) {
             const float *r = vp0 + ((size_t)s * p.Hg + h) * kVisPart;
             const float e = ex2(__ldcg(r) - mx);
-            wv[s * kMaxHeads + h] = e;
+            wv[s * p.Hg + h] = e;
             sum += __ldcg(r + 1) * e;
         }
         for (int c = lane; c < p.Sc; c += 32) {
             const float *r = tp0 + ((size_t)c * p.Hg + h) * kTxtPart;
             const float m = __ldcg(r);
             const float e = (m != -INFINITY) ? ex2(m - mx) : 0.f;
-            wt[c * kMaxHeads + h] = e;
+            wt[c * p.Hg + h] = e;
             sum += (m != -INFINITY) ? __ldcg(r + 1) * e : 0.f;
         }
         #pragma unroll
@@ -862,8 +864,8 @@ __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
         if (lane == 0 && p.ustat != nullptr)
             *reinterpret_cast<float2 *>(p.ustat + ((size_t)unit * p.Hg + h) * 2) = make_float2(mx, inv);
         __syncwarp();
-        for (int s = lane; s < p.S; s += 32) wv[s * kMaxHeads + h] *= inv;
-        for (int c = lane; c < p.Sc; c += 32) wt[c * kMaxHeads + h] *= inv;
+        for (int s = lane; s < p.S; s += 32) wv[s * p.Hg + h] *= inv;
+        for (int c = lane; c < p.Sc; c += 32) wt[c * p.Hg + h] *= inv;
     }
     __syncthreads();
     for (int task = tid; task < p.Hg * 64; task += 256) {
@@ -872,11 +874,11 @@ __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
         float a0 = 0.f, a1 = 0.f;
         int s = 0;
         for (; s + 2 <= p.S; s += 2) {
-            a0 = fmaf(__ldcg(r + (size_t)s * p.Hg * kVisPart), wv[s * kMaxHeads + h], a0);
-            a1 = fmaf(__ldcg(r + (size_t)(s + 1) * p.Hg * kVisPart), wv[(s + 1) * kMaxHeads + h], a1);
+            a0 = fmaf(__ldcg(r + (size_t)s * p.Hg * kVisPart), wv[s * p.Hg + h], a0);
+            a1 = fmaf(__ldcg(r + (size_t)(s + 1) * p.Hg * kVisPart), wv[(s + 1) * p.Hg + h], a1);
         }
-        if (s < p.S) a0 = fmaf(__ldcg(r + (size_t)s * p.Hg * kVisPart), wv[s * kMaxHeads + h], a0);
-        uf[h][f] = a0 + a1;
+        if (s < p.S) a0 = fmaf(__ldcg(r + (size_t)s * p.Hg * kVisPart), wv[s * p.Hg + h], a0);
+        uf[h * 64 + f] = a0 + a1;
     }
     for (int task = tid; task < p.Hg * 128; task += 256) {
         const int h = task >> 7, f = task & 127;
@@ -884,16 +886,16 @@ __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
         float a0 = 0.f, a1 = 0.f;
         int c = 0;
         for (; c + 2 <= p.Sc; c += 2) {
-            a0 = fmaf(__ldcg(r + (size_t)c * p.Hg * kTxtPart), wt[c * kMaxHeads + h], a0);
-            a1 = fmaf(__ldcg(r + (size_t)(c + 1) * p.Hg * kTxtPart), wt[(c + 1) * kMaxHeads + h], a1);
+            a0 = fmaf(__ldcg(r + (size_t)c * p.Hg * kTxtPart), wt[c * p.Hg + h], a0);
+            a1 = fmaf(__ldcg(r + (size_t)(c + 1) * p.Hg * kTxtPart), wt[(c + 1) * p.Hg + h], a1);
         }
-        if (c < p.Sc) a0 = fmaf(__ldcg(r + (size_t)c * p.Hg * kTxtPart), wt[c * kMaxHeads + h], a0);
-        wf[h][f] = a0 + a1;
+        if (c < p.Sc) a0 = fmaf(__ldcg(r + (size_t)c * p.Hg * kTxtPart), wt[c * p.Hg + h], a0);
+        wf[h * 128 + f] = a0 + a1;
     }
     __syncthreads();
     const int j = tid >> 6, d = (2 * tid) & 127;
     const int lb = unit / p.groups, G = unit % p.groups;
-    const uint32_t *bv = reinterpret_cast<const uint32_t *>(p.BV + (size_t)unit * 64 * 512) + tid;
+    const uint32_t *bv = reinterpret_cast<const uint32_t *>(bvg) + tid;
     float acc[8][2];
     #pragma unroll
     for (int hh = 0; hh < 8; ++hh) acc[hh][0] = acc[hh][1] = 0.f;
@@ -909,7 +911,7 @@ __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
             #pragma unroll
             for (int hh = 0; hh < 8; ++hh) {
                 if (hh < p.per_kv) {
-                    const float x = uf[h0 + hh][i0 + i];
+                    const float x = uf[(h0 + hh) * 64 + i0 + i];
                     acc[hh][0] = fmaf(x, b0, acc[hh][0]);
                     acc[hh][1] = fmaf(x, b1, acc[hh][1]);
                 }
@@ -921,17 +923,11 @@ __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
         if (hh < p.per_kv) {
             const int h = h0 + hh;
             *reinterpret_cast<uint32_t *>(p.out + ((size_t)lb * p.n_q + (size_t)G * p.Hg + h) * 128 + d) =
-                pack_bf16(acc[hh][0] + wf[h][d], acc[hh][1] + wf[h][d + 1]);
+                pack_bf16(acc[hh][0] + wf[h * 128 + d], acc[hh][1] + wf[h * 128 + d + 1]);
         }
     }
 }
 
-}  // namespace decode
-}  // namespace kvpack
-
-namespace kvpack {
-namespace decode {
-// one block per SM: the opt-in shared-memory limit per block on sm_100 is 232448 bytes
 static_assert(2 * (vis::smem_bytes<1>() + 1024) <= 233472, "visual kernel (16 head rows): two blocks per SM");
 static_assert(vis::smem_bytes<2>() <= 232448, "visual kernel (32 head rows) shared memory");
 static_assert(text::smem_bytes() <= 232448, "text kernel shared memory");

@@ -111,7 +111,7 @@ kvpack_status device_info(DeviceInfo **out) {
             cudaFuncSetAttribute(dc::text::text_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)dc::text::smem_bytes()) != cudaSuccess ||
             cudaFuncSetAttribute(dc::finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)dc::finish_smem_bytes((kMaxT + 255) / 256, (KVPACK_MAX_TEXT + kTextChunk - 1) / kTextChunk)) != cudaSuccess)
+                                 (int)dc::kFinishSmemMax) != cudaSuccess)
             return KVPACK_ERR_CUDA;
         // all of the SM's shared memory for these kernels (two visual blocks of the 16-row variant)
         if (cudaFuncSetAttribute(dc::vis::vis_kernel<1>, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
@@ -347,7 +347,7 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     // 4. combine and project through B_V
     dc::FinishParams fp{BV, vpart, Sc > 0 ? tpart : nullptr, out, mass != nullptr ? ustat : nullptr,
                         Hg, per_kv, d->n_q_heads, groups, pl.S, Sc};
-    dc::finish_kernel<<<pl.units, 256, dc::finish_smem_bytes(pl.S, Sc), st>>>(fp);
+    dc::finish_kernel<<<pl.units, 256, dc::finish_smem_bytes(pl.S, Sc, Hg), st>>>(fp);
     if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
     if (mass == nullptr) return KVPACK_OK;
 
