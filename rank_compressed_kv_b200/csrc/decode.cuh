@@ -347,7 +347,8 @@ namespace vis {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSub = 64;        // tokens per sub-chunk: one LO stage
-constexpr int kSubMeta = 8;     // sub-chunk metadata ring per warp (at most kSlots sub-chunks are in flight)
+constexpr int kMaxItemTok = 2048;               // tokens per item, at most
+constexpr int kMaxItemWords = kMaxItemTok / 32;
 
 // Geometry per head-block count.  Up to 16 query heads per unit: two blocks per
 // SM.  Up to 32: one block per SM with a deeper ring.
@@ -378,8 +379,10 @@ template <int NMB>
 struct Smem {
     using C = Cfg<NMB>;
     alignas(1024) unsigned char ring[kWarps][C::kSlots][C::kSlotBytes];
-    uint8_t hi_list[kWarps][kSubMeta][kSub];                 // sub-chunk-relative positions of full-rank tokens
-    int meta[kWarps][kSubMeta][8];                           // item, unit, t0, n, n_hi, w0, w1, flags
+    uint16_t hi_list[kWarps][kMaxItemTok];                   // item-relative positions of the issue side's item's
+                                                             // full-rank tokens
+    uint32_t mw[kWarps][kMaxItemWords];                      // that item's mask words
+    int desc[kWarps][C::kSlots][6];                          // per ring slot: flags, item, n, w0, w1
     uint64_t full[kWarps][C::kSlots];
     int abort;
 };
@@ -436,19 +439,21 @@ __device__ __forceinline__ void lazy_update(float (&s)[NT][4], float (&m)[2], fl
 }
 
 // Persistent, one or two 256-thread blocks per SM; every warp works alone.
-// A warp fetches items (unit, chunk of tps tokens) from a global counter and
-// streams each through a private ring, 64 tokens (a sub-chunk) at a time: one
-// TMA stage of C_lo rows of K and V (skipped when every token is full-rank)
-// and one gathered stage (C_lo + C_hi rows of K and V, cp.async) per 16
-// full-rank tokens.  With heads on M and tokens on N of mma.sync m16n8k16:
+// A warp fetches items (unit, chunk of tps <= 2048 tokens) from a global
+// counter and streams each through a private ring: the unit's q~, then one
+// TMA stage of C_lo rows of K and V per 64-token sub-chunk (skipped when every
+// token of it is full-rank), then the item's full-rank tokens 16 at a time
+// (C_lo + C_hi rows of K and V gathered by cp.async; the issue side lists
+// them once per item, so only the item's last gathered stage is partial).
+// With heads on M and tokens on N of mma.sync m16n8k16:
 //   scores  s = q~ C_K^T  (q~ as a bf16 hi + lo pair, C_K exact in bf16)
 //   softmax online per head row; P stays in registers as the A operand of
 //   values  u += P C_V    (rank 16 over the LO tokens, rank 64 for HI tokens;
 //                          a token with its mask bit set gets logit -inf in LO)
 // At the item's end the warp writes the partial (max, sum, u) of each head.
-// The unit's q~ (hi and lo planes) travels through the same ring: an item's
-// first sub-chunk begins with kQStages bulk-copied stages that the consumer
-// takes into registers.
+// The unit's q~ (hi and lo planes) travels through the same ring: an item
+// begins with kQStages bulk-copied stages that the consumer takes into
+// registers.  Every ring slot carries a small descriptor of its stage.
 template <int NMB>
 __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const __grid_constant__ Params p) {
     using C = Cfg<NMB>;
@@ -469,62 +474,79 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
     __syncthreads();
 
     // ------------------------------------------------------------ issue side
-    int i_item = -1, i_sc = 0, i_nsc = 0, i_st = 0, i_nst = 0, i_nq = 0;
-    uint32_t i_seq = 0, c_seq = 0, i_sub = 0, c_sub = 0;
+    constexpr int kTypeQ = 0, kTypeLo = 1, kTypeHi = 2, kFirst = 4, kLast = 8;
+    int i_item = -1, i_unit = 0, i_t0 = 0, i_n = 0;   // the item being issued
+    int i_q = 0, i_sub = 0, i_lo = 0, i_hi = 0, i_nhi = 0, i_left = 0;   // i_lo: LO stages still to issue
+    uint32_t i_seq = 0, c_seq = 0;
     bool i_done = false;
     auto fetch = [&]() -> int {
         int v = 0;
         if (lane == 0) v = (int)atomicAdd(p.counter, 1u);
         return __shfl_sync(0xffffffffu, v, 0);
     };
-    // sub-chunk i_sc of the issue side's item into meta slot i_sub % kSubMeta
-    auto begin_sub = [&]() {
-        const int ms = i_sub % kSubMeta;
-        const int unit = i_item / p.S, t0 = (i_item % p.S) * p.tps + kSub * i_sc;
-        const int n = min(kSub, p.T - t0);
-        uint32_t w = 0u;
-        if (lane < 2 && 32 * lane < n) {
-            w = __ldg(p.mask + (size_t)unit * p.nwords + (t0 >> 5) + lane);
-            const int nb = n - 32 * lane;
-            if (nb < 32) w &= (1u << nb) - 1u;
-        }
-        const uint32_t w0 = __shfl_sync(0xffffffffu, w, 0), w1 = __shfl_sync(0xffffffffu, w, 1);
-        const int c0 = __popc(w0), n_hi = c0 + __popc(w1);
-        const uint32_t below = (1u << lane) - 1u;
-        if ((w0 >> lane) & 1u) sm.hi_list[warp][ms][__popc(w0 & below)] = (uint8_t)lane;
-        if ((w1 >> lane) & 1u) sm.hi_list[warp][ms][c0 + __popc(w1 & below)] = (uint8_t)(32 + lane);
-        if (lane == 0) {
-            int *m = sm.meta[warp][ms];
-            m[0] = i_item; m[1] = unit; m[2] = t0; m[3] = n; m[4] = n_hi; m[5] = (int)w0; m[6] = (int)w1;
-            m[7] = (i_sc == 0 ? 1 : 0) | (i_sc + 1 == i_nsc ? 2 : 0);
-        }
-        __syncwarp();
-        i_nq = i_sc == 0 ? C::kQStages : 0;
-        i_nst = i_nq + (n_hi < n ? 1 : 0) + (n_hi + kHiTok - 1) / kHiTok;
-        i_st = 0;
-    };
+    // the next item: its mask words and the list of its full-rank tokens
     auto begin_item = [&]() -> bool {
         const int it = fetch();
         if (it >= p.n_items) return false;
         i_item = it;
-        const int t0 = (it % p.S) * p.tps;
-        i_nsc = (min(p.tps, p.T - t0) + kSub - 1) / kSub;
-        i_sc = 0;
+        i_unit = it / p.S;
+        i_t0 = (it % p.S) * p.tps;
+        i_n = min(p.tps, p.T - i_t0);
+        const int nw = (i_n + 31) >> 5;
+        int base = 0, n_lo_st = 0;
+        for (int w0 = 0; w0 < nw; w0 += 32) {
+            const int wi = w0 + lane;
+            uint32_t w = 0u;
+            if (wi < nw) {
+                w = __ldg(p.mask + (size_t)i_unit * p.nwords + (i_t0 >> 5) + wi);
+                const int nb = i_n - 32 * wi;
+                if (nb < 32) w &= (1u << nb) - 1u;
+                sm.mw[warp][wi] = w;
+            }
+            const int c = __popc(w);
+            int incl = c;
+            #pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += v;
+            }
+            int r = base + incl - c;
+            uint32_t bits = w;
+            while (bits) {
+                sm.hi_list[warp][r++] = (uint16_t)(32 * wi + __ffs(bits) - 1);
+                bits &= bits - 1u;
+            }
+            // sub-chunks (word pairs) with a reduced-rank token need a LO stage
+            const int c_pair = c + __shfl_down_sync(0xffffffffu, c, 1);
+            const int nsub_tok = min(kSub, i_n - 32 * wi);
+            const bool lo_st = (lane & 1) == 0 && wi < nw && c_pair < nsub_tok;
+            n_lo_st += __popc(__ballot_sync(0xffffffffu, lo_st));
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        i_nhi = base;
+        i_hi = 0;
+        i_sub = 0;
+        i_lo = n_lo_st;
+        i_q = 0;
+        i_left = C::kQStages + n_lo_st + (i_nhi + kHiTok - 1) / kHiTok;
+        __syncwarp();
         return true;
     };
+    // issue the item's next stage (the item has one)
     auto issue_stage = [&]() {
-        const int ms = i_sub % kSubMeta;
-        const int *m = sm.meta[warp][ms];
-        const int unit = m[1], t0 = m[2], n = m[3], n_hi = m[4];
         const int slot = i_seq % kSlots;
         unsigned char *dst = sm.ring[warp][slot];
         uint64_t *bar = &sm.full[warp][slot];
+        int type, n = 0;
+        uint32_t w0 = 0u, w1 = 0u;
         __syncwarp();
-        if (i_st < i_nq) {
+        if (i_q < C::kQStages) {
             // q~ of the unit: the hi plane (NMB == 1: then the lo plane in the slot's second half),
             // Hg rows of 128 bytes; the consumer zeroes the rows past Hg in registers
+            type = kTypeQ | (i_q == 0 ? kFirst : 0);
+            n = i_q;
             if (lane == 0) {
-                const unsigned char *src = p.qt + (size_t)unit * qblock_bytes(p.Hg);
+                const unsigned char *src = p.qt + (size_t)i_unit * qblock_bytes(p.Hg);
                 const uint32_t bytes = (uint32_t)p.Hg * 128u;
                 fence_proxy_async();
                 if (C::kQStages == 1) {
@@ -533,30 +555,43 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
                     bulk_g2s(dst + kHalf, src + bytes, bytes, bar);
                 } else {
                     mbar_arrive_tx(bar, bytes);
-                    bulk_g2s(dst, src + (size_t)i_st * bytes, bytes, bar);
+                    bulk_g2s(dst, src + (size_t)i_q * bytes, bytes, bar);
                 }
             } else {
                 mbar_arrive(bar);
             }
-        } else if (i_st == i_nq && n_hi < n) {
-            // all 64 rows of K and V: the value MMA reads every row (masked rows get p = 0,
-            // which must meet finite data -- neighbouring rows, or zeros past the unit's end)
+            ++i_q;
+        } else if (i_lo > 0) {
+            // the next sub-chunk with a reduced-rank token (one exists): all 64 rows of K and V (the value MMA reads
+            // every row; masked rows get p = 0, which must meet finite data -- neighbouring rows, or zeros
+            // past the unit's end)
+            while (true) {
+                n = min(kSub, i_n - kSub * i_sub);
+                w0 = sm.mw[warp][2 * i_sub];
+                w1 = n > 32 ? sm.mw[warp][2 * i_sub + 1] : 0u;
+                if (__popc(w0) + __popc(w1) < n) break;
+                ++i_sub;
+            }
+            type = kTypeLo;
+            const int t0 = i_t0 + kSub * i_sub;
             if (lane == 0) {
                 fence_proxy_async();
                 mbar_arrive_tx(bar, 4u * 1024u);
-                tma_3d(dst, &p.tm_ck, 0, t0, unit, bar);
-                tma_3d(dst + 1024, &p.tm_ck, 0, t0 + 32, unit, bar);
-                tma_3d(dst + kHalf, &p.tm_cv, 0, t0, unit, bar);
-                tma_3d(dst + kHalf + 1024, &p.tm_cv, 0, t0 + 32, unit, bar);
+                tma_3d(dst, &p.tm_ck, 0, t0, i_unit, bar);
+                tma_3d(dst + 1024, &p.tm_ck, 0, t0 + 32, i_unit, bar);
+                tma_3d(dst + kHalf, &p.tm_cv, 0, t0, i_unit, bar);
+                tma_3d(dst + kHalf + 1024, &p.tm_cv, 0, t0 + 32, i_unit, bar);
             } else {
                 mbar_arrive(bar);
             }
+            ++i_sub;
+            --i_lo;
         } else {
             // kHiTok full-rank tokens: C_lo + C_hi rows of K and V gathered into 128-byte rows
             // (16-byte chunk c of row r stored at c ^ (r & 7)); rows past the count are zero
-            const int hs = i_st - i_nq - (n_hi < n ? 1 : 0);
-            const int cnt = min(kHiTok, n_hi - kHiTok * hs);
-            const size_t ubase = (size_t)unit * p.T + t0;
+            type = kTypeHi;
+            n = min(kHiTok, i_nhi - i_hi);
+            const size_t ubase = (size_t)i_unit * p.T + i_t0;
             #pragma unroll
             for (int i = 0; i < kHiTok / 4; ++i) {
                 const int idx = lane + 32 * i;
@@ -564,8 +599,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
                 const int pos = (ch ^ (r & 7)) << 4;
                 unsigned char *dk = dst + r * 128 + pos;
                 unsigned char *dv = dst + kHalf + r * 128 + pos;
-                if (r < cnt) {
-                    const size_t row = ubase + sm.hi_list[warp][ms][kHiTok * hs + r];
+                if (r < n) {
+                    const size_t row = ubase + sm.hi_list[warp][i_hi + r];
                     if (ch < 2) {
                         cp_async16(dk, p.CK_lo + row * 16 + ch * 8);
                         cp_async16(dv, p.CV_lo + row * 16 + ch * 8);
@@ -579,23 +614,23 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
                 }
             }
             cp_async_arrive_noinc(bar);
+            i_hi += n;
         }
-        ++i_st;
-        if (i_st == i_nst) ++i_sub;
+        --i_left;
+        if (i_left == 0) type |= kLast;
+        if (lane == 0) {
+            int *d = sm.desc[warp][slot];
+            d[0] = type; d[1] = i_item; d[2] = n; d[3] = (int)w0; d[4] = (int)w1;
+        }
+        __syncwarp();
         ++i_seq;
     };
-    // issue while the ring has room and the metadata ring has a free entry
+    // issue while the ring has room
     auto pump = [&]() {
         while (!i_done && i_seq - c_seq < (uint32_t)kSlots) {
-            if (i_st == i_nst) {
-                if (i_sub - c_sub >= (uint32_t)kSubMeta) return;
-                if (i_item >= 0 && i_sc + 1 < i_nsc) {
-                    ++i_sc;
-                } else {
-                    if (!begin_item()) { i_done = true; return; }
-                }
-                begin_sub();
-                continue;
+            if (i_left == 0 && !begin_item()) {
+                i_done = true;
+                return;
             }
             issue_stage();
         }
@@ -723,54 +758,43 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
 
     while (ok) {
         pump();
-        if (c_sub == i_sub && c_seq == i_seq) break;   // nothing issued and nothing left to issue
-        const int ms = c_sub % kSubMeta;
-        const int *mt = sm.meta[warp][ms];
-        const int item = mt[0], n = mt[3], n_hi = mt[4], flags = mt[7];
-        const uint32_t w0 = (uint32_t)mt[5], w1 = (uint32_t)mt[6];
-        const int nq = (flags & 1) ? C::kQStages : 0;   // an item's first sub-chunk starts with its q~
-        const int nst = nq + (n_hi < n ? 1 : 0) + (n_hi + kHiTok - 1) / kHiTok;
-        for (int st = 0; st < nst; ++st) {
-            const int slot = c_seq % kSlots;
-            if (!mbar_wait(&sm.full[warp][slot], (c_seq / kSlots) & 1u, abort)) { ok = false; break; }
-            const uint32_t sb = smem_u32(sm.ring[warp][slot]);
-            if (st < nq) {
-                if (st == 0) {   // a new item: fresh softmax state
+        if (c_seq == i_seq) break;   // nothing in flight, nothing left to issue
+        const int slot = c_seq % kSlots;
+        if (!mbar_wait(&sm.full[warp][slot], (c_seq / kSlots) & 1u, abort)) { ok = false; break; }
+        const int *dsc = sm.desc[warp][slot];
+        const int type = dsc[0], item = dsc[1], n = dsc[2];
+        const uint32_t sb = smem_u32(sm.ring[warp][slot]);
+        if ((type & 3) == kTypeQ) {
+            if (type & kFirst) {   // a new item: fresh softmax state
+                #pragma unroll
+                for (int mb = 0; mb < NMB; ++mb) {
+                    m[mb][0] = m[mb][1] = kRefInit;
+                    l[mb][0] = l[mb][1] = 0.f;
                     #pragma unroll
-                    for (int mb = 0; mb < NMB; ++mb) {
-                        m[mb][0] = m[mb][1] = kRefInit;
-                        l[mb][0] = l[mb][1] = 0.f;
-                        #pragma unroll
-                        for (int a = 0; a < 8; ++a) u[mb][a][0] = u[mb][a][1] = u[mb][a][2] = u[mb][a][3] = 0.f;
-                    }
+                    for (int a = 0; a < 8; ++a) u[mb][a][0] = u[mb][a][1] = u[mb][a][2] = u[mb][a][3] = 0.f;
                 }
-                if (C::kQStages == 1) {
-                    load_plane(sb, qh);
-                    load_plane(sb + kHalf, ql);
-                } else if (st == 0) {
-                    load_plane(sb, qh);
-                } else {
-                    load_plane(sb, ql);
-                }
-            } else if (st == nq && n_hi < n) {
-                if (NMB == 1) {   // two 32-token halves: fewer live scores
-                    do_lo(sb, w0, 0u, n, std::integral_constant<int, 4>{});
-                    if (n > 32) do_lo(sb + 1024, w1, 0u, n - 32, std::integral_constant<int, 4>{});
-                } else {
-                    do_lo(sb, w0, w1, n, std::integral_constant<int, 8>{});
-                }
-            } else {
-                const int hs = st - nq - (n_hi < n ? 1 : 0);
-                do_hi(sb, min(kHiTok, n_hi - kHiTok * hs));
             }
-            ++c_seq;
-            __syncwarp();
-            pump();
+            if (C::kQStages == 1) {
+                load_plane(sb, qh);
+                load_plane(sb + kHalf, ql);
+            } else if (n == 0) {
+                load_plane(sb, qh);
+            } else {
+                load_plane(sb, ql);
+            }
+        } else if ((type & 3) == kTypeLo) {
+            const uint32_t w0 = (uint32_t)dsc[3], w1 = (uint32_t)dsc[4];
+            if (NMB == 1) {   // two 32-token halves: fewer live scores
+                do_lo(sb, w0, 0u, n, std::integral_constant<int, 4>{});
+                if (n > 32) do_lo(sb + 1024, w1, 0u, n - 32, std::integral_constant<int, 4>{});
+            } else {
+                do_lo(sb, w0, w1, n, std::integral_constant<int, 8>{});
+            }
+        } else {
+            do_hi(sb, n);
         }
-        if (!ok) break;
-        ++c_sub;
-        if (flags & 2) {
-            // last sub-chunk: the partial of the item -- per head row: max, sum, u[64]
+        if (type & kLast) {
+            // the item's partial -- per head row: max, sum, u[64]
             float *dst = p.part + (size_t)item * p.Hg * kVisPart;
             #pragma unroll
             for (int mb = 0; mb < NMB; ++mb)
@@ -790,6 +814,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<NMB>::kBlocks) vis_kernel(const 
                     }
                 }
         }
+        ++c_seq;
+        __syncwarp();
     }
     if (!ok) *abort = 1;
     // copies still in flight (only after an abort) must land before the block exits

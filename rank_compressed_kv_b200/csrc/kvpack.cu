@@ -72,6 +72,7 @@ DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
     const int S0 = (int)((T + tgt - 1) / tgt);
     pl.tps = ((T + S0 - 1) / S0 + 63) / 64 * 64;
     pl.S = (T + pl.tps - 1) / pl.tps;
+    static_assert(kvpack::decode::vis::kMaxItemTok >= 2048, "visual items of up to 2048 tokens");
     pl.Sc_max = (d->L_text_cap + kTextChunk - 1) / kTextChunk;
     size_t off = 0;
     pl.off_qt = off;
