@@ -29,7 +29,8 @@ constexpr int kChunk = 64;          // tokens of one unit per chunk
 constexpr int kSlots = 4;           // ring slots per warp
 constexpr int kSlotBytes = 2048;    // 64 C_K lo rows (32 B), or kHiTok gathered C_K rows (128 B)
 constexpr int kHiTok = 16;          // full-rank tokens per gathered stage
-constexpr int kMeta = 8;            // chunk metadata ring (the issue side runs at most kSlots chunks ahead)
+constexpr int kSegChunks = 32;      // chunks of one unit per segment: 2048 tokens, 64 mask words
+constexpr int kSegTok = kSegChunks * kChunk;
 
 struct Params {
     CUtensorMap tm_ck;              // C_K lo: 3D {16, T, units}, box {16, 32, 1}, 32-byte swizzle
@@ -43,18 +44,22 @@ struct Params {
 
 struct Smem {
     alignas(1024) unsigned char ring[kWarps][kSlots][kSlotBytes];
-    uint8_t hi_list[kWarps][kMeta][kChunk];   // chunk-relative positions of the full-rank tokens
-    int meta[kWarps][kMeta][6];               // unit, t0, n, n_hi, mask words 0 and 1
+    uint16_t hi_list[kWarps][kSegTok];        // segment-relative positions of the issue side's full-rank tokens
+    uint32_t mw[kWarps][kSegTok / 32];        // that segment's mask words
+    int desc[kWarps][kSlots][6];              // per ring slot: type, unit, t0, n, mask words 0 and 1
+    uint16_t pos[kWarps][kSlots][kHiTok];     // per gathered slot: the tokens' positions in the unit
     uint64_t full[kWarps][kSlots];
     int abort;
 };
 
 constexpr size_t smem_bytes() { return sizeof(Smem) + 1024; }
 
-// Every warp owns a contiguous range of chunks (unit, 64 tokens) and streams
-// it through a private ring: per chunk one TMA stage of C_K lo rows (skipped
-// when every token is full-rank) and one gathered stage per 16 full-rank
-// tokens.  Logits with tokens on M and heads on N (NT tiles of 8) of mma.sync
+// Every warp owns a contiguous range of chunks (unit, 64 tokens), taken in
+// segments of up to 32 chunks of one unit, and streams it through a private
+// ring: per chunk one TMA stage of C_K lo rows (skipped when every token is
+// full-rank), then the segment's full-rank tokens 16 at a time (C_lo + C_hi
+// rows gathered by cp.async; the issue side lists them once per segment).
+// Logits with tokens on M and heads on N (NT tiles of 8) of mma.sync
 // m16n8k16, q~ as a bf16 hi + lo pair held in registers for the whole unit.
 template <int NT>
 __global__ void __launch_bounds__(kThreads, NT <= 2 ? 2 : 1) mass_kernel(const __grid_constant__ Params p) {
@@ -76,88 +81,123 @@ __global__ void __launch_bounds__(kThreads, NT <= 2 ? 2 : 1) mass_kernel(const _
     const int c_begin = (int)(wg * p.n_chunks / W), c_end = (int)((wg + 1) * p.n_chunks / W);
 
     // ------------------------------------------------------------ issue side
-    int i_c = c_begin, i_st = 0, i_nst = 0;
+    constexpr int kTypeLo = 0, kTypeHi = 1;
+    int i_c = c_begin;                               // first chunk of the next segment
+    int i_unit = 0, i_t0 = 0, i_n = 0;               // the segment being issued
+    int i_sub = 0, i_lo = 0, i_hi = 0, i_nhi = 0, i_left = 0;
     uint32_t i_seq = 0, c_seq = 0;
     bool i_done = c_begin >= c_end;
-    auto begin_chunk = [&](int c) {
-        const int ms = (c - c_begin) % kMeta;
-        const int unit = c / p.cpu, t0 = (c % p.cpu) * kChunk;
-        const int n = min(kChunk, p.T - t0);
-        uint32_t w = 0u;
-        if (lane < 2 && 32 * lane < n) {
-            w = __ldg(p.mask + (size_t)unit * p.nwords + (t0 >> 5) + lane);
-            const int nb = n - 32 * lane;
-            if (nb < 32) w &= (1u << nb) - 1u;
+    auto begin_segment = [&]() -> bool {
+        if (i_c >= c_end) return false;
+        i_unit = i_c / p.cpu;
+        const int k0 = i_c % p.cpu;
+        const int nch = min(min(kSegChunks, p.cpu - k0), c_end - i_c);
+        i_c += nch;
+        i_t0 = k0 * kChunk;
+        i_n = min(nch * kChunk, p.T - i_t0);
+        const int nw = (i_n + 31) >> 5;
+        int base = 0, n_lo_st = 0;
+        for (int w0 = 0; w0 < nw; w0 += 32) {
+            const int wi = w0 + lane;
+            uint32_t w = 0u;
+            if (wi < nw) {
+                w = __ldg(p.mask + (size_t)i_unit * p.nwords + (i_t0 >> 5) + wi);
+                const int nb = i_n - 32 * wi;
+                if (nb < 32) w &= (1u << nb) - 1u;
+                sm.mw[warp][wi] = w;
+            }
+            const int c = __popc(w);
+            int incl = c;
+            #pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += v;
+            }
+            int r = base + incl - c;
+            uint32_t bits = w;
+            while (bits) {
+                sm.hi_list[warp][r++] = (uint16_t)(32 * wi + __ffs(bits) - 1);
+                bits &= bits - 1u;
+            }
+            const int c_pair = c + __shfl_down_sync(0xffffffffu, c, 1);
+            const bool lo_st = (lane & 1) == 0 && wi < nw && c_pair < min(kChunk, i_n - 32 * wi);
+            n_lo_st += __popc(__ballot_sync(0xffffffffu, lo_st));
+            base += __shfl_sync(0xffffffffu, incl, 31);
         }
-        const uint32_t w0 = __shfl_sync(0xffffffffu, w, 0), w1 = __shfl_sync(0xffffffffu, w, 1);
-        const int c0 = __popc(w0), n_hi = c0 + __popc(w1);
-        const uint32_t below = (1u << lane) - 1u;
-        if ((w0 >> lane) & 1u) sm.hi_list[warp][ms][__popc(w0 & below)] = (uint8_t)lane;
-        if ((w1 >> lane) & 1u) sm.hi_list[warp][ms][c0 + __popc(w1 & below)] = (uint8_t)(32 + lane);
-        if (lane == 0) {
-            int *m = sm.meta[warp][ms];
-            m[0] = unit; m[1] = t0; m[2] = n; m[3] = n_hi; m[4] = (int)w0; m[5] = (int)w1;
-        }
+        i_nhi = base;
+        i_hi = 0;
+        i_sub = 0;
+        i_lo = n_lo_st;
+        i_left = n_lo_st + (i_nhi + kHiTok - 1) / kHiTok;
         __syncwarp();
-        i_nst = (n_hi < n ? 1 : 0) + (n_hi + kHiTok - 1) / kHiTok;
-        i_st = 0;
+        return true;
     };
     auto issue_stage = [&]() {
-        const int ms = (i_c - c_begin) % kMeta;
-        const int *m = sm.meta[warp][ms];
-        const int unit = m[0], t0 = m[1], n = m[2], n_hi = m[3];
         const int slot = i_seq % kSlots;
         unsigned char *dst = sm.ring[warp][slot];
         uint64_t *bar = &sm.full[warp][slot];
+        int type, n, t0 = 0;
+        uint32_t w0 = 0u, w1 = 0u;
         __syncwarp();
-        if (i_st == 0 && n_hi < n) {
+        if (i_lo > 0) {
+            // the next chunk with a reduced-rank token (one exists)
+            while (true) {
+                n = min(kChunk, i_n - kChunk * i_sub);
+                w0 = sm.mw[warp][2 * i_sub];
+                w1 = n > 32 ? sm.mw[warp][2 * i_sub + 1] : 0u;
+                if (__popc(w0) + __popc(w1) < n) break;
+                ++i_sub;
+            }
+            type = kTypeLo;
+            t0 = i_t0 + kChunk * i_sub;
             const int nb = (n + 31) >> 5;
             if (lane == 0) {
                 fence_proxy_async();
                 mbar_arrive_tx(bar, (uint32_t)nb * 1024u);
-                for (int b = 0; b < nb; ++b) tma_3d(dst + 1024 * b, &p.tm_ck, 0, t0 + 32 * b, unit, bar);
+                for (int b = 0; b < nb; ++b) tma_3d(dst + 1024 * b, &p.tm_ck, 0, t0 + 32 * b, i_unit, bar);
             } else {
                 mbar_arrive(bar);
             }
+            ++i_sub;
+            --i_lo;
         } else {
-            // kHiTok full-rank tokens: C_lo + C_hi rows gathered into 128-byte rows
-            // (16-byte chunk c of row r stored at c ^ (r & 7)); rows past the count are left alone
-            const int hs = i_st - (n_hi < n ? 1 : 0);
-            const int cnt = min(kHiTok, n_hi - kHiTok * hs);
-            const size_t ubase = (size_t)unit * p.T + t0;
+            // kHiTok full-rank tokens: C_lo + C_hi into 128-byte rows (16-byte chunk c of row r at
+            // c ^ (r & 7)); rows past the count are left alone
+            type = kTypeHi;
+            n = min(kHiTok, i_nhi - i_hi);
+            const size_t ubase = (size_t)i_unit * p.T + i_t0;
+            if (lane < n) sm.pos[warp][slot][lane] = (uint16_t)(i_t0 + sm.hi_list[warp][i_hi + lane]);
             #pragma unroll
             for (int i = 0; i < kHiTok / 4; ++i) {
                 const int idx = lane + 32 * i;
                 const int r = idx >> 3, ch = idx & 7;
-                if (r < cnt) {
-                    const size_t row = ubase + sm.hi_list[warp][ms][kHiTok * hs + r];
+                if (r < n) {
+                    const size_t row = ubase + sm.hi_list[warp][i_hi + r];
                     const uint16_t *src = ch < 2 ? p.CK_lo + row * 16 + ch * 8 : p.CK_hi + row * 48 + (ch - 2) * 8;
                     cp_async16(dst + r * 128 + ((ch ^ (r & 7)) << 4), src);
                 }
             }
             cp_async_arrive_noinc(bar);
+            i_hi += n;
         }
-        ++i_st;
+        --i_left;
+        if (lane == 0) {
+            int *d = sm.desc[warp][slot];
+            d[0] = type; d[1] = i_unit; d[2] = t0; d[3] = n; d[4] = (int)w0; d[5] = (int)w1;
+        }
+        __syncwarp();
         ++i_seq;
     };
-    // issue while the ring has room, at most kMeta - 1 chunks ahead of the consumer
-    int c_c = c_begin;   // chunk the consumer is on
     auto pump = [&]() {
         while (!i_done && i_seq - c_seq < (uint32_t)kSlots) {
-            if (i_st == i_nst) {
-                if (i_c + 1 >= c_end) { i_done = true; return; }
-                if (i_c + 1 - c_c >= kMeta) return;
-                ++i_c;
-                begin_chunk(i_c);
-                continue;
+            if (i_left == 0 && !begin_segment()) {
+                i_done = true;
+                return;
             }
             issue_stage();
         }
     };
-    if (!i_done) {
-        begin_chunk(i_c);
-        pump();
-    }
+    pump();
 
     // ---------------------------------------------------------- consumer side
     uint32_t qh[4][NT][2], ql[4][NT][2];   // q~^T as B fragments: k-step kb, head tile nt
@@ -204,82 +244,73 @@ __global__ void __launch_bounds__(kThreads, NT <= 2 ? 2 : 1) mass_kernel(const _
         v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
     };
 
-    for (; c_c < c_end; ++c_c) {
+    bool ok = true;
+    while (true) {
         pump();
-        const int ms = (c_c - c_begin) % kMeta;
-        const int unit = sm.meta[warp][ms][0], t0 = sm.meta[warp][ms][1], n = sm.meta[warp][ms][2];
-        const int n_hi = sm.meta[warp][ms][3];
-        const uint32_t w0 = (uint32_t)sm.meta[warp][ms][4], w1 = (uint32_t)sm.meta[warp][ms][5];
+        if (c_seq == i_seq) break;   // nothing in flight, nothing left to issue
+        const int slot = c_seq % kSlots;
+        if (!mbar_wait(&sm.full[warp][slot], (c_seq / kSlots) & 1u, abort)) { ok = false; break; }
+        const int *dsc = sm.desc[warp][slot];
+        const int type = dsc[0], unit = dsc[1], t0 = dsc[2], n = dsc[3];
         if (unit != cur_unit) {
             load_unit(unit);
             cur_unit = unit;
         }
-        float *mrow = p.mass + (size_t)unit * p.T + t0;
-        const int nst = (n_hi < n ? 1 : 0) + (n_hi + kHiTok - 1) / kHiTok;
-        bool ok = true;
-        for (int st = 0; st < nst; ++st) {
-            const int slot = c_seq % kSlots;
-            if (!mbar_wait(&sm.full[warp][slot], (c_seq / kSlots) & 1u, abort)) { ok = false; break; }
-            const uint32_t sb = smem_u32(sm.ring[warp][slot]);
-            if (st == 0 && n_hi < n) {
-                // C_K lo rows of the chunk (32-byte rows, 32-byte swizzle: chunk c of row r at c ^ ((r >> 2) & 1))
-                #pragma unroll
-                for (int mt = 0; mt < kChunk / 16; ++mt) {
-                    if (16 * mt < n) {
-                        uint32_t a[4];
-                        const int row = 16 * mt + (lane & 7) + (((lane >> 3) & 1) << 3);
-                        const int ch = lane >> 4;
-                        ldsm_x4(sb + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), a[0], a[1], a[2], a[3]);
-                        float s[NT][4];
-                        #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-                            mma_bf16(s[nt], a, qh[0][nt][0], qh[0][nt][1]);
-                            mma_bf16(s[nt], a, ql[0][nt][0], ql[0][nt][1]);
-                        }
-                        float v0, v1;
-                        tile_mass(s, v0, v1);
-                        if (tig < 2) {
-                            const int r = 16 * mt + g + 8 * tig;
-                            const uint32_t wd = r < 32 ? w0 : w1;
-                            if (r < n && !((wd >> (r & 31)) & 1u)) mrow[r] = tig ? v1 : v0;
-                        }
-                    }
-                }
-            } else {
-                const int hs = st - (n_hi < n ? 1 : 0);
-                const int cnt = min(kHiTok, n_hi - kHiTok * hs);
-                float s[NT][4];
-                #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-                #pragma unroll
-                for (int kb = 0; kb < 4; ++kb) {
+        float *mrow = p.mass + (size_t)unit * p.T;
+        const uint32_t sb = smem_u32(sm.ring[warp][slot]);
+        if (type == kTypeLo) {
+            // C_K lo rows of the chunk (32-byte rows, 32-byte swizzle: chunk c of row r at c ^ ((r >> 2) & 1))
+            const uint32_t w0 = (uint32_t)dsc[4], w1 = (uint32_t)dsc[5];
+            #pragma unroll
+            for (int mt = 0; mt < kChunk / 16; ++mt) {
+                if (16 * mt < n) {
                     uint32_t a[4];
-                    const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
-                    const int ch = 2 * kb + (lane >> 4);
-                    ldsm_x4(sb + row * 128 + ((ch ^ (row & 7)) << 4), a[0], a[1], a[2], a[3]);
+                    const int row = 16 * mt + (lane & 7) + (((lane >> 3) & 1) << 3);
+                    const int ch = lane >> 4;
+                    ldsm_x4(sb + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), a[0], a[1], a[2], a[3]);
+                    float s[NT][4];
                     #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        mma_bf16(s[nt], a, qh[kb][nt][0], qh[kb][nt][1]);
-                        mma_bf16(s[nt], a, ql[kb][nt][0], ql[kb][nt][1]);
+                        s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+                        mma_bf16(s[nt], a, qh[0][nt][0], qh[0][nt][1]);
+                        mma_bf16(s[nt], a, ql[0][nt][0], ql[0][nt][1]);
+                    }
+                    float v0, v1;
+                    tile_mass(s, v0, v1);
+                    if (tig < 2) {
+                        const int r = 16 * mt + g + 8 * tig;
+                        const uint32_t wd = r < 32 ? w0 : w1;
+                        if (r < n && !((wd >> (r & 31)) & 1u)) mrow[t0 + r] = tig ? v1 : v0;
                     }
                 }
-                float v0, v1;
-                tile_mass(s, v0, v1);
-                if (tig < 2) {
-                    const int r = g + 8 * tig;
-                    if (r < cnt) mrow[sm.hi_list[warp][ms][kHiTok * hs + r]] = tig ? v1 : v0;
+            }
+        } else {
+            float s[NT][4];
+            #pragma unroll
+            for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+            #pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+                uint32_t a[4];
+                const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
+                const int ch = 2 * kb + (lane >> 4);
+                ldsm_x4(sb + row * 128 + ((ch ^ (row & 7)) << 4), a[0], a[1], a[2], a[3]);
+                #pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    mma_bf16(s[nt], a, qh[kb][nt][0], qh[kb][nt][1]);
+                    mma_bf16(s[nt], a, ql[kb][nt][0], ql[kb][nt][1]);
                 }
             }
-            ++c_seq;
-            __syncwarp();
-            pump();
+            float v0, v1;
+            tile_mass(s, v0, v1);
+            if (tig < 2) {
+                const int r = g + 8 * tig;
+                if (r < n) mrow[sm.pos[warp][slot][r]] = tig ? v1 : v0;
+            }
         }
-        if (!ok) {
-            *abort = 1;
-            break;
-        }
+        ++c_seq;
+        __syncwarp();
     }
+    if (!ok) *abort = 1;
     // copies still in flight (only after an abort) must land before the block exits
     while (c_seq < i_seq) {
         const int slot = c_seq % kSlots;
