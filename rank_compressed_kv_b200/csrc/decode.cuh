@@ -848,11 +848,15 @@ __host__ __device__ constexpr size_t finish_smem_bytes(int S, int Sc, int Hg) {
 }
 constexpr size_t kFinishSmemMax = 200 * 1024;
 
-// One block per unit.  Per head, the unit-wide max M and sum L over every visual and text
+// One block per unit.  When the unit has many partials, thread 0 first asks
+// for the unit's B_V (64 KB) to be brought into L2, so that it streams from
+// DRAM while the partials are combined.  Per head, the unit-wide max M and sum L over every visual and text
 // partial give each partial the weight 2^(m - M) / L; u / l and w / l are
 // weighted sums with the feature index across threads (coalesced).  Then
 // o_h = (u_h / l_h) B_V[:, 128 j(h) ..] + w_h / l_h, thread t owning output
 // columns 2t, 2t+1 of the unit's 512 (KV head t / 64).
+// PK = query heads per KV head (the projection's inner loop is unrolled over exactly PK heads).
+template <int PK>
 __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
     extern __shared__ float fsm[];
     float *wv = fsm;                              // [S][Hg]
@@ -863,6 +867,7 @@ __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
     const float *vp0 = p.vpart + (size_t)unit * p.S * p.Hg * kVisPart;
     const float *tp0 = p.tpart + (size_t)unit * p.Sc * p.Hg * kTxtPart;
     const uint16_t *bvg = p.BV + (size_t)unit * 64 * 512;
+    if (tid == 0 && p.S + p.Sc > 8) bulk_prefetch_l2(bvg, 64 * 512 * 2);   // long combine: overlap B_V
 
     for (int h = warp; h < p.Hg; h += 8) {
         float mx = -INFINITY;
@@ -894,38 +899,52 @@ __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
         for (int c = lane; c < p.Sc; c += 32) wt[c * p.Hg + h] *= inv;
     }
     __syncthreads();
-    for (int task = tid; task < p.Hg * 64; task += 256) {
-        const int h = task >> 6, f = task & 63;
-        const float *r = vp0 + (size_t)h * kVisPart + 2 + f;
-        float a0 = 0.f, a1 = 0.f;
-        int s = 0;
-        for (; s + 2 <= p.S; s += 2) {
-            a0 = fmaf(__ldcg(r + (size_t)s * p.Hg * kVisPart), wv[s * p.Hg + h], a0);
-            a1 = fmaf(__ldcg(r + (size_t)(s + 1) * p.Hg * kVisPart), wv[(s + 1) * p.Hg + h], a1);
+    // weighted sums: thread tid takes the tasks tid, tid + 256, ... K at a time (K = the tasks per
+    // thread, up to 4), so that the partial loads of K sums are in flight together
+    auto combine_k = [&](auto kc, const float *base, int row, int n_task, int npart, const float *wgt, float *dst,
+                         int shift) {
+        constexpr int K = decltype(kc)::value;
+        const size_t st = (size_t)p.Hg * row;
+        for (int t0 = tid; t0 < n_task; t0 += K * 256) {
+            const float *r[K];
+            int hk[K];
+            bool ok[K];
+            #pragma unroll
+            for (int k = 0; k < K; ++k) {
+                const int task = t0 + 256 * k;
+                ok[k] = task < n_task;
+                hk[k] = ok[k] ? task >> shift : 0;
+                r[k] = base + (size_t)hk[k] * row + 2 + (ok[k] ? (task & ((1 << shift) - 1)) : 0);
+            }
+            float acc[K];
+            #pragma unroll
+            for (int k = 0; k < K; ++k) acc[k] = 0.f;
+            for (int s2 = 0; s2 < npart; ++s2) {
+                #pragma unroll
+                for (int k = 0; k < K; ++k)
+                    if (ok[k]) acc[k] = fmaf(__ldcg(r[k] + s2 * st), wgt[s2 * p.Hg + hk[k]], acc[k]);
+            }
+            #pragma unroll
+            for (int k = 0; k < K; ++k)
+                if (ok[k]) dst[t0 + 256 * k] = acc[k];
         }
-        if (s < p.S) a0 = fmaf(__ldcg(r + (size_t)s * p.Hg * kVisPart), wv[s * p.Hg + h], a0);
-        uf[h * 64 + f] = a0 + a1;
-    }
-    for (int task = tid; task < p.Hg * 128; task += 256) {
-        const int h = task >> 7, f = task & 127;
-        const float *r = tp0 + (size_t)h * kTxtPart + 2 + f;
-        float a0 = 0.f, a1 = 0.f;
-        int c = 0;
-        for (; c + 2 <= p.Sc; c += 2) {
-            a0 = fmaf(__ldcg(r + (size_t)c * p.Hg * kTxtPart), wt[c * p.Hg + h], a0);
-            a1 = fmaf(__ldcg(r + (size_t)(c + 1) * p.Hg * kTxtPart), wt[(c + 1) * p.Hg + h], a1);
-        }
-        if (c < p.Sc) a0 = fmaf(__ldcg(r + (size_t)c * p.Hg * kTxtPart), wt[c * p.Hg + h], a0);
-        wf[h * 128 + f] = a0 + a1;
-    }
+    };
+    auto combine = [&](const float *base, int row, int n_task, int npart, const float *wgt, float *dst, int shift) {
+        const int per = (n_task + 255) / 256;
+        if (per <= 1) combine_k(std::integral_constant<int, 1>(), base, row, n_task, npart, wgt, dst, shift);
+        else if (per == 2) combine_k(std::integral_constant<int, 2>(), base, row, n_task, npart, wgt, dst, shift);
+        else combine_k(std::integral_constant<int, 4>(), base, row, n_task, npart, wgt, dst, shift);
+    };
+    combine(vp0, kVisPart, p.Hg * 64, p.S, wv, uf, 6);
+    combine(tp0, kTxtPart, p.Hg * 128, p.Sc, wt, wf, 7);
     __syncthreads();
     const int j = tid >> 6, d = (2 * tid) & 127;
     const int lb = unit / p.groups, G = unit % p.groups;
     const uint32_t *bv = reinterpret_cast<const uint32_t *>(bvg) + tid;
-    float acc[8][2];
+    float acc[PK][2];
     #pragma unroll
-    for (int hh = 0; hh < 8; ++hh) acc[hh][0] = acc[hh][1] = 0.f;
-    const int h0 = j * p.per_kv;
+    for (int hh = 0; hh < PK; ++hh) acc[hh][0] = acc[hh][1] = 0.f;
+    const int h0 = j * PK;
     #pragma unroll 4
     for (int i0 = 0; i0 < 64; i0 += 16) {
         uint32_t braw[16];
@@ -935,22 +954,18 @@ __global__ void __launch_bounds__(256) finish_kernel(const FinishParams p) {
         for (int i = 0; i < 16; ++i) {
             const float b0 = __uint_as_float(braw[i] << 16), b1 = __uint_as_float(braw[i] & 0xffff0000u);
             #pragma unroll
-            for (int hh = 0; hh < 8; ++hh) {
-                if (hh < p.per_kv) {
-                    const float x = uf[(h0 + hh) * 64 + i0 + i];
-                    acc[hh][0] = fmaf(x, b0, acc[hh][0]);
-                    acc[hh][1] = fmaf(x, b1, acc[hh][1]);
-                }
+            for (int hh = 0; hh < PK; ++hh) {
+                const float x = uf[(h0 + hh) * 64 + i0 + i];
+                acc[hh][0] = fmaf(x, b0, acc[hh][0]);
+                acc[hh][1] = fmaf(x, b1, acc[hh][1]);
             }
         }
     }
     #pragma unroll
-    for (int hh = 0; hh < 8; ++hh) {
-        if (hh < p.per_kv) {
-            const int h = h0 + hh;
-            *reinterpret_cast<uint32_t *>(p.out + ((size_t)lb * p.n_q + (size_t)G * p.Hg + h) * 128 + d) =
-                pack_bf16(acc[hh][0] + wf[h * 128 + d], acc[hh][1] + wf[h * 128 + d + 1]);
-        }
+    for (int hh = 0; hh < PK; ++hh) {
+        const int h = h0 + hh;
+        *reinterpret_cast<uint32_t *>(p.out + ((size_t)lb * p.n_q + (size_t)G * p.Hg + h) * 128 + d) =
+            pack_bf16(acc[hh][0] + wf[h * 128 + d], acc[hh][1] + wf[h * 128 + d + 1]);
     }
 }
 

@@ -97,6 +97,31 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
+// finish_kernel is instantiated for 1..8 query heads per KV head
+template <int PK>
+bool finish_attr_one() {
+    return cudaFuncSetAttribute(kvpack::decode::finish_kernel<PK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kvpack::decode::kFinishSmemMax) == cudaSuccess;
+}
+bool finish_attrs() {
+    return finish_attr_one<1>() && finish_attr_one<2>() && finish_attr_one<3>() && finish_attr_one<4>() &&
+           finish_attr_one<5>() && finish_attr_one<6>() && finish_attr_one<7>() && finish_attr_one<8>();
+}
+cudaError_t launch_finish(int per_kv, const kvpack::decode::FinishParams &fp, int units, size_t smem, cudaStream_t st) {
+    namespace dc = kvpack::decode;
+    switch (per_kv) {
+        case 1: dc::finish_kernel<1><<<units, 256, smem, st>>>(fp); break;
+        case 2: dc::finish_kernel<2><<<units, 256, smem, st>>>(fp); break;
+        case 3: dc::finish_kernel<3><<<units, 256, smem, st>>>(fp); break;
+        case 4: dc::finish_kernel<4><<<units, 256, smem, st>>>(fp); break;
+        case 5: dc::finish_kernel<5><<<units, 256, smem, st>>>(fp); break;
+        case 6: dc::finish_kernel<6><<<units, 256, smem, st>>>(fp); break;
+        case 7: dc::finish_kernel<7><<<units, 256, smem, st>>>(fp); break;
+        default: dc::finish_kernel<8><<<units, 256, smem, st>>>(fp); break;
+    }
+    return cudaGetLastError();
+}
+
 kvpack_status device_info(DeviceInfo **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVPACK_ERR_CUDA;
@@ -111,8 +136,7 @@ kvpack_status device_info(DeviceInfo **out) {
                                  (int)dc::vis::smem_bytes<2>()) != cudaSuccess ||
             cudaFuncSetAttribute(dc::text::text_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)dc::text::smem_bytes()) != cudaSuccess ||
-            cudaFuncSetAttribute(dc::finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)dc::kFinishSmemMax) != cudaSuccess)
+            !finish_attrs())
             return KVPACK_ERR_CUDA;
         // all of the SM's shared memory for these kernels (two visual blocks of the 16-row variant)
         if (cudaFuncSetAttribute(dc::vis::vis_kernel<1>, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
@@ -348,7 +372,8 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     // 4. combine and project through B_V
     dc::FinishParams fp{BV, vpart, Sc > 0 ? tpart : nullptr, out, mass != nullptr ? ustat : nullptr,
                         Hg, per_kv, d->n_q_heads, groups, pl.S, Sc};
-    dc::finish_kernel<<<pl.units, 256, dc::finish_smem_bytes(pl.S, Sc, Hg), st>>>(fp);
+    if (launch_finish(per_kv, fp, pl.units, dc::finish_smem_bytes(pl.S, Sc, Hg), st) != cudaSuccess)
+        return KVPACK_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
     if (mass == nullptr) return KVPACK_OK;
 
