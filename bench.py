@@ -265,7 +265,8 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
     # end-to-end through the public API with host buffers: every step's q comes from pinned host
     # memory and its output goes back to pinned host memory.  The copies run on a second stream,
     # double-buffered, so step i + 1's upload and step i's download overlap the computation, as a
-    # serving loop would run them; each step still moves its own bytes.
+    # serving loop would run them; each step still moves its own bytes.  The text lengths are those
+    # of the device-timed steps, so the two numbers time the same work.
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -290,7 +291,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
             stream.wait_event(ev_d2h[b])        # outd[b] has been read back
         kv.select(dims, n_layers, mass, None, 0.0, k_hi, mask)
         kv.decode_attn(dims, n_layers, qd[b], c["CK_lo"], c["CK_hi"], c["BK"], c["CV_lo"], c["CV_hi"], c["BV"],
-                       c["K_text"], c["V_text"], min(L0 + s, Lcap), mask, 1.0, outd[b], mass, ws)
+                       c["K_text"], c["V_text"], min(L0 + W + 1 + i, Lcap), mask, 1.0, outd[b], mass, ws)
         ev_done[b].record(stream)
         if i + 1 < K:                            # next step's q, once step i - 1 has finished reading qd[1 - b]
             with torch.cuda.stream(hs):
@@ -313,6 +314,50 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
     e2e_value = world * w.batch / (e2e_ms / 1e3)
     qbytes = q_host[0].numel() * 2
     obytes = out.numel() * 2
+
+    # per-layer launches, as a framework that runs attention layer by layer would call the
+    # library: one kvpack_select and one kvpack_decode_attn per layer (layer slices of the same
+    # buffers), captured once into a CUDA graph and replayed K times; the text length stays at the
+    # captured value
+    upl = w.units_per_layer
+    dims1 = kv.Dims(batch=w.batch, n_q_heads=w.n_q, n_kv_heads=w.n_kv, T_vis=T, L_text_cap=Lcap)
+    ws1 = torch.empty(kv.decode_workspace(dims1, 1), dtype=torch.uint8, device=dev)
+    L_g = min(L0 + W + 1 + 2 * K, Lcap)
+    qg = q_dev[0]
+
+    def per_layer_step():
+        for l in range(n_layers):
+            u0, u1, r0, r1 = l * upl, (l + 1) * upl, l * w.batch, (l + 1) * w.batch
+            kv.select(dims1, 1, mass[u0:u1], None, 0.0, k_hi, mask[u0:u1])
+            kv.decode_attn(dims1, 1, qg[r0:r1], c["CK_lo"][u0:u1], c["CK_hi"][u0:u1], c["BK"][u0:u1],
+                           c["CV_lo"][u0:u1], c["CV_hi"][u0:u1], c["BV"][u0:u1], c["K_text"][u0:u1],
+                           c["V_text"][u0:u1], L_g, mask[u0:u1], 1.0, out[r0:r1], mass[u0:u1], ws1)
+
+    per_layer_step()                      # library set-up outside the capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        per_layer_step()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(K):
+        graph.replay()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    st = kv.last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {kv.STATUS_NAMES[st]} in the per-layer graph")
+    g_ms = g0.elapsed_time(g1) / K
+    if dist:
+        t = torch.tensor([g_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        g_ms = float(t[0])
+    del graph
 
     # roofline of the dominant launch (kvpack_decode_attn), algorithmic bytes per launch
     hbm, _, peak_kind = measured_peaks()
@@ -352,6 +397,9 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
         "e2e": {"value": round(e2e_value, 1), "unit": "query-tokens/s", "h2d_bytes_per_step": qbytes,
                 "d2h_bytes_per_step": obytes, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": 6 * K,   # per step: select, text (q~ projection + text tail), text statistics, visual, finish, mass
+        "per_layer_graph": {"value": round(world * w.batch / (g_ms / 1e3), 1), "unit": "query-tokens/s",
+                            "ms_per_step": round(g_ms, 4), "launches_per_step": 6 * n_layers, "text_len": L_g,
+                            "mode": "per layer: kvpack_select + kvpack_decode_attn, captured in one CUDA graph"},
         "clocks": clk,
         "wall_s_timed": round(wall, 3),
     }

@@ -12,9 +12,11 @@
   orthonormal rows, C's column norms are sigma, C^T C is diagonal, the
   residual is the discarded energy) plus the generator's known leading
   singular values.
-* the decode -> select chain over C0's 8 steps: decode parity at every step on
-  the GPU's own mask, and the GPU's next mask equal to the oracle's wherever
-  the oracle's mass is decided (relative gap to the k-th largest > 1e-3)."""
+* the decode -> select chain over C0's 8 steps, with importance = mass
+  (alpha = 0) and with the moving average alpha = 0.5 carried on each side:
+  decode parity at every step on the GPU's own mask, and the GPU's next mask
+  equal to the oracle's wherever the oracle's importance is decided (relative
+  gap to the k-th largest > 1e-3)."""
 import numpy as np
 import pytest
 import torch
@@ -132,7 +134,8 @@ def test_compress_one_unit_at_T65536():
     assert abs(res - (tot - float((s * s).sum()))) <= 5e-2 * res + 1e-5 * tot
 
 
-def test_decode_select_chain_c0():
+@pytest.mark.parametrize("alpha", [0.0, 0.5])
+def test_decode_select_chain_c0(alpha):
     import rank_compressed_kv_b200 as kv
     w = synth.WORKLOADS["C0"]
     T, U, steps = w.T, w.units, w.steps
@@ -146,6 +149,8 @@ def test_decode_select_chain_c0():
     dev["CV_lo"], dev["CV_hi"] = bf(CV[..., :16]), bf(CV[..., 16:])
     ws = torch.empty(kv.decode_workspace(dims, 1), dtype=torch.uint8, device=DEV)
     mask = u32(np.stack([synth.all_ones_mask(T)] * U))
+    score = torch.zeros(U, T, dtype=torch.float32, device=DEV)    # the GPU's importance state
+    ref_score = np.zeros((U, T), dtype=np.float32)                  # the oracle's, from its own masses
     for step in range(steps):
         L = w.text0 + step
         q_np = np.stack([synth.query(w, 0, b, step) for b in range(w.batch)])
@@ -167,13 +172,14 @@ def test_decode_select_chain_c0():
         np.testing.assert_allclose(got_m, ref_m, rtol=1e-4, atol=1e-10)
         # next mask: GPU selection from its own mass vs the oracle's from the oracle's mass
         nxt = torch.empty_like(mask)
-        kv.select(dims, 1, mass, None, 0.0, w.k_hi, nxt)
+        kv.select(dims, 1, mass, score if alpha > 0 else None, alpha, w.k_hi, nxt)
         got_next = nxt.cpu().numpy().view(np.uint32)
-        ref_next, _ = oracle.select(ref_m.astype(np.float32), w.k_hi)
+        ref_next, ref_score = oracle.select(ref_m.astype(np.float32), w.k_hi, alpha=alpha, score=ref_score)
+        keys = ref_score if alpha > 0 else ref_m
         bits = lambda m: ((m[:, np.arange(T) >> 5] >> (np.arange(T) & 31).astype(np.uint32)) & 1).astype(bool)
         gb, rb = bits(got_next), bits(ref_next)
         for u in range(U):
-            theta = np.sort(ref_m[u])[::-1][w.k_hi - 1]
-            decided = np.abs(ref_m[u] - theta) > 1e-3 * theta
-            assert np.array_equal(gb[u][decided], rb[u][decided]), f"step {step} unit {u}"
+            theta = np.sort(keys[u])[::-1][w.k_hi - 1]
+            decided = np.abs(keys[u] - theta) > 1e-3 * theta
+            assert np.array_equal(gb[u][decided], rb[u][decided]), f"alpha {alpha} step {step} unit {u}"
         mask = nxt
