@@ -69,9 +69,36 @@ def measured_peaks():
     try:
         with open(path) as f:
             mp = json.load(f)
-        return float(mp["hbm_gbs"]), float(mp["bf16_tflops"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+        return float(mp["hbm_gbs"]), float(mp["bf16_tflops"]), "measured (MEASURED_PEAKS.json)"
     except Exception:
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback (profiling recipe)"
+
+
+class Ranks:
+    """The bench's steps across ranks: barriers and max-over-ranks reductions of device
+    times.  Every rank takes the same steps in the same order; without a process group
+    (one GPU) they are no-ops.  The backend is NCCL on the GPUs and gloo for the CPU tests."""
+
+    def __init__(self, dist=None, device="cpu"):
+        self.dist, self.device = dist, device
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, *values):
+        if self.dist is None:
+            return tuple(float(v) for v in values)
+        import torch
+        t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return tuple(float(x) for x in t.cpu())
+
+
+def whole_job_value(world: int, batch: int, ms_per_step: float) -> float:
+    """Query tokens per second of the whole job: every rank decodes its own batch (weak
+    scaling), and the step time is the slowest rank's."""
+    return world * batch / (ms_per_step / 1e3)
 
 
 DECODE_SOURCES = ("decode.cuh", "mass.cuh", "common.cuh", "kvpack.cu")
@@ -192,6 +219,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
         import torch.distributed as dist
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    ranks = Ranks(dist, dev)
 
     K, W = args.steps, args.warmup
     T, L0 = w.T, w.text0
@@ -233,8 +261,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    if dist:
-        dist.barrier()
+    ranks.barrier()
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     ev0.record(stream)
@@ -253,14 +280,9 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
         raise RuntimeError(f"device status {kv.STATUS_NAMES[st]} during the timed region")
     ms_total = ev0.elapsed_time(ev1)
     dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
-    if dist:
-        t = torch.tensor([ms_total, sum(dec_ms)], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, dec_sum = float(t[0]), float(t[1])
-    else:
-        dec_sum = sum(dec_ms)
+    ms_total, dec_sum = ranks.max(ms_total, sum(dec_ms))
     ms_step = ms_total / K
-    value = world * w.batch / (ms_step / 1e3)
+    value = whole_job_value(world, w.batch, ms_step)
 
     # end-to-end through the public API with host buffers: every step's q comes from pinned host
     # memory and its output goes back to pinned host memory.  The copies run on a second stream,
@@ -268,8 +290,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
     # serving loop would run them; each step still moves its own bytes.  The text lengths are those
     # of the device-timed steps, so the two numbers time the same work.
     torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
+    ranks.barrier()
     hs, ds = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)   # uploads, downloads
     qd = [torch.empty_like(q_dev[0]) for _ in range(2)]
     outd = [torch.empty_like(out) for _ in range(2)]
@@ -306,12 +327,8 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
     stream.wait_event(ev_d2h[(K - 1) % 2])
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / K
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e_value = world * w.batch / (e2e_ms / 1e3)
+    e2e_ms, = ranks.max(e0.elapsed_time(e1) / K)
+    e2e_value = whole_job_value(world, w.batch, e2e_ms)
     qbytes = q_host[0].numel() * 2
     obytes = out.numel() * 2
 
@@ -341,8 +358,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
     for _ in range(3):
         graph.replay()
     torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
+    ranks.barrier()
     g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     g0.record(stream)
     for _ in range(K):
@@ -352,11 +368,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
     st = kv.last_device_status()
     if st != 0:
         raise RuntimeError(f"device status {kv.STATUS_NAMES[st]} in the per-layer graph")
-    g_ms = g0.elapsed_time(g1) / K
-    if dist:
-        t = torch.tensor([g_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        g_ms = float(t[0])
+    g_ms, = ranks.max(g0.elapsed_time(g1) / K)
     del graph
 
     # roofline of the dominant launch (kvpack_decode_attn), algorithmic bytes per launch
@@ -397,7 +409,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
         "e2e": {"value": round(e2e_value, 1), "unit": "query-tokens/s", "h2d_bytes_per_step": qbytes,
                 "d2h_bytes_per_step": obytes, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": 6 * K,   # per step: select, text (q~ projection + text tail), text statistics, visual, finish, mass
-        "per_layer_graph": {"value": round(world * w.batch / (g_ms / 1e3), 1), "unit": "query-tokens/s",
+        "per_layer_graph": {"value": round(whole_job_value(world, w.batch, g_ms), 1), "unit": "query-tokens/s",
                             "ms_per_step": round(g_ms, 4), "launches_per_step": 6 * n_layers, "text_len": L_g,
                             "mode": "per layer: kvpack_select + kvpack_decode_attn, captured in one CUDA graph"},
         "clocks": clk,
@@ -407,8 +419,8 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
     if args.compress and rank == 0:
         line["compress"] = bench_compress(kv, torch, w, dev)
+    ranks.barrier()
     if dist:
-        dist.barrier()
         dist.destroy_process_group()
     return line
 

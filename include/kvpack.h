@@ -131,8 +131,9 @@ kvpack_status kvpack_compress(const kvpack_dims *dims, int32_t n_layers,
  * decompressed cache; K and V are never materialised.  Accumulation is fp32;
  * out is rounded to bf16.  mass may be NULL.  0 <= L_text <= L_text_cap.
  * ws must hold kvpack_decode_workspace(dims, n_layers) bytes; contents on
- * entry do not matter.  Device status KVPACK_ERR_TIMEOUT if a wait between
- * the thread blocks sharing a unit expired (out and mass are then invalid).
+ * entry do not matter.  No thread block waits on another; device status
+ * KVPACK_ERR_TIMEOUT means a bounded wait for a copy into shared memory
+ * expired (out and mass are then invalid).
  */
 size_t kvpack_decode_workspace(const kvpack_dims *dims, int32_t n_layers);
 kvpack_status kvpack_decode_attn(const kvpack_dims *dims, int32_t n_layers,
@@ -153,8 +154,8 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *dims, int32_t n_layers,
  * can stall on device-wide synchronisation.  This entry point has no
  * counterpart in the paper; it only changes where the scratch lives.
  *
- * The scratch (rank-space queries, per-split partial results and arrival
- * counters) is a fixed array of KVPACK_NOALLOC_SCRATCH_BYTES compiled into
+ * The scratch (rank-space queries, per-chunk partial results, the units'
+ * softmax statistics and two work counters) is a fixed array of KVPACK_NOALLOC_SCRATCH_BYTES compiled into
  * the library as device memory.  Every GPU that loads the library holds
  * that array until the process exits.  The call itself allocates nothing
  * and calls no allocating routine.
@@ -166,8 +167,8 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *dims, int32_t n_layers,
  *   KVPACK_NOALLOC_SCRATCH_BYTES returns KVPACK_ERR_WORKSPACE and launches
  *   nothing; split the layers over several calls instead.
  * - All calls on a device share the one array, and it keeps the last call's
- *   contents.  The kernels rewrite every part they read, and clear the
- *   arrival counters themselves before use.  Calls that overlap on the GPU
+ *   contents.  The kernels rewrite every part they read, and the work
+ *   counters are cleared on the stream before use.  Calls that overlap on the GPU
  *   (two streams, or two threads with their own streams) race on the array
  *   and give wrong results: order them on one stream or with events.
  * Arguments and results are those of kvpack_decode_attn minus ws / ws_bytes.
