@@ -10,15 +10,16 @@
 // coefficients are summed in rank space and projected back through B_V once
 // per head.  K and V are never materialised.
 //
-// Four launches, each streaming its own bytes once:
-//   text_kernel    q~ = scale * log2(e) * B_K[:, 128 j(h) ..] q_h per (unit, KV head), split into
-//                  bf16 hi + lo; and the text tail (plain bf16 K/V) per (unit, KV head, chunk of
-//                  tokens): partial (max, sum, w = sum p V) per query head
-//   text_stats     the text tail's (max, sum) per head folded over its chunks, one warp per unit
-//   vis_kernel     the compressed visual tokens per (unit, split of tokens): partial
-//                  (max, sum, u = sum p C_V) per query head, then -- once every split
-//                  of the unit has published -- the attention mass of each token
-//   finish_kernel  combines the partials of a unit and projects: o_h = (u B_V + w) / l
+// Four of the decode call's five launches live here (the fifth, the attention
+// mass of every visual token, is mass.cuh), each streaming its own bytes once:
+//   text_kernel        q~ = scale * log2(e) * B_K[:, 128 j(h) ..] q_h per (unit, KV head), split
+//                      into bf16 hi + lo; and the text tail (plain bf16 K/V) per (unit, KV head,
+//                      chunk of tokens): partial (max, sum, w = sum p V) per query head
+//   text_stats_kernel  the text tail's (max, sum) per head folded over its chunks, one warp per unit
+//   vis_kernel         the compressed visual tokens per (unit, chunk of tokens), one warp per
+//                      item: partial (max, sum, u = sum p C_V) per query head
+//   finish_kernel      combines the partials of a unit and projects: o_h = (u B_V + w) / l, and
+//                      publishes the unit's (max, 1/sum) per head for the mass pass
 // Logits are kept in the log2 domain (the scale folds log2(e)).
 #pragma once
 
@@ -31,9 +32,8 @@
 namespace kvpack {
 namespace decode {
 
-constexpr int kMaxHeads = 32;
 constexpr int kTxtPart = 130;   // per (unit, text chunk, head): max, sum, w[128]
-constexpr int kVisPart = 66;    // per (unit, visual split, head): max, sum, u[64]
+constexpr int kVisPart = 66;    // per (unit, visual chunk, head): max, sum, u[64]
 
 // =================================================================== query block
 
