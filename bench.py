@@ -39,6 +39,9 @@ from synth import cases  # noqa: E402
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 POOL = 8   # distinct host-generated units tiled over the cache
+# kernels of ours launched per step: kvpack_select (1) + kvpack_decode_attn (q~/text, text statistics,
+# visual, finish, mass)
+LAUNCHES_PER_STEP = 6
 
 
 # ------------------------------------------------------------------ accounting
@@ -207,23 +210,12 @@ def build_cache(kv, torch, w: synth.Workload, Lcap: int, dev):
     return c
 
 
-def run_ours(args, w: synth.Workload, rank: int, world: int):
-    import torch
-    import rank_compressed_kv_b200 as kv
-
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    ranks = Ranks(dist, dev)
-
-    K, W = args.steps, args.warmup
+def measure_workload(kv, torch, w: synth.Workload, K: int, W: int, dev, ranks, world: int, headline: bool):
+    """Device-timed decode steps of one workload (select + decode over all layers), the same
+    steps as per-layer calls in one CUDA graph, and, for the headline workload, the end-to-end
+    leg with host buffers.  Returns the measurements as a dict."""
     T, L0 = w.T, w.text0
-    Lcap = L0 + W + K + 1
+    Lcap = L0 + W + 2 * K + 2
     k_hi = w.k_hi
     dims = kv.Dims(batch=w.batch, n_q_heads=w.n_q, n_kv_heads=w.n_kv, T_vis=T, L_text_cap=Lcap)
     n_layers = w.layers
@@ -233,7 +225,6 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
                                .view(np.int16)).view(torch.bfloat16).pin_memory() for s in range(NQ)]
     q_dev = [qh.to(dev) for qh in q_host]
     out = torch.empty(n_layers * w.batch, w.n_q, 128, dtype=torch.bfloat16, device=dev)
-    out_host = torch.empty_like(out, device="cpu").pin_memory()
     mass = torch.zeros(w.units, T, dtype=torch.float32, device=dev)
     nwords = (T + 31) // 32
     mask = torch.empty(w.units, nwords, dtype=torch.int32, device=dev)
@@ -245,19 +236,17 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
         kv.decode_attn(dims, n_layers, q, c["CK_lo"], c["CK_hi"], c["BK"], c["CV_lo"], c["CV_hi"], c["BV"],
                        c["K_text"], c["V_text"], L0 + step, mask, 1.0, out, mass, ws)
 
-    def step_fn(step, q):
-        kv.select(dims, n_layers, mass, None, 0.0, k_hi, mask)
-        decode(step, q)
-
     # step 0: all tokens at full rank (no previous mass), then warm-up steps
     decode(0, q_dev[0])
     for s in range(1, W + 1):
-        step_fn(s, q_dev[s % NQ])
+        kv.select(dims, n_layers, mass, None, 0.0, k_hi, mask)
+        decode(s, q_dev[s % NQ])
     torch.cuda.synchronize()
 
     # device-resident timed region: events per decode launch and around the whole run
     ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    local = dev.index if dev.index is not None else 0
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
@@ -277,76 +266,78 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
     clk = clocks.stop()
     st = kv.last_device_status()
     if st != 0:
-        raise RuntimeError(f"device status {kv.STATUS_NAMES[st]} during the timed region")
+        raise RuntimeError(f"device status {kv.STATUS_NAMES[st]} during the timed region ({w.name})")
     ms_total = ev0.elapsed_time(ev1)
     dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
     ms_total, dec_sum = ranks.max(ms_total, sum(dec_ms))
     ms_step = ms_total / K
-    value = whole_job_value(world, w.batch, ms_step)
+    res = {"w": w, "ms_step": ms_step, "dec_avg_ms": dec_sum / K, "clocks": clk, "wall": wall,
+           "L_mean": L0 + W + 1 + (K - 1) / 2.0}
 
-    # end-to-end through the public API with host buffers: every step's q comes from pinned host
-    # memory and its output goes back to pinned host memory.  The copies run on a second stream,
-    # double-buffered, so step i + 1's upload and step i's download overlap the computation, as a
-    # serving loop would run them; each step still moves its own bytes.  The text lengths are those
-    # of the device-timed steps, so the two numbers time the same work.
-    torch.cuda.synchronize()
-    ranks.barrier()
-    hs, ds = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)   # uploads, downloads
-    qd = [torch.empty_like(q_dev[0]) for _ in range(2)]
-    outd = [torch.empty_like(out) for _ in range(2)]
-    outh = [out_host, torch.empty_like(out, device="cpu").pin_memory()]
-    ev_q = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_d2h = [torch.cuda.Event() for _ in range(2)]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s_base = W + 1 + K
-    e0.record(stream)
-    hs.wait_event(e0)
-    with torch.cuda.stream(hs):
-        qd[0].copy_(q_host[s_base % NQ], non_blocking=True)
-        ev_q[0].record(hs)
-    for i in range(K):
-        s, b = s_base + i, i % 2
-        stream.wait_event(ev_q[b])
-        if i >= 2:
-            stream.wait_event(ev_d2h[b])        # outd[b] has been read back
-        kv.select(dims, n_layers, mass, None, 0.0, k_hi, mask)
-        kv.decode_attn(dims, n_layers, qd[b], c["CK_lo"], c["CK_hi"], c["BK"], c["CV_lo"], c["CV_hi"], c["BV"],
-                       c["K_text"], c["V_text"], min(L0 + W + 1 + i, Lcap), mask, 1.0, outd[b], mass, ws)
-        ev_done[b].record(stream)
-        if i + 1 < K:                            # next step's q, once step i - 1 has finished reading qd[1 - b]
-            with torch.cuda.stream(hs):
-                if i >= 1:
-                    hs.wait_event(ev_done[1 - b])
-                qd[1 - b].copy_(q_host[(s + 1) % NQ], non_blocking=True)
-                ev_q[1 - b].record(hs)
-        with torch.cuda.stream(ds):              # this step's output
-            ds.wait_event(ev_done[b])
-            outh[b].copy_(outd[b], non_blocking=True)
-            ev_d2h[b].record(ds)
-    stream.wait_event(ev_d2h[(K - 1) % 2])
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms, = ranks.max(e0.elapsed_time(e1) / K)
-    e2e_value = whole_job_value(world, w.batch, e2e_ms)
-    qbytes = q_host[0].numel() * 2
-    obytes = out.numel() * 2
+    if headline:
+        # end-to-end through the public API with host buffers: every step's q comes from pinned host
+        # memory and its output goes back to pinned host memory.  The copies run on a second stream,
+        # double-buffered, so step i + 1's upload and step i's download overlap the computation, as a
+        # serving loop would run them; each step still moves its own bytes.  The text lengths are those
+        # of the device-timed steps, so the two numbers time the same work.
+        out_host = torch.empty_like(out, device="cpu").pin_memory()
+        torch.cuda.synchronize()
+        ranks.barrier()
+        hs, ds = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)   # uploads, downloads
+        qd = [torch.empty_like(q_dev[0]) for _ in range(2)]
+        outd = [torch.empty_like(out) for _ in range(2)]
+        outh = [out_host, torch.empty_like(out, device="cpu").pin_memory()]
+        ev_q = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_d2h = [torch.cuda.Event() for _ in range(2)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s_base = W + 1 + K
+        e0.record(stream)
+        hs.wait_event(e0)
+        with torch.cuda.stream(hs):
+            qd[0].copy_(q_host[s_base % NQ], non_blocking=True)
+            ev_q[0].record(hs)
+        for i in range(K):
+            s, b = s_base + i, i % 2
+            stream.wait_event(ev_q[b])
+            if i >= 2:
+                stream.wait_event(ev_d2h[b])        # outd[b] has been read back
+            kv.select(dims, n_layers, mass, None, 0.0, k_hi, mask)
+            kv.decode_attn(dims, n_layers, qd[b], c["CK_lo"], c["CK_hi"], c["BK"], c["CV_lo"], c["CV_hi"],
+                           c["BV"], c["K_text"], c["V_text"], L0 + W + 1 + i, mask, 1.0, outd[b], mass, ws)
+            ev_done[b].record(stream)
+            if i + 1 < K:                            # next step's q, once step i - 1 has finished reading qd[1 - b]
+                with torch.cuda.stream(hs):
+                    if i >= 1:
+                        hs.wait_event(ev_done[1 - b])
+                    qd[1 - b].copy_(q_host[(s + 1) % NQ], non_blocking=True)
+                    ev_q[1 - b].record(hs)
+            with torch.cuda.stream(ds):              # this step's output
+                ds.wait_event(ev_done[b])
+                outh[b].copy_(outd[b], non_blocking=True)
+                ev_d2h[b].record(ds)
+        stream.wait_event(ev_d2h[(K - 1) % 2])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms, = ranks.max(e0.elapsed_time(e1) / K)
+        res["e2e_ms"] = e2e_ms
+        res["h2d"] = q_host[0].numel() * 2
+        res["d2h"] = out.numel() * 2
 
     # per-layer launches, as a framework that runs attention layer by layer would call the
     # library: one kvpack_select and one kvpack_decode_attn per layer (layer slices of the same
     # buffers), captured once into a CUDA graph and replayed K times; the text length stays at the
     # captured value
     upl = w.units_per_layer
-    dims1 = kv.Dims(batch=w.batch, n_q_heads=w.n_q, n_kv_heads=w.n_kv, T_vis=T, L_text_cap=Lcap)
-    ws1 = torch.empty(kv.decode_workspace(dims1, 1), dtype=torch.uint8, device=dev)
-    L_g = min(L0 + W + 1 + 2 * K, Lcap)
+    ws1 = torch.empty(kv.decode_workspace(dims, 1), dtype=torch.uint8, device=dev)
+    L_g = L0 + W + 1 + 2 * K
     qg = q_dev[0]
 
     def per_layer_step():
         for l in range(n_layers):
             u0, u1, r0, r1 = l * upl, (l + 1) * upl, l * w.batch, (l + 1) * w.batch
-            kv.select(dims1, 1, mass[u0:u1], None, 0.0, k_hi, mask[u0:u1])
-            kv.decode_attn(dims1, 1, qg[r0:r1], c["CK_lo"][u0:u1], c["CK_hi"][u0:u1], c["BK"][u0:u1],
+            kv.select(dims, 1, mass[u0:u1], None, 0.0, k_hi, mask[u0:u1])
+            kv.decode_attn(dims, 1, qg[r0:r1], c["CK_lo"][u0:u1], c["CK_hi"][u0:u1], c["BK"][u0:u1],
                            c["CV_lo"][u0:u1], c["CV_hi"][u0:u1], c["BV"][u0:u1], c["K_text"][u0:u1],
                            c["V_text"][u0:u1], L_g, mask[u0:u1], 1.0, out[r0:r1], mass[u0:u1], ws1)
 
@@ -367,17 +358,68 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
     torch.cuda.synchronize()
     st = kv.last_device_status()
     if st != 0:
-        raise RuntimeError(f"device status {kv.STATUS_NAMES[st]} in the per-layer graph")
+        raise RuntimeError(f"device status {kv.STATUS_NAMES[st]} in the per-layer graph ({w.name})")
     g_ms, = ranks.max(g0.elapsed_time(g1) / K)
     del graph
+    res["graph_ms"] = g_ms
+    res["L_graph"] = L_g
+    del c, ws, ws1
+    torch.cuda.empty_cache()
+    return res
 
-    # roofline of the dominant launch (kvpack_decode_attn), algorithmic bytes per launch
+
+def roofline_block(w: synth.Workload, L_mean: float, dec_avg_ms: float):
+    """Roofline of the dominant call (kvpack_decode_attn): algorithmic bytes per launch over its
+    CUDA-event duration, against the measured copy bandwidth."""
     hbm, _, peak_kind = measured_peaks()
-    L_mean = L0 + W + 1 + (K - 1) / 2.0
-    dbytes = decode_bytes(w, L_mean, k_hi)
-    dec_avg_ms = dec_sum / K
+    dbytes = decode_bytes(w, L_mean, w.k_hi)
     achieved = dbytes / (dec_avg_ms / 1e3) / 1e9
-    sbytes = step_bytes(w, L_mean, k_hi)
+    return {"bound": "hbm",
+            "kernel": "kvpack_decode_attn (all of its kernels on one stream)",
+            "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "frac_of_8TBps": round(achieved / 8000.0, 4),
+            "peak_kind": peak_kind,
+            "bytes_per_launch": int(dbytes), "avg_launch_ms": round(dec_avg_ms, 4),
+            "traffic": recorded_traffic("decode", w.name)}
+
+
+def config_block(res, world: int):
+    """The per-workload summary that goes under "configs" in the bench line."""
+    w = res["w"]
+    return {"workload": f"{w.name}: batch {w.batch} x {w.layers} layers, {w.n_q} q / {w.n_kv} kv heads, "
+                        f"T={w.T} visual + {w.text0}+step text, top {round(w.hi_frac * 100)}% full rank",
+            "value": round(whole_job_value(world, w.batch, res["ms_step"]), 1), "unit": "query-tokens/s",
+            "ms_per_step": round(res["ms_step"], 4),
+            "us_per_decode_call": round(res["dec_avg_ms"] * 1e3, 1),
+            "roofline": roofline_block(w, res["L_mean"], res["dec_avg_ms"]),
+            "per_layer_graph": {"value": round(whole_job_value(world, w.batch, res["graph_ms"]), 1),
+                                "ms_per_step": round(res["graph_ms"], 4), "text_len": res["L_graph"]},
+            "clocks": res["clocks"]}
+
+
+EXTRA_CONFIGS = (("C2", 0.25), ("C3", 0.25), ("C4", 0.25), ("C4", 0.10))
+
+
+def run_ours(args, w: synth.Workload, rank: int, world: int):
+    import torch
+    import rank_compressed_kv_b200 as kv
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    ranks = Ranks(dist, dev)
+
+    K, W = args.steps, args.warmup
+    res = measure_workload(kv, torch, w, K, W, dev, ranks, world, headline=True)
+    ms_step = res["ms_step"]
+    value = whole_job_value(world, w.batch, ms_step)
+    L_mean = res["L_mean"]
+    sbytes = step_bytes(w, L_mean, w.k_hi)
     line = {
         "metric": "compressed-KV decode attn query-tokens/s and achieved HBM GB/s vs 8 TB/s peak",
         "value": round(value, 1),
@@ -392,33 +434,39 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
         "dtype": "bf16",
         "data": "synthetic (seeded low-rank-plus-noise compressed cache, 8 generated units tiled)",
         "config": {"workload": f"{w.name}: batch {w.batch} x {w.layers} layers, {w.n_q} q / {w.n_kv} kv heads, "
-                               f"T={T} visual + {L0}+step text, r=64/16, top {int(w.hi_frac * 100)}% full rank",
+                               f"T={w.T} visual + {w.text0}+step text, r=64/16, top {round(w.hi_frac * 100)}% full rank",
                    "global_batch": world * w.batch, "units": w.units, "hi_frac": w.hi_frac,
                    "parallelism": f"dp{world}" if world > 1 else "single-gpu",
                    "l2": "inputs larger than L2 (no flush needed)",
                    "step": "kvpack_select + kvpack_decode_attn over all layers"},
         "step_bytes": int(sbytes),
         "step_GBps": round(sbytes / (ms_step / 1e3) / 1e9, 1),
-        "roofline": {"bound": "hbm",
-                     "kernel": "kvpack_decode_attn (text_kernel, text_stats_kernel, vis_kernel, finish_kernel, mass_kernel on one stream)",
-                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "frac_of_8TBps": round(achieved / 8000.0, 4),
-                     "peak_kind": peak_kind,
-                     "bytes_per_launch": int(dbytes), "avg_launch_ms": round(dec_avg_ms, 4),
-                     "traffic": recorded_traffic("decode", w.name)},
-        "e2e": {"value": round(e2e_value, 1), "unit": "query-tokens/s", "h2d_bytes_per_step": qbytes,
-                "d2h_bytes_per_step": obytes, "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": 6 * K,   # per step: select, text (q~ projection + text tail), text statistics, visual, finish, mass
-        "per_layer_graph": {"value": round(whole_job_value(world, w.batch, g_ms), 1), "unit": "query-tokens/s",
-                            "ms_per_step": round(g_ms, 4), "launches_per_step": 6 * n_layers, "text_len": L_g,
+        "roofline": roofline_block(w, L_mean, res["dec_avg_ms"]),
+        "e2e": {"value": round(whole_job_value(world, w.batch, res["e2e_ms"]), 1), "unit": "query-tokens/s",
+                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
+                "ms_per_step": round(res["e2e_ms"], 4)},
+        "gpu_launches": LAUNCHES_PER_STEP * K,
+        "per_layer_graph": {"value": round(whole_job_value(world, w.batch, res["graph_ms"]), 1),
+                            "unit": "query-tokens/s", "ms_per_step": round(res["graph_ms"], 4),
+                            "launches_per_step": LAUNCHES_PER_STEP * w.layers, "text_len": res["L_graph"],
                             "mode": "per layer: kvpack_select + kvpack_decode_attn, captured in one CUDA graph"},
-        "clocks": clk,
-        "wall_s_timed": round(wall, 3),
+        "clocks": res["clocks"],
+        "wall_s_timed": round(res["wall"], 3),
     }
+    if not args.headline_only:
+        # the workloads the HBM-roofline target is set on, measured the same way (device-resident,
+        # CUDA events, max over ranks); the headline value above stays the first workload's
+        K2 = max(10, min(K, args.config_steps))
+        blocks = {}
+        for name, f in EXTRA_CONFIGS:
+            wx = synth.WORKLOADS[name].with_hi_frac(f)
+            blocks[f"{name}@{round(f * 100)}%"] = config_block(
+                measure_workload(kv, torch, wx, K2, W, dev, ranks, world, headline=False), world)
+        line["configs"] = blocks
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
-    if args.compress and rank == 0:
-        line["compress"] = bench_compress(kv, torch, w, dev)
+    if not args.no_compress and rank == 0:
+        line["compress"] = {n: bench_compress(kv, torch, synth.WORKLOADS[n], dev) for n in ("C2", "C4")}
     ranks.barrier()
     if dist:
         dist.destroy_process_group()
@@ -426,8 +474,10 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
 
 
 def bench_compress(kv, torch, w, dev):
-    """kvpack_compress on one layer of the workload (K side), timed with CUDA events; per-kernel
-    device times from the CUDA profiler give the Gram's rate against the measured bf16 peak."""
+    """kvpack_compress on one layer of the workload (K side: batch x groups units), timed with CUDA
+    events; per-kernel device times from the CUDA profiler give the Gram's rate against the measured
+    bf16 peak.  The Gram's algorithmic count is the symmetric rank-k update T n (n + 1) per matrix
+    (the kernel computes the upper 128-row bands and mirrors them)."""
     from torch.profiler import profile, ProfilerActivity
     units = w.batch * (w.n_kv // 4)
     dims = kv.Dims(batch=units, n_q_heads=4, n_kv_heads=4, T_vis=w.T, L_text_cap=1)
@@ -458,19 +508,24 @@ def bench_compress(kv, torch, w, dev):
     kern = {}
     for e in prof.events():
         if e.device_type.name == "CUDA":
-            name = e.name.split("(")[0].split("::")[-1]
+            name = e.name.split("(")[0].split("::")[-1].split("<")[0]
             kern[name] = kern.get(name, 0.0) + e.device_time_total / 1e3
     _, bf16, peak_kind = measured_peaks()
     gram_ms = kern.get("gram_tc_kernel", float("nan"))
-    full = 2.0 * units * w.T * 512 * 512                  # the full product X^T X
-    executed = full * (128 * (512 + 384 + 256 + 128)) / (512 * 512)   # upper bands as computed
-    return {"units": units, "T": w.T, "ms_per_layer_matrix": round(e0.elapsed_time(e1), 3), "status": st,
+    n = 512
+    syrk = float(units) * w.T * n * (n + 1)                 # symmetric rank-k update: the algorithmic count
+    full = 2.0 * units * w.T * n * n                         # the full product X^T X, for reference
+    tf = syrk / (gram_ms / 1e3) / 1e12
+    del X, C_lo, C_hi, B, sig, ws
+    torch.cuda.empty_cache()
+    return {"workload": f"{w.name}: one layer, K side, {units} units of T={w.T}", "units": units, "T": w.T,
+            "ms_per_layer_matrix": round(e0.elapsed_time(e1), 3), "status": kv.STATUS_NAMES.get(st, st),
             "kernel_ms": {k: round(v, 3) for k, v in kern.items()},
-            "gram": {"full_2Tn2_tflops": round(full / (gram_ms / 1e3) / 1e12, 1),
-                     "executed_tflops": round(executed / (gram_ms / 1e3) / 1e12, 1),
-                     "peak_tflops": bf16, "peak_kind": peak_kind,
-                     "frac_full_2Tn2": round(full / (gram_ms / 1e3) / 1e12 / bf16, 4),
-                     "frac_executed": round(executed / (gram_ms / 1e3) / 1e12 / bf16, 4)}}
+            "gram": {"bound": "tensor", "count": "SYRK T*n*(n+1) per matrix", "flops": syrk,
+                     "achieved": round(tf, 1), "unit": "TFLOP/s", "peak": bf16, "peak_kind": peak_kind,
+                     "frac": round(tf / bf16, 4),
+                     "full_product_tflops": round(full / (gram_ms / 1e3) / 1e12, 1),
+                     "kernel_ms": round(gram_ms, 4)}}
 
 
 # ------------------------------------------------------------------ oracle (CPU) arm
@@ -569,7 +624,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--compress", action="store_true", help="also time kvpack_compress on the workload")
+    ap.add_argument("--no-compress", action="store_true", help="skip the kvpack_compress block")
+    ap.add_argument("--headline-only", action="store_true", help="measure the --config workload only")
+    ap.add_argument("--config-steps", type=int, default=50, help="timed steps of each extra workload")
+    ap.add_argument("--only-compress", action="store_true",
+                    help="time kvpack_compress on one layer of --config only (a small case for profiler captures)")
     ap.add_argument("--layers", type=int, default=None,
                     help="run the config with fewer layers (a small case for profiler captures; named in the line)")
     args = ap.parse_args()
@@ -589,6 +648,13 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args, w)), flush=True)
+        return
+    if args.only_compress:
+        import torch
+        import rank_compressed_kv_b200 as kv
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        print(json.dumps(bench_compress(kv, torch, w, torch.device("cuda", torch.cuda.current_device()))),
+              flush=True)
         return
     line = run_ours(args, w, rank, world)
     if rank == 0:

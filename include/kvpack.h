@@ -12,8 +12,8 @@
  * The cache is cut into independent UNITS.  A unit is one (layer l, batch
  * row b, KV-head group G): the K (or V) vectors of its g = 4 KV heads,
  * concatenated along the feature axis, form one T x 512 matrix that is
- * compressed by one SVD ("the heads are merged before the SVD", Methodologie
- * 2.A on the fr page).  Unit index: u = (l * batch + b) * n_groups + G, with
+ * compressed by one SVD (multi-head compression joins a group's heads before
+ * factoring: Methodologie 2.A on the fr page).  Unit index: u = (l * batch + b) * n_groups + G, with
  * n_groups = n_kv_heads / 4, so one layer is a contiguous run of units.
  * Query head h of (l, b) belongs to group G = h / Hg, Hg = 4 * n_q / n_kv,
  * and within its group reads KV head j(h) = (h % Hg) / (n_q / n_kv).
@@ -155,14 +155,18 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *dims, int32_t n_layers,
  * counterpart in the paper; it only changes where the scratch lives.
  *
  * The scratch (rank-space queries, per-chunk partial results, the units'
- * softmax statistics and two work counters) is a fixed array of KVPACK_NOALLOC_SCRATCH_BYTES compiled into
- * the library as device memory.  Every GPU that loads the library holds
- * that array until the process exits.  The call itself allocates nothing
- * and calls no allocating routine.
+ * softmax statistics and the work counters) is a fixed array of
+ * KVPACK_NOALLOC_SCRATCH_BYTES compiled into the library as device memory.
+ * The call itself allocates nothing and calls no allocating routine.
  *
- * - The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current) and sets the kernels'
- *   attributes; make that first call before any stream capture.
+ * - Where the array lives: CUDA loads the library's device code, and places
+ *   the array, on a device the first time any kvpack call runs there (lazy
+ *   module loading, the default); from then on that GPU holds the array
+ *   until the process exits.  Make one kvpack call per device at start-up,
+ *   before any stream capture, so that this happens outside the serving loop.
+ * - Every call looks the array's device address up afresh (with the
+ *   caller's device current), so a context that was torn down and created
+ *   again (cudaDeviceReset) is handled like a first use.
  * - A call whose kvpack_decode_workspace(dims, n_layers) exceeds
  *   KVPACK_NOALLOC_SCRATCH_BYTES returns KVPACK_ERR_WORKSPACE and launches
  *   nothing; split the layers over several calls instead.
@@ -172,6 +176,7 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *dims, int32_t n_layers,
  *   (two streams, or two threads with their own streams) race on the array
  *   and give wrong results: order them on one stream or with events.
  * Arguments and results are those of kvpack_decode_attn minus ws / ws_bytes.
+ * kvpack_noalloc_scratch_bytes() returns KVPACK_NOALLOC_SCRATCH_BYTES.
  */
 #define KVPACK_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 kvpack_status kvpack_decode_attn_noalloc(const kvpack_dims *dims, int32_t n_layers,
@@ -181,6 +186,7 @@ kvpack_status kvpack_decode_attn_noalloc(const kvpack_dims *dims, int32_t n_laye
                                          const uint16_t *K_text, const uint16_t *V_text, int32_t L_text,
                                          const uint32_t *mask, float softmax_scale,
                                          uint16_t *out, float *mass, void *stream);
+size_t kvpack_noalloc_scratch_bytes(void);
 
 /* ------------------------------------------------------------------ rank choice
  * kvpack_select -- importance update and rank mask for the next step, every

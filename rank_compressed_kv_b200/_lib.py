@@ -82,6 +82,7 @@ _L.kvpack_decode_attn.restype = ctypes.c_int
 _L.kvpack_decode_attn_noalloc.argtypes = [_dims_p, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                           _vp, ctypes.c_float, _vp, _vp, _vp]
 _L.kvpack_decode_attn_noalloc.restype = ctypes.c_int
+_L.kvpack_noalloc_scratch_bytes.restype = _sz
 _L.kvpack_select.argtypes = [_dims_p, _i32, _vp, _vp, ctypes.c_float, _i32, _vp, _vp]
 _L.kvpack_select.restype = ctypes.c_int
 
@@ -161,7 +162,7 @@ def decode_attn_noalloc(dims: Dims, n_layers: int, q, CK_lo, CK_hi, BK, CV_lo, C
            "kvpack_decode_attn_noalloc")
 
 
-NOALLOC_SCRATCH_BYTES = 64 << 20
+NOALLOC_SCRATCH_BYTES = int(_L.kvpack_noalloc_scratch_bytes())
 
 
 def select(dims: Dims, n_layers: int, mass, score, alpha: float, k_hi: int, mask_out, stream=None):

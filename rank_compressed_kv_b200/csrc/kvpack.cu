@@ -91,6 +91,7 @@ DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
 
 struct DeviceInfo {
     bool ready = false;
+    unsigned long long ctx_id = 0;       // the context the attributes below were set in
     int sms = 0;
     int mass_blocks[4] = {0, 0, 0, 0};   // resident blocks per SM of mass_kernel<1..4>
 };
@@ -122,12 +123,48 @@ cudaError_t launch_finish(int per_kv, const kvpack::decode::FinishParams &fp, in
     return cudaGetLastError();
 }
 
+// Unique id of the calling thread's current context (cuCtxGetId, looked up once through the
+// runtime).  Kernel attributes belong to a context: one torn down and created again
+// (cudaDeviceReset) needs them set afresh.
+kvpack_status current_context_id(unsigned long long *id) {
+    using GetCtx = CUresult (*)(CUcontext *);
+    using GetId = CUresult (*)(CUcontext, unsigned long long *);
+    static GetCtx get_ctx = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f1 = nullptr, *f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) == cudaSuccess &&
+            q2 == cudaDriverEntryPointSuccess) {
+            get_ctx = reinterpret_cast<GetCtx>(f1);
+            get_id = reinterpret_cast<GetId>(f2);
+        }
+    });
+    if (get_ctx == nullptr || get_id == nullptr) return KVPACK_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return KVPACK_ERR_CUDA;
+    if (ctx == nullptr) {   // a thread without a current context: bind the device's primary context
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return KVPACK_ERR_CUDA;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return KVPACK_ERR_CUDA;
+    }
+    if (get_id(ctx, id) != CUDA_SUCCESS) return KVPACK_ERR_CUDA;
+    return KVPACK_OK;
+}
+
 kvpack_status device_info(DeviceInfo **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVPACK_ERR_CUDA;
+    unsigned long long ctx_id = 0;
+    if (current_context_id(&ctx_id) != KVPACK_OK) return KVPACK_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_dev_mu);
     DeviceInfo &di = g_dev[dev];
-    if (!di.ready) {
+    if (!di.ready || di.ctx_id != ctx_id) {
+        di.ready = false;
+        di.ctx_id = ctx_id;
         if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return KVPACK_ERR_CUDA;
         namespace dc = kvpack::decode;
         if (cudaFuncSetAttribute(dc::vis::vis_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -409,35 +446,29 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
 //
 // For callers that cannot give the library device memory (a framework-owned
 // plugin with no workspace hook, a serving loop that bans allocator calls):
-// the decode scratch lives in this fixed device array, which every GPU that
-// loads the library holds until exit.  Host code must not pass the array's
-// name to a kernel -- on the host it is only a stand-in -- so its device
-// address is looked up once per device and cached.
+// the decode scratch lives in this fixed device array, which every GPU holds
+// from the library's first use there until exit.  Host code must not pass the
+// array's name to a kernel -- on the host it is only a stand-in -- so its
+// device address is looked up with the caller's device current.  The lookup
+// runs on every call and is not cached: a context torn down and created
+// again (cudaDeviceReset) places the array at a new address.
 
 namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[KVPACK_NOALLOC_SCRATCH_BYTES];
 
-void *g_noalloc_addr[kMaxDevices];
-std::mutex g_noalloc_mu;
-
-// First call on a device: look the array up with that device current.
 kvpack_status noalloc_scratch(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVPACK_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (g_noalloc_addr[dev] == nullptr) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KVPACK_ERR_CUDA;
-        g_noalloc_addr[dev] = p;
-    }
-    *out = g_noalloc_addr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KVPACK_ERR_CUDA;
+    *out = p;
     return KVPACK_OK;
 }
 
 }  // namespace
 
 extern "C" {
+
+size_t kvpack_noalloc_scratch_bytes(void) { return KVPACK_NOALLOC_SCRATCH_BYTES; }
 
 kvpack_status kvpack_decode_attn_noalloc(const kvpack_dims *d, int32_t n_layers, const uint16_t *q,
                                          const uint16_t *CK_lo, const uint16_t *CK_hi, const uint16_t *BK,

@@ -1,8 +1,8 @@
 """Parity at the workloads' full sizes, in the launch configuration bench.py times.
 
 * decode + select over every unit of C1..C4 (the bench's device cache: eight
-  generated units tiled over all units, a 25 % rank mask chosen by
-  kvpack_select from a random mass): selection bit-exact against the oracle's
+  generated units tiled over all units, a 25 % rank mask -- and 10 % for C4's
+  sweep -- chosen by kvpack_select from a random mass): selection bit-exact against the oracle's
   on the same fp32 mass, outputs and attention mass against the fp64 oracle
   on sampled units (first, last, middle and an odd unit), and, on every unit,
   properties that hold at any size (finite outputs; mass >= 0 summing to at
@@ -48,10 +48,10 @@ def _oracle_units(w, pool, units, q_np, mask_np, T, L):
     return oracle.decode(CK, BK, CV, BV, Kt, Vt, mask_np, qu)
 
 
-@pytest.mark.parametrize("name", ["C1", "C2", "C3", "C4"])
-def test_decode_and_select_at_full_size(name):
+@pytest.mark.parametrize("name,hi_frac", [("C1", 0.25), ("C2", 0.25), ("C3", 0.25), ("C4", 0.25), ("C4", 0.10)])
+def test_decode_and_select_at_full_size(name, hi_frac):
     import rank_compressed_kv_b200 as kv
-    w = synth.WORKLOADS[name]
+    w = synth.WORKLOADS[name].with_hi_frac(hi_frac)
     T, U, Lcap, L = w.T, w.units, w.text0 + 2, w.text0 + 1
     dims = kv.Dims(batch=w.batch, n_q_heads=w.n_q, n_kv_heads=w.n_kv, T_vis=T, L_text_cap=Lcap)
     c = bench.build_cache(kv, torch, w, Lcap, DEV)

@@ -185,3 +185,30 @@ def test_large_logits_do_not_overflow():
     CK, BK, CV, BV, Kt, Vt, mask, q, bits = _rand_unit(6, T, L, Hg)
     o, m = oracle.decode(CK, BK, CV, BV, Kt, Vt, mask, q * 1e5)
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(m))
+
+
+def test_rank_zero_tokens_act_as_zero_key_and_value():
+    """r_lo = 0 (a low-importance token is not decompressed at all, de summary 2.B): such a
+    token's reconstruction is zero, so the step equals a full-rank step in which those tokens'
+    coefficients are zero; all of them get the same mass."""
+    T, L, Hg = 45, 6, 8
+    CK, BK, CV, BV, Kt, Vt, mask, q, bits = _rand_unit(77, T, L, Hg)
+    out0, mass0 = oracle.decode(CK, BK, CV, BV, Kt, Vt, mask, q, r_lo=0)
+    CKz, CVz = CK.copy(), CV.copy()
+    CKz[0, ~bits] = 0.0
+    CVz[0, ~bits] = 0.0
+    ones = np.full_like(mask, 0xFFFFFFFF)
+    ref_o, ref_m = oracle.decode(CKz, BK, CVz, BV, Kt, Vt, ones, q, r_lo=64)
+    np.testing.assert_allclose(out0, ref_o, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(mass0, ref_m, rtol=1e-12, atol=1e-16)
+    m_low = mass0[0, ~bits]
+    assert np.all(np.abs(m_low - m_low[0]) <= 1e-15 * abs(m_low[0]))
+
+
+def test_all_rank_zero_without_text_is_uniform_and_zero():
+    T, Hg = 37, 4
+    CK, BK, CV, BV, Kt, Vt, mask, q, bits = _rand_unit(3, T, 0, Hg)
+    zero = np.zeros_like(mask)
+    out, mass = oracle.decode(CK, BK, CV, BV, Kt, Vt, zero, q, r_lo=0)
+    assert np.all(out == 0.0)
+    np.testing.assert_allclose(mass[0], np.full(T, Hg / T), rtol=1e-14)
