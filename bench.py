@@ -104,7 +104,7 @@ def whole_job_value(world: int, batch: int, ms_per_step: float) -> float:
     return world * batch / (ms_per_step / 1e3)
 
 
-DECODE_SOURCES = ("decode.cuh", "mass.cuh", "common.cuh", "kvpack.cu")
+DECODE_SOURCES = ("decode.cuh", "rstream.cuh", "common.cuh", "kvpack.cu")
 
 
 def sources_digest(names=DECODE_SOURCES) -> str:
@@ -210,7 +210,8 @@ def build_cache(kv, torch, w: synth.Workload, Lcap: int, dev):
     return c
 
 
-def measure_workload(kv, torch, w: synth.Workload, K: int, W: int, dev, ranks, world: int, headline: bool):
+def measure_workload(kv, torch, w: synth.Workload, K: int, W: int, dev, ranks, world: int, headline: bool,
+                     baselines: bool = False):
     """Device-timed decode steps of one workload (select + decode over all layers), the same
     steps as per-layer calls in one CUDA graph, and, for the headline workload, the end-to-end
     leg with host buffers.  Returns the measurements as a dict."""
@@ -363,9 +364,75 @@ def measure_workload(kv, torch, w: synth.Workload, K: int, W: int, dev, ranks, w
     del graph
     res["graph_ms"] = g_ms
     res["L_graph"] = L_g
-    del c, ws, ws1
+    del ws1
+    if baselines:
+        res["baselines"] = measure_baselines(kv, torch, w, dims, c, mask, q_dev[0], out, ws, L0 + W + 1, dev, ranks,
+                                             max(3, min(K, 10)))
+    del c, ws
     torch.cuda.empty_cache()
     return res
+
+
+def measure_baselines(kv, torch, w, dims, c, mask, q, out, ws, L_text, dev, ranks, K):
+    """The rank-space decode call against the two routes it replaces, on the same cache, mask and
+    query: standard attention over the uncompressed bf16 cache (T + L tokens, built here by
+    decompressing every token at full rank), and decompress-then-attend (materialise K^ and V^ at
+    each token's rank, then the same dense attention).  CUDA events around K calls of each."""
+    n_layers, T = w.layers, w.T
+    U = w.units
+    Lc = T + L_text
+    dims_full = kv.Dims(batch=w.batch, n_q_heads=w.n_q, n_kv_heads=w.n_kv, T_vis=T, L_text_cap=dims.L_text_cap)
+    Kd = torch.empty((U, Lc, 4, 128), dtype=torch.bfloat16, device=dev)
+    Vd = torch.empty((U, Lc, 4, 128), dtype=torch.bfloat16, device=dev)
+    Kd[:, T:].copy_(c["K_text"][:, :L_text])
+    Vd[:, T:].copy_(c["V_text"][:, :L_text])
+    ones = torch.full_like(mask, -1)
+    kv.decompress(dims_full, n_layers, c["CK_lo"], c["CK_hi"], c["BK"], c["CV_lo"], c["CV_hi"], c["BV"], ones,
+                  Kd, Vd, Lc)
+    wsd = torch.empty(kv.dense_decode_workspace(dims, n_layers, Lc), dtype=torch.uint8, device=dev)
+    mass = torch.empty(U, T, dtype=torch.float32, device=dev)
+
+    def rank_space():
+        kv.decode_attn(dims, n_layers, q, c["CK_lo"], c["CK_hi"], c["BK"], c["CV_lo"], c["CV_hi"], c["BV"],
+                       c["K_text"], c["V_text"], L_text, mask, 1.0, out, mass, ws)
+
+    def dense():
+        kv.dense_decode_attn(dims, n_layers, q, Kd, Vd, Lc, Lc, 1.0, out, wsd)
+
+    def decompress_then_attend():
+        kv.decompress(dims, n_layers, c["CK_lo"], c["CK_hi"], c["BK"], c["CV_lo"], c["CV_hi"], c["BV"], mask,
+                      Kd, Vd, Lc)
+        kv.dense_decode_attn(dims, n_layers, q, Kd, Vd, Lc, Lc, 1.0, out, wsd)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        ranks.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms, = ranks.max(e0.elapsed_time(e1) / K)
+        return ms
+
+    r_ms = timed(rank_space)
+    d_ms = timed(dense)
+    dta_ms = timed(decompress_then_attend)
+    st = kv.last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {kv.STATUS_NAMES[st]} in the baselines ({w.name})")
+    hbm, _, _ = measured_peaks()
+    dense_bytes = U * Lc * 512 * 2 * 2 + 2 * U * w.Hg * 128 * 2
+    del Kd, Vd, wsd
+    torch.cuda.empty_cache()
+    return {"text_len": L_text, "calls_timed": K,
+            "rank_space_ms": round(r_ms, 4), "dense_ms": round(d_ms, 4), "decompress_then_attend_ms": round(dta_ms, 4),
+            "speedup_vs_dense": round(d_ms / r_ms, 2), "speedup_vs_decompress_then_attend": round(dta_ms / r_ms, 2),
+            "dense_GBps": round(dense_bytes / (d_ms / 1e3) / 1e9, 1), "dense_frac": round(dense_bytes / (d_ms / 1e3) / 1e9 / hbm, 4),
+            "note": "rank-space call also writes the attention mass; the baselines write the output only"}
 
 
 def roofline_block(w: synth.Workload, L_mean: float, dec_avg_ms: float):
@@ -394,7 +461,8 @@ def config_block(res, world: int):
             "roofline": roofline_block(w, res["L_mean"], res["dec_avg_ms"]),
             "per_layer_graph": {"value": round(whole_job_value(world, w.batch, res["graph_ms"]), 1),
                                 "ms_per_step": round(res["graph_ms"], 4), "text_len": res["L_graph"]},
-            "clocks": res["clocks"]}
+            "clocks": res["clocks"],
+            "baselines": res.get("baselines")}
 
 
 EXTRA_CONFIGS = (("C2", 0.25), ("C3", 0.25), ("C4", 0.25), ("C4", 0.10))
@@ -415,7 +483,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
     ranks = Ranks(dist, dev)
 
     K, W = args.steps, args.warmup
-    res = measure_workload(kv, torch, w, K, W, dev, ranks, world, headline=True)
+    res = measure_workload(kv, torch, w, K, W, dev, ranks, world, headline=True, baselines=not args.no_baselines)
     ms_step = res["ms_step"]
     value = whole_job_value(world, w.batch, ms_step)
     L_mean = res["L_mean"]
@@ -452,6 +520,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
                             "mode": "per layer: kvpack_select + kvpack_decode_attn, captured in one CUDA graph"},
         "clocks": res["clocks"],
         "wall_s_timed": round(res["wall"], 3),
+        "baselines": res.get("baselines"),
     }
     if not args.headline_only:
         # the workloads the HBM-roofline target is set on, measured the same way (device-resident,
@@ -461,7 +530,8 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
         for name, f in EXTRA_CONFIGS:
             wx = synth.WORKLOADS[name].with_hi_frac(f)
             blocks[f"{name}@{round(f * 100)}%"] = config_block(
-                measure_workload(kv, torch, wx, K2, W, dev, ranks, world, headline=False), world)
+                measure_workload(kv, torch, wx, K2, W, dev, ranks, world, headline=False,
+                                 baselines=not args.no_baselines), world)
         line["configs"] = blocks
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
@@ -626,6 +696,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-compress", action="store_true", help="skip the kvpack_compress block")
     ap.add_argument("--headline-only", action="store_true", help="measure the --config workload only")
+    ap.add_argument("--no-baselines", action="store_true", help="skip the dense and decompress-then-attend baselines")
     ap.add_argument("--config-steps", type=int, default=50, help="timed steps of each extra workload")
     ap.add_argument("--only-compress", action="store_true",
                     help="time kvpack_compress on one layer of --config only (a small case for profiler captures)")

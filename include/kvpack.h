@@ -77,7 +77,10 @@ typedef enum {
 
 /*
  * Shape of the cache.  Supported: group == 4, head_dim == 128, rank == 64,
- * rank_lo == 16, n_kv_heads a positive multiple of 4, n_q_heads a positive
+ * rank_lo == 16 (a low-importance token is decompressed at rank 16), or
+ * rank_lo == 0 (it is not decompressed at all: its key and value are taken as
+ * zero -- the variant of Methodik 2.B on the de page; the coefficient layout is
+ * the same), n_kv_heads a positive multiple of 4, n_q_heads a positive
  * multiple of n_kv_heads with Hg = 4 * n_q / n_kv <= 32, batch >= 1,
  * 1 <= T_vis <= KVPACK_MAX_T, 0 <= L_text_cap <= KVPACK_MAX_TEXT.
  */
@@ -121,7 +124,7 @@ kvpack_status kvpack_compress(const kvpack_dims *dims, int32_t n_layers,
  * page: high-score tokens are decompressed at the full rank R_kv, the others
  * at R_kv/4).  For each query head h of the unit, j = j(h):
  *   q~_h    = B_K[:, 128 j : 128 j + 128] q_h                       (rank space, 64)
- *   rho_t   = 64 if mask bit t else 16
+ *   rho_t   = 64 if mask bit t else dims.rank_lo (16, or 0: logit 0, no value)
  *   s_h,t   = scale * sum_{i < rho_t} C_K[t, i] q~_h[i]             (visual, t < T)
  *   s_h,T+u = scale * q_h . K_text[u, j]                           (text, u < L_text)
  *   p_h     = softmax over the T + L_text logits
@@ -131,7 +134,8 @@ kvpack_status kvpack_compress(const kvpack_dims *dims, int32_t n_layers,
  * decompressed cache; K and V are never materialised.  Accumulation is fp32;
  * out is rounded to bf16.  mass may be NULL.  0 <= L_text <= L_text_cap.
  * ws must hold kvpack_decode_workspace(dims, n_layers) bytes; contents on
- * entry do not matter.  No thread block waits on another; device status
+ * entry do not matter.  The work split depends on the shapes alone, so
+ * repeated calls give identical bits.  No thread block waits on another; device status
  * KVPACK_ERR_TIMEOUT means a bounded wait for a copy into shared memory
  * expired (out and mass are then invalid).
  */
@@ -204,6 +208,38 @@ kvpack_status kvpack_select(const kvpack_dims *dims, int32_t n_layers,
                             const float *mass, float *score, float alpha, int32_t k_hi,
                             uint32_t *mask_out, void *stream);
 
+/* ------------------------------------------------------------------ baselines
+ * The two routes the rank-space decode is measured against.  The fr summary
+ * (§4, results) credits the method's fused kernels with a 2.4x lower latency
+ * than a standard implementation; these entry points give that comparison a
+ * B200 counterpart.  They share the text kernel's streaming attention.
+ *
+ * kvpack_dense_decode_attn -- standard decode attention over an uncompressed
+ * bf16 cache: for each query head h of a unit (KV head j = j(h)),
+ *   o_h = softmax_u(scale * q_h . K[u, j]) V[u, j]   over the first L rows
+ * of K, V [units][L_cap][4][128] (visual and text tokens alike).  ws must hold
+ * kvpack_dense_decode_workspace(dims, n_layers, L_cap) bytes.  1 <= L <= L_cap
+ * <= 4 * KVPACK_MAX_T.  dims.T_vis is not used beyond argument checks.
+ *
+ * kvpack_decompress -- decompress every visual token at its own rank, the
+ * first half of the decompress-then-attend route (fr summary 2.B):
+ *   K^_t = sum_{i < rho_t} C_K[t, i] B_K[i, :],  V^_t likewise,
+ *   rho_t = 64 if mask bit t, else dims.rank_lo (16, or 0 for tokens that are
+ *   not decompressed at all)
+ * written in bf16 (round to nearest even, fp32 accumulation) to rows 0 .. T-1
+ * of K_out, V_out [units][L_cap][4][128]; rows T .. L_cap-1 are left as they
+ * are (the caller's text tail), so kvpack_dense_decode_attn over T + L_text
+ * rows then attends over the decompressed cache.  L_cap >= T_vis.
+ */
+size_t kvpack_dense_decode_workspace(const kvpack_dims *dims, int32_t n_layers, int32_t L_cap);
+kvpack_status kvpack_dense_decode_attn(const kvpack_dims *dims, int32_t n_layers, const uint16_t *q,
+                                       const uint16_t *K, const uint16_t *V, int32_t L_cap, int32_t L,
+                                       float softmax_scale, uint16_t *out, void *ws, size_t ws_bytes, void *stream);
+kvpack_status kvpack_decompress(const kvpack_dims *dims, int32_t n_layers,
+                                const uint16_t *CK_lo, const uint16_t *CK_hi, const uint16_t *BK,
+                                const uint16_t *CV_lo, const uint16_t *CV_hi, const uint16_t *BV,
+                                const uint32_t *mask, uint16_t *K_out, uint16_t *V_out, int32_t L_cap, void *stream);
+
 /* ------------------------------------------------------------------ helpers */
 
 /* Human-readable name of a status. */
@@ -224,6 +260,17 @@ kvpack_status kvpack_last_device_status(void *stream);
 kvpack_status kvpack_footprint(const kvpack_dims *dims, int32_t n_layers, int32_t L_text, uint64_t out[3]);
 
 int32_t kvpack_version(void);
+
+/*
+ * Diagnostic, no counterpart in the paper: checks the library's failure path.
+ * Launches one thread that waits on a shared-memory barrier for a 16-byte
+ * transfer that is never issued, with the bounded wait every kernel here uses
+ * but a limit of `cycles` SM clocks (1 .. about 2e9) instead of about one
+ * second.  The wait expires, the kernel records KVPACK_ERR_TIMEOUT in the
+ * device error word and returns: kvpack_last_device_status() then reports
+ * KVPACK_ERR_TIMEOUT and the context stays usable.  Nothing is copied.
+ */
+kvpack_status kvpack_selftest_bounded_wait(int64_t cycles, void *stream);
 
 #ifdef __cplusplus
 }

@@ -27,10 +27,14 @@ from ._lib import (  # noqa: F401
     decode_attn_noalloc,
     NOALLOC_SCRATCH_BYTES,
     decode_workspace,
+    decompress,
+    dense_decode_attn,
+    dense_decode_workspace,
     footprint,
     last_device_status,
     lib,
     library_path,
     select,
+    selftest_bounded_wait,
     version,
 )

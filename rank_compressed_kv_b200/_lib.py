@@ -83,6 +83,14 @@ _L.kvpack_decode_attn_noalloc.argtypes = [_dims_p, _i32, _vp, _vp, _vp, _vp, _vp
                                           _vp, ctypes.c_float, _vp, _vp, _vp]
 _L.kvpack_decode_attn_noalloc.restype = ctypes.c_int
 _L.kvpack_noalloc_scratch_bytes.restype = _sz
+_L.kvpack_dense_decode_workspace.argtypes = [_dims_p, _i32, _i32]
+_L.kvpack_dense_decode_workspace.restype = _sz
+_L.kvpack_dense_decode_attn.argtypes = [_dims_p, _i32, _vp, _vp, _vp, _i32, _i32, ctypes.c_float, _vp, _vp, _sz, _vp]
+_L.kvpack_dense_decode_attn.restype = ctypes.c_int
+_L.kvpack_decompress.argtypes = [_dims_p, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
+_L.kvpack_decompress.restype = ctypes.c_int
+_L.kvpack_selftest_bounded_wait.argtypes = [ctypes.c_int64, _vp]
+_L.kvpack_selftest_bounded_wait.restype = ctypes.c_int
 _L.kvpack_select.argtypes = [_dims_p, _i32, _vp, _vp, ctypes.c_float, _i32, _vp, _vp]
 _L.kvpack_select.restype = ctypes.c_int
 
@@ -168,6 +176,30 @@ NOALLOC_SCRATCH_BYTES = int(_L.kvpack_noalloc_scratch_bytes())
 def select(dims: Dims, n_layers: int, mass, score, alpha: float, k_hi: int, mask_out, stream=None):
     _check(_L.kvpack_select(ctypes.byref(dims.c()), n_layers, _ptr(mass), _ptr(score), float(alpha), int(k_hi),
                             _ptr(mask_out), _stream(stream)), "kvpack_select")
+
+
+def dense_decode_workspace(dims: Dims, n_layers: int, L_cap: int) -> int:
+    return int(_L.kvpack_dense_decode_workspace(ctypes.byref(dims.c()), n_layers, L_cap))
+
+
+def dense_decode_attn(dims: Dims, n_layers: int, q, K, V, L_cap: int, L: int, scale: float, out, ws, stream=None):
+    """Standard attention over an uncompressed bf16 cache [units][L_cap][4][128] (the baseline)."""
+    _check(_L.kvpack_dense_decode_attn(ctypes.byref(dims.c()), n_layers, _ptr(q), _ptr(K), _ptr(V), L_cap, L,
+                                       float(scale), _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "kvpack_dense_decode_attn")
+
+
+def decompress(dims: Dims, n_layers: int, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, mask, K_out, V_out, L_cap: int,
+               stream=None):
+    """Every visual token decompressed at its rank into rows 0..T-1 of K_out, V_out [units][L_cap][4][128]."""
+    _check(_L.kvpack_decompress(ctypes.byref(dims.c()), n_layers, _ptr(CK_lo), _ptr(CK_hi), _ptr(BK), _ptr(CV_lo),
+                                _ptr(CV_hi), _ptr(BV), _ptr(mask), _ptr(K_out), _ptr(V_out), L_cap, _stream(stream)),
+           "kvpack_decompress")
+
+
+def selftest_bounded_wait(cycles: int, stream=None):
+    """Run the bounded-wait self-test (a wait that nothing completes; expect KVPACK_ERR_TIMEOUT next)."""
+    _check(_L.kvpack_selftest_bounded_wait(int(cycles), _stream(stream)), "kvpack_selftest_bounded_wait")
 
 
 def last_device_status(stream=None) -> int:

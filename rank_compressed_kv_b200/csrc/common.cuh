@@ -50,15 +50,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and
-// raises *abort) if *abort was already set or the wait expired.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
-    if (*abort) return false;
+// raises *abort) if the phase has not completed and *abort is set or the wait
+// expired.  A completed phase is reported as such even after an abort, so
+// threads that wait on the same phase agree on the outcome.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, volatile int *abort, long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
     long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             report_error(KVPACK_ERR_TIMEOUT);
             *abort = 1;
             return false;
@@ -66,10 +68,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return mbar_wait_for(bar, parity, abort, kWaitCycles);
+}
+
+// ------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the
+// previous kernel on the stream is still running; it must not touch that
+// kernel's outputs before griddep_wait(), which returns once the previous grid
+// has completed and its memory is visible (immediately for a normal launch).
+// griddep_launch_dependents() lets the next such kernel start early.
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ cp.async
 
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+
+// 16-byte copy that writes zeros instead when !valid (the source is then not read).
+__device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src, bool valid) {
+    const int n = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(n)
+                 : "memory");
 }
 
 // Arrive on the mbarrier when all of this thread's earlier cp.async copies have

@@ -65,11 +65,6 @@ inline Workspace carve(void *ws, int units) {
     return w;
 }
 
-__device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src, bool valid) {
-    const int n = valid ? 16 : 0;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(n)
-                 : "memory");
-}
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
@@ -229,6 +224,7 @@ __device__ int eig_jacobi(float *Y, EigSmem &sm) {
 
 struct EigParams {
     Workspace ws;
+    int max_iter;       // iteration cap (at most kMaxIter)
     uint16_t *B;        // [units][64][512]
     float *sigma;       // [units][64] or null
     int units;
@@ -258,7 +254,7 @@ __global__ void __launch_bounds__(kEigThreads, 1) eig_kernel(EigParams p) {
     __syncthreads();
 
     bool converged = false, jacobi_ok = true;
-    for (int it = 0; it < kMaxIter; ++it) {
+    for (int it = 0; it < p.max_iter; ++it) {
         // Y = G Q  (Q in the smem buffer), Y^T to global
         eig_gemm(Gu, sm.buf, Ytu);
         __threadfence_block();
@@ -314,7 +310,7 @@ __global__ void __launch_bounds__(kEigThreads, 1) eig_kernel(EigParams p) {
         __syncthreads();
         if (tid < kP) sm.prev_sorted[tid] = sm.lam_sorted[tid];
         converged = sm.done != 0;
-        const bool last = converged || it == kMaxIter - 1;
+        const bool last = converged || it == p.max_iter - 1;
 
         // Q for the next iteration: normalised columns in sorted order, bf16 hi / lo rows
         {
@@ -624,7 +620,7 @@ inline kvpack_status prepare_device() {
 }
 
 inline kvpack_status run(int units, int T, const uint16_t *X, const CUtensorMap &tm_x, uint16_t *C_lo,
-                         uint16_t *C_hi, uint16_t *B, float *sigma, void *ws, int sms, cudaStream_t st) {
+                         uint16_t *C_hi, uint16_t *B, float *sigma, void *ws, int sms, int max_iter, cudaStream_t st) {
     (void)sms;
     Workspace w = carve(ws, units);
     GramTcParams gp;
@@ -639,7 +635,7 @@ inline kvpack_status run(int units, int T, const uint16_t *X, const CUtensorMap 
     const int per_unit = gp.splits[0] + gp.splits[1] + gp.splits[2] + gp.splits[3];
     gram_tc_kernel<<<units * per_unit, kGtThreads, gram_tc_smem(), st>>>(gp);
     if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
-    EigParams ep{w, B, sigma, units};
+    EigParams ep{w, max_iter, B, sigma, units};
     eig_kernel<<<units, kEigThreads, sizeof(EigSmem), st>>>(ep);
     if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
     const int tiles = (T + kProjTok - 1) / kProjTok;

@@ -1,9 +1,12 @@
 // kvpack.cu -- the C ABI of libkvpack (see include/kvpack.h): argument
 // validation, workspace planning and kernel launches.  Everything that
-// computes runs in the kernels of decode.cuh, select.cuh and compress.cuh.
+// computes runs in the kernels of decode.cuh, rstream.cuh, select.cuh and
+// compress.cuh.
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -11,7 +14,8 @@
 #include "kvpack.h"
 #include "common.cuh"
 #include "decode.cuh"
-#include "mass.cuh"
+#include "rstream.cuh"
+#include "baseline.cuh"
 #include "select.cuh"
 #include "compress.cuh"
 
@@ -29,7 +33,7 @@ kvpack_status check_dims(const kvpack_dims *d, int32_t n_layers) {
     if (d->batch <= 0 || d->n_q_heads <= 0 || d->n_kv_heads <= 0 || d->T_vis <= 0 || d->L_text_cap < 0)
         return KVPACK_ERR_INVALID_ARG;
     if (d->group != KVPACK_GROUP || d->head_dim != KVPACK_HEAD_DIM || d->rank != KVPACK_RANK ||
-        d->rank_lo != KVPACK_RANK_LO)
+        (d->rank_lo != KVPACK_RANK_LO && d->rank_lo != 0))
         return KVPACK_ERR_UNSUPPORTED;
     if (d->n_kv_heads % KVPACK_GROUP != 0 || d->n_q_heads % d->n_kv_heads != 0) return KVPACK_ERR_UNSUPPORTED;
     if ((d->n_q_heads / d->n_kv_heads) * KVPACK_GROUP > 32) return KVPACK_ERR_UNSUPPORTED;
@@ -47,43 +51,51 @@ inline int hg(const kvpack_dims *d) { return (d->n_q_heads / d->n_kv_heads) * KV
 
 // Text tail: work items of kTextChunk tokens per (unit, KV head).
 constexpr int kTextChunk = 64;
+// The visual passes are sized for a full B200 (148 SMs) whatever the device, so the
+// workspace, the work split and hence the results depend on the shapes alone.
+constexpr int kPlanSMs = 148;
+
+namespace rs = kvpack::decode::rs;
 
 struct DecodePlan {
-    int nmb, S, tps, units, Hg, Sc_max;
-    size_t off_qt, off_tp, off_vp, off_ustat, off_counter, total;
+    int units, Hg, NH, tpu, nwords, Sc_max;
+    long long ntiles;
+    int cta_s, cta_v, nslot_s, nslot_v;
+    size_t off_qt, off_tp, off_sp, off_ustat, off_vp, off_counter, total;
 };
+
+inline int round_heads(int Hg) { return Hg <= 4 ? 4 : Hg <= 8 ? 8 : Hg <= 16 ? 16 : 32; }
+
+// Most partial slots any unit gets when NT tiles are split over C CTAs (tpu tiles per unit).
+inline int max_slots(long long NT, long long C, int tpu) { return (int)(((long long)tpu * C + NT - 1) / NT) + 1; }
 
 DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
     DecodePlan pl{};
     pl.Hg = hg(d);
-    pl.nmb = (pl.Hg <= 16) ? 1 : 2;
+    pl.NH = round_heads(pl.Hg);
     pl.units = n_units(d, n_layers);
-    // Visual items (unit, chunk of tps tokens) for warps that fetch work from a counter:
-    // about six per warp of a full B200 (148 SMs x 16 or 8 warps), so the last round is
-    // short; chunks are whole 64-token sub-chunks, between 256 and 2048 tokens, and a
-    // unit's chunks are as even as the 64-token grain allows.  The plan depends on the
-    // shapes alone, so the workspace size does too.
     const int T = d->T_vis;
-    const long long warps = (pl.nmb == 1) ? 148LL * 16 : 148LL * 8;
-    long long tgt = ((long long)pl.units * T) / (6 * warps);
-    tgt = (tgt + 63) / 64 * 64;
-    if (tgt < 256) tgt = 256;
-    if (tgt > 2048) tgt = 2048;
-    const int S0 = (int)((T + tgt - 1) / tgt);
-    pl.tps = ((T + S0 - 1) / S0 + 63) / 64 * 64;
-    pl.S = (T + pl.tps - 1) / pl.tps;
-    static_assert(kvpack::decode::vis::kMaxItemTok >= 2048, "visual items of up to 2048 tokens");
+    pl.tpu = (T + rs::kTile - 1) / rs::kTile;
+    pl.nwords = (T + 31) / 32;
+    pl.ntiles = (long long)pl.units * pl.tpu;
+    const int blocks = pl.NH <= 16 ? 2 : 1;     // resident CTAs per SM of both visual passes
+    pl.cta_s = (int)(pl.ntiles < (long long)kPlanSMs * blocks ? pl.ntiles : (long long)kPlanSMs * blocks);
+    pl.cta_v = pl.cta_s;
+    pl.nslot_s = max_slots(pl.ntiles, pl.cta_s, pl.tpu);
+    pl.nslot_v = max_slots(pl.ntiles, pl.cta_v, pl.tpu);
     pl.Sc_max = (d->L_text_cap + kTextChunk - 1) / kTextChunk;
     size_t off = 0;
     pl.off_qt = off;
     off = align256(off + (size_t)pl.units * kvpack::decode::qblock_bytes(pl.Hg));
     pl.off_tp = off;
     off = align256(off + (size_t)pl.units * pl.Sc_max * pl.Hg * kvpack::decode::kTxtPart * sizeof(float));
-    pl.off_vp = off;
-    off = align256(off + (size_t)pl.units * pl.S * pl.Hg * kvpack::decode::kVisPart * sizeof(float));
+    pl.off_sp = off;
+    off = align256(off + (size_t)pl.units * pl.nslot_s * pl.Hg * 2 * sizeof(float));
     pl.off_ustat = off;
     off = align256(off + (size_t)pl.units * pl.Hg * 2 * sizeof(float));
-    pl.off_counter = off;   // work counters: [0] text kernel, [1] visual kernel
+    pl.off_vp = off;
+    off = align256(off + (size_t)pl.units * pl.nslot_v * pl.Hg * 64 * sizeof(float));
+    pl.off_counter = off;   // work counter of the text kernel
     off = align256(off + 4 * sizeof(unsigned int));
     pl.total = off;
     return pl;
@@ -93,34 +105,64 @@ struct DeviceInfo {
     bool ready = false;
     unsigned long long ctx_id = 0;       // the context the attributes below were set in
     int sms = 0;
-    int mass_blocks[4] = {0, 0, 0, 0};   // resident blocks per SM of mass_kernel<1..4>
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
-// finish_kernel is instantiated for 1..8 query heads per KV head
-template <int PK>
-bool finish_attr_one() {
-    return cudaFuncSetAttribute(kvpack::decode::finish_kernel<PK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kvpack::decode::kFinishSmemMax) == cudaSuccess;
+template <int NH, bool VALUE>
+bool rs_attr() {
+    const void *fn = (const void *)rs::rs_kernel<NH, VALUE>;
+    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rs::smem_bytes<NH, VALUE>()) ==
+               cudaSuccess &&
+           cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) == cudaSuccess;
 }
-bool finish_attrs() {
-    return finish_attr_one<1>() && finish_attr_one<2>() && finish_attr_one<3>() && finish_attr_one<4>() &&
-           finish_attr_one<5>() && finish_attr_one<6>() && finish_attr_one<7>() && finish_attr_one<8>();
+bool rs_attrs() {
+    return rs_attr<4, false>() && rs_attr<4, true>() && rs_attr<8, false>() && rs_attr<8, true>() &&
+           rs_attr<16, false>() && rs_attr<16, true>() && rs_attr<32, false>() && rs_attr<32, true>();
 }
-cudaError_t launch_finish(int per_kv, const kvpack::decode::FinishParams &fp, int units, size_t smem, cudaStream_t st) {
-    namespace dc = kvpack::decode;
-    switch (per_kv) {
-        case 1: dc::finish_kernel<1><<<units, 256, smem, st>>>(fp); break;
-        case 2: dc::finish_kernel<2><<<units, 256, smem, st>>>(fp); break;
-        case 3: dc::finish_kernel<3><<<units, 256, smem, st>>>(fp); break;
-        case 4: dc::finish_kernel<4><<<units, 256, smem, st>>>(fp); break;
-        case 5: dc::finish_kernel<5><<<units, 256, smem, st>>>(fp); break;
-        case 6: dc::finish_kernel<6><<<units, 256, smem, st>>>(fp); break;
-        case 7: dc::finish_kernel<7><<<units, 256, smem, st>>>(fp); break;
-        default: dc::finish_kernel<8><<<units, 256, smem, st>>>(fp); break;
+
+// Launch on `st` with programmatic stream serialization: the kernel may start while the
+// previous kernel on the stream drains, and waits for it (griddep_wait) before reading its
+// outputs.
+template <typename... Args, typename... Params>
+cudaError_t launch_pdl(void (*kernel)(Params...), int grid, int threads, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <bool VALUE>
+cudaError_t launch_rs(int NH, const rs::Params &rp, int grid, cudaStream_t st) {
+    switch (NH) {
+        case 4: return launch_pdl(rs::rs_kernel<4, VALUE>, grid, rs::kThreads, rs::smem_bytes<4, VALUE>(), st, rp);
+        case 8: return launch_pdl(rs::rs_kernel<8, VALUE>, grid, rs::kThreads, rs::smem_bytes<8, VALUE>(), st, rp);
+        case 16: return launch_pdl(rs::rs_kernel<16, VALUE>, grid, rs::kThreads, rs::smem_bytes<16, VALUE>(), st, rp);
+        default: return launch_pdl(rs::rs_kernel<32, VALUE>, grid, rs::kThreads, rs::smem_bytes<32, VALUE>(), st, rp);
     }
-    return cudaGetLastError();
+}
+
+// finish_kernel is instantiated for 1..8 query heads per KV head
+cudaError_t launch_finish(int per_kv, const rs::FinishParams &fp, int units, cudaStream_t st) {
+    const int grid = units * 4;
+    switch (per_kv) {
+        case 1: return launch_pdl(rs::finish_kernel<1>, grid, 128, 0, st, fp);
+        case 2: return launch_pdl(rs::finish_kernel<2>, grid, 128, 0, st, fp);
+        case 3: return launch_pdl(rs::finish_kernel<3>, grid, 128, 0, st, fp);
+        case 4: return launch_pdl(rs::finish_kernel<4>, grid, 128, 0, st, fp);
+        case 5: return launch_pdl(rs::finish_kernel<5>, grid, 128, 0, st, fp);
+        case 6: return launch_pdl(rs::finish_kernel<6>, grid, 128, 0, st, fp);
+        case 7: return launch_pdl(rs::finish_kernel<7>, grid, 128, 0, st, fp);
+        default: return launch_pdl(rs::finish_kernel<8>, grid, 128, 0, st, fp);
+    }
 }
 
 // Unique id of the calling thread's current context (cuCtxGetId, looked up once through the
@@ -167,41 +209,16 @@ kvpack_status device_info(DeviceInfo **out) {
         di.ctx_id = ctx_id;
         if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return KVPACK_ERR_CUDA;
         namespace dc = kvpack::decode;
-        if (cudaFuncSetAttribute(dc::vis::vis_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)dc::vis::smem_bytes<1>()) != cudaSuccess ||
-            cudaFuncSetAttribute(dc::vis::vis_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)dc::vis::smem_bytes<2>()) != cudaSuccess ||
-            cudaFuncSetAttribute(dc::text::text_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(dc::text::text_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)dc::text::smem_bytes()) != cudaSuccess ||
-            !finish_attrs())
+            cudaFuncSetAttribute(dc::text::text_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+                cudaSuccess ||
+            !rs_attrs() ||
+            cudaFuncSetAttribute(kvpack::baseline::decompress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(kvpack::baseline::DecSmem)) != cudaSuccess ||
+            cudaFuncSetAttribute(kvpack::select::select_kernel<64, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kvpack::select::select_smem_bytes<64, 32>()) != cudaSuccess)
             return KVPACK_ERR_CUDA;
-        // all of the SM's shared memory for these kernels (two visual blocks of the 16-row variant)
-        if (cudaFuncSetAttribute(dc::vis::vis_kernel<1>, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
-            cudaFuncSetAttribute(dc::vis::vis_kernel<2>, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
-            cudaFuncSetAttribute(dc::text::text_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
-            return KVPACK_ERR_CUDA;
-        {
-            const void *mk[4] = {(const void *)dc::mass::mass_kernel<1>, (const void *)dc::mass::mass_kernel<2>,
-                                 (const void *)dc::mass::mass_kernel<3>, (const void *)dc::mass::mass_kernel<4>};
-            for (int i = 0; i < 4; ++i) {
-                if (cudaFuncSetAttribute(mk[i], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dc::mass::smem_bytes()) != cudaSuccess ||
-                    cudaFuncSetAttribute(mk[i], cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
-                    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.mass_blocks[i], mk[i], dc::mass::kThreads,
-                                                                  dc::mass::smem_bytes()) != cudaSuccess ||
-                    di.mass_blocks[i] < 1)
-                    return KVPACK_ERR_CUDA;
-            }
-        }
-        int b1 = 0, b2 = 0, bt = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b1, dc::vis::vis_kernel<1>, dc::vis::kThreads,
-                                                          dc::vis::smem_bytes<1>()) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b2, dc::vis::vis_kernel<2>, dc::vis::kThreads,
-                                                          dc::vis::smem_bytes<2>()) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bt, dc::text::text_kernel, dc::text::kThreads,
-                                                          dc::text::smem_bytes()) != cudaSuccess)
-            return KVPACK_ERR_CUDA;
-        // the visual kernels are sized for Cfg::kBlocks resident blocks per SM
-        if (b1 != dc::vis::Cfg<1>::kBlocks || b2 != dc::vis::Cfg<2>::kBlocks || bt < 1) return KVPACK_ERR_CUDA;
         kvpack_status cs = kvpack::compress::prepare_device();
         if (cs != KVPACK_OK) return cs;
         di.ready = true;
@@ -243,7 +260,8 @@ cudaError_t launch_select(const kvpack::select::Params &p, cudaStream_t st) {
         const int grid = (p.n_units + 7) / 8;
         kvpack::select::select_kernel<KPT, 1><<<grid, 256, 0, st>>>(p);
     } else {
-        kvpack::select::select_kernel<KPT, 32><<<p.n_units, 1024, 0, st>>>(p);
+        constexpr size_t smem = kvpack::select::select_smem_bytes<KPT, 32>();   // set up in device_info
+        kvpack::select::select_kernel<KPT, 32><<<p.n_units, 1024, smem, st>>>(p);
     }
     return cudaGetLastError();
 }
@@ -325,8 +343,7 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     for (const void *ptr : ptrs)
         if (ptr && !aligned16(ptr)) return KVPACK_ERR_ALIGNMENT;
     const DecodePlan pl = plan_decode(d, n_layers);
-    if (pl.S <= 0) return KVPACK_ERR_UNSUPPORTED;
-    if ((long long)pl.units * d->T_vis * 3 >= (1LL << 31)) return KVPACK_ERR_UNSUPPORTED;   // int32 gather rows
+    if ((long long)pl.units * d->T_vis * 3 >= (1LL << 31)) return KVPACK_ERR_UNSUPPORTED;   // int32 rows
     if (ws == nullptr || ws_bytes < pl.total) return KVPACK_ERR_WORKSPACE;
     DeviceInfo *di = nullptr;
     if ((s = device_info(&di)) != KVPACK_OK) return s;
@@ -342,12 +359,13 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     unsigned char *w = static_cast<unsigned char *>(ws);
     unsigned char *qt = w + pl.off_qt;
     float *tpart = reinterpret_cast<float *>(w + pl.off_tp);
-    float *vpart = reinterpret_cast<float *>(w + pl.off_vp);
+    float *spart = reinterpret_cast<float *>(w + pl.off_sp);
     float *ustat = reinterpret_cast<float *>(w + pl.off_ustat);
+    float *vpart = reinterpret_cast<float *>(w + pl.off_vp);
     unsigned int *counter = reinterpret_cast<unsigned int *>(w + pl.off_counter);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    // the work counters start at zero
+    // the text kernel's work counter starts at zero
     if (cudaMemsetAsync(counter, 0, 4 * sizeof(unsigned int), st) != cudaSuccess) return KVPACK_ERR_CUDA;
 
     // 1. q~ per (unit, KV head) and the text tail partials, one persistent launch
@@ -378,66 +396,34 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
         if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
     }
 
-    // 2. the text tail's (max, sum) per head of each unit, into its query block
-    dc::text::text_stats_kernel<<<(pl.units + 7) / 8, 256, 0, st>>>(tpart, qt, pl.units, Hg, Sc);
-    if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
-
-    // 3. visual partials and the attention mass
+    // 2-4. the visual tokens: softmax statistics, the unit-wide statistics, then the value pass
+    rs::Params rp;
+    std::memset(&rp, 0, sizeof(rp));
     {
-        dc::vis::Params vp;
-        std::memset(&vp, 0, sizeof(vp));
         const cuuint64_t dims[3] = {16, (cuuint64_t)T, (cuuint64_t)pl.units};
         const cuuint64_t strides[2] = {32, (cuuint64_t)T * 32};
-        const cuuint32_t box[3] = {16, 32, 1};
-        if (!encode_bf16(enc, &vp.tm_ck, CK_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B) ||
-            !encode_bf16(enc, &vp.tm_cv, CV_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B))
+        const cuuint32_t box[3] = {16, 256, 1};
+        if (!encode_bf16(enc, &rp.tm_ck, CK_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B) ||
+            !encode_bf16(enc, &rp.tm_cv, CV_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B))
             return KVPACK_ERR_CUDA;
-        vp.CK_lo = CK_lo; vp.CK_hi = CK_hi; vp.CV_lo = CV_lo; vp.CV_hi = CV_hi;
-        vp.qt = qt; vp.mask = mask; vp.part = vpart; vp.counter = counter + 1;
-        vp.n_units = pl.units; vp.T = T; vp.Hg = Hg; vp.S = pl.S; vp.tps = pl.tps; vp.nwords = (T + 31) / 32;
-        vp.n_items = pl.units * pl.S;
-        const int resident = di->sms * (pl.nmb == 1 ? dc::vis::Cfg<1>::kBlocks : dc::vis::Cfg<2>::kBlocks);
-        const int need = (vp.n_items + dc::vis::kWarps - 1) / dc::vis::kWarps;
-        const int grid = need < resident ? need : resident;
-        void *args[] = {&vp};
-        const void *fn = (pl.nmb == 1) ? (const void *)dc::vis::vis_kernel<1> : (const void *)dc::vis::vis_kernel<2>;
-        const size_t smem = (pl.nmb == 1) ? dc::vis::smem_bytes<1>() : dc::vis::smem_bytes<2>();
-        const cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(dc::vis::kThreads), args, smem, st);
-        if (e != cudaSuccess) return KVPACK_ERR_CUDA;
     }
-
-    // 4. combine and project through B_V
-    dc::FinishParams fp{BV, vpart, Sc > 0 ? tpart : nullptr, out, mass != nullptr ? ustat : nullptr,
-                        Hg, per_kv, d->n_q_heads, groups, pl.S, Sc};
-    if (launch_finish(per_kv, fp, pl.units, dc::finish_smem_bytes(pl.S, Sc, Hg), st) != cudaSuccess)
+    rp.CK_lo = CK_lo; rp.CK_hi = CK_hi; rp.CV_lo = CV_lo; rp.CV_hi = CV_hi;
+    rp.qt = qt; rp.mask = mask; rp.ustat = ustat;
+    rp.units = pl.units; rp.T = T; rp.Hg = Hg; rp.nwords = pl.nwords; rp.tpu = pl.tpu;
+    rp.rank0 = d->rank_lo == 0 ? 1 : 0; rp.ntiles = pl.ntiles;
+    rp.part = spart; rp.nslot = pl.nslot_s; rp.mass = nullptr;
+    if (launch_rs<false>(pl.NH, rp, pl.cta_s, st) != cudaSuccess) return KVPACK_ERR_CUDA;
+    if (launch_pdl(rs::combine_kernel, (pl.units + 7) / 8, 256, 0, st, (const float *)spart, (const float *)tpart,
+                   ustat, pl.units, Hg, Sc, pl.nslot_s, pl.ntiles, pl.tpu, pl.cta_s) != cudaSuccess)
         return KVPACK_ERR_CUDA;
-    if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
-    if (mass == nullptr) return KVPACK_OK;
+    rp.part = vpart; rp.nslot = pl.nslot_v; rp.mass = mass;
+    if (launch_rs<true>(pl.NH, rp, pl.cta_v, st) != cudaSuccess) return KVPACK_ERR_CUDA;
 
-    // 5. the attention mass of every visual token under the unit's final (max, sum)
-    {
-        dc::mass::Params mp;
-        std::memset(&mp, 0, sizeof(mp));
-        const cuuint64_t dims[3] = {16, (cuuint64_t)T, (cuuint64_t)pl.units};
-        const cuuint64_t strides[2] = {32, (cuuint64_t)T * 32};
-        const cuuint32_t box[3] = {16, 32, 1};
-        if (!encode_bf16(enc, &mp.tm_ck, CK_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B)) return KVPACK_ERR_CUDA;
-        mp.CK_lo = CK_lo; mp.CK_hi = CK_hi; mp.qt = qt; mp.ustat = ustat; mp.mask = mask; mp.mass = mass;
-        mp.T = T; mp.Hg = Hg; mp.nwords = (T + 31) / 32; mp.cpu = (T + dc::mass::kChunk - 1) / dc::mass::kChunk;
-        mp.n_chunks = pl.units * mp.cpu;
-        const int nt = (Hg + 7) / 8;
-        const int resident = di->sms * di->mass_blocks[nt - 1];
-        const int need = (mp.n_chunks + dc::mass::kWarps - 1) / dc::mass::kWarps;
-        const int grid = need < resident ? need : resident;
-        const size_t smem = dc::mass::smem_bytes();
-        switch (nt) {
-            case 1: dc::mass::mass_kernel<1><<<grid, dc::mass::kThreads, smem, st>>>(mp); break;
-            case 2: dc::mass::mass_kernel<2><<<grid, dc::mass::kThreads, smem, st>>>(mp); break;
-            case 3: dc::mass::mass_kernel<3><<<grid, dc::mass::kThreads, smem, st>>>(mp); break;
-            default: dc::mass::mass_kernel<4><<<grid, dc::mass::kThreads, smem, st>>>(mp); break;
-        }
-    }
-    return (cudaGetLastError() == cudaSuccess) ? KVPACK_OK : KVPACK_ERR_CUDA;
+    // 5. combine the partials and project through B_V
+    rs::FinishParams fp{BV, vpart, Sc > 0 ? tpart : nullptr, ustat, out, Hg, per_kv, d->n_q_heads, groups, Sc,
+                        pl.nslot_v, pl.tpu, pl.cta_v, pl.ntiles};
+    if (launch_finish(per_kv, fp, pl.units, st) != cudaSuccess) return KVPACK_ERR_CUDA;
+    return KVPACK_OK;
 }
 
 }  // extern "C"
@@ -485,6 +471,143 @@ kvpack_status kvpack_decode_attn_noalloc(const kvpack_dims *d, int32_t n_layers,
                               softmax_scale, out, mass, ws, KVPACK_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+// ------------------------------------------------------------------ baselines
+
+namespace {
+
+size_t dense_workspace(int units, int Hg, int L_cap) {
+    const int Sc = (L_cap + kvpack::baseline::kDenseChunk - 1) / kvpack::baseline::kDenseChunk;
+    return align256((size_t)units * (Sc > 0 ? Sc : 1) * Hg * kvpack::decode::kTxtPart * sizeof(float)) + 256;
+}
+
+cudaError_t launch_dense_finish(int per_kv, const kvpack::baseline::DenseFinishParams &fp, int units, cudaStream_t st) {
+    namespace bl = kvpack::baseline;
+    const int grid = units * 4;
+    switch (per_kv) {
+        case 1: bl::dense_finish_kernel<1><<<grid, 128, 0, st>>>(fp); break;
+        case 2: bl::dense_finish_kernel<2><<<grid, 128, 0, st>>>(fp); break;
+        case 3: bl::dense_finish_kernel<3><<<grid, 128, 0, st>>>(fp); break;
+        case 4: bl::dense_finish_kernel<4><<<grid, 128, 0, st>>>(fp); break;
+        case 5: bl::dense_finish_kernel<5><<<grid, 128, 0, st>>>(fp); break;
+        case 6: bl::dense_finish_kernel<6><<<grid, 128, 0, st>>>(fp); break;
+        case 7: bl::dense_finish_kernel<7><<<grid, 128, 0, st>>>(fp); break;
+        default: bl::dense_finish_kernel<8><<<grid, 128, 0, st>>>(fp); break;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kvpack_dense_decode_workspace(const kvpack_dims *d, int32_t n_layers, int32_t L_cap) {
+    if (check_dims(d, n_layers) != KVPACK_OK || L_cap < 1) return 0;
+    return dense_workspace(n_units(d, n_layers), hg(d), L_cap);
+}
+
+kvpack_status kvpack_dense_decode_attn(const kvpack_dims *d, int32_t n_layers, const uint16_t *q, const uint16_t *K,
+                                       const uint16_t *V, int32_t L_cap, int32_t L, float softmax_scale,
+                                       uint16_t *out, void *ws, size_t ws_bytes, void *stream) {
+    kvpack_status s = check_dims(d, n_layers);
+    if (s != KVPACK_OK) return s;
+    if (L_cap < 1 || L < 1 || L > L_cap || (long long)L_cap > 4LL * KVPACK_MAX_T) return KVPACK_ERR_INVALID_ARG;
+    if (!q || !K || !V || !out) return KVPACK_ERR_INVALID_ARG;
+    if (!(softmax_scale == softmax_scale) || softmax_scale <= 0.f) return KVPACK_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, K, V, out, ws};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KVPACK_ERR_ALIGNMENT;
+    const int units = n_units(d, n_layers), Hg = hg(d), per_kv = d->n_q_heads / d->n_kv_heads;
+    const size_t need = dense_workspace(units, Hg, L_cap);
+    if (ws == nullptr || ws_bytes < need) return KVPACK_ERR_WORKSPACE;
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != KVPACK_OK) return s;
+    PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+    if ((s = tensor_map_encoder(&enc)) != KVPACK_OK) return s;
+    namespace dc = kvpack::decode;
+    const int ct = kvpack::baseline::kDenseChunk, Sc = (L + ct - 1) / ct;
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    float *tpart = reinterpret_cast<float *>(w);
+    unsigned int *counter = reinterpret_cast<unsigned int *>(w + need - 256);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(counter, 0, 4 * sizeof(unsigned int), st) != cudaSuccess) return KVPACK_ERR_CUDA;
+    dc::text::Params tp;
+    std::memset(&tp, 0, sizeof(tp));
+    {
+        const cuuint64_t dims[4] = {128, 4, (cuuint64_t)L, (cuuint64_t)units};
+        const cuuint64_t strides[3] = {256, 1024, (cuuint64_t)L_cap * 1024};
+        const cuuint32_t box[4] = {64, 1, 16, 1};
+        if (!encode_bf16(enc, &tp.tm_k, K, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_bf16(enc, &tp.tm_v, V, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return KVPACK_ERR_CUDA;
+    }
+    tp.q = q; tp.part = tpart; tp.qt = nullptr; tp.counter = counter;
+    tp.n_units = units; tp.L = L; tp.Hg = Hg; tp.per_kv = per_kv; tp.n_q = d->n_q_heads;
+    tp.groups = d->n_kv_heads / KVPACK_GROUP; tp.Sc = Sc; tp.ct = ct; tp.n_qitems = 0;
+    tp.n_items = units * 4 * Sc; tp.scale2 = softmax_scale * 1.4426950408889634f;
+    const int grid = tp.n_items < di->sms ? tp.n_items : di->sms;
+    dc::text::text_kernel<<<grid, dc::text::kThreads, dc::text::smem_bytes(), st>>>(tp);
+    if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
+    kvpack::baseline::DenseFinishParams fp{tpart, out, Hg, d->n_q_heads, d->n_kv_heads / KVPACK_GROUP, Sc};
+    return launch_dense_finish(per_kv, fp, units, st) == cudaSuccess ? KVPACK_OK : KVPACK_ERR_CUDA;
+}
+
+kvpack_status kvpack_decompress(const kvpack_dims *d, int32_t n_layers, const uint16_t *CK_lo, const uint16_t *CK_hi,
+                                const uint16_t *BK, const uint16_t *CV_lo, const uint16_t *CV_hi, const uint16_t *BV,
+                                const uint32_t *mask, uint16_t *K_out, uint16_t *V_out, int32_t L_cap, void *stream) {
+    kvpack_status s = check_dims(d, n_layers);
+    if (s != KVPACK_OK) return s;
+    if (L_cap < d->T_vis) return KVPACK_ERR_INVALID_ARG;
+    if (!CK_lo || !CK_hi || !BK || !CV_lo || !CV_hi || !BV || !mask || !K_out || !V_out) return KVPACK_ERR_INVALID_ARG;
+    const void *ptrs[] = {CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, mask, K_out, V_out};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return KVPACK_ERR_ALIGNMENT;
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != KVPACK_OK) return s;
+    namespace bl = kvpack::baseline;
+    bl::DecompressParams p{};
+    p.C_lo[0] = CK_lo; p.C_hi[0] = CK_hi; p.B[0] = BK;
+    p.C_lo[1] = CV_lo; p.C_hi[1] = CV_hi; p.B[1] = BV;
+    p.mask = mask; p.out[0] = K_out; p.out[1] = V_out;
+    p.T = d->T_vis; p.L_cap = L_cap; p.nwords = (d->T_vis + 31) / 32;
+    p.tiles = (d->T_vis + bl::kDecTok - 1) / bl::kDecTok; p.rank_lo = d->rank_lo;
+    const long long grid = (long long)n_units(d, n_layers) * p.tiles;
+    if (grid >= (1LL << 31)) return KVPACK_ERR_UNSUPPORTED;
+    bl::decompress_kernel<<<(unsigned)grid, bl::kDecThreads, sizeof(bl::DecSmem), static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? KVPACK_OK : KVPACK_ERR_CUDA;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ bounded-wait self-test
+
+namespace {
+
+// One thread announces a 16-byte transfer on a fresh barrier and waits for it; no copy is
+// issued, so the library's bounded wait must give up after `cycles`, record
+// KVPACK_ERR_TIMEOUT in the error word and return.
+__global__ void wait_selftest_kernel(long long cycles) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        kvpack::mbar_init(&bar, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        kvpack::mbar_arrive_tx(&bar, 16u);
+        kvpack::mbar_wait_for(&bar, 0u, &abort_flag, cycles);
+    }
+}
+
+}  // namespace
+
+extern "C" kvpack_status kvpack_selftest_bounded_wait(int64_t cycles, void *stream) {
+    if (cycles < 1 || cycles > kvpack::kWaitCycles) return KVPACK_ERR_INVALID_ARG;
+    wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((long long)cycles);
+    return cudaGetLastError() == cudaSuccess ? KVPACK_OK : KVPACK_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ select
 
 kvpack_status kvpack_select(const kvpack_dims *d, int32_t n_layers, const float *mass, float *score, float alpha,
@@ -496,6 +619,8 @@ kvpack_status kvpack_select(const kvpack_dims *d, int32_t n_layers, const float 
     if (!(alpha >= 0.f && alpha < 1.f)) return KVPACK_ERR_INVALID_ARG;
     if (alpha != 0.f && score == nullptr) return KVPACK_ERR_INVALID_ARG;
     if (!aligned16(mass) || !aligned16(mask_out) || (score && !aligned16(score))) return KVPACK_ERR_ALIGNMENT;
+    DeviceInfo *di = nullptr;
+    if ((s = device_info(&di)) != KVPACK_OK) return s;
     kvpack::select::Params p{};
     p.mass = mass; p.score = score; p.alpha = alpha; p.k = k_hi; p.T = d->T_vis;
     p.nwords = (d->T_vis + 31) / 32; p.n_units = n_units(d, n_layers); p.mask = mask_out;
@@ -542,7 +667,14 @@ kvpack_status kvpack_compress(const kvpack_dims *d, int32_t n_layers, const uint
         const cuuint32_t box[3] = {64, 64, 1};
         if (!encode_bf16(enc, &tm_x, X, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVPACK_ERR_CUDA;
     }
-    return kvpack::compress::run(units, d->T_vis, X, tm_x, C_lo, C_hi, B, sigma, ws, di->sms,
+    // KVPACK_EIG_MAX_ITER (1 .. the built-in cap) lowers the eigen-solver's iteration cap: a test
+    // knob that drives the KVPACK_ERR_NOCONVERGE path without any change to the inputs
+    int max_iter = kvpack::compress::kMaxIter;
+    if (const char *e = std::getenv("KVPACK_EIG_MAX_ITER")) {
+        const int v = std::atoi(e);
+        if (v >= 1 && v < max_iter) max_iter = v;
+    }
+    return kvpack::compress::run(units, d->T_vis, X, tm_x, C_lo, C_hi, B, sigma, ws, di->sms, max_iter,
                                  static_cast<cudaStream_t>(stream));
 }
 

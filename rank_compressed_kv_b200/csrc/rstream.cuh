@@ -1,0 +1,829 @@
+// rstream.cuh -- the visual half of an AttentionPack decode step as two streaming
+// passes over the rank-compressed cache, with the scores on the 5th-generation
+// tensor cores.
+//
+// Method ("Attention-aware Inference Optimizations for Large Vision-Language
+// Models with Memory-efficient Decoding", technical summaries 2.B on the
+// es / fr / de pages): a token with a high importance score is decompressed at
+// the full rank, the others at a quarter of it (or, in the de summary's
+// variant, not at all).  Decompression is folded into the attention by
+// associativity: with q~ = B_K[:, slice] q in rank space, a token's logit is
+// C_K[t, :rho_t] . q~[:rho_t]; the softmax-weighted V coefficients are summed
+// in rank space and projected through B_V once per head (finish kernel).
+//
+//   stats pass  per segment of a unit's tokens: max and sum of 2^s per query
+//               head (s = the logit in the log2 domain), from C_K only
+//   value pass  with the unit's final (M, 1/L) per head known (combine
+//               kernel): p' = 2^(s - M); the attention mass of every token,
+//               sum_h p'_h / L_h; and u_h = sum_t p'_t C_V[t, :rho_t]
+//
+// Work split: the units' tokens, flattened in 128-token tiles, are cut into
+// one contiguous range per CTA; a CTA walks its range unit by unit
+// ("segments") and writes one partial per segment, so a unit has at most a
+// few partials whatever its length.
+//
+// A CTA has six warps:
+//   warp 0     producer: per 512-token block of the segment, one TMA tile of
+//              the C_lo rows (K, and V in the value pass; 32-byte rows,
+//              32-byte swizzle) unless every token of the block is full-rank;
+//              the block's full-rank tokens join a queue, and every 128 of them
+//              (and the rest at the segment's end) are gathered by cp.async as
+//              128-byte rows (C_lo + C_hi, 128-byte swizzle) into a HI tile;
+//              the unit's q~ (bf16 hi and lo planes) by bulk copy per segment
+//   warp 1     tensor memory owner and MMA issuer: per tile, S = C q~^T with
+//              tokens on M = 128 (the tensor-memory lanes) and the query heads
+//              on N, as two bf16 products (q~ hi, q~ lo) accumulated in fp32:
+//              K = 16 (one k-step) for a LO sub-tile, 64 (four) for a HI tile
+//   warps 2-5  consumers: thread = token.  Each reads its token's logits for
+//              every head from tensor memory (tcgen05.ld) and does the
+//              per-token work; in the value pass it writes its row of p' to
+//              shared memory, and the warp adds u^T += C_V^T P for its 32 tokens
+//              with mma.sync (ranks on M, heads on N).
+// Every ring slot carries a descriptor of its tile; one barrier triple per slot
+// (data landed / scores ready / slot free) orders the roles, and a slot's
+// tensor-memory score buffer is reused with the slot.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "decode.cuh"
+
+namespace kvpack {
+namespace decode {
+namespace rs {
+
+constexpr int kWarps = 6;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTile = 128;          // tokens per tensor-memory tile (M of the score MMA)
+constexpr int kHiRing = 1024;       // producer's queue of pending full-rank token positions
+constexpr int kMaskWin = 2048;      // producer's window of mask words (65536 tokens)
+constexpr int kDescInts = 8 + 64;   // header + up to 16 mask words (LO) or 128 uint16 positions (HI)
+constexpr int kTypeLo = 0, kTypeHi = 1, kTypeEnd = 2;
+constexpr int kFlagFirst = 1 << 8, kFlagLast = 1 << 9;
+constexpr float kRefInit = -1e30f;
+constexpr float kLazy = 8.f;        // a per-thread reference max moves when a logit exceeds it by 2^8
+
+// Geometry per (query heads NH, pass).  NH is the unit's Hg rounded up to 4, 8, 16 or 32.  Every
+// ring slot is 16 KB: the statistics pass streams K only (a LO tile of 512 tokens of 32-byte
+// rows, a HI tile of 128 tokens of 128-byte rows), the value pass K and V (256 and 64 tokens).
+// A 64-token HI tile still runs the 128-row score MMA; rows 64-127 read the V half of the slot
+// and their scores are never used.
+template <int NH, bool VALUE>
+struct Cfg {
+    static constexpr int kNHP = NH < 16 ? 16 : NH;                  // N of the score MMA
+    static constexpr int kPH = NH < 8 ? 8 : NH;                      // heads per row of P (mma.sync n8 tiles)
+    static constexpr int kBlocks = NH <= 16 ? 2 : 1;                 // resident CTAs per SM
+    static constexpr int kLoTok = VALUE ? 256 : 512;                 // tokens per LO tile
+    static constexpr int kHiTok = VALUE ? 64 : 128;                  // tokens per HI tile
+    static constexpr int kSub = kLoTok / kTile;                      // 128-token sub-tiles per LO tile
+    static constexpr int kSlotBytes = 16384;
+    static constexpr int kVOff = 8192;                               // value pass: V rows after the K rows
+    static constexpr int kSlots = VALUE ? (NH <= 16 ? 4 : 8) : 4;
+    static constexpr int kSCols = kSub * kNHP;                       // tensor-memory columns of one slot's scores
+    static constexpr int kTmemCols = kSlots * kSCols;                // 128, 256 or 512
+    static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "power-of-two allocation");
+    static_assert(kLoTok / 32 <= 16 && kHiTok <= 128, "descriptor capacity");
+};
+
+struct Params {
+    CUtensorMap tm_ck, tm_cv;       // C_lo planes: 3D {16, T, units}, box {16, 256, 1}, 32-byte swizzle
+    const uint16_t *CK_lo, *CK_hi, *CV_lo, *CV_hi;
+    const unsigned char *qt;        // [units][qblock_bytes(Hg)]: q~ hi, lo planes (from text_kernel)
+    const uint32_t *mask;           // [units][nwords]
+    const float *ustat;             // value pass: [units][Hg][2] = (M, 1/L)
+    float *part;                    // stats: [units][nslot][Hg][2] = (m, l); value: [units][nslot][Hg][64] = u
+    float *mass;                    // value pass: [units][T] or null
+    int units, T, Hg, nwords, tpu, nslot, rank0;
+    long long ntiles;               // units * tpu
+};
+
+// Flattened 128-token tiles [x0, x1) of CTA c among C: x0 = floor(c NT / C).  The CTA that
+// holds tile x is floor(((x + 1) C - 1) / NT); a unit's partial slot is its CTA's offset
+// from the CTA holding the unit's first tile.
+__host__ __device__ inline long long tile_begin(long long c, long long C, long long NT) { return c * NT / C; }
+__host__ __device__ inline long long cta_of_tile(long long x, long long C, long long NT) { return ((x + 1) * C - 1) / NT; }
+
+template <int NH, bool VALUE>
+struct Smem {
+    using C = Cfg<NH, VALUE>;
+    alignas(1024) unsigned char slot[C::kSlots][C::kSlotBytes];
+    alignas(1024) unsigned char qbuf[2][2][C::kNHP * 128];          // [q slot][hi, lo][rows of 128 B]
+    int desc[C::kSlots][kDescInts];
+    uint32_t mwin[kMaskWin];                                        // producer's window of the CTA's mask words
+    uint16_t hi_ring[kHiRing];
+    unsigned char pbuf[VALUE ? 4 : 1][VALUE ? 32 * C::kPH * 2 : 16];   // value pass: P rows of each consumer warp
+    float merge[VALUE ? 3 : 4][VALUE ? NH * 64 : NH * 2];           // partial merge across the consumer warps
+    uint64_t full[C::kSlots], sfull[C::kSlots], empty[C::kSlots], qfull[2], qempty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int NH, bool VALUE>
+constexpr size_t smem_bytes() { return sizeof(Smem<NH, VALUE>) + 1024; }
+
+// ------------------------------------------------------------------ tcgen05 helpers
+
+// Shared-memory descriptor of a K-major operand in swizzled 8-row atoms: SBO = byte
+// stride between 8-row groups; the leading offset is unused for swizzled K-major tiles.
+// swz: 6 = 32-byte swizzle, 2 = 128-byte swizzle.
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr, uint32_t sbo, uint32_t swz) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)swz << 61;
+    return d;
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_kk(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]);
+
+template <>
+__device__ __forceinline__ void tmem_ld<4>(uint32_t taddr, float (&v)[4]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]) : "r"(taddr) : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld<8>(uint32_t taddr, float (&v)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+                 : "r"(taddr) : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, float (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
+          "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+        : "r"(taddr) : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, float (&v)[32]) {
+    tmem_ld32(taddr, v);
+}
+
+// ------------------------------------------------------------------ the kernel
+
+template <int NH, bool VALUE>
+__global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(const __grid_constant__ Params p) {
+    using C = Cfg<NH, VALUE>;
+    constexpr int kSlots = C::kSlots, kNHP = C::kNHP, kPH = C::kPH;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t base0 = smem_u32(smem_raw);
+    Smem<NH, VALUE> &sm = *reinterpret_cast<Smem<NH, VALUE> *>(smem_raw + ((1024u - (base0 & 1023u)) & 1023u));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int *abort = &sm.abort;
+
+    const long long NT = p.ntiles, CT = gridDim.x;
+    const long long x0 = tile_begin(blockIdx.x, CT, NT), x1 = tile_begin(blockIdx.x + 1, CT, NT);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kSlots; ++s) {
+            mbar_init(&sm.full[s], 32);
+            mbar_init(&sm.sfull[s], 1);
+            mbar_init(&sm.empty[s], 4);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.qfull[s], 1);
+            mbar_init(&sm.qempty[s], 1);
+        }
+        sm.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    // q~ rows past Hg stay zero for the whole kernel (the bulk copies write Hg rows), so the
+    // scores of padding heads are exactly zero
+    for (int i = threadIdx.x; i < 2 * 2 * kNHP * 128 / 16; i += kThreads)
+        reinterpret_cast<uint4 *>(&sm.qbuf[0][0][0])[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async();
+    if (warp == 1) tmem_alloc(&sm.tmem_base, C::kTmemCols);
+    tmem_fence_before();
+    __syncthreads();
+    tmem_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    // everything above overlaps the previous kernel's tail; its outputs (q~, the unit
+    // statistics) are read only from here on
+    griddep_launch_dependents();
+    griddep_wait();
+
+    if (warp == 0) {
+        // =============================================================== producer
+        uint32_t seq = 0, qseq = 0;
+        unsigned hi_head = 0, hi_tail = 0;
+        bool ok = true;
+        // wait until slot s may be refilled (its previous tile has been consumed)
+        auto acquire = [&](int s) -> bool {
+            if (seq >= (uint32_t)kSlots && !mbar_wait(&sm.empty[s], ((seq / kSlots) - 1) & 1u, abort)) return false;
+            return true;
+        };
+        // The CTA's mask words are one contiguous run (its tiles are consecutive 128-token tiles
+        // and a unit's words follow the previous unit's), read into shared memory a window at a
+        // time so that no tile waits on a global load of its mask.
+        const long long gw_end = (x1 - 1) / p.tpu * p.nwords +
+                                 (min(p.T, (int)((x1 - 1) % p.tpu + 1) * kTile) + 31) / 32;
+        long long wbase = -1;
+        auto mask_words = [&](long long gw, int nw) -> const uint32_t * {
+            if (wbase < 0 || gw < wbase || gw + nw > wbase + kMaskWin) {
+                wbase = gw;
+                const int cnt = (int)min((long long)kMaskWin, gw_end - gw);
+                __syncwarp();
+                for (int i = lane; i < cnt; i += 32) sm.mwin[i] = __ldg(p.mask + gw + i);
+                __syncwarp();
+            }
+            return sm.mwin + (gw - wbase);
+        };
+        long long x = x0;
+        while (ok && x < x1) {
+            const int unit = (int)(x / p.tpu);
+            const long long ue = (long long)(unit + 1) * p.tpu;
+            const long long xe = x1 < ue ? x1 : ue;
+            const int tok0 = (int)(x - (long long)unit * p.tpu) * kTile;
+            const int tok1 = min(p.T, (int)(xe - (long long)unit * p.tpu) * kTile);
+            const int pslot = (int)(blockIdx.x - cta_of_tile((long long)unit * p.tpu, CT, NT));
+            x = xe;
+            // the unit's q~ into the next q slot
+            const int qs = qseq & 1;
+            if (qseq >= 2 && !mbar_wait(&sm.qempty[qs], ((qseq >> 1) - 1) & 1u, abort)) { ok = false; break; }
+            if (lane == 0) {
+                const unsigned char *src = p.qt + (size_t)unit * qblock_bytes(p.Hg);
+                const uint32_t bytes = (uint32_t)p.Hg * 128u;
+                fence_proxy_async();
+                mbar_arrive_tx(&sm.qfull[qs], 2 * bytes);
+                bulk_g2s(&sm.qbuf[qs][0][0], src, bytes, &sm.qfull[qs]);
+                bulk_g2s(&sm.qbuf[qs][1][0], src + bytes, bytes, &sm.qfull[qs]);
+            }
+            ++qseq;
+            bool first = true;
+            for (int tok = tok0; tok < tok1 && ok; tok += C::kLoTok) {
+                const int n = min(C::kLoTok, tok1 - tok);
+                // the block's mask words (bits past n cleared) and its full-rank tokens
+                const uint32_t *mw = mask_words((long long)unit * p.nwords + (tok >> 5), (n + 31) >> 5);
+                uint32_t wd = 0u;
+                if (lane < C::kLoTok / 32 && 32 * lane < n) {
+                    wd = mw[lane];
+                    const int nb = n - 32 * lane;
+                    if (nb < 32) wd &= (1u << nb) - 1u;
+                }
+                const int c = __popc(wd);
+                int incl = c;
+                #pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+                    if (lane >= d) incl += v;
+                }
+                const int nhi = __shfl_sync(0xffffffffu, incl, 31);
+                {
+                    unsigned r = hi_tail + (unsigned)(incl - c);
+                    uint32_t bits = wd;
+                    while (bits) {
+                        sm.hi_ring[r % kHiRing] = (uint16_t)(tok + 32 * lane + __ffs(bits) - 1);
+                        ++r;
+                        bits &= bits - 1u;
+                    }
+                }
+                hi_tail += (unsigned)nhi;
+                __syncwarp();
+                const bool final_blk = tok + C::kLoTok >= tok1;
+                const unsigned pend = hi_tail - hi_head;
+                const int hi_now = (int)(pend / C::kHiTok) + ((final_blk && (pend % C::kHiTok) != 0) ? 1 : 0);
+                if (nhi < n) {
+                    // ------------------------------------------------ LO tile
+                    const int s = seq % kSlots;
+                    if (!acquire(s)) { ok = false; break; }
+                    int *d = sm.desc[s];
+                    if (lane == 0) {
+                        d[0] = kTypeLo | (first ? kFlagFirst : 0) | ((final_blk && hi_now == 0) ? kFlagLast : 0);
+                        d[1] = unit; d[2] = tok; d[3] = n; d[4] = pslot; d[5] = qs;
+                    }
+                    if (lane < C::kLoTok / 32) d[8 + lane] = (int)wd;
+                    first = false;
+                    if (!p.rank0) {
+                        const int nb = (n + 255) >> 8;   // 256-row boxes
+                        if (lane == 0) {
+                            unsigned char *dst = sm.slot[s];
+                            fence_proxy_async();
+                            mbar_arrive_tx(&sm.full[s], (uint32_t)nb * 8192u * (VALUE ? 2u : 1u));
+                            for (int b = 0; b < nb; ++b) {
+                                tma_3d(dst + 8192 * b, &p.tm_ck, 0, tok + 256 * b, unit, &sm.full[s]);
+                                if (VALUE) tma_3d(dst + C::kVOff + 8192 * b, &p.tm_cv, 0, tok + 256 * b, unit, &sm.full[s]);
+                            }
+                        } else {
+                            mbar_arrive(&sm.full[s]);
+                        }
+                    } else {
+                        mbar_arrive(&sm.full[s]);
+                    }
+                    ++seq;
+                }
+                for (int i = 0; i < hi_now && ok; ++i) {
+                    // ------------------------------------------------ HI tile
+                    const int s = seq % kSlots;
+                    if (!acquire(s)) { ok = false; break; }
+                    const int nh = (int)min((unsigned)C::kHiTok, hi_tail - hi_head);
+                    int *d = sm.desc[s];
+                    uint16_t *pos = reinterpret_cast<uint16_t *>(d + 8);
+                    if (lane == 0) {
+                        d[0] = kTypeHi | (first ? kFlagFirst : 0) | ((final_blk && i == hi_now - 1) ? kFlagLast : 0);
+                        d[1] = unit; d[2] = 0; d[3] = nh; d[4] = pslot; d[5] = qs;
+                    }
+                    #pragma unroll
+                    for (int k = 0; k < C::kHiTok / 32; ++k) {
+                        const int r = lane + 32 * k;
+                        pos[r] = r < nh ? sm.hi_ring[(hi_head + r) % kHiRing] : (uint16_t)0;
+                    }
+                    first = false;
+                    __syncwarp();
+                    // C_lo + C_hi rows into 128-byte rows (16-byte chunk c of row r at c ^ (r & 7));
+                    // V rows past nh are zero-filled (their p is zero, and 0 * stale data must stay 0)
+                    unsigned char *dst = sm.slot[s];
+                    const size_t ubase = (size_t)unit * p.T;
+                    #pragma unroll 4
+                    for (int k = 0; k < C::kHiTok * 8 / 32; ++k) {
+                        const int idx = lane + 32 * k;
+                        const int r = idx >> 3, ch = idx & 7;
+                        const bool valid = r < nh;
+                        const size_t row = ubase + pos[r];
+                        const int off = r * 128 + ((ch ^ (r & 7)) << 4);
+                        const uint16_t *sk = ch < 2 ? p.CK_lo + row * 16 + ch * 8 : p.CK_hi + row * 48 + (ch - 2) * 8;
+                        if (valid) cp_async16(dst + off, sk);
+                        if (VALUE) {
+                            const uint16_t *sv = ch < 2 ? p.CV_lo + row * 16 + ch * 8 : p.CV_hi + row * 48 + (ch - 2) * 8;
+                            cp_async16_zfill(dst + C::kVOff + off, sv, valid);
+                        }
+                    }
+                    cp_async_arrive(&sm.full[s]);   // raises the pending count; arrives when the copies land
+                    mbar_arrive(&sm.full[s]);       // releases this lane's descriptor writes
+                    hi_head += (unsigned)nh;
+                    ++seq;
+                }
+            }
+        }
+        // end marker
+        if (ok) {
+            const int s = seq % kSlots;
+            if (acquire(s)) {
+                if (lane == 0) sm.desc[s][0] = kTypeEnd;
+                mbar_arrive(&sm.full[s]);
+                ++seq;
+            } else {
+                ok = false;
+            }
+        }
+        if (!ok) *abort = 1;
+        // copies still in flight (only after an abort) must land before the block exits
+        cp_async_wait_all();
+        for (uint32_t k = (seq > (uint32_t)kSlots ? seq - kSlots : 0u); k < seq; ++k) {
+            const long long t0 = clock64();
+            while (!mbar_try_wait(&sm.full[k % kSlots], (k / kSlots) & 1u) && clock64() - t0 < kWaitCycles) {}
+        }
+    } else if (warp == 1) {
+        // =============================================================== MMA issuer
+        if (lane == 0) {
+            uint32_t seq = 0, qseq = 0, last_sfull = 0xffffffffu;
+            const uint32_t id_s = idesc_bf16_kk(128, kNHP);
+            while (true) {
+                const int s = seq % kSlots;
+                if (!mbar_wait(&sm.full[s], (seq / kSlots) & 1u, abort)) break;
+                // the descriptor is read before the commit below: once the consumers are done the
+                // producer may rewrite it
+                const int *d = sm.desc[s];
+                const int hdr = d[0];
+                const int type = hdr & 0xff;
+                if (type == kTypeEnd) break;
+                const int qs = d[5], n = d[3];
+                if (hdr & kFlagFirst) {
+                    if (!mbar_wait(&sm.qfull[qs], (qseq >> 1) & 1u, abort)) break;
+                    ++qseq;
+                }
+                const bool has_s = type == kTypeHi || !p.rank0;
+                if (has_s) {
+                    if (type == kTypeHi) fence_proxy_async();   // the gathered rows were written by cp.async
+                    tmem_fence_after();
+                    const uint32_t dcol = tmem + (uint32_t)(s * C::kSCols);
+                    const uint32_t qh = smem_u32(&sm.qbuf[qs][0][0]), ql = smem_u32(&sm.qbuf[qs][1][0]);
+                    const uint32_t sb = smem_u32(sm.slot[s]);
+                    if (type == kTypeLo) {
+                        for (int sub = 0; sub * kTile < n; ++sub) {
+                            const uint64_t a = desc_kmajor(sb + 4096u * sub, 256u, 6u);
+                            umma_bf16(dcol + sub * kNHP, a, desc_kmajor(qh, 1024u, 2u), id_s, 0u);
+                            umma_bf16(dcol + sub * kNHP, a, desc_kmajor(ql, 1024u, 2u), id_s, 1u);
+                        }
+                    } else {
+                        #pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t a = desc_kmajor(sb + 32u * k, 1024u, 2u);
+                            umma_bf16(dcol, a, desc_kmajor(qh + 32u * k, 1024u, 2u), id_s, k > 0 ? 1u : 0u);
+                            umma_bf16(dcol, a, desc_kmajor(ql + 32u * k, 1024u, 2u), id_s, 1u);
+                        }
+                    }
+                    umma_commit(&sm.sfull[s]);
+                    last_sfull = seq;
+                } else {
+                    mbar_arrive(&sm.sfull[s]);   // keeps the slot's score-barrier phases in step
+                }
+                if (hdr & kFlagLast) umma_commit(&sm.qempty[qs]);
+                ++seq;
+            }
+            // MMAs still in flight (only after an abort) must finish before tensor memory is freed
+            if (last_sfull != 0xffffffffu) {
+                const long long t0 = clock64();
+                while (!mbar_try_wait(&sm.sfull[last_sfull % kSlots], (last_sfull / kSlots) & 1u) &&
+                       clock64() - t0 < kWaitCycles) {}
+            }
+        }
+        __syncwarp();
+    } else {
+        // =============================================================== consumers
+        const int q = warp & 3;                       // tensor-memory lane quarter
+        const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+        const int g = lane >> 2, tig = lane & 3;
+        uint32_t seq = 0;
+        // per-segment state
+        float m[NH], l[NH];                            // stats pass: this thread's reference max and sum per head
+        float Mh[NH], ILh[NH];                         // value pass: the unit's (M, 1/L) per head
+        float u[4][kPH / 8][4];                        // value pass: u^T (ranks on M, heads on N) of this warp
+        (void)m; (void)l; (void)Mh; (void)ILh; (void)u;
+        int unit = 0, pslot = 0;
+        unsigned char *pb = sm.pbuf[VALUE ? q : 0];
+        const uint32_t pb_s = smem_u32(pb);
+        while (true) {
+            const int s = seq % kSlots;
+            if (!mbar_wait(&sm.full[s], (seq / kSlots) & 1u, abort)) break;
+            const int *d = sm.desc[s];
+            const int hdr = d[0];                    // read before this warp releases the slot
+            const int type = hdr & 0xff;
+            if (type == kTypeEnd) break;
+            const int n = d[3];
+            if (hdr & kFlagFirst) {
+                unit = d[1];
+                pslot = d[4];
+                if (VALUE) {
+                    #pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        float2 st = make_float2(0.f, 0.f);
+                        if (h < p.Hg) st = __ldg(reinterpret_cast<const float2 *>(p.ustat + ((size_t)unit * p.Hg + h) * 2));
+                        Mh[h] = st.x;
+                        ILh[h] = st.y;
+                    }
+                    #pragma unroll
+                    for (int a = 0; a < 4; ++a)
+                        #pragma unroll
+                        for (int b = 0; b < kPH / 8; ++b) u[a][b][0] = u[a][b][1] = u[a][b][2] = u[a][b][3] = 0.f;
+                } else {
+                    #pragma unroll
+                    for (int h = 0; h < NH; ++h) { m[h] = kRefInit; l[h] = 0.f; }
+                }
+            }
+            const bool has_s = type == kTypeHi || !p.rank0;
+            if (!mbar_wait(&sm.sfull[s], (seq / kSlots) & 1u, abort)) break;
+            tmem_fence_after();
+            const int nsub = type == kTypeLo ? (n + kTile - 1) / kTile : 1;
+            const uint32_t sb = smem_u32(sm.slot[s]);
+            // the scores of up to kLd sub-tiles are loaded from tensor memory before one wait
+            constexpr int kLd = (C::kSub * NH <= 64) ? C::kSub : (64 / NH > 0 ? 64 / NH : 1);
+            for (int sub0 = 0; sub0 < nsub; sub0 += kLd) {
+                float scv[kLd][NH];
+                #pragma unroll
+                for (int j = 0; j < kLd; ++j) {
+                    const int sub = sub0 + j;
+                    if (has_s && sub < nsub && sub * kTile + 32 * q < n) {
+                        constexpr int NL = NH < 4 ? 4 : NH;
+                        float v[NL];
+                        tmem_ld<NL>(tmem + lane_addr + (uint32_t)(s * C::kSCols + sub * kNHP), v);
+                        #pragma unroll
+                        for (int h = 0; h < NH; ++h) scv[j][h] = v[h];
+                    } else {
+                        #pragma unroll
+                        for (int h = 0; h < NH; ++h) scv[j][h] = 0.f;
+                    }
+                }
+                if (has_s) tmem_wait_ld();
+                #pragma unroll
+                for (int j = 0; j < kLd; ++j) {
+                const int sub = sub0 + j;
+                if (sub >= nsub || sub * kTile + 32 * q >= n) continue;   // no token of this warp here
+                const int r = sub * kTile + 32 * q + lane;    // row of this thread's token in the tile
+                bool take;
+                int pos;
+                if (type == kTypeLo) {
+                    const uint32_t wd = (uint32_t)d[8 + 4 * sub + q];
+                    take = r < n && !((wd >> lane) & 1u);
+                    pos = d[2] + r;
+                } else {
+                    take = r < n;
+                    pos = reinterpret_cast<const uint16_t *>(d + 8)[r];
+                }
+                const float (&sc)[NH] = scv[j];
+                if (!VALUE) {
+                    // ---------------------------------------------------- stats
+                    if (take) {
+                        float mx = sc[0] - m[0];
+                        #pragma unroll
+                        for (int h = 1; h < NH; ++h) mx = fmaxf(mx, sc[h] - m[h]);
+                        if (mx > kLazy) {
+                            #pragma unroll
+                            for (int h = 0; h < NH; ++h)
+                                if (sc[h] > m[h]) {
+                                    l[h] *= ex2(m[h] - sc[h]);
+                                    m[h] = sc[h];
+                                }
+                        }
+                        #pragma unroll
+                        for (int h = 0; h < NH; ++h) l[h] += ex2(sc[h] - m[h]);
+                    }
+                } else {
+                    // ---------------------------------------------------- value
+                    float pr[kPH];
+                    float ms0 = 0.f, ms1 = 0.f;
+                    #pragma unroll
+                    for (int h = 0; h < kPH; ++h) {
+                        if (h < NH) {
+                            const float e = take ? ex2(sc[h] - Mh[h]) : 0.f;
+                            pr[h] = e;
+                            if (h & 1) ms1 = fmaf(e, ILh[h], ms1);
+                            else ms0 = fmaf(e, ILh[h], ms0);
+                        } else {
+                            pr[h] = 0.f;
+                        }
+                    }
+                    if (take && p.mass != nullptr) p.mass[(size_t)unit * p.T + pos] = ms0 + ms1;
+                    const bool do_u = type == kTypeHi || !p.rank0;
+                    if (do_u) {
+                        // this thread's P row (kPH bf16), 16-byte chunks swizzled against bank conflicts
+                        const int prow = lane;
+                        #pragma unroll
+                        for (int c = 0; c < kPH / 8; ++c) {
+                            uint4 v;
+                            v.x = pack_bf16(pr[8 * c + 0], pr[8 * c + 1]);
+                            v.y = pack_bf16(pr[8 * c + 2], pr[8 * c + 3]);
+                            v.z = pack_bf16(pr[8 * c + 4], pr[8 * c + 5]);
+                            v.w = pack_bf16(pr[8 * c + 6], pr[8 * c + 7]);
+                            int pc = c;
+                            if (kPH == 16) pc = c ^ ((prow >> 2) & 1);
+                            if (kPH == 32) pc = c ^ ((prow >> 1) & 3);
+                            *reinterpret_cast<uint4 *>(pb + prow * (kPH * 2) + pc * 16) = v;
+                        }
+                        __syncwarp();
+                        // u^T += C_V^T P over the warp's 32 tokens (two k-steps of 16)
+                        #pragma unroll
+                        for (int kk = 0; kk < 2; ++kk) {
+                            uint32_t bfr[kPH / 8][2];
+                            #pragma unroll
+                            for (int np = 0; np < (kPH + 15) / 16; ++np) {
+                                const int row = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
+                                int ch = 2 * np + (lane >> 4);
+                                if (kPH == 8) ch = 0;
+                                int pc = ch;
+                                if (kPH == 16) pc = ch ^ ((row >> 2) & 1);
+                                if (kPH == 32) pc = ch ^ ((row >> 1) & 3);
+                                uint32_t r0, r1, r2, r3;
+                                if (kPH == 8) {
+                                    // x2: tokens 0-7 and 8-15 of the 8 heads
+                                    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+                                                 : "=r"(r0), "=r"(r1) : "r"(pb_s + row * (kPH * 2) + (pc << 4)));
+                                    bfr[0][0] = r0;
+                                    bfr[0][1] = r1;
+                                } else {
+                                    ldsm_x4_t(pb_s + row * (kPH * 2) + (pc << 4), r0, r1, r2, r3);
+                                    bfr[2 * np][0] = r0;
+                                    bfr[2 * np][1] = r1;
+                                    bfr[2 * np + 1][0] = r2;
+                                    bfr[2 * np + 1][1] = r3;
+                                }
+                            }
+                            const int tb = sub * kTile + 32 * q + 16 * kk;   // first token row of the k-step
+                            if (type == kTypeLo) {
+                                uint32_t a[4];
+                                const int row = tb + (lane & 7) + ((lane >> 4) << 3);
+                                const int ch = (lane >> 3) & 1;
+                                ldsm_x4_t(sb + C::kVOff + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), a[0], a[1], a[2], a[3]);
+                                #pragma unroll
+                                for (int nt = 0; nt < kPH / 8; ++nt) mma_bf16(u[0][nt], a, bfr[nt][0], bfr[nt][1]);
+                            } else {
+                                #pragma unroll
+                                for (int mt = 0; mt < 4; ++mt) {
+                                    uint32_t a[4];
+                                    const int row = tb + (lane & 7) + ((lane >> 4) << 3);
+                                    const int ch = 2 * mt + ((lane >> 3) & 1);
+                                    ldsm_x4_t(sb + C::kVOff + row * 128 + ((ch ^ (row & 7)) << 4), a[0], a[1], a[2], a[3]);
+                                    #pragma unroll
+                                    for (int nt = 0; nt < kPH / 8; ++nt) mma_bf16(u[mt][nt], a, bfr[nt][0], bfr[nt][1]);
+                                }
+                            }
+                        }
+                        __syncwarp();
+                    }
+                }
+                }
+            }
+            // this slot is free once every consumer warp has read its scores (and, in the value pass, its V rows)
+            tmem_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[s]);
+
+            if (hdr & kFlagLast) {
+                // ---------------------------------------------------------- the segment's partial
+                if (!VALUE) {
+                    // (m, l) per head: over the warp's lanes, then over the four warps in a fixed order
+                    #pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        float mw = m[h];
+                        #pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) mw = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, o));
+                        float lw = l[h] * ex2(m[h] - mw);
+                        #pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+                        if (lane == 0) {
+                            sm.merge[q][2 * h] = mw;
+                            sm.merge[q][2 * h + 1] = lw;
+                        }
+                    }
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    if (q == 0 && lane < NH && lane < p.Hg) {
+                        float mx = sm.merge[0][2 * lane];
+                        #pragma unroll
+                        for (int w = 1; w < 4; ++w) mx = fmaxf(mx, sm.merge[w][2 * lane]);
+                        float sum = 0.f;
+                        #pragma unroll
+                        for (int w = 0; w < 4; ++w) sum += sm.merge[w][2 * lane + 1] * ex2(sm.merge[w][2 * lane] - mx);
+                        float *dst = p.part + (((size_t)unit * p.nslot + pslot) * p.Hg + lane) * 2;
+                        dst[0] = mx;
+                        dst[1] = sum;
+                    }
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                } else {
+                    // u per head: warps 1-3 park theirs in shared memory, warp 0 adds them in order
+                    if (q != 0) {
+                        #pragma unroll
+                        for (int mt = 0; mt < 4; ++mt)
+                            #pragma unroll
+                            for (int nt = 0; nt < kPH / 8; ++nt)
+                                #pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int rr = 16 * mt + g + 8 * (e >> 1), hh = 8 * nt + 2 * tig + (e & 1);
+                                    if (hh < NH) sm.merge[q - 1][hh * 64 + rr] = u[mt][nt][e];
+                                }
+                    }
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    if (q == 0) {
+                        float *dst = p.part + ((size_t)unit * p.nslot + pslot) * p.Hg * 64;
+                        #pragma unroll
+                        for (int mt = 0; mt < 4; ++mt)
+                            #pragma unroll
+                            for (int nt = 0; nt < kPH / 8; ++nt)
+                                #pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int rr = 16 * mt + g + 8 * (e >> 1), hh = 8 * nt + 2 * tig + (e & 1);
+                                    if (hh < NH && hh < p.Hg) {
+                                        float v = u[mt][nt][e];
+                                        v += sm.merge[0][hh * 64 + rr];
+                                        v += sm.merge[1][hh * 64 + rr];
+                                        v += sm.merge[2][hh * 64 + rr];
+                                        dst[hh * 64 + rr] = v;
+                                    }
+                                }
+                    }
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                }
+            }
+            ++seq;
+        }
+    }
+
+    tmem_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tmem_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ combine
+
+// Per unit and query head (one warp per unit, a lane per head): the unit-wide max M and
+// sum L over the stats pass's segment partials and the text tail's chunk partials; writes
+// (M, 1/L) for the value pass and the finish.
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ spart, const float *__restrict__ tpart,
+                                                      float *__restrict__ ustat, int units, int Hg, int Sc, int nslot,
+                                                      long long ntiles, int tpu, int cta_s) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const int unit = blockIdx.x * 8 + (threadIdx.x >> 5), h = threadIdx.x & 31;
+    if (unit >= units || h >= Hg) return;
+    const long long f = (long long)unit * tpu;
+    const int c0 = (int)cta_of_tile(f, cta_s, ntiles), c1 = (int)cta_of_tile(f + tpu - 1, cta_s, ntiles);
+    const float *sp = spart + ((size_t)unit * nslot * Hg + h) * 2;
+    const float *tp = tpart + (size_t)unit * Sc * Hg * kTxtPart + (size_t)h * kTxtPart;
+    float mx = -INFINITY;
+    for (int k = 0; k <= c1 - c0; ++k) mx = fmaxf(mx, sp[(size_t)k * Hg * 2]);
+    for (int c = 0; c < Sc; ++c) mx = fmaxf(mx, tp[(size_t)c * Hg * kTxtPart]);
+    float sum = 0.f;
+    for (int k = 0; k <= c1 - c0; ++k) sum += sp[(size_t)k * Hg * 2 + 1] * ex2(sp[(size_t)k * Hg * 2] - mx);
+    for (int c = 0; c < Sc; ++c) {
+        const float mc = tp[(size_t)c * Hg * kTxtPart];
+        if (mc != -INFINITY) sum += tp[(size_t)c * Hg * kTxtPart + 1] * ex2(mc - mx);
+    }
+    *reinterpret_cast<float2 *>(ustat + ((size_t)unit * Hg + h) * 2) = make_float2(mx, 1.f / sum);
+}
+
+// ------------------------------------------------------------------ finish
+
+struct FinishParams {
+    const uint16_t *BV;       // [units][64][512]
+    const float *vpart;       // [units][nslot][Hg][64]: u = sum p' C_V per segment
+    const float *tpart;       // [units][Sc][Hg][kTxtPart] or null
+    const float *ustat;       // [units][Hg][2]: (M, 1/L)
+    uint16_t *out;            // [(layer, batch)][n_q][128]
+    int Hg, per_kv, n_q, groups, Sc, nslot, tpu, cta_v;
+    long long ntiles;
+};
+
+// One block of 128 threads per (unit, KV head j): u_h = the sum of the unit's segment
+// partials, w_h = the text chunks' sums weighted by 2^(m_c - M_h), then
+// o_h = (u_h B_V[:, 128 j ..] + w_h) / L_h for the PK query heads of KV head j, thread t
+// owning output feature t.  The loads of each stage are independent of one another (the
+// chunk weights are computed once into shared memory first), so they are all in flight at once.
+constexpr int kFinishMaxChunks = 64;   // text chunks whose weights are staged; longer tails loop
+
+template <int PK>
+__global__ void __launch_bounds__(128) finish_kernel(const FinishParams p) {
+    __shared__ float uf[PK][64];
+    __shared__ float ew[PK][kFinishMaxChunks];
+    __shared__ float ms[PK][2];
+    griddep_wait();
+    const int unit = blockIdx.x >> 2, j = blockIdx.x & 3, tid = threadIdx.x;
+    const int h0 = j * PK;
+    // B_V[:, 128 j + tid] for all 64 ranks: issued first, used last
+    const uint16_t *bv = p.BV + (size_t)unit * 64 * 512 + 128 * j + tid;
+    uint16_t braw[64];
+    #pragma unroll
+    for (int r = 0; r < 64; ++r) braw[r] = __ldcs(bv + (size_t)r * 512);
+    if (tid < PK) {
+        const float2 st = __ldg(reinterpret_cast<const float2 *>(p.ustat + ((size_t)unit * p.Hg + h0 + tid) * 2));
+        ms[tid][0] = st.x;
+        ms[tid][1] = st.y;
+    }
+    const long long f = (long long)unit * p.tpu;
+    const int ns = (int)(cta_of_tile(f + p.tpu - 1, p.cta_v, p.ntiles) - cta_of_tile(f, p.cta_v, p.ntiles)) + 1;
+    for (int i = tid; i < PK * 64; i += 128) {
+        const int hh = i >> 6, r = i & 63;
+        const float *src = p.vpart + ((size_t)unit * p.nslot * p.Hg + h0 + hh) * 64 + r;
+        float a = 0.f;
+        for (int k = 0; k < ns; ++k) a += __ldcg(src + (size_t)k * p.Hg * 64);
+        uf[hh][r] = a;
+    }
+    __syncthreads();
+    float wacc[PK];
+    #pragma unroll
+    for (int hh = 0; hh < PK; ++hh) wacc[hh] = 0.f;
+    if (p.tpart != nullptr) {
+        const float *tp0 = p.tpart + ((size_t)unit * p.Sc * p.Hg + h0) * kTxtPart;
+        for (int c0 = 0; c0 < p.Sc; c0 += kFinishMaxChunks) {
+            const int nc = min(kFinishMaxChunks, p.Sc - c0);
+            for (int i = tid; i < PK * nc; i += 128) {
+                const int hh = i / nc, c = i % nc;
+                const float mc = __ldcg(tp0 + ((size_t)(c0 + c) * p.Hg + hh) * kTxtPart);
+                ew[hh][c] = mc != -INFINITY ? ex2(mc - ms[hh][0]) : 0.f;
+            }
+            __syncthreads();
+            #pragma unroll
+            for (int hh = 0; hh < PK; ++hh) {
+                const float *tp = tp0 + (size_t)hh * kTxtPart + 2 + tid;
+                float a0 = 0.f, a1 = 0.f;
+                int c = 0;
+                for (; c + 1 < nc; c += 2) {
+                    a0 = fmaf(__ldcg(tp + (size_t)(c0 + c) * p.Hg * kTxtPart), ew[hh][c], a0);
+                    a1 = fmaf(__ldcg(tp + (size_t)(c0 + c + 1) * p.Hg * kTxtPart), ew[hh][c + 1], a1);
+                }
+                if (c < nc) a0 = fmaf(__ldcg(tp + (size_t)(c0 + c) * p.Hg * kTxtPart), ew[hh][c], a0);
+                wacc[hh] += a0 + a1;
+            }
+            __syncthreads();
+        }
+    }
+    float acc[PK];
+    #pragma unroll
+    for (int hh = 0; hh < PK; ++hh) acc[hh] = 0.f;
+    #pragma unroll
+    for (int r = 0; r < 64; ++r) {
+        const float b = __uint_as_float((uint32_t)braw[r] << 16);
+        #pragma unroll
+        for (int hh = 0; hh < PK; ++hh) acc[hh] = fmaf(uf[hh][r], b, acc[hh]);
+    }
+    const int lb = unit / p.groups, G = unit % p.groups;
+    #pragma unroll
+    for (int hh = 0; hh < PK; ++hh) {
+        const float o = (acc[hh] + wacc[hh]) * ms[hh][1];
+        p.out[((size_t)lb * p.n_q + (size_t)G * p.Hg + h0 + hh) * 128 + tid] = float_to_bf16_bits(o);
+    }
+}
+
+}  // namespace rs
+}  // namespace decode
+}  // namespace kvpack

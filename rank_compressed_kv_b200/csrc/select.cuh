@@ -86,9 +86,22 @@ __device__ __forceinline__ int group_exclusive_scan(int v, int *red) {
     }
 }
 
+// Keys of the unit: KR per thread in registers, the other KS = KPT - KR in shared memory
+// (a 1024-thread block has 64 registers per thread, too few for 64 keys and the rest).
+template <int KPT, int NW>
+struct KeySplit {
+    static constexpr int KR = (NW > 1 && KPT > 32) ? 32 : KPT;
+    static constexpr int KS = KPT - KR;
+};
+
+template <int KPT, int NW>
+constexpr size_t select_smem_bytes() { return (size_t)KeySplit<KPT, NW>::KS * 32 * NW * sizeof(uint32_t); }
+
 template <int KPT, int NW>
 __global__ void __launch_bounds__(NW == 1 ? 256 : 32 * NW) select_kernel(Params p) {
+    constexpr int KR = KeySplit<KPT, NW>::KR, KS = KeySplit<KPT, NW>::KS;
     __shared__ int red[64];
+    extern __shared__ uint32_t skeys[];     // [KS][threads]: key KR + i of thread r at [i][r]
     int unit, r;
     if constexpr (NW == 1) {
         unit = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -102,20 +115,23 @@ __global__ void __launch_bounds__(NW == 1 ? 256 : 32 * NW) select_kernel(Params 
     const size_t ub = (size_t)unit * T;
     const float one_minus = __fsub_rn(1.0f, p.alpha);
 
-    uint32_t key[KPT];
-    #pragma unroll
-    for (int i = 0; i < KPT; ++i) {
+    auto load_key = [&](int i) -> uint32_t {
         const int t = r * KPT + i;
-        key[i] = 0u;
-        if (t < T) {
-            const float m = p.mass[ub + t];
-            float x;
-            if (p.alpha == 0.0f) x = m;
-            else x = __fmaf_rn(p.alpha, p.score[ub + t], __fmul_rn(one_minus, m));
-            if (p.score != nullptr) p.score[ub + t] = x;
-            key[i] = ordered_key(x);
-        }
+        if (t >= T) return 0u;
+        const float m = p.mass[ub + t];
+        float x;
+        if (p.alpha == 0.0f) x = m;
+        else x = __fmaf_rn(p.alpha, p.score[ub + t], __fmul_rn(one_minus, m));
+        if (p.score != nullptr) p.score[ub + t] = x;
+        return ordered_key(x);
+    };
+    uint32_t key[KR];
+    #pragma unroll
+    for (int i = 0; i < KR; ++i) key[i] = load_key(i);
+    if constexpr (KS > 0) {
+        for (int i = 0; i < KS; ++i) skeys[i * blockDim.x + r] = load_key(KR + i);
     }
+    auto skey = [&](int i) -> uint32_t { return skeys[i * blockDim.x + r]; };
 
     uint32_t *out = p.mask + (size_t)unit * p.nwords;
     if (p.k <= 0) {
@@ -129,14 +145,25 @@ __global__ void __launch_bounds__(NW == 1 ? 256 : 32 * NW) select_kernel(Params 
         const uint32_t cand = theta | (1u << bit);
         int c = 0;
         #pragma unroll
-        for (int i = 0; i < KPT; ++i) c += (key[i] >= cand) ? 1 : 0;
+        for (int i = 0; i < KR; ++i) c += (key[i] >= cand) ? 1 : 0;
+        if constexpr (KS > 0) {
+            #pragma unroll 8
+            for (int i = 0; i < KS; ++i) c += (skey(i) >= cand) ? 1 : 0;
+        }
         if (group_sum<NW>(c, red) >= p.k) theta = cand;
     }
     int gt = 0, eq = 0;
     #pragma unroll
-    for (int i = 0; i < KPT; ++i) {
+    for (int i = 0; i < KR; ++i) {
         gt += (key[i] > theta) ? 1 : 0;
         eq += (key[i] == theta) ? 1 : 0;
+    }
+    if constexpr (KS > 0) {
+        for (int i = 0; i < KS; ++i) {
+            const uint32_t kk = skey(i);
+            gt += (kk > theta) ? 1 : 0;
+            eq += (kk == theta) ? 1 : 0;
+        }
     }
     const int need = p.k - group_sum<NW>(gt, red);      // equal keys to take, >= 1
     int before = group_exclusive_scan<NW>(eq, red);     // equal keys at lower token indices
@@ -149,8 +176,11 @@ __global__ void __launch_bounds__(NW == 1 ? 256 : 32 * NW) select_kernel(Params 
             #pragma unroll
             for (int b = 0; b < 32; ++b) {
                 const int i = wd * 32 + b;
-                bool s = key[i] > theta;
-                if (key[i] == theta) { s = before < need; ++before; }
+                uint32_t kk;
+                if (i < KR) kk = key[i < KR ? i : 0];
+                else kk = skey(i - KR);
+                bool s = kk > theta;
+                if (kk == theta) { s = before < need; ++before; }
                 if (s) bits |= 1u << b;
             }
             const int widx = r * (KPT / 32) + wd;

@@ -17,8 +17,8 @@ def u32(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint32).view(np.int32)).to(DEV)
 
 
-def run_decode(kv, w, c, n_layers, T, Lcap, L_text, scale=1.0, want_mass=True):
-    dims = kv.Dims(batch=w.batch, n_q_heads=w.n_q, n_kv_heads=w.n_kv, T_vis=T, L_text_cap=Lcap)
+def run_decode(kv, w, c, n_layers, T, Lcap, L_text, scale=1.0, want_mass=True, rank_lo=16):
+    dims = kv.Dims(batch=w.batch, n_q_heads=w.n_q, n_kv_heads=w.n_kv, T_vis=T, L_text_cap=Lcap, rank_lo=rank_lo)
     g = {k: bf(c[k]) for k in ("q", "CK_lo", "CK_hi", "BK", "CV_lo", "CV_hi", "BV", "K_text", "V_text")}
     mask = u32(c["mask"])
     out = torch.full((n_layers * w.batch, w.n_q, 128), float("nan"), dtype=torch.bfloat16, device=DEV)
@@ -32,10 +32,11 @@ def run_decode(kv, w, c, n_layers, T, Lcap, L_text, scale=1.0, want_mass=True):
     return o, (mass.cpu().numpy() if want_mass else None)
 
 
-def oracle_decode(w, c, L_text, scale=1.0):
+def oracle_decode(w, c, L_text, scale=1.0, rank_lo=16):
     f = oracle.bf16_to_f64
     return oracle.decode(f(c["CK"]), f(c["BK"]), f(c["CV"]), f(c["BV"]), f(c["K_text"][:, :L_text]),
-                         f(c["V_text"][:, :L_text]), c["mask"], f(cases.per_unit_queries(w, c["q"])), scale=scale)
+                         f(c["V_text"][:, :L_text]), c["mask"], f(cases.per_unit_queries(w, c["q"])), scale=scale,
+                         r_lo=rank_lo)
 
 
 def assert_decode_close(w, got_out, got_mass, ref_out, ref_mass, mass_rtol=1e-4):

@@ -64,6 +64,7 @@ def test_decode_rejects_bad_arguments_before_launch(kv):
     assert _call_decode(kv, _dims(kv, n_q_heads=12)) == 3
     assert _call_decode(kv, _dims(kv, n_q_heads=72, n_kv_heads=8)) == 3      # Hg = 36 > 32
     assert _call_decode(kv, _dims(kv, T_vis=65537)) == 3
+    assert _call_decode(kv, _dims(kv, rank_lo=8)) == 3          # reduced rank is 16 or 0 (not decompressed)
     assert _call_decode(kv, _dims(kv, T_vis=0)) == 1
     assert _call_decode(kv, _dims(kv, batch=0)) == 1
     assert _call_decode(kv, _dims(kv), n_layers=0) == 1
@@ -91,6 +92,11 @@ def test_compress_rejects_bad_arguments_before_launch(kv):
     assert lib.kvpack_compress(ctypes.byref(d.c()), 1, 0x1000, 0x1000, 0x1000, 0x1000, None, 0x1000, ws - 1, None) == 4
     assert lib.kvpack_compress(ctypes.byref(d.c()), 1, 0x1002, 0x1000, 0x1000, 0x1000, None, 0x1000, ws, None) == 2
     assert lib.kvpack_compress(ctypes.byref(d.c()), 1, None, 0x1000, 0x1000, 0x1000, None, 0x1000, ws, None) == 1
+
+
+def test_rank_zero_variant_is_a_supported_shape(kv):
+    assert kv.decode_workspace(_dims(kv, rank_lo=0), 1) == kv.decode_workspace(_dims(kv), 1) > 0
+    assert kv.decode_workspace(_dims(kv, rank_lo=8), 1) == 0
 
 
 def test_workspace_grows_with_splits(kv):

@@ -2,9 +2,9 @@
 
 Small shapes that still span several 128-token tiles, HI stages and text
 stages, with ragged tails, T = 1, empty text, all-full / all-reduced masks,
-every head-group size (Hg 4 / 16 / 28 / 32), units split into many visual
-items (long_split14: 79 items of 256 tokens) and multi-layer, multi-batch unit
-indexing."""
+every head-group size (Hg 4 / 8 / 16 / 28 / 32), a unit split over many CTAs
+(long_split: 20000 tokens), multi-layer, multi-batch unit indexing, and the
+rank-0 variant (low-importance tokens not decompressed at all: r_lo = 0)."""
 import numpy as np
 import pytest
 
@@ -15,29 +15,34 @@ from gpu_util import assert_decode_close, oracle_decode, run_decode
 pytestmark = pytest.mark.gpu
 
 CASES = [
-    # name,          batch, layers, n_q, n_kv, T,     Lcap, L_text, mask
-    ("c0",           1, 1, 8, 8, 576, 32, 32, "random"),
-    ("ragged_T",     1, 1, 8, 8, 1000, 40, 37, "random"),
-    ("T1",           2, 1, 8, 8, 1, 4, 3, "ones"),
-    ("T1_lowrank",   1, 1, 8, 8, 1, 4, 0, "zeros"),
-    ("no_text",      1, 2, 8, 8, 200, 16, 0, "random"),
-    ("all_full",     1, 1, 8, 8, 333, 20, 20, "ones"),
-    ("all_reduced",  1, 1, 8, 8, 333, 20, 20, "zeros"),
-    ("gqa16_split2", 2, 1, 32, 8, 3000, 64, 50, "random"),
-    ("gqa28_split3", 1, 2, 28, 4, 2000, 48, 48, "random"),
-    ("gqa32",        1, 1, 64, 8, 900, 16, 9, "random"),
-    ("many_units",   3, 2, 16, 16, 100, 8, 5, "random"),
-    ("long_split14", 1, 1, 32, 8, 20000, 300, 271, "random"),
+    # name,          batch, layers, n_q, n_kv, T,     Lcap, L_text, mask, r_lo
+    ("c0",           1, 1, 8, 8, 576, 32, 32, "random", 16),
+    ("ragged_T",     1, 1, 8, 8, 1000, 40, 37, "random", 16),
+    ("T1",           2, 1, 8, 8, 1, 4, 3, "ones", 16),
+    ("T1_lowrank",   1, 1, 8, 8, 1, 4, 0, "zeros", 16),
+    ("no_text",      1, 2, 8, 8, 200, 16, 0, "random", 16),
+    ("all_full",     1, 1, 8, 8, 333, 20, 20, "ones", 16),
+    ("all_reduced",  1, 1, 8, 8, 333, 20, 20, "zeros", 16),
+    ("gqa8",         1, 1, 16, 8, 700, 16, 16, "random", 16),
+    ("gqa16_split2", 2, 1, 32, 8, 3000, 64, 50, "random", 16),
+    ("gqa28_split3", 1, 2, 28, 4, 2000, 48, 48, "random", 16),
+    ("gqa32",        1, 1, 64, 8, 900, 16, 9, "random", 16),
+    ("many_units",   3, 2, 16, 16, 100, 8, 5, "random", 16),
+    ("long_split",   1, 1, 32, 8, 20000, 300, 271, "random", 16),
+    ("rank0_c0",     1, 1, 8, 8, 576, 32, 32, "random", 0),
+    ("rank0_gqa28",  1, 1, 28, 4, 2000, 48, 30, "random", 0),
+    ("rank0_no_text", 2, 1, 32, 8, 3000, 8, 0, "random", 0),
+    ("rank0_all_zero", 1, 1, 8, 8, 300, 8, 5, "zeros", 0),
 ]
 
 
-@pytest.mark.parametrize("name,batch,layers,n_q,n_kv,T,Lcap,L_text,mask", CASES, ids=[c[0] for c in CASES])
-def test_decode_matches_oracle(name, batch, layers, n_q, n_kv, T, Lcap, L_text, mask):
+@pytest.mark.parametrize("name,batch,layers,n_q,n_kv,T,Lcap,L_text,mask,r_lo", CASES, ids=[c[0] for c in CASES])
+def test_decode_matches_oracle(name, batch, layers, n_q, n_kv, T, Lcap, L_text, mask, r_lo):
     import rank_compressed_kv_b200 as kv
     w = synth.Workload(name, 100 + len(name), batch, layers, n_q, n_kv, T, Lcap, 1, "lowrank32")
     c = cases.decode_case(w, n_layers=layers, T=T, Lcap=Lcap, mask=mask)
-    got_o, got_m = run_decode(kv, w, c, layers, T, Lcap, L_text)
-    ref_o, ref_m = oracle_decode(w, c, L_text)
+    got_o, got_m = run_decode(kv, w, c, layers, T, Lcap, L_text, rank_lo=r_lo)
+    ref_o, ref_m = oracle_decode(w, c, L_text, rank_lo=r_lo)
     assert np.all(np.isfinite(got_o))
     assert_decode_close(w, got_o, got_m, ref_o, ref_m)
 
