@@ -149,6 +149,44 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *dims, int32_t n_layers,
                                  uint16_t *out, float *mass,
                                  void *ws, size_t ws_bytes, void *stream);
 
+/* ------------------------------------------- decode step, text compressed too
+ * kvpack_decode_attn_tb -- the decode step of kvpack_decode_attn when the text
+ * tokens are SVD-compressed as well, with a basis of their own (the visual and
+ * the text tokens are factored separately: Methodologie 2.A on the fr page,
+ * Metodologia 2.A on the es page).  A unit's attention then runs over
+ *   T visual tokens    at their mask's rank, through the visual basis (as in
+ *                      kvpack_decode_attn),
+ *   tb->L_c text tokens at the full rank 64, through the text basis:
+ *                      s_h,t = scale * C_K'[t, :] . (B_K'[:, 128 j : +128] q_h),
+ *                      value C_V'[t, :] B_V'[:, 128 j : +128],
+ *   L_text tokens      of the uncompressed tail (the tokens generated since the
+ *                      text was compressed), as in kvpack_decode_attn,
+ * with one softmax over all T + L_c + L_text logits.  The text planes follow the
+ * visual layouts with L_c in place of T (C_K' lo [units][L_c][16], hi
+ * [units][L_c][48], B_K' [units][64][512], the same for V); mass covers the
+ * visual tokens only.  tb->L_c = 0 gives exactly kvpack_decode_attn.
+ * ws must hold kvpack_decode_tb_workspace(dims, n_layers, tb->L_c) bytes; all
+ * other arguments, results and errors are those of kvpack_decode_attn, plus
+ * KVPACK_ERR_INVALID_ARG for a null tb, L_c < 0 or > KVPACK_MAX_T, or a null
+ * text plane when L_c > 0.
+ */
+typedef struct kvpack_text_basis {
+    const uint16_t *CK_lo, *CK_hi, *BK;
+    const uint16_t *CV_lo, *CV_hi, *BV;
+    int32_t L_c;
+} kvpack_text_basis;
+
+size_t kvpack_decode_tb_workspace(const kvpack_dims *dims, int32_t n_layers, int32_t L_c);
+kvpack_status kvpack_decode_attn_tb(const kvpack_dims *dims, int32_t n_layers,
+                                    const uint16_t *q,
+                                    const uint16_t *CK_lo, const uint16_t *CK_hi, const uint16_t *BK,
+                                    const uint16_t *CV_lo, const uint16_t *CV_hi, const uint16_t *BV,
+                                    const kvpack_text_basis *tb,
+                                    const uint16_t *K_text, const uint16_t *V_text, int32_t L_text,
+                                    const uint32_t *mask, float softmax_scale,
+                                    uint16_t *out, float *mass,
+                                    void *ws, size_t ws_bytes, void *stream);
+
 /* ---------------------------------------------------- decode step, no allocation
  * kvpack_decode_attn_noalloc -- the same decode step as kvpack_decode_attn,
  * for callers that cannot hand the library any device memory of their own:

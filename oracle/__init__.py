@@ -18,6 +18,9 @@ computes, and the passage of the method it follows:
                by its mask bit, then dense softmax attention over visual
                tokens plus the uncompressed text tail; also the attention
                mass each visual token received.
+  decode_tb -- the same step with the text tokens compressed too, by a basis
+               of their own (pages 2.A): they are decompressed at the full
+               rank and attended together with the uncompressed tail.
   select    -- importance = moving average (alpha) of attention mass; the k
                largest get the full rank next step, ties to the lower index.
 
@@ -143,6 +146,24 @@ def decode(CK, BK, CV, BV, Ktext, Vtext, mask, q, r_lo=16, scale=1.0, want_mass=
                            _ptr(Ktext, _dp), _ptr(Vtext, _dp), _ptr(m, _u32p), _ptr(q, _dp), float(scale),
                            _ptr(out, _dp), _ptr(mass, _dp) if want_mass else None)
     return out, mass
+
+
+def decode_tb(CK, BK, CV, BV, CKt, BKt, CVt, BVt, Ktail, Vtail, mask, q, r_lo=16, scale=1.0, want_mass=True):
+    """One decode step when the text tokens are compressed too, with a basis of their own
+    (technical summaries 2.A on the es / fr / de pages: visual and text tokens are factored
+    separately).  The L_c compressed text tokens are decompressed at the full rank,
+    K' = C_K' B_K' and V' = C_V' B_V' (fp64 products, reshaped to [L_c, 4, 128]), and placed
+    before the uncompressed tail; the step is then decode() over T visual + L_c + L_tail tokens.
+
+    CKt, CVt [U,L_c,64]; BKt, BVt [U,64,512]; Ktail, Vtail [U,L,4,128].  Returns out, mass [U,T].
+    """
+    CKt, BKt, CVt, BVt = (_f64(a) for a in (CKt, BKt, CVt, BVt))
+    U, Lc, _ = CKt.shape
+    Kd = np.matmul(CKt, BKt).reshape(U, Lc, 4, 128)
+    Vd = np.matmul(CVt, BVt).reshape(U, Lc, 4, 128)
+    Kall = np.concatenate([Kd, _f64(Ktail)], axis=1)
+    Vall = np.concatenate([Vd, _f64(Vtail)], axis=1)
+    return decode(CK, BK, CV, BV, Kall, Vall, mask, q, r_lo=r_lo, scale=scale, want_mass=want_mass)
 
 
 # --------------------------------------------------------------- select

@@ -12,6 +12,8 @@ Functions mirror the C entry points:
     compress(dims, n_layers, X, C_lo, C_hi, B, sigma, ws)
     decode_attn(dims, n_layers, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV,
                 K_text, V_text, L_text, mask, scale, out, mass, ws)
+    decode_attn_tb(dims, n_layers, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV,
+                   text_basis, K_text, V_text, L_text, mask, scale, out, mass, ws)
     select(dims, n_layers, mass, score, alpha, k_hi, mask_out)
 
 bf16 arrays are torch.bfloat16 (or int16 views of bf16 bits); masks are
@@ -25,6 +27,8 @@ from ._lib import (  # noqa: F401
     compress_workspace,
     decode_attn,
     decode_attn_noalloc,
+    decode_attn_tb,
+    decode_tb_workspace,
     NOALLOC_SCRATCH_BYTES,
     decode_workspace,
     decompress,

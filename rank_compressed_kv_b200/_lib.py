@@ -83,6 +83,18 @@ _L.kvpack_decode_attn_noalloc.argtypes = [_dims_p, _i32, _vp, _vp, _vp, _vp, _vp
                                           _vp, ctypes.c_float, _vp, _vp, _vp]
 _L.kvpack_decode_attn_noalloc.restype = ctypes.c_int
 _L.kvpack_noalloc_scratch_bytes.restype = _sz
+
+
+class _CTextBasis(ctypes.Structure):
+    _fields_ = [("CK_lo", _vp), ("CK_hi", _vp), ("BK", _vp), ("CV_lo", _vp), ("CV_hi", _vp), ("BV", _vp),
+                ("L_c", _i32)]
+
+
+_L.kvpack_decode_tb_workspace.argtypes = [_dims_p, _i32, _i32]
+_L.kvpack_decode_tb_workspace.restype = _sz
+_L.kvpack_decode_attn_tb.argtypes = [_dims_p, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(_CTextBasis),
+                                     _vp, _vp, _i32, _vp, ctypes.c_float, _vp, _vp, _vp, _sz, _vp]
+_L.kvpack_decode_attn_tb.restype = ctypes.c_int
 _L.kvpack_dense_decode_workspace.argtypes = [_dims_p, _i32, _i32]
 _L.kvpack_dense_decode_workspace.restype = _sz
 _L.kvpack_dense_decode_attn.argtypes = [_dims_p, _i32, _vp, _vp, _vp, _i32, _i32, ctypes.c_float, _vp, _vp, _sz, _vp]
@@ -171,6 +183,22 @@ def decode_attn_noalloc(dims: Dims, n_layers: int, q, CK_lo, CK_hi, BK, CV_lo, C
 
 
 NOALLOC_SCRATCH_BYTES = int(_L.kvpack_noalloc_scratch_bytes())
+
+
+def decode_tb_workspace(dims: Dims, n_layers: int, L_c: int) -> int:
+    return int(_L.kvpack_decode_tb_workspace(ctypes.byref(dims.c()), n_layers, int(L_c)))
+
+
+def decode_attn_tb(dims: Dims, n_layers: int, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, text_basis, K_text, V_text,
+                   L_text: int, mask, scale: float, out, mass, ws, stream=None):
+    """decode_attn with the text tokens compressed by a basis of their own: text_basis =
+    (CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, L_c) in the visual planes' layouts with L_c tokens."""
+    tk_lo, tk_hi, tbk, tv_lo, tv_hi, tbv, L_c = text_basis
+    tb = _CTextBasis(_ptr(tk_lo), _ptr(tk_hi), _ptr(tbk), _ptr(tv_lo), _ptr(tv_hi), _ptr(tbv), int(L_c))
+    _check(_L.kvpack_decode_attn_tb(ctypes.byref(dims.c()), n_layers, _ptr(q), _ptr(CK_lo), _ptr(CK_hi), _ptr(BK),
+                                    _ptr(CV_lo), _ptr(CV_hi), _ptr(BV), ctypes.byref(tb), _ptr(K_text),
+                                    _ptr(V_text), L_text, _ptr(mask), float(scale), _ptr(out), _ptr(mass), _ptr(ws),
+                                    _nbytes(ws), _stream(stream)), "kvpack_decode_attn_tb")
 
 
 def select(dims: Dims, n_layers: int, mass, score, alpha: float, k_hi: int, mask_out, stream=None):

@@ -9,14 +9,12 @@
 //                      generation tensor cores (tcgen05.mma, accumulator in tensor
 //                      memory, operands staged by TMA); only the upper 128-row bands
 //                      right of the diagonal are computed, then mirrored.
-//   2. eig_kernel      top-64 eigenpairs of G by blocked subspace iteration
-//                      with p = 96 columns: Y = G Q (three-product bf16 split
-//                      on the tensor cores, ~fp32 accurate), then Y is
-//                      orthonormalised by one-sided Jacobi in shared memory,
-//                      which also aligns the basis with the Ritz vectors of G
-//                      (the column norms are the Ritz estimates of lambda).
-//                      Stops when the leading 64 estimates move by less than
-//                      5e-4 relative; sigma_i = sqrt(lambda_i), B = Q_r^T.
+//   2. eig_kernel      top-64 eigenpairs of G by blocked subspace (orthogonal)
+//                      iteration with p = 96 columns: Y = G Q (three-product bf16
+//                      split on the tensor cores, ~fp32 accurate), Rayleigh-Ritz
+//                      every second iteration (96 x 96 Jacobi), Cholesky QR of the
+//                      columns scaled by their Ritz values; sigma_i = sqrt(theta_i),
+//                      B = the leading 64 Ritz vectors.
 //   3. project_kernel  C = X Q_r (Q_r carried as a bf16 hi + lo pair), rounded
 //                      to bf16 and written as the C_lo / C_hi planes.
 #pragma once
@@ -30,16 +28,17 @@ constexpr int kN = 512;               // features per unit (4 KV heads x 128)
 constexpr int kP = 96;                // subspace dimension (64 + 32 oversampling)
 constexpr int kR = 64;                // rank kept
 constexpr int kQPitch = 400;          // bytes per row of the bf16 Q layout: hi[96] | lo[96] | pad
-constexpr int kMaxIter = 40;
-constexpr int kMaxSweeps = 12;
+constexpr int kMaxIter = 60;
+constexpr int kMaxSweeps = 16;        // Jacobi sweeps of one 96 x 96 Rayleigh-Ritz problem
 constexpr float kConvTol = 2e-3f;     // estimated remaining relative error of the top-64 sigma
-constexpr float kJacobiTol = 2e-5f;   // off-orthogonality tolerance (fp32 dot products of length 512)
 
 struct Workspace {
     float *G;            // [units][512][512]
     float *Yt;           // [units][96][512]   Y = G Q, column-major
+    float *Zt;           // [units][96][512]   Z = Y V Theta^-1 (Rayleigh-Ritz iterations), column-major
+    float *Qt;           // [units][96][512]   Q in fp32, column-major
     unsigned char *Qg;   // [units][512][kQPitch]  Q as bf16 hi / lo, columns sorted by Ritz value
-    float *info;         // [units][4]: iterations, Jacobi sweeps of the last iteration, last change, error estimate
+    float *info;         // [units][4]: iterations, Jacobi sweeps of the last Rayleigh-Ritz step, last change, error estimate
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -52,16 +51,23 @@ inline size_t ws_info(int units) { return align256((size_t)units * 4 * 4); }
 
 inline size_t workspace_bytes(int units, int T) {
     (void)T;
-    return ws_G(units) + ws_Yt(units) + ws_Qg(units) + ws_info(units);
+    return ws_G(units) + 3 * ws_Yt(units) + ws_Qg(units) + ws_info(units);
 }
 
 inline Workspace carve(void *ws, int units) {
     unsigned char *p = static_cast<unsigned char *>(ws);
     Workspace w;
     w.G = reinterpret_cast<float *>(p);
-    w.Yt = reinterpret_cast<float *>(p + ws_G(units));
-    w.Qg = p + ws_G(units) + ws_Yt(units);
-    w.info = reinterpret_cast<float *>(p + ws_G(units) + ws_Yt(units) + ws_Qg(units));
+    p += ws_G(units);
+    w.Yt = reinterpret_cast<float *>(p);
+    p += ws_Yt(units);
+    w.Zt = reinterpret_cast<float *>(p);
+    p += ws_Yt(units);
+    w.Qt = reinterpret_cast<float *>(p);
+    p += ws_Yt(units);
+    w.Qg = p;
+    p += ws_Qg(units);
+    w.info = reinterpret_cast<float *>(p);
     return w;
 }
 
@@ -74,29 +80,65 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 
 // ================================================================== eigen-solver
+//
+// Orthogonal (blocked subspace) iteration on G with p = 96 columns and a Rayleigh-Ritz step
+// on the first and every second iteration:
+//   Y = G Q                       tensor cores, three-product bf16 split (~fp32 accurate)
+//   Rayleigh-Ritz iterations:     H = Q^T Y (96 x 96) = V Theta V^T by cyclic two-sided Jacobi;
+//                                 Z = Y V Theta^-1, columns sorted by Ritz value
+//   other iterations:             Z = Y D^-1, D = diag(Q^T Y) (the columns' Rayleigh quotients)
+//   Q = Z R^-1 with Z^T Z = R^T R (Cholesky QR)
+// Dividing each column by its Ritz value / Rayleigh quotient leaves Z's columns near unit
+// length and near orthogonal, so a single fp32 Cholesky QR pass is accurate; the triangular R
+// keeps Gram-Schmidt order (largest first), so between Rayleigh-Ritz steps the columns stay
+// close to eigenvectors, as in orthogonal iteration.  The iteration stops when the Ritz
+// estimates of the leading 64 sigma move by less than kConvTol between Rayleigh-Ritz steps
+// (extrapolated with the observed contraction rate); B = the leading 64 Ritz vectors,
+// sigma_i = sqrt(theta_i).
+//
+// One 512-thread block per unit.  The 96 x 96 work (H, Z^T Z, Jacobi, Cholesky, R^-1) lives in
+// shared memory; Y, Z and Q (96 columns of 512 fp32, one column per row of the array) live in
+// the workspace, which stays in L2.
 
 constexpr int kEigThreads = 512;
 constexpr int kEigWarps = kEigThreads / 32;
+constexpr int kStageRows = 32;          // rows of Y per staged chunk of a 96 x 96 product
+constexpr int kStagePitch = kP + 1;     // staged chunks are stored transposed, padded
+constexpr float kJacTol = 1e-6f;        // rotate when |a_pq| > kJacTol sqrt(|a_pp a_qq|) ...
+constexpr float kJacFloor = 1e-7f;      // ... and |a_pq| > kJacFloor max |a_ii| (fp32 rounding level)
+constexpr float kPivTol = 1e-4f;        // Cholesky pivot below this fraction of its diagonal: dependent column
+constexpr float kThetaFloor = 1e-7f;    // Ritz values below this fraction of the largest are taken as zero
+
+struct EigWork {                        // the 96 x 96 phase, laid over the Q buffer
+    float A[kP * kP];                   // H or W = Z^T Z (row-major)
+    float V[kP * kP];                   // Jacobi rotations, then the Cholesky factor R
+    float M[kP * kP];                   // the matrix that mixes the columns of Y or Z
+    float st[2][kStageRows * kStagePitch];
+};
 
 struct EigSmem {
-    alignas(128) unsigned char buf[kN * kQPitch];   // Q (bf16 hi/lo rows) or Y^T (fp32 columns)
-    float lam[kP];          // Ritz estimates of this iteration (unsorted, by column)
-    float lam_sorted[kP];
-    float prev_sorted[kP];
-    int rank[kP];           // sorted position of each column
-    int inv[kP];            // column at each sorted position
+    alignas(128) unsigned char buf[kN * kQPitch];   // Q as bf16 hi / lo rows for the product | EigWork
+    float theta[kP];        // Ritz values, sorted (descending)
+    float prev[kP];         // the previous Rayleigh-Ritz step's sorted values
+    float scale[kP];        // column scale of Z (1 / Rayleigh quotient), 0 for a dead column
+    float diag0[kP];        // diagonal of W before the Cholesky updates
+    int inv[kP];            // column of H at each sorted position
+    int rot_p[kP / 2], rot_q[kP / 2];
+    float rot_c[kP / 2], rot_s[kP / 2];
+    float amax;
     int rotations;
     int done;
-    int sweeps;
     float prev_change;
 };
-static_assert(kN * kQPitch >= kP * kN * 4, "buffer must hold Y^T too");
+static_assert(sizeof(EigWork) <= kN * kQPitch, "the 96 x 96 phase must fit in the Q buffer");
 
-// Deterministic +-1 start vectors (a multiplicative hash of row and column).
+// Start vectors: 96 columns of a 512 x 512 Sylvester-Hadamard matrix with hashed row signs,
+// scaled by 1/sqrt(512) (exactly orthonormal).
 __device__ __forceinline__ float start_entry(int r, int c) {
-    uint32_t h = (uint32_t)(r * 2654435761u) ^ (uint32_t)((c + 1) * 2246822519u);
-    h ^= h >> 15; h *= 2654435761u; h ^= h >> 13;
-    return (h & 1u) ? 0.04419417382415922f : -0.04419417382415922f;   // +-1/sqrt(512)
+    uint32_t h = (uint32_t)(r + 1) * 2654435761u;
+    h ^= h >> 15; h *= 2246822519u; h ^= h >> 13;
+    const int par = (__popc((uint32_t)r & (uint32_t)(c + 1)) + (int)(h & 1u)) & 1;
+    return par ? -0.04419417382415922f : 0.04419417382415922f;
 }
 
 // Y = G Q for one matrix: warp w computes rows [32w, 32w+32) x 96 columns with
@@ -167,59 +209,206 @@ __device__ void eig_gemm(const float *__restrict__ Gu, const unsigned char *qbuf
             }
 }
 
-// One-sided Jacobi on the columns of Y^T (96 columns of 512 fp32 in shared
-// memory), parallel round-robin pair order: 48 disjoint pairs per round, 95
-// rounds per sweep; a warp rotates 3 pairs per round.  Returns the sweeps used,
-// or -1 if kMaxSweeps passed without convergence.
-__device__ int eig_jacobi(float *Y, EigSmem &sm) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int sweep = 1; sweep <= kMaxSweeps; ++sweep) {
-        if (threadIdx.x == 0) sm.rotations = 0;
+// C[i][j] = sum_r At[i][r] Bt[j][r] for i, j < 96, where At and Bt hold 96 columns of 512
+// fp32 (column i contiguous).  Chunks of 32 rows are staged transposed in shared memory;
+// thread t accumulates rows 3 (t / 16) .. +2 and columns 6 (t % 16) .. +5 of C in fp32.
+__device__ void small_gram(const float *__restrict__ At, const float *__restrict__ Bt, float *C, EigWork &wk) {
+    const int tid = threadIdx.x;
+    const int i0 = 3 * (tid >> 4), j0 = 6 * (tid & 15);
+    float acc[3][6];
+    #pragma unroll
+    for (int x = 0; x < 3; ++x)
+        #pragma unroll
+        for (int y = 0; y < 6; ++y) acc[x][y] = 0.f;
+    for (int r0 = 0; r0 < kN; r0 += kStageRows) {
         __syncthreads();
-        int mine = 0;
-        for (int r = 0; r < kP - 1; ++r) {
-            for (int k = warp; k < kP / 2; k += kEigWarps) {
-                int a, b;
-                if (k == 0) { a = r; b = kP - 1; }
-                else { a = (r + k) % (kP - 1); b = (r - k + kP - 1) % (kP - 1); }
-                float *ya = Y + a * kN, *yb = Y + b * kN;
-                float al = 0.f, be = 0.f, ga = 0.f;
-                float va[16], vb[16];
+        for (int idx = tid; idx < kP * kStageRows; idx += kEigThreads) {
+            const int c = idx / kStageRows, r = idx % kStageRows;
+            wk.st[0][r * kStagePitch + c] = __ldcg(At + (size_t)c * kN + r0 + r);
+            wk.st[1][r * kStagePitch + c] = __ldcg(Bt + (size_t)c * kN + r0 + r);
+        }
+        __syncthreads();
+        #pragma unroll 4
+        for (int r = 0; r < kStageRows; ++r) {
+            const float *a = &wk.st[0][r * kStagePitch + i0];
+            const float *b = &wk.st[1][r * kStagePitch + j0];
+            float av[3], bv[6];
+            #pragma unroll
+            for (int x = 0; x < 3; ++x) av[x] = a[x];
+            #pragma unroll
+            for (int y = 0; y < 6; ++y) bv[y] = b[y];
+            #pragma unroll
+            for (int x = 0; x < 3; ++x)
                 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    va[j] = ya[lane + 32 * j];
-                    vb[j] = yb[lane + 32 * j];
-                    al = fmaf(va[j], va[j], al);
-                    be = fmaf(vb[j], vb[j], be);
-                    ga = fmaf(va[j], vb[j], ga);
-                }
+                for (int y = 0; y < 6; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+        }
+    }
+    #pragma unroll
+    for (int x = 0; x < 3; ++x)
+        #pragma unroll
+        for (int y = 0; y < 6; ++y) C[(i0 + x) * kP + j0 + y] = acc[x][y];
+    __syncthreads();
+}
+
+// out[j][r] = sum_i in[i][r] M[i][j] for the 96 columns j (in and out: 96 columns of 512 fp32,
+// column-contiguous; one thread per row r).  Optional outputs: out (fp32), the bf16 hi / lo row
+// layout qg, and the bf16 rows of the basis B (its first 64 columns, B[j][r]).
+__device__ void rowmix(const float *__restrict__ in, const float *M, float *__restrict__ out,
+                       unsigned char *__restrict__ qg, uint16_t *__restrict__ Bout) {
+    const int r = threadIdx.x;
+    #pragma unroll 1
+    for (int h = 0; h < kP; h += 48) {
+        float acc[48];
+        #pragma unroll
+        for (int j = 0; j < 48; ++j) acc[j] = 0.f;
+        #pragma unroll 4
+        for (int i = 0; i < kP; ++i) {
+            const float x = __ldcg(in + (size_t)i * kN + r);
+            const float4 *m = reinterpret_cast<const float4 *>(M + i * kP + h);
+            #pragma unroll
+            for (int q = 0; q < 12; ++q) {
+                const float4 v = m[q];
+                acc[4 * q + 0] = fmaf(x, v.x, acc[4 * q + 0]);
+                acc[4 * q + 1] = fmaf(x, v.y, acc[4 * q + 1]);
+                acc[4 * q + 2] = fmaf(x, v.z, acc[4 * q + 2]);
+                acc[4 * q + 3] = fmaf(x, v.w, acc[4 * q + 3]);
+            }
+        }
+        if (out != nullptr) {
+            #pragma unroll
+            for (int j = 0; j < 48; ++j) out[(size_t)(h + j) * kN + r] = acc[j];
+        }
+        if (qg != nullptr) {
+            unsigned char *row = qg + (size_t)r * kQPitch;
+            #pragma unroll
+            for (int c8 = 0; c8 < 48; c8 += 8) {
+                uint32_t hw[4], lw[4];
                 #pragma unroll
-                for (int d = 16; d > 0; d >>= 1) {
-                    al += __shfl_xor_sync(0xffffffffu, al, d);
-                    be += __shfl_xor_sync(0xffffffffu, be, d);
-                    ga += __shfl_xor_sync(0xffffffffu, ga, d);
-                }
-                if (al > 0.f && be > 0.f && fabsf(ga) > kJacobiTol * sqrtf(al * be)) {
-                    ++mine;
-                    const float zeta = (be - al) / (2.f * ga);
+                for (int e = 0; e < 4; ++e) split2(acc[c8 + 2 * e], acc[c8 + 2 * e + 1], hw[e], lw[e]);
+                *reinterpret_cast<uint4 *>(row + (h + c8) * 2) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(row + kP * 2 + (h + c8) * 2) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+        }
+        if (Bout != nullptr) {
+            #pragma unroll
+            for (int j = 0; j < 48; ++j)
+                if (h + j < kR) Bout[(size_t)(h + j) * kN + r] = float_to_bf16_bits(acc[j]);
+        }
+    }
+}
+
+// Cyclic two-sided Jacobi on the symmetric 96 x 96 matrix A (row-major, both triangles),
+// V = the product of the rotations (A -> V^T A V).  Parallel round-robin order: 48 disjoint
+// pairs per round, 95 rounds per sweep; each 2 x 2 block of A is rotated in place by one
+// thread.  Returns the sweeps used, or -1 after kMaxSweeps without convergence.
+__device__ int jacobi96(float *A, float *V, EigSmem &sm) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    for (int e = tid; e < kP * kP; e += kEigThreads) V[e] = (e / kP == e % kP) ? 1.f : 0.f;
+    for (int sweep = 1; sweep <= kMaxSweeps; ++sweep) {
+        __syncthreads();
+        if (tid < 32) {
+            float m = 0.f;
+            for (int i = lane; i < kP; i += 32) m = fmaxf(m, fabsf(A[i * kP + i]));
+            #pragma unroll
+            for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
+            if (lane == 0) { sm.amax = m; sm.rotations = 0; }
+        }
+        __syncthreads();
+        const float floor_a = kJacFloor * sm.amax;
+        for (int rd = 0; rd < kP - 1; ++rd) {
+            if (tid < kP / 2) {
+                const int k = tid;
+                int p, q;
+                if (k == 0) { p = rd; q = kP - 1; }
+                else { p = (rd + k) % (kP - 1); q = (rd - k + kP - 1) % (kP - 1); }
+                const float app = A[p * kP + p], aqq = A[q * kP + q], apq = A[p * kP + q];
+                float c = 1.f, s = 0.f;
+                if (fabsf(apq) > kJacTol * sqrtf(fabsf(app * aqq)) && fabsf(apq) > floor_a) {
+                    const float zeta = (aqq - app) / (2.f * apq);
                     const float t = copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
-                    const float c = rsqrtf(1.f + t * t), s = c * t;
-                    #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        ya[lane + 32 * j] = c * va[j] - s * vb[j];
-                        yb[lane + 32 * j] = s * va[j] + c * vb[j];
-                    }
+                    c = 1.f / sqrtf(1.f + t * t);
+                    s = c * t;
+                    atomicAdd(&sm.rotations, 1);
                 }
+                sm.rot_p[k] = p; sm.rot_q[k] = q; sm.rot_c[k] = c; sm.rot_s[k] = s;
+            }
+            __syncthreads();
+            for (int blk = tid; blk < (kP / 2) * (kP / 2); blk += kEigThreads) {
+                const int a = blk / (kP / 2), b = blk % (kP / 2);
+                const float sa = sm.rot_s[a], sb = sm.rot_s[b];
+                if (sa == 0.f && sb == 0.f) continue;
+                const float ca = sm.rot_c[a], cb = sm.rot_c[b];
+                const int pa = sm.rot_p[a], qa = sm.rot_q[a], pb = sm.rot_p[b], qb = sm.rot_q[b];
+                const float x11 = A[pa * kP + pb], x12 = A[pa * kP + qb];
+                const float x21 = A[qa * kP + pb], x22 = A[qa * kP + qb];
+                const float y11 = ca * x11 - sa * x21, y12 = ca * x12 - sa * x22;   // rows
+                const float y21 = sa * x11 + ca * x21, y22 = sa * x12 + ca * x22;
+                float z11 = cb * y11 - sb * y12, z12 = sb * y11 + cb * y12;          // columns
+                float z21 = cb * y21 - sb * y22, z22 = sb * y21 + cb * y22;
+                if (a == b) z12 = z21 = 0.f;                                        // the annihilated pair
+                A[pa * kP + pb] = z11; A[pa * kP + qb] = z12;
+                A[qa * kP + pb] = z21; A[qa * kP + qb] = z22;
+            }
+            for (int e = tid; e < kP * (kP / 2); e += kEigThreads) {
+                const int i = e / (kP / 2), k = e % (kP / 2);
+                const float s = sm.rot_s[k];
+                if (s == 0.f) continue;
+                const float c = sm.rot_c[k];
+                const int p = sm.rot_p[k], q = sm.rot_q[k];
+                const float vp = V[i * kP + p], vq = V[i * kP + q];
+                V[i * kP + p] = c * vp - s * vq;
+                V[i * kP + q] = s * vp + c * vq;
             }
             __syncthreads();
         }
-        if (lane == 0 && mine) atomicAdd(&sm.rotations, mine);
-        __syncthreads();
-        const int rot = sm.rotations;
-        __syncthreads();
-        if (rot == 0) return sweep;
+        if (sm.rotations == 0) return sweep;
     }
     return -1;
+}
+
+// W = R^T R (R upper triangular, written to R; the lower triangle is zeroed).  A holds W on
+// entry and is overwritten by the trailing updates.  A pivot at or below kPivTol of its
+// column's original diagonal marks a dependent (or dead) column: its row of R is zero.
+__device__ void cholesky96(float *A, float *R, EigSmem &sm) {
+    const int tid = threadIdx.x;
+    if (tid < kP) sm.diag0[tid] = A[tid * kP + tid];
+    for (int e = tid; e < kP * kP; e += kEigThreads) R[e] = 0.f;
+    __syncthreads();
+    for (int k = 0; k < kP; ++k) {
+        const float piv = A[k * kP + k];
+        const bool ok = piv > kPivTol * sm.diag0[k] && piv > 0.f;
+        const float rk = ok ? sqrtf(piv) : 0.f;
+        const float inv_piv = ok ? 1.f / piv : 0.f;
+        for (int j = k + tid; j < kP; j += kEigThreads) R[k * kP + j] = ok ? A[k * kP + j] / rk : 0.f;
+        const int n = kP - 1 - k;
+        for (int e = tid; e < n * n; e += kEigThreads) {
+            const int i = k + 1 + e / n, j = k + 1 + e % n;
+            if (j < i) continue;
+            A[i * kP + j] -= A[k * kP + i] * A[k * kP + j] * inv_piv;
+        }
+        __syncthreads();
+    }
+}
+
+// X = R^-1 for the upper-triangular R of cholesky96 (a zero row of R gives a zero row and
+// column of X), computed bottom-up: X_ii = 1 / R_ii, X_ij = -(sum_{i<k<=j} R_ik X_kj) / R_ii.
+// Four threads share each column's sum.
+__device__ void tri_inverse96(const float *R, float *X) {
+    const int tid = threadIdx.x;
+    for (int e = tid; e < kP * kP; e += kEigThreads) X[e] = 0.f;
+    __syncthreads();
+    const int j = tid >> 2, part = tid & 3;     // 384 threads: 96 columns x 4
+    for (int i = kP - 1; i >= 0; --i) {
+        if (j < kP) {                            // whole warps (threads 0 .. 383)
+            float s = 0.f;
+            for (int k = i + 1 + part; k <= j; k += 4) s = fmaf(R[i * kP + k], X[k * kP + j], s);
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            s += __shfl_xor_sync(0xffffffffu, s, 2);
+            const float rii = R[i * kP + i];
+            if (part == 0 && j >= i) X[i * kP + j] = rii > 0.f ? (j == i ? 1.f / rii : -s / rii) : 0.f;
+        }
+        __syncthreads();
+    }
 }
 
 struct EigParams {
@@ -233,115 +422,132 @@ struct EigParams {
 __global__ void __launch_bounds__(kEigThreads, 1) eig_kernel(EigParams p) {
     extern __shared__ __align__(128) unsigned char eig_smem_raw[];
     EigSmem &sm = *reinterpret_cast<EigSmem *>(eig_smem_raw);
+    EigWork &wk = *reinterpret_cast<EigWork *>(sm.buf);
     const int unit = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const float *Gu = p.ws.G + (size_t)unit * kN * kN;
-    float *Ytu = p.ws.Yt + (size_t)unit * kP * kN;
+    float *Yt = p.ws.Yt + (size_t)unit * kP * kN;
+    float *Zt = p.ws.Zt + (size_t)unit * kP * kN;
+    float *Qt = p.ws.Qt + (size_t)unit * kP * kN;
     unsigned char *Qgu = p.ws.Qg + (size_t)unit * kN * kQPitch;
-    float *Ys = reinterpret_cast<float *>(sm.buf);
 
-    // Q0 in the bf16 layout: row r = [hi 96 | lo 96]
-    for (int i = tid; i < kN * kP; i += kEigThreads) {
-        const int r = i / kP, c = i % kP;
-        const float v = start_entry(r, c);
-        const uint16_t h = float_to_bf16_bits(v);
+    // Q0: fp32 columns in Qt and bf16 hi / lo rows in shared memory (thread = row)
+    {
+        const int r = tid;
         uint16_t *row = reinterpret_cast<uint16_t *>(sm.buf + r * kQPitch);
-        row[c] = h;
-        row[kP + c] = float_to_bf16_bits(v - bf16_bits_to_float(h));
+        for (int c = 0; c < kP; ++c) {
+            const float v = start_entry(r, c);
+            Qt[(size_t)c * kN + r] = v;
+            const uint16_t h = float_to_bf16_bits(v);
+            row[c] = h;
+            row[kP + c] = float_to_bf16_bits(v - bf16_bits_to_float(h));
+        }
     }
-    if (tid < kP) sm.prev_sorted[tid] = 0.f;
     if (tid == 0) { sm.done = 0; sm.prev_change = 1.f; }
     __syncthreads();
 
-    bool converged = false, jacobi_ok = true;
-    for (int it = 0; it < p.max_iter; ++it) {
-        // Y = G Q  (Q in the smem buffer), Y^T to global
-        eig_gemm(Gu, sm.buf, Ytu);
-        __threadfence_block();
+    bool converged = false, jacobi_ok = true, have_prev = false;
+    int sweeps = 0;
+    for (int it = 1; it <= p.max_iter; ++it) {
+        eig_gemm(Gu, sm.buf, Yt);                       // Y = G Q
         __syncthreads();
-        // Y^T into shared memory (column-major fp32)
-        for (int i = tid; i < kP * kN / 4; i += kEigThreads)
-            reinterpret_cast<float4 *>(Ys)[i] = __ldcg(reinterpret_cast<const float4 *>(Ytu) + i);
-        __syncthreads();
-        const int sw = eig_jacobi(Ys, sm);
-        jacobi_ok = sw >= 0;
-        if (tid == 0) sm.sweeps = sw;
-        // column norms = Ritz estimates of lambda
-        for (int c = warp; c < kP; c += kEigWarps) {
-            float s = 0.f;
-            for (int j = lane; j < kN; j += 32) s = fmaf(Ys[c * kN + j], Ys[c * kN + j], s);
-            #pragma unroll
-            for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
-            if (lane == 0) sm.lam[c] = sqrtf(s);
-        }
-        __syncthreads();
-        if (tid < kP) {
-            const float v = sm.lam[tid];
-            int rk = 0;
-            for (int c = 0; c < kP; ++c) {
-                const float u = sm.lam[c];
-                rk += (u > v || (u == v && c < tid)) ? 1 : 0;
-            }
-            sm.rank[tid] = rk;
-            sm.inv[rk] = tid;
-            sm.lam_sorted[rk] = v;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            // components below 1e-6 of the largest are numerically zero (rank-deficient G) and
-            // are left out of the test
-            // largest relative change of sigma = sqrt(lambda) among the leading 64; with the
-            // ratio of successive changes as the contraction rate rho, the remaining error is
-            // about change * rho / (1 - rho)
-            float worst = 0.f;
-            const float floor_l = 1e-6f * sm.lam_sorted[0];
-            for (int i = 0; i < kR; ++i) {
-                if (sm.lam_sorted[i] <= floor_l) continue;
-                const float a = sqrtf(sm.lam_sorted[i]), b = sqrtf(sm.prev_sorted[i]);
-                worst = fmaxf(worst, fabsf(a - b) / a);
-            }
-            const float rho = fminf(worst / fmaxf(sm.prev_change, 1e-30f), 0.95f);
-            const float est = worst * rho / (1.f - rho);
-            sm.done = (it >= 2 && est < kConvTol && worst < kConvTol) ? 1 : 0;
-            sm.prev_change = worst;
-            float *inf = p.ws.info + (size_t)unit * 4;
-            inf[0] = (float)(it + 1); inf[1] = (float)sm.sweeps; inf[2] = worst; inf[3] = est;
-        }
-        __syncthreads();
-        if (tid < kP) sm.prev_sorted[tid] = sm.lam_sorted[tid];
-        converged = sm.done != 0;
-        const bool last = converged || it == p.max_iter - 1;
-
-        // Q for the next iteration: normalised columns in sorted order, bf16 hi / lo rows
-        {
-            const int r = tid;   // one row per thread
-            unsigned char *dst = Qgu + (size_t)r * kQPitch;
-            for (int c8 = 0; c8 < kP; c8 += 8) {
-                uint32_t hw[4], lw[4];
-                #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int c0 = sm.inv[c8 + 2 * e], c1 = sm.inv[c8 + 2 * e + 1];
-                    const float x0 = sm.lam[c0] > 0.f ? Ys[c0 * kN + r] / sm.lam[c0] : 0.f;
-                    const float x1 = sm.lam[c1] > 0.f ? Ys[c1 * kN + r] / sm.lam[c1] : 0.f;
-                    split2(x0, x1, hw[e], lw[e]);
+        const bool rr = it == 1 || (it & 1) == 0 || it == p.max_iter;
+        const float *zsrc;
+        if (rr) {
+            small_gram(Qt, Yt, wk.A, wk);               // H = Q^T Y
+            for (int e = tid; e < kP * kP; e += kEigThreads) {
+                const int i = e / kP, j = e % kP;
+                if (i < j) {
+                    const float v = 0.5f * (wk.A[e] + wk.A[j * kP + i]);
+                    wk.A[e] = v;
+                    wk.A[j * kP + i] = v;
                 }
-                *reinterpret_cast<uint4 *>(dst + c8 * 2) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4 *>(dst + kP * 2 + c8 * 2) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
             }
-        }
-        if (last) {
-            // basis B = Q_r^T (bf16) and singular values sigma_i = sqrt(lambda_i)
-            uint16_t *Bu = p.B + (size_t)unit * kR * kN;
-            for (int i = tid; i < kR * kN; i += kEigThreads) {
-                const int row = i / kN, col = i % kN;
-                const int c = sm.inv[row];
-                Bu[i] = float_to_bf16_bits(sm.lam[c] > 0.f ? Ys[c * kN + col] / sm.lam[c] : 0.f);
+            __syncthreads();
+            sweeps = jacobi96(wk.A, wk.V, sm);
+            if (sweeps < 0) jacobi_ok = false;
+            __syncthreads();
+            if (tid < kP) {                              // sort the Ritz values, descending
+                const float v = wk.A[tid * kP + tid];
+                int rk = 0;
+                for (int c = 0; c < kP; ++c) {
+                    const float u = wk.A[c * kP + c];
+                    rk += (u > v || (u == v && c < tid)) ? 1 : 0;
+                }
+                sm.inv[rk] = tid;
+                sm.theta[rk] = v;
             }
-            if (p.sigma != nullptr && tid < kR) p.sigma[(size_t)unit * kR + tid] = sqrtf(sm.lam_sorted[tid]);
-            break;
+            __syncthreads();
+            if (tid == 0) {
+                // largest relative change of sigma = sqrt(theta) among the leading 64 since the
+                // previous Rayleigh-Ritz step (components below kThetaFloor of the largest are
+                // numerically zero and left out); with the ratio of successive changes as the
+                // contraction rate rho, the remaining error is about change * rho / (1 - rho)
+                float worst = 0.f;
+                const float floor_t = kThetaFloor * sm.theta[0];
+                for (int i = 0; i < kR; ++i) {
+                    if (sm.theta[i] <= floor_t) continue;
+                    const float a = sqrtf(sm.theta[i]), b = sqrtf(fmaxf(sm.prev[i], 0.f));
+                    worst = fmaxf(worst, fabsf(a - b) / a);
+                }
+                const float rho = fminf(worst / fmaxf(sm.prev_change, 1e-30f), 0.95f);
+                const float est = worst * rho / (1.f - rho);
+                sm.done = (have_prev && est < kConvTol && worst < kConvTol) ? 1 : 0;
+                sm.prev_change = worst;
+                float *inf = p.ws.info + (size_t)unit * 4;
+                inf[0] = (float)it; inf[1] = (float)sweeps; inf[2] = worst; inf[3] = est;
+            }
+            __syncthreads();
+            if (tid < kP) sm.prev[tid] = sm.theta[tid];
+            have_prev = true;
+            converged = sm.done != 0;
+            const bool last = converged || it == p.max_iter;
+            const float floor_t = kThetaFloor * fmaxf(sm.theta[0], 0.f);
+            // M = V (sorted columns), scaled by 1 / theta for Z; plain for the final Ritz vectors
+            for (int e = tid; e < kP * kP; e += kEigThreads) {
+                const int i = e / kP, j = e % kP;
+                const float th = sm.theta[j];
+                const float v = wk.V[i * kP + sm.inv[j]];
+                wk.M[e] = last ? v : (th > floor_t ? v / th : 0.f);
+            }
+            __syncthreads();
+            if (last) {
+                // Ritz vectors U = Q V: basis B = U_r^T (bf16) and Q_r for the projection
+                rowmix(Qt, wk.M, nullptr, Qgu, p.B + (size_t)unit * kR * kN);
+                if (p.sigma != nullptr && tid < kR) p.sigma[(size_t)unit * kR + tid] = sqrtf(fmaxf(sm.theta[tid], 0.f));
+                break;
+            }
+            rowmix(Yt, wk.M, Zt, nullptr, nullptr);     // Z = Y V Theta^-1
+            if (tid < kP) sm.scale[tid] = 1.f;
+            zsrc = Zt;
+        } else {
+            // Rayleigh quotients d_j = q_j . y_j; Z = Y D^-1
+            for (int c = warp; c < kP; c += kEigWarps) {
+                float s = 0.f;
+                for (int j = lane; j < kN; j += 32) s = fmaf(__ldcg(Qt + (size_t)c * kN + j), __ldcg(Yt + (size_t)c * kN + j), s);
+                #pragma unroll
+                for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
+                if (lane == 0) sm.scale[c] = s;
+            }
+            __syncthreads();
+            if (tid < kP) {
+                const float d = sm.scale[tid];
+                sm.scale[tid] = d > kThetaFloor * sm.prev[0] ? 1.f / d : 0.f;
+            }
+            zsrc = Yt;
         }
         __syncthreads();
-        // reload Q into shared memory for the next product
+        // Cholesky QR of Z = zsrc * diag(scale): W = S^T (zsrc^T zsrc) S = R^T R, Q = zsrc S R^-1
+        small_gram(zsrc, zsrc, wk.A, wk);
+        for (int e = tid; e < kP * kP; e += kEigThreads) wk.A[e] *= sm.scale[e / kP] * sm.scale[e % kP];
+        __syncthreads();
+        cholesky96(wk.A, wk.V, sm);
+        tri_inverse96(wk.V, wk.M);
+        for (int e = tid; e < kP * kP; e += kEigThreads) wk.M[e] *= sm.scale[e / kP];
+        __syncthreads();
+        rowmix(zsrc, wk.M, Qt, Qgu, nullptr);
+        __syncthreads();
+        // Q (bf16 hi / lo rows) into shared memory for the next product
         for (int i = tid; i < kN * kQPitch / 16; i += kEigThreads)
             reinterpret_cast<uint4 *>(sm.buf)[i] = __ldcg(reinterpret_cast<const uint4 *>(Qgu) + i);
         __syncthreads();

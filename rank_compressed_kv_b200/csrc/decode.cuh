@@ -48,9 +48,11 @@ constexpr int kTile = 16;
 struct Params {
     CUtensorMap tm_k, tm_v;    // text: 4D {128, 4, L, units}, box {64, 1, 16, 1}, 128-byte swizzle
     CUtensorMap tm_bk;         // B_K: 3D {512, 64, units}, box {64, 64, 1}, 128-byte swizzle
+    CUtensorMap tm_bk2;        // the text tokens' own B_K (same layout), when they are compressed too
     const uint16_t *q;
     float *part;               // [units][Sc][Hg][kTxtPart]
     unsigned char *qt;         // [units][qblock_bytes(Hg)]: q~ written here
+    unsigned char *qt2;        // the same for the text tokens' basis, or null
     unsigned int *counter;     // work counter, zero at launch
     int n_units, L, Hg, per_kv, n_q, groups, Sc, ct, n_qitems, n_items;
     float scale2;
@@ -69,7 +71,8 @@ constexpr size_t smem_bytes() { return sizeof(Smem) + 1024; }
 // a global counter.  Items 0 .. n_qitems-1 project the query to rank space for
 // (unit, KV head j): two stages of B_K (64 rank rows x 64 columns each), q~^T =
 // B_K[:, 128 j ..] q^T on mma.sync (ranks on M, the KV head's query heads on N),
-// written as the bf16 hi + lo pair of the unit's query block.  The others are
+// written as the bf16 hi + lo pair of the unit's query block (items 4 units ..
+// 8 units - 1, when present, do the same with the text tokens' basis).  The others are
 // text items -- (unit, KV head j, chunk of ct text tokens): per 16-token tile,
 // S = K q^T with tokens on M and the query heads on N, an online softmax down
 // the columns, and w^T += V^T P (the transposed P from movmatrix); at the end of
@@ -96,7 +99,7 @@ __global__ void __launch_bounds__(kThreads, 1) text_kernel(const __grid_constant
         return __shfl_sync(0xffffffffu, v, 0);
     };
     // (unit, KV head) of an item
-    auto unit_of = [&](int it) { return it < p.n_qitems ? it >> 2 : (it - p.n_qitems) / (4 * p.Sc); };
+    auto unit_of = [&](int it) { return it < p.n_qitems ? (it % (4 * p.n_units)) >> 2 : (it - p.n_qitems) / (4 * p.Sc); };
     auto kvh_of = [&](int it) { return it < p.n_qitems ? it & 3 : ((it - p.n_qitems) / p.Sc) & 3; };
     auto n_tok = [&](int it) { const int c = (it - p.n_qitems) % p.Sc; return min(p.ct, p.L - c * p.ct); };
     auto n_tiles = [&](int it) { return it < p.n_qitems ? 2 : (n_tok(it) + kTile - 1) / kTile; };
@@ -123,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1) text_kernel(const __grid_constant
             fence_proxy_async();
             mbar_arrive_tx(bar, kSlotBytes);
             if (i_item < p.n_qitems) {
-                tma_3d(dst, &p.tm_bk, 128 * j + 64 * i_tile, 0, unit, bar);
+                tma_3d(dst, i_item >= 4 * p.n_units ? &p.tm_bk2 : &p.tm_bk, 128 * j + 64 * i_tile, 0, unit, bar);
             } else {
                 const int tok = ((i_item - p.n_qitems) % p.Sc) * p.ct + i_tile * kTile;
                 tma_4d(dst, &p.tm_k, 0, j, tok, unit, bar);
@@ -208,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1) text_kernel(const __grid_constant
             if (c_tile == c_ntiles) {
                 // wt[mt][e]: rank 16 mt + g (+8 for e >= 2), head 2 tig + (e & 1) of KV head j
                 const int unit = unit_of(c_item), j = kvh_of(c_item);
-                uint16_t *qt = reinterpret_cast<uint16_t *>(p.qt + (size_t)unit * qblock_bytes(p.Hg));
+                unsigned char *qb = c_item >= 4 * p.n_units ? p.qt2 : p.qt;
+                uint16_t *qt = reinterpret_cast<uint16_t *>(qb + (size_t)unit * qblock_bytes(p.Hg));
                 #pragma unroll
                 for (int mt = 0; mt < 4; ++mt)
                     #pragma unroll

@@ -62,6 +62,10 @@ struct DecodePlan {
     long long ntiles;
     int cta_s, cta_v, nslot_s, nslot_v;
     size_t off_qt, off_tp, off_sp, off_ustat, off_vp, off_counter, total;
+    // the text tokens' own rank-space passes (text compressed too); absent when L_c = 0
+    int L_c, tpu2, nwords2, cta2, nslot2;
+    long long ntiles2;
+    size_t off_qt2, off_sp2, off_vp2, off_mask2;
 };
 
 inline int round_heads(int Hg) { return Hg <= 4 ? 4 : Hg <= 8 ? 8 : Hg <= 16 ? 16 : 32; }
@@ -69,7 +73,7 @@ inline int round_heads(int Hg) { return Hg <= 4 ? 4 : Hg <= 8 ? 8 : Hg <= 16 ? 1
 // Most partial slots any unit gets when NT tiles are split over C CTAs (tpu tiles per unit).
 inline int max_slots(long long NT, long long C, int tpu) { return (int)(((long long)tpu * C + NT - 1) / NT) + 1; }
 
-DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
+DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers, int L_c = 0) {
     DecodePlan pl{};
     pl.Hg = hg(d);
     pl.NH = round_heads(pl.Hg);
@@ -97,6 +101,22 @@ DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers) {
     off = align256(off + (size_t)pl.units * pl.nslot_v * pl.Hg * 64 * sizeof(float));
     pl.off_counter = off;   // work counter of the text kernel
     off = align256(off + 4 * sizeof(unsigned int));
+    pl.L_c = L_c;
+    if (L_c > 0) {
+        pl.tpu2 = (L_c + rs::kTile - 1) / rs::kTile;
+        pl.nwords2 = (L_c + 31) / 32;
+        pl.ntiles2 = (long long)pl.units * pl.tpu2;
+        pl.cta2 = (int)(pl.ntiles2 < (long long)kPlanSMs * blocks ? pl.ntiles2 : (long long)kPlanSMs * blocks);
+        pl.nslot2 = max_slots(pl.ntiles2, pl.cta2, pl.tpu2);
+        pl.off_qt2 = off;
+        off = align256(off + (size_t)pl.units * kvpack::decode::qblock_bytes(pl.Hg));
+        pl.off_sp2 = off;
+        off = align256(off + (size_t)pl.units * pl.nslot2 * pl.Hg * 2 * sizeof(float));
+        pl.off_vp2 = off;
+        off = align256(off + (size_t)pl.units * pl.nslot2 * pl.Hg * 64 * sizeof(float));
+        pl.off_mask2 = off;     // every text token at the full rank
+        off = align256(off + (size_t)pl.units * pl.nwords2 * sizeof(uint32_t));
+    }
     pl.total = off;
     return pl;
 }
@@ -150,18 +170,23 @@ cudaError_t launch_rs(int NH, const rs::Params &rp, int grid, cudaStream_t st) {
     }
 }
 
-// finish_kernel is instantiated for 1..8 query heads per KV head
-cudaError_t launch_finish(int per_kv, const rs::FinishParams &fp, int units, cudaStream_t st) {
-    const int grid = units * 4;
+// finish_kernel is instantiated for 1..8 query heads per KV head, and for a whole unit per
+// block (many units) or one KV head per block (few units)
+template <int PK>
+cudaError_t launch_finish_pk(const rs::FinishParams &fp, int units, int sms, cudaStream_t st) {
+    if (units >= 2 * sms) return launch_pdl(rs::finish_kernel<PK, 4>, units, 512, 0, st, fp);
+    return launch_pdl(rs::finish_kernel<PK, 1>, units * 4, 128, 0, st, fp);
+}
+cudaError_t launch_finish(int per_kv, const rs::FinishParams &fp, int units, int sms, cudaStream_t st) {
     switch (per_kv) {
-        case 1: return launch_pdl(rs::finish_kernel<1>, grid, 128, 0, st, fp);
-        case 2: return launch_pdl(rs::finish_kernel<2>, grid, 128, 0, st, fp);
-        case 3: return launch_pdl(rs::finish_kernel<3>, grid, 128, 0, st, fp);
-        case 4: return launch_pdl(rs::finish_kernel<4>, grid, 128, 0, st, fp);
-        case 5: return launch_pdl(rs::finish_kernel<5>, grid, 128, 0, st, fp);
-        case 6: return launch_pdl(rs::finish_kernel<6>, grid, 128, 0, st, fp);
-        case 7: return launch_pdl(rs::finish_kernel<7>, grid, 128, 0, st, fp);
-        default: return launch_pdl(rs::finish_kernel<8>, grid, 128, 0, st, fp);
+        case 1: return launch_finish_pk<1>(fp, units, sms, st);
+        case 2: return launch_finish_pk<2>(fp, units, sms, st);
+        case 3: return launch_finish_pk<3>(fp, units, sms, st);
+        case 4: return launch_finish_pk<4>(fp, units, sms, st);
+        case 5: return launch_finish_pk<5>(fp, units, sms, st);
+        case 6: return launch_finish_pk<6>(fp, units, sms, st);
+        case 7: return launch_finish_pk<7>(fp, units, sms, st);
+        default: return launch_finish_pk<8>(fp, units, sms, st);
     }
 }
 
@@ -215,9 +240,7 @@ kvpack_status device_info(DeviceInfo **out) {
                 cudaSuccess ||
             !rs_attrs() ||
             cudaFuncSetAttribute(kvpack::baseline::decompress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(kvpack::baseline::DecSmem)) != cudaSuccess ||
-            cudaFuncSetAttribute(kvpack::select::select_kernel<64, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kvpack::select::select_smem_bytes<64, 32>()) != cudaSuccess)
+                                 (int)sizeof(kvpack::baseline::DecSmem)) != cudaSuccess)
             return KVPACK_ERR_CUDA;
         kvpack_status cs = kvpack::compress::prepare_device();
         if (cs != KVPACK_OK) return cs;
@@ -254,29 +277,17 @@ bool encode_bf16(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const vo
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KPT, int NW>
-cudaError_t launch_select(const kvpack::select::Params &p, cudaStream_t st) {
-    if (NW == 1) {
-        const int grid = (p.n_units + 7) / 8;
-        kvpack::select::select_kernel<KPT, 1><<<grid, 256, 0, st>>>(p);
-    } else {
-        constexpr size_t smem = kvpack::select::select_smem_bytes<KPT, 32>();   // set up in device_info
-        kvpack::select::select_kernel<KPT, 32><<<p.n_units, 1024, smem, st>>>(p);
-    }
+template <int KPT>
+cudaError_t launch_select_warp(const kvpack::select::Params &p, cudaStream_t st) {
+    kvpack::select::select_warp_kernel<KPT><<<(p.n_units + 7) / 8, 256, 0, st>>>(p);
     return cudaGetLastError();
 }
 
-template <int NW>
-cudaError_t select_dispatch(int kpt, const kvpack::select::Params &p, cudaStream_t st) {
-    switch (kpt) {
-        case 1: return launch_select<1, NW>(p, st);
-        case 2: return launch_select<2, NW>(p, st);
-        case 4: return launch_select<4, NW>(p, st);
-        case 8: return launch_select<8, NW>(p, st);
-        case 16: return launch_select<16, NW>(p, st);
-        case 32: return launch_select<32, NW>(p, st);
-        default: return launch_select<64, NW>(p, st);
-    }
+template <int KPT>
+cudaError_t launch_select_cluster(const kvpack::select::Params &p, cudaStream_t st) {
+    namespace sl = kvpack::select;
+    sl::select_cluster_kernel<KPT><<<p.n_units * sl::kClusterCtas, sl::kClusterThreads, 0, st>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -326,14 +337,29 @@ size_t kvpack_decode_workspace(const kvpack_dims *d, int32_t n_layers) {
     return plan_decode(d, n_layers).total;
 }
 
-kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const uint16_t *q,
-                                 const uint16_t *CK_lo, const uint16_t *CK_hi, const uint16_t *BK,
-                                 const uint16_t *CV_lo, const uint16_t *CV_hi, const uint16_t *BV,
-                                 const uint16_t *K_text, const uint16_t *V_text, int32_t L_text,
-                                 const uint32_t *mask, float softmax_scale, uint16_t *out, float *mass,
-                                 void *ws, size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// The decode step; tb (the text tokens compressed with a basis of their own) may be null.
+kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t *q, const uint16_t *CK_lo,
+                          const uint16_t *CK_hi, const uint16_t *BK, const uint16_t *CV_lo, const uint16_t *CV_hi,
+                          const uint16_t *BV, const kvpack_text_basis *tb, const uint16_t *K_text,
+                          const uint16_t *V_text, int32_t L_text, const uint32_t *mask, float softmax_scale,
+                          uint16_t *out, float *mass, void *ws, size_t ws_bytes, void *stream) {
     kvpack_status s = check_dims(d, n_layers);
     if (s != KVPACK_OK) return s;
+    const int L_c = tb != nullptr ? tb->L_c : 0;
+    if (tb != nullptr) {
+        if (L_c < 0 || L_c > kMaxT) return KVPACK_ERR_INVALID_ARG;
+        if (L_c > 0) {
+            const void *tp[] = {tb->CK_lo, tb->CK_hi, tb->BK, tb->CV_lo, tb->CV_hi, tb->BV};
+            for (const void *ptr : tp) {
+                if (ptr == nullptr) return KVPACK_ERR_INVALID_ARG;
+                if (!aligned16(ptr)) return KVPACK_ERR_ALIGNMENT;
+            }
+        }
+    }
     if (L_text < 0 || L_text > d->L_text_cap) return KVPACK_ERR_INVALID_ARG;
     if (!q || !CK_lo || !CK_hi || !BK || !CV_lo || !CV_hi || !BV || !mask || !out) return KVPACK_ERR_INVALID_ARG;
     if (L_text > 0 && (!K_text || !V_text)) return KVPACK_ERR_INVALID_ARG;
@@ -342,8 +368,9 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
                           L_text > 0 ? K_text : nullptr, L_text > 0 ? V_text : nullptr};
     for (const void *ptr : ptrs)
         if (ptr && !aligned16(ptr)) return KVPACK_ERR_ALIGNMENT;
-    const DecodePlan pl = plan_decode(d, n_layers);
+    const DecodePlan pl = plan_decode(d, n_layers, L_c);
     if ((long long)pl.units * d->T_vis * 3 >= (1LL << 31)) return KVPACK_ERR_UNSUPPORTED;   // int32 rows
+    if ((long long)pl.units * L_c * 3 >= (1LL << 31)) return KVPACK_ERR_UNSUPPORTED;
     if (ws == nullptr || ws_bytes < pl.total) return KVPACK_ERR_WORKSPACE;
     DeviceInfo *di = nullptr;
     if ((s = device_info(&di)) != KVPACK_OK) return s;
@@ -363,10 +390,16 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     float *ustat = reinterpret_cast<float *>(w + pl.off_ustat);
     float *vpart = reinterpret_cast<float *>(w + pl.off_vp);
     unsigned int *counter = reinterpret_cast<unsigned int *>(w + pl.off_counter);
+    unsigned char *qt2 = L_c > 0 ? w + pl.off_qt2 : nullptr;
+    float *spart2 = L_c > 0 ? reinterpret_cast<float *>(w + pl.off_sp2) : nullptr;
+    float *vpart2 = L_c > 0 ? reinterpret_cast<float *>(w + pl.off_vp2) : nullptr;
+    uint32_t *mask2 = L_c > 0 ? reinterpret_cast<uint32_t *>(w + pl.off_mask2) : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    // the text kernel's work counter starts at zero
+    // the text kernel's work counter starts at zero; the text tokens' own mask is all ones
     if (cudaMemsetAsync(counter, 0, 4 * sizeof(unsigned int), st) != cudaSuccess) return KVPACK_ERR_CUDA;
+    if (L_c > 0 && cudaMemsetAsync(mask2, 0xFF, (size_t)pl.units * pl.nwords2 * sizeof(uint32_t), st) != cudaSuccess)
+        return KVPACK_ERR_CUDA;
 
     // 1. q~ per (unit, KV head) and the text tail partials, one persistent launch
     {
@@ -386,17 +419,20 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
             const cuuint32_t box[3] = {64, 64, 1};
             if (!encode_bf16(enc, &tp.tm_bk, BK, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
                 return KVPACK_ERR_CUDA;
+            if (L_c > 0 && !encode_bf16(enc, &tp.tm_bk2, tb->BK, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+                return KVPACK_ERR_CUDA;
         }
-        tp.q = q; tp.part = tpart; tp.qt = qt; tp.counter = counter;
+        tp.q = q; tp.part = tpart; tp.qt = qt; tp.qt2 = qt2; tp.counter = counter;
         tp.n_units = pl.units; tp.L = L_text; tp.Hg = Hg; tp.per_kv = per_kv; tp.n_q = d->n_q_heads;
-        tp.groups = groups; tp.Sc = Sc; tp.ct = kTextChunk; tp.n_qitems = pl.units * 4;
+        tp.groups = groups; tp.Sc = Sc; tp.ct = kTextChunk; tp.n_qitems = pl.units * 4 * (L_c > 0 ? 2 : 1);
         tp.n_items = tp.n_qitems + pl.units * 4 * Sc; tp.scale2 = scale2;
         const int grid = tp.n_items < di->sms ? tp.n_items : di->sms;
         dc::text::text_kernel<<<grid, dc::text::kThreads, dc::text::smem_bytes(), st>>>(tp);
         if (cudaGetLastError() != cudaSuccess) return KVPACK_ERR_CUDA;
     }
 
-    // 2-4. the visual tokens: softmax statistics, the unit-wide statistics, then the value pass
+    // 2-4. the visual tokens (and the text tokens' own rank space): softmax statistics, the
+    // unit-wide statistics, then the value passes
     rs::Params rp;
     std::memset(&rp, 0, sizeof(rp));
     {
@@ -411,19 +447,79 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
     rp.qt = qt; rp.mask = mask; rp.ustat = ustat;
     rp.units = pl.units; rp.T = T; rp.Hg = Hg; rp.nwords = pl.nwords; rp.tpu = pl.tpu;
     rp.rank0 = d->rank_lo == 0 ? 1 : 0; rp.ntiles = pl.ntiles;
+    rs::Params rp2;
+    std::memset(&rp2, 0, sizeof(rp2));
+    if (L_c > 0) {
+        const cuuint64_t dims[3] = {16, (cuuint64_t)L_c, (cuuint64_t)pl.units};
+        const cuuint64_t strides[2] = {32, (cuuint64_t)L_c * 32};
+        const cuuint32_t box[3] = {16, 256, 1};
+        if (!encode_bf16(enc, &rp2.tm_ck, tb->CK_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B) ||
+            !encode_bf16(enc, &rp2.tm_cv, tb->CV_lo, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_32B))
+            return KVPACK_ERR_CUDA;
+        rp2.CK_lo = tb->CK_lo; rp2.CK_hi = tb->CK_hi; rp2.CV_lo = tb->CV_lo; rp2.CV_hi = tb->CV_hi;
+        rp2.qt = qt2; rp2.mask = mask2; rp2.ustat = ustat;
+        rp2.units = pl.units; rp2.T = L_c; rp2.Hg = Hg; rp2.nwords = pl.nwords2; rp2.tpu = pl.tpu2;
+        rp2.rank0 = 0; rp2.ntiles = pl.ntiles2;
+    }
     rp.part = spart; rp.nslot = pl.nslot_s; rp.mass = nullptr;
     if (launch_rs<false>(pl.NH, rp, pl.cta_s, st) != cudaSuccess) return KVPACK_ERR_CUDA;
-    if (launch_pdl(rs::combine_kernel, (pl.units + 7) / 8, 256, 0, st, (const float *)spart, (const float *)tpart,
-                   ustat, pl.units, Hg, Sc, pl.nslot_s, pl.ntiles, pl.tpu, pl.cta_s) != cudaSuccess)
+    if (L_c > 0) {
+        rp2.part = spart2; rp2.nslot = pl.nslot2; rp2.mass = nullptr;
+        if (launch_rs<false>(pl.NH, rp2, pl.cta2, st) != cudaSuccess) return KVPACK_ERR_CUDA;
+    }
+    const rs::Segs sv{spart, pl.nslot_s, pl.tpu, pl.cta_s, pl.ntiles};
+    const rs::Segs s2{spart2, pl.nslot2, pl.tpu2, pl.cta2, pl.ntiles2};
+    if (launch_pdl(rs::combine_kernel, (pl.units + 7) / 8, 256, 0, st, sv, s2, (const float *)tpart, ustat, pl.units,
+                   Hg, Sc) != cudaSuccess)
         return KVPACK_ERR_CUDA;
     rp.part = vpart; rp.nslot = pl.nslot_v; rp.mass = mass;
     if (launch_rs<true>(pl.NH, rp, pl.cta_v, st) != cudaSuccess) return KVPACK_ERR_CUDA;
+    if (L_c > 0) {
+        rp2.part = vpart2; rp2.nslot = pl.nslot2; rp2.mass = nullptr;
+        if (launch_rs<true>(pl.NH, rp2, pl.cta2, st) != cudaSuccess) return KVPACK_ERR_CUDA;
+    }
 
-    // 5. combine the partials and project through B_V
-    rs::FinishParams fp{BV, vpart, Sc > 0 ? tpart : nullptr, ustat, out, Hg, per_kv, d->n_q_heads, groups, Sc,
-                        pl.nslot_v, pl.tpu, pl.cta_v, pl.ntiles};
-    if (launch_finish(per_kv, fp, pl.units, st) != cudaSuccess) return KVPACK_ERR_CUDA;
+    // 5. combine the partials and project through B_V (and the text tokens' B_V)
+    rs::FinishParams fp{};
+    fp.BV = BV; fp.vpart = vpart; fp.tpart = Sc > 0 ? tpart : nullptr; fp.ustat = ustat; fp.out = out;
+    fp.Hg = Hg; fp.per_kv = per_kv; fp.n_q = d->n_q_heads; fp.groups = groups; fp.Sc = Sc;
+    fp.nslot = pl.nslot_v; fp.tpu = pl.tpu; fp.cta_v = pl.cta_v; fp.ntiles = pl.ntiles;
+    if (L_c > 0) {
+        fp.BV2 = tb->BV; fp.vpart2 = vpart2; fp.nslot2 = pl.nslot2; fp.tpu2 = pl.tpu2; fp.cta_v2 = pl.cta2;
+        fp.ntiles2 = pl.ntiles2;
+    }
+    if (launch_finish(per_kv, fp, pl.units, di->sms, st) != cudaSuccess) return KVPACK_ERR_CUDA;
     return KVPACK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const uint16_t *q,
+                                 const uint16_t *CK_lo, const uint16_t *CK_hi, const uint16_t *BK,
+                                 const uint16_t *CV_lo, const uint16_t *CV_hi, const uint16_t *BV,
+                                 const uint16_t *K_text, const uint16_t *V_text, int32_t L_text,
+                                 const uint32_t *mask, float softmax_scale, uint16_t *out, float *mass,
+                                 void *ws, size_t ws_bytes, void *stream) {
+    return decode_impl(d, n_layers, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, nullptr, K_text, V_text, L_text, mask,
+                       softmax_scale, out, mass, ws, ws_bytes, stream);
+}
+
+size_t kvpack_decode_tb_workspace(const kvpack_dims *d, int32_t n_layers, int32_t L_c) {
+    if (check_dims(d, n_layers) != KVPACK_OK || L_c < 0 || L_c > kMaxT) return 0;
+    return plan_decode(d, n_layers, L_c).total;
+}
+
+kvpack_status kvpack_decode_attn_tb(const kvpack_dims *d, int32_t n_layers, const uint16_t *q,
+                                    const uint16_t *CK_lo, const uint16_t *CK_hi, const uint16_t *BK,
+                                    const uint16_t *CV_lo, const uint16_t *CV_hi, const uint16_t *BV,
+                                    const kvpack_text_basis *tb, const uint16_t *K_text, const uint16_t *V_text,
+                                    int32_t L_text, const uint32_t *mask, float softmax_scale, uint16_t *out,
+                                    float *mass, void *ws, size_t ws_bytes, void *stream) {
+    if (tb == nullptr) return KVPACK_ERR_INVALID_ARG;
+    return decode_impl(d, n_layers, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, tb, K_text, V_text, L_text, mask,
+                       softmax_scale, out, mass, ws, ws_bytes, stream);
 }
 
 }  // extern "C"
@@ -627,14 +723,30 @@ kvpack_status kvpack_select(const kvpack_dims *d, int32_t n_layers, const float 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     const int T = d->T_vis;
+    namespace sl = kvpack::select;
     if (T <= 32 * 64) {
         int kpt = 1;
         while (32 * kpt < T) kpt <<= 1;
-        e = select_dispatch<1>(kpt, p, st);
+        switch (kpt) {
+            case 1: e = launch_select_warp<1>(p, st); break;
+            case 2: e = launch_select_warp<2>(p, st); break;
+            case 4: e = launch_select_warp<4>(p, st); break;
+            case 8: e = launch_select_warp<8>(p, st); break;
+            case 16: e = launch_select_warp<16>(p, st); break;
+            case 32: e = launch_select_warp<32>(p, st); break;
+            default: e = launch_select_warp<64>(p, st); break;
+        }
     } else {
         int kpt = 1;
-        while (1024 * kpt < T) kpt <<= 1;
-        e = select_dispatch<32>(kpt, p, st);
+        while (sl::kClusterCtas * sl::kClusterThreads * kpt < T) kpt <<= 1;
+        switch (kpt) {
+            case 1: e = launch_select_cluster<1>(p, st); break;
+            case 2: e = launch_select_cluster<2>(p, st); break;
+            case 4: e = launch_select_cluster<4>(p, st); break;
+            case 8: e = launch_select_cluster<8>(p, st); break;
+            case 16: e = launch_select_cluster<16>(p, st); break;
+            default: e = launch_select_cluster<32>(p, st); break;
+        }
     }
     return (e == cudaSuccess) ? KVPACK_OK : KVPACK_ERR_CUDA;
 }

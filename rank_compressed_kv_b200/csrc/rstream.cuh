@@ -57,18 +57,23 @@ constexpr int kWarps = 6;
 constexpr int kThreads = kWarps * 32;
 constexpr int kTile = 128;          // tokens per tensor-memory tile (M of the score MMA)
 constexpr int kHiRing = 1024;       // producer's queue of pending full-rank token positions
-constexpr int kMaskWin = 2048;      // producer's window of mask words (65536 tokens)
+constexpr int kMaskWin = 1024;      // producer's window of mask words (32768 tokens)
 constexpr int kDescInts = 8 + 64;   // header + up to 16 mask words (LO) or 128 uint16 positions (HI)
 constexpr int kTypeLo = 0, kTypeHi = 1, kTypeEnd = 2;
 constexpr int kFlagFirst = 1 << 8, kFlagLast = 1 << 9;
 constexpr float kRefInit = -1e30f;
 constexpr float kLazy = 8.f;        // a per-thread reference max moves when a logit exceeds it by 2^8
 
-// Geometry per (query heads NH, pass).  NH is the unit's Hg rounded up to 4, 8, 16 or 32.  Every
-// ring slot is 16 KB: the statistics pass streams K only (a LO tile of 512 tokens of 32-byte
-// rows, a HI tile of 128 tokens of 128-byte rows), the value pass K and V (256 and 64 tokens).
-// A 64-token HI tile still runs the 128-row score MMA; rows 64-127 read the V half of the slot
-// and their scores are never used.
+// Geometry per (query heads NH, pass).  NH is the unit's Hg rounded up to 4, 8, 16 or 32.
+// Three rings per CTA, released independently:
+//   K slots   the C_K part of a tile (statistics pass: a LO tile of 512 tokens of 32-byte rows
+//             or a HI tile of 128 tokens of 128-byte rows, 16 KB; value pass: 256 or 64 tokens,
+//             8 KB), freed by the score MMA's completion (tcgen05.commit) -- the consumers
+//             never read them
+//   V slots   the C_V part of a value-pass tile (8 KB), freed by the consumers after their V sums
+//   S buffers tensor-memory scores of a tile (kSub x kNHP columns), freed by the consumers
+// A 64-token HI tile of the value pass still runs the 128-row score MMA; rows 64-127 read the
+// 8 KB that follow the slot and their scores are never used.
 template <int NH, bool VALUE>
 struct Cfg {
     static constexpr int kNHP = NH < 16 ? 16 : NH;                  // N of the score MMA
@@ -77,11 +82,13 @@ struct Cfg {
     static constexpr int kLoTok = VALUE ? 256 : 512;                 // tokens per LO tile
     static constexpr int kHiTok = VALUE ? 64 : 128;                  // tokens per HI tile
     static constexpr int kSub = kLoTok / kTile;                      // 128-token sub-tiles per LO tile
-    static constexpr int kSlotBytes = 16384;
-    static constexpr int kVOff = 8192;                               // value pass: V rows after the K rows
-    static constexpr int kSlots = VALUE ? (NH <= 16 ? 4 : 8) : 4;
-    static constexpr int kSCols = kSub * kNHP;                       // tensor-memory columns of one slot's scores
-    static constexpr int kTmemCols = kSlots * kSCols;                // 128, 256 or 512
+    static constexpr int kKBytes = VALUE ? 8192 : 16384;
+    static constexpr int kVBytes = 8192;
+    static constexpr int kNK = VALUE ? (NH <= 16 ? 5 : 8) : (NH <= 16 ? 5 : 10);
+    static constexpr int kNV = VALUE ? (NH <= 16 ? 4 : 8) : 1;
+    static constexpr int kNS = 4;
+    static constexpr int kSCols = kSub * kNHP;                       // tensor-memory columns of one S buffer
+    static constexpr int kTmemCols = kNS * kSCols;                   // 128, 256 or 512
     static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "power-of-two allocation");
     static_assert(kLoTok / 32 <= 16 && kHiTok <= 128, "descriptor capacity");
 };
@@ -107,20 +114,30 @@ __host__ __device__ inline long long cta_of_tile(long long x, long long C, long 
 template <int NH, bool VALUE>
 struct Smem {
     using C = Cfg<NH, VALUE>;
-    alignas(1024) unsigned char slot[C::kSlots][C::kSlotBytes];
+    alignas(1024) unsigned char kslot[C::kNK][C::kKBytes];
+    alignas(1024) unsigned char vslot[C::kNV][VALUE ? C::kVBytes : 16];   // follows the K slots (see Cfg)
     alignas(1024) unsigned char qbuf[2][2][C::kNHP * 128];          // [q slot][hi, lo][rows of 128 B]
-    int desc[C::kSlots][kDescInts];
+    int kdesc[C::kNK][kDescInts];                                   // written by the producer with the K slot
+    int sdesc[C::kNS][kDescInts];                                   // copied by the MMA warp for the consumers
     uint32_t mwin[kMaskWin];                                        // producer's window of the CTA's mask words
     uint16_t hi_ring[kHiRing];
     unsigned char pbuf[VALUE ? 4 : 1][VALUE ? 32 * C::kPH * 2 : 16];   // value pass: P rows of each consumer warp
     float merge[VALUE ? 3 : 4][VALUE ? NH * 64 : NH * 2];           // partial merge across the consumer warps
-    uint64_t full[C::kSlots], sfull[C::kSlots], empty[C::kSlots], qfull[2], qempty[2];
+    uint64_t kfull[C::kNK], kempty[C::kNK], vfull[C::kNV], vempty[C::kNV], sfull[C::kNS], sfree[C::kNS];
+    uint64_t qfull[2], qempty[2], mdone;
     uint32_t tmem_base;
     int abort;
 };
 
 template <int NH, bool VALUE>
 constexpr size_t smem_bytes() { return sizeof(Smem<NH, VALUE>) + 1024; }
+
+// resident CTAs per SM as planned: 228 KB of shared memory per SM, 1 KB of it reserved per CTA
+template <int NH, bool VALUE>
+constexpr bool smem_fits() { return Cfg<NH, VALUE>::kBlocks * (smem_bytes<NH, VALUE>() + 1024) <= 233472; }
+static_assert(smem_fits<4, false>() && smem_fits<4, true>() && smem_fits<8, false>() && smem_fits<8, true>(), "smem");
+static_assert(smem_fits<16, false>() && smem_fits<16, true>(), "shared memory of two CTAs per SM");
+static_assert(smem_fits<32, false>() && smem_fits<32, true>(), "shared memory of one CTA per SM");
 
 // ------------------------------------------------------------------ tcgen05 helpers
 
@@ -174,7 +191,7 @@ __device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, float (&v)[32]) {
 template <int NH, bool VALUE>
 __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(const __grid_constant__ Params p) {
     using C = Cfg<NH, VALUE>;
-    constexpr int kSlots = C::kSlots, kNHP = C::kNHP, kPH = C::kPH;
+    constexpr int kNK = C::kNK, kNV = C::kNV, kNS = C::kNS, kNHP = C::kNHP, kPH = C::kPH;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t base0 = smem_u32(smem_raw);
     Smem<NH, VALUE> &sm = *reinterpret_cast<Smem<NH, VALUE> *>(smem_raw + ((1024u - (base0 & 1023u)) & 1023u));
@@ -185,15 +202,23 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
     const long long x0 = tile_begin(blockIdx.x, CT, NT), x1 = tile_begin(blockIdx.x + 1, CT, NT);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kSlots; ++s) {
-            mbar_init(&sm.full[s], 32);
+        for (int s = 0; s < kNK; ++s) {
+            mbar_init(&sm.kfull[s], 32);
+            mbar_init(&sm.kempty[s], 1);
+        }
+        for (int s = 0; s < kNV; ++s) {
+            mbar_init(&sm.vfull[s], 32);
+            mbar_init(&sm.vempty[s], 4);
+        }
+        for (int s = 0; s < kNS; ++s) {
             mbar_init(&sm.sfull[s], 1);
-            mbar_init(&sm.empty[s], 4);
+            mbar_init(&sm.sfree[s], 4);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.qfull[s], 1);
             mbar_init(&sm.qempty[s], 1);
         }
+        mbar_init(&sm.mdone, 1);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -217,10 +242,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
         uint32_t seq = 0, qseq = 0;
         unsigned hi_head = 0, hi_tail = 0;
         bool ok = true;
-        // wait until slot s may be refilled (its previous tile has been consumed)
-        auto acquire = [&](int s) -> bool {
-            if (seq >= (uint32_t)kSlots && !mbar_wait(&sm.empty[s], ((seq / kSlots) - 1) & 1u, abort)) return false;
-            return true;
+        // wait until the K slot (and, in the value pass, the V slot) of tile `seq` may be refilled
+        auto acquire_k = [&](int ks) -> bool {
+            return seq < (uint32_t)kNK || mbar_wait(&sm.kempty[ks], ((seq / kNK) - 1) & 1u, abort);
+        };
+        auto acquire_v = [&](int vs) -> bool {
+            return seq < (uint32_t)kNV || mbar_wait(&sm.vempty[vs], ((seq / kNV) - 1) & 1u, abort);
         };
         // The CTA's mask words are one contiguous run (its tiles are consecutive 128-token tiles
         // and a unit's words follow the previous unit's), read into shared memory a window at a
@@ -238,6 +265,22 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             }
             return sm.mwin + (gw - wbase);
         };
+        // 128-byte rows (C_lo + C_hi, 16-byte chunk c of row r at c ^ (r & 7)) of the listed tokens;
+        // rows past n are zero-filled when `zero` (their p is zero, and 0 * stale data must stay 0)
+        auto gather = [&](unsigned char *dst, const uint16_t *lo, const uint16_t *hi, const uint16_t *pos, int n,
+                          size_t ubase, bool zero) {
+            #pragma unroll 4
+            for (int k = 0; k < C::kHiTok * 8 / 32; ++k) {
+                const int idx = lane + 32 * k;
+                const int r = idx >> 3, ch = idx & 7;
+                const bool valid = r < n;
+                const size_t row = ubase + pos[r];
+                const uint16_t *src = ch < 2 ? lo + row * 16 + ch * 8 : hi + row * 48 + (ch - 2) * 8;
+                unsigned char *d = dst + r * 128 + ((ch ^ (r & 7)) << 4);
+                if (zero) cp_async16_zfill(d, src, valid);
+                else if (valid) cp_async16(d, src);
+            }
+        };
         long long x = x0;
         while (ok && x < x1) {
             const int unit = (int)(x / p.tpu);
@@ -246,6 +289,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             const int tok0 = (int)(x - (long long)unit * p.tpu) * kTile;
             const int tok1 = min(p.T, (int)(xe - (long long)unit * p.tpu) * kTile);
             const int pslot = (int)(blockIdx.x - cta_of_tile((long long)unit * p.tpu, CT, NT));
+            const size_t ubase = (size_t)unit * p.T;
             x = xe;
             // the unit's q~ into the next q slot
             const int qs = qseq & 1;
@@ -294,39 +338,51 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 const int hi_now = (int)(pend / C::kHiTok) + ((final_blk && (pend % C::kHiTok) != 0) ? 1 : 0);
                 if (nhi < n) {
                     // ------------------------------------------------ LO tile
-                    const int s = seq % kSlots;
-                    if (!acquire(s)) { ok = false; break; }
-                    int *d = sm.desc[s];
+                    const int ks = seq % kNK;
+                    if (!acquire_k(ks)) { ok = false; break; }
+                    int *d = sm.kdesc[ks];
                     if (lane == 0) {
                         d[0] = kTypeLo | (first ? kFlagFirst : 0) | ((final_blk && hi_now == 0) ? kFlagLast : 0);
                         d[1] = unit; d[2] = tok; d[3] = n; d[4] = pslot; d[5] = qs;
                     }
                     if (lane < C::kLoTok / 32) d[8 + lane] = (int)wd;
                     first = false;
+                    const int nb = (n + 255) >> 8;   // 256-row boxes of 32-byte rows
                     if (!p.rank0) {
-                        const int nb = (n + 255) >> 8;   // 256-row boxes
                         if (lane == 0) {
-                            unsigned char *dst = sm.slot[s];
                             fence_proxy_async();
-                            mbar_arrive_tx(&sm.full[s], (uint32_t)nb * 8192u * (VALUE ? 2u : 1u));
-                            for (int b = 0; b < nb; ++b) {
-                                tma_3d(dst + 8192 * b, &p.tm_ck, 0, tok + 256 * b, unit, &sm.full[s]);
-                                if (VALUE) tma_3d(dst + C::kVOff + 8192 * b, &p.tm_cv, 0, tok + 256 * b, unit, &sm.full[s]);
-                            }
+                            mbar_arrive_tx(&sm.kfull[ks], (uint32_t)nb * 8192u);
+                            for (int b = 0; b < nb; ++b)
+                                tma_3d(sm.kslot[ks] + 8192 * b, &p.tm_ck, 0, tok + 256 * b, unit, &sm.kfull[ks]);
                         } else {
-                            mbar_arrive(&sm.full[s]);
+                            mbar_arrive(&sm.kfull[ks]);
                         }
                     } else {
-                        mbar_arrive(&sm.full[s]);
+                        mbar_arrive(&sm.kfull[ks]);
+                    }
+                    if (VALUE) {
+                        const int vs = seq % kNV;
+                        if (!acquire_v(vs)) { ok = false; break; }
+                        if (!p.rank0) {
+                            if (lane == 0) {
+                                fence_proxy_async();
+                                mbar_arrive_tx(&sm.vfull[vs], 8192u);
+                                tma_3d(sm.vslot[vs], &p.tm_cv, 0, tok, unit, &sm.vfull[vs]);
+                            } else {
+                                mbar_arrive(&sm.vfull[vs]);
+                            }
+                        } else {
+                            mbar_arrive(&sm.vfull[vs]);
+                        }
                     }
                     ++seq;
                 }
                 for (int i = 0; i < hi_now && ok; ++i) {
                     // ------------------------------------------------ HI tile
-                    const int s = seq % kSlots;
-                    if (!acquire(s)) { ok = false; break; }
+                    const int ks = seq % kNK;
+                    if (!acquire_k(ks)) { ok = false; break; }
                     const int nh = (int)min((unsigned)C::kHiTok, hi_tail - hi_head);
-                    int *d = sm.desc[s];
+                    int *d = sm.kdesc[ks];
                     uint16_t *pos = reinterpret_cast<uint16_t *>(d + 8);
                     if (lane == 0) {
                         d[0] = kTypeHi | (first ? kFlagFirst : 0) | ((final_blk && i == hi_now - 1) ? kFlagLast : 0);
@@ -339,63 +395,73 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                     }
                     first = false;
                     __syncwarp();
-                    // C_lo + C_hi rows into 128-byte rows (16-byte chunk c of row r at c ^ (r & 7));
-                    // V rows past nh are zero-filled (their p is zero, and 0 * stale data must stay 0)
-                    unsigned char *dst = sm.slot[s];
-                    const size_t ubase = (size_t)unit * p.T;
-                    #pragma unroll 4
-                    for (int k = 0; k < C::kHiTok * 8 / 32; ++k) {
-                        const int idx = lane + 32 * k;
-                        const int r = idx >> 3, ch = idx & 7;
-                        const bool valid = r < nh;
-                        const size_t row = ubase + pos[r];
-                        const int off = r * 128 + ((ch ^ (r & 7)) << 4);
-                        const uint16_t *sk = ch < 2 ? p.CK_lo + row * 16 + ch * 8 : p.CK_hi + row * 48 + (ch - 2) * 8;
-                        if (valid) cp_async16(dst + off, sk);
-                        if (VALUE) {
-                            const uint16_t *sv = ch < 2 ? p.CV_lo + row * 16 + ch * 8 : p.CV_hi + row * 48 + (ch - 2) * 8;
-                            cp_async16_zfill(dst + C::kVOff + off, sv, valid);
-                        }
+                    gather(sm.kslot[ks], p.CK_lo, p.CK_hi, pos, nh, ubase, false);
+                    cp_async_arrive(&sm.kfull[ks]);   // raises the pending count; arrives when the copies land
+                    mbar_arrive(&sm.kfull[ks]);       // releases this lane's descriptor writes
+                    if (VALUE) {
+                        const int vs = seq % kNV;
+                        if (!acquire_v(vs)) { ok = false; break; }
+                        gather(sm.vslot[vs], p.CV_lo, p.CV_hi, pos, nh, ubase, true);
+                        cp_async_arrive(&sm.vfull[vs]);
+                        mbar_arrive(&sm.vfull[vs]);
                     }
-                    cp_async_arrive(&sm.full[s]);   // raises the pending count; arrives when the copies land
-                    mbar_arrive(&sm.full[s]);       // releases this lane's descriptor writes
                     hi_head += (unsigned)nh;
                     ++seq;
                 }
             }
         }
-        // end marker
+        // end marker (K ring only: the MMA warp passes it on to the consumers)
+        bool ended = false;
         if (ok) {
-            const int s = seq % kSlots;
-            if (acquire(s)) {
-                if (lane == 0) sm.desc[s][0] = kTypeEnd;
-                mbar_arrive(&sm.full[s]);
-                ++seq;
+            const int ks = seq % kNK;
+            if (acquire_k(ks)) {
+                if (lane == 0) sm.kdesc[ks][0] = kTypeEnd;
+                mbar_arrive(&sm.kfull[ks]);
+                ended = true;
             } else {
                 ok = false;
             }
         }
         if (!ok) *abort = 1;
-        // copies still in flight (only after an abort) must land before the block exits
+        // Copies still in flight (possible only when a role gave up) must land before the block
+        // exits: wait for the data phases of the last tiles of each ring.  A parity wait is only
+        // meaningful while its phase is the slot's latest, so on the K ring the slot that carried
+        // the end marker (whose tile was consumed before the marker could be written) is skipped.
         cp_async_wait_all();
-        for (uint32_t k = (seq > (uint32_t)kSlots ? seq - kSlots : 0u); k < seq; ++k) {
+        const uint32_t kfirst = seq > (uint32_t)kNK ? seq - kNK + (ended ? 1u : 0u) : 0u;
+        for (uint32_t k = kfirst; k < seq; ++k) {
             const long long t0 = clock64();
-            while (!mbar_try_wait(&sm.full[k % kSlots], (k / kSlots) & 1u) && clock64() - t0 < kWaitCycles) {}
+            while (!mbar_try_wait(&sm.kfull[k % kNK], (k / kNK) & 1u) && clock64() - t0 < kWaitCycles) {}
+        }
+        if (VALUE) {
+            for (uint32_t k = (seq > (uint32_t)kNV ? seq - kNV : 0u); k < seq; ++k) {
+                const long long t0 = clock64();
+                while (!mbar_try_wait(&sm.vfull[k % kNV], (k / kNV) & 1u) && clock64() - t0 < kWaitCycles) {}
+            }
         }
     } else if (warp == 1) {
         // =============================================================== MMA issuer
         if (lane == 0) {
-            uint32_t seq = 0, qseq = 0, last_sfull = 0xffffffffu;
+            uint32_t seq = 0, qseq = 0;
+            bool issued = false;
             const uint32_t id_s = idesc_bf16_kk(128, kNHP);
             while (true) {
-                const int s = seq % kSlots;
-                if (!mbar_wait(&sm.full[s], (seq / kSlots) & 1u, abort)) break;
-                // the descriptor is read before the commit below: once the consumers are done the
-                // producer may rewrite it
-                const int *d = sm.desc[s];
+                const int ks = seq % kNK, sb = seq % kNS;
+                if (!mbar_wait(&sm.kfull[ks], (seq / kNK) & 1u, abort)) break;
+                // the S buffer (scores and descriptor) of the tile kNS back must have been read
+                if (seq >= (uint32_t)kNS && !mbar_wait(&sm.sfree[sb], ((seq / kNS) - 1) & 1u, abort)) break;
+                // the descriptor moves on with the scores: the K slot is released by the MMA's completion
+                const int *d = sm.kdesc[ks];
+                int *sd = sm.sdesc[sb];
                 const int hdr = d[0];
                 const int type = hdr & 0xff;
-                if (type == kTypeEnd) break;
+                if (type == kTypeEnd) {
+                    sd[0] = kTypeEnd;
+                    mbar_arrive(&sm.sfull[sb]);
+                    break;
+                }
+                #pragma unroll 8
+                for (int i = 0; i < kDescInts; ++i) sd[i] = d[i];
                 const int qs = d[5], n = d[3];
                 if (hdr & kFlagFirst) {
                     if (!mbar_wait(&sm.qfull[qs], (qseq >> 1) & 1u, abort)) break;
@@ -405,36 +471,39 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 if (has_s) {
                     if (type == kTypeHi) fence_proxy_async();   // the gathered rows were written by cp.async
                     tmem_fence_after();
-                    const uint32_t dcol = tmem + (uint32_t)(s * C::kSCols);
+                    const uint32_t dcol = tmem + (uint32_t)(sb * C::kSCols);
                     const uint32_t qh = smem_u32(&sm.qbuf[qs][0][0]), ql = smem_u32(&sm.qbuf[qs][1][0]);
-                    const uint32_t sb = smem_u32(sm.slot[s]);
+                    const uint32_t kb = smem_u32(sm.kslot[ks]);
                     if (type == kTypeLo) {
                         for (int sub = 0; sub * kTile < n; ++sub) {
-                            const uint64_t a = desc_kmajor(sb + 4096u * sub, 256u, 6u);
+                            const uint64_t a = desc_kmajor(kb + 4096u * sub, 256u, 6u);
                             umma_bf16(dcol + sub * kNHP, a, desc_kmajor(qh, 1024u, 2u), id_s, 0u);
                             umma_bf16(dcol + sub * kNHP, a, desc_kmajor(ql, 1024u, 2u), id_s, 1u);
                         }
                     } else {
                         #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            const uint64_t a = desc_kmajor(sb + 32u * k, 1024u, 2u);
+                            const uint64_t a = desc_kmajor(kb + 32u * k, 1024u, 2u);
                             umma_bf16(dcol, a, desc_kmajor(qh + 32u * k, 1024u, 2u), id_s, k > 0 ? 1u : 0u);
                             umma_bf16(dcol, a, desc_kmajor(ql + 32u * k, 1024u, 2u), id_s, 1u);
                         }
                     }
-                    umma_commit(&sm.sfull[s]);
-                    last_sfull = seq;
+                    umma_commit(&sm.sfull[sb]);
+                    umma_commit(&sm.kempty[ks]);
+                    issued = true;
                 } else {
-                    mbar_arrive(&sm.sfull[s]);   // keeps the slot's score-barrier phases in step
+                    mbar_arrive(&sm.sfull[sb]);   // keeps the rings' phases in step
+                    mbar_arrive(&sm.kempty[ks]);
                 }
                 if (hdr & kFlagLast) umma_commit(&sm.qempty[qs]);
                 ++seq;
             }
-            // MMAs still in flight (only after an abort) must finish before tensor memory is freed
-            if (last_sfull != 0xffffffffu) {
+            // MMAs still in flight (possible only after an abort) must finish before tensor memory
+            // is freed: one more commit, to a barrier of its own, arrives once all of them are done
+            if (issued) {
+                umma_commit(&sm.mdone);
                 const long long t0 = clock64();
-                while (!mbar_try_wait(&sm.sfull[last_sfull % kSlots], (last_sfull / kSlots) & 1u) &&
-                       clock64() - t0 < kWaitCycles) {}
+                while (!mbar_try_wait(&sm.mdone, 0u) && clock64() - t0 < kWaitCycles) {}
             }
         }
         __syncwarp();
@@ -452,11 +521,13 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
         int unit = 0, pslot = 0;
         unsigned char *pb = sm.pbuf[VALUE ? q : 0];
         const uint32_t pb_s = smem_u32(pb);
-        while (true) {
-            const int s = seq % kSlots;
-            if (!mbar_wait(&sm.full[s], (seq / kSlots) & 1u, abort)) break;
-            const int *d = sm.desc[s];
-            const int hdr = d[0];                    // read before this warp releases the slot
+        bool failed = false;
+        while (!failed) {
+            const int sb = seq % kNS, vs = seq % kNV;
+            if (!mbar_wait(&sm.sfull[sb], (seq / kNS) & 1u, abort)) break;
+            tmem_fence_after();
+            const int *d = sm.sdesc[sb];
+            const int hdr = d[0];
             const int type = hdr & 0xff;
             if (type == kTypeEnd) break;
             const int n = d[3];
@@ -481,13 +552,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 }
             }
             const bool has_s = type == kTypeHi || !p.rank0;
-            if (!mbar_wait(&sm.sfull[s], (seq / kSlots) & 1u, abort)) break;
-            tmem_fence_after();
             const int nsub = type == kTypeLo ? (n + kTile - 1) / kTile : 1;
-            const uint32_t sb = smem_u32(sm.slot[s]);
+            const uint32_t vb = smem_u32(sm.vslot[vs]);
+            bool v_ready = false;
             // the scores of up to kLd sub-tiles are loaded from tensor memory before one wait
             constexpr int kLd = (C::kSub * NH <= 64) ? C::kSub : (64 / NH > 0 ? 64 / NH : 1);
-            for (int sub0 = 0; sub0 < nsub; sub0 += kLd) {
+            for (int sub0 = 0; sub0 < nsub && !failed; sub0 += kLd) {
                 float scv[kLd][NH];
                 #pragma unroll
                 for (int j = 0; j < kLd; ++j) {
@@ -495,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                     if (has_s && sub < nsub && sub * kTile + 32 * q < n) {
                         constexpr int NL = NH < 4 ? 4 : NH;
                         float v[NL];
-                        tmem_ld<NL>(tmem + lane_addr + (uint32_t)(s * C::kSCols + sub * kNHP), v);
+                        tmem_ld<NL>(tmem + lane_addr + (uint32_t)(sb * C::kSCols + sub * kNHP), v);
                         #pragma unroll
                         for (int h = 0; h < NH; ++h) scv[j][h] = v[h];
                     } else {
@@ -554,6 +624,10 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                     }
                     if (take && p.mass != nullptr) p.mass[(size_t)unit * p.T + pos] = ms0 + ms1;
                     const bool do_u = type == kTypeHi || !p.rank0;
+                    if (do_u && !v_ready) {
+                        if (!mbar_wait(&sm.vfull[vs], (seq / C::kNV) & 1u, abort)) { failed = true; break; }
+                        v_ready = true;
+                    }
                     if (do_u) {
                         // this thread's P row (kPH bf16), 16-byte chunks swizzled against bank conflicts
                         const int prow = lane;
@@ -602,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                                 uint32_t a[4];
                                 const int row = tb + (lane & 7) + ((lane >> 4) << 3);
                                 const int ch = (lane >> 3) & 1;
-                                ldsm_x4_t(sb + C::kVOff + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), a[0], a[1], a[2], a[3]);
+                                ldsm_x4_t(vb + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), a[0], a[1], a[2], a[3]);
                                 #pragma unroll
                                 for (int nt = 0; nt < kPH / 8; ++nt) mma_bf16(u[0][nt], a, bfr[nt][0], bfr[nt][1]);
                             } else {
@@ -611,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                                     uint32_t a[4];
                                     const int row = tb + (lane & 7) + ((lane >> 4) << 3);
                                     const int ch = 2 * mt + ((lane >> 3) & 1);
-                                    ldsm_x4_t(sb + C::kVOff + row * 128 + ((ch ^ (row & 7)) << 4), a[0], a[1], a[2], a[3]);
+                                    ldsm_x4_t(vb + row * 128 + ((ch ^ (row & 7)) << 4), a[0], a[1], a[2], a[3]);
                                     #pragma unroll
                                     for (int nt = 0; nt < kPH / 8; ++nt) mma_bf16(u[mt][nt], a, bfr[nt][0], bfr[nt][1]);
                                 }
@@ -622,10 +696,16 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 }
                 }
             }
-            // this slot is free once every consumer warp has read its scores (and, in the value pass, its V rows)
+            if (failed) break;
+            // the V slot (value pass) and the S buffer are free once every consumer warp is done
+            if (VALUE) {
+                if (!v_ready && !mbar_wait(&sm.vfull[vs], (seq / kNV) & 1u, abort)) break;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.vempty[vs]);
+            }
             tmem_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.empty[s]);
+            if (lane == 0) mbar_arrive(&sm.sfree[sb]);
 
             if (hdr & kFlagLast) {
                 // ---------------------------------------------------------- the segment's partial
@@ -694,6 +774,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             }
             ++seq;
         }
+        if (failed) *abort = 1;
     }
 
     tmem_fence_before();
@@ -707,27 +788,47 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
 // ------------------------------------------------------------------ combine
 
 // Per unit and query head (one warp per unit, a lane per head): the unit-wide max M and
-// sum L over the stats pass's segment partials and the text tail's chunk partials; writes
-// (M, 1/L) for the value pass and the finish.
-__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ spart, const float *__restrict__ tpart,
-                                                      float *__restrict__ ustat, int units, int Hg, int Sc, int nslot,
-                                                      long long ntiles, int tpu, int cta_s) {
+// sum L over the statistics pass's segment partials, those of the text tokens' own
+// rank-space pass when the text is compressed too, and the text tail's chunk partials;
+// writes (M, 1/L) for the value passes and the finish.
+struct Segs {
+    const float *part;      // [units][nslot][Hg][2] = (m, l), or null
+    int nslot, tpu, ctas;
+    long long ntiles;
+};
+
+// partials of a unit: one per CTA that holds some of its tiles
+__device__ __forceinline__ int seg_count(const Segs &s, int unit) {
+    const long long f = (long long)unit * s.tpu;
+    return (int)(cta_of_tile(f + s.tpu - 1, s.ctas, s.ntiles) - cta_of_tile(f, s.ctas, s.ntiles)) + 1;
+}
+
+__global__ void __launch_bounds__(256) combine_kernel(const Segs sv, const Segs st, const float *__restrict__ tpart,
+                                                      float *__restrict__ ustat, int units, int Hg, int Sc) {
     griddep_launch_dependents();
     griddep_wait();
     const int unit = blockIdx.x * 8 + (threadIdx.x >> 5), h = threadIdx.x & 31;
     if (unit >= units || h >= Hg) return;
-    const long long f = (long long)unit * tpu;
-    const int c0 = (int)cta_of_tile(f, cta_s, ntiles), c1 = (int)cta_of_tile(f + tpu - 1, cta_s, ntiles);
-    const float *sp = spart + ((size_t)unit * nslot * Hg + h) * 2;
     const float *tp = tpart + (size_t)unit * Sc * Hg * kTxtPart + (size_t)h * kTxtPart;
-    float mx = -INFINITY;
-    for (int k = 0; k <= c1 - c0; ++k) mx = fmaxf(mx, sp[(size_t)k * Hg * 2]);
-    for (int c = 0; c < Sc; ++c) mx = fmaxf(mx, tp[(size_t)c * Hg * kTxtPart]);
-    float sum = 0.f;
-    for (int k = 0; k <= c1 - c0; ++k) sum += sp[(size_t)k * Hg * 2 + 1] * ex2(sp[(size_t)k * Hg * 2] - mx);
-    for (int c = 0; c < Sc; ++c) {
-        const float mc = tp[(size_t)c * Hg * kTxtPart];
-        if (mc != -INFINITY) sum += tp[(size_t)c * Hg * kTxtPart + 1] * ex2(mc - mx);
+    float mx = -INFINITY, sum = 0.f;
+    #pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {       // the maximum first, then the sum
+        for (int which = 0; which < 2; ++which) {
+            const Segs &sg = which == 0 ? sv : st;
+            if (sg.part == nullptr) continue;
+            const int n = seg_count(sg, unit);
+            const float *sp = sg.part + ((size_t)unit * sg.nslot * Hg + h) * 2;
+            for (int k = 0; k < n; ++k) {
+                const float m = sp[(size_t)k * Hg * 2];
+                if (pass == 0) mx = fmaxf(mx, m);
+                else sum += sp[(size_t)k * Hg * 2 + 1] * ex2(m - mx);
+            }
+        }
+        for (int c = 0; c < Sc; ++c) {
+            const float mc = tp[(size_t)c * Hg * kTxtPart];
+            if (pass == 0) mx = fmaxf(mx, mc);
+            else if (mc != -INFINITY) sum += tp[(size_t)c * Hg * kTxtPart + 1] * ex2(mc - mx);
+        }
     }
     *reinterpret_cast<float2 *>(ustat + ((size_t)unit * Hg + h) * 2) = make_float2(mx, 1.f / sum);
 }
@@ -737,6 +838,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 struct FinishParams {
     const uint16_t *BV;       // [units][64][512]
     const float *vpart;       // [units][nslot][Hg][64]: u = sum p' C_V per segment
+    const uint16_t *BV2;      // the text tokens' own B_V, or null
+    const float *vpart2;      // [units][nslot2][Hg][64]: their u per segment
+    int nslot2, tpu2, cta_v2;
+    long long ntiles2;
     const float *tpart;       // [units][Sc][Hg][kTxtPart] or null
     const float *ustat;       // [units][Hg][2]: (M, 1/L)
     uint16_t *out;            // [(layer, batch)][n_q][128]
@@ -744,49 +849,67 @@ struct FinishParams {
     long long ntiles;
 };
 
-// One block of 128 threads per (unit, KV head j): u_h = the sum of the unit's segment
-// partials, w_h = the text chunks' sums weighted by 2^(m_c - M_h), then
-// o_h = (u_h B_V[:, 128 j ..] + w_h) / L_h for the PK query heads of KV head j, thread t
-// owning output feature t.  The loads of each stage are independent of one another (the
-// chunk weights are computed once into shared memory first), so they are all in flight at once.
+// One block per (unit, JPB KV heads), 128 threads per KV head j: u_h = the sum of the unit's
+// segment partials, w_h = the text chunks' sums weighted by 2^(m_c - M_h), then
+// o_h = (u_h B_V[:, 128 j ..] + u2_h B_V2[:, 128 j ..] + w_h) / L_h for the PK query heads of
+// each KV head (u2, B_V2: the text tokens' own rank space, when the text is compressed), thread t
+// owning output feature t % 128 of KV head j0 + t / 128.  The loads of each stage are
+// independent of one another (the chunk weights are computed once into shared memory first),
+// so they are all in flight at once.  JPB = 4 (a whole unit per block) when units are many,
+// 1 when few, so that the launch fills the GPU either way.
 constexpr int kFinishMaxChunks = 64;   // text chunks whose weights are staged; longer tails loop
 
-template <int PK>
-__global__ void __launch_bounds__(128) finish_kernel(const FinishParams p) {
-    __shared__ float uf[PK][64];
-    __shared__ float ew[PK][kFinishMaxChunks];
-    __shared__ float ms[PK][2];
+template <int PK, int JPB>
+__global__ void __launch_bounds__(128 * JPB) finish_kernel(const FinishParams p) {
+    constexpr int NHB = PK * JPB;           // query heads of the block
+    __shared__ float uf[NHB][64];
+    __shared__ float uf2[NHB][64];
+    __shared__ float ew[NHB][kFinishMaxChunks];
+    __shared__ float ms[NHB][2];
     griddep_wait();
-    const int unit = blockIdx.x >> 2, j = blockIdx.x & 3, tid = threadIdx.x;
-    const int h0 = j * PK;
-    // B_V[:, 128 j + tid] for all 64 ranks: issued first, used last
-    const uint16_t *bv = p.BV + (size_t)unit * 64 * 512 + 128 * j + tid;
+    constexpr int kBlocksPerUnit = 4 / JPB;
+    const int unit = blockIdx.x / kBlocksPerUnit, tid = threadIdx.x;
+    const int j0 = (blockIdx.x % kBlocksPerUnit) * JPB, jj = tid >> 7, dcol = tid & 127;
+    const int hb0 = j0 * PK;                // first query head of the block (within the unit)
+    // B_V[:, 128 (j0 + jj) + dcol] for all 64 ranks: issued first, used last
+    const uint16_t *bv = p.BV + (size_t)unit * 64 * 512 + 128 * j0 + tid;
     uint16_t braw[64];
     #pragma unroll
     for (int r = 0; r < 64; ++r) braw[r] = __ldcs(bv + (size_t)r * 512);
-    if (tid < PK) {
-        const float2 st = __ldg(reinterpret_cast<const float2 *>(p.ustat + ((size_t)unit * p.Hg + h0 + tid) * 2));
+    if (tid < NHB) {
+        const float2 st = __ldg(reinterpret_cast<const float2 *>(p.ustat + ((size_t)unit * p.Hg + hb0 + tid) * 2));
         ms[tid][0] = st.x;
         ms[tid][1] = st.y;
     }
     const long long f = (long long)unit * p.tpu;
     const int ns = (int)(cta_of_tile(f + p.tpu - 1, p.cta_v, p.ntiles) - cta_of_tile(f, p.cta_v, p.ntiles)) + 1;
-    for (int i = tid; i < PK * 64; i += 128) {
+    for (int i = tid; i < NHB * 64; i += 128 * JPB) {
         const int hh = i >> 6, r = i & 63;
-        const float *src = p.vpart + ((size_t)unit * p.nslot * p.Hg + h0 + hh) * 64 + r;
+        const float *src = p.vpart + ((size_t)unit * p.nslot * p.Hg + hb0 + hh) * 64 + r;
         float a = 0.f;
         for (int k = 0; k < ns; ++k) a += __ldcg(src + (size_t)k * p.Hg * 64);
         uf[hh][r] = a;
+    }
+    if (p.vpart2 != nullptr) {
+        const long long f2 = (long long)unit * p.tpu2;
+        const int ns2 = (int)(cta_of_tile(f2 + p.tpu2 - 1, p.cta_v2, p.ntiles2) - cta_of_tile(f2, p.cta_v2, p.ntiles2)) + 1;
+        for (int i = tid; i < NHB * 64; i += 128 * JPB) {
+            const int hh = i >> 6, r = i & 63;
+            const float *src = p.vpart2 + ((size_t)unit * p.nslot2 * p.Hg + hb0 + hh) * 64 + r;
+            float a = 0.f;
+            for (int k = 0; k < ns2; ++k) a += __ldcg(src + (size_t)k * p.Hg * 64);
+            uf2[hh][r] = a;
+        }
     }
     __syncthreads();
     float wacc[PK];
     #pragma unroll
     for (int hh = 0; hh < PK; ++hh) wacc[hh] = 0.f;
     if (p.tpart != nullptr) {
-        const float *tp0 = p.tpart + ((size_t)unit * p.Sc * p.Hg + h0) * kTxtPart;
+        const float *tp0 = p.tpart + ((size_t)unit * p.Sc * p.Hg + hb0) * kTxtPart;
         for (int c0 = 0; c0 < p.Sc; c0 += kFinishMaxChunks) {
             const int nc = min(kFinishMaxChunks, p.Sc - c0);
-            for (int i = tid; i < PK * nc; i += 128) {
+            for (int i = tid; i < NHB * nc; i += 128 * JPB) {
                 const int hh = i / nc, c = i % nc;
                 const float mc = __ldcg(tp0 + ((size_t)(c0 + c) * p.Hg + hh) * kTxtPart);
                 ew[hh][c] = mc != -INFINITY ? ex2(mc - ms[hh][0]) : 0.f;
@@ -794,14 +917,15 @@ __global__ void __launch_bounds__(128) finish_kernel(const FinishParams p) {
             __syncthreads();
             #pragma unroll
             for (int hh = 0; hh < PK; ++hh) {
-                const float *tp = tp0 + (size_t)hh * kTxtPart + 2 + tid;
+                const int hb = jj * PK + hh;
+                const float *tp = tp0 + (size_t)hb * kTxtPart + 2 + dcol;
                 float a0 = 0.f, a1 = 0.f;
                 int c = 0;
                 for (; c + 1 < nc; c += 2) {
-                    a0 = fmaf(__ldcg(tp + (size_t)(c0 + c) * p.Hg * kTxtPart), ew[hh][c], a0);
-                    a1 = fmaf(__ldcg(tp + (size_t)(c0 + c + 1) * p.Hg * kTxtPart), ew[hh][c + 1], a1);
+                    a0 = fmaf(__ldcg(tp + (size_t)(c0 + c) * p.Hg * kTxtPart), ew[hb][c], a0);
+                    a1 = fmaf(__ldcg(tp + (size_t)(c0 + c + 1) * p.Hg * kTxtPart), ew[hb][c + 1], a1);
                 }
-                if (c < nc) a0 = fmaf(__ldcg(tp + (size_t)(c0 + c) * p.Hg * kTxtPart), ew[hh][c], a0);
+                if (c < nc) a0 = fmaf(__ldcg(tp + (size_t)(c0 + c) * p.Hg * kTxtPart), ew[hb][c], a0);
                 wacc[hh] += a0 + a1;
             }
             __syncthreads();
@@ -814,13 +938,23 @@ __global__ void __launch_bounds__(128) finish_kernel(const FinishParams p) {
     for (int r = 0; r < 64; ++r) {
         const float b = __uint_as_float((uint32_t)braw[r] << 16);
         #pragma unroll
-        for (int hh = 0; hh < PK; ++hh) acc[hh] = fmaf(uf[hh][r], b, acc[hh]);
+        for (int hh = 0; hh < PK; ++hh) acc[hh] = fmaf(uf[jj * PK + hh][r], b, acc[hh]);
+    }
+    if (p.BV2 != nullptr) {
+        const uint16_t *bv2 = p.BV2 + (size_t)unit * 64 * 512 + 128 * j0 + tid;
+        #pragma unroll 8
+        for (int r = 0; r < 64; ++r) {
+            const float b = __uint_as_float((uint32_t)__ldcs(bv2 + (size_t)r * 512) << 16);
+            #pragma unroll
+            for (int hh = 0; hh < PK; ++hh) acc[hh] = fmaf(uf2[jj * PK + hh][r], b, acc[hh]);
+        }
     }
     const int lb = unit / p.groups, G = unit % p.groups;
     #pragma unroll
     for (int hh = 0; hh < PK; ++hh) {
-        const float o = (acc[hh] + wacc[hh]) * ms[hh][1];
-        p.out[((size_t)lb * p.n_q + (size_t)G * p.Hg + h0 + hh) * 128 + tid] = float_to_bf16_bits(o);
+        const int hb = jj * PK + hh;
+        const float o = (acc[hh] + wacc[hh]) * ms[hb][1];
+        p.out[((size_t)lb * p.n_q + (size_t)G * p.Hg + hb0 + hb) * 128 + dcol] = float_to_bf16_bits(o);
     }
 }
 

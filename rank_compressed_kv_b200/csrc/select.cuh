@@ -13,7 +13,7 @@
 // correct sort with ties to the lower index.
 //
 // Small T (<= 2048): one warp per unit, 8 units per block.
-// Large T (<= 65536): one 1024-thread block per unit.
+// Large T (<= 65536): a cluster of 8 CTAs of 256 threads per unit (up to 32 keys per thread).
 #pragma once
 
 #include "common.cuh"
@@ -36,139 +36,12 @@ struct Params {
     uint32_t *mask;
 };
 
-// Sum over the threads that share a unit.  NW == 1: the warp; otherwise the block.
-template <int NW>
-__device__ __forceinline__ int group_sum(int v, int *red) {
-    v = __reduce_add_sync(0xffffffffu, v);
-    if constexpr (NW == 1) {
-        return v;
-    } else {
-        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-        if (lane == 0) red[warp] = v;
-        __syncthreads();
-        int s = (lane < NW) ? red[lane] : 0;
-        s = __reduce_add_sync(0xffffffffu, s);
-        __syncthreads();
-        return s;
-    }
-}
-
-// Exclusive prefix sum over the unit's threads in thread order.
-template <int NW>
-__device__ __forceinline__ int group_exclusive_scan(int v, int *red) {
-    const int lane = threadIdx.x & 31;
-    int incl = v;
-    #pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += o;
-    }
-    if constexpr (NW == 1) {
-        return incl - v;
-    } else {
-        const int warp = threadIdx.x >> 5;
-        if (lane == 31) red[warp] = incl;
-        __syncthreads();
-        if (warp == 0) {
-            int w = (lane < NW) ? red[lane] : 0;
-            int wi = w;
-            #pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const int o = __shfl_up_sync(0xffffffffu, wi, d);
-                if (lane >= d) wi += o;
-            }
-            red[32 + lane] = wi - w;
-        }
-        __syncthreads();
-        const int base = red[32 + warp];
-        __syncthreads();
-        return base + incl - v;
-    }
-}
-
-// Keys of the unit: KR per thread in registers, the other KS = KPT - KR in shared memory
-// (a 1024-thread block has 64 registers per thread, too few for 64 keys and the rest).
-template <int KPT, int NW>
-struct KeySplit {
-    static constexpr int KR = (NW > 1 && KPT > 32) ? 32 : KPT;
-    static constexpr int KS = KPT - KR;
-};
-
-template <int KPT, int NW>
-constexpr size_t select_smem_bytes() { return (size_t)KeySplit<KPT, NW>::KS * 32 * NW * sizeof(uint32_t); }
-
-template <int KPT, int NW>
-__global__ void __launch_bounds__(NW == 1 ? 256 : 32 * NW) select_kernel(Params p) {
-    constexpr int KR = KeySplit<KPT, NW>::KR, KS = KeySplit<KPT, NW>::KS;
-    __shared__ int red[64];
-    extern __shared__ uint32_t skeys[];     // [KS][threads]: key KR + i of thread r at [i][r]
-    int unit, r;
-    if constexpr (NW == 1) {
-        unit = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-        r = threadIdx.x & 31;
-        if (unit >= p.n_units) return;      // whole warp leaves together
-    } else {
-        unit = blockIdx.x;
-        r = threadIdx.x;
-    }
-    const int T = p.T;
-    const size_t ub = (size_t)unit * T;
-    const float one_minus = __fsub_rn(1.0f, p.alpha);
-
-    auto load_key = [&](int i) -> uint32_t {
-        const int t = r * KPT + i;
-        if (t >= T) return 0u;
-        const float m = p.mass[ub + t];
-        float x;
-        if (p.alpha == 0.0f) x = m;
-        else x = __fmaf_rn(p.alpha, p.score[ub + t], __fmul_rn(one_minus, m));
-        if (p.score != nullptr) p.score[ub + t] = x;
-        return ordered_key(x);
-    };
-    uint32_t key[KR];
-    #pragma unroll
-    for (int i = 0; i < KR; ++i) key[i] = load_key(i);
-    if constexpr (KS > 0) {
-        for (int i = 0; i < KS; ++i) skeys[i * blockDim.x + r] = load_key(KR + i);
-    }
-    auto skey = [&](int i) -> uint32_t { return skeys[i * blockDim.x + r]; };
-
-    uint32_t *out = p.mask + (size_t)unit * p.nwords;
-    if (p.k <= 0) {
-        for (int wd = r; wd < p.nwords; wd += 32 * NW) out[wd] = 0u;
-        return;
-    }
-
-    // theta = largest x with #{key >= x} >= k  (the k-th largest key)
-    uint32_t theta = 0u;
-    for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t cand = theta | (1u << bit);
-        int c = 0;
-        #pragma unroll
-        for (int i = 0; i < KR; ++i) c += (key[i] >= cand) ? 1 : 0;
-        if constexpr (KS > 0) {
-            #pragma unroll 8
-            for (int i = 0; i < KS; ++i) c += (skey(i) >= cand) ? 1 : 0;
-        }
-        if (group_sum<NW>(c, red) >= p.k) theta = cand;
-    }
-    int gt = 0, eq = 0;
-    #pragma unroll
-    for (int i = 0; i < KR; ++i) {
-        gt += (key[i] > theta) ? 1 : 0;
-        eq += (key[i] == theta) ? 1 : 0;
-    }
-    if constexpr (KS > 0) {
-        for (int i = 0; i < KS; ++i) {
-            const uint32_t kk = skey(i);
-            gt += (kk > theta) ? 1 : 0;
-            eq += (kk == theta) ? 1 : 0;
-        }
-    }
-    const int need = p.k - group_sum<NW>(gt, red);      // equal keys to take, >= 1
-    int before = group_exclusive_scan<NW>(eq, red);     // equal keys at lower token indices
-
-    // bits of this thread's KPT tokens, then whole mask words
+// Mask bits of a thread's KPT consecutive tokens (thread index r of the unit): keys above theta,
+// and the first `need` keys equal to theta in token order (`before` of them precede this
+// thread's).  KPT >= 32: whole words per thread; otherwise the words are shared within a warp.
+template <int KPT>
+__device__ __forceinline__ void write_bits(const uint32_t (&key)[KPT], uint32_t theta, int need, int before, int r,
+                                           uint32_t *out, int nwords) {
     if constexpr (KPT >= 32) {
         #pragma unroll
         for (int wd = 0; wd < KPT / 32; ++wd) {
@@ -176,15 +49,12 @@ __global__ void __launch_bounds__(NW == 1 ? 256 : 32 * NW) select_kernel(Params 
             #pragma unroll
             for (int b = 0; b < 32; ++b) {
                 const int i = wd * 32 + b;
-                uint32_t kk;
-                if (i < KR) kk = key[i < KR ? i : 0];
-                else kk = skey(i - KR);
-                bool s = kk > theta;
-                if (kk == theta) { s = before < need; ++before; }
+                bool s = key[i] > theta;
+                if (key[i] == theta) { s = before < need; ++before; }
                 if (s) bits |= 1u << b;
             }
             const int widx = r * (KPT / 32) + wd;
-            if (widx < p.nwords) out[widx] = bits;
+            if (widx < nwords) out[widx] = bits;
         }
     } else {
         uint32_t bits = 0u;
@@ -198,8 +68,178 @@ __global__ void __launch_bounds__(NW == 1 ? 256 : 32 * NW) select_kernel(Params 
         #pragma unroll
         for (int d = 1; d < share; d <<= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, d);
         const int widx = (r * KPT) >> 5;
-        if ((r % share) == 0 && widx < p.nwords) out[widx] = bits;
+        if ((r % share) == 0 && widx < nwords) out[widx] = bits;
     }
+}
+
+// ------------------------------------------------------------ small T: one warp per unit
+
+template <int KPT>
+__global__ void __launch_bounds__(256) select_warp_kernel(Params p) {
+    const int unit = blockIdx.x * 8 + (threadIdx.x >> 5), r = threadIdx.x & 31;
+    if (unit >= p.n_units) return;          // whole warp leaves together
+    const int T = p.T;
+    const size_t ub = (size_t)unit * T;
+    const float one_minus = __fsub_rn(1.0f, p.alpha);
+    uint32_t key[KPT];
+    #pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+        const int t = r * KPT + i;
+        key[i] = 0u;
+        if (t < T) {
+            const float m = p.mass[ub + t];
+            float x;
+            if (p.alpha == 0.0f) x = m;
+            else x = __fmaf_rn(p.alpha, p.score[ub + t], __fmul_rn(one_minus, m));
+            if (p.score != nullptr) p.score[ub + t] = x;
+            key[i] = ordered_key(x);
+        }
+    }
+    uint32_t *out = p.mask + (size_t)unit * p.nwords;
+    if (p.k <= 0) {
+        for (int wd = r; wd < p.nwords; wd += 32) out[wd] = 0u;
+        return;
+    }
+    // theta = largest x with #{key >= x} >= k  (the k-th largest key)
+    uint32_t theta = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = theta | (1u << bit);
+        int c = 0;
+        #pragma unroll
+        for (int i = 0; i < KPT; ++i) c += (key[i] >= cand) ? 1 : 0;
+        if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= p.k) theta = cand;
+    }
+    int gt = 0, eq = 0;
+    #pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+        gt += (key[i] > theta) ? 1 : 0;
+        eq += (key[i] == theta) ? 1 : 0;
+    }
+    const int need = p.k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);   // equal keys to take, >= 1
+    int incl = eq;
+    #pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, d);
+        if (r >= d) incl += o;
+    }
+    int before = incl - eq;                 // equal keys at lower token indices
+    write_bits<KPT>(key, theta, need, before, r, out, p.nwords);
+}
+
+// ------------------------------------------------------------ large T: a cluster of CTAs per unit
+//
+// The unit's keys are spread over kClusterCtas CTAs of 256 threads (KPT keys per thread, in
+// registers).  Each counting pass sums the CTA's count, stores it into every CTA's shared
+// memory (distributed shared memory) and meets the others at one cluster barrier; the count
+// buffers alternate between passes, so a CTA that runs ahead never overwrites counts another
+// is still reading.  CTA rank order is token order, so the tie scan over CTAs is a prefix of
+// their equal-key counts.
+constexpr int kClusterCtas = 8;
+constexpr int kClusterThreads = 256;
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// store v into word `idx` of the shared array `arr` of the CTA with cluster rank `cta`
+__device__ __forceinline__ void st_cluster(int *arr, int idx, uint32_t cta, int v) {
+    uint32_t local = smem_u32(arr + idx), remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(cta));
+    asm volatile("st.shared::cluster.u32 [%0], %1;" :: "r"(remote), "r"(v) : "memory");
+}
+
+template <int KPT>
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterThreads)
+    select_cluster_kernel(Params p) {
+    __shared__ int red[2][8];
+    __shared__ int counts[2][3][kClusterCtas];   // [parity][count, gt, eq][cta]
+    const uint32_t rank = cluster_rank();
+    const int unit = blockIdx.x / kClusterCtas;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int r = (int)rank * kClusterThreads + tid;   // thread index within the unit
+    const int T = p.T;
+    const size_t ub = (size_t)unit * T;
+    const float one_minus = __fsub_rn(1.0f, p.alpha);
+    uint32_t key[KPT];
+    #pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+        const int t = r * KPT + i;
+        key[i] = 0u;
+        if (t < T) {
+            const float m = p.mass[ub + t];
+            float x;
+            if (p.alpha == 0.0f) x = m;
+            else x = __fmaf_rn(p.alpha, p.score[ub + t], __fmul_rn(one_minus, m));
+            if (p.score != nullptr) p.score[ub + t] = x;
+            key[i] = ordered_key(x);
+        }
+    }
+    uint32_t *out = p.mask + (size_t)unit * p.nwords;
+    if (p.k <= 0) {   // uniform across the cluster: no barrier is skipped by only some CTAs
+        for (int wd = r; wd < p.nwords; wd += kClusterCtas * kClusterThreads) out[wd] = 0u;
+        return;
+    }
+    // sum of v over the cluster's threads (slot c of the parity's buffers), plus, if asked,
+    // the sum over the CTAs of lower rank
+    int par = 0;
+    auto cluster_sum = [&](int v, int slot, int *lower) -> int {
+        v = (int)__reduce_add_sync(0xffffffffu, (unsigned)v);
+        if (lane == 0) red[par][warp] = v;
+        __syncthreads();
+        if (warp == 0) {
+            int s = lane < kClusterThreads / 32 ? red[par][lane] : 0;
+            s = (int)__reduce_add_sync(0xffffffffu, (unsigned)s);
+            if (lane < kClusterCtas) st_cluster(&counts[par][slot][0], (int)rank, (uint32_t)lane, s);
+        }
+        cluster_sync_all();
+        int tot = 0, low = 0;
+        #pragma unroll
+        for (int c = 0; c < kClusterCtas; ++c) {
+            const int x = counts[par][slot][c];
+            tot += x;
+            low += c < (int)rank ? x : 0;
+        }
+        if (lower) *lower = low;
+        par ^= 1;
+        return tot;
+    };
+    uint32_t theta = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = theta | (1u << bit);
+        int c = 0;
+        #pragma unroll
+        for (int i = 0; i < KPT; ++i) c += (key[i] >= cand) ? 1 : 0;
+        if (cluster_sum(c, 0, nullptr) >= p.k) theta = cand;
+    }
+    int gt = 0, eq = 0;
+    #pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+        gt += (key[i] > theta) ? 1 : 0;
+        eq += (key[i] == theta) ? 1 : 0;
+    }
+    const int need = p.k - cluster_sum(gt, 1, nullptr);   // equal keys to take, >= 1
+    // equal keys at lower token indices: CTAs of lower rank, then lower threads of this CTA
+    int low_ctas = 0;
+    int incl = eq;
+    #pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += o;
+    }
+    __shared__ int wsum[kClusterThreads / 32];
+    if (lane == 31) wsum[warp] = incl;
+    cluster_sum(eq, 2, &low_ctas);                         // also orders wsum's writes before the reads
+    int low_warps = 0;
+    for (int w2 = 0; w2 < warp; ++w2) low_warps += wsum[w2];
+    int before = low_ctas + low_warps + incl - eq;
+    write_bits<KPT>(key, theta, need, before, r, out, p.nwords);
+    cluster_sync_all();   // no CTA leaves while another may still store into its shared memory
 }
 
 }  // namespace select

@@ -33,7 +33,7 @@ RANK = 64
 RANK_LO = 16
 NOISE_STD = 0.05
 
-K_VIS, V_VIS, K_TEXT, V_TEXT, QUERY, COEF_K, COEF_V, MASK = range(8)
+K_VIS, V_VIS, K_TEXT, V_TEXT, QUERY, COEF_K, COEF_V, MASK, COEF_TK, COEF_TV = range(10)
 
 
 @dataclass(frozen=True)
@@ -183,11 +183,21 @@ def compressed_unit(w: Workload, layer: int, b: int, g: int, kind: int, T: int =
     B [64, 512] with orthonormal rows.  bf16 bits.  Used where a decode-step input is wanted
     without running a compression first."""
     T = w.T if T is None else T
-    gen = rng(w, layer, b, g, COEF_K if kind == K_VIS else COEF_V)
+    return _coefficients(rng(w, layer, b, g, COEF_K if kind == K_VIS else COEF_V), T)
+
+
+def _coefficients(gen: np.random.Generator, T: int):
     sig = coefficient_sigmas(T)
     C = gen.standard_normal((T, RANK)) * (sig / math.sqrt(T))[None, :]
     B = _orthonormal_columns(gen, FEAT, RANK).T
     return to_bf16_bits(C), to_bf16_bits(B)
+
+
+def text_compressed_unit(w: Workload, layer: int, b: int, g: int, kind: int, L_c: int):
+    """Synthetic compressed text of one unit (the text tokens factored with a basis of their own):
+    coefficients C [L_c, 64] and basis B [64, 512] drawn like compressed_unit's, from their own
+    stream (kind = K_TEXT or V_TEXT).  bf16 bits."""
+    return _coefficients(rng(w, layer, b, g, COEF_TK if kind == K_TEXT else COEF_TV), L_c)
 
 
 def random_mask(w: Workload, layer: int, b: int, g: int, T: int = None, k: int = None, step: int = 0) -> np.ndarray:

@@ -74,6 +74,29 @@ def test_decode_rejects_bad_arguments_before_launch(kv):
     assert _call_decode(kv, _dims(kv), ws_bytes=16) == 4
 
 
+def test_text_basis_decode_rejects_bad_arguments_before_launch(kv):
+    lib = kv.lib()
+    d = _dims(kv)
+    ptr = 0x10000
+
+    def call(tb, ws=None, L_c=None):
+        n = kv.decode_tb_workspace(d, 1, L_c if L_c is not None else (tb.L_c if tb is not None else 0))
+        return lib.kvpack_decode_attn_tb(ctypes.byref(d.c()), 1, *([ptr] * 7), ctypes.byref(tb) if tb else None,
+                                         ptr, ptr, 8, ptr, 1.0, ptr, ptr, ptr, n if ws is None else ws, None)
+
+    TB = kv._lib._CTextBasis
+    assert call(None) == 1                                             # no text basis
+    assert call(TB(ptr, ptr, ptr, ptr, ptr, None, 100)) == 1           # a missing plane
+    assert call(TB(ptr, ptr, ptr, ptr, ptr, ptr + 8, 100)) == 2        # a misaligned plane
+    assert call(TB(ptr, ptr, ptr, ptr, ptr, ptr, -1), ws=1 << 30) == 1
+    assert call(TB(ptr, ptr, ptr, ptr, ptr, ptr, 65537), ws=1 << 30) == 1
+    assert call(TB(ptr, ptr, ptr, ptr, ptr, ptr, 100), ws=16) == 4
+    # the text tokens' own passes need room of their own; none at L_c = 0
+    assert kv.decode_tb_workspace(d, 1, 0) == kv.decode_workspace(d, 1)
+    assert kv.decode_tb_workspace(d, 1, 512) > kv.decode_workspace(d, 1)
+    assert kv.decode_tb_workspace(d, 1, -1) == 0
+
+
 def test_select_rejects_bad_arguments_before_launch(kv):
     lib = kv.lib()
     d = _dims(kv).c()

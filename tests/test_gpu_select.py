@@ -1,6 +1,7 @@
 """GPU top-k rank selection vs the oracle on identical fp32 input: bit-exact,
 including ties (to the lower index), -0 / +0, NaN, k in {0, 1, T}, every size
-regime of the kernel (warp per unit up to T = 2048, block per unit above) and
+regime of the kernel (warp per unit up to T = 2048, a cluster of 8 CTAs per unit above,
+with 1 to 32 keys per thread) and
 the moving-average importance update."""
 import math
 
@@ -39,7 +40,7 @@ def _run(kv, m, k, alpha=0.0, score=None):
     return out.cpu().numpy().view(np.uint32), (sd.cpu().numpy() if sd is not None else None)
 
 
-@pytest.mark.parametrize("T", [1, 7, 31, 32, 33, 576, 1000, 2047, 2048, 2049, 2304, 6272, 20000, 65536])
+@pytest.mark.parametrize("T", [1, 7, 31, 32, 33, 576, 1000, 2047, 2048, 2049, 2304, 4097, 6272, 20000, 32768, 65536])
 def test_select_bit_exact(T):
     import rank_compressed_kv_b200 as kv
     m = _mass(T, T)

@@ -212,3 +212,54 @@ def test_all_rank_zero_without_text_is_uniform_and_zero():
     out, mass = oracle.decode(CK, BK, CV, BV, Kt, Vt, zero, q, r_lo=0)
     assert np.all(out == 0.0)
     np.testing.assert_allclose(mass[0], np.full(T, Hg / T), rtol=1e-14)
+
+
+# ----------------------------------------------------------------- text compressed too
+
+def _text_factors(seed, L, exact_rank=64):
+    """Text K / V of rank <= 64 with exact factors: K = C B, B with orthonormal rows."""
+    g = np.random.default_rng(seed)
+    out = []
+    for _ in range(2):
+        B = np.linalg.qr(g.standard_normal((512, 64)))[0].T
+        C = g.standard_normal((L, 64)) * (np.arange(64) < exact_rank)
+        out += [C[None], B[None]]
+    return out   # CKt, BKt, CVt, BVt
+
+
+def test_text_basis_equals_its_decompressed_tail():
+    """The compressed text tokens act exactly like the uncompressed tokens C B they factor."""
+    CK, BK, CV, BV, Kt, Vt, mask, q, _ = _rand_unit(71, 300, 9, 8)
+    CKt, BKt, CVt, BVt = _text_factors(72, 40)
+    Kd = (CKt[0] @ BKt[0]).reshape(1, 40, 4, 128)
+    Vd = (CVt[0] @ BVt[0]).reshape(1, 40, 4, 128)
+    o1, m1 = oracle.decode_tb(CK, BK, CV, BV, CKt, BKt, CVt, BVt, Kt, Vt, mask, q)
+    o2, m2 = oracle.decode(CK, BK, CV, BV, np.concatenate([Kd, Kt], 1), np.concatenate([Vd, Vt], 1), mask, q)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(m1, m2, rtol=0, atol=1e-15)
+
+
+def test_text_basis_without_text_tokens_is_the_plain_step():
+    CK, BK, CV, BV, Kt, Vt, mask, q, _ = _rand_unit(73, 200, 5, 16)
+    z = np.zeros((1, 0, 64))
+    zb = np.linalg.qr(np.random.default_rng(74).standard_normal((512, 64)))[0].T[None]
+    o1, m1 = oracle.decode_tb(CK, BK, CV, BV, z, zb, z, zb, Kt, Vt, mask, q)
+    o2, m2 = oracle.decode(CK, BK, CV, BV, Kt, Vt, mask, q)
+    assert np.array_equal(o1, o2) and np.array_equal(m1, m2)
+
+
+def test_text_basis_rank_space_route():
+    """Closed form of the text tokens' part: their logits are C_K' (B_K' q) and their value sum
+    (sum p C_V') B_V', so a query orthogonal to every B_K' row gives them logit 0."""
+    CK, BK, CV, BV, Kt, Vt, mask, q, _ = _rand_unit(75, 64, 0, 4)
+    CKt, BKt, CVt, BVt = _text_factors(76, 30)
+    # project the query of every head onto the orthogonal complement of its KV head's text basis slice
+    qq = q.copy()
+    for h in range(4):
+        Bj = BKt[0][:, 128 * h:128 * h + 128]          # Hg = 4: one query head per KV head
+        Pj = np.linalg.qr(Bj.T)[0]                      # orthonormal basis of span(B_j^T) (128 x 64)
+        qq[0, h] -= Pj @ (Pj.T @ qq[0, h])
+    big = 1e3 * np.ones_like(CKt)                        # any coefficients: the logits stay 0
+    o1, _ = oracle.decode_tb(CK, BK, CV, BV, big, BKt, CVt, BVt, Kt, Vt, mask, qq)
+    o2, _ = oracle.decode_tb(CK, BK, CV, BV, 0 * big, BKt, CVt, BVt, Kt, Vt, mask, qq)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-9)
