@@ -435,6 +435,79 @@ def measure_baselines(kv, torch, w, dims, c, mask, q, out, ws, L_text, dev, rank
             "note": "rank-space call also writes the attention mass; the baselines write the output only"}
 
 
+def measure_text_basis(kv, torch, w: synth.Workload, dev, ranks, K: int):
+    """The decode call with the text tokens compressed too (kvpack_decode_attn_tb: the workload's
+    text0 prompt tokens factored with a basis of their own, attended at the full rank, plus one
+    uncompressed generated token) against the same attention with all text0 + 1 text tokens
+    uncompressed (kvpack_decode_attn), on the same visual cache, mask and query.  CUDA events
+    around K calls of each; algorithmic bytes per call for both."""
+    n_layers, T, U, L_c = w.layers, w.T, w.units, w.text0
+    Lcap = L_c + 1
+    dims = kv.Dims(batch=w.batch, n_q_heads=w.n_q, n_kv_heads=w.n_kv, T_vis=T, L_text_cap=Lcap)
+    c = build_cache(kv, torch, w, Lcap, dev)
+    pool = []
+    for i in range(POOL):
+        ck, bk = synth.text_compressed_unit(w, 0, i % w.batch, i % w.groups, synth.K_TEXT, L_c)
+        cv, bv = synth.text_compressed_unit(w, 0, i % w.batch, i % w.groups, synth.V_TEXT, L_c)
+        pool.append((ck, bk, cv, bv))
+
+    def tile(j, sl, shape):
+        arr = np.stack([p[j] if sl is None else p[j][..., sl] for p in pool])
+        src = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).to(dev)
+        idx = torch.arange(U, device=dev) % POOL
+        return src[idx].reshape((U,) + shape).contiguous().view(torch.bfloat16)
+
+    tb = (tile(0, slice(0, 16), (L_c, 16)), tile(0, slice(16, 64), (L_c, 48)), tile(1, None, (64, 512)),
+          tile(2, slice(0, 16), (L_c, 16)), tile(2, slice(16, 64), (L_c, 48)), tile(3, None, (64, 512)), L_c)
+    q = torch.from_numpy(np.stack([synth.query(w, l, b, 1) for l in range(n_layers) for b in range(w.batch)])
+                         .view(np.int16)).view(torch.bfloat16).to(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(77 + w.seed)
+    mask = torch.empty(U, (T + 31) // 32, dtype=torch.int32, device=dev)
+    kv.select(dims, n_layers, torch.rand(U, T, generator=gen, device=dev), None, 0.0, w.k_hi, mask)
+    out = torch.empty(n_layers * w.batch, w.n_q, 128, dtype=torch.bfloat16, device=dev)
+    mass = torch.empty(U, T, dtype=torch.float32, device=dev)
+    ws_plain = torch.empty(kv.decode_workspace(dims, n_layers), dtype=torch.uint8, device=dev)
+    ws_tb = torch.empty(kv.decode_tb_workspace(dims, n_layers, L_c), dtype=torch.uint8, device=dev)
+
+    def plain():
+        kv.decode_attn(dims, n_layers, q, c["CK_lo"], c["CK_hi"], c["BK"], c["CV_lo"], c["CV_hi"], c["BV"],
+                       c["K_text"], c["V_text"], L_c + 1, mask, 1.0, out, mass, ws_plain)
+
+    def compressed_text():
+        kv.decode_attn_tb(dims, n_layers, q, c["CK_lo"], c["CK_hi"], c["BK"], c["CV_lo"], c["CV_hi"], c["BV"], tb,
+                          c["K_text"], c["V_text"], 1, mask, 1.0, out, mass, ws_tb)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ranks.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms, = ranks.max(e0.elapsed_time(e1) / K)
+        return ms
+
+    p_ms = timed(plain)
+    t_ms = timed(compressed_text)
+    st = kv.last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {kv.STATUS_NAMES[st]} in the text-basis leg ({w.name})")
+    plain_bytes = decode_bytes(w, L_c + 1, w.k_hi)
+    tb_bytes = plain_bytes - U * L_c * 512 * 2 * 2 + U * (L_c * 64 * 2 * 2 + 2 * 64 * 512 * 2 + ((L_c + 31) // 32) * 4)
+    del c, tb, ws_plain, ws_tb
+    torch.cuda.empty_cache()
+    return {"workload": f"{w.name}: {L_c} prompt text tokens compressed (rank 64, own basis) + 1 generated token",
+            "calls_timed": K, "text_uncompressed_ms": round(p_ms, 4), "text_compressed_ms": round(t_ms, 4),
+            "speedup": round(p_ms / t_ms, 2), "bytes_text_uncompressed": int(plain_bytes),
+            "bytes_text_compressed": int(tb_bytes),
+            "GBps_text_compressed": round(tb_bytes / (t_ms / 1e3) / 1e9, 1)}
+
+
 def roofline_block(w: synth.Workload, L_mean: float, dec_avg_ms: float):
     """Roofline of the dominant call (kvpack_decode_attn): algorithmic bytes per launch over its
     CUDA-event duration, against the measured copy bandwidth."""
@@ -522,6 +595,8 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
         "wall_s_timed": round(res["wall"], 3),
         "baselines": res.get("baselines"),
     }
+    if not args.no_baselines:
+        line["text_basis"] = measure_text_basis(kv, torch, w, dev, ranks, max(10, min(K, args.config_steps)))
     if not args.headline_only:
         # the workloads the HBM-roofline target is set on, measured the same way (device-resident,
         # CUDA events, max over ranks); the headline value above stays the first workload's

@@ -106,6 +106,7 @@ constexpr int kStageRows = 32;          // rows of Y per staged chunk of a 96 x 
 constexpr int kStagePitch = kP + 1;     // staged chunks are stored transposed, padded
 constexpr float kJacTol = 1e-6f;        // rotate when |a_pq| > kJacTol sqrt(|a_pp a_qq|) ...
 constexpr float kJacFloor = 1e-7f;      // ... and |a_pq| > kJacFloor max |a_ii| (fp32 rounding level)
+constexpr float kJacQuad = 1e-3f;       // a sweep whose largest ratio is below this is the last (~sqrt(kJacTol))
 constexpr float kPivTol = 1e-4f;        // Cholesky pivot below this fraction of its diagonal: dependent column
 constexpr float kThetaFloor = 1e-7f;    // Ritz values below this fraction of the largest are taken as zero
 
@@ -126,7 +127,7 @@ struct EigSmem {
     int rot_p[kP / 2], rot_q[kP / 2];
     float rot_c[kP / 2], rot_s[kP / 2];
     float amax;
-    int rotations;
+    float red2[2];
     int done;
     float prev_change;
 };
@@ -300,9 +301,13 @@ __device__ void rowmix(const float *__restrict__ in, const float *M, float *__re
 // Cyclic two-sided Jacobi on the symmetric 96 x 96 matrix A (row-major, both triangles),
 // V = the product of the rotations (A -> V^T A V).  Parallel round-robin order: 48 disjoint
 // pairs per round, 95 rounds per sweep; each 2 x 2 block of A is rotated in place by one
-// thread.  Returns the sweeps used, or -1 after kMaxSweeps without convergence.
+// thread.  The largest relative off-diagonal |a_pq| / sqrt(|a_pp a_qq|) met in a sweep decides
+// the end: none above kJacTol means converged; all below sqrt(kJacTol) means this sweep's
+// rotations leave them near kJacTol (Jacobi converges quadratically), so no further sweep is
+// run.  Returns the sweeps used, or -1 after kMaxSweeps without convergence.
 __device__ int jacobi96(float *A, float *V, EigSmem &sm) {
     const int tid = threadIdx.x, lane = tid & 31;
+    constexpr int kPairs = kP / 2;
     for (int e = tid; e < kP * kP; e += kEigThreads) V[e] = (e / kP == e % kP) ? 1.f : 0.f;
     for (int sweep = 1; sweep <= kMaxSweeps; ++sweep) {
         __syncthreads();
@@ -311,30 +316,32 @@ __device__ int jacobi96(float *A, float *V, EigSmem &sm) {
             for (int i = lane; i < kP; i += 32) m = fmaxf(m, fabsf(A[i * kP + i]));
             #pragma unroll
             for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
-            if (lane == 0) { sm.amax = m; sm.rotations = 0; }
+            if (lane == 0) sm.amax = m;
         }
         __syncthreads();
         const float floor_a = kJacFloor * sm.amax;
+        float worst = 0.f;                      // rotating threads: largest relative off-diagonal seen
         for (int rd = 0; rd < kP - 1; ++rd) {
-            if (tid < kP / 2) {
+            if (tid < kPairs) {
                 const int k = tid;
                 int p, q;
                 if (k == 0) { p = rd; q = kP - 1; }
                 else { p = (rd + k) % (kP - 1); q = (rd - k + kP - 1) % (kP - 1); }
                 const float app = A[p * kP + p], aqq = A[q * kP + q], apq = A[p * kP + q];
                 float c = 1.f, s = 0.f;
-                if (fabsf(apq) > kJacTol * sqrtf(fabsf(app * aqq)) && fabsf(apq) > floor_a) {
+                const float ref = sqrtf(fabsf(app * aqq));
+                if (fabsf(apq) > floor_a) worst = fmaxf(worst, fabsf(apq) / fmaxf(ref, 1e-30f));
+                if (fabsf(apq) > kJacTol * ref && fabsf(apq) > floor_a) {
                     const float zeta = (aqq - app) / (2.f * apq);
                     const float t = copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
                     c = 1.f / sqrtf(1.f + t * t);
                     s = c * t;
-                    atomicAdd(&sm.rotations, 1);
                 }
                 sm.rot_p[k] = p; sm.rot_q[k] = q; sm.rot_c[k] = c; sm.rot_s[k] = s;
             }
             __syncthreads();
-            for (int blk = tid; blk < (kP / 2) * (kP / 2); blk += kEigThreads) {
-                const int a = blk / (kP / 2), b = blk % (kP / 2);
+            for (int blk = tid; blk < kPairs * kPairs; blk += kEigThreads) {
+                const int a = blk / kPairs, b = blk - a * kPairs;
                 const float sa = sm.rot_s[a], sb = sm.rot_s[b];
                 if (sa == 0.f && sb == 0.f) continue;
                 const float ca = sm.rot_c[a], cb = sm.rot_c[b];
@@ -349,8 +356,8 @@ __device__ int jacobi96(float *A, float *V, EigSmem &sm) {
                 A[pa * kP + pb] = z11; A[pa * kP + qb] = z12;
                 A[qa * kP + pb] = z21; A[qa * kP + qb] = z22;
             }
-            for (int e = tid; e < kP * (kP / 2); e += kEigThreads) {
-                const int i = e / (kP / 2), k = e % (kP / 2);
+            for (int e = tid; e < kP * kPairs; e += kEigThreads) {
+                const int i = e / kPairs, k = e - i * kPairs;
                 const float s = sm.rot_s[k];
                 if (s == 0.f) continue;
                 const float c = sm.rot_c[k];
@@ -361,7 +368,16 @@ __device__ int jacobi96(float *A, float *V, EigSmem &sm) {
             }
             __syncthreads();
         }
-        if (sm.rotations == 0) return sweep;
+        // the sweep's largest relative off-diagonal over the 48 rotating threads (warps 0 and 1)
+        if (tid < 64) {
+            float m = worst;
+            #pragma unroll
+            for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
+            if (lane == 0) sm.red2[tid >> 5] = m;
+        }
+        __syncthreads();
+        const float sweep_worst = fmaxf(sm.red2[0], sm.red2[1]);
+        if (sweep_worst <= kJacTol || sweep_worst < kJacQuad) return sweep;
     }
     return -1;
 }
@@ -369,43 +385,65 @@ __device__ int jacobi96(float *A, float *V, EigSmem &sm) {
 // W = R^T R (R upper triangular, written to R; the lower triangle is zeroed).  A holds W on
 // entry and is overwritten by the trailing updates.  A pivot at or below kPivTol of its
 // column's original diagonal marks a dependent (or dead) column: its row of R is zero.
+// Trailing updates: thread (ti, tj) of a 16 x 32 grid takes rows k+1+ti+16m, columns k+1+tj+32n.
 __device__ void cholesky96(float *A, float *R, EigSmem &sm) {
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, ti = tid >> 5, tj = tid & 31;
     if (tid < kP) sm.diag0[tid] = A[tid * kP + tid];
     for (int e = tid; e < kP * kP; e += kEigThreads) R[e] = 0.f;
     __syncthreads();
     for (int k = 0; k < kP; ++k) {
         const float piv = A[k * kP + k];
         const bool ok = piv > kPivTol * sm.diag0[k] && piv > 0.f;
-        const float rk = ok ? sqrtf(piv) : 0.f;
-        const float inv_piv = ok ? 1.f / piv : 0.f;
-        for (int j = k + tid; j < kP; j += kEigThreads) R[k * kP + j] = ok ? A[k * kP + j] / rk : 0.f;
-        const int n = kP - 1 - k;
-        for (int e = tid; e < n * n; e += kEigThreads) {
-            const int i = k + 1 + e / n, j = k + 1 + e % n;
-            if (j < i) continue;
-            A[i * kP + j] -= A[k * kP + i] * A[k * kP + j] * inv_piv;
+        if (ok) {
+            const float rk = sqrtf(piv), inv_piv = 1.f / piv, inv_rk = 1.f / rk;
+            if (tid >= k && tid < kP) R[k * kP + tid] = tid == k ? rk : A[k * kP + tid] * inv_rk;
+            for (int i = k + 1 + ti; i < kP; i += 16) {
+                const float aki = A[k * kP + i] * inv_piv;
+                for (int j = i + ((tj - (i - k - 1)) & 31); j < kP; j += 32) {
+                    // columns j >= i of row i, each thread a fixed residue of j - (k + 1) mod 32
+                    A[i * kP + j] -= aki * A[k * kP + j];
+                }
+            }
         }
         __syncthreads();
     }
 }
 
 // X = R^-1 for the upper-triangular R of cholesky96 (a zero row of R gives a zero row and
-// column of X), computed bottom-up: X_ii = 1 / R_ii, X_ij = -(sum_{i<k<=j} R_ik X_kj) / R_ii.
-// Four threads share each column's sum.
-__device__ void tri_inverse96(const float *R, float *X) {
-    const int tid = threadIdx.x;
+// column of X), by 16 x 16 blocks: the six diagonal blocks are inverted by back substitution,
+// one warp each, a column per lane; then, block row by block row from the bottom,
+// X_IJ = -X_II (sum_{I<K<=J} R_IK X_KJ) for every J > I at once.
+__device__ void tri_inverse96(const float *R, float *X, float *T) {
+    constexpr int kB = 16, kNB = kP / kB;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     for (int e = tid; e < kP * kP; e += kEigThreads) X[e] = 0.f;
     __syncthreads();
-    const int j = tid >> 2, part = tid & 3;     // 384 threads: 96 columns x 4
-    for (int i = kP - 1; i >= 0; --i) {
-        if (j < kP) {                            // whole warps (threads 0 .. 383)
-            float s = 0.f;
-            for (int k = i + 1 + part; k <= j; k += 4) s = fmaf(R[i * kP + k], X[k * kP + j], s);
-            s += __shfl_xor_sync(0xffffffffu, s, 1);
-            s += __shfl_xor_sync(0xffffffffu, s, 2);
+    if (warp < kNB && lane < kB) {
+        const int o = warp * kB, j = o + lane;
+        for (int i = j; i >= o; --i) {
             const float rii = R[i * kP + i];
-            if (part == 0 && j >= i) X[i * kP + j] = rii > 0.f ? (j == i ? 1.f / rii : -s / rii) : 0.f;
+            float sum = i == j ? 1.f : 0.f;
+            for (int k = i + 1; k <= j; ++k) sum = fmaf(-R[i * kP + k], X[k * kP + j], sum);
+            X[i * kP + j] = rii > 0.f ? sum / rii : 0.f;
+        }
+    }
+    __syncthreads();
+    for (int I = kNB - 2; I >= 0; --I) {
+        const int oI = I * kB, ncol = kP - (oI + kB);        // columns right of the diagonal block
+        // T = R[I rows, (I, J] ] X[(I, J], J cols] for every column of the blocks right of I
+        for (int e = tid; e < kB * ncol; e += kEigThreads) {
+            const int i = e / ncol, jc = oI + kB + (e - (e / ncol) * ncol);
+            const int kend = jc;                               // X[k][jc] = 0 for k > jc
+            float sum = 0.f;
+            for (int k = oI + kB; k <= kend; ++k) sum = fmaf(R[(oI + i) * kP + k], X[k * kP + jc], sum);
+            T[i * kP + jc] = sum;
+        }
+        __syncthreads();
+        for (int e = tid; e < kB * ncol; e += kEigThreads) {
+            const int i = e / ncol, jc = oI + kB + (e - (e / ncol) * ncol);
+            float sum = 0.f;
+            for (int k = i; k < kB; ++k) sum = fmaf(X[(oI + i) * kP + oI + k], T[k * kP + jc], sum);
+            X[(oI + i) * kP + jc] = -sum;
         }
         __syncthreads();
     }
@@ -542,7 +580,7 @@ __global__ void __launch_bounds__(kEigThreads, 1) eig_kernel(EigParams p) {
         for (int e = tid; e < kP * kP; e += kEigThreads) wk.A[e] *= sm.scale[e / kP] * sm.scale[e % kP];
         __syncthreads();
         cholesky96(wk.A, wk.V, sm);
-        tri_inverse96(wk.V, wk.M);
+        tri_inverse96(wk.V, wk.M, wk.A);
         for (int e = tid; e < kP * kP; e += kEigThreads) wk.M[e] *= sm.scale[e / kP];
         __syncthreads();
         rowmix(zsrc, wk.M, Qt, Qgu, nullptr);

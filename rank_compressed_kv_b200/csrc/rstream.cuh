@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
         // meaningful while its phase is the slot's latest, so on the K ring the slot that carried
         // the end marker (whose tile was consumed before the marker could be written) is skipped.
         cp_async_wait_all();
-        const uint32_t kfirst = seq > (uint32_t)kNK ? seq - kNK + (ended ? 1u : 0u) : 0u;
+        const uint32_t kfirst = seq >= (uint32_t)kNK ? seq - kNK + (ended ? 1u : 0u) : 0u;
         for (uint32_t k = kfirst; k < seq; ++k) {
             const long long t0 = clock64();
             while (!mbar_try_wait(&sm.kfull[k % kNK], (k / kNK) & 1u) && clock64() - t0 < kWaitCycles) {}
