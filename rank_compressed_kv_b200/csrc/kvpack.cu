@@ -174,8 +174,8 @@ cudaError_t launch_rs(int NH, const rs::Params &rp, int grid, cudaStream_t st) {
 // block (many units) or one KV head per block (few units)
 template <int PK>
 cudaError_t launch_finish_pk(const rs::FinishParams &fp, int units, int sms, cudaStream_t st) {
-    if (units >= 2 * sms) return launch_pdl(rs::finish_kernel<PK, 4>, units, 512, 0, st, fp);
-    return launch_pdl(rs::finish_kernel<PK, 1>, units * 4, 128, 0, st, fp);
+    if (units >= 2 * sms) return launch_pdl(rs::finish_kernel<PK, 4>, units, 256, 0, st, fp);
+    return launch_pdl(rs::finish_kernel<PK, 1>, units * 4, 64, 0, st, fp);
 }
 cudaError_t launch_finish(int per_kv, const rs::FinishParams &fp, int units, int sms, cudaStream_t st) {
     switch (per_kv) {
@@ -284,6 +284,12 @@ cudaError_t launch_select_warp(const kvpack::select::Params &p, cudaStream_t st)
 }
 
 template <int KPT>
+cudaError_t launch_select_block(const kvpack::select::Params &p, cudaStream_t st) {
+    kvpack::select::select_block_kernel<KPT><<<p.n_units, kvpack::select::kBlockThreads, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <int KPT>
 cudaError_t launch_select_cluster(const kvpack::select::Params &p, cudaStream_t st) {
     namespace sl = kvpack::select;
     sl::select_cluster_kernel<KPT><<<p.n_units * sl::kClusterCtas, sl::kClusterThreads, 0, st>>>(p);
@@ -381,7 +387,12 @@ kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t
 
     const int T = d->T_vis, Hg = pl.Hg, per_kv = d->n_q_heads / d->n_kv_heads;
     const int groups = d->n_kv_heads / KVPACK_GROUP;
-    const int Sc = (L_text + kTextChunk - 1) / kTextChunk;
+    // text chunks: 64 tokens, doubled (up to 1024) while the items would still fill the GPU twice
+    // over (148 SMs x 8 warps), so that a long tail on few units keeps many items and a short tail
+    // on many units writes one partial per (unit, KV head)
+    int ct = kTextChunk;
+    while (ct < 1024 && (long long)pl.units * 4 * ((L_text + 2 * ct - 1) / (2 * ct)) >= 2LL * kPlanSMs * 8 * 2) ct <<= 1;
+    const int Sc = (L_text + ct - 1) / ct;
     const float scale2 = softmax_scale * 1.4426950408889634f;
     unsigned char *w = static_cast<unsigned char *>(ws);
     unsigned char *qt = w + pl.off_qt;
@@ -424,7 +435,7 @@ kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t
         }
         tp.q = q; tp.part = tpart; tp.qt = qt; tp.qt2 = qt2; tp.counter = counter;
         tp.n_units = pl.units; tp.L = L_text; tp.Hg = Hg; tp.per_kv = per_kv; tp.n_q = d->n_q_heads;
-        tp.groups = groups; tp.Sc = Sc; tp.ct = kTextChunk; tp.n_qitems = pl.units * 4 * (L_c > 0 ? 2 : 1);
+        tp.groups = groups; tp.Sc = Sc; tp.ct = ct; tp.n_qitems = pl.units * 4 * (L_c > 0 ? 2 : 1);
         tp.n_items = tp.n_qitems + pl.units * 4 * Sc; tp.scale2 = scale2;
         const int grid = tp.n_items < di->sms ? tp.n_items : di->sms;
         dc::text::text_kernel<<<grid, dc::text::kThreads, dc::text::smem_bytes(), st>>>(tp);
@@ -736,6 +747,11 @@ kvpack_status kvpack_select(const kvpack_dims *d, int32_t n_layers, const float 
             case 32: e = launch_select_warp<32>(p, st); break;
             default: e = launch_select_warp<64>(p, st); break;
         }
+    } else if (T <= sl::kBlockThreads * 32) {
+        int kpt = 16;
+        while (sl::kBlockThreads * kpt < T) kpt <<= 1;
+        if (kpt == 16) e = launch_select_block<16>(p, st);
+        else e = launch_select_block<32>(p, st);
     } else {
         int kpt = 1;
         while (sl::kClusterCtas * sl::kClusterThreads * kpt < T) kpt <<= 1;

@@ -53,8 +53,12 @@ namespace kvpack {
 namespace decode {
 namespace rs {
 
-constexpr int kWarps = 6;
+constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
+constexpr int kGatherWarp = 6;              // warps 6 and 7 gather the full-rank tokens' rows
+constexpr int kGatherThreads = 64;
+constexpr int kND = 12;                     // descriptor ring (written by the producer, freed by the consumers)
+constexpr int kNQ = 4;                      // queue of full-rank tiles handed to the gather warp
 constexpr int kTile = 128;          // tokens per tensor-memory tile (M of the score MMA)
 constexpr int kHiRing = 1024;       // producer's queue of pending full-rank token positions
 constexpr int kMaskWin = 1024;      // producer's window of mask words (32768 tokens)
@@ -117,13 +121,14 @@ struct Smem {
     alignas(1024) unsigned char kslot[C::kNK][C::kKBytes];
     alignas(1024) unsigned char vslot[C::kNV][VALUE ? C::kVBytes : 16];   // follows the K slots (see Cfg)
     alignas(1024) unsigned char qbuf[2][2][C::kNHP * 128];          // [q slot][hi, lo][rows of 128 B]
-    int kdesc[C::kNK][kDescInts];                                   // written by the producer with the K slot
-    int sdesc[C::kNS][kDescInts];                                   // copied by the MMA warp for the consumers
+    int kdesc[kND][kDescInts];                                      // tile descriptors, written once by the producer
+    int hiq[kNQ][8];                                                // full-rank tiles for the gather warp
     uint32_t mwin[kMaskWin];                                        // producer's window of the CTA's mask words
     uint16_t hi_ring[kHiRing];
     unsigned char pbuf[VALUE ? 4 : 1][VALUE ? 32 * C::kPH * 2 : 16];   // value pass: P rows of each consumer warp
     float merge[VALUE ? 3 : 4][VALUE ? NH * 64 : NH * 2];           // partial merge across the consumer warps
     uint64_t kfull[C::kNK], kempty[C::kNK], vfull[C::kNV], vempty[C::kNV], sfull[C::kNS], sfree[C::kNS];
+    uint64_t dfree[kND], gready[kNQ], gfree[kNQ];
     uint64_t qfull[2], qempty[2], mdone;
     uint32_t tmem_base;
     int abort;
@@ -202,13 +207,19 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
     const long long x0 = tile_begin(blockIdx.x, CT, NT), x1 = tile_begin(blockIdx.x + 1, CT, NT);
 
     if (threadIdx.x == 0) {
+        // data slots complete with the producer's 32 lanes and the gather warps' 64 threads
         for (int s = 0; s < kNK; ++s) {
-            mbar_init(&sm.kfull[s], 32);
+            mbar_init(&sm.kfull[s], 32 + kGatherThreads);
             mbar_init(&sm.kempty[s], 1);
         }
         for (int s = 0; s < kNV; ++s) {
-            mbar_init(&sm.vfull[s], 32);
+            mbar_init(&sm.vfull[s], 32 + kGatherThreads);
             mbar_init(&sm.vempty[s], 4);
+        }
+        for (int s = 0; s < kND; ++s) mbar_init(&sm.dfree[s], 4);
+        for (int s = 0; s < kNQ; ++s) {
+            mbar_init(&sm.gready[s], 1);
+            mbar_init(&sm.gfree[s], kGatherThreads);
         }
         for (int s = 0; s < kNS; ++s) {
             mbar_init(&sm.sfull[s], 1);
@@ -265,21 +276,22 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             }
             return sm.mwin + (gw - wbase);
         };
-        // 128-byte rows (C_lo + C_hi, 16-byte chunk c of row r at c ^ (r & 7)) of the listed tokens;
-        // rows past n are zero-filled when `zero` (their p is zero, and 0 * stale data must stay 0)
-        auto gather = [&](unsigned char *dst, const uint16_t *lo, const uint16_t *hi, const uint16_t *pos, int n,
-                          size_t ubase, bool zero) {
-            #pragma unroll 4
-            for (int k = 0; k < C::kHiTok * 8 / 32; ++k) {
-                const int idx = lane + 32 * k;
-                const int r = idx >> 3, ch = idx & 7;
-                const bool valid = r < n;
-                const size_t row = ubase + pos[r];
-                const uint16_t *src = ch < 2 ? lo + row * 16 + ch * 8 : hi + row * 48 + (ch - 2) * 8;
-                unsigned char *d = dst + r * 128 + ((ch ^ (r & 7)) << 4);
-                if (zero) cp_async16_zfill(d, src, valid);
-                else if (valid) cp_async16(d, src);
+        // wait until descriptor ds of tile `seq` may be rewritten (the consumers are done with it)
+        auto acquire_d = [&](int ds) -> bool {
+            return seq < (uint32_t)kND || mbar_wait(&sm.dfree[ds], ((seq / kND) - 1) & 1u, abort);
+        };
+        // hand a full-rank tile (K slot ks, V slot vs, descriptor ds) to the gather warp; ks < 0 ends it
+        uint32_t hseq = 0;
+        auto push_gather = [&](int ks, int vs, int ds, int n, int unit) -> bool {
+            const int hq = hseq % kNQ;
+            if (hseq >= (uint32_t)kNQ && !mbar_wait(&sm.gfree[hq], ((hseq / kNQ) - 1) & 1u, abort)) return false;
+            if (lane == 0) {
+                int *e = sm.hiq[hq];
+                e[0] = ks; e[1] = vs; e[2] = ds; e[3] = n; e[4] = unit;
+                mbar_arrive(&sm.gready[hq]);
             }
+            ++hseq;
+            return true;
         };
         long long x = x0;
         while (ok && x < x1) {
@@ -338,51 +350,48 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 const int hi_now = (int)(pend / C::kHiTok) + ((final_blk && (pend % C::kHiTok) != 0) ? 1 : 0);
                 if (nhi < n) {
                     // ------------------------------------------------ LO tile
-                    const int ks = seq % kNK;
-                    if (!acquire_k(ks)) { ok = false; break; }
-                    int *d = sm.kdesc[ks];
+                    const int ks = seq % kNK, ds = seq % kND, vs = seq % kNV;
+                    if (!acquire_k(ks) || !acquire_d(ds) || (VALUE && !acquire_v(vs))) { ok = false; break; }
+                    int *d = sm.kdesc[ds];
                     if (lane == 0) {
                         d[0] = kTypeLo | (first ? kFlagFirst : 0) | ((final_blk && hi_now == 0) ? kFlagLast : 0);
                         d[1] = unit; d[2] = tok; d[3] = n; d[4] = pslot; d[5] = qs;
                     }
                     if (lane < C::kLoTok / 32) d[8 + lane] = (int)wd;
                     first = false;
+                    __syncwarp();
+                    // lane 0 issues the copies and arrives for itself and for the gather warp's
+                    // lanes (which have nothing to add to a LO tile); the other lanes' arrivals
+                    // release their descriptor writes
                     const int nb = (n + 255) >> 8;   // 256-row boxes of 32-byte rows
-                    if (!p.rank0) {
-                        if (lane == 0) {
+                    if (lane == 0) {
+                        if (!p.rank0) {
                             fence_proxy_async();
                             mbar_arrive_tx(&sm.kfull[ks], (uint32_t)nb * 8192u);
                             for (int b = 0; b < nb; ++b)
                                 tma_3d(sm.kslot[ks] + 8192 * b, &p.tm_ck, 0, tok + 256 * b, unit, &sm.kfull[ks]);
-                        } else {
-                            mbar_arrive(&sm.kfull[ks]);
-                        }
-                    } else {
-                        mbar_arrive(&sm.kfull[ks]);
-                    }
-                    if (VALUE) {
-                        const int vs = seq % kNV;
-                        if (!acquire_v(vs)) { ok = false; break; }
-                        if (!p.rank0) {
-                            if (lane == 0) {
-                                fence_proxy_async();
+                            if (VALUE) {
                                 mbar_arrive_tx(&sm.vfull[vs], 8192u);
                                 tma_3d(sm.vslot[vs], &p.tm_cv, 0, tok, unit, &sm.vfull[vs]);
-                            } else {
-                                mbar_arrive(&sm.vfull[vs]);
                             }
                         } else {
-                            mbar_arrive(&sm.vfull[vs]);
+                            mbar_arrive(&sm.kfull[ks]);
+                            if (VALUE) mbar_arrive(&sm.vfull[vs]);
                         }
+                        mbar_arrive_cnt(&sm.kfull[ks], kGatherThreads);
+                        if (VALUE) mbar_arrive_cnt(&sm.vfull[vs], kGatherThreads);
+                    } else {
+                        mbar_arrive(&sm.kfull[ks]);
+                        if (VALUE) mbar_arrive(&sm.vfull[vs]);
                     }
                     ++seq;
                 }
                 for (int i = 0; i < hi_now && ok; ++i) {
-                    // ------------------------------------------------ HI tile
-                    const int ks = seq % kNK;
-                    if (!acquire_k(ks)) { ok = false; break; }
+                    // ------------------------------------------------ HI tile: positions here, rows by the gather warp
+                    const int ks = seq % kNK, ds = seq % kND, vs = seq % kNV;
+                    if (!acquire_k(ks) || !acquire_d(ds) || (VALUE && !acquire_v(vs))) { ok = false; break; }
                     const int nh = (int)min((unsigned)C::kHiTok, hi_tail - hi_head);
-                    int *d = sm.kdesc[ks];
+                    int *d = sm.kdesc[ds];
                     uint16_t *pos = reinterpret_cast<uint16_t *>(d + 8);
                     if (lane == 0) {
                         d[0] = kTypeHi | (first ? kFlagFirst : 0) | ((final_blk && i == hi_now - 1) ? kFlagLast : 0);
@@ -395,39 +404,32 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                     }
                     first = false;
                     __syncwarp();
-                    gather(sm.kslot[ks], p.CK_lo, p.CK_hi, pos, nh, ubase, false);
-                    cp_async_arrive(&sm.kfull[ks]);   // raises the pending count; arrives when the copies land
+                    if (!push_gather(ks, vs, ds, nh, unit)) { ok = false; break; }
                     mbar_arrive(&sm.kfull[ks]);       // releases this lane's descriptor writes
-                    if (VALUE) {
-                        const int vs = seq % kNV;
-                        if (!acquire_v(vs)) { ok = false; break; }
-                        gather(sm.vslot[vs], p.CV_lo, p.CV_hi, pos, nh, ubase, true);
-                        cp_async_arrive(&sm.vfull[vs]);
-                        mbar_arrive(&sm.vfull[vs]);
-                    }
+                    if (VALUE) mbar_arrive(&sm.vfull[vs]);
                     hi_head += (unsigned)nh;
                     ++seq;
                 }
             }
         }
-        // end marker (K ring only: the MMA warp passes it on to the consumers)
+        // end markers: the K ring's (the MMA warp passes it on to the consumers) and the gather warp's
         bool ended = false;
         if (ok) {
-            const int ks = seq % kNK;
-            if (acquire_k(ks)) {
-                if (lane == 0) sm.kdesc[ks][0] = kTypeEnd;
+            const int ks = seq % kNK, ds = seq % kND;
+            if (acquire_k(ks) && acquire_d(ds)) {
+                if (lane == 0) sm.kdesc[ds][0] = kTypeEnd;
+                __syncwarp();
                 mbar_arrive(&sm.kfull[ks]);
-                ended = true;
-            } else {
-                ok = false;
+                if (lane == 0) mbar_arrive_cnt(&sm.kfull[ks], kGatherThreads);
+                ended = push_gather(-1, 0, 0, 0, 0);
             }
+            ok = ended;
         }
         if (!ok) *abort = 1;
         // Copies still in flight (possible only when a role gave up) must land before the block
         // exits: wait for the data phases of the last tiles of each ring.  A parity wait is only
         // meaningful while its phase is the slot's latest, so on the K ring the slot that carried
         // the end marker (whose tile was consumed before the marker could be written) is skipped.
-        cp_async_wait_all();
         const uint32_t kfirst = seq >= (uint32_t)kNK ? seq - kNK + (ended ? 1u : 0u) : 0u;
         for (uint32_t k = kfirst; k < seq; ++k) {
             const long long t0 = clock64();
@@ -439,29 +441,76 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 while (!mbar_try_wait(&sm.vfull[k % kNV], (k / kNV) & 1u) && clock64() - t0 < kWaitCycles) {}
             }
         }
+    } else if (warp >= kGatherWarp) {
+        // =============================================================== gather warps
+        // 128-byte rows (C_lo + C_hi, 16-byte chunk c of row r at c ^ (r & 7)) of a HI tile's
+        // tokens into its K slot (and V slot); V rows past n are zero-filled (their p is zero, and
+        // 0 * stale data must stay 0).  Thread g copies chunk g % 8 of rows g / 8 + 8 i, so its
+        // source column and its swizzled destination column are fixed.
+        const int g = threadIdx.x - kGatherWarp * 32, ch = g & 7, r0 = g >> 3;
+        const int dcol = (ch ^ (r0 & 7)) << 4;
+        auto gather = [&](unsigned char *dst, const uint16_t *lo, const uint16_t *hi, const uint16_t *pos, int n,
+                          size_t ubase, bool zero) {
+            const uint16_t *base = ch < 2 ? lo + ch * 8 : hi + (ch - 2) * 8;
+            const int stride = ch < 2 ? 16 : 48;
+            #pragma unroll 4
+            for (int r = r0; r < C::kHiTok; r += kGatherThreads / 8) {
+                const bool valid = r < n;
+                const uint16_t *src = base + (ubase + pos[r]) * stride;
+                unsigned char *dp = dst + r * 128 + dcol;
+                if (zero) cp_async16_zfill(dp, src, valid);
+                else if (valid) cp_async16(dp, src);
+            }
+        };
+        uint32_t h = 0;
+        while (true) {
+            const int hq = h % kNQ;
+            if (!mbar_wait(&sm.gready[hq], (h / kNQ) & 1u, abort)) break;
+            const int *e = sm.hiq[hq];
+            const int ks = e[0], vs = e[1], ds = e[2], n = e[3], unit = e[4];
+            mbar_arrive(&sm.gfree[hq]);
+            if (ks < 0) break;
+            // the positions stay valid until the consumers free the descriptor, which needs this
+            // tile's data first
+            const uint16_t *pos = reinterpret_cast<const uint16_t *>(sm.kdesc[ds] + 8);
+            const size_t ubase = (size_t)unit * p.T;
+            gather(sm.kslot[ks], p.CK_lo, p.CK_hi, pos, n, ubase, false);
+            cp_async_arrive(&sm.kfull[ks]);   // raises the pending count; arrives when the copies land
+            mbar_arrive(&sm.kfull[ks]);
+            if (VALUE) {
+                gather(sm.vslot[vs], p.CV_lo, p.CV_hi, pos, n, ubase, true);
+                cp_async_arrive(&sm.vfull[vs]);
+                mbar_arrive(&sm.vfull[vs]);
+            }
+            ++h;
+        }
+        cp_async_wait_all();
     } else if (warp == 1) {
         // =============================================================== MMA issuer
         if (lane == 0) {
             uint32_t seq = 0, qseq = 0;
             bool issued = false;
             const uint32_t id_s = idesc_bf16_kk(128, kNHP);
+            // shared-memory descriptors, formed once: K slot 0 as a LO operand (32-byte rows) and as a
+            // HI operand (128-byte rows), and the q~ planes of q slot 0; a slot, q slot, sub-tile or
+            // k-step moves the start address, the low field of the descriptor (address / 16)
+            const uint64_t dlo0 = desc_kmajor(smem_u32(sm.kslot[0]), 256u, 6u);
+            const uint64_t dhi0 = desc_kmajor(smem_u32(sm.kslot[0]), 1024u, 2u);
+            const uint64_t dqh0 = desc_kmajor(smem_u32(&sm.qbuf[0][0][0]), 1024u, 2u);
+            const uint64_t dql0 = desc_kmajor(smem_u32(&sm.qbuf[0][1][0]), 1024u, 2u);
+            constexpr uint32_t kSlotStep = C::kKBytes >> 4, kQStep = (2 * C::kNHP * 128) >> 4;
             while (true) {
                 const int ks = seq % kNK, sb = seq % kNS;
                 if (!mbar_wait(&sm.kfull[ks], (seq / kNK) & 1u, abort)) break;
-                // the S buffer (scores and descriptor) of the tile kNS back must have been read
+                // the S buffer of the tile kNS back must have been read
                 if (seq >= (uint32_t)kNS && !mbar_wait(&sm.sfree[sb], ((seq / kNS) - 1) & 1u, abort)) break;
-                // the descriptor moves on with the scores: the K slot is released by the MMA's completion
-                const int *d = sm.kdesc[ks];
-                int *sd = sm.sdesc[sb];
+                const int *d = sm.kdesc[seq % kND];
                 const int hdr = d[0];
                 const int type = hdr & 0xff;
                 if (type == kTypeEnd) {
-                    sd[0] = kTypeEnd;
                     mbar_arrive(&sm.sfull[sb]);
                     break;
                 }
-                #pragma unroll 8
-                for (int i = 0; i < kDescInts; ++i) sd[i] = d[i];
                 const int qs = d[5], n = d[3];
                 if (hdr & kFlagFirst) {
                     if (!mbar_wait(&sm.qfull[qs], (qseq >> 1) & 1u, abort)) break;
@@ -472,20 +521,22 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                     if (type == kTypeHi) fence_proxy_async();   // the gathered rows were written by cp.async
                     tmem_fence_after();
                     const uint32_t dcol = tmem + (uint32_t)(sb * C::kSCols);
-                    const uint32_t qh = smem_u32(&sm.qbuf[qs][0][0]), ql = smem_u32(&sm.qbuf[qs][1][0]);
-                    const uint32_t kb = smem_u32(sm.kslot[ks]);
+                    const uint64_t qh = dqh0 + (uint64_t)(qs * kQStep), ql = dql0 + (uint64_t)(qs * kQStep);
                     if (type == kTypeLo) {
-                        for (int sub = 0; sub * kTile < n; ++sub) {
-                            const uint64_t a = desc_kmajor(kb + 4096u * sub, 256u, 6u);
-                            umma_bf16(dcol + sub * kNHP, a, desc_kmajor(qh, 1024u, 2u), id_s, 0u);
-                            umma_bf16(dcol + sub * kNHP, a, desc_kmajor(ql, 1024u, 2u), id_s, 1u);
-                        }
+                        const uint64_t a0 = dlo0 + (uint64_t)(ks * kSlotStep);
+                        // the q~ hi products of all sub-tiles first (independent accumulators), then
+                        // the lo products that add into them
+                        const int nsub = (n + kTile - 1) / kTile;
+                        for (int sub = 0; sub < nsub; ++sub)
+                            umma_bf16(dcol + sub * kNHP, a0 + (uint64_t)(sub * (4096 >> 4)), qh, id_s, 0u);
+                        for (int sub = 0; sub < nsub; ++sub)
+                            umma_bf16(dcol + sub * kNHP, a0 + (uint64_t)(sub * (4096 >> 4)), ql, id_s, 1u);
                     } else {
+                        const uint64_t a0 = dhi0 + (uint64_t)(ks * kSlotStep);
                         #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            const uint64_t a = desc_kmajor(kb + 32u * k, 1024u, 2u);
-                            umma_bf16(dcol, a, desc_kmajor(qh + 32u * k, 1024u, 2u), id_s, k > 0 ? 1u : 0u);
-                            umma_bf16(dcol, a, desc_kmajor(ql + 32u * k, 1024u, 2u), id_s, 1u);
+                            umma_bf16(dcol, a0 + 2u * k, qh + 2u * k, id_s, k > 0 ? 1u : 0u);
+                            umma_bf16(dcol, a0 + 2u * k, ql + 2u * k, id_s, 1u);
                         }
                     }
                     umma_commit(&sm.sfull[sb]);
@@ -526,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             const int sb = seq % kNS, vs = seq % kNV;
             if (!mbar_wait(&sm.sfull[sb], (seq / kNS) & 1u, abort)) break;
             tmem_fence_after();
-            const int *d = sm.sdesc[sb];
+            const int *d = sm.kdesc[seq % kND];
             const int hdr = d[0];
             const int type = hdr & 0xff;
             if (type == kTypeEnd) break;
@@ -705,7 +756,10 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             }
             tmem_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.sfree[sb]);
+            if (lane == 0) {
+                mbar_arrive(&sm.sfree[sb]);
+                mbar_arrive(&sm.dfree[seq % kND]);
+            }
 
             if (hdr & kFlagLast) {
                 // ---------------------------------------------------------- the segment's partial
@@ -849,33 +903,57 @@ struct FinishParams {
     long long ntiles;
 };
 
-// One block per (unit, JPB KV heads), 128 threads per KV head j: u_h = the sum of the unit's
-// segment partials, w_h = the text chunks' sums weighted by 2^(m_c - M_h), then
-// o_h = (u_h B_V[:, 128 j ..] + u2_h B_V2[:, 128 j ..] + w_h) / L_h for the PK query heads of
-// each KV head (u2, B_V2: the text tokens' own rank space, when the text is compressed), thread t
-// owning output feature t % 128 of KV head j0 + t / 128.  The loads of each stage are
-// independent of one another (the chunk weights are computed once into shared memory first),
-// so they are all in flight at once.  JPB = 4 (a whole unit per block) when units are many,
-// 1 when few, so that the launch fills the GPU either way.
+// One block per (unit, JPB KV heads), two warps per KV head j.  Thread (g, f) of a KV head owns
+// output features 8f .. 8f+7 (f < 16) and rank group g < 4 (ranks 16g .. 16g+15, and the text
+// chunks c = g mod 4): u_h = the sum of the unit's segment partials, w_h = the text chunks' sums
+// weighted by 2^(m_c - M_h), then
+//   o_h = (u_h B_V[:, 128 j ..] + u2_h B_V2[:, 128 j ..] + w_h) / L_h
+// for the PK query heads of the KV head (u2, B_V2: the text tokens' own rank space, when the
+// text is compressed).  B_V rows are read 16 bytes at a time and issued first; the four rank
+// groups' sums meet through a shuffle (the two groups of a warp) and shared memory (the two
+// warps).  JPB = 4 (a whole unit per block) when units are many, 1 when few, so that the launch
+// fills the GPU either way.
 constexpr int kFinishMaxChunks = 64;   // text chunks whose weights are staged; longer tails loop
 
+template <int PK>
+__device__ __forceinline__ void finish_project(const uint16_t *__restrict__ bv, const float (*uf)[64], int hb, int rg,
+                                               float (&acc)[PK][8]) {
+    uint4 raw[16];
+    #pragma unroll
+    for (int i = 0; i < 16; ++i) raw[i] = __ldcs(reinterpret_cast<const uint4 *>(bv + (size_t)(16 * rg + i) * 512));
+    #pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+        float b[8];
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            b[2 * e] = __uint_as_float(w[e] << 16);
+            b[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+        }
+        #pragma unroll
+        for (int hh = 0; hh < PK; ++hh) {
+            const float u = uf[hb + hh][16 * rg + i];
+            #pragma unroll
+            for (int f = 0; f < 8; ++f) acc[hh][f] = fmaf(u, b[f], acc[hh][f]);
+        }
+    }
+}
+
 template <int PK, int JPB>
-__global__ void __launch_bounds__(128 * JPB) finish_kernel(const FinishParams p) {
+__global__ void __launch_bounds__(64 * JPB) finish_kernel(const FinishParams p) {
     constexpr int NHB = PK * JPB;           // query heads of the block
     __shared__ float uf[NHB][64];
     __shared__ float uf2[NHB][64];
     __shared__ float ew[NHB][kFinishMaxChunks];
     __shared__ float ms[NHB][2];
+    __shared__ float red[JPB][PK][128];
     griddep_wait();
     constexpr int kBlocksPerUnit = 4 / JPB;
-    const int unit = blockIdx.x / kBlocksPerUnit, tid = threadIdx.x;
-    const int j0 = (blockIdx.x % kBlocksPerUnit) * JPB, jj = tid >> 7, dcol = tid & 127;
+    const int unit = blockIdx.x / kBlocksPerUnit, tid = threadIdx.x, lane = tid & 31;
+    const int j0 = (blockIdx.x % kBlocksPerUnit) * JPB, jj = tid >> 6;
+    const int half = (tid >> 5) & 1, fg = lane & 15, rg = 2 * half + (lane >> 4);
     const int hb0 = j0 * PK;                // first query head of the block (within the unit)
-    // B_V[:, 128 (j0 + jj) + dcol] for all 64 ranks: issued first, used last
-    const uint16_t *bv = p.BV + (size_t)unit * 64 * 512 + 128 * j0 + tid;
-    uint16_t braw[64];
-    #pragma unroll
-    for (int r = 0; r < 64; ++r) braw[r] = __ldcs(bv + (size_t)r * 512);
+    const int hb = jj * PK;                 // this KV head's first query head within the block
     if (tid < NHB) {
         const float2 st = __ldg(reinterpret_cast<const float2 *>(p.ustat + ((size_t)unit * p.Hg + hb0 + tid) * 2));
         ms[tid][0] = st.x;
@@ -883,7 +961,7 @@ __global__ void __launch_bounds__(128 * JPB) finish_kernel(const FinishParams p)
     }
     const long long f = (long long)unit * p.tpu;
     const int ns = (int)(cta_of_tile(f + p.tpu - 1, p.cta_v, p.ntiles) - cta_of_tile(f, p.cta_v, p.ntiles)) + 1;
-    for (int i = tid; i < NHB * 64; i += 128 * JPB) {
+    for (int i = tid; i < NHB * 64; i += 64 * JPB) {
         const int hh = i >> 6, r = i & 63;
         const float *src = p.vpart + ((size_t)unit * p.nslot * p.Hg + hb0 + hh) * 64 + r;
         float a = 0.f;
@@ -893,7 +971,7 @@ __global__ void __launch_bounds__(128 * JPB) finish_kernel(const FinishParams p)
     if (p.vpart2 != nullptr) {
         const long long f2 = (long long)unit * p.tpu2;
         const int ns2 = (int)(cta_of_tile(f2 + p.tpu2 - 1, p.cta_v2, p.ntiles2) - cta_of_tile(f2, p.cta_v2, p.ntiles2)) + 1;
-        for (int i = tid; i < NHB * 64; i += 128 * JPB) {
+        for (int i = tid; i < NHB * 64; i += 64 * JPB) {
             const int hh = i >> 6, r = i & 63;
             const float *src = p.vpart2 + ((size_t)unit * p.nslot2 * p.Hg + hb0 + hh) * 64 + r;
             float a = 0.f;
@@ -902,59 +980,66 @@ __global__ void __launch_bounds__(128 * JPB) finish_kernel(const FinishParams p)
         }
     }
     __syncthreads();
-    float wacc[PK];
+    float acc[PK][8];
     #pragma unroll
-    for (int hh = 0; hh < PK; ++hh) wacc[hh] = 0.f;
+    for (int hh = 0; hh < PK; ++hh)
+        #pragma unroll
+        for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
+    const size_t col = (size_t)unit * 64 * 512 + 128 * (j0 + jj) + 8 * fg;
+    finish_project<PK>(p.BV + col, uf, hb, rg, acc);
+    if (p.BV2 != nullptr) finish_project<PK>(p.BV2 + col, uf2, hb, rg, acc);
     if (p.tpart != nullptr) {
         const float *tp0 = p.tpart + ((size_t)unit * p.Sc * p.Hg + hb0) * kTxtPart;
         for (int c0 = 0; c0 < p.Sc; c0 += kFinishMaxChunks) {
             const int nc = min(kFinishMaxChunks, p.Sc - c0);
-            for (int i = tid; i < NHB * nc; i += 128 * JPB) {
+            __syncthreads();
+            for (int i = tid; i < NHB * nc; i += 64 * JPB) {
                 const int hh = i / nc, c = i % nc;
                 const float mc = __ldcg(tp0 + ((size_t)(c0 + c) * p.Hg + hh) * kTxtPart);
                 ew[hh][c] = mc != -INFINITY ? ex2(mc - ms[hh][0]) : 0.f;
             }
             __syncthreads();
-            #pragma unroll
-            for (int hh = 0; hh < PK; ++hh) {
-                const int hb = jj * PK + hh;
-                const float *tp = tp0 + (size_t)hb * kTxtPart + 2 + dcol;
-                float a0 = 0.f, a1 = 0.f;
-                int c = 0;
-                for (; c + 1 < nc; c += 2) {
-                    a0 = fmaf(__ldcg(tp + (size_t)(c0 + c) * p.Hg * kTxtPart), ew[hb][c], a0);
-                    a1 = fmaf(__ldcg(tp + (size_t)(c0 + c + 1) * p.Hg * kTxtPart), ew[hb][c + 1], a1);
+            for (int c = rg; c < nc; c += 4) {
+                #pragma unroll
+                for (int hh = 0; hh < PK; ++hh) {
+                    const float wgt = ew[hb + hh][c];
+                    const float *src = tp0 + ((size_t)(c0 + c) * p.Hg + hb + hh) * kTxtPart + 2 + 8 * fg;
+                    // rows of kTxtPart = 130 floats: 8-byte aligned, read as float2
+                    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 v = __ldcg(reinterpret_cast<const float2 *>(src) + e);
+                        acc[hh][2 * e] = fmaf(wgt, v.x, acc[hh][2 * e]);
+                        acc[hh][2 * e + 1] = fmaf(wgt, v.y, acc[hh][2 * e + 1]);
+                    }
                 }
-                if (c < nc) a0 = fmaf(__ldcg(tp + (size_t)(c0 + c) * p.Hg * kTxtPart), ew[hb][c], a0);
-                wacc[hh] += a0 + a1;
             }
-            __syncthreads();
         }
     }
-    float acc[PK];
+    // the four rank groups: lanes f and f + 16 of a warp, then the KV head's two warps
     #pragma unroll
-    for (int hh = 0; hh < PK; ++hh) acc[hh] = 0.f;
-    #pragma unroll
-    for (int r = 0; r < 64; ++r) {
-        const float b = __uint_as_float((uint32_t)braw[r] << 16);
+    for (int hh = 0; hh < PK; ++hh)
         #pragma unroll
-        for (int hh = 0; hh < PK; ++hh) acc[hh] = fmaf(uf[jj * PK + hh][r], b, acc[hh]);
-    }
-    if (p.BV2 != nullptr) {
-        const uint16_t *bv2 = p.BV2 + (size_t)unit * 64 * 512 + 128 * j0 + tid;
-        #pragma unroll 8
-        for (int r = 0; r < 64; ++r) {
-            const float b = __uint_as_float((uint32_t)__ldcs(bv2 + (size_t)r * 512) << 16);
+        for (int e = 0; e < 8; ++e) acc[hh][e] += __shfl_xor_sync(0xffffffffu, acc[hh][e], 16);
+    if (half == 1 && lane < 16) {
+        #pragma unroll
+        for (int hh = 0; hh < PK; ++hh)
             #pragma unroll
-            for (int hh = 0; hh < PK; ++hh) acc[hh] = fmaf(uf2[jj * PK + hh][r], b, acc[hh]);
-        }
+            for (int e = 0; e < 8; ++e) red[jj][hh][8 * fg + e] = acc[hh][e];
     }
-    const int lb = unit / p.groups, G = unit % p.groups;
-    #pragma unroll
-    for (int hh = 0; hh < PK; ++hh) {
-        const int hb = jj * PK + hh;
-        const float o = (acc[hh] + wacc[hh]) * ms[hb][1];
-        p.out[((size_t)lb * p.n_q + (size_t)G * p.Hg + hb0 + hb) * 128 + dcol] = float_to_bf16_bits(o);
+    __syncthreads();
+    if (half == 0 && lane < 16) {
+        const int lb = unit / p.groups, G = unit % p.groups;
+        #pragma unroll
+        for (int hh = 0; hh < PK; ++hh) {
+            const float il = ms[hb + hh][1];
+            uint32_t w[4];
+            #pragma unroll
+            for (int e = 0; e < 4; ++e)
+                w[e] = pack_bf16((acc[hh][2 * e] + red[jj][hh][8 * fg + 2 * e]) * il,
+                                 (acc[hh][2 * e + 1] + red[jj][hh][8 * fg + 2 * e + 1]) * il);
+            uint16_t *dst = p.out + ((size_t)lb * p.n_q + (size_t)G * p.Hg + hb0 + hb + hh) * 128 + 8 * fg;
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
     }
 }
 

@@ -13,6 +13,7 @@
 // correct sort with ties to the lower index.
 //
 // Small T (<= 2048): one warp per unit, 8 units per block.
+// Medium T (<= 8192): one block of 256 threads per unit.
 // Large T (<= 65536): a cluster of 8 CTAs of 256 threads per unit (up to 32 keys per thread).
 #pragma once
 
@@ -124,6 +125,80 @@ __global__ void __launch_bounds__(256) select_warp_kernel(Params p) {
     }
     int before = incl - eq;                 // equal keys at lower token indices
     write_bits<KPT>(key, theta, need, before, r, out, p.nwords);
+}
+
+// ------------------------------------------------------------ medium T: one block per unit
+//
+// 256 threads, KPT keys each (T <= 256 KPT).  A counting pass sums the warps' counts through
+// shared memory with one barrier; the two count buffers alternate between passes, so a thread
+// that runs ahead never overwrites counts another is still reading.
+constexpr int kBlockThreads = 256;
+
+template <int KPT>
+__global__ void __launch_bounds__(kBlockThreads) select_block_kernel(Params p) {
+    __shared__ int red[2][kBlockThreads / 32];
+    __shared__ int wsum[kBlockThreads / 32];
+    const int unit = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int T = p.T;
+    const size_t ub = (size_t)unit * T;
+    const float one_minus = __fsub_rn(1.0f, p.alpha);
+    uint32_t key[KPT];
+    #pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+        const int t = tid * KPT + i;
+        key[i] = 0u;
+        if (t < T) {
+            const float m = p.mass[ub + t];
+            float x;
+            if (p.alpha == 0.0f) x = m;
+            else x = __fmaf_rn(p.alpha, p.score[ub + t], __fmul_rn(one_minus, m));
+            if (p.score != nullptr) p.score[ub + t] = x;
+            key[i] = ordered_key(x);
+        }
+    }
+    uint32_t *out = p.mask + (size_t)unit * p.nwords;
+    if (p.k <= 0) {
+        for (int wd = tid; wd < p.nwords; wd += kBlockThreads) out[wd] = 0u;
+        return;
+    }
+    int par = 0;
+    auto block_sum = [&](int v) -> int {
+        v = (int)__reduce_add_sync(0xffffffffu, (unsigned)v);
+        if (lane == 0) red[par][warp] = v;
+        __syncthreads();
+        int tot = 0;
+        #pragma unroll
+        for (int w = 0; w < kBlockThreads / 32; ++w) tot += red[par][w];
+        par ^= 1;
+        return tot;
+    };
+    uint32_t theta = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = theta | (1u << bit);
+        int c = 0;
+        #pragma unroll
+        for (int i = 0; i < KPT; ++i) c += (key[i] >= cand) ? 1 : 0;
+        if (block_sum(c) >= p.k) theta = cand;
+    }
+    int gt = 0, eq = 0;
+    #pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+        gt += (key[i] > theta) ? 1 : 0;
+        eq += (key[i] == theta) ? 1 : 0;
+    }
+    const int need = p.k - block_sum(gt);   // equal keys to take, >= 1
+    int incl = eq;
+    #pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += o;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int before = incl - eq;                  // equal keys at lower token indices
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    write_bits<KPT>(key, theta, need, before, tid, out, p.nwords);
 }
 
 // ------------------------------------------------------------ large T: a cluster of CTAs per unit

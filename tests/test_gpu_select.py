@@ -40,7 +40,7 @@ def _run(kv, m, k, alpha=0.0, score=None):
     return out.cpu().numpy().view(np.uint32), (sd.cpu().numpy() if sd is not None else None)
 
 
-@pytest.mark.parametrize("T", [1, 7, 31, 32, 33, 576, 1000, 2047, 2048, 2049, 2304, 4097, 6272, 20000, 32768, 65536])
+@pytest.mark.parametrize("T", [1, 7, 31, 32, 33, 576, 1000, 2047, 2048, 2049, 2304, 4096, 4097, 6272, 8192, 8193, 20000, 32768, 65536])
 def test_select_bit_exact(T):
     import rank_compressed_kv_b200 as kv
     m = _mass(T, T)
