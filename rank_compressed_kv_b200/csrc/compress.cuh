@@ -104,9 +104,9 @@ constexpr int kEigThreads = 512;
 constexpr int kEigWarps = kEigThreads / 32;
 constexpr int kStageRows = 32;          // rows of Y per staged chunk of a 96 x 96 product
 constexpr int kStagePitch = kP + 1;     // staged chunks are stored transposed, padded
-constexpr float kJacTol = 1e-5f;        // rotate when |a_pq| > kJacTol sqrt(|a_pp a_qq|) ...
-constexpr float kJacFloor = 1e-6f;      // ... and |a_pq| > kJacFloor max |a_ii| (the level of the product's rounding)
-constexpr float kJacQuad = 3e-3f;       // a sweep whose largest ratio is below this is the last (~sqrt(kJacTol))
+constexpr float kJacTol = 1e-6f;        // rotate when |a_pq| > kJacTol sqrt(|a_pp a_qq|) ...
+constexpr float kJacFloor = 1e-7f;      // ... and |a_pq| > kJacFloor max |a_ii| (fp32 rounding level)
+constexpr float kJacQuad = 1e-3f;       // a sweep whose largest ratio is below this is the last (~sqrt(kJacTol))
 constexpr float kPivTol = 1e-4f;        // Cholesky pivot below this fraction of its diagonal: dependent column
 constexpr float kThetaFloor = 1e-7f;    // Ritz values below this fraction of the largest are taken as zero
 
