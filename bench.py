@@ -368,6 +368,8 @@ def measure_workload(kv, torch, w: synth.Workload, K: int, W: int, dev, ranks, w
     if baselines:
         res["baselines"] = measure_baselines(kv, torch, w, dims, c, mask, q_dev[0], out, ws, L0 + W + 1, dev, ranks,
                                              max(3, min(K, 10)))
+        res["q4"] = measure_q4(kv, torch, w, dims, c, mask, q_dev[0], out, ws, L0 + W + 1, dev, ranks,
+                               max(3, min(K, 20)))
     del c, ws
     torch.cuda.empty_cache()
     return res
@@ -508,6 +510,62 @@ def measure_text_basis(kv, torch, w: synth.Workload, dev, ranks, K: int):
             "GBps_text_compressed": round(tb_bytes / (t_ms / 1e3) / 1e9, 1)}
 
 
+def measure_q4(kv, torch, w: synth.Workload, dims, c, mask, q, out, ws, L_text, dev, ranks, K: int):
+    """The decode call over 4-bit visual coefficients (kvpack_quantize4 once, then
+    kvpack_decode_attn_q4) against the 16-bit call, on the same cache, mask and query.  CUDA events
+    around K calls of each; algorithmic bytes per call for the 4-bit one (codes and exponents at
+    each token's rank, K and V, instead of the 16-bit rows)."""
+    n_layers, T, U = w.layers, w.T, w.units
+    planes = []
+    for side in ("K", "V"):
+        Q_lo = torch.empty((U, T, 8), dtype=torch.uint8, device=dev)
+        Q_hi = torch.empty((U, T, 24), dtype=torch.uint8, device=dev)
+        E = torch.empty((U, T, 2), dtype=torch.int8, device=dev)
+        kv.quantize4(dims, n_layers, T, c[f"C{side}_lo"], c[f"C{side}_hi"], Q_lo, Q_hi, E)
+        planes.append((Q_lo, Q_hi, E))
+    mass = torch.empty(U, T, dtype=torch.float32, device=dev)
+
+    def sixteen():
+        kv.decode_attn(dims, n_layers, q, c["CK_lo"], c["CK_hi"], c["BK"], c["CV_lo"], c["CV_hi"], c["BV"],
+                       c["K_text"], c["V_text"], L_text, mask, 1.0, out, mass, ws)
+
+    def four():
+        (a, b, e), (f, g, h) = planes
+        kv.decode_attn_q4(dims, n_layers, q, a, b, e, c["BK"], f, g, h, c["BV"], c["K_text"], c["V_text"], L_text,
+                          mask, 1.0, out, mass, ws)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ranks.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms, = ranks.max(e0.elapsed_time(e1) / K)
+        return ms
+
+    s_ms = timed(sixteen)
+    f_ms = timed(four)
+    st = kv.last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {kv.STATUS_NAMES[st]} in the 4-bit leg ({w.name})")
+    k = w.k_hi
+    sixteen_bytes = decode_bytes(w, L_text, k)
+    four_bytes = sixteen_bytes - U * ((k * 64 + (T - k) * 16) * 2 * 2) + U * ((k * 34 + (T - k) * 9) * 2)
+    hbm, _, _ = measured_peaks()
+    del planes
+    torch.cuda.empty_cache()
+    return {"calls_timed": K, "sixteen_bit_ms": round(s_ms, 4), "four_bit_ms": round(f_ms, 4),
+            "speedup": round(s_ms / f_ms, 2), "bytes_four_bit": int(four_bytes),
+            "GBps_four_bit": round(four_bytes / (f_ms / 1e3) / 1e9, 1),
+            "frac_four_bit": round(four_bytes / (f_ms / 1e3) / 1e9 / hbm, 4),
+            "format": "int4 codes, a power-of-two scale per token and plane (ranks 0-15, 16-63)"}
+
+
 def roofline_block(w: synth.Workload, L_mean: float, dec_avg_ms: float):
     """Roofline of the dominant call (kvpack_decode_attn): algorithmic bytes per launch over its
     CUDA-event duration, against the measured copy bandwidth."""
@@ -535,7 +593,7 @@ def config_block(res, world: int):
             "per_layer_graph": {"value": round(whole_job_value(world, w.batch, res["graph_ms"]), 1),
                                 "ms_per_step": round(res["graph_ms"], 4), "text_len": res["L_graph"]},
             "clocks": res["clocks"],
-            "baselines": res.get("baselines")}
+            "baselines": res.get("baselines"), "q4": res.get("q4")}
 
 
 EXTRA_CONFIGS = (("C2", 0.25), ("C3", 0.25), ("C4", 0.25), ("C4", 0.10))
@@ -594,6 +652,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int):
         "clocks": res["clocks"],
         "wall_s_timed": round(res["wall"], 3),
         "baselines": res.get("baselines"),
+        "q4": res.get("q4"),
     }
     if not args.no_baselines:
         line["text_basis"] = measure_text_basis(kv, torch, w, dev, ranks, max(10, min(K, args.config_steps)))

@@ -187,6 +187,39 @@ kvpack_status kvpack_decode_attn_tb(const kvpack_dims *dims, int32_t n_layers,
                                     uint16_t *out, float *mass,
                                     void *ws, size_t ws_bytes, void *stream);
 
+/* -------------------------------------------------------- 4-bit coefficients
+ * The pages compose the compression with 4-bit quantisation (Contribuciones §3 on
+ * the es page, Compatibilite §4 on the fr page, Ergebnisse §4 on the de page) but
+ * fix no format.  This library's format: per token and plane (ranks 0..15 and
+ * 16..63) symmetric int4 codes q in [-7, 7] and one power-of-two scale 2^e, e the
+ * smallest integer with 7 * 2^e >= max |c| (0 for an all-zero plane, clamped to
+ * [-127, 127]); q = round-half-even(c / 2^e) -- the block format of the OCP
+ * microscaling (MX) specification with an E8M0 scale.  The value is q * 2^e.
+ *   Q_lo [units][T][8]   codes of ranks 0..15, code 2k in the low nibble of byte k
+ *   Q_hi [units][T][24]  codes of ranks 16..63, same packing
+ *   E    [units][T][2]   int8 exponents (e of ranks 0..15, e of ranks 16..63)
+ * A reduced-rank token then costs 9 bytes per plane set and a full-rank one 34.
+ *
+ * kvpack_quantize4 -- codes and exponents of the 16-bit planes C_lo, C_hi (every
+ * token of n_layers layers' units; T tokens per unit).
+ * kvpack_decode_attn_q4 -- kvpack_decode_attn with the visual coefficients given as
+ * 4-bit planes (K: QK_lo, QK_hi, EK; V: QV_lo, QV_hi, EV): the attention of the
+ * dequantized coefficients, dequantized on the fly inside the decode (never
+ * written to memory).  Workspace, other arguments, results and errors are those
+ * of kvpack_decode_attn.
+ */
+kvpack_status kvpack_quantize4(const kvpack_dims *dims, int32_t n_layers, int32_t T,
+                               const uint16_t *C_lo, const uint16_t *C_hi,
+                               uint8_t *Q_lo, uint8_t *Q_hi, int8_t *E, void *stream);
+kvpack_status kvpack_decode_attn_q4(const kvpack_dims *dims, int32_t n_layers,
+                                    const uint16_t *q,
+                                    const uint8_t *QK_lo, const uint8_t *QK_hi, const int8_t *EK, const uint16_t *BK,
+                                    const uint8_t *QV_lo, const uint8_t *QV_hi, const int8_t *EV, const uint16_t *BV,
+                                    const uint16_t *K_text, const uint16_t *V_text, int32_t L_text,
+                                    const uint32_t *mask, float softmax_scale,
+                                    uint16_t *out, float *mass,
+                                    void *ws, size_t ws_bytes, void *stream);
+
 /* ---------------------------------------------------- decode step, no allocation
  * kvpack_decode_attn_noalloc -- the same decode step as kvpack_decode_attn,
  * for callers that cannot hand the library any device memory of their own:

@@ -21,6 +21,8 @@ computes, and the passage of the method it follows:
   decode_tb -- the same step with the text tokens compressed too, by a basis
                of their own (pages 2.A): they are decompressed at the full
                rank and attended together with the uncompressed tail.
+  quantize4 -- 4-bit coefficients (int4 codes, a power-of-two scale per token
+               and plane) and their exact dequantisation.
   select    -- importance = moving average (alpha) of attention mass; the k
                largest get the full rank next step, ties to the lower index.
 
@@ -164,6 +166,55 @@ def decode_tb(CK, BK, CV, BV, CKt, BKt, CVt, BVt, Ktail, Vtail, mask, q, r_lo=16
     Kall = np.concatenate([Kd, _f64(Ktail)], axis=1)
     Vall = np.concatenate([Vd, _f64(Vtail)], axis=1)
     return decode(CK, BK, CV, BV, Kall, Vall, mask, q, r_lo=r_lo, scale=scale, want_mass=want_mass)
+
+
+# --------------------------------------------------------------- 4-bit coefficients
+
+def quantize4(C):
+    """4-bit coefficients with a power-of-two scale per token and plane (the pages' composition of
+    the compression with 4-bit quantisation: es page 3 Contribuciones, fr page 4 Compatibilite;
+    they fix no format, so this build takes symmetric int4 codes with a shared power-of-two scale,
+    the block format of the OCP microscaling (MX) specification with E8M0 scales).
+
+    C: [..., T, 64] coefficients (bf16 values as float64).  For each token the planes of ranks
+    0..15 and 16..63 get their own exponent e = the smallest integer with 7 * 2^e >= max |c|
+    (e = 0 for an all-zero plane), and codes q = round-half-even(c / 2^e) in [-7, 7].  Returns
+    codes int8 [..., T, 64] and exponents int8 [..., T, 2]."""
+    C = np.asarray(C, dtype=np.float64)
+    codes = np.zeros(C.shape, dtype=np.int8)
+    exps = np.zeros(C.shape[:-1] + (2,), dtype=np.int8)
+    for pl, (a, b) in enumerate(((0, 16), (16, 64))):
+        X = C[..., a:b]
+        amax = np.abs(X).max(axis=-1)
+        nz = amax > 0
+        # amax = m 2^k with m in [0.5, 1): the smallest e with 7 * 2^e >= amax is k - 3 or k - 2
+        _, k = np.frexp(np.where(nz, amax, 1.0))
+        k = k.astype(np.int64)
+        e = np.where(np.ldexp(7.0, k - 3) >= amax, k - 3, k - 2)
+        e = np.where(nz, e, 0)
+        e = np.clip(e, -127, 127)
+        q = np.rint(X / np.ldexp(1.0, e)[..., None])
+        codes[..., a:b] = np.clip(q, -7, 7).astype(np.int8)
+        exps[..., pl] = e.astype(np.int8)
+    return codes, exps
+
+
+def dequantize4(codes, exps):
+    """c = q * 2^e per plane (exact in binary floating point)."""
+    codes = np.asarray(codes, dtype=np.float64)
+    e = np.asarray(exps, dtype=np.int64)
+    out = codes.copy()
+    out[..., :16] *= np.ldexp(1.0, e[..., 0])[..., None]
+    out[..., 16:] *= np.ldexp(1.0, e[..., 1])[..., None]
+    return out
+
+
+def pack4(codes):
+    """int4 codes [..., 64] -> bytes: lo plane [..., 8], hi plane [..., 24]; code 2k in the low nibble of
+    byte k, two's complement."""
+    u = (np.asarray(codes, dtype=np.int16) & 0xF).astype(np.uint8)
+    packed = (u[..., 0::2] | (u[..., 1::2] << 4)).astype(np.uint8)
+    return np.ascontiguousarray(packed[..., :8]), np.ascontiguousarray(packed[..., 8:])
 
 
 # --------------------------------------------------------------- select

@@ -14,6 +14,9 @@ Functions mirror the C entry points:
                 K_text, V_text, L_text, mask, scale, out, mass, ws)
     decode_attn_tb(dims, n_layers, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV,
                    text_basis, K_text, V_text, L_text, mask, scale, out, mass, ws)
+    quantize4(dims, n_layers, T, C_lo, C_hi, Q_lo, Q_hi, E)
+    decode_attn_q4(dims, n_layers, q, QK_lo, QK_hi, EK, BK, QV_lo, QV_hi, EV, BV,
+                   K_text, V_text, L_text, mask, scale, out, mass, ws)
     select(dims, n_layers, mass, score, alpha, k_hi, mask_out)
 
 bf16 arrays are torch.bfloat16 (or int16 views of bf16 bits); masks are
@@ -29,6 +32,8 @@ from ._lib import (  # noqa: F401
     decode_attn_noalloc,
     decode_attn_tb,
     decode_tb_workspace,
+    decode_attn_q4,
+    quantize4,
     NOALLOC_SCRATCH_BYTES,
     decode_workspace,
     decompress,

@@ -90,6 +90,11 @@ class _CTextBasis(ctypes.Structure):
                 ("L_c", _i32)]
 
 
+_L.kvpack_quantize4.argtypes = [_dims_p, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
+_L.kvpack_quantize4.restype = ctypes.c_int
+_L.kvpack_decode_attn_q4.argtypes = [_dims_p, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
+                                     ctypes.c_float, _vp, _vp, _vp, _sz, _vp]
+_L.kvpack_decode_attn_q4.restype = ctypes.c_int
 _L.kvpack_decode_tb_workspace.argtypes = [_dims_p, _i32, _i32]
 _L.kvpack_decode_tb_workspace.restype = _sz
 _L.kvpack_decode_attn_tb.argtypes = [_dims_p, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(_CTextBasis),
@@ -183,6 +188,21 @@ def decode_attn_noalloc(dims: Dims, n_layers: int, q, CK_lo, CK_hi, BK, CV_lo, C
 
 
 NOALLOC_SCRATCH_BYTES = int(_L.kvpack_noalloc_scratch_bytes())
+
+
+def quantize4(dims: Dims, n_layers: int, T: int, C_lo, C_hi, Q_lo, Q_hi, E, stream=None):
+    """4-bit codes (uint8, two per byte) and int8 exponents of the 16-bit coefficient planes."""
+    _check(_L.kvpack_quantize4(ctypes.byref(dims.c()), n_layers, int(T), _ptr(C_lo), _ptr(C_hi), _ptr(Q_lo),
+                               _ptr(Q_hi), _ptr(E), _stream(stream)), "kvpack_quantize4")
+
+
+def decode_attn_q4(dims: Dims, n_layers: int, q, QK_lo, QK_hi, EK, BK, QV_lo, QV_hi, EV, BV, K_text, V_text,
+                   L_text: int, mask, scale: float, out, mass, ws, stream=None):
+    """decode_attn over 4-bit visual coefficients, dequantized inside the decode."""
+    _check(_L.kvpack_decode_attn_q4(ctypes.byref(dims.c()), n_layers, _ptr(q), _ptr(QK_lo), _ptr(QK_hi), _ptr(EK),
+                                    _ptr(BK), _ptr(QV_lo), _ptr(QV_hi), _ptr(EV), _ptr(BV), _ptr(K_text),
+                                    _ptr(V_text), L_text, _ptr(mask), float(scale), _ptr(out), _ptr(mass),
+                                    _ptr(ws), _nbytes(ws), _stream(stream)), "kvpack_decode_attn_q4")
 
 
 def decode_tb_workspace(dims: Dims, n_layers: int, L_c: int) -> int:

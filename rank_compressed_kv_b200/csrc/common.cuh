@@ -57,9 +57,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete.  Returns false (and
 // raises *abort) if the phase has not completed and *abort is set or the wait
 // expired.  A completed phase is reported as such even after an abort, so
-// threads that wait on the same phase agree on the outcome.
-__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, volatile int *abort, long long limit) {
-    if (mbar_try_wait(bar, parity)) return true;
+// threads that wait on the same phase agree on the outcome.  The first test is
+// inline; the spin is one shared out-of-line routine, which keeps the kernels'
+// code (and its instruction-cache footprint) small.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, volatile int *abort, long long limit) {
     if (*abort) return false;
     long long t0 = clock64();
     while (true) {
@@ -71,6 +72,11 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, vo
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, volatile int *abort, long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, abort, limit);
 }
 
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {

@@ -129,16 +129,20 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
-template <int NH, bool VALUE>
+template <int NH, bool VALUE, bool Q4>
 bool rs_attr() {
-    const void *fn = (const void *)rs::rs_kernel<NH, VALUE>;
+    const void *fn = (const void *)rs::rs_kernel<NH, VALUE, Q4>;
     return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rs::smem_bytes<NH, VALUE>()) ==
                cudaSuccess &&
            cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) == cudaSuccess;
 }
 bool rs_attrs() {
-    return rs_attr<4, false>() && rs_attr<4, true>() && rs_attr<8, false>() && rs_attr<8, true>() &&
-           rs_attr<16, false>() && rs_attr<16, true>() && rs_attr<32, false>() && rs_attr<32, true>();
+    return rs_attr<4, false, false>() && rs_attr<4, true, false>() && rs_attr<8, false, false>() &&
+           rs_attr<8, true, false>() && rs_attr<16, false, false>() && rs_attr<16, true, false>() &&
+           rs_attr<32, false, false>() && rs_attr<32, true, false>() && rs_attr<4, false, true>() &&
+           rs_attr<4, true, true>() && rs_attr<8, false, true>() && rs_attr<8, true, true>() &&
+           rs_attr<16, false, true>() && rs_attr<16, true, true>() && rs_attr<32, false, true>() &&
+           rs_attr<32, true, true>();
 }
 
 // Launch on `st` with programmatic stream serialization: the kernel may start while the
@@ -160,14 +164,20 @@ cudaError_t launch_pdl(void (*kernel)(Params...), int grid, int threads, size_t 
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+template <bool VALUE, bool Q4>
+cudaError_t launch_rs_q(int NH, const rs::Params &rp, int grid, cudaStream_t st) {
+    switch (NH) {
+        case 4: return launch_pdl(rs::rs_kernel<4, VALUE, Q4>, grid, rs::kThreads, rs::smem_bytes<4, VALUE>(), st, rp);
+        case 8: return launch_pdl(rs::rs_kernel<8, VALUE, Q4>, grid, rs::kThreads, rs::smem_bytes<8, VALUE>(), st, rp);
+        case 16:
+            return launch_pdl(rs::rs_kernel<16, VALUE, Q4>, grid, rs::kThreads, rs::smem_bytes<16, VALUE>(), st, rp);
+        default:
+            return launch_pdl(rs::rs_kernel<32, VALUE, Q4>, grid, rs::kThreads, rs::smem_bytes<32, VALUE>(), st, rp);
+    }
+}
 template <bool VALUE>
 cudaError_t launch_rs(int NH, const rs::Params &rp, int grid, cudaStream_t st) {
-    switch (NH) {
-        case 4: return launch_pdl(rs::rs_kernel<4, VALUE>, grid, rs::kThreads, rs::smem_bytes<4, VALUE>(), st, rp);
-        case 8: return launch_pdl(rs::rs_kernel<8, VALUE>, grid, rs::kThreads, rs::smem_bytes<8, VALUE>(), st, rp);
-        case 16: return launch_pdl(rs::rs_kernel<16, VALUE>, grid, rs::kThreads, rs::smem_bytes<16, VALUE>(), st, rp);
-        default: return launch_pdl(rs::rs_kernel<32, VALUE>, grid, rs::kThreads, rs::smem_bytes<32, VALUE>(), st, rp);
-    }
+    return rp.QK_lo != nullptr ? launch_rs_q<VALUE, true>(NH, rp, grid, st) : launch_rs_q<VALUE, false>(NH, rp, grid, st);
 }
 
 // finish_kernel is instantiated for 1..8 query heads per KV head, and for a whole unit per
@@ -347,10 +357,17 @@ size_t kvpack_decode_workspace(const kvpack_dims *d, int32_t n_layers) {
 
 namespace {
 
-// The decode step; tb (the text tokens compressed with a basis of their own) may be null.
+// 4-bit visual coefficients (quant.cuh) in place of the 16-bit planes
+struct Q4Planes {
+    const uint8_t *QK_lo, *QK_hi, *QV_lo, *QV_hi;
+    const int8_t *EK, *EV;
+};
+
+// The decode step; tb (the text tokens compressed with a basis of their own) and q4 (4-bit
+// visual coefficients, when CK_lo .. CV_hi are null) may be null.
 kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t *q, const uint16_t *CK_lo,
                           const uint16_t *CK_hi, const uint16_t *BK, const uint16_t *CV_lo, const uint16_t *CV_hi,
-                          const uint16_t *BV, const kvpack_text_basis *tb, const uint16_t *K_text,
+                          const uint16_t *BV, const Q4Planes *q4, const kvpack_text_basis *tb, const uint16_t *K_text,
                           const uint16_t *V_text, int32_t L_text, const uint32_t *mask, float softmax_scale,
                           uint16_t *out, float *mass, void *ws, size_t ws_bytes, void *stream) {
     kvpack_status s = check_dims(d, n_layers);
@@ -367,7 +384,15 @@ kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t
         }
     }
     if (L_text < 0 || L_text > d->L_text_cap) return KVPACK_ERR_INVALID_ARG;
-    if (!q || !CK_lo || !CK_hi || !BK || !CV_lo || !CV_hi || !BV || !mask || !out) return KVPACK_ERR_INVALID_ARG;
+    if (!q || !BK || !BV || !mask || !out) return KVPACK_ERR_INVALID_ARG;
+    if (q4 == nullptr && (!CK_lo || !CK_hi || !CV_lo || !CV_hi)) return KVPACK_ERR_INVALID_ARG;
+    if (q4 != nullptr) {
+        const void *qp[] = {q4->QK_lo, q4->QK_hi, q4->QV_lo, q4->QV_hi, q4->EK, q4->EV};
+        for (const void *ptr : qp) {
+            if (ptr == nullptr) return KVPACK_ERR_INVALID_ARG;
+            if (!aligned16(ptr)) return KVPACK_ERR_ALIGNMENT;
+        }
+    }
     if (L_text > 0 && (!K_text || !V_text)) return KVPACK_ERR_INVALID_ARG;
     if (!(softmax_scale == softmax_scale) || softmax_scale <= 0.f) return KVPACK_ERR_INVALID_ARG;
     const void *ptrs[] = {q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, mask, out, mass, ws,
@@ -446,7 +471,10 @@ kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t
     // unit-wide statistics, then the value passes
     rs::Params rp;
     std::memset(&rp, 0, sizeof(rp));
-    {
+    if (q4 != nullptr) {
+        rp.QK_lo = q4->QK_lo; rp.QK_hi = q4->QK_hi; rp.QV_lo = q4->QV_lo; rp.QV_hi = q4->QV_hi;
+        rp.EK = q4->EK; rp.EV = q4->EV;
+    } else {
         const cuuint64_t dims[3] = {16, (cuuint64_t)T, (cuuint64_t)pl.units};
         const cuuint64_t strides[2] = {32, (cuuint64_t)T * 32};
         const cuuint32_t box[3] = {16, 256, 1};
@@ -513,8 +541,8 @@ kvpack_status kvpack_decode_attn(const kvpack_dims *d, int32_t n_layers, const u
                                  const uint16_t *K_text, const uint16_t *V_text, int32_t L_text,
                                  const uint32_t *mask, float softmax_scale, uint16_t *out, float *mass,
                                  void *ws, size_t ws_bytes, void *stream) {
-    return decode_impl(d, n_layers, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, nullptr, K_text, V_text, L_text, mask,
-                       softmax_scale, out, mass, ws, ws_bytes, stream);
+    return decode_impl(d, n_layers, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, nullptr, nullptr, K_text, V_text, L_text,
+                       mask, softmax_scale, out, mass, ws, ws_bytes, stream);
 }
 
 size_t kvpack_decode_tb_workspace(const kvpack_dims *d, int32_t n_layers, int32_t L_c) {
@@ -529,8 +557,35 @@ kvpack_status kvpack_decode_attn_tb(const kvpack_dims *d, int32_t n_layers, cons
                                     int32_t L_text, const uint32_t *mask, float softmax_scale, uint16_t *out,
                                     float *mass, void *ws, size_t ws_bytes, void *stream) {
     if (tb == nullptr) return KVPACK_ERR_INVALID_ARG;
-    return decode_impl(d, n_layers, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, tb, K_text, V_text, L_text, mask,
+    return decode_impl(d, n_layers, q, CK_lo, CK_hi, BK, CV_lo, CV_hi, BV, nullptr, tb, K_text, V_text, L_text, mask,
                        softmax_scale, out, mass, ws, ws_bytes, stream);
+}
+
+kvpack_status kvpack_quantize4(const kvpack_dims *d, int32_t n_layers, int32_t T, const uint16_t *C_lo,
+                               const uint16_t *C_hi, uint8_t *Q_lo, uint8_t *Q_hi, int8_t *E, void *stream) {
+    kvpack_status s = check_dims(d, n_layers);
+    if (s != KVPACK_OK) return s;
+    if (T < 1 || T > kMaxT) return KVPACK_ERR_INVALID_ARG;
+    if (!C_lo || !C_hi || !Q_lo || !Q_hi || !E) return KVPACK_ERR_INVALID_ARG;
+    const void *ptrs[] = {C_lo, C_hi, Q_lo, Q_hi, E};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return KVPACK_ERR_ALIGNMENT;
+    const long long rows = (long long)n_units(d, n_layers) * T;
+    const long long blocks = (rows + 255) / 256;
+    kvpack::quant::quantize4_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        C_lo, C_hi, Q_lo, Q_hi, E, rows);
+    return cudaGetLastError() == cudaSuccess ? KVPACK_OK : KVPACK_ERR_CUDA;
+}
+
+kvpack_status kvpack_decode_attn_q4(const kvpack_dims *d, int32_t n_layers, const uint16_t *q,
+                                    const uint8_t *QK_lo, const uint8_t *QK_hi, const int8_t *EK, const uint16_t *BK,
+                                    const uint8_t *QV_lo, const uint8_t *QV_hi, const int8_t *EV, const uint16_t *BV,
+                                    const uint16_t *K_text, const uint16_t *V_text, int32_t L_text,
+                                    const uint32_t *mask, float softmax_scale, uint16_t *out, float *mass, void *ws,
+                                    size_t ws_bytes, void *stream) {
+    const Q4Planes q4{QK_lo, QK_hi, QV_lo, QV_hi, EK, EV};
+    return decode_impl(d, n_layers, q, nullptr, nullptr, BK, nullptr, nullptr, BV, &q4, nullptr, K_text, V_text, L_text,
+                       mask, softmax_scale, out, mass, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -48,6 +48,7 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "quant.cuh"
 
 namespace kvpack {
 namespace decode {
@@ -100,6 +101,8 @@ struct Cfg {
 struct Params {
     CUtensorMap tm_ck, tm_cv;       // C_lo planes: 3D {16, T, units}, box {16, 256, 1}, 32-byte swizzle
     const uint16_t *CK_lo, *CK_hi, *CV_lo, *CV_hi;
+    const uint8_t *QK_lo, *QK_hi, *QV_lo, *QV_hi;   // 4-bit planes (quant.cuh), when the kernel is Q4
+    const int8_t *EK, *EV;                           // their exponents [units][T][2]
     const unsigned char *qt;        // [units][qblock_bytes(Hg)]: q~ hi, lo planes (from text_kernel)
     const uint32_t *mask;           // [units][nwords]
     const float *ustat;             // value pass: [units][Hg][2] = (M, 1/L)
@@ -143,6 +146,7 @@ constexpr bool smem_fits() { return Cfg<NH, VALUE>::kBlocks * (smem_bytes<NH, VA
 static_assert(smem_fits<4, false>() && smem_fits<4, true>() && smem_fits<8, false>() && smem_fits<8, true>(), "smem");
 static_assert(smem_fits<16, false>() && smem_fits<16, true>(), "shared memory of two CTAs per SM");
 static_assert(smem_fits<32, false>() && smem_fits<32, true>(), "shared memory of one CTA per SM");
+static_assert(kGatherThreads == 64, "the 4-bit gather assumes 64 threads");
 
 // ------------------------------------------------------------------ tcgen05 helpers
 
@@ -193,7 +197,10 @@ __device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, float (&v)[32]) {
 
 // ------------------------------------------------------------------ the kernel
 
-template <int NH, bool VALUE>
+// Q4: the coefficients are 4-bit (quant.cuh); the gather warps then dequantize every tile, LO and
+// HI, into the same shared-memory layouts the TMA and cp.async copies produce, so the score MMA
+// and the consumers are unchanged.
+template <int NH, bool VALUE, bool Q4>
 __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(const __grid_constant__ Params p) {
     using C = Cfg<NH, VALUE>;
     constexpr int kNK = C::kNK, kNV = C::kNV, kNS = C::kNS, kNHP = C::kNHP, kPH = C::kPH;
@@ -282,12 +289,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
         };
         // hand a full-rank tile (K slot ks, V slot vs, descriptor ds) to the gather warp; ks < 0 ends it
         uint32_t hseq = 0;
-        auto push_gather = [&](int ks, int vs, int ds, int n, int unit) -> bool {
+        auto push_gather = [&](int ks, int vs, int ds, int n, int unit, int type, int tok) -> bool {
             const int hq = hseq % kNQ;
             if (hseq >= (uint32_t)kNQ && !mbar_wait(&sm.gfree[hq], ((hseq / kNQ) - 1) & 1u, abort)) return false;
             if (lane == 0) {
                 int *e = sm.hiq[hq];
-                e[0] = ks; e[1] = vs; e[2] = ds; e[3] = n; e[4] = unit;
+                e[0] = ks; e[1] = vs; e[2] = ds; e[3] = n; e[4] = unit; e[5] = type; e[6] = tok;
                 mbar_arrive(&sm.gready[hq]);
             }
             ++hseq;
@@ -301,7 +308,6 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             const int tok0 = (int)(x - (long long)unit * p.tpu) * kTile;
             const int tok1 = min(p.T, (int)(xe - (long long)unit * p.tpu) * kTile);
             const int pslot = (int)(blockIdx.x - cta_of_tile((long long)unit * p.tpu, CT, NT));
-            const size_t ubase = (size_t)unit * p.T;
             x = xe;
             // the unit's q~ into the next q slot
             const int qs = qseq & 1;
@@ -360,11 +366,15 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                     if (lane < C::kLoTok / 32) d[8 + lane] = (int)wd;
                     first = false;
                     __syncwarp();
-                    // lane 0 issues the copies and arrives for itself and for the gather warp's
-                    // lanes (which have nothing to add to a LO tile); the other lanes' arrivals
-                    // release their descriptor writes
+                    // lane 0 issues the copies and arrives for itself and for the gather warps
+                    // (which have nothing to add to a LO tile); the other lanes' arrivals
+                    // release their descriptor writes.  4-bit rows go to the gather warps instead.
                     const int nb = (n + 255) >> 8;   // 256-row boxes of 32-byte rows
-                    if (lane == 0) {
+                    if (Q4 && !p.rank0) {
+                        if (!push_gather(ks, vs, ds, n, unit, kTypeLo, tok)) { ok = false; break; }
+                        mbar_arrive(&sm.kfull[ks]);
+                        if (VALUE) mbar_arrive(&sm.vfull[vs]);
+                    } else if (lane == 0) {
                         if (!p.rank0) {
                             fence_proxy_async();
                             mbar_arrive_tx(&sm.kfull[ks], (uint32_t)nb * 8192u);
@@ -404,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                     }
                     first = false;
                     __syncwarp();
-                    if (!push_gather(ks, vs, ds, nh, unit)) { ok = false; break; }
+                    if (!push_gather(ks, vs, ds, nh, unit, kTypeHi, 0)) { ok = false; break; }
                     mbar_arrive(&sm.kfull[ks]);       // releases this lane's descriptor writes
                     if (VALUE) mbar_arrive(&sm.vfull[vs]);
                     hi_head += (unsigned)nh;
@@ -421,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 __syncwarp();
                 mbar_arrive(&sm.kfull[ks]);
                 if (lane == 0) mbar_arrive_cnt(&sm.kfull[ks], kGatherThreads);
-                ended = push_gather(-1, 0, 0, 0, 0);
+                ended = push_gather(-1, 0, 0, 0, 0, kTypeEnd, 0);
             }
             ok = ended;
         }
@@ -467,13 +477,99 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             const int hq = h % kNQ;
             if (!mbar_wait(&sm.gready[hq], (h / kNQ) & 1u, abort)) break;
             const int *e = sm.hiq[hq];
-            const int ks = e[0], vs = e[1], ds = e[2], n = e[3], unit = e[4];
+            const int ks = e[0], vs = e[1], ds = e[2], n = e[3], unit = e[4], type = e[5], tok = e[6];
             mbar_arrive(&sm.gfree[hq]);
             if (ks < 0) break;
             // the positions stay valid until the consumers free the descriptor, which needs this
             // tile's data first
             const uint16_t *pos = reinterpret_cast<const uint16_t *>(sm.kdesc[ds] + 8);
             const size_t ubase = (size_t)unit * p.T;
+            if constexpr (Q4) {
+                // dequantize into the layouts of the 16-bit path: LO rows of 32 bytes (32-byte
+                // swizzle), HI rows of 128 bytes (128-byte swizzle); rows past n are zero
+                constexpr int RL = C::kLoTok / kGatherThreads, RH = C::kHiTok / kGatherThreads;
+                struct LoRows { uint2 w[RL]; int ex[RL]; };
+                struct HiRows { uint2 w[RH][4]; char2 ee[RH]; };
+                auto lo_load = [&](LoRows &L, const uint8_t *Q, const int8_t *E) {
+                    #pragma unroll
+                    for (int i = 0; i < RL; ++i) {
+                        const int t = g + kGatherThreads * i;
+                        L.w[i] = make_uint2(0u, 0u);
+                        L.ex[i] = 0;
+                        if (t < n) {
+                            const size_t row = ubase + tok + t;
+                            L.w[i] = __ldg(reinterpret_cast<const uint2 *>(Q + row * 8));
+                            L.ex[i] = __ldg(E + row * 2);
+                        }
+                    }
+                };
+                auto lo_store = [&](const LoRows &L, unsigned char *dst) {
+                    #pragma unroll
+                    for (int i = 0; i < RL; ++i) {
+                        const int t = g + kGatherThreads * i;
+                        const int sw = (t >> 2) & 1;
+                        *reinterpret_cast<uint4 *>(dst + t * 32 + (sw << 4)) = quant::dq8(L.w[i].x, L.ex[i]);
+                        *reinterpret_cast<uint4 *>(dst + t * 32 + ((1 ^ sw) << 4)) = quant::dq8(L.w[i].y, L.ex[i]);
+                    }
+                };
+                auto hi_load = [&](HiRows &H, const uint8_t *QL, const uint8_t *QH, const int8_t *E) {
+                    #pragma unroll
+                    for (int i = 0; i < RH; ++i) {
+                        const int r = g + kGatherThreads * i;
+                        #pragma unroll
+                        for (int k = 0; k < 4; ++k) H.w[i][k] = make_uint2(0u, 0u);
+                        H.ee[i] = make_char2(0, 0);
+                        if (r < n) {
+                            const size_t row = ubase + pos[r];
+                            H.w[i][0] = __ldg(reinterpret_cast<const uint2 *>(QL + row * 8));
+                            const uint2 *hq2 = reinterpret_cast<const uint2 *>(QH + row * 24);
+                            H.w[i][1] = __ldg(hq2);
+                            H.w[i][2] = __ldg(hq2 + 1);
+                            H.w[i][3] = __ldg(hq2 + 2);
+                            H.ee[i] = __ldg(reinterpret_cast<const char2 *>(E + row * 2));
+                        }
+                    }
+                };
+                auto hi_store = [&](const HiRows &H, unsigned char *dst) {
+                    #pragma unroll
+                    for (int i = 0; i < RH; ++i) {
+                        const int r = g + kGatherThreads * i;
+                        #pragma unroll
+                        for (int c8 = 0; c8 < 8; ++c8) {
+                            const uint32_t word = (c8 & 1) ? H.w[i][c8 >> 1].y : H.w[i][c8 >> 1].x;
+                            *reinterpret_cast<uint4 *>(dst + r * 128 + ((c8 ^ (r & 7)) << 4)) =
+                                quant::dq8(word, c8 < 2 ? H.ee[i].x : H.ee[i].y);
+                        }
+                    }
+                };
+                // every load of a tile (K and V) is issued before the first is used, so one memory
+                // latency is paid per tile
+                if (type == kTypeLo) {
+                    LoRows K4, V4;
+                    lo_load(K4, p.QK_lo, p.EK);
+                    if (VALUE) lo_load(V4, p.QV_lo, p.EV);
+                    lo_store(K4, sm.kslot[ks]);
+                    fence_proxy_async();              // the score MMA reads these rows through the async proxy
+                    mbar_arrive(&sm.kfull[ks]);
+                    if (VALUE) {
+                        lo_store(V4, sm.vslot[vs]);
+                        mbar_arrive(&sm.vfull[vs]);
+                    }
+                } else {
+                    HiRows K4, V4;
+                    hi_load(K4, p.QK_lo, p.QK_hi, p.EK);
+                    if (VALUE) hi_load(V4, p.QV_lo, p.QV_hi, p.EV);
+                    hi_store(K4, sm.kslot[ks]);
+                    fence_proxy_async();
+                    mbar_arrive(&sm.kfull[ks]);
+                    if (VALUE) {
+                        hi_store(V4, sm.vslot[vs]);
+                        mbar_arrive(&sm.vfull[vs]);
+                    }
+                }
+                ++h;
+                continue;
+            }
             gather(sm.kslot[ks], p.CK_lo, p.CK_hi, pos, n, ubase, false);
             cp_async_arrive(&sm.kfull[ks]);   // raises the pending count; arrives when the copies land
             mbar_arrive(&sm.kfull[ks]);
@@ -518,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 }
                 const bool has_s = type == kTypeHi || !p.rank0;
                 if (has_s) {
-                    if (type == kTypeHi) fence_proxy_async();   // the gathered rows were written by cp.async
+                    if (type == kTypeHi || Q4) fence_proxy_async();   // rows written by cp.async or stores
                     tmem_fence_after();
                     const uint32_t dcol = tmem + (uint32_t)(sb * C::kSCols);
                     const uint64_t qh = dqh0 + (uint64_t)(qs * kQStep), ql = dql0 + (uint64_t)(qs * kQStep);
@@ -696,7 +792,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                         }
                         __syncwarp();
                         // u^T += C_V^T P over the warp's 32 tokens (two k-steps of 16)
-                        #pragma unroll
+                        #pragma unroll 1
                         for (int kk = 0; kk < 2; ++kk) {
                             uint32_t bfr[kPH / 8][2];
                             #pragma unroll

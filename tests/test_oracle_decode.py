@@ -263,3 +263,60 @@ def test_text_basis_rank_space_route():
     o1, _ = oracle.decode_tb(CK, BK, CV, BV, big, BKt, CVt, BVt, Kt, Vt, mask, qq)
     o2, _ = oracle.decode_tb(CK, BK, CV, BV, 0 * big, BKt, CVt, BVt, Kt, Vt, mask, qq)
     np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-9)
+
+
+# ----------------------------------------------------------------- 4-bit coefficients
+
+def test_quantize4_exponent_and_codes_by_brute_force():
+    """e is the smallest integer with 7 * 2^e >= max |c| (searched over all candidates), codes
+    are c / 2^e rounded half to even, and |q| <= 7."""
+    g = np.random.default_rng(81)
+    C = g.standard_normal((40, 64)) * np.exp(g.uniform(-20, 20, size=(40, 1)))
+    C[3] = 0.0                                  # an all-zero token
+    C[5, :16] = 0.0                             # an all-zero plane
+    C[7, :16] = np.linspace(-3.0, 3.0, 16)
+    C[7, 0] = 7 * 2.0 ** 3                      # the maximum exactly on 7 * 2^e
+    C[8, :16] = 0.0
+    C[8, 1] = 2.5 * 2.0 ** -4                   # a tie, rounded to even
+    C[8, 0] = 7 * 2.0 ** -4
+    q, e = oracle.quantize4(C)
+    for t in range(C.shape[0]):
+        for pl, (a, b) in enumerate(((0, 16), (16, 64))):
+            amax = np.abs(C[t, a:b]).max()
+            if amax == 0:
+                assert e[t, pl] == 0 and np.all(q[t, a:b] == 0)
+                continue
+            best = min(x for x in range(-200, 200) if 7 * 2.0 ** x >= amax)
+            assert e[t, pl] == best
+            assert np.all(np.abs(q[t, a:b]) <= 7)
+            for i in range(a, b):
+                v = C[t, i] / 2.0 ** best
+                r = np.floor(v + 0.5)
+                if r - v == 0.5 and r % 2 == 1:   # a tie goes to the even neighbour
+                    r -= 1
+                assert q[t, i] == r
+    assert e[7, 0] == 3 and q[7, 0] == 7
+    assert q[8, 1] == 2                          # 2.5 -> 2
+
+
+def test_quantize4_round_trip_and_error_bound():
+    g = np.random.default_rng(82)
+    C = g.standard_normal((100, 64))
+    q, e = oracle.quantize4(C)
+    D = oracle.dequantize4(q, e)
+    step = np.concatenate([np.repeat(2.0 ** e[:, :1], 16, axis=1), np.repeat(2.0 ** e[:, 1:], 48, axis=1)], axis=1)
+    assert np.all(np.abs(D - C) <= step / 2)    # half a step at most
+    q2, e2 = oracle.quantize4(D)                 # grid values are fixed points
+    assert np.array_equal(q2, q) and np.array_equal(e2, e)
+
+
+def test_pack4_layout():
+    codes = np.arange(-7, 8).tolist() * 5
+    codes = np.array(codes[:64], dtype=np.int8)[None]
+    lo, hi = oracle.pack4(codes)
+    assert lo.shape == (1, 8) and hi.shape == (1, 24)
+    flat = np.concatenate([lo, hi], axis=1)[0]
+    for k in range(32):
+        low, high = int(flat[k]) & 0xF, int(flat[k]) >> 4
+        sx = lambda v: v - 16 if v >= 8 else v
+        assert sx(low) == codes[0, 2 * k] and sx(high) == codes[0, 2 * k + 1]
