@@ -371,9 +371,21 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                     // release their descriptor writes.  4-bit rows go to the gather warps instead.
                     const int nb = (n + 255) >> 8;   // 256-row boxes of 32-byte rows
                     if (Q4 && !p.rank0) {
-                        if (!push_gather(ks, vs, ds, n, unit, kTypeLo, tok)) { ok = false; break; }
+                        // 4-bit rows: the producer dequantizes LO tiles itself, in parallel with the
+                        // gather warps' HI tiles, and arrives for the gather warps
+                        const size_t base = (size_t)unit * p.T + tok;
+                        if (VALUE)
+                            quant::lo_rows_kv<C::kLoTok / 32, 32>(sm.kslot[ks], sm.vslot[vs], p.QK_lo, p.EK, p.QV_lo,
+                                                                  p.EV, base, n, lane);
+                        else
+                            quant::lo_rows<C::kLoTok / 32, 32>(sm.kslot[ks], p.QK_lo, p.EK, base, n, lane);
+                        fence_proxy_async();          // the score MMA reads these rows through the async proxy
                         mbar_arrive(&sm.kfull[ks]);
                         if (VALUE) mbar_arrive(&sm.vfull[vs]);
+                        if (lane == 0) {
+                            mbar_arrive_cnt(&sm.kfull[ks], kGatherThreads);
+                            if (VALUE) mbar_arrive_cnt(&sm.vfull[vs], kGatherThreads);
+                        }
                     } else if (lane == 0) {
                         if (!p.rank0) {
                             fence_proxy_async();
@@ -477,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             const int hq = h % kNQ;
             if (!mbar_wait(&sm.gready[hq], (h / kNQ) & 1u, abort)) break;
             const int *e = sm.hiq[hq];
-            const int ks = e[0], vs = e[1], ds = e[2], n = e[3], unit = e[4], type = e[5], tok = e[6];
+            const int ks = e[0], vs = e[1], ds = e[2], n = e[3], unit = e[4];
             mbar_arrive(&sm.gfree[hq]);
             if (ks < 0) break;
             // the positions stay valid until the consumers free the descriptor, which needs this
@@ -485,33 +497,10 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             const uint16_t *pos = reinterpret_cast<const uint16_t *>(sm.kdesc[ds] + 8);
             const size_t ubase = (size_t)unit * p.T;
             if constexpr (Q4) {
-                // dequantize into the layouts of the 16-bit path: LO rows of 32 bytes (32-byte
-                // swizzle), HI rows of 128 bytes (128-byte swizzle); rows past n are zero
-                constexpr int RL = C::kLoTok / kGatherThreads, RH = C::kHiTok / kGatherThreads;
-                struct LoRows { uint2 w[RL]; int ex[RL]; };
+                // dequantize a HI tile into the layout of the 16-bit path (128-byte rows, 128-byte
+                // swizzle); rows past n are zero.  (LO tiles of 4-bit rows are the producer's.)
+                constexpr int RH = C::kHiTok / kGatherThreads;
                 struct HiRows { uint2 w[RH][4]; char2 ee[RH]; };
-                auto lo_load = [&](LoRows &L, const uint8_t *Q, const int8_t *E) {
-                    #pragma unroll
-                    for (int i = 0; i < RL; ++i) {
-                        const int t = g + kGatherThreads * i;
-                        L.w[i] = make_uint2(0u, 0u);
-                        L.ex[i] = 0;
-                        if (t < n) {
-                            const size_t row = ubase + tok + t;
-                            L.w[i] = __ldg(reinterpret_cast<const uint2 *>(Q + row * 8));
-                            L.ex[i] = __ldg(E + row * 2);
-                        }
-                    }
-                };
-                auto lo_store = [&](const LoRows &L, unsigned char *dst) {
-                    #pragma unroll
-                    for (int i = 0; i < RL; ++i) {
-                        const int t = g + kGatherThreads * i;
-                        const int sw = (t >> 2) & 1;
-                        *reinterpret_cast<uint4 *>(dst + t * 32 + (sw << 4)) = quant::dq8(L.w[i].x, L.ex[i]);
-                        *reinterpret_cast<uint4 *>(dst + t * 32 + ((1 ^ sw) << 4)) = quant::dq8(L.w[i].y, L.ex[i]);
-                    }
-                };
                 auto hi_load = [&](HiRows &H, const uint8_t *QL, const uint8_t *QH, const int8_t *E) {
                     #pragma unroll
                     for (int i = 0; i < RH; ++i) {
@@ -544,18 +533,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 };
                 // every load of a tile (K and V) is issued before the first is used, so one memory
                 // latency is paid per tile
-                if (type == kTypeLo) {
-                    LoRows K4, V4;
-                    lo_load(K4, p.QK_lo, p.EK);
-                    if (VALUE) lo_load(V4, p.QV_lo, p.EV);
-                    lo_store(K4, sm.kslot[ks]);
-                    fence_proxy_async();              // the score MMA reads these rows through the async proxy
-                    mbar_arrive(&sm.kfull[ks]);
-                    if (VALUE) {
-                        lo_store(V4, sm.vslot[vs]);
-                        mbar_arrive(&sm.vfull[vs]);
-                    }
-                } else {
+                {
                     HiRows K4, V4;
                     hi_load(K4, p.QK_lo, p.QK_hi, p.EK);
                     if (VALUE) hi_load(V4, p.QV_lo, p.QV_hi, p.EV);
