@@ -104,7 +104,7 @@ def whole_job_value(world: int, batch: int, ms_per_step: float) -> float:
     return world * batch / (ms_per_step / 1e3)
 
 
-DECODE_SOURCES = ("decode.cuh", "rstream.cuh", "common.cuh", "kvpack.cu")
+DECODE_SOURCES = ("decode.cuh", "rstream.cuh", "quant.cuh", "common.cuh", "kvpack.cu")
 
 
 def sources_digest(names=DECODE_SOURCES) -> str:

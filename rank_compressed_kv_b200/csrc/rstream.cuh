@@ -680,8 +680,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             const int nsub = type == kTypeLo ? (n + kTile - 1) / kTile : 1;
             const uint32_t vb = smem_u32(sm.vslot[vs]);
             bool v_ready = false;
-            // the scores of up to kLd sub-tiles are loaded from tensor memory before one wait
-            constexpr int kLd = (C::kSub * NH <= 64) ? C::kSub : (64 / NH > 0 ? 64 / NH : 1);
+            // the scores of one sub-tile are loaded from tensor memory before each wait
+            constexpr int kLd = 1;   // measured: batching the loads of several sub-tiles was slower (larger code)
             for (int sub0 = 0; sub0 < nsub && !failed; sub0 += kLd) {
                 float scv[kLd][NH];
                 #pragma unroll
