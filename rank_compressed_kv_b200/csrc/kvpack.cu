@@ -61,11 +61,12 @@ struct DecodePlan {
     int units, Hg, NH, tpu, nwords, Sc_max;
     long long ntiles;
     int cta_s, cta_v, nslot_s, nslot_v;
-    size_t off_qt, off_tp, off_sp, off_ustat, off_vp, off_counter, total;
+    size_t off_qt, off_tp, off_sp, off_ustat, off_vp, off_counter, off_hipos, off_hicnt, total;
+    int Tp;   // stride of a unit's list of full-rank positions (T rounded up to 8)
     // the text tokens' own rank-space passes (text compressed too); absent when L_c = 0
-    int L_c, tpu2, nwords2, cta2, nslot2;
+    int L_c, tpu2, nwords2, cta2, nslot2, Tp2;
     long long ntiles2;
-    size_t off_qt2, off_sp2, off_vp2, off_mask2;
+    size_t off_qt2, off_sp2, off_vp2, off_mask2, off_hipos2, off_hicnt2;
 };
 
 inline int round_heads(int Hg) { return Hg <= 4 ? 4 : Hg <= 8 ? 8 : Hg <= 16 ? 16 : 32; }
@@ -101,6 +102,11 @@ DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers, int L_c = 0) {
     off = align256(off + (size_t)pl.units * pl.nslot_v * pl.Hg * 64 * sizeof(float));
     pl.off_counter = off;   // work counter of the text kernel
     off = align256(off + 4 * sizeof(unsigned int));
+    pl.Tp = (T + 7) & ~7;
+    pl.off_hipos = off;
+    off = align256(off + (size_t)pl.units * pl.Tp * sizeof(uint16_t));
+    pl.off_hicnt = off;
+    off = align256(off + (size_t)pl.units * pl.tpu * sizeof(int));
     pl.L_c = L_c;
     if (L_c > 0) {
         pl.tpu2 = (L_c + rs::kTile - 1) / rs::kTile;
@@ -116,6 +122,11 @@ DecodePlan plan_decode(const kvpack_dims *d, int32_t n_layers, int L_c = 0) {
         off = align256(off + (size_t)pl.units * pl.nslot2 * pl.Hg * 64 * sizeof(float));
         pl.off_mask2 = off;     // every text token at the full rank
         off = align256(off + (size_t)pl.units * pl.nwords2 * sizeof(uint32_t));
+        pl.Tp2 = (L_c + 7) & ~7;
+        pl.off_hipos2 = off;
+        off = align256(off + (size_t)pl.units * pl.Tp2 * sizeof(uint16_t));
+        pl.off_hicnt2 = off;
+        off = align256(off + (size_t)pl.units * pl.tpu2 * sizeof(int));
     }
     pl.total = off;
     return pl;
@@ -484,6 +495,11 @@ kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t
     }
     rp.CK_lo = CK_lo; rp.CK_hi = CK_hi; rp.CV_lo = CV_lo; rp.CV_hi = CV_hi;
     rp.qt = qt; rp.mask = mask; rp.ustat = ustat;
+    uint16_t *hipos = reinterpret_cast<uint16_t *>(w + pl.off_hipos);
+    int *hicnt = reinterpret_cast<int *>(w + pl.off_hicnt);
+    uint16_t *hipos2 = L_c > 0 ? reinterpret_cast<uint16_t *>(w + pl.off_hipos2) : nullptr;
+    int *hicnt2 = L_c > 0 ? reinterpret_cast<int *>(w + pl.off_hicnt2) : nullptr;
+    rp.hipos = hipos; rp.hicnt = hicnt; rp.Tp = pl.Tp;
     rp.units = pl.units; rp.T = T; rp.Hg = Hg; rp.nwords = pl.nwords; rp.tpu = pl.tpu;
     rp.rank0 = d->rank_lo == 0 ? 1 : 0; rp.ntiles = pl.ntiles;
     rs::Params rp2;
@@ -497,8 +513,25 @@ kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t
             return KVPACK_ERR_CUDA;
         rp2.CK_lo = tb->CK_lo; rp2.CK_hi = tb->CK_hi; rp2.CV_lo = tb->CV_lo; rp2.CV_hi = tb->CV_hi;
         rp2.qt = qt2; rp2.mask = mask2; rp2.ustat = ustat;
+        rp2.hipos = hipos2; rp2.hicnt = hicnt2; rp2.Tp = pl.Tp2;
         rp2.units = pl.units; rp2.T = L_c; rp2.Hg = Hg; rp2.nwords = pl.nwords2; rp2.tpu = pl.tpu2;
         rp2.rank0 = 0; rp2.ntiles = pl.ntiles2;
+    }
+    {
+        // each unit's full-rank positions, for the HI tiles of both passes
+        const rs::HiposParams ha{mask, hipos, hicnt, pl.units, T, pl.nwords, pl.tpu, pl.Tp};
+        const rs::HiposParams hb =
+            L_c > 0 ? rs::HiposParams{mask2, hipos2, hicnt2, pl.units, L_c, pl.nwords2, pl.tpu2, pl.Tp2} : ha;
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)pl.units, L_c > 0 ? 2u : 1u);
+        cfg.blockDim = dim3((unsigned)rs::kHpThreads);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, rs::hipos_kernel, ha, hb) != cudaSuccess) return KVPACK_ERR_CUDA;
     }
     rp.part = spart; rp.nslot = pl.nslot_s; rp.mass = nullptr;
     if (launch_rs<false>(pl.NH, rp, pl.cta_s, st) != cudaSuccess) return KVPACK_ERR_CUDA;

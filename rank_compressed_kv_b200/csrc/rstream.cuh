@@ -22,14 +22,15 @@
 // ("segments") and writes one partial per segment, so a unit has at most a
 // few partials whatever its length.
 //
-// A CTA has six warps:
+// A CTA has eight warps:
 //   warp 0     producer: per 512-token block of the segment, one TMA tile of
 //              the C_lo rows (K, and V in the value pass; 32-byte rows,
 //              32-byte swizzle) unless every token of the block is full-rank;
-//              the block's full-rank tokens join a queue, and every 128 of them
-//              (and the rest at the segment's end) are gathered by cp.async as
-//              128-byte rows (C_lo + C_hi, 128-byte swizzle) into a HI tile;
-//              the unit's q~ (bf16 hi and lo planes) by bulk copy per segment
+//              the block's full-rank tokens are counted, and every 128 of them
+//              (and the rest at the segment's end) make a HI tile: a run of the
+//              unit's list of full-rank positions (hipos_kernel, ahead of the
+//              passes) lands in the tile's descriptor by bulk copy; the unit's
+//              q~ (bf16 hi and lo planes) by bulk copy per segment
 //   warp 1     tensor memory owner and MMA issuer: per tile, S = C q~^T with
 //              tokens on M = 128 (the tensor-memory lanes) and the query heads
 //              on N, as two bf16 products (q~ hi, q~ lo) accumulated in fp32:
@@ -39,6 +40,8 @@
 //              per-token work; in the value pass it writes its row of p' to
 //              shared memory, and the warp adds u^T += C_V^T P for its 32 tokens
 //              with mma.sync (ranks on M, heads on N).
+//   warps 6-7  gather: a HI tile's rows, 128 bytes each (C_lo + C_hi, 128-byte
+//              swizzle), by cp.async from the positions in its descriptor
 // Every ring slot carries a descriptor of its tile; one barrier triple per slot
 // (data landed / scores ready / slot free) orders the roles, and a slot's
 // tensor-memory score buffer is reused with the slot.
@@ -61,9 +64,7 @@ constexpr int kGatherThreads = 64;
 constexpr int kND = 12;                     // descriptor ring (written by the producer, freed by the consumers)
 constexpr int kNQ = 4;                      // queue of full-rank tiles handed to the gather warp
 constexpr int kTile = 128;          // tokens per tensor-memory tile (M of the score MMA)
-constexpr int kHiRing = 1024;       // producer's queue of pending full-rank token positions
-constexpr int kMaskWin = 1024;      // producer's window of mask words (32768 tokens)
-constexpr int kDescInts = 8 + 64;   // header + up to 16 mask words (LO) or 128 uint16 positions (HI)
+constexpr int kDescInts = 8 + 68;   // header + up to 16 mask words (LO) or 8 + 128 uint16 positions (HI)
 constexpr int kTypeLo = 0, kTypeHi = 1, kTypeEnd = 2;
 constexpr int kFlagFirst = 1 << 8, kFlagLast = 1 << 9;
 constexpr float kRefInit = -1e30f;
@@ -71,26 +72,27 @@ constexpr float kLazy = 8.f;        // a per-thread reference max moves when a l
 
 // Geometry per (query heads NH, pass).  NH is the unit's Hg rounded up to 4, 8, 16 or 32.
 // Three rings per CTA, released independently:
-//   K slots   the C_K part of a tile (statistics pass: a LO tile of 512 tokens of 32-byte rows
-//             or a HI tile of 128 tokens of 128-byte rows, 16 KB; value pass: 256 or 64 tokens,
-//             8 KB), freed by the score MMA's completion (tcgen05.commit) -- the consumers
-//             never read them
-//   V slots   the C_V part of a value-pass tile (8 KB), freed by the consumers after their V sums
+//   K slots   the C_K part of a tile: a LO tile of 512 tokens of 32-byte rows or a HI tile of 128
+//             tokens of 128-byte rows, 16 KB, freed by the score MMA's completion
+//             (tcgen05.commit) -- the consumers never read them
+//   V slots   the C_V part of a value-pass tile (the same geometry, 16 KB), freed by the consumers
+//             after their V sums
 //   S buffers tensor-memory scores of a tile (kSub x kNHP columns), freed by the consumers
-// A 64-token HI tile of the value pass still runs the 128-row score MMA; rows 64-127 read the
-// 8 KB that follow the slot and their scores are never used.
 template <int NH, bool VALUE>
 struct Cfg {
     static constexpr int kNHP = NH < 16 ? 16 : NH;                  // N of the score MMA
     static constexpr int kPH = NH < 8 ? 8 : NH;                      // heads per row of P (mma.sync n8 tiles)
     static constexpr int kBlocks = NH <= 16 ? 2 : 1;                 // resident CTAs per SM
-    static constexpr int kLoTok = VALUE ? 256 : 512;                 // tokens per LO tile
-    static constexpr int kHiTok = VALUE ? 64 : 128;                  // tokens per HI tile
+    static constexpr int kLoTok = 512;                               // tokens per LO tile
+    static constexpr int kHiTok = 128;                               // tokens per HI tile
     static constexpr int kSub = kLoTok / kTile;                      // 128-token sub-tiles per LO tile
-    static constexpr int kKBytes = VALUE ? 8192 : 16384;
-    static constexpr int kVBytes = 8192;
-    static constexpr int kNK = VALUE ? (NH <= 16 ? 5 : 8) : (NH <= 16 ? 5 : 10);
-    static constexpr int kNV = VALUE ? (NH <= 16 ? 4 : 8) : 1;
+    static constexpr int kKBytes = 16384;
+    static constexpr int kVBytes = 16384;
+    // the V slots stay with a tile until its consumers are done, the K slots only until its score
+    // MMA is (which runs up to kNS tiles ahead of them): the value pass holds more V than K slots
+    static constexpr int kNK = VALUE ? (NH <= 16 ? 2 : 5) : (NH <= 16 ? 5 : 10);
+    static constexpr int kNV = VALUE ? (NH <= 16 ? 3 : 5) : 1;
+    static constexpr int kMaskWin = VALUE && NH <= 16 ? 512 : 1024;   // producer's window of mask words
     static constexpr int kNS = 4;
     static constexpr int kSCols = kSub * kNHP;                       // tensor-memory columns of one S buffer
     static constexpr int kTmemCols = kNS * kSCols;                   // 128, 256 or 512
@@ -105,10 +107,12 @@ struct Params {
     const int8_t *EK, *EV;                           // their exponents [units][T][2]
     const unsigned char *qt;        // [units][qblock_bytes(Hg)]: q~ hi, lo planes (from text_kernel)
     const uint32_t *mask;           // [units][nwords]
+    const uint16_t *hipos;          // [units][Tp]: each unit's full-rank token positions, ascending (hipos_kernel)
+    const int *hicnt;               // [units][tpu]: full-rank tokens of the unit before each tile
     const float *ustat;             // value pass: [units][Hg][2] = (M, 1/L)
     float *part;                    // stats: [units][nslot][Hg][2] = (m, l); value: [units][nslot][Hg][64] = u
     float *mass;                    // value pass: [units][T] or null
-    int units, T, Hg, nwords, tpu, nslot, rank0;
+    int units, T, Hg, nwords, tpu, nslot, rank0, Tp;
     long long ntiles;               // units * tpu
 };
 
@@ -122,12 +126,11 @@ template <int NH, bool VALUE>
 struct Smem {
     using C = Cfg<NH, VALUE>;
     alignas(1024) unsigned char kslot[C::kNK][C::kKBytes];
-    alignas(1024) unsigned char vslot[C::kNV][VALUE ? C::kVBytes : 16];   // follows the K slots (see Cfg)
+    alignas(1024) unsigned char vslot[C::kNV][VALUE ? C::kVBytes : 16];
     alignas(1024) unsigned char qbuf[2][2][C::kNHP * 128];          // [q slot][hi, lo][rows of 128 B]
     int kdesc[kND][kDescInts];                                      // tile descriptors, written once by the producer
     int hiq[kNQ][8];                                                // full-rank tiles for the gather warp
-    uint32_t mwin[kMaskWin];                                        // producer's window of the CTA's mask words
-    uint16_t hi_ring[kHiRing];
+    uint32_t mwin[C::kMaskWin];                                     // producer's window of the CTA's mask words
     unsigned char pbuf[VALUE ? 4 : 1][VALUE ? 32 * C::kPH * 2 : 16];   // value pass: P rows of each consumer warp
     float merge[VALUE ? 3 : 4][VALUE ? NH * 64 : NH * 2];           // partial merge across the consumer warps
     uint64_t kfull[C::kNK], kempty[C::kNK], vfull[C::kNV], vempty[C::kNV], sfull[C::kNS], sfree[C::kNS];
@@ -258,7 +261,6 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
     if (warp == 0) {
         // =============================================================== producer
         uint32_t seq = 0, qseq = 0;
-        unsigned hi_head = 0, hi_tail = 0;
         bool ok = true;
         // wait until the K slot (and, in the value pass, the V slot) of tile `seq` may be refilled
         auto acquire_k = [&](int ks) -> bool {
@@ -274,9 +276,9 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                                  (min(p.T, (int)((x1 - 1) % p.tpu + 1) * kTile) + 31) / 32;
         long long wbase = -1;
         auto mask_words = [&](long long gw, int nw) -> const uint32_t * {
-            if (wbase < 0 || gw < wbase || gw + nw > wbase + kMaskWin) {
+            if (wbase < 0 || gw < wbase || gw + nw > wbase + C::kMaskWin) {
                 wbase = gw;
-                const int cnt = (int)min((long long)kMaskWin, gw_end - gw);
+                const int cnt = (int)min((long long)C::kMaskWin, gw_end - gw);
                 __syncwarp();
                 for (int i = lane; i < cnt; i += 32) sm.mwin[i] = __ldg(p.mask + gw + i);
                 __syncwarp();
@@ -287,19 +289,33 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
         auto acquire_d = [&](int ds) -> bool {
             return seq < (uint32_t)kND || mbar_wait(&sm.dfree[ds], ((seq / kND) - 1) & 1u, abort);
         };
-        // hand a full-rank tile (K slot ks, V slot vs, descriptor ds) to the gather warp; ks < 0 ends it
+        // hand a full-rank tile (K slot ks, V slot vs, descriptor ds) to the gather warps; ks < 0 ends
+        // them.  A tile's token positions (pos_bytes from src) land in its descriptor by a bulk copy
+        // that completes on the queue entry's barrier, so the gather warps start once they are there.
         uint32_t hseq = 0;
-        auto push_gather = [&](int ks, int vs, int ds, int n, int unit, int type, int tok) -> bool {
+        auto push_gather = [&](int ks, int vs, int ds, int n, int unit, int skew, const uint16_t *src,
+                               uint32_t pos_bytes) -> bool {
             const int hq = hseq % kNQ;
             if (hseq >= (uint32_t)kNQ && !mbar_wait(&sm.gfree[hq], ((hseq / kNQ) - 1) & 1u, abort)) return false;
             if (lane == 0) {
                 int *e = sm.hiq[hq];
-                e[0] = ks; e[1] = vs; e[2] = ds; e[3] = n; e[4] = unit; e[5] = type; e[6] = tok;
-                mbar_arrive(&sm.gready[hq]);
+                e[0] = ks; e[1] = vs; e[2] = ds; e[3] = n; e[4] = unit; e[5] = skew;
+                if (pos_bytes > 0) {
+                    fence_proxy_async();   // the descriptor's earlier readers went through the generic proxy
+                    mbar_arrive_tx(&sm.gready[hq], pos_bytes);
+                    bulk_g2s(sm.kdesc[ds] + 8, src, pos_bytes, &sm.gready[hq]);
+                } else {
+                    mbar_arrive(&sm.gready[hq]);
+                }
             }
             ++hseq;
             return true;
         };
+        // full-rank tokens of the CTA's first unit before its first tile: a unit's list of full-rank
+        // positions starts at its first token, and only the CTA's first segment can start inside a unit
+        int hi_first = 0;
+        if (lane == 0 && x0 < x1 && x0 % p.tpu != 0) hi_first = __ldg(p.hicnt + x0);
+        hi_first = __shfl_sync(0xffffffffu, hi_first, 0);
         long long x = x0;
         while (ok && x < x1) {
             const int unit = (int)(x / p.tpu);
@@ -308,6 +324,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             const int tok0 = (int)(x - (long long)unit * p.tpu) * kTile;
             const int tok1 = min(p.T, (int)(xe - (long long)unit * p.tpu) * kTile);
             const int pslot = (int)(blockIdx.x - cta_of_tile((long long)unit * p.tpu, CT, NT));
+            const size_t hi_base = (size_t)unit * p.Tp + (x == x0 ? hi_first : 0);
             x = xe;
             // the unit's q~ into the next q slot
             const int qs = qseq & 1;
@@ -322,9 +339,10 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             }
             ++qseq;
             bool first = true;
+            unsigned hi_head = 0, hi_tail = 0;   // the segment's full-rank tokens: emitted, passed
             for (int tok = tok0; tok < tok1 && ok; tok += C::kLoTok) {
                 const int n = min(C::kLoTok, tok1 - tok);
-                // the block's mask words (bits past n cleared) and its full-rank tokens
+                // the block's mask words (bits past n cleared) and its count of full-rank tokens
                 const uint32_t *mw = mask_words((long long)unit * p.nwords + (tok >> 5), (n + 31) >> 5);
                 uint32_t wd = 0u;
                 if (lane < C::kLoTok / 32 && 32 * lane < n) {
@@ -332,25 +350,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                     const int nb = n - 32 * lane;
                     if (nb < 32) wd &= (1u << nb) - 1u;
                 }
-                const int c = __popc(wd);
-                int incl = c;
-                #pragma unroll
-                for (int d = 1; d < 32; d <<= 1) {
-                    const int v = __shfl_up_sync(0xffffffffu, incl, d);
-                    if (lane >= d) incl += v;
-                }
-                const int nhi = __shfl_sync(0xffffffffu, incl, 31);
-                {
-                    unsigned r = hi_tail + (unsigned)(incl - c);
-                    uint32_t bits = wd;
-                    while (bits) {
-                        sm.hi_ring[r % kHiRing] = (uint16_t)(tok + 32 * lane + __ffs(bits) - 1);
-                        ++r;
-                        bits &= bits - 1u;
-                    }
-                }
+                const int nhi = (int)__reduce_add_sync(0xffffffffu, (unsigned)__popc(wd));
                 hi_tail += (unsigned)nhi;
-                __syncwarp();
                 const bool final_blk = tok + C::kLoTok >= tok1;
                 const unsigned pend = hi_tail - hi_head;
                 const int hi_now = (int)(pend / C::kHiTok) + ((final_blk && (pend % C::kHiTok) != 0) ? 1 : 0);
@@ -393,8 +394,9 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                             for (int b = 0; b < nb; ++b)
                                 tma_3d(sm.kslot[ks] + 8192 * b, &p.tm_ck, 0, tok + 256 * b, unit, &sm.kfull[ks]);
                             if (VALUE) {
-                                mbar_arrive_tx(&sm.vfull[vs], 8192u);
-                                tma_3d(sm.vslot[vs], &p.tm_cv, 0, tok, unit, &sm.vfull[vs]);
+                                mbar_arrive_tx(&sm.vfull[vs], (uint32_t)nb * 8192u);
+                                for (int b = 0; b < nb; ++b)
+                                    tma_3d(sm.vslot[vs] + 8192 * b, &p.tm_cv, 0, tok + 256 * b, unit, &sm.vfull[vs]);
                             }
                         } else {
                             mbar_arrive(&sm.kfull[ks]);
@@ -409,24 +411,26 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                     ++seq;
                 }
                 for (int i = 0; i < hi_now && ok; ++i) {
-                    // ------------------------------------------------ HI tile: positions here, rows by the gather warp
+                    // ------------------------------------------------ HI tile: positions and rows by the gather warps
                     const int ks = seq % kNK, ds = seq % kND, vs = seq % kNV;
                     if (!acquire_k(ks) || !acquire_d(ds) || (VALUE && !acquire_v(vs))) { ok = false; break; }
                     const int nh = (int)min((unsigned)C::kHiTok, hi_tail - hi_head);
+                    // the bulk copy starts on a 16-byte boundary of the list (p.Tp is a multiple of 8):
+                    // the tile's first position is entry `skew` of the copied run
+                    const size_t idx = hi_base + hi_head;
+                    const int skew = (int)(idx & 7u);
+                    const uint32_t bytes = ((uint32_t)(skew + nh) * 2u + 15u) & ~15u;
                     int *d = sm.kdesc[ds];
-                    uint16_t *pos = reinterpret_cast<uint16_t *>(d + 8);
                     if (lane == 0) {
                         d[0] = kTypeHi | (first ? kFlagFirst : 0) | ((final_blk && i == hi_now - 1) ? kFlagLast : 0);
-                        d[1] = unit; d[2] = 0; d[3] = nh; d[4] = pslot; d[5] = qs;
-                    }
-                    #pragma unroll
-                    for (int k = 0; k < C::kHiTok / 32; ++k) {
-                        const int r = lane + 32 * k;
-                        pos[r] = r < nh ? sm.hi_ring[(hi_head + r) % kHiRing] : (uint16_t)0;
+                        d[1] = unit; d[2] = skew; d[3] = nh; d[4] = pslot; d[5] = qs;
                     }
                     first = false;
                     __syncwarp();
-                    if (!push_gather(ks, vs, ds, nh, unit, kTypeHi, 0)) { ok = false; break; }
+                    if (!push_gather(ks, vs, ds, nh, unit, skew, p.hipos + (idx - (size_t)skew), bytes)) {
+                        ok = false;
+                        break;
+                    }
                     mbar_arrive(&sm.kfull[ks]);       // releases this lane's descriptor writes
                     if (VALUE) mbar_arrive(&sm.vfull[vs]);
                     hi_head += (unsigned)nh;
@@ -443,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 __syncwarp();
                 mbar_arrive(&sm.kfull[ks]);
                 if (lane == 0) mbar_arrive_cnt(&sm.kfull[ks], kGatherThreads);
-                ended = push_gather(-1, 0, 0, 0, 0, kTypeEnd, 0);
+                ended = push_gather(-1, 0, 0, 0, 0, 0, nullptr, 0u);
             }
             ok = ended;
         }
@@ -478,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             #pragma unroll 4
             for (int r = r0; r < C::kHiTok; r += kGatherThreads / 8) {
                 const bool valid = r < n;
-                const uint16_t *src = base + (ubase + pos[r]) * stride;
+                const uint16_t *src = base + (ubase + (valid ? pos[r] : 0)) * stride;
                 unsigned char *dp = dst + r * 128 + dcol;
                 if (zero) cp_async16_zfill(dp, src, valid);
                 else if (valid) cp_async16(dp, src);
@@ -489,12 +493,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
             const int hq = h % kNQ;
             if (!mbar_wait(&sm.gready[hq], (h / kNQ) & 1u, abort)) break;
             const int *e = sm.hiq[hq];
-            const int ks = e[0], vs = e[1], ds = e[2], n = e[3], unit = e[4];
+            const int ks = e[0], vs = e[1], ds = e[2], n = e[3], unit = e[4], skew = e[5];
             mbar_arrive(&sm.gfree[hq]);
             if (ks < 0) break;
-            // the positions stay valid until the consumers free the descriptor, which needs this
-            // tile's data first
-            const uint16_t *pos = reinterpret_cast<const uint16_t *>(sm.kdesc[ds] + 8);
+            // the positions (landed with the queue entry) stay valid until the consumers free the
+            // descriptor, which needs this tile's data first
+            const uint16_t *pos = reinterpret_cast<const uint16_t *>(sm.kdesc[ds] + 8) + skew;
             const size_t ubase = (size_t)unit * p.T;
             if constexpr (Q4) {
                 // dequantize a HI tile into the layout of the 16-bit path (128-byte rows, 128-byte
@@ -712,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                     pos = d[2] + r;
                 } else {
                     take = r < n;
-                    pos = reinterpret_cast<const uint16_t *>(d + 8)[r];
+                    pos = r < n ? reinterpret_cast<const uint16_t *>(d + 8)[d[2] + r] : 0;
                 }
                 const float (&sc)[NH] = scv[j];
                 if (!VALUE) {
@@ -911,6 +915,62 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
         tmem_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
+}
+
+// ------------------------------------------------------------------ full-rank positions
+
+// Each unit's full-rank token positions in ascending order (hipos[unit][0 .. count)) and, per
+// 128-token tile, the count of full-rank tokens before it (hicnt[unit][tile]): the visual
+// passes' HI tiles are runs of that list.  One block per unit (blockIdx.y picks the mask: the
+// visual tokens', or the compressed text tokens' own); thread t scans a contiguous run of words.
+constexpr int kHpThreads = 256;
+struct HiposParams {
+    const uint32_t *mask;    // [units][nwords]
+    uint16_t *hipos;         // [units][Tp]
+    int *hicnt;              // [units][tpu]
+    int units, T, nwords, tpu, Tp;
+};
+
+__global__ void __launch_bounds__(kHpThreads) hipos_kernel(const HiposParams a, const HiposParams b) {
+    griddep_launch_dependents();
+    const HiposParams &p = blockIdx.y == 0 ? a : b;
+    const int unit = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ int wsum[kHpThreads / 32];
+    if (unit < p.units) {
+        const int wpt = (p.nwords + kHpThreads - 1) / kHpThreads;
+        const int w0 = min(p.nwords, (int)threadIdx.x * wpt), w1 = min(p.nwords, w0 + wpt);
+        const uint32_t *mk = p.mask + (size_t)unit * p.nwords;
+        auto word = [&](int w) -> uint32_t {
+            uint32_t v = __ldg(mk + w);
+            const int nb = p.T - 32 * w;
+            if (nb < 32) v &= (1u << nb) - 1u;
+            return v;
+        };
+        int c = 0;
+        for (int w = w0; w < w1; ++w) c += __popc(word(w));
+        int incl = c;
+        #pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        int base = incl - c;
+        for (int i = 0; i < warp; ++i) base += wsum[i];
+        uint16_t *out = p.hipos + (size_t)unit * p.Tp;
+        int *cnt = p.hicnt + (size_t)unit * p.tpu;
+        for (int w = w0; w < w1; ++w) {
+            if ((w & 3) == 0) cnt[w >> 2] = base;   // a tile is four words
+            uint32_t bits = word(w);
+            while (bits) {
+                out[base++] = (uint16_t)(32 * w + __ffs(bits) - 1);
+                bits &= bits - 1u;
+            }
+        }
+    }
+    // the next kernel's wait then also covers the kernel before this one
+    griddep_wait();
 }
 
 // ------------------------------------------------------------------ combine
