@@ -83,6 +83,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     return mbar_wait_for(bar, parity, abort, kWaitCycles);
 }
 
+// Named barrier `id` over `count` threads (a multiple of 32) of the block.
+__device__ __forceinline__ void named_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(count) : "memory");
+}
+
+// Global fp32 add without a return value (performed at L2).
+__device__ __forceinline__ void red_add_f32(float *addr, float v) {
+    asm volatile("red.global.add.f32 [%0], %1;" :: "l"(addr), "f"(v) : "memory");
+}
+
 // ------------------------------------------------------ programmatic dependent launch
 // A kernel launched with programmatic stream serialization may start while the
 // previous kernel on the stream is still running; it must not touch that

@@ -178,12 +178,18 @@ cudaError_t launch_pdl(void (*kernel)(Params...), int grid, int threads, size_t 
 template <bool VALUE, bool Q4>
 cudaError_t launch_rs_q(int NH, const rs::Params &rp, int grid, cudaStream_t st) {
     switch (NH) {
-        case 4: return launch_pdl(rs::rs_kernel<4, VALUE, Q4>, grid, rs::kThreads, rs::smem_bytes<4, VALUE>(), st, rp);
-        case 8: return launch_pdl(rs::rs_kernel<8, VALUE, Q4>, grid, rs::kThreads, rs::smem_bytes<8, VALUE>(), st, rp);
+        case 4:
+            return launch_pdl(rs::rs_kernel<4, VALUE, Q4>, grid, rs::Cfg<4, VALUE>::kThreads, rs::smem_bytes<4, VALUE>(),
+                              st, rp);
+        case 8:
+            return launch_pdl(rs::rs_kernel<8, VALUE, Q4>, grid, rs::Cfg<8, VALUE>::kThreads, rs::smem_bytes<8, VALUE>(),
+                              st, rp);
         case 16:
-            return launch_pdl(rs::rs_kernel<16, VALUE, Q4>, grid, rs::kThreads, rs::smem_bytes<16, VALUE>(), st, rp);
+            return launch_pdl(rs::rs_kernel<16, VALUE, Q4>, grid, rs::Cfg<16, VALUE>::kThreads, rs::smem_bytes<16, VALUE>(),
+                              st, rp);
         default:
-            return launch_pdl(rs::rs_kernel<32, VALUE, Q4>, grid, rs::kThreads, rs::smem_bytes<32, VALUE>(), st, rp);
+            return launch_pdl(rs::rs_kernel<32, VALUE, Q4>, grid, rs::Cfg<32, VALUE>::kThreads, rs::smem_bytes<32, VALUE>(),
+                              st, rp);
     }
 }
 template <bool VALUE>
@@ -519,9 +525,12 @@ kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t
     }
     {
         // each unit's full-rank positions, for the HI tiles of both passes
-        const rs::HiposParams ha{mask, hipos, hicnt, pl.units, T, pl.nwords, pl.tpu, pl.Tp};
+        // with two consumer groups (32 heads) the value pass adds the groups' shares of a token's
+        // attention mass into the zeroed output
+        float *mass0 = pl.NH >= 32 ? mass : nullptr;
+        const rs::HiposParams ha{mask, hipos, hicnt, mass0, pl.units, T, pl.nwords, pl.tpu, pl.Tp};
         const rs::HiposParams hb =
-            L_c > 0 ? rs::HiposParams{mask2, hipos2, hicnt2, pl.units, L_c, pl.nwords2, pl.tpu2, pl.Tp2} : ha;
+            L_c > 0 ? rs::HiposParams{mask2, hipos2, hicnt2, nullptr, pl.units, L_c, pl.nwords2, pl.tpu2, pl.Tp2} : ha;
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3((unsigned)pl.units, L_c > 0 ? 2u : 1u);
         cfg.blockDim = dim3((unsigned)rs::kHpThreads);

@@ -57,9 +57,8 @@ namespace kvpack {
 namespace decode {
 namespace rs {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
 constexpr int kGatherWarp = 6;              // warps 6 and 7 gather the full-rank tokens' rows
+constexpr int kConsumer2 = 8;               // warps 8-11: the second consumer group (kSplit = 2)
 constexpr int kGatherThreads = 64;
 constexpr int kND = 12;                     // descriptor ring (written by the producer, freed by the consumers)
 constexpr int kNQ = 4;                      // queue of full-rank tiles handed to the gather warp
@@ -81,7 +80,12 @@ constexpr float kLazy = 8.f;        // a per-thread reference max moves when a l
 template <int NH, bool VALUE>
 struct Cfg {
     static constexpr int kNHP = NH < 16 ? 16 : NH;                  // N of the score MMA
-    static constexpr int kPH = NH < 8 ? 8 : NH;                      // heads per row of P (mma.sync n8 tiles)
+    // consumer warp groups: each has four warps (one per tensor-memory lane quarter) and NH / kSplit heads
+    // (measured: two groups pay off at 32 heads; at 16 they run no faster than one group of two CTAs per SM)
+    static constexpr int kSplit = NH >= 32 ? 2 : 1;
+    static constexpr int kHS = NH / kSplit;
+    static constexpr int kPHS = kHS < 8 ? 8 : kHS;                   // heads per row of a group's P (mma.sync n8 tiles)
+    static constexpr int kThreads = (8 + 4 * (kSplit - 1)) * 32;
     static constexpr int kBlocks = NH <= 16 ? 2 : 1;                 // resident CTAs per SM
     static constexpr int kLoTok = 512;                               // tokens per LO tile
     static constexpr int kHiTok = 128;                               // tokens per HI tile
@@ -131,7 +135,7 @@ struct Smem {
     int kdesc[kND][kDescInts];                                      // tile descriptors, written once by the producer
     int hiq[kNQ][8];                                                // full-rank tiles for the gather warp
     uint32_t mwin[C::kMaskWin];                                     // producer's window of the CTA's mask words
-    unsigned char pbuf[VALUE ? 4 : 1][VALUE ? 32 * C::kPH * 2 : 16];   // value pass: P rows of each consumer warp
+    unsigned char pbuf[VALUE ? 4 * C::kSplit : 1][VALUE ? 32 * C::kPHS * 2 : 16];   // value pass: P rows per consumer warp
     float merge[VALUE ? 3 : 4][VALUE ? NH * 64 : NH * 2];           // partial merge across the consumer warps
     uint64_t kfull[C::kNK], kempty[C::kNK], vfull[C::kNV], vempty[C::kNV], sfull[C::kNS], sfree[C::kNS];
     uint64_t dfree[kND], gready[kNQ], gfree[kNQ];
@@ -204,9 +208,9 @@ __device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, float (&v)[32]) {
 // HI, into the same shared-memory layouts the TMA and cp.async copies produce, so the score MMA
 // and the consumers are unchanged.
 template <int NH, bool VALUE, bool Q4>
-__global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(const __grid_constant__ Params p) {
     using C = Cfg<NH, VALUE>;
-    constexpr int kNK = C::kNK, kNV = C::kNV, kNS = C::kNS, kNHP = C::kNHP, kPH = C::kPH;
+    constexpr int kNK = C::kNK, kNV = C::kNV, kNS = C::kNS, kNHP = C::kNHP;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t base0 = smem_u32(smem_raw);
     Smem<NH, VALUE> &sm = *reinterpret_cast<Smem<NH, VALUE> *>(smem_raw + ((1024u - (base0 & 1023u)) & 1023u));
@@ -224,16 +228,16 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
         }
         for (int s = 0; s < kNV; ++s) {
             mbar_init(&sm.vfull[s], 32 + kGatherThreads);
-            mbar_init(&sm.vempty[s], 4);
+            mbar_init(&sm.vempty[s], 4 * C::kSplit);
         }
-        for (int s = 0; s < kND; ++s) mbar_init(&sm.dfree[s], 4);
+        for (int s = 0; s < kND; ++s) mbar_init(&sm.dfree[s], 4 * C::kSplit);
         for (int s = 0; s < kNQ; ++s) {
             mbar_init(&sm.gready[s], 1);
             mbar_init(&sm.gfree[s], kGatherThreads);
         }
         for (int s = 0; s < kNS; ++s) {
             mbar_init(&sm.sfull[s], 1);
-            mbar_init(&sm.sfree[s], 4);
+            mbar_init(&sm.sfree[s], 4 * C::kSplit);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.qfull[s], 1);
@@ -245,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
     }
     // q~ rows past Hg stay zero for the whole kernel (the bulk copies write Hg rows), so the
     // scores of padding heads are exactly zero
-    for (int i = threadIdx.x; i < 2 * 2 * kNHP * 128 / 16; i += kThreads)
+    for (int i = threadIdx.x; i < 2 * 2 * kNHP * 128 / 16; i += C::kThreads)
         reinterpret_cast<uint4 *>(&sm.qbuf[0][0][0])[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async();
     if (warp == 1) tmem_alloc(&sm.tmem_base, C::kTmemCols);
@@ -467,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 while (!mbar_try_wait(&sm.vfull[k % kNV], (k / kNV) & 1u) && clock64() - t0 < kWaitCycles) {}
             }
         }
-    } else if (warp >= kGatherWarp) {
+    } else if (warp >= kGatherWarp && warp < kGatherWarp + 2) {
         // =============================================================== gather warps
         // 128-byte rows (C_lo + C_hi, 16-byte chunk c of row r at c ^ (r & 7)) of a HI tile's
         // tokens into its K slot (and V slot); V rows past n are zero-filled (their p is zero, and
@@ -638,17 +642,21 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
         __syncwarp();
     } else {
         // =============================================================== consumers
+        // kSplit groups of four warps share each tile: group cg takes heads [cg HS, cg HS + HS)
+        constexpr int HS = C::kHS, PHS = C::kPHS, NCW = 4 * C::kSplit;
         const int q = warp & 3;                       // tensor-memory lane quarter
+        const int cg = warp >= kConsumer2 ? 1 : 0;
+        const int h0 = cg * HS;
         const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
         const int g = lane >> 2, tig = lane & 3;
         uint32_t seq = 0;
         // per-segment state
-        float m[NH], l[NH];                            // stats pass: this thread's reference max and sum per head
-        float Mh[NH], ILh[NH];                         // value pass: the unit's (M, 1/L) per head
-        float u[4][kPH / 8][4];                        // value pass: u^T (ranks on M, heads on N) of this warp
+        float m[HS], l[HS];                            // stats pass: this thread's reference max and sum per head
+        float Mh[HS], ILh[HS];                         // value pass: the unit's (M, 1/L) per head
+        float u[4][PHS / 8][4];                        // value pass: u^T (ranks on M, heads on N) of this warp
         (void)m; (void)l; (void)Mh; (void)ILh; (void)u;
         int unit = 0, pslot = 0;
-        unsigned char *pb = sm.pbuf[VALUE ? q : 0];
+        unsigned char *pb = sm.pbuf[VALUE ? 4 * cg + q : 0];
         const uint32_t pb_s = smem_u32(pb);
         bool failed = false;
         while (!failed) {
@@ -665,48 +673,38 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 pslot = d[4];
                 if (VALUE) {
                     #pragma unroll
-                    for (int h = 0; h < NH; ++h) {
+                    for (int h = 0; h < HS; ++h) {
                         float2 st = make_float2(0.f, 0.f);
-                        if (h < p.Hg) st = __ldg(reinterpret_cast<const float2 *>(p.ustat + ((size_t)unit * p.Hg + h) * 2));
+                        if (h0 + h < p.Hg)
+                            st = __ldg(reinterpret_cast<const float2 *>(p.ustat + ((size_t)unit * p.Hg + h0 + h) * 2));
                         Mh[h] = st.x;
                         ILh[h] = st.y;
                     }
                     #pragma unroll
                     for (int a = 0; a < 4; ++a)
                         #pragma unroll
-                        for (int b = 0; b < kPH / 8; ++b) u[a][b][0] = u[a][b][1] = u[a][b][2] = u[a][b][3] = 0.f;
+                        for (int b = 0; b < PHS / 8; ++b) u[a][b][0] = u[a][b][1] = u[a][b][2] = u[a][b][3] = 0.f;
                 } else {
                     #pragma unroll
-                    for (int h = 0; h < NH; ++h) { m[h] = kRefInit; l[h] = 0.f; }
+                    for (int h = 0; h < HS; ++h) { m[h] = kRefInit; l[h] = 0.f; }
                 }
             }
             const bool has_s = type == kTypeHi || !p.rank0;
             const int nsub = type == kTypeLo ? (n + kTile - 1) / kTile : 1;
             const uint32_t vb = smem_u32(sm.vslot[vs]);
             bool v_ready = false;
-            // the scores of one sub-tile are loaded from tensor memory before each wait
-            constexpr int kLd = 1;   // measured: batching the loads of several sub-tiles was slower (larger code)
-            for (int sub0 = 0; sub0 < nsub && !failed; sub0 += kLd) {
-                float scv[kLd][NH];
-                #pragma unroll
-                for (int j = 0; j < kLd; ++j) {
-                    const int sub = sub0 + j;
-                    if (has_s && sub < nsub && sub * kTile + 32 * q < n) {
-                        constexpr int NL = NH < 4 ? 4 : NH;
-                        float v[NL];
-                        tmem_ld<NL>(tmem + lane_addr + (uint32_t)(sb * C::kSCols + sub * kNHP), v);
-                        #pragma unroll
-                        for (int h = 0; h < NH; ++h) scv[j][h] = v[h];
-                    } else {
-                        #pragma unroll
-                        for (int h = 0; h < NH; ++h) scv[j][h] = 0.f;
-                    }
+            // the scores of one sub-tile (this group's heads) are loaded from tensor memory before each wait
+            for (int sub = 0; sub < nsub && !failed; ++sub) {
+                if (sub * kTile + 32 * q >= n) continue;   // no token of this warp here
+                constexpr int NL = HS < 4 ? 4 : HS;
+                float sc[NL];
+                if (has_s) {
+                    tmem_ld<NL>(tmem + lane_addr + (uint32_t)(sb * C::kSCols + sub * kNHP + h0), sc);
+                    tmem_wait_ld();
+                } else {
+                    #pragma unroll
+                    for (int h = 0; h < NL; ++h) sc[h] = 0.f;
                 }
-                if (has_s) tmem_wait_ld();
-                #pragma unroll
-                for (int j = 0; j < kLd; ++j) {
-                const int sub = sub0 + j;
-                if (sub >= nsub || sub * kTile + 32 * q >= n) continue;   // no token of this warp here
                 const int r = sub * kTile + 32 * q + lane;    // row of this thread's token in the tile
                 bool take;
                 int pos;
@@ -718,31 +716,30 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                     take = r < n;
                     pos = r < n ? reinterpret_cast<const uint16_t *>(d + 8)[d[2] + r] : 0;
                 }
-                const float (&sc)[NH] = scv[j];
                 if (!VALUE) {
                     // ---------------------------------------------------- stats
                     if (take) {
                         float mx = sc[0] - m[0];
                         #pragma unroll
-                        for (int h = 1; h < NH; ++h) mx = fmaxf(mx, sc[h] - m[h]);
+                        for (int h = 1; h < HS; ++h) mx = fmaxf(mx, sc[h] - m[h]);
                         if (mx > kLazy) {
                             #pragma unroll
-                            for (int h = 0; h < NH; ++h)
+                            for (int h = 0; h < HS; ++h)
                                 if (sc[h] > m[h]) {
                                     l[h] *= ex2(m[h] - sc[h]);
                                     m[h] = sc[h];
                                 }
                         }
                         #pragma unroll
-                        for (int h = 0; h < NH; ++h) l[h] += ex2(sc[h] - m[h]);
+                        for (int h = 0; h < HS; ++h) l[h] += ex2(sc[h] - m[h]);
                     }
                 } else {
                     // ---------------------------------------------------- value
-                    float pr[kPH];
+                    float pr[PHS];
                     float ms0 = 0.f, ms1 = 0.f;
                     #pragma unroll
-                    for (int h = 0; h < kPH; ++h) {
-                        if (h < NH) {
+                    for (int h = 0; h < PHS; ++h) {
+                        if (h < HS) {
                             const float e = take ? ex2(sc[h] - Mh[h]) : 0.f;
                             pr[h] = e;
                             if (h & 1) ms1 = fmaf(e, ILh[h], ms1);
@@ -751,49 +748,55 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                             pr[h] = 0.f;
                         }
                     }
-                    if (take && p.mass != nullptr) p.mass[(size_t)unit * p.T + pos] = ms0 + ms1;
+                    // the token's attention mass: each head group adds its heads' share into the
+                    // zeroed output (two addends onto zero: the same sum in either order)
+                    if (take && p.mass != nullptr) {
+                        float *dst = p.mass + (size_t)unit * p.T + pos;
+                        if (C::kSplit == 1) *dst = ms0 + ms1;
+                        else red_add_f32(dst, ms0 + ms1);
+                    }
                     const bool do_u = type == kTypeHi || !p.rank0;
                     if (do_u && !v_ready) {
                         if (!mbar_wait(&sm.vfull[vs], (seq / C::kNV) & 1u, abort)) { failed = true; break; }
                         v_ready = true;
                     }
                     if (do_u) {
-                        // this thread's P row (kPH bf16), 16-byte chunks swizzled against bank conflicts
+                        // this thread's P row (PHS bf16), 16-byte chunks swizzled against bank conflicts
                         const int prow = lane;
                         #pragma unroll
-                        for (int c = 0; c < kPH / 8; ++c) {
+                        for (int c = 0; c < PHS / 8; ++c) {
                             uint4 v;
                             v.x = pack_bf16(pr[8 * c + 0], pr[8 * c + 1]);
                             v.y = pack_bf16(pr[8 * c + 2], pr[8 * c + 3]);
                             v.z = pack_bf16(pr[8 * c + 4], pr[8 * c + 5]);
                             v.w = pack_bf16(pr[8 * c + 6], pr[8 * c + 7]);
                             int pc = c;
-                            if (kPH == 16) pc = c ^ ((prow >> 2) & 1);
-                            if (kPH == 32) pc = c ^ ((prow >> 1) & 3);
-                            *reinterpret_cast<uint4 *>(pb + prow * (kPH * 2) + pc * 16) = v;
+                            if (PHS == 16) pc = c ^ ((prow >> 2) & 1);
+                            if (PHS == 32) pc = c ^ ((prow >> 1) & 3);
+                            *reinterpret_cast<uint4 *>(pb + prow * (PHS * 2) + pc * 16) = v;
                         }
                         __syncwarp();
                         // u^T += C_V^T P over the warp's 32 tokens (two k-steps of 16)
                         #pragma unroll 1
                         for (int kk = 0; kk < 2; ++kk) {
-                            uint32_t bfr[kPH / 8][2];
+                            uint32_t bfr[PHS / 8][2];
                             #pragma unroll
-                            for (int np = 0; np < (kPH + 15) / 16; ++np) {
+                            for (int np = 0; np < (PHS + 15) / 16; ++np) {
                                 const int row = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
                                 int ch = 2 * np + (lane >> 4);
-                                if (kPH == 8) ch = 0;
+                                if (PHS == 8) ch = 0;
                                 int pc = ch;
-                                if (kPH == 16) pc = ch ^ ((row >> 2) & 1);
-                                if (kPH == 32) pc = ch ^ ((row >> 1) & 3);
+                                if (PHS == 16) pc = ch ^ ((row >> 2) & 1);
+                                if (PHS == 32) pc = ch ^ ((row >> 1) & 3);
                                 uint32_t r0, r1, r2, r3;
-                                if (kPH == 8) {
+                                if (PHS == 8) {
                                     // x2: tokens 0-7 and 8-15 of the 8 heads
                                     asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
-                                                 : "=r"(r0), "=r"(r1) : "r"(pb_s + row * (kPH * 2) + (pc << 4)));
+                                                 : "=r"(r0), "=r"(r1) : "r"(pb_s + row * (PHS * 2) + (pc << 4)));
                                     bfr[0][0] = r0;
                                     bfr[0][1] = r1;
                                 } else {
-                                    ldsm_x4_t(pb_s + row * (kPH * 2) + (pc << 4), r0, r1, r2, r3);
+                                    ldsm_x4_t(pb_s + row * (PHS * 2) + (pc << 4), r0, r1, r2, r3);
                                     bfr[2 * np][0] = r0;
                                     bfr[2 * np][1] = r1;
                                     bfr[2 * np + 1][0] = r2;
@@ -807,7 +810,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                                 const int ch = (lane >> 3) & 1;
                                 ldsm_x4_t(vb + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), a[0], a[1], a[2], a[3]);
                                 #pragma unroll
-                                for (int nt = 0; nt < kPH / 8; ++nt) mma_bf16(u[0][nt], a, bfr[nt][0], bfr[nt][1]);
+                                for (int nt = 0; nt < PHS / 8; ++nt) mma_bf16(u[0][nt], a, bfr[nt][0], bfr[nt][1]);
                             } else {
                                 #pragma unroll
                                 for (int mt = 0; mt < 4; ++mt) {
@@ -816,13 +819,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                                     const int ch = 2 * mt + ((lane >> 3) & 1);
                                     ldsm_x4_t(vb + row * 128 + ((ch ^ (row & 7)) << 4), a[0], a[1], a[2], a[3]);
                                     #pragma unroll
-                                    for (int nt = 0; nt < kPH / 8; ++nt) mma_bf16(u[mt][nt], a, bfr[nt][0], bfr[nt][1]);
+                                    for (int nt = 0; nt < PHS / 8; ++nt) mma_bf16(u[mt][nt], a, bfr[nt][0], bfr[nt][1]);
                                 }
                             }
                         }
                         __syncwarp();
                     }
-                }
                 }
             }
             if (failed) break;
@@ -844,7 +846,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                 if (!VALUE) {
                     // (m, l) per head: over the warp's lanes, then over the four warps in a fixed order
                     #pragma unroll
-                    for (int h = 0; h < NH; ++h) {
+                    for (int h = 0; h < HS; ++h) {
                         float mw = m[h];
                         #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) mw = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, o));
@@ -852,12 +854,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                         #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
                         if (lane == 0) {
-                            sm.merge[q][2 * h] = mw;
-                            sm.merge[q][2 * h + 1] = lw;
+                            sm.merge[q][2 * (h0 + h)] = mw;
+                            sm.merge[q][2 * (h0 + h) + 1] = lw;
                         }
                     }
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
-                    if (q == 0 && lane < NH && lane < p.Hg) {
+                    named_sync(1, 32 * NCW);
+                    if (q == 0 && cg == 0 && lane < NH && lane < p.Hg) {
                         float mx = sm.merge[0][2 * lane];
                         #pragma unroll
                         for (int w = 1; w < 4; ++w) mx = fmaxf(mx, sm.merge[w][2 * lane]);
@@ -868,40 +870,42 @@ __global__ void __launch_bounds__(kThreads, Cfg<NH, VALUE>::kBlocks) rs_kernel(c
                         dst[0] = mx;
                         dst[1] = sum;
                     }
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    named_sync(1, 32 * NCW);
                 } else {
-                    // u per head: warps 1-3 park theirs in shared memory, warp 0 adds them in order
+                    // u per head: warps 1-3 of each group park theirs in shared memory, warp 0 adds them
+                    // in order
                     if (q != 0) {
                         #pragma unroll
                         for (int mt = 0; mt < 4; ++mt)
                             #pragma unroll
-                            for (int nt = 0; nt < kPH / 8; ++nt)
+                            for (int nt = 0; nt < PHS / 8; ++nt)
                                 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
                                     const int rr = 16 * mt + g + 8 * (e >> 1), hh = 8 * nt + 2 * tig + (e & 1);
-                                    if (hh < NH) sm.merge[q - 1][hh * 64 + rr] = u[mt][nt][e];
+                                    if (hh < HS) sm.merge[q - 1][(h0 + hh) * 64 + rr] = u[mt][nt][e];
                                 }
                     }
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    named_sync(1, 32 * NCW);
                     if (q == 0) {
                         float *dst = p.part + ((size_t)unit * p.nslot + pslot) * p.Hg * 64;
                         #pragma unroll
                         for (int mt = 0; mt < 4; ++mt)
                             #pragma unroll
-                            for (int nt = 0; nt < kPH / 8; ++nt)
+                            for (int nt = 0; nt < PHS / 8; ++nt)
                                 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
                                     const int rr = 16 * mt + g + 8 * (e >> 1), hh = 8 * nt + 2 * tig + (e & 1);
-                                    if (hh < NH && hh < p.Hg) {
+                                    if (hh < HS && h0 + hh < p.Hg) {
+                                        const int H = h0 + hh;
                                         float v = u[mt][nt][e];
-                                        v += sm.merge[0][hh * 64 + rr];
-                                        v += sm.merge[1][hh * 64 + rr];
-                                        v += sm.merge[2][hh * 64 + rr];
-                                        dst[hh * 64 + rr] = v;
+                                        v += sm.merge[0][H * 64 + rr];
+                                        v += sm.merge[1][H * 64 + rr];
+                                        v += sm.merge[2][H * 64 + rr];
+                                        dst[H * 64 + rr] = v;
                                     }
                                 }
                     }
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    named_sync(1, 32 * NCW);
                 }
             }
             ++seq;
@@ -928,6 +932,7 @@ struct HiposParams {
     const uint32_t *mask;    // [units][nwords]
     uint16_t *hipos;         // [units][Tp]
     int *hicnt;              // [units][tpu]
+    float *mass;             // [units][T], zeroed here when the value pass adds into it (or null)
     int units, T, nwords, tpu, Tp;
 };
 
@@ -936,6 +941,10 @@ __global__ void __launch_bounds__(kHpThreads) hipos_kernel(const HiposParams a, 
     const HiposParams &p = blockIdx.y == 0 ? a : b;
     const int unit = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     __shared__ int wsum[kHpThreads / 32];
+    if (unit < p.units && p.mass != nullptr) {
+        float *ms = p.mass + (size_t)unit * p.T;
+        for (int i = threadIdx.x; i < p.T; i += kHpThreads) ms[i] = 0.f;
+    }
     if (unit < p.units) {
         const int wpt = (p.nwords + kHpThreads - 1) / kHpThreads;
         const int w0 = min(p.nwords, (int)threadIdx.x * wpt), w1 = min(p.nwords, w0 + wpt);
