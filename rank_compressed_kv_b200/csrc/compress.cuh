@@ -469,6 +469,17 @@ __global__ void __launch_bounds__(kEigThreads, 1) eig_kernel(EigParams p) {
     float *Qt = p.ws.Qt + (size_t)unit * kP * kN;
     unsigned char *Qgu = p.ws.Qg + (size_t)unit * kN * kQPitch;
 
+    // the Gram kernel writes the diagonal 128-row blocks of G and the blocks right of them; the
+    // blocks left of the diagonal are their transposes
+    {
+        float *Gw = p.ws.G + (size_t)unit * kN * kN;
+        for (int e = tid; e < kN * kN; e += kEigThreads) {
+            const int r = e / kN, c = e % kN;
+            if ((c >> 7) < (r >> 7)) Gw[e] = __ldcg(Gw + (size_t)c * kN + r);
+        }
+    }
+    __syncthreads();
+
     // Q0: fp32 columns in Qt and bf16 hi / lo rows in shared memory (thread = row)
     {
         const int r = tid;
@@ -699,9 +710,10 @@ __global__ void __launch_bounds__(kProjThreads, 1) project_kernel(const uint16_t
 //     K row; the band's own 128 features are the first two boxes of the stage);
 //   * tcgen05.commit releases a stage once its MMAs have read it;
 //   * four warps move the accumulator (one tensor-memory lane per feature row) to
-//     G and mirror the off-diagonal part into the lower triangle.
-// Long token ranges are split 4:3:2:1 over the bands (equal work per block) and
-// the splits add into a zeroed G with fp32 atomics.
+//     G (the eigen-solver fills the lower triangle from it).
+// When the units alone leave SMs idle, the bands' token ranges are split (more
+// splits for the wider bands, equal work per block, one wave of blocks) and the
+// splits add into a zeroed G with fp32 atomics.
 constexpr int kGtTok = 64;         // tokens per stage
 constexpr int kGtStages = 3;
 constexpr int kGtThreads = 128;
@@ -825,14 +837,6 @@ __global__ void __launch_bounds__(kGtThreads, 1) gram_tc_kernel(const __grid_con
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<float4 *>(grow + J0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
                 }
-                if (J0 >= 128 * (I + 1)) {   // off the diagonal block: mirror (lanes write consecutive rows)
-                    float *gcol = p.G + (size_t)unit * 512 * 512 + row;
-                    #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        if (p.atomic) atomicAdd(gcol + (size_t)(J0 + j) * 512, v[j]);
-                        else gcol[(size_t)(J0 + j) * 512] = v[j];
-                    }
-                }
             }
         }
     }
@@ -844,10 +848,22 @@ __global__ void __launch_bounds__(kGtThreads, 1) gram_tc_kernel(const __grid_con
     }
 }
 
-// block counts of the four bands: equal work per block (4:3:2:1) once T is long
-inline void gram_tc_splits(int T, int (&sp)[4]) {
-    const int f = T >= 8192 ? (T + 8191) / 8192 : 0;
-    for (int I = 0; I < 4; ++I) sp[I] = f ? f * (4 - I) : 1;
+// Token splits of the four bands (band I has 4 - I column blocks of work per token): while a further
+// split of every unit still fits one wave of blocks, split the band whose blocks are the longest
+// (at least 16 chunks of 64 tokens per split)
+inline void gram_tc_splits(int units, int T, int sms, int (&sp)[4]) {
+    for (int I = 0; I < 4; ++I) sp[I] = 1;
+    const int nch = (T + kGtTok - 1) / kGtTok;
+    while (true) {
+        int total = 0, best = -1;
+        for (int I = 0; I < 4; ++I) total += sp[I];
+        if ((long long)units * (total + 1) > sms) break;
+        for (int I = 0; I < 4; ++I)
+            if (nch >= 16 * (sp[I] + 1) &&
+                (best < 0 || (4 - I) * sp[best] > (4 - best) * sp[I])) best = I;
+        if (best < 0) break;
+        ++sp[best];
+    }
 }
 
 inline size_t gram_tc_smem() { return sizeof(GramTcSmem) + 1024; }
@@ -865,15 +881,14 @@ inline kvpack_status prepare_device() {
 
 inline kvpack_status run(int units, int T, const uint16_t *X, const CUtensorMap &tm_x, uint16_t *C_lo,
                          uint16_t *C_hi, uint16_t *B, float *sigma, void *ws, int sms, int max_iter, cudaStream_t st) {
-    (void)sms;
     Workspace w = carve(ws, units);
     GramTcParams gp;
     gp.tm_x = tm_x;
     gp.G = w.G;
     gp.T = T;
     gp.units = units;
-    gram_tc_splits(T, gp.splits);
-    gp.atomic = gp.splits[3] > 1 ? 1 : 0;
+    gram_tc_splits(units, T, sms, gp.splits);
+    gp.atomic = (gp.splits[0] > 1 || gp.splits[1] > 1 || gp.splits[2] > 1 || gp.splits[3] > 1) ? 1 : 0;
     if (gp.atomic && cudaMemsetAsync(w.G, 0, (size_t)units * 512 * 512 * sizeof(float), st) != cudaSuccess)
         return KVPACK_ERR_CUDA;
     const int per_unit = gp.splits[0] + gp.splits[1] + gp.splits[2] + gp.splits[3];
