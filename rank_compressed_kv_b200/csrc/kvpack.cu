@@ -528,11 +528,15 @@ kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t
         // with two consumer groups (32 heads) the value pass adds the groups' shares of a token's
         // attention mass into the zeroed output
         float *mass0 = pl.NH >= 32 ? mass : nullptr;
-        const rs::HiposParams ha{mask, hipos, hicnt, mass0, pl.units, T, pl.nwords, pl.tpu, pl.Tp};
-        const rs::HiposParams hb =
-            L_c > 0 ? rs::HiposParams{mask2, hipos2, hicnt2, nullptr, pl.units, L_c, pl.nwords2, pl.tpu2, pl.Tp2} : ha;
+        const rs::HiposParams ha{mask, hipos, hicnt, mass0, pl.units, T, pl.nwords, pl.tpu, pl.Tp,
+                                 rs::hipos_group(pl.nwords)};
+        const rs::HiposParams hb = L_c > 0 ? rs::HiposParams{mask2, hipos2, hicnt2, nullptr, pl.units, L_c, pl.nwords2,
+                                                             pl.tpu2, pl.Tp2, rs::hipos_group(pl.nwords2)}
+                                           : ha;
+        // blocks: enough for the set with the fewer units per block
+        const int upb = rs::kHpThreads / (ha.tpg > hb.tpg ? ha.tpg : hb.tpg);
         cudaLaunchConfig_t cfg{};
-        cfg.gridDim = dim3((unsigned)pl.units, L_c > 0 ? 2u : 1u);
+        cfg.gridDim = dim3((unsigned)((pl.units + upb - 1) / upb), L_c > 0 ? 2u : 1u);
         cfg.blockDim = dim3((unsigned)rs::kHpThreads);
         cfg.stream = st;
         cudaLaunchAttribute attr[1];

@@ -925,48 +925,60 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
 
 // Each unit's full-rank token positions in ascending order (hipos[unit][0 .. count)) and, per
 // 128-token tile, the count of full-rank tokens before it (hicnt[unit][tile]): the visual
-// passes' HI tiles are runs of that list.  One block per unit (blockIdx.y picks the mask: the
-// visual tokens', or the compressed text tokens' own); thread t scans a contiguous run of words.
+// passes' HI tiles are runs of that list.  A group of tpg threads (32 .. 256, the unit's word
+// count rounded up to a power of two) per unit, kHpThreads / tpg units per block (blockIdx.y picks
+// the mask: the visual tokens', or the compressed text tokens' own); thread t of a group scans a
+// contiguous run of words.
 constexpr int kHpThreads = 256;
 struct HiposParams {
     const uint32_t *mask;    // [units][nwords]
     uint16_t *hipos;         // [units][Tp]
     int *hicnt;              // [units][tpu]
     float *mass;             // [units][T], zeroed here when the value pass adds into it (or null)
-    int units, T, nwords, tpu, Tp;
+    int units, T, nwords, tpu, Tp, tpg;
 };
+
+__host__ __device__ inline int hipos_group(int nwords) {
+    int t = 32;
+    while (t < kHpThreads && t < nwords) t <<= 1;
+    return t;
+}
 
 __global__ void __launch_bounds__(kHpThreads) hipos_kernel(const HiposParams a, const HiposParams b) {
     griddep_launch_dependents();
     const HiposParams &p = blockIdx.y == 0 ? a : b;
-    const int unit = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tpg = p.tpg, t = threadIdx.x % tpg, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int unit = blockIdx.x * (kHpThreads / tpg) + threadIdx.x / tpg;
+    const int w_first = (threadIdx.x / tpg) * (tpg / 32);   // the group's first warp
     __shared__ int wsum[kHpThreads / 32];
-    if (unit < p.units && p.mass != nullptr) {
+    const bool live = unit < p.units;
+    if (live && p.mass != nullptr) {
         float *ms = p.mass + (size_t)unit * p.T;
-        for (int i = threadIdx.x; i < p.T; i += kHpThreads) ms[i] = 0.f;
+        for (int i = t; i < p.T; i += tpg) ms[i] = 0.f;
     }
-    if (unit < p.units) {
-        const int wpt = (p.nwords + kHpThreads - 1) / kHpThreads;
-        const int w0 = min(p.nwords, (int)threadIdx.x * wpt), w1 = min(p.nwords, w0 + wpt);
-        const uint32_t *mk = p.mask + (size_t)unit * p.nwords;
-        auto word = [&](int w) -> uint32_t {
-            uint32_t v = __ldg(mk + w);
-            const int nb = p.T - 32 * w;
-            if (nb < 32) v &= (1u << nb) - 1u;
-            return v;
-        };
-        int c = 0;
+    const int wpt = (p.nwords + tpg - 1) / tpg;
+    const int w0 = min(p.nwords, t * wpt), w1 = min(p.nwords, w0 + wpt);
+    const uint32_t *mk = p.mask + (size_t)(live ? unit : 0) * p.nwords;
+    auto word = [&](int w) -> uint32_t {
+        uint32_t v = __ldg(mk + w);
+        const int nb = p.T - 32 * w;
+        if (nb < 32) v &= (1u << nb) - 1u;
+        return v;
+    };
+    int c = 0;
+    if (live)
         for (int w = w0; w < w1; ++w) c += __popc(word(w));
-        int incl = c;
-        #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        if (lane == 31) wsum[warp] = incl;
-        __syncthreads();
+    int incl = c;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (live) {
         int base = incl - c;
-        for (int i = 0; i < warp; ++i) base += wsum[i];
+        for (int i = w_first; i < warp; ++i) base += wsum[i];
         uint16_t *out = p.hipos + (size_t)unit * p.Tp;
         int *cnt = p.hicnt + (size_t)unit * p.tpu;
         for (int w = w0; w < w1; ++w) {
