@@ -533,11 +533,12 @@ kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t
         const rs::HiposParams hb = L_c > 0 ? rs::HiposParams{mask2, hipos2, hicnt2, nullptr, pl.units, L_c, pl.nwords2,
                                                              pl.tpu2, pl.Tp2, rs::hipos_group(pl.nwords2)}
                                            : ha;
-        // blocks: enough for the set with the fewer units per block
-        const int upb = rs::kHpThreads / (ha.tpg > hb.tpg ? ha.tpg : hb.tpg);
+        // 256-thread blocks unless a unit's group is larger; enough blocks for the set with the fewer
+        // units per block
+        const int tpg = ha.tpg > hb.tpg ? ha.tpg : hb.tpg, threads = tpg > 256 ? tpg : 256, upb = threads / tpg;
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3((unsigned)((pl.units + upb - 1) / upb), L_c > 0 ? 2u : 1u);
-        cfg.blockDim = dim3((unsigned)rs::kHpThreads);
+        cfg.blockDim = dim3((unsigned)threads);
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

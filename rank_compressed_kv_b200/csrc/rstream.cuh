@@ -925,11 +925,12 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
 
 // Each unit's full-rank token positions in ascending order (hipos[unit][0 .. count)) and, per
 // 128-token tile, the count of full-rank tokens before it (hicnt[unit][tile]): the visual
-// passes' HI tiles are runs of that list.  A group of tpg threads (32 .. 256, the unit's word
-// count rounded up to a power of two) per unit, kHpThreads / tpg units per block (blockIdx.y picks
+// passes' HI tiles are runs of that list.  A group of tpg threads (32 .. 1024, the unit's word
+// count rounded up to a power of two) per unit, blockDim / tpg units per block (blockIdx.y picks
 // the mask: the visual tokens', or the compressed text tokens' own); thread t of a group scans a
 // contiguous run of words.
-constexpr int kHpThreads = 256;
+constexpr int kHpThreads = 1024;     // most threads per block (blocks are 256 threads unless a unit needs more)
+constexpr int kHpWords = 8;       // mask words a thread keeps in registers
 struct HiposParams {
     const uint32_t *mask;    // [units][nwords]
     uint16_t *hipos;         // [units][Tp]
@@ -948,7 +949,7 @@ __global__ void __launch_bounds__(kHpThreads) hipos_kernel(const HiposParams a, 
     griddep_launch_dependents();
     const HiposParams &p = blockIdx.y == 0 ? a : b;
     const int tpg = p.tpg, t = threadIdx.x % tpg, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int unit = blockIdx.x * (kHpThreads / tpg) + threadIdx.x / tpg;
+    const int unit = blockIdx.x * (blockDim.x / tpg) + threadIdx.x / tpg;
     const int w_first = (threadIdx.x / tpg) * (tpg / 32);   // the group's first warp
     __shared__ int wsum[kHpThreads / 32];
     const bool live = unit < p.units;
@@ -965,9 +966,16 @@ __global__ void __launch_bounds__(kHpThreads) hipos_kernel(const HiposParams a, 
         if (nb < 32) v &= (1u << nb) - 1u;
         return v;
     };
+    // a thread's words stay in registers when they are at most kHpWords (masks up to 65536 tokens)
+    uint32_t wv[kHpWords];
     int c = 0;
+    #pragma unroll
+    for (int i = 0; i < kHpWords; ++i) {
+        wv[i] = live && w0 + i < w1 ? word(w0 + i) : 0u;
+        c += __popc(wv[i]);
+    }
     if (live)
-        for (int w = w0; w < w1; ++w) c += __popc(word(w));
+        for (int w = w0 + kHpWords; w < w1; ++w) c += __popc(word(w));
     int incl = c;
     #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -981,14 +989,17 @@ __global__ void __launch_bounds__(kHpThreads) hipos_kernel(const HiposParams a, 
         for (int i = w_first; i < warp; ++i) base += wsum[i];
         uint16_t *out = p.hipos + (size_t)unit * p.Tp;
         int *cnt = p.hicnt + (size_t)unit * p.tpu;
-        for (int w = w0; w < w1; ++w) {
+        auto emit = [&](int w, uint32_t bits) {
             if ((w & 3) == 0) cnt[w >> 2] = base;   // a tile is four words
-            uint32_t bits = word(w);
             while (bits) {
                 out[base++] = (uint16_t)(32 * w + __ffs(bits) - 1);
                 bits &= bits - 1u;
             }
-        }
+        };
+        #pragma unroll
+        for (int i = 0; i < kHpWords; ++i)
+            if (w0 + i < w1) emit(w0 + i, wv[i]);
+        for (int w = w0 + kHpWords; w < w1; ++w) emit(w, word(w));
     }
     // the next kernel's wait then also covers the kernel before this one
     griddep_wait();
