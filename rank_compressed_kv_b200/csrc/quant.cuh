@@ -159,11 +159,15 @@ __device__ __forceinline__ void lo_rows(unsigned char *dst, const uint8_t *__res
     }
 }
 
-// The same for the K and the V planes of the same rows, all loads first
+// The same for the K and the V planes of the same rows, the loads of eight rows first
 template <int R, int NT>
 __device__ __forceinline__ void lo_rows_kv(unsigned char *dk, unsigned char *dv, const uint8_t *__restrict__ QK,
                                            const int8_t *__restrict__ EK, const uint8_t *__restrict__ QV,
                                            const int8_t *__restrict__ EV, size_t base, int n, int t0) {
+    if constexpr (R > 8) {
+        lo_rows_kv<8, NT>(dk, dv, QK, EK, QV, EV, base, n, t0);
+        lo_rows_kv<R - 8, NT>(dk, dv, QK, EK, QV, EV, base, n, t0 + 8 * NT);
+    } else {
     uint2 wk[R], wv[R];
     int ek[R], ev[R];
     #pragma unroll
@@ -186,6 +190,7 @@ __device__ __forceinline__ void lo_rows_kv(unsigned char *dk, unsigned char *dv,
         *reinterpret_cast<uint4 *>(dk + t * 32 + ((1 ^ sw) << 4)) = dq8(wk[i].y, ek[i]);
         *reinterpret_cast<uint4 *>(dv + t * 32 + (sw << 4)) = dq8(wv[i].x, ev[i]);
         *reinterpret_cast<uint4 *>(dv + t * 32 + ((1 ^ sw) << 4)) = dq8(wv[i].y, ev[i]);
+    }
     }
 }
 

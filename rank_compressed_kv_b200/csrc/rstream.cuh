@@ -298,12 +298,12 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
         // that completes on the queue entry's barrier, so the gather warps start once they are there.
         uint32_t hseq = 0;
         auto push_gather = [&](int ks, int vs, int ds, int n, int unit, int skew, const uint16_t *src,
-                               uint32_t pos_bytes) -> bool {
+                               uint32_t pos_bytes, int type = kTypeHi, int tok = 0) -> bool {
             const int hq = hseq % kNQ;
             if (hseq >= (uint32_t)kNQ && !mbar_wait(&sm.gfree[hq], ((hseq / kNQ) - 1) & 1u, abort)) return false;
             if (lane == 0) {
                 int *e = sm.hiq[hq];
-                e[0] = ks; e[1] = vs; e[2] = ds; e[3] = n; e[4] = unit; e[5] = skew;
+                e[0] = ks; e[1] = vs; e[2] = ds; e[3] = n; e[4] = unit; e[5] = skew; e[6] = type; e[7] = tok;
                 if (pos_bytes > 0) {
                     fence_proxy_async();   // the descriptor's earlier readers went through the generic proxy
                     mbar_arrive_tx(&sm.gready[hq], pos_bytes);
@@ -376,21 +376,18 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
                     // release their descriptor writes.  4-bit rows go to the gather warps instead.
                     const int nb = (n + 255) >> 8;   // 256-row boxes of 32-byte rows
                     if (Q4 && !p.rank0) {
-                        // 4-bit rows: the producer dequantizes LO tiles itself, in parallel with the
-                        // gather warps' HI tiles, and arrives for the gather warps
+                        // 4-bit rows: the producer dequantizes the first half of a LO tile's rows and
+                        // the gather warps the second half (they arrive for themselves)
                         const size_t base = (size_t)unit * p.T + tok;
                         if (VALUE)
-                            quant::lo_rows_kv<C::kLoTok / 32, 32>(sm.kslot[ks], sm.vslot[vs], p.QK_lo, p.EK, p.QV_lo,
+                            quant::lo_rows_kv<C::kLoTok / 64, 32>(sm.kslot[ks], sm.vslot[vs], p.QK_lo, p.EK, p.QV_lo,
                                                                   p.EV, base, n, lane);
                         else
-                            quant::lo_rows<C::kLoTok / 32, 32>(sm.kslot[ks], p.QK_lo, p.EK, base, n, lane);
+                            quant::lo_rows<C::kLoTok / 64, 32>(sm.kslot[ks], p.QK_lo, p.EK, base, n, lane);
                         fence_proxy_async();          // the score MMA reads these rows through the async proxy
+                        if (!push_gather(ks, vs, ds, n, unit, 0, nullptr, 0u, kTypeLo, tok)) { ok = false; break; }
                         mbar_arrive(&sm.kfull[ks]);
                         if (VALUE) mbar_arrive(&sm.vfull[vs]);
-                        if (lane == 0) {
-                            mbar_arrive_cnt(&sm.kfull[ks], kGatherThreads);
-                            if (VALUE) mbar_arrive_cnt(&sm.vfull[vs], kGatherThreads);
-                        }
                     } else if (lane == 0) {
                         if (!p.rank0) {
                             fence_proxy_async();
@@ -497,7 +494,7 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
             const int hq = h % kNQ;
             if (!mbar_wait(&sm.gready[hq], (h / kNQ) & 1u, abort)) break;
             const int *e = sm.hiq[hq];
-            const int ks = e[0], vs = e[1], ds = e[2], n = e[3], unit = e[4], skew = e[5];
+            const int ks = e[0], vs = e[1], ds = e[2], n = e[3], unit = e[4], skew = e[5], etype = e[6], etok = e[7];
             mbar_arrive(&sm.gfree[hq]);
             if (ks < 0) break;
             // the positions (landed with the queue entry) stay valid until the consumers free the
@@ -505,8 +502,24 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
             const uint16_t *pos = reinterpret_cast<const uint16_t *>(sm.kdesc[ds] + 8) + skew;
             const size_t ubase = (size_t)unit * p.T;
             if constexpr (Q4) {
+                if (etype == kTypeLo) {
+                    // the second half of a LO tile's rows (the producer dequantizes the first)
+                    const size_t base = ubase + etok;
+                    constexpr int kHalf = C::kLoTok / 2;
+                    if (VALUE)
+                        quant::lo_rows_kv<kHalf / kGatherThreads, kGatherThreads>(
+                            sm.kslot[ks], sm.vslot[vs], p.QK_lo, p.EK, p.QV_lo, p.EV, base, n, kHalf + g);
+                    else
+                        quant::lo_rows<kHalf / kGatherThreads, kGatherThreads>(sm.kslot[ks], p.QK_lo, p.EK, base, n,
+                                                                              kHalf + g);
+                    fence_proxy_async();
+                    mbar_arrive(&sm.kfull[ks]);
+                    if (VALUE) mbar_arrive(&sm.vfull[vs]);
+                    ++h;
+                    continue;
+                }
                 // dequantize a HI tile into the layout of the 16-bit path (128-byte rows, 128-byte
-                // swizzle); rows past n are zero.  (LO tiles of 4-bit rows are the producer's.)
+                // swizzle); rows past n are zero
                 constexpr int RH = C::kHiTok / kGatherThreads;
                 struct HiRows { uint2 w[RH][4]; char2 ee[RH]; };
                 auto hi_load = [&](HiRows &H, const uint8_t *QL, const uint8_t *QH, const int8_t *E) {
