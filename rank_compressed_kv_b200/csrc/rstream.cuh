@@ -671,6 +671,31 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
         int unit = 0, pslot = 0;
         unsigned char *pb = sm.pbuf[VALUE ? 4 * cg + q : 0];
         const uint32_t pb_s = smem_u32(pb);
+        float *mrow = nullptr;                         // value pass: the segment's unit's row of the mass
+        // Per-lane parts of the value pass's shared-memory addresses.  A k-step's first row is a
+        // multiple of 16, so every swizzle term depends on the lane alone.
+        const int ra = (lane & 7) + ((lane >> 4) << 3);                // A (C_V^T): row within the k-step
+        const int rb = (lane & 7) + (((lane >> 3) & 1) << 3);          // B (P): row within the k-step
+        const uint32_t offA_lo = (uint32_t)(ra * 32 + ((((lane >> 3) & 1) ^ ((ra >> 2) & 1)) << 4));
+        uint32_t offA_hi[4], offB[(PHS + 15) / 16], offP[PHS / 8];
+        #pragma unroll
+        for (int mt = 0; mt < 4; ++mt)
+            offA_hi[mt] = (uint32_t)(ra * 128 + (((2 * mt + ((lane >> 3) & 1)) ^ (lane & 7)) << 4));
+        #pragma unroll
+        for (int np = 0; np < (PHS + 15) / 16; ++np) {
+            int ch = PHS == 8 ? 0 : 2 * np + (lane >> 4);
+            if (PHS == 16) ch ^= (rb >> 2) & 1;
+            if (PHS == 32) ch ^= (rb >> 1) & 3;
+            offB[np] = (uint32_t)(rb * (PHS * 2) + (ch << 4));
+        }
+        #pragma unroll
+        for (int c = 0; c < PHS / 8; ++c) {
+            int pc = c;
+            if (PHS == 16) pc = c ^ ((lane >> 2) & 1);
+            if (PHS == 32) pc = c ^ ((lane >> 1) & 3);
+            offP[c] = (uint32_t)(lane * (PHS * 2) + pc * 16);
+        }
+        (void)offA_lo; (void)offA_hi; (void)offB; (void)offP; (void)mrow;
         bool failed = false;
         while (!failed) {
             const int sb = seq % kNS, vs = seq % kNV;
@@ -685,6 +710,7 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
                 unit = d[1];
                 pslot = d[4];
                 if (VALUE) {
+                    mrow = p.mass != nullptr ? p.mass + (size_t)unit * p.T : nullptr;
                     #pragma unroll
                     for (int h = 0; h < HS; ++h) {
                         float2 st = make_float2(0.f, 0.f);
@@ -763,10 +789,9 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
                     }
                     // the token's attention mass: each head group adds its heads' share into the
                     // zeroed output (two addends onto zero: the same sum in either order)
-                    if (take && p.mass != nullptr) {
-                        float *dst = p.mass + (size_t)unit * p.T + pos;
-                        if (C::kSplit == 1) *dst = ms0 + ms1;
-                        else red_add_f32(dst, ms0 + ms1);
+                    if (take && mrow != nullptr) {
+                        if (C::kSplit == 1) mrow[pos] = ms0 + ms1;
+                        else red_add_f32(mrow + pos, ms0 + ms1);
                     }
                     const bool do_u = type == kTypeHi || !p.rank0;
                     if (do_u && !v_ready) {
@@ -775,7 +800,6 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
                     }
                     if (do_u) {
                         // this thread's P row (PHS bf16), 16-byte chunks swizzled against bank conflicts
-                        const int prow = lane;
                         #pragma unroll
                         for (int c = 0; c < PHS / 8; ++c) {
                             uint4 v;
@@ -783,54 +807,43 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
                             v.y = pack_bf16(pr[8 * c + 2], pr[8 * c + 3]);
                             v.z = pack_bf16(pr[8 * c + 4], pr[8 * c + 5]);
                             v.w = pack_bf16(pr[8 * c + 6], pr[8 * c + 7]);
-                            int pc = c;
-                            if (PHS == 16) pc = c ^ ((prow >> 2) & 1);
-                            if (PHS == 32) pc = c ^ ((prow >> 1) & 3);
-                            *reinterpret_cast<uint4 *>(pb + prow * (PHS * 2) + pc * 16) = v;
+                            *reinterpret_cast<uint4 *>(pb + offP[c]) = v;
                         }
                         __syncwarp();
                         // u^T += C_V^T P over the warp's 32 tokens (two k-steps of 16)
+                        const uint32_t a_lo = vb + (uint32_t)((sub * kTile + 32 * q) * 32) + offA_lo;
+                        const uint32_t a_hi = vb + (uint32_t)((32 * q) * 128);
                         #pragma unroll 1
                         for (int kk = 0; kk < 2; ++kk) {
                             uint32_t bfr[PHS / 8][2];
                             #pragma unroll
                             for (int np = 0; np < (PHS + 15) / 16; ++np) {
-                                const int row = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
-                                int ch = 2 * np + (lane >> 4);
-                                if (PHS == 8) ch = 0;
-                                int pc = ch;
-                                if (PHS == 16) pc = ch ^ ((row >> 2) & 1);
-                                if (PHS == 32) pc = ch ^ ((row >> 1) & 3);
+                                const uint32_t ba = pb_s + (uint32_t)(kk * 16 * PHS * 2) + offB[np];
                                 uint32_t r0, r1, r2, r3;
                                 if (PHS == 8) {
                                     // x2: tokens 0-7 and 8-15 of the 8 heads
                                     asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
-                                                 : "=r"(r0), "=r"(r1) : "r"(pb_s + row * (PHS * 2) + (pc << 4)));
+                                                 : "=r"(r0), "=r"(r1) : "r"(ba));
                                     bfr[0][0] = r0;
                                     bfr[0][1] = r1;
                                 } else {
-                                    ldsm_x4_t(pb_s + row * (PHS * 2) + (pc << 4), r0, r1, r2, r3);
+                                    ldsm_x4_t(ba, r0, r1, r2, r3);
                                     bfr[2 * np][0] = r0;
                                     bfr[2 * np][1] = r1;
                                     bfr[2 * np + 1][0] = r2;
                                     bfr[2 * np + 1][1] = r3;
                                 }
                             }
-                            const int tb = sub * kTile + 32 * q + 16 * kk;   // first token row of the k-step
                             if (type == kTypeLo) {
                                 uint32_t a[4];
-                                const int row = tb + (lane & 7) + ((lane >> 4) << 3);
-                                const int ch = (lane >> 3) & 1;
-                                ldsm_x4_t(vb + row * 32 + ((ch ^ ((row >> 2) & 1)) << 4), a[0], a[1], a[2], a[3]);
+                                ldsm_x4_t(a_lo + (uint32_t)(kk * 16 * 32), a[0], a[1], a[2], a[3]);
                                 #pragma unroll
                                 for (int nt = 0; nt < PHS / 8; ++nt) mma_bf16(u[0][nt], a, bfr[nt][0], bfr[nt][1]);
                             } else {
                                 #pragma unroll
                                 for (int mt = 0; mt < 4; ++mt) {
                                     uint32_t a[4];
-                                    const int row = tb + (lane & 7) + ((lane >> 4) << 3);
-                                    const int ch = 2 * mt + ((lane >> 3) & 1);
-                                    ldsm_x4_t(vb + row * 128 + ((ch ^ (row & 7)) << 4), a[0], a[1], a[2], a[3]);
+                                    ldsm_x4_t(a_hi + (uint32_t)(kk * 16 * 128) + offA_hi[mt], a[0], a[1], a[2], a[3]);
                                     #pragma unroll
                                     for (int nt = 0; nt < PHS / 8; ++nt) mma_bf16(u[mt][nt], a, bfr[nt][0], bfr[nt][1]);
                                 }
