@@ -67,7 +67,7 @@ constexpr int kDescInts = 8 + 68;   // header + up to 16 mask words (LO) or 8 + 
 constexpr int kTypeLo = 0, kTypeHi = 1, kTypeEnd = 2;
 constexpr int kFlagFirst = 1 << 8, kFlagLast = 1 << 9;
 constexpr float kRefInit = -1e30f;
-constexpr float kLazy = 8.f;        // a per-thread reference max moves when a logit exceeds it by 2^8
+constexpr float kLazy = 8.f;        // a per-thread reference sits 2^8 above the largest logit at its last move
 
 // Geometry per (query heads NH, pass).  NH is the unit's Hg rounded up to 4, 8, 16 or 32.
 // Three rings per CTA, released independently:
@@ -758,15 +758,17 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
                 if (!VALUE) {
                     // ---------------------------------------------------- stats
                     if (take) {
-                        float mx = sc[0] - m[0];
+                        // m[h] is kept kLazy above the largest logit at its last move, so the test is
+                        // one comparison per head and every term 2^(s - m) is at most 1
+                        bool up = false;
                         #pragma unroll
-                        for (int h = 1; h < HS; ++h) mx = fmaxf(mx, sc[h] - m[h]);
-                        if (mx > kLazy) {
+                        for (int h = 0; h < HS; ++h) up |= sc[h] > m[h];
+                        if (up) {
                             #pragma unroll
                             for (int h = 0; h < HS; ++h)
                                 if (sc[h] > m[h]) {
-                                    l[h] *= ex2(m[h] - sc[h]);
-                                    m[h] = sc[h];
+                                    l[h] *= ex2(m[h] - (sc[h] + kLazy));
+                                    m[h] = sc[h] + kLazy;
                                 }
                         }
                         #pragma unroll
