@@ -251,6 +251,78 @@ __device__ void small_gram(const float *__restrict__ At, const float *__restrict
     __syncthreads();
 }
 
+// The same product on the tensor cores: both operands split into bf16 hi + lo planes, three
+// products (hi hi, hi lo, lo hi) with fp32 accumulation (~2^-16 relative, as the G Q product).
+// 32-row chunks of the contraction are staged in shared memory as bf16 rows of 32 (one row per
+// column i or j: K-major for both mma.sync operands; the 16-byte chunk c of row x sits at
+// c ^ ((x >> 1) & 3), so the 8-row ldmatrix reads are free of bank conflicts); warp w < 12
+// computes columns 8w .. 8w + 7 of C for all 96 rows.
+__device__ void small_gram_tc(const float *__restrict__ At, const float *__restrict__ Bt, float *C, EigWork &wk) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, tig = lane & 3;
+    // planes of 96 rows x 64 bytes: A hi, A lo, B hi, B lo
+    unsigned char *st = reinterpret_cast<unsigned char *>(&wk.st[0][0]);
+    const uint32_t st_s = smem_u32(st);
+    constexpr uint32_t kPlane = kP * 64;
+    static_assert(4 * kPlane <= sizeof(wk.st), "staging planes");
+    float acc[6][4];
+    #pragma unroll
+    for (int mt = 0; mt < 6; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    for (int r0 = 0; r0 < kN; r0 += 32) {
+        __syncthreads();
+        // stage: thread t takes operand t / 256, column c, rows 4 q4 .. 4 q4 + 3 of the chunk
+        for (int i = tid; i < 2 * kP * 8; i += kEigThreads) {
+            const int op = i / (kP * 8), c = (i / 8) % kP, q4 = i % 8;
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>((op ? Bt : At) + (size_t)c * kN + r0 + 4 * q4));
+            uint32_t h01, l01, h23, l23;
+            split2(v.x, v.y, h01, l01);
+            split2(v.z, v.w, h23, l23);
+            const uint32_t off = (uint32_t)c * 64 + ((((q4 >> 1) ^ ((c >> 1) & 3))) << 4) + (q4 & 1) * 8;
+            unsigned char *hp = st + (2 * op) * kPlane + off, *lp = st + (2 * op + 1) * kPlane + off;
+            *reinterpret_cast<uint2 *>(hp) = make_uint2(h01, h23);
+            *reinterpret_cast<uint2 *>(lp) = make_uint2(l01, l23);
+        }
+        __syncthreads();
+        if (warp < 12) {
+            #pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+                // B (the warp's 8 columns, k 16 ks ..): rows n = 8 warp + (lane & 7), chunk 2 ks + ((lane >> 3) & 1)
+                const int nrow = 8 * warp + (lane & 7);
+                const uint32_t boff = (uint32_t)nrow * 64 + (((2 * ks + ((lane >> 3) & 1)) ^ ((nrow >> 1) & 3)) << 4);
+                uint32_t bh0, bh1, bl0, bl1;
+                asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+                             : "=r"(bh0), "=r"(bh1) : "r"(st_s + 2 * kPlane + boff));
+                asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+                             : "=r"(bl0), "=r"(bl1) : "r"(st_s + 3 * kPlane + boff));
+                #pragma unroll
+                for (int mt = 0; mt < 6; ++mt) {
+                    // A (rows 16 mt ..): matrices (rows 0-7, k 0-7), (8-15, 0-7), (0-7, 8-15), (8-15, 8-15)
+                    const int arow = 16 * mt + (lane & 7) + (((lane >> 3) & 1) << 3);
+                    const uint32_t aoff =
+                        (uint32_t)arow * 64 + (((2 * ks + ((lane >> 4) & 1)) ^ ((arow >> 1) & 3)) << 4);
+                    uint32_t ah[4], al[4];
+                    ldsm_x4(st_s + aoff, ah[0], ah[1], ah[2], ah[3]);
+                    ldsm_x4(st_s + kPlane + aoff, al[0], al[1], al[2], al[3]);
+                    mma_bf16(acc[mt], ah, bh0, bh1);
+                    mma_bf16(acc[mt], ah, bl0, bl1);
+                    mma_bf16(acc[mt], al, bh0, bh1);
+                }
+            }
+        }
+    }
+    if (warp < 12) {
+        #pragma unroll
+        for (int mt = 0; mt < 6; ++mt) {
+            const int r = 16 * mt + g, c = 8 * warp + 2 * tig;
+            C[r * kP + c] = acc[mt][0];
+            C[r * kP + c + 1] = acc[mt][1];
+            C[(r + 8) * kP + c] = acc[mt][2];
+            C[(r + 8) * kP + c + 1] = acc[mt][3];
+        }
+    }
+    __syncthreads();
+}
+
 // out[j][r] = sum_i in[i][r] M[i][j] for the 96 columns j (in and out: 96 columns of 512 fp32,
 // column-contiguous; one thread per row r).  Optional outputs: out (fp32), the bf16 hi / lo row
 // layout qg, and the bf16 rows of the basis B (its first 64 columns, B[j][r]).
@@ -503,7 +575,7 @@ __global__ void __launch_bounds__(kEigThreads, 1) eig_kernel(EigParams p) {
         const bool rr = it == 1 || (it % 3) == 0 || it == p.max_iter;   // measured: every third beats every second
         const float *zsrc;
         if (rr) {
-            small_gram(Qt, Yt, wk.A, wk);               // H = Q^T Y
+            small_gram_tc(Qt, Yt, wk.A, wk);            // H = Q^T Y
             for (int e = tid; e < kP * kP; e += kEigThreads) {
                 const int i = e / kP, j = e % kP;
                 if (i < j) {
@@ -587,7 +659,7 @@ __global__ void __launch_bounds__(kEigThreads, 1) eig_kernel(EigParams p) {
         }
         __syncthreads();
         // Cholesky QR of Z = zsrc * diag(scale): W = S^T (zsrc^T zsrc) S = R^T R, Q = zsrc S R^-1
-        small_gram(zsrc, zsrc, wk.A, wk);
+        small_gram_tc(zsrc, zsrc, wk.A, wk);
         for (int e = tid; e < kP * kP; e += kEigThreads) wk.A[e] *= sm.scale[e / kP] * sm.scale[e % kP];
         __syncthreads();
         cholesky96(wk.A, wk.V, sm);
