@@ -13,7 +13,9 @@ def unit_inputs(w: Workload, layer: int, b: int, g: int, T: int, Lcap: int, mask
                 step: int = 0):
     """One unit's compressed cache, text tail and rank mask.
 
-    mask: "random" (k random bits, default k = ceil(hi_frac T)), "ones", "zeros".
+    mask: "random" (k random bits, default k = ceil(hi_frac T)), "ones", "zeros", "blocks" (runs of
+    512 full-rank and 512 reduced tokens, the first run 256 long, so runs straddle 128-token tiles),
+    "prefix" (the first k tokens full-rank).
     Returns dict: CK, CV [T, 64]; BK, BV [64, 512]; K_text, V_text [Lcap, 4, 128]; mask [ceil(T/32)] uint32.
     """
     CK, BK = compressed_unit(w, layer, b, g, K_VIS, T)
@@ -26,6 +28,15 @@ def unit_inputs(w: Workload, layer: int, b: int, g: int, T: int, Lcap: int, mask
         m = all_ones_mask(T)
     elif mask == "zeros":
         m = np.zeros((T + 31) // 32, dtype=np.uint32)
+    elif mask in ("blocks", "prefix"):
+        t = np.arange(T)
+        if mask == "blocks":
+            bits = ((t + 256) // 512) % 2 == 1
+        else:
+            bits = t < (k if k is not None else int(np.ceil(w.hi_frac * T)))
+        padded = np.zeros(((T + 31) // 32) * 32, dtype=bool)
+        padded[:T] = bits
+        m = (padded.reshape(-1, 32).astype(np.uint64) << np.arange(32, dtype=np.uint64)).sum(axis=1).astype(np.uint32)
     else:
         raise ValueError(mask)
     return dict(CK=CK, CV=CV, BK=BK, BV=BV, K_text=Kt, V_text=Vt, mask=m)

@@ -33,6 +33,12 @@ CASES = [
     ("rank0_gqa28",  1, 1, 28, 4, 2000, 48, 30, "random", 0),
     ("rank0_no_text", 2, 1, 32, 8, 3000, 8, 0, "random", 0),
     ("rank0_all_zero", 1, 1, 8, 8, 300, 8, 5, "zeros", 0),
+    # runs of full-rank tokens: blocks without a LO tile, HI tiles that span blocks, units split
+    # over many CTAs (segments starting inside a unit, past full-rank tokens)
+    ("blocks",       1, 2, 32, 8, 5000, 24, 20, "blocks", 16),
+    ("blocks_gqa28", 1, 1, 28, 4, 4100, 16, 7, "blocks", 16),
+    ("prefix_long",  2, 1, 16, 8, 9000, 16, 12, "prefix", 16),
+    ("rank0_blocks", 1, 1, 32, 8, 3000, 8, 4, "blocks", 0),
 ]
 
 
