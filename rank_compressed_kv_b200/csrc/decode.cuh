@@ -32,7 +32,8 @@ constexpr int kTxtPart = 130;   // per (unit, text chunk, head): max, sum, w[128
 // =================================================================== query block
 
 // Per unit, the query block the visual passes copy plane by plane:
-//   [2][Hg][64] bf16  q~ hi then lo (128-byte rows, 16-byte chunk c stored at c ^ (h & 7))
+//   [2][Hg][64] bf16  q~ hi then lo (128-byte rows, 16-byte chunk c stored at c ^ (r & 7) with r the
+//                     row the head lands in: h, or h + 2 for heads >= qsplit in the 28-head form)
 __host__ __device__ constexpr size_t qblock_bytes(int Hg) { return (size_t)Hg * 2 * 128; }
 
 // ========================================================================= text
@@ -55,6 +56,7 @@ struct Params {
     unsigned char *qt2;        // the same for the text tokens' basis, or null
     unsigned int *counter;     // work counter, zero at launch
     int n_units, L, Hg, per_kv, n_q, groups, Sc, ct, n_qitems, n_items;
+    int qsplit;                // heads >= qsplit sit 2 rows lower in the visual passes' q~ tile (28-head form)
     float scale2;
 };
 
@@ -223,7 +225,8 @@ __global__ void __launch_bounds__(kThreads, 1) text_kernel(const __grid_constant
                             const float v = wt[mt][e] * p.scale2;
                             const uint16_t hi = float_to_bf16_bits(v);
                             const uint16_t lo = float_to_bf16_bits(v - bf16_bits_to_float(hi));
-                            const int off = h * 64 + ((((i >> 3) ^ (h & 7)) & 7) << 3) + (i & 7);
+                            const int ph = h + (h >= p.qsplit ? 2 : 0);   // the row it lands in
+                            const int off = h * 64 + ((((i >> 3) ^ (ph & 7)) & 7) << 3) + (i & 7);
                             qt[off] = hi;
                             qt[p.Hg * 64 + off] = lo;
                         }

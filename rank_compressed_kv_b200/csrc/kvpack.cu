@@ -69,7 +69,7 @@ struct DecodePlan {
     size_t off_qt2, off_sp2, off_vp2, off_mask2, off_hipos2, off_hicnt2;
 };
 
-inline int round_heads(int Hg) { return Hg <= 4 ? 4 : Hg <= 8 ? 8 : Hg <= 16 ? 16 : 32; }
+inline int round_heads(int Hg) { return Hg <= 4 ? 4 : Hg <= 8 ? 8 : Hg <= 16 ? 16 : Hg <= 28 ? 28 : 32; }
 
 // Most partial slots any unit gets when NT tiles are split over C CTAs (tpu tiles per unit).
 inline int max_slots(long long NT, long long C, int tpu) { return (int)(((long long)tpu * C + NT - 1) / NT) + 1; }
@@ -150,10 +150,11 @@ bool rs_attr() {
 bool rs_attrs() {
     return rs_attr<4, false, false>() && rs_attr<4, true, false>() && rs_attr<8, false, false>() &&
            rs_attr<8, true, false>() && rs_attr<16, false, false>() && rs_attr<16, true, false>() &&
-           rs_attr<32, false, false>() && rs_attr<32, true, false>() && rs_attr<4, false, true>() &&
-           rs_attr<4, true, true>() && rs_attr<8, false, true>() && rs_attr<8, true, true>() &&
-           rs_attr<16, false, true>() && rs_attr<16, true, true>() && rs_attr<32, false, true>() &&
-           rs_attr<32, true, true>();
+           rs_attr<28, false, false>() && rs_attr<28, true, false>() && rs_attr<32, false, false>() &&
+           rs_attr<32, true, false>() && rs_attr<4, false, true>() && rs_attr<4, true, true>() &&
+           rs_attr<8, false, true>() && rs_attr<8, true, true>() && rs_attr<16, false, true>() &&
+           rs_attr<16, true, true>() && rs_attr<28, false, true>() && rs_attr<28, true, true>() &&
+           rs_attr<32, false, true>() && rs_attr<32, true, true>();
 }
 
 // Launch on `st` with programmatic stream serialization: the kernel may start while the
@@ -186,6 +187,9 @@ cudaError_t launch_rs_q(int NH, const rs::Params &rp, int grid, cudaStream_t st)
                               st, rp);
         case 16:
             return launch_pdl(rs::rs_kernel<16, VALUE, Q4>, grid, rs::Cfg<16, VALUE>::kThreads, rs::smem_bytes<16, VALUE>(),
+                              st, rp);
+        case 28:
+            return launch_pdl(rs::rs_kernel<28, VALUE, Q4>, grid, rs::Cfg<28, VALUE>::kThreads, rs::smem_bytes<28, VALUE>(),
                               st, rp);
         default:
             return launch_pdl(rs::rs_kernel<32, VALUE, Q4>, grid, rs::Cfg<32, VALUE>::kThreads, rs::smem_bytes<32, VALUE>(),
@@ -476,6 +480,7 @@ kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t
                 return KVPACK_ERR_CUDA;
         }
         tp.q = q; tp.part = tpart; tp.qt = qt; tp.qt2 = qt2; tp.counter = counter;
+        tp.qsplit = pl.NH == 28 ? 14 : 1 << 30;
         tp.n_units = pl.units; tp.L = L_text; tp.Hg = Hg; tp.per_kv = per_kv; tp.n_q = d->n_q_heads;
         tp.groups = groups; tp.Sc = Sc; tp.ct = ct; tp.n_qitems = pl.units * 4 * (L_c > 0 ? 2 : 1);
         tp.n_items = tp.n_qitems + pl.units * 4 * Sc; tp.scale2 = scale2;
@@ -525,9 +530,9 @@ kvpack_status decode_impl(const kvpack_dims *d, int32_t n_layers, const uint16_t
     }
     {
         // each unit's full-rank positions, for the HI tiles of both passes
-        // with two consumer groups (32 heads) the value pass adds the groups' shares of a token's
-        // attention mass into the zeroed output
-        float *mass0 = pl.NH >= 32 ? mass : nullptr;
+        // with two consumer groups (28 or 32 heads) the value pass adds the groups' shares of a
+        // token's attention mass into the zeroed output
+        float *mass0 = pl.NH >= 28 ? mass : nullptr;
         const rs::HiposParams ha{mask, hipos, hicnt, mass0, pl.units, T, pl.nwords, pl.tpu, pl.Tp,
                                  rs::hipos_group(pl.nwords)};
         const rs::HiposParams hb = L_c > 0 ? rs::HiposParams{mask2, hipos2, hicnt2, nullptr, pl.units, L_c, pl.nwords2,
@@ -750,6 +755,7 @@ kvpack_status kvpack_dense_decode_attn(const kvpack_dims *d, int32_t n_layers, c
             return KVPACK_ERR_CUDA;
     }
     tp.q = q; tp.part = tpart; tp.qt = nullptr; tp.counter = counter;
+    tp.qsplit = 1 << 30;
     tp.n_units = units; tp.L = L; tp.Hg = Hg; tp.per_kv = per_kv; tp.n_q = d->n_q_heads;
     tp.groups = d->n_kv_heads / KVPACK_GROUP; tp.Sc = Sc; tp.ct = ct; tp.n_qitems = 0;
     tp.n_items = units * 4 * Sc; tp.scale2 = softmax_scale * 1.4426950408889634f;

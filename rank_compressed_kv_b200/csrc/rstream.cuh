@@ -69,7 +69,9 @@ constexpr int kFlagFirst = 1 << 8, kFlagLast = 1 << 9;
 constexpr float kRefInit = -1e30f;
 constexpr float kLazy = 8.f;        // a per-thread reference sits 2^8 above the largest logit at its last move
 
-// Geometry per (query heads NH, pass).  NH is the unit's Hg rounded up to 4, 8, 16 or 32.
+// Geometry per (query heads NH, pass).  NH is the unit's Hg rounded up to 4, 8, 16, 28 or 32.  In the
+// 28-head form the two consumer groups' 14 heads sit at tensor-memory columns 0-13 and 16-29 (the
+// q~ rows of heads 14-27 two rows lower), so each group's loads start on a 16-column boundary.
 // Three rings per CTA, released independently:
 //   K slots   the C_K part of a tile: a LO tile of 512 tokens of 32-byte rows or a HI tile of 128
 //             tokens of 128-byte rows, 16 KB, freed by the score MMA's completion
@@ -79,12 +81,13 @@ constexpr float kLazy = 8.f;        // a per-thread reference sits 2^8 above the
 //   S buffers tensor-memory scores of a tile (kSub x kNHP columns), freed by the consumers
 template <int NH, bool VALUE>
 struct Cfg {
-    static constexpr int kNHP = NH < 16 ? 16 : NH;                  // N of the score MMA
+    static constexpr int kNHP = NH < 16 ? 16 : (NH + 15) / 16 * 16;  // N of the score MMA
     // consumer warp groups: each has four warps (one per tensor-memory lane quarter) and NH / kSplit heads
     // (measured: two groups pay off at 32 heads; at 16 they run no faster than one group of two CTAs per SM)
-    static constexpr int kSplit = NH >= 32 ? 2 : 1;
+    static constexpr int kSplit = NH >= 28 ? 2 : 1;
     static constexpr int kHS = NH / kSplit;
-    static constexpr int kPHS = kHS < 8 ? 8 : kHS;                   // heads per row of a group's P (mma.sync n8 tiles)
+    static constexpr int kPHS = kHS <= 8 ? 8 : kHS <= 16 ? 16 : 32;   // heads per row of a group's P (mma.sync n8 tiles)
+    static constexpr int kGCol = kNHP / kSplit;                      // tensor-memory columns of a group
     static constexpr int kThreads = (8 + 4 * (kSplit - 1)) * 32;
     static constexpr int kBlocks = NH <= 16 ? 2 : 1;                 // resident CTAs per SM
     static constexpr int kLoTok = 512;                               // tokens per LO tile
@@ -152,7 +155,8 @@ template <int NH, bool VALUE>
 constexpr bool smem_fits() { return Cfg<NH, VALUE>::kBlocks * (smem_bytes<NH, VALUE>() + 1024) <= 233472; }
 static_assert(smem_fits<4, false>() && smem_fits<4, true>() && smem_fits<8, false>() && smem_fits<8, true>(), "smem");
 static_assert(smem_fits<16, false>() && smem_fits<16, true>(), "shared memory of two CTAs per SM");
-static_assert(smem_fits<32, false>() && smem_fits<32, true>(), "shared memory of one CTA per SM");
+static_assert(smem_fits<28, false>() && smem_fits<28, true>() && smem_fits<32, false>() && smem_fits<32, true>(),
+              "shared memory of one CTA per SM");
 static_assert(kGatherThreads == 64, "the 4-bit gather assumes 64 threads");
 
 // ------------------------------------------------------------------ tcgen05 helpers
@@ -338,8 +342,17 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
                 const uint32_t bytes = (uint32_t)p.Hg * 128u;
                 fence_proxy_async();
                 mbar_arrive_tx(&sm.qfull[qs], 2 * bytes);
-                bulk_g2s(&sm.qbuf[qs][0][0], src, bytes, &sm.qfull[qs]);
-                bulk_g2s(&sm.qbuf[qs][1][0], src + bytes, bytes, &sm.qfull[qs]);
+                if (NH == 28 && p.Hg > 14) {
+                    // heads 14 .. Hg-1 two rows lower (columns 16 on of the scores)
+                    const uint32_t b0 = 14u * 128u, b1 = bytes - b0;
+                    for (int pl = 0; pl < 2; ++pl) {
+                        bulk_g2s(&sm.qbuf[qs][pl][0], src + pl * bytes, b0, &sm.qfull[qs]);
+                        bulk_g2s(&sm.qbuf[qs][pl][16 * 128], src + pl * bytes + b0, b1, &sm.qfull[qs]);
+                    }
+                } else {
+                    bulk_g2s(&sm.qbuf[qs][0][0], src, bytes, &sm.qfull[qs]);
+                    bulk_g2s(&sm.qbuf[qs][1][0], src + bytes, bytes, &sm.qfull[qs]);
+                }
             }
             ++qseq;
             bool first = true;
@@ -735,10 +748,10 @@ __global__ void __launch_bounds__(Cfg<NH, VALUE>::kThreads, Cfg<NH, VALUE>::kBlo
             // the scores of one sub-tile (this group's heads) are loaded from tensor memory before each wait
             for (int sub = 0; sub < nsub && !failed; ++sub) {
                 if (sub * kTile + 32 * q >= n) continue;   // no token of this warp here
-                constexpr int NL = HS < 4 ? 4 : HS;
+                constexpr int NL = HS <= 4 ? 4 : HS <= 8 ? 8 : HS <= 16 ? 16 : 32;   // columns loaded
                 float sc[NL];
                 if (has_s) {
-                    tmem_ld<NL>(tmem + lane_addr + (uint32_t)(sb * C::kSCols + sub * kNHP + h0), sc);
+                    tmem_ld<NL>(tmem + lane_addr + (uint32_t)(sb * C::kSCols + sub * kNHP + cg * C::kGCol), sc);
                     tmem_wait_ld();
                 } else {
                     #pragma unroll
