@@ -211,53 +211,13 @@ __device__ void eig_gemm(const float *__restrict__ Gu, const unsigned char *qbuf
 }
 
 // C[i][j] = sum_r At[i][r] Bt[j][r] for i, j < 96, where At and Bt hold 96 columns of 512
-// fp32 (column i contiguous).  Chunks of 32 rows are staged transposed in shared memory;
-// thread t accumulates rows 3 (t / 16) .. +2 and columns 6 (t % 16) .. +5 of C in fp32.
-__device__ void small_gram(const float *__restrict__ At, const float *__restrict__ Bt, float *C, EigWork &wk) {
-    const int tid = threadIdx.x;
-    const int i0 = 3 * (tid >> 4), j0 = 6 * (tid & 15);
-    float acc[3][6];
-    #pragma unroll
-    for (int x = 0; x < 3; ++x)
-        #pragma unroll
-        for (int y = 0; y < 6; ++y) acc[x][y] = 0.f;
-    for (int r0 = 0; r0 < kN; r0 += kStageRows) {
-        __syncthreads();
-        for (int idx = tid; idx < kP * kStageRows; idx += kEigThreads) {
-            const int c = idx / kStageRows, r = idx % kStageRows;
-            wk.st[0][r * kStagePitch + c] = __ldcg(At + (size_t)c * kN + r0 + r);
-            wk.st[1][r * kStagePitch + c] = __ldcg(Bt + (size_t)c * kN + r0 + r);
-        }
-        __syncthreads();
-        #pragma unroll 4
-        for (int r = 0; r < kStageRows; ++r) {
-            const float *a = &wk.st[0][r * kStagePitch + i0];
-            const float *b = &wk.st[1][r * kStagePitch + j0];
-            float av[3], bv[6];
-            #pragma unroll
-            for (int x = 0; x < 3; ++x) av[x] = a[x];
-            #pragma unroll
-            for (int y = 0; y < 6; ++y) bv[y] = b[y];
-            #pragma unroll
-            for (int x = 0; x < 3; ++x)
-                #pragma unroll
-                for (int y = 0; y < 6; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
-        }
-    }
-    #pragma unroll
-    for (int x = 0; x < 3; ++x)
-        #pragma unroll
-        for (int y = 0; y < 6; ++y) C[(i0 + x) * kP + j0 + y] = acc[x][y];
-    __syncthreads();
-}
-
-// The same product on the tensor cores: both operands split into bf16 hi + lo planes, three
-// products (hi hi, hi lo, lo hi) with fp32 accumulation (~2^-16 relative, as the G Q product).
+// fp32 (column i contiguous), on the tensor cores: both operands split into bf16 hi + lo
+// planes, three products (hi hi, hi lo, lo hi) with fp32 accumulation (~2^-16 relative, as the G Q product).
 // 32-row chunks of the contraction are staged in shared memory as bf16 rows of 32 (one row per
 // column i or j: K-major for both mma.sync operands; the 16-byte chunk c of row x sits at
 // c ^ ((x >> 1) & 3), so the 8-row ldmatrix reads are free of bank conflicts); warp w < 12
 // computes columns 8w .. 8w + 7 of C for all 96 rows.
-__device__ void small_gram_tc(const float *__restrict__ At, const float *__restrict__ Bt, float *C, EigWork &wk) {
+__device__ void small_gram(const float *__restrict__ At, const float *__restrict__ Bt, float *C, EigWork &wk) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, tig = lane & 3;
     // planes of 96 rows x 64 bytes: A hi, A lo, B hi, B lo
@@ -575,7 +535,7 @@ __global__ void __launch_bounds__(kEigThreads, 1) eig_kernel(EigParams p) {
         const bool rr = it == 1 || (it % 3) == 0 || it == p.max_iter;   // measured: every third beats every second
         const float *zsrc;
         if (rr) {
-            small_gram_tc(Qt, Yt, wk.A, wk);            // H = Q^T Y
+            small_gram(Qt, Yt, wk.A, wk);            // H = Q^T Y
             for (int e = tid; e < kP * kP; e += kEigThreads) {
                 const int i = e / kP, j = e % kP;
                 if (i < j) {
@@ -659,7 +619,7 @@ __global__ void __launch_bounds__(kEigThreads, 1) eig_kernel(EigParams p) {
         }
         __syncthreads();
         // Cholesky QR of Z = zsrc * diag(scale): W = S^T (zsrc^T zsrc) S = R^T R, Q = zsrc S R^-1
-        small_gram_tc(zsrc, zsrc, wk.A, wk);
+        small_gram(zsrc, zsrc, wk.A, wk);
         for (int e = tid; e < kP * kP; e += kEigThreads) wk.A[e] *= sm.scale[e / kP] * sm.scale[e % kP];
         __syncthreads();
         cholesky96(wk.A, wk.V, sm);
