@@ -102,8 +102,8 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 constexpr int kEigThreads = 512;
 constexpr int kEigWarps = kEigThreads / 32;
-constexpr int kStageRows = 32;          // rows of Y per staged chunk of a 96 x 96 product
-constexpr int kStagePitch = kP + 1;     // staged chunks are stored transposed, padded
+constexpr int kStageRows = 32;          // contraction rows per staged chunk of a 96 x 96 product
+constexpr int kStagePitch = kP + 1;     // the staging buffer: 2 x 32 x 97 floats, room for four bf16 planes
 constexpr float kJacTol = 1e-6f;        // rotate when |a_pq| > kJacTol sqrt(|a_pp a_qq|) ...
 constexpr float kJacFloor = 1e-7f;      // ... and |a_pq| > kJacFloor max |a_ii| (fp32 rounding level)
 constexpr float kJacQuad = 1e-3f;       // a sweep whose largest ratio is below this is the last (~sqrt(kJacTol))
@@ -212,7 +212,8 @@ __device__ void eig_gemm(const float *__restrict__ Gu, const unsigned char *qbuf
 
 // C[i][j] = sum_r At[i][r] Bt[j][r] for i, j < 96, where At and Bt hold 96 columns of 512
 // fp32 (column i contiguous), on the tensor cores: both operands split into bf16 hi + lo
-// planes, three products (hi hi, hi lo, lo hi) with fp32 accumulation (~2^-16 relative, as the G Q product).
+// planes, three products (hi hi, hi lo, lo hi) with fp32 accumulation (~2^-16 relative, as the
+// G Q product).
 // 32-row chunks of the contraction are staged in shared memory as bf16 rows of 32 (one row per
 // column i or j: K-major for both mma.sync operands; the 16-byte chunk c of row x sits at
 // c ^ ((x >> 1) & 3), so the 8-row ldmatrix reads are free of bank conflicts); warp w < 12
