@@ -30,7 +30,7 @@ constexpr int kR = 64;                // rank kept
 constexpr int kQPitch = 400;          // bytes per row of the bf16 Q layout: hi[96] | lo[96] | pad
 constexpr int kMaxIter = 60;
 constexpr int kMaxSweeps = 16;        // Jacobi sweeps of one 96 x 96 Rayleigh-Ritz problem
-constexpr float kConvTol = 2e-3f;     // estimated remaining relative error of the top-64 sigma
+constexpr float kConvTol = 3e-3f;     // estimated remaining relative error of the top-64 sigma (bound: 1e-2)
 
 struct Workspace {
     float *G;            // [units][512][512]
