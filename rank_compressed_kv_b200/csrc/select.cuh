@@ -4,9 +4,11 @@
 //
 // One unit's T keys are held in registers, KPT consecutive tokens per thread
 // (blocked layout, so thread order is token order).  The k-th largest key
-// theta is built bit by bit from the most significant end: a candidate bit
-// is kept when at least k keys are >= the candidate (32 counting passes over
-// registers, no data movement).  Then every key > theta is selected, plus the
+// theta is built from the most significant end: a candidate bit is kept when
+// at least k keys are >= the candidate (counting passes over registers, no
+// data movement; one bit per pass, two in the cluster kernel, whose passes
+// end at a cluster barrier).  The search stops early at an accepted candidate
+// with exactly k keys at or above it: those k keys are the top k.  Then every key > theta is selected, plus the
 // first (k - #greater) keys equal to theta in token order (an exclusive scan
 // of per-thread equal counts).  Keys are fp32 mapped to order-preserving
 // uint32 (-0 as +0, NaN lowest), so the result is exact and matches any
@@ -73,6 +75,28 @@ __device__ __forceinline__ void write_bits(const uint32_t (&key)[KPT], uint32_t 
     }
 }
 
+// Two bits of theta per counting pass (the cluster kernel, where a pass costs a cluster barrier):
+// with the bits above b fixed, the thread counts its keys >= theta | j 2^b for j = 1, 2, 3 (j = 1
+// and 2 packed as n1 + (n2 << 16): a CTA's count stays below 2^16), and the pass keeps
+// the largest j whose count over the unit is >= k.  The counts fall with j, so this is the same
+// theta as two one-bit passes (bit b + 1 kept iff n2 >= k; then bit b iff n3 >= k, or n1 >= k).
+template <int KPT>
+__device__ __forceinline__ void count3(const uint32_t (&key)[KPT], uint32_t theta, int b, int &n12, int &n3) {
+    const uint32_t c1 = theta | (1u << b), c2 = theta | (2u << b), c3 = theta | (3u << b);
+    int a = 0, d = 0;
+    #pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+        a += (key[i] >= c1 ? 1 : 0) + (key[i] >= c2 ? 0x10000 : 0);
+        d += key[i] >= c3 ? 1 : 0;
+    }
+    n12 = a;
+    n3 = d;
+}
+
+__device__ __forceinline__ uint32_t digit2(int n1, int n2, int n3, int k) {
+    return n3 >= k ? 3u : n2 >= k ? 2u : n1 >= k ? 1u : 0u;
+}
+
 // ------------------------------------------------------------ small T: one warp per unit
 
 template <int KPT>
@@ -101,14 +125,17 @@ __global__ void __launch_bounds__(256) select_warp_kernel(Params p) {
         for (int wd = r; wd < p.nwords; wd += 32) out[wd] = 0u;
         return;
     }
-    // theta = largest x with #{key >= x} >= k  (the k-th largest key)
+    // theta = largest x with #{key >= x} >= k  (the k-th largest key), or the first accepted
+    // candidate with exactly k keys above it
     uint32_t theta = 0u;
     for (int bit = 31; bit >= 0; --bit) {
         const uint32_t cand = theta | (1u << bit);
         int c = 0;
         #pragma unroll
         for (int i = 0; i < KPT; ++i) c += (key[i] >= cand) ? 1 : 0;
-        if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= p.k) theta = cand;
+        const int n = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+        if (n >= p.k) theta = cand;
+        if (n == p.k) break;
     }
     int gt = 0, eq = 0;
     #pragma unroll
@@ -116,7 +143,7 @@ __global__ void __launch_bounds__(256) select_warp_kernel(Params p) {
         gt += (key[i] > theta) ? 1 : 0;
         eq += (key[i] == theta) ? 1 : 0;
     }
-    const int need = p.k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);   // equal keys to take, >= 1
+    const int need = p.k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);   // equal keys to take
     int incl = eq;
     #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -179,7 +206,9 @@ __global__ void __launch_bounds__(kBlockThreads) select_block_kernel(Params p) {
         int c = 0;
         #pragma unroll
         for (int i = 0; i < KPT; ++i) c += (key[i] >= cand) ? 1 : 0;
-        if (block_sum(c) >= p.k) theta = cand;
+        const int n = block_sum(c);          // the same value in every thread: all leave together
+        if (n >= p.k) theta = cand;
+        if (n == p.k) break;
     }
     int gt = 0, eq = 0;
     #pragma unroll
@@ -187,7 +216,7 @@ __global__ void __launch_bounds__(kBlockThreads) select_block_kernel(Params p) {
         gt += (key[i] > theta) ? 1 : 0;
         eq += (key[i] == theta) ? 1 : 0;
     }
-    const int need = p.k - block_sum(gt);   // equal keys to take, >= 1
+    const int need = p.k - block_sum(gt);   // equal keys to take
     int incl = eq;
     #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -232,8 +261,10 @@ __device__ __forceinline__ void st_cluster(int *arr, int idx, uint32_t cta, int 
 template <int KPT>
 __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterThreads)
     select_cluster_kernel(Params p) {
-    __shared__ int red[2][8];
-    __shared__ int counts[2][3][kClusterCtas];   // [parity][count, gt, eq][cta]
+    static_assert(kClusterThreads * KPT < 0x10000, "packed counts");
+    static_assert(kClusterThreads / 32 == 8 && kClusterCtas == 8, "warp and CTA sums: groups of 8 lanes");
+    __shared__ int red[2][2][kClusterThreads / 32];   // [parity][packed pair, third count][warp]
+    __shared__ int counts[2][2][kClusterCtas];       // [parity][packed pair, third count][cta]
     const uint32_t rank = cluster_rank();
     const int unit = blockIdx.x / kClusterCtas;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -260,37 +291,51 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
         for (int wd = r; wd < p.nwords; wd += kClusterCtas * kClusterThreads) out[wd] = 0u;
         return;
     }
-    // sum of v over the cluster's threads (slot c of the parity's buffers), plus, if asked,
-    // the sum over the CTAs of lower rank
+    cluster_sync_all();   // every CTA of the cluster has started before any stores into its shared memory
+    // sums over the unit's threads of a packed pair of counts (ab = a + (b << 16)) and of a third
+    // count c: each CTA's sums go into every CTA's buffers of this parity (lane 8 j + d of warp 0
+    // stores sum j into CTA d), one cluster barrier, then each CTA adds the 8 CTAs' fields; also
+    // the b field summed over the CTAs of lower rank
     int par = 0;
-    auto cluster_sum = [&](int v, int slot, int *lower) -> int {
-        v = (int)__reduce_add_sync(0xffffffffu, (unsigned)v);
-        if (lane == 0) red[par][warp] = v;
+    auto cluster_sum = [&](int ab, int c, int &a_tot, int &b_tot, int &c_tot, int &b_lower) {
+        ab = (int)__reduce_add_sync(0xffffffffu, (unsigned)ab);
+        c = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+        if (lane == 0) {
+            red[par][0][warp] = ab;
+            red[par][1][warp] = c;
+        }
         __syncthreads();
         if (warp == 0) {
-            int s = lane < kClusterThreads / 32 ? red[par][lane] : 0;
-            s = (int)__reduce_add_sync(0xffffffffu, (unsigned)s);
-            if (lane < kClusterCtas) st_cluster(&counts[par][slot][0], (int)rank, (uint32_t)lane, s);
+            int s = lane < 16 ? red[par][lane >> 3][lane & 7] : 0;
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            s += __shfl_xor_sync(0xffffffffu, s, 2);
+            s += __shfl_xor_sync(0xffffffffu, s, 4);
+            if (lane < 16) st_cluster(&counts[par][lane >> 3][0], (int)rank, (uint32_t)(lane & 7), s);
         }
         cluster_sync_all();
-        int tot = 0, low = 0;
+        int sa = 0, sb = 0, sc = 0, lb = 0;
         #pragma unroll
-        for (int c = 0; c < kClusterCtas; ++c) {
-            const int x = counts[par][slot][c];
-            tot += x;
-            low += c < (int)rank ? x : 0;
+        for (int d = 0; d < kClusterCtas; ++d) {
+            const int x = counts[par][0][d];
+            sa += x & 0xFFFF;
+            sb += x >> 16;
+            sc += counts[par][1][d];
+            lb += d < (int)rank ? x >> 16 : 0;
         }
-        if (lower) *lower = low;
+        a_tot = sa;
+        b_tot = sb;
+        c_tot = sc;
+        b_lower = lb;
         par ^= 1;
-        return tot;
     };
     uint32_t theta = 0u;
-    for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t cand = theta | (1u << bit);
-        int c = 0;
-        #pragma unroll
-        for (int i = 0; i < KPT; ++i) c += (key[i] >= cand) ? 1 : 0;
-        if (cluster_sum(c, 0, nullptr) >= p.k) theta = cand;
+    for (int b = 30; b >= 0; b -= 2) {
+        int n12, n3, t1, t2, t3, unused;
+        count3<KPT>(key, theta, b, n12, n3);
+        cluster_sum(n12, n3, t1, t2, t3, unused);     // the same sums in every CTA: all leave together
+        const uint32_t d = digit2(t1, t2, t3, p.k);
+        theta |= d << b;
+        if (d != 0u && (d == 3u ? t3 : d == 2u ? t2 : t1) == p.k) break;
     }
     int gt = 0, eq = 0;
     #pragma unroll
@@ -298,9 +343,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
         gt += (key[i] > theta) ? 1 : 0;
         eq += (key[i] == theta) ? 1 : 0;
     }
-    const int need = p.k - cluster_sum(gt, 1, nullptr);   // equal keys to take, >= 1
     // equal keys at lower token indices: CTAs of lower rank, then lower threads of this CTA
-    int low_ctas = 0;
     int incl = eq;
     #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -308,8 +351,10 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
         if (lane >= d) incl += o;
     }
     __shared__ int wsum[kClusterThreads / 32];
-    if (lane == 31) wsum[warp] = incl;
-    cluster_sum(eq, 2, &low_ctas);                         // also orders wsum's writes before the reads
+    if (lane == 31) wsum[warp] = incl;                     // read after the sum's barriers
+    int gt_tot, eq_tot, unused, low_ctas;
+    cluster_sum(gt + (eq << 16), 0, gt_tot, eq_tot, unused, low_ctas);
+    const int need = p.k - gt_tot;                         // equal keys to take
     int low_warps = 0;
     for (int w2 = 0; w2 < warp; ++w2) low_warps += wsum[w2];
     int before = low_ctas + low_warps + incl - eq;
