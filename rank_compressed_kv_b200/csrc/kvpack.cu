@@ -844,21 +844,27 @@ kvpack_status kvpack_select(const kvpack_dims *d, int32_t n_layers, const float 
     const int T = d->T_vis;
     namespace sl = kvpack::select;
     if (T <= 32 * 64) {
-        int kpt = 1;
-        while (32 * kpt < T) kpt <<= 1;
-        switch (kpt) {
-            case 1: e = launch_select_warp<1>(p, st); break;
-            case 2: e = launch_select_warp<2>(p, st); break;
-            case 4: e = launch_select_warp<4>(p, st); break;
-            case 8: e = launch_select_warp<8>(p, st); break;
-            case 16: e = launch_select_warp<16>(p, st); break;
-            case 32: e = launch_select_warp<32>(p, st); break;
-            default: e = launch_select_warp<64>(p, st); break;
-        }
+        // rows of 32 tokens, rounded up to an instantiated count
+        const int rows = (T + 31) / 32;
+        if (rows <= 1) e = launch_select_warp<1>(p, st);
+        else if (rows <= 2) e = launch_select_warp<2>(p, st);
+        else if (rows <= 4) e = launch_select_warp<4>(p, st);
+        else if (rows <= 8) e = launch_select_warp<8>(p, st);
+        else if (rows <= 12) e = launch_select_warp<12>(p, st);
+        else if (rows <= 16) e = launch_select_warp<16>(p, st);
+        else if (rows <= 18) e = launch_select_warp<18>(p, st);
+        else if (rows <= 24) e = launch_select_warp<24>(p, st);
+        else if (rows <= 32) e = launch_select_warp<32>(p, st);
+        else if (rows <= 48) e = launch_select_warp<48>(p, st);
+        else e = launch_select_warp<64>(p, st);
     } else if (T <= sl::kBlockThreads * 32) {
-        int kpt = 16;
-        while (sl::kBlockThreads * kpt < T) kpt <<= 1;
-        if (kpt == 16) e = launch_select_block<16>(p, st);
+        // rows of 256 tokens (9 to 32 here), rounded up to an instantiated count
+        const int rows = (T + sl::kBlockThreads - 1) / sl::kBlockThreads;
+        if (rows <= 9) e = launch_select_block<9>(p, st);
+        else if (rows <= 12) e = launch_select_block<12>(p, st);
+        else if (rows <= 16) e = launch_select_block<16>(p, st);
+        else if (rows <= 20) e = launch_select_block<20>(p, st);
+        else if (rows <= 25) e = launch_select_block<25>(p, st);
         else e = launch_select_block<32>(p, st);
     } else {
         int kpt = 1;

@@ -2,20 +2,21 @@
 // technical summary 2.B on the fr page: a moving average of the accumulated
 // attention ranks the tokens; the top 25 % keep the full rank).
 //
-// One unit's T keys are held in registers, KPT consecutive tokens per thread
-// (blocked layout, so thread order is token order).  The k-th largest key
-// theta is built from the most significant end: a candidate bit is kept when
-// at least k keys are >= the candidate (counting passes over registers, no
-// data movement; one bit per pass, two in the cluster kernel, whose passes
-// end at a cluster barrier).  The search stops early at an accepted candidate
-// with exactly k keys at or above it: those k keys are the top k.  Then every key > theta is selected, plus the
-// first (k - #greater) keys equal to theta in token order (an exclusive scan
-// of per-thread equal counts).  Keys are fp32 mapped to order-preserving
-// uint32 (-0 as +0, NaN lowest), so the result is exact and matches any
-// correct sort with ties to the lower index.
+// One unit's T keys are held in registers, KPT per thread: strided (key i of
+// thread r is token i * threads + r) in the warp and block forms, blocked (KPT
+// consecutive tokens) in the cluster form.  The k-th largest key theta is
+// built from the most significant end: a candidate bit is kept when at least
+// k keys are >= the candidate (counting passes over registers, no data
+// movement; one bit per pass, two in the cluster kernel, whose passes end at
+// a cluster barrier).  The search stops early at an accepted candidate with
+// exactly k keys at or above it: those k keys are the top k.  Then every key
+// > theta is selected, plus the first (k - #greater) keys equal to theta in
+// token order.  Keys are fp32 mapped to order-preserving uint32 (-0 as +0,
+// NaN lowest), so the result is exact and matches any correct sort with ties
+// to the lower index.
 //
-// Small T (<= 2048): one warp per unit, 8 units per block.
-// Medium T (<= 8192): one block of 256 threads per unit.
+// Small T (<= 2048): one warp per unit, 8 units per block (up to 64 keys per lane).
+// Medium T (<= 8192): one block of 256 threads per unit (9 to 32 keys per thread).
 // Large T (<= 65536): a cluster of 8 CTAs of 256 threads per unit (up to 32 keys per thread).
 #pragma once
 
@@ -39,9 +40,9 @@ struct Params {
     uint32_t *mask;
 };
 
-// Mask bits of a thread's KPT consecutive tokens (thread index r of the unit): keys above theta,
-// and the first `need` keys equal to theta in token order (`before` of them precede this
-// thread's).  KPT >= 32: whole words per thread; otherwise the words are shared within a warp.
+// Mask bits of a thread's KPT consecutive tokens (blocked layout, thread index r of the unit):
+// keys above theta, and the first `need` keys equal to theta in token order (`before` of them
+// precede this thread's).  KPT >= 32: whole words per thread; otherwise the words are shared within a warp.
 template <int KPT>
 __device__ __forceinline__ void write_bits(const uint32_t (&key)[KPT], uint32_t theta, int need, int before, int r,
                                            uint32_t *out, int nwords) {
@@ -98,10 +99,12 @@ __device__ __forceinline__ uint32_t digit2(int n1, int n2, int n3, int k) {
 }
 
 // ------------------------------------------------------------ small T: one warp per unit
-
+//
+// Strided layout: key i of lane l is token 32 i + l, so every load is coalesced, mask word i is
+// the warp's ballot over row i, and KPT (rows) is ceil(T / 32) rounded up to an instantiated size.
 template <int KPT>
 __global__ void __launch_bounds__(256) select_warp_kernel(Params p) {
-    const int unit = blockIdx.x * 8 + (threadIdx.x >> 5), r = threadIdx.x & 31;
+    const int unit = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (unit >= p.n_units) return;          // whole warp leaves together
     const int T = p.T;
     const size_t ub = (size_t)unit * T;
@@ -109,7 +112,7 @@ __global__ void __launch_bounds__(256) select_warp_kernel(Params p) {
     uint32_t key[KPT];
     #pragma unroll
     for (int i = 0; i < KPT; ++i) {
-        const int t = r * KPT + i;
+        const int t = 32 * i + lane;
         key[i] = 0u;
         if (t < T) {
             const float m = p.mass[ub + t];
@@ -122,7 +125,7 @@ __global__ void __launch_bounds__(256) select_warp_kernel(Params p) {
     }
     uint32_t *out = p.mask + (size_t)unit * p.nwords;
     if (p.k <= 0) {
-        for (int wd = r; wd < p.nwords; wd += 32) out[wd] = 0u;
+        for (int wd = lane; wd < p.nwords; wd += 32) out[wd] = 0u;
         return;
     }
     // theta = largest x with #{key >= x} >= k  (the k-th largest key), or the first accepted
@@ -137,34 +140,46 @@ __global__ void __launch_bounds__(256) select_warp_kernel(Params p) {
         if (n >= p.k) theta = cand;
         if (n == p.k) break;
     }
-    int gt = 0, eq = 0;
+    int gt = 0;
+    #pragma unroll
+    for (int i = 0; i < KPT; ++i) gt += (key[i] > theta) ? 1 : 0;
+    const int need = p.k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);   // equal keys to take
+    // rows in token order: keys above theta, and the first `need` keys equal to theta (padding
+    // keys, t >= T, are 0 and come last)
+    const uint32_t lower = (1u << lane) - 1u;
+    int before = 0;                         // equal keys in the rows above
+    uint32_t word = 0u;
     #pragma unroll
     for (int i = 0; i < KPT; ++i) {
-        gt += (key[i] > theta) ? 1 : 0;
-        eq += (key[i] == theta) ? 1 : 0;
+        const bool eq = key[i] == theta;
+        const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+        const bool sel = key[i] > theta || (eq && before + __popc(eqm & lower) < need);
+        const uint32_t w = __ballot_sync(0xffffffffu, sel);
+        before += __popc(eqm);
+        if (lane == (i & 31)) word = w;
+        if ((i & 31) == 31 || i == KPT - 1) {   // lanes 0 .. (i & 31) hold words (i & ~31) + lane
+            const int wd = (i & ~31) + lane;
+            if (lane <= (i & 31) && wd < p.nwords) out[wd] = word;
+        }
     }
-    const int need = p.k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);   // equal keys to take
-    int incl = eq;
-    #pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, d);
-        if (r >= d) incl += o;
-    }
-    int before = incl - eq;                 // equal keys at lower token indices
-    write_bits<KPT>(key, theta, need, before, r, out, p.nwords);
 }
 
 // ------------------------------------------------------------ medium T: one block per unit
 //
-// 256 threads, KPT keys each (T <= 256 KPT).  A counting pass sums the warps' counts through
-// shared memory with one barrier; the two count buffers alternate between passes, so a thread
-// that runs ahead never overwrites counts another is still reading.
+// 256 threads, strided as the warp form: key i of thread r is token 256 i + r (row i = mask
+// words 8 i .. 8 i + 7, one per warp), KPT = ceil(T / 256) rounded up to an instantiated size.
+// A counting pass sums the warps' counts through shared memory with one barrier; the two count
+// buffers alternate between passes, so a thread that runs ahead never overwrites counts another
+// is still reading.  When not every key equal to theta is taken, a key's rank among the equal
+// ones comes from per-row, per-warp counts in shared memory.
 constexpr int kBlockThreads = 256;
 
 template <int KPT>
 __global__ void __launch_bounds__(kBlockThreads) select_block_kernel(Params p) {
-    __shared__ int red[2][kBlockThreads / 32];
-    __shared__ int wsum[kBlockThreads / 32];
+    constexpr int kWarps = kBlockThreads / 32;
+    static_assert(kBlockThreads * KPT < 0x10000, "packed counts");
+    __shared__ int red[2][kWarps];
+    __shared__ int rows[KPT][kWarps];       // keys equal to theta per row and warp (ordered ties)
     const int unit = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = p.T;
@@ -173,7 +188,7 @@ __global__ void __launch_bounds__(kBlockThreads) select_block_kernel(Params p) {
     uint32_t key[KPT];
     #pragma unroll
     for (int i = 0; i < KPT; ++i) {
-        const int t = tid * KPT + i;
+        const int t = kBlockThreads * i + tid;
         key[i] = 0u;
         if (t < T) {
             const float m = p.mass[ub + t];
@@ -196,7 +211,7 @@ __global__ void __launch_bounds__(kBlockThreads) select_block_kernel(Params p) {
         __syncthreads();
         int tot = 0;
         #pragma unroll
-        for (int w = 0; w < kBlockThreads / 32; ++w) tot += red[par][w];
+        for (int w = 0; w < kWarps; ++w) tot += red[par][w];
         par ^= 1;
         return tot;
     };
@@ -216,18 +231,41 @@ __global__ void __launch_bounds__(kBlockThreads) select_block_kernel(Params p) {
         gt += (key[i] > theta) ? 1 : 0;
         eq += (key[i] == theta) ? 1 : 0;
     }
-    const int need = p.k - block_sum(gt);   // equal keys to take
-    int incl = eq;
-    #pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += o;
+    const int both = block_sum(gt + (eq << 16));
+    const int need = p.k - (both & 0xFFFF);  // equal keys to take
+    const bool take_all = (both >> 16) <= need;   // block-uniform
+    if (!take_all) {
+        #pragma unroll
+        for (int i = 0; i < KPT; ++i) {
+            const uint32_t eqm = __ballot_sync(0xffffffffu, key[i] == theta);
+            if (lane == 0) rows[i][warp] = __popc(eqm);
+        }
+        __syncthreads();
     }
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    int before = incl - eq;                  // equal keys at lower token indices
-    for (int w = 0; w < warp; ++w) before += wsum[w];
-    write_bits<KPT>(key, theta, need, before, tid, out, p.nwords);
+    const uint32_t lower = (1u << lane) - 1u;
+    int before = 0;                          // equal keys in the rows above (ordered ties only)
+    uint32_t word = 0u;
+    #pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+        const bool eqk = key[i] == theta;
+        bool sel = key[i] > theta;
+        if (take_all) {
+            sel = sel || eqk;
+        } else {
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eqk);
+            int b = before + __popc(eqm & lower);
+            for (int w = 0; w < warp; ++w) b += rows[i][w];
+            if (eqk) sel = b < need;
+            #pragma unroll
+            for (int w = 0; w < kWarps; ++w) before += rows[i][w];
+        }
+        const uint32_t wbits = __ballot_sync(0xffffffffu, sel);
+        if (lane == (i & 31)) word = wbits;
+        if ((i & 31) == 31 || i == KPT - 1) {   // lanes 0 .. (i & 31) hold rows (i & ~31) + lane
+            const int wd = ((i & ~31) + lane) * kWarps + warp;
+            if (lane <= (i & 31) && wd < p.nwords) out[wd] = word;
+        }
+    }
 }
 
 // ------------------------------------------------------------ large T: a cluster of CTAs per unit
