@@ -40,8 +40,8 @@ def _run(kv, m, k, alpha=0.0, score=None):
     return out.cpu().numpy().view(np.uint32), (sd.cpu().numpy() if sd is not None else None)
 
 
-# every instantiated size: warp rows 1, 2, 4, 8, 12, 16, 18, 24, 32, 48, 64; block rows 9, 12, 16,
-# 20, 25, 32; cluster keys per thread 8, 16, 32 (the sizes T > 8192 reaches)
+# every size the dispatch reaches: warp rows 1, 2, 4, 8, 12, 16, 18, 24, 32, 48, 64; block rows 9, 12, 16,
+# 20, 25, 32; cluster keys per thread 8, 16, 32
 @pytest.mark.parametrize("T", [1, 7, 31, 32, 33, 100, 200, 380, 500, 576, 700, 1000, 1500, 2047, 2048, 2049,
                                2304, 2600, 4096, 4097, 5000, 5200, 6272, 8192, 8193, 20000, 32768, 65536])
 def test_select_bit_exact(T):
