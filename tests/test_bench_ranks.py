@@ -83,3 +83,20 @@ def test_reference_arm_runs_on_rank_zero_only(rank, monkeypatch, capsys):
         assert calls == ["C0"] and json.loads(printed) == {"impl": "reference"}
     else:
         assert calls == [] and printed == ""
+
+
+def test_recorded_traffic_only_for_the_sources_it_was_taken_on(tmp_path, monkeypatch):
+    """The committed DRAM traffic is reported only while the decode sources hash to the digest
+    stored with it; any edit of those sources turns it into null (a re-capture is due)."""
+    csrc = tmp_path / "rank_compressed_kv_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for n in bench.DECODE_SOURCES:
+        (csrc / n).write_text(f"// {n}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    rec = {"decode:C2": {"bytes_per_launch": 12345, "sources_sha256_16": bench.sources_digest()}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    assert bench.recorded_traffic("decode", "C2") == 12345
+    assert bench.recorded_traffic("decode", "C3") is None          # no record for this workload
+    (csrc / bench.DECODE_SOURCES[0]).write_text("// edited\n")
+    assert bench.recorded_traffic("decode", "C2") is None          # sources changed since the capture
